@@ -1,0 +1,485 @@
+"""Benchmark of the IndexMem hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2] [--budget 1024]
+    python bench.py --impl reference ...     # the CPU oracle on a bounded sample
+
+A step is one pass of the whole path over one batch of the workload:
+indexer scoring with the streaming per-key max (chunked for long contexts),
+top-B selection and compaction, the latent-memory update from the evicted
+tokens, then the decode steps over the retained cache with the memory readout.
+The metric counts tokens through the path: the b*L context keys scored and
+evicted plus the b*n_decode decoded tokens, per second.
+
+Under torchrun every rank runs its own replica on its own GPU (the batch
+units are independent; no collective on the data path): weak scaling, the
+time is the max over ranks and the value counts the tokens of all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from learned_kv_cache_indexmem_b200 import binding, synth  # noqa: E402
+from learned_kv_cache_indexmem_b200.layer import IndexMemLayer  # noqa: E402
+
+METRIC = "evicted-cache decode tokens/s + indexer keys/s; % of HBM / tensor-core roofline"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples nvidia-smi during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 6:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[2:6]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workload
+
+class Job:
+    """One replica of the workload on one GPU, inputs resident in HBM."""
+
+    def __init__(self, wl, B, device, seed):
+        self.wl, self.B, self.dev = wl, B, device
+        s = wl.shape
+        self.batch, self.L, self.n_dec = wl.batch, wl.L, wl.n_decode
+        self.cap = B + self.n_dec
+        w = synth.make_weights(s, seed, device)
+        self.inp = synth.make_layer_inputs(wl, w, seed, device)
+        self.decin = synth.make_decode_inputs(wl, w, self.n_dec, seed, device)
+        if wl.needles:
+            synth.plant_needles(wl, self.inp["K"], self.decin["q"], wl.needles, seed)
+        self.w = w
+        self.layer = IndexMemLayer.from_shape(s, w)
+        self.st = self.layer.new_state(self.batch, self.L, B, self.cap, device)
+        self.layer.workspace(self.batch, self.L, B, device)
+        self.zero_M = torch.zeros_like(self.st.M)
+        self.zero_b = torch.zeros_like(self.st.bstab)
+        self.len0 = torch.full_like(self.st.cache_len, B)
+        self.out = torch.empty(self.n_dec, self.batch, s.n_q_heads, s.head_dim, dtype=s.torch_dtype,
+                               device=device)
+        ch = wl.prefill_chunk
+        self.ranges = ([(i, min(self.L, i + ch)) for i in range(0, self.L, ch)] if ch else
+                       [(0, self.L)])
+        self.stream = torch.cuda.Stream(device)   # capture needs a non-default stream
+        self.graph = None
+
+    # kernels per call (see the library's launchers)
+    def launches_per_step(self):
+        n_e = self.L - self.B
+        return 2 * len(self.ranges) + 2 + (2 if n_e > 0 else 0) + self.n_dec
+
+    def reset(self):
+        self.st.cache_len.copy_(self.len0)
+        self.st.M.copy_(self.zero_M)
+        self.st.bstab.copy_(self.zero_b)
+
+    def prefill(self):
+        d = self.inp
+        self.layer.score_and_evict(d["X"], d["Q"], d["K"], d["V"], self.st, self.B,
+                                   q_ranges=self.ranges, stream=self.stream)
+
+    def memory(self):
+        self.layer.update_memory(self.inp["K"], self.inp["V"], self.st, self.B,
+                                 chunk=self.wl.mem_chunk, stream=self.stream)
+
+    def decode_loop(self):
+        for s in range(self.n_dec):
+            self.layer.decode(self.decin["q"][s], self.decin["k_new"][s], self.decin["v_new"][s],
+                              self.st, out=self.out[s], stream=self.stream)
+
+    def capture_decode(self):
+        """The decode steps as one CUDA graph (removes per-launch host overhead)."""
+        with torch.cuda.stream(self.stream):
+            self.reset()
+            self.prefill()
+            self.memory()
+            self.decode_loop()          # warm (and exercise) outside capture
+        torch.cuda.synchronize()
+        self.layer.sync(self.stream)
+        with torch.cuda.stream(self.stream):
+            self.reset()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream):
+            self.decode_loop()
+        torch.cuda.synchronize()
+        self.graph = g
+
+    def step(self, ev=None):
+        with torch.cuda.stream(self.stream):
+            self._step(ev)
+
+    def _step(self, ev):
+        self.reset()
+        if ev: ev[0].record(self.stream)
+        self.prefill()
+        if ev: ev[1].record(self.stream)
+        self.memory()
+        if ev: ev[2].record(self.stream)
+        if self.graph is not None:
+            self.graph.replay()
+        else:
+            self.decode_loop()
+        if ev: ev[3].record(self.stream)
+
+    # algorithmic work -------------------------------------------------------
+    def decode_bytes_per_launch(self):
+        """K/V rows read (cache incl. the new row), memory state, q in, out,
+        new row written; averaged over the decode steps of a step."""
+        s = self.wl.shape
+        es = 2 if s.dtype == "bf16" else 4
+        row = s.n_kv_heads * s.head_dim * es * 2
+        avg_rows = self.B + (self.n_dec + 1) / 2.0
+        mstate = s.n_kv_heads * (s.mem_r * s.head_dim + s.mem_r) * 4
+        qo = 2 * s.n_q_heads * s.head_dim * es
+        return self.batch * (avg_rows * row + mstate + qo + row / 2)
+
+    def prefill_bytes(self):
+        s = self.wl.shape
+        es = 2 if s.dtype == "bf16" else 4
+        xq = self.batch * self.L * (s.hidden + s.n_q_heads * s.head_dim) * es
+        kv_ret = 2 * self.batch * self.B * s.n_kv_heads * s.head_dim * es * 2
+        return xq + kv_ret
+
+    def memory_bytes(self):
+        s = self.wl.shape
+        es = 2 if s.dtype == "bf16" else 4
+        return self.batch * (self.L - self.B) * s.n_kv_heads * s.head_dim * es * 2
+
+    def scoring_flops(self):
+        pairs = 0
+        for (q0, q1) in self.ranges:
+            # pairs (s, t) with t <= s, s in [q0, q1)
+            pairs += (q1 * (q1 + 1) - q0 * (q0 + 1)) // 2
+        return 2 * self.wl.shape.idx_dim * pairs * self.batch
+
+    def tokens_per_step(self):
+        return self.batch * (self.L + self.n_dec)
+
+
+# ------------------------------------------------------------------ e2e
+
+def run_e2e(job, steps, warmup):
+    """Same step through the public API with the step's inputs in pinned host
+    memory: H2D copies of X, Q, K, V and the decode inputs, D2H of the decode
+    outputs and the retained indices, all inside the timed region."""
+    dev_in = [job.inp[k] for k in ("X", "Q", "K", "V")] + \
+             [job.decin[k] for k in ("q", "k_new", "v_new")]
+    host_in = [t.cpu().pin_memory() for t in dev_in]
+    host_out = torch.empty(job.out.shape, dtype=job.out.dtype).pin_memory()
+    host_idx = torch.empty(job.st.idx_retained.shape, dtype=torch.int32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_out.numel() * host_out.element_size() + host_idx.numel() * 4
+
+    def one():
+        with torch.cuda.stream(job.stream):
+            for h, d in zip(host_in, dev_in):
+                d.copy_(h, non_blocking=True)
+            job.step()
+            host_out.copy_(job.out, non_blocking=True)
+            host_idx.copy_(job.st.idx_retained, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(job.stream)
+    for _ in range(steps):
+        one()
+    b.record(job.stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps, h2d, d2h
+
+
+# ------------------------------------------------------------------ cpu oracle
+
+def cpu_oracle_sample(wl, B, budget_s=20.0):
+    """Times the CPU oracle on a bounded sample of the workload and scales each
+    stage to the full step by its unit count. Returns (seconds per full step,
+    description of the sample, threads used)."""
+    from oracle import indexmem_oracle as om
+    s = wl.shape
+    torch.manual_seed(0)
+    Ls = min(wl.L, 2048)                       # one sequence, first Ls tokens
+    w = synth.make_weights(s, wl.seed, "cpu")
+    inp = synth.make_layer_inputs(wl, w, wl.seed, "cpu", L=Ls, batch=1)
+    t0 = time.perf_counter()
+    qhat, khat, gate = om.indexer_features(inp["X"], inp["Q"], w["W_iq"], w["W_ik"], w["w_ig"])
+    t_feat = (time.perf_counter() - t0) / Ls                      # per token
+    keys = np.arange(0, Ls, max(1, Ls // 64))
+    t0 = time.perf_counter()
+    om.pooled_importance(qhat, khat, gate, keys=keys)
+    pairs_s = sum(Ls - k for k in keys)
+    t_pair = (time.perf_counter() - t0) / pairs_s                  # per causal pair
+    I = np.random.default_rng(0).standard_normal((1, wl.L))
+    t0 = time.perf_counter()
+    R, E = om.select_budget(I, B)
+    t_sel = time.perf_counter() - t0                               # per sequence
+    n_mem = min(512, Ls - 1)
+    Em = np.arange(n_mem)[None]
+    t0 = time.perf_counter()
+    M, bs = om.memory_update(inp["K"], inp["V"], Em, w["W_phi"], s.lam)
+    t_mem = (time.perf_counter() - t0) / n_mem                     # per evicted token
+    n_steps = 4
+    dec = synth.make_decode_inputs(wl, w, n_steps, wl.seed, "cpu", batch=1)
+    Bs = min(B, Ls)
+    KR, VR = om.compact(inp["K"].float().numpy(), inp["V"].float().numpy(), np.arange(Bs)[None],
+                        Bs + n_steps)
+    f = lambda t: t.float().numpy().astype(np.float64)
+    clen = np.array([Bs])
+    t0 = time.perf_counter()
+    for st in range(n_steps):
+        _, clen, _, _, _ = om.decode_step(f(dec["q"][st]), f(dec["k_new"][st]), f(dec["v_new"][st]),
+                                          KR, VR, clen, M, bs, f(w["W_phi"]), f(w["w_gate"]))
+    t_dec = (time.perf_counter() - t0) / n_steps * (B + wl.n_decode / 2) / (Bs + n_steps / 2)
+    pairs_full = wl.batch * wl.L * (wl.L + 1) / 2
+    full = (t_feat * wl.batch * wl.L + t_pair * pairs_full + t_sel * wl.batch +
+            t_mem * wl.batch * (wl.L - B) + t_dec * wl.batch * wl.n_decode)
+    sample = ("1 sequence: indexer features of %d tokens, pooled importance of %d keys over "
+              "their causal queries, selection of %d scores, memory update of %d tokens, %d "
+              "decode steps at budget %d; each stage scaled to the full step by its unit count "
+              "(tokens, causal pairs, sequences, evicted tokens, decode tokens x cache length)"
+              % (Ls, len(keys), wl.L, n_mem, n_steps, Bs))
+    return full, sample
+
+
+def oracle_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [os.cpu_count()])
+    except Exception:
+        return os.cpu_count()
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="c2", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--budget", type=int, default=None)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = synth.WORKLOADS[a.workload]
+    B = a.budget or wl.budget
+    if wl.n_layers != 1:
+        raise SystemExit("the bench step covers single-layer workloads (c0-c3)")
+    config = {"workload": "%s: batch %d, L=%d, budget B=%d (%.1f%% eviction), %d decode steps, "
+                          "%s, Llama-3.1-8B-shaped layer" % (
+                              wl.name, wl.batch, wl.L, B, 100.0 * (wl.L - B) / wl.L, wl.n_decode,
+                              wl.shape.dtype),
+              "batch": wl.batch, "L": wl.L, "budget": B, "n_decode": wl.n_decode,
+              "prefill_chunk": wl.prefill_chunk,
+              "l2": "inputs larger than L2: X, Q, K, V (%.2f GiB) are read every step" % (
+                  wl.batch * wl.L * (wl.shape.hidden + wl.shape.n_q_heads * wl.shape.head_dim +
+                                     2 * wl.shape.n_kv_heads * wl.shape.head_dim) *
+                  (2 if wl.shape.dtype == "bf16" else 4) / 2 ** 30),
+              "parallelism": "replica per GPU" if world > 1 else "1 GPU"}
+
+    if a.impl == "reference":
+        if rank != 0:
+            return
+        per_step = []
+        desc = None
+        for i in range(a.warmup + a.steps):
+            t, desc = cpu_oracle_sample(wl, B)
+            if i >= a.warmup:
+                per_step.append(t)
+        t = statistics.mean(per_step)
+        tok = wl.batch * (wl.L + wl.n_decode)
+        v = tok / t
+        cores = oracle_threads()
+        print(json.dumps({
+            "metric": METRIC, "value": v, "unit": "tokens/s", "impl": "reference",
+            "n_gpus": 1, "steps": a.steps, "warmup": a.warmup, "ms_per_step": t * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config,
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}))
+        return
+
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    binding.load()
+    job = Job(wl, B, dev, wl.seed + 1000 * rank)
+    job.capture_decode()
+    for _ in range(a.warmup):
+        job.step()
+    torch.cuda.synchronize()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(a.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                          else local)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    start.record(job.stream)
+    for i in range(a.steps):
+        job.step(ev[i])
+    end.record(job.stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = start.elapsed_time(end) / a.steps
+    stage_ms = {
+        "prefill": statistics.mean(e[0].elapsed_time(e[1]) for e in ev),
+        "memory": statistics.mean(e[1].elapsed_time(e[2]) for e in ev),
+        "decode": statistics.mean(e[2].elapsed_time(e[3]) for e in ev),
+    }
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    layer_sync_ok = True
+    try:
+        job.layer.sync(job.stream)
+    except binding.IndexMemError:
+        layer_sync_ok = False
+
+    peaks = load_peaks()
+    tokens = job.tokens_per_step() * world
+    value = tokens / (ms / 1e3)
+    dec_launch_ms = stage_ms["decode"] / job.n_dec
+    dec_bytes = job.decode_bytes_per_launch()
+    achieved = dec_bytes / (dec_launch_ms / 1e3) / 1e9
+    peak = peaks["hbm_gbs"]
+    stages = {
+        "prefill_score_select_compact": {
+            "ms": stage_ms["prefill"],
+            "indexer_keys_per_s": job.batch * job.L / (stage_ms["prefill"] / 1e3),
+            "scoring_tflops_if_all_time": job.scoring_flops() / (stage_ms["prefill"] / 1e3) / 1e12},
+        "memory_update": {
+            "ms": stage_ms["memory"],
+            "evicted_tokens_per_s": job.batch * (job.L - B) / max(stage_ms["memory"], 1e-9) * 1e3,
+            "GBps": job.memory_bytes() / max(stage_ms["memory"], 1e-9) / 1e6},
+        "decode": {"ms": stage_ms["decode"], "ms_per_launch": dec_launch_ms,
+                   "tokens_per_s": job.batch * job.n_dec / (stage_ms["decode"] / 1e3),
+                   "GBps": achieved},
+    }
+    e2e = None
+    if not a.no_e2e:
+        e2e_ms, h2d, d2h = run_e2e(job, max(2, a.steps // 2), 1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        t_full, desc = cpu_oracle_sample(wl, B)
+        cpu = {"value": job.tokens_per_step() / t_full, "unit": "tokens/s",
+               "cores": oracle_threads(), "kind": "oracle", "sample": desc}
+    if world > 1:
+        torch.distributed.barrier()
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if wl.shape.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": config,
+            "roofline": {"kernel": "decode", "bound": "hbm", "achieved": achieved, "peak": peak,
+                         "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                         "peak_source": peaks["source"]},
+            "stages": stages,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "gpu_launches": job.launches_per_step() * a.steps,
+            "device_errors": not layer_sync_ok,
+        }))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

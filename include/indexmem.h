@@ -1,0 +1,178 @@
+/*
+ * indexmem.h -- C ABI of the IndexMem hot path on NVIDIA B200 (sm_100a).
+ *
+ * IndexMem keeps a bounded KV cache by learned eviction and compensates the
+ * evicted tokens with a small latent memory. Sources, cited by page title and
+ * section:
+ *   [IM-sum]  "IndexMem: learned KV-cache eviction with latent memory",
+ *             technical summary (gist.science), §1 Problem, §2.A Learnable
+ *             indexer, §2.B Latent memory, §4 Experimental results.
+ *   [IM-abs]  "IndexMem: Learned KV-Cache Eviction with Latent Memory for
+ *             Long-Context LLM Inference", arXiv abstract.
+ *
+ * Conventions for every entry point
+ *   - Tensor arguments are DEVICE pointers owned by the caller, row-major and
+ *     contiguous, 16-byte aligned. The library never frees or retains them
+ *     beyond the call (weights passed to imem_init are copied/repacked).
+ *   - Work is enqueued asynchronously on the caller's cudaStream_t (passed as
+ *     void* so this header needs no CUDA include; 0 = legacy default stream).
+ *   - Arguments are validated on the host before anything is launched; an
+ *     invalid call returns an error status and enqueues nothing.
+ *   - Errors raised on the device (a bounded wait that ran out) are recorded
+ *     in the context and reported by imem_sync(). No entry point throws.
+ *   - A context is bound to the device that was current at imem_init; calls
+ *     must be made with that device current. Calls that share a context or a
+ *     workspace must be ordered on one stream.
+ *
+ * Data types: IMEM_FP32 or IMEM_BF16 (the "model dtype") applies to X, Q, K, V,
+ * the indexer weights, decode inputs, the retained cache and the decode output.
+ * The memory state M, b and its weights W_phi, w_gate are always fp32.
+ */
+#ifndef INDEXMEM_H
+#define INDEXMEM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  IMEM_OK = 0,
+  IMEM_ERR_INVALID_ARG = 1,  /* null pointer, bad enum, negative size        */
+  IMEM_ERR_SHAPE = 2,        /* sizes inconsistent (e.g. B > L, q_end > L)   */
+  IMEM_ERR_ALIGN = 3,        /* a pointer is not 16-byte aligned             */
+  IMEM_ERR_UNSUPPORTED = 4,  /* a dimension this build has no kernel for    */
+  IMEM_ERR_CUDA = 5,         /* a CUDA runtime call failed                  */
+  IMEM_ERR_TIMEOUT = 6       /* a bounded device-side wait ran out          */
+} imem_status;
+
+typedef enum { IMEM_FP32 = 0, IMEM_BF16 = 1 } imem_dtype;
+
+/* Layer configuration.
+ * Supported by this build: head_dim in {64,128}; idx_dim in {32,64};
+ * idx_heads == n_q_heads (one indexer head per attention query head,
+ * [IM-sum] §2.A: the multi-head queries are down-projected);
+ * n_q_heads % n_kv_heads == 0 with a group of at most 8; hidden % 64 == 0;
+ * mem_r in {16,32,...,128}; 0 < lambda <= 1. */
+typedef struct {
+  int hidden;        /* H: hidden size of the model                        */
+  int n_q_heads;     /* Hq                                                  */
+  int n_kv_heads;    /* Hkv                                                 */
+  int head_dim;      /* d                                                   */
+  int idx_heads;     /* H_I, must equal n_q_heads                           */
+  int idx_dim;       /* d_I: indexer dimension                              */
+  int mem_r;         /* r: memory feature dimension                         */
+  float lambda;      /* memory decay per evicted token                      */
+  float eps;         /* readout denominator epsilon (1e-6 by default)       */
+  int dtype;         /* imem_dtype                                          */
+  float gate_override; /* NaN: learned gate g(q); otherwise g forced to it  */
+} imem_config;
+
+/* Layer weights, device pointers, read once by imem_init (repacked into the
+ * context, so the caller may free them afterwards).
+ *   W_idx_q [H_I, d, d_I]   model dtype  query down-projection per head
+ *   W_idx_k [H, d_I]        model dtype  shared indexer key from hidden
+ *   w_idx_g [H, H_I]        model dtype  head-gate logits from hidden
+ *   W_phi   [r, d]          fp32         memory feature map phi(x) = W_phi x
+ *   w_gate  [Hq, d]         fp32         readout gate g(q) = sigmoid(w_gate[h].q)
+ * ([IM-sum] §2.A Architecture; §2.B Mechanism, slow weights.) */
+typedef struct {
+  const void* W_idx_q;
+  const void* W_idx_k;
+  const void* w_idx_g;
+  const float* W_phi;
+  const float* w_gate;
+} imem_weights;
+
+typedef struct imem_ctx imem_ctx;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* imem_status_string(imem_status s);
+
+/* Creates a context for one layer on the current device: validates cfg,
+ * repacks the weights into the kernels' layouts (device memory owned by the
+ * context) and allocates a 4-byte device error word. Synchronous.
+ * Errors: INVALID_ARG (null cfg/weights/out), UNSUPPORTED (see imem_config),
+ * ALIGN, CUDA. On error *out is set to NULL. */
+imem_status imem_init(const imem_config* cfg, const imem_weights* w, imem_ctx** out);
+
+/* Releases the context and its device memory (synchronises the device).
+ * NULL is accepted. */
+void imem_destroy(imem_ctx* ctx);
+
+/* Bytes of caller-owned device workspace that score_and_evict, update_memory
+ * and decode need for `batch` sequences of context length L and budget B.
+ * The workspace must be zero-filled once before its first use (it holds
+ * counters that every call leaves at zero again) and must be the same buffer
+ * across the chunked score_and_evict calls of one prefill (it keeps the
+ * indexer keys of earlier chunks). Errors: INVALID_ARG, SHAPE. */
+imem_status imem_workspace_size(imem_ctx* ctx, int batch, int L, int B, size_t* bytes);
+
+/* Indexer scoring with streaming per-key max, then (optionally) top-B
+ * selection and compaction.  ([IM-sum] §2.A Function/Training: dense scores
+ * A[s,t] pooled per key by a running max without forming the L x L matrix;
+ * §1 token eviction; §4 90% eviction; §2.A pre-eviction by query ranges.)
+ *
+ * Inputs (model dtype): X [batch, L, H], Q [batch, L, Hq, d], K, V [batch, L, Hkv, d].
+ * Only rows [q_begin, q_end) of X and Q are read by this call.
+ * running_max [batch, L] fp32, in/out: for keys t in [q_begin, q_end) it is
+ *   reset to -inf, then for all keys t < q_end
+ *   I[t] = max(I[t], max_{s in [max(t,q_begin), q_end)} A[s,t]).
+ *   Calling with consecutive ranges [0,c),[c,2c),...,[.,L) is chunked prefill.
+ * finalize = 1 (requires q_end == L): selects R = the B largest I (ties to the
+ *   lower position), writes idx_retained [batch, B] and idx_evicted
+ *   [batch, L-B] (int32, ascending) and gathers K_ret/V_ret[:, :B] =
+ *   K/V[R] into K_ret, V_ret [batch, cap, Hkv, d] (cap >= B; rows >= B are not
+ *   written). finalize = 0 leaves those outputs untouched (may be NULL).
+ * Errors: INVALID_ARG, SHAPE (B < 1, B > L, q ranges, cap < B), ALIGN,
+ * UNSUPPORTED, CUDA. */
+imem_status imem_score_and_evict(imem_ctx* ctx, int batch, int L, int B,
+                                 const void* X, const void* Q, const void* K, const void* V,
+                                 float* running_max, int q_begin, int q_end, int finalize,
+                                 int32_t* idx_retained, int32_t* idx_evicted,
+                                 void* K_ret, void* V_ret, int cap,
+                                 void* workspace, void* stream);
+
+/* Latent-memory update from the evicted tokens ([IM-sum] §2.B Mechanism,
+ * fast weights: decayed outer-product accumulation into M and stabiliser b).
+ * For every sequence and KV head h, with phi(x) = W_phi x and the evicted
+ * positions E[0..n) (ascending, from idx_evicted [batch, n_evicted]):
+ *   M_h <- lambda^n M_h + sum_i lambda^(n-1-i) phi(k_{E[i],h}) v_{E[i],h}^T
+ *   b_h <- lambda^n b_h + sum_i lambda^(n-1-i) phi(k_{E[i],h})
+ * which equals the sequential update M <- lambda M + phi(k) v^T in order.
+ * K, V [batch, L, Hkv, d] model dtype; M [batch, Hkv, r, d] fp32 in/out;
+ * bstab [batch, Hkv, r] fp32 in/out. `chunk` = evicted tokens per work unit
+ * (a multiple of 64, e.g. 512). n_evicted = 0 leaves M and b unchanged.
+ * Errors: INVALID_ARG, SHAPE, ALIGN, CUDA. */
+imem_status imem_update_memory(imem_ctx* ctx, int batch, int L, const void* K, const void* V,
+                               const int32_t* idx_evicted, int n_evicted, int chunk,
+                               float* M, float* bstab, void* workspace, void* stream);
+
+/* One decode step over the retained cache with the gated memory readout
+ * ([IM-sum] §2.B Output: o = o_attn + g(q) m(q); [IM-abs]).
+ * q [batch, Hq, d]; k_new, v_new [batch, Hkv, d] are appended at row
+ * cache_len[s] of K_ret/V_ret [batch, cap, Hkv, d] and cache_len [batch]
+ * (int32, device) is incremented. Query head h uses KV head h/(Hq/Hkv):
+ *   o_attn = softmax(q K^T / sqrt(d)) V over rows [0, cache_len] (new row incl.)
+ *   u = W_phi q; m = M_kv^T u / (b_kv . u + eps); g = sigmoid(w_gate[h] . q)
+ *   out = o_attn + g m            (out [batch, Hq, d], model dtype)
+ * M, bstab are read only. A sequence whose cache is full (cache_len >= cap)
+ * is left unchanged and its output row is not written; imem_sync reports it.
+ * Errors: INVALID_ARG, SHAPE, ALIGN, CUDA. */
+imem_status imem_decode(imem_ctx* ctx, int batch, const void* q, const void* k_new,
+                        const void* v_new, void* K_ret, void* V_ret, int32_t* cache_len,
+                        int cap, const float* M, const float* bstab, void* out,
+                        void* workspace, void* stream);
+
+/* Waits for the stream, then reports the first error the device recorded for
+ * this context since the last imem_sync (TIMEOUT for a bounded wait that ran
+ * out, SHAPE for a decode into a full cache) or a CUDA error, and clears it. */
+imem_status imem_sync(imem_ctx* ctx, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INDEXMEM_H */

@@ -1,0 +1,283 @@
+// api.cu -- the C ABI (include/indexmem.h): host-side validation, context
+// and workspace layout, and dispatch to the kernels. Nothing here computes
+// part of the method; every step runs in a kernel.
+#include <cuda_runtime.h>
+
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+struct imem_ctx {
+  imem::Ctx c;
+};
+
+namespace imem {
+
+int decode_splits(int batch, int n_kv_heads, int cap);
+int memory_groups(int batch, int n_kv_heads, int n_e, int chunk);
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+Workspace workspace_layout(const Ctx& c, int batch, int L) {
+  // Regions that do not depend on L come first, so that decode (which is not
+  // told L) finds them at the same offsets.
+  Workspace w;
+  size_t off = 0;
+  const size_t units = (size_t)batch * c.cfg.n_kv_heads;
+  w.dec_cnt_off = off;
+  off = align_up(off + (units + batch) * sizeof(int), 256);
+  // decode partials: at most (2*148 + units) split states of a GQA group
+  w.dec_part_off = off;
+  off = align_up(off + (2 * 148 + units) * c.group * (size_t)(c.cfg.head_dim + 4) * sizeof(float), 256);
+  // memory partials: at most (2*148 + units) runs of an r x d (+ r) state
+  w.mem_part_off = off;
+  off = align_up(off + (2 * 148 + units) * ((size_t)c.cfg.mem_r * c.cfg.head_dim + c.cfg.mem_r) *
+                           sizeof(float), 256);
+  w.sel_off = off;
+  off = align_up(off + 256, 256);
+  w.qt_off = off;
+  off = align_up(off + (size_t)batch * L * c.cfg.idx_dim * sizeof(float), 256);
+  w.kh_off = off;
+  off = align_up(off + (size_t)batch * L * c.cfg.idx_dim * sizeof(float), 256);
+  w.total = off;
+  return w;
+}
+
+}  // namespace imem
+
+using imem::Ctx;
+
+namespace {
+
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+inline imem_status check_ptr(const void* p) {
+  if (!p) return IMEM_ERR_INVALID_ARG;
+  if (!aligned16(p)) return IMEM_ERR_ALIGN;
+  return IMEM_OK;
+}
+
+#define IMEM_CHECK(expr)                 \
+  do {                                   \
+    imem_status s__ = (expr);            \
+    if (s__ != IMEM_OK) return s__;      \
+  } while (0)
+
+inline imem_status cuda_status(cudaError_t e) {
+  return e == cudaSuccess ? IMEM_OK : IMEM_ERR_CUDA;
+}
+
+imem_status check_device(const Ctx& c) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return IMEM_ERR_CUDA;
+  return dev == c.device ? IMEM_OK : IMEM_ERR_INVALID_ARG;
+}
+
+size_t dtype_size(int dt) { return dt == IMEM_BF16 ? 2 : 4; }
+
+}  // namespace
+
+extern "C" {
+
+const char* imem_status_string(imem_status s) {
+  switch (s) {
+    case IMEM_OK: return "IMEM_OK";
+    case IMEM_ERR_INVALID_ARG: return "IMEM_ERR_INVALID_ARG";
+    case IMEM_ERR_SHAPE: return "IMEM_ERR_SHAPE";
+    case IMEM_ERR_ALIGN: return "IMEM_ERR_ALIGN";
+    case IMEM_ERR_UNSUPPORTED: return "IMEM_ERR_UNSUPPORTED";
+    case IMEM_ERR_CUDA: return "IMEM_ERR_CUDA";
+    case IMEM_ERR_TIMEOUT: return "IMEM_ERR_TIMEOUT";
+  }
+  return "IMEM_ERR_UNKNOWN";
+}
+
+imem_status imem_init(const imem_config* cfg, const imem_weights* w, imem_ctx** out) {
+  if (!out) return IMEM_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!cfg || !w) return IMEM_ERR_INVALID_ARG;
+  const imem_config& k = *cfg;
+  if (k.dtype != IMEM_FP32 && k.dtype != IMEM_BF16) return IMEM_ERR_INVALID_ARG;
+  if (k.hidden <= 0 || k.n_q_heads <= 0 || k.n_kv_heads <= 0 || k.head_dim <= 0 ||
+      k.idx_heads <= 0 || k.idx_dim <= 0 || k.mem_r <= 0)
+    return IMEM_ERR_INVALID_ARG;
+  if (!(k.lambda > 0.f && k.lambda <= 1.f) || !(k.eps >= 0.f) || isinf(k.eps))
+    return IMEM_ERR_INVALID_ARG;
+  if (k.idx_heads != k.n_q_heads) return IMEM_ERR_UNSUPPORTED;
+  if (k.n_q_heads % k.n_kv_heads) return IMEM_ERR_SHAPE;
+  const int group = k.n_q_heads / k.n_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8) return IMEM_ERR_UNSUPPORTED;
+  if (k.head_dim != 64 && k.head_dim != 128) return IMEM_ERR_UNSUPPORTED;
+  if (k.idx_dim != 32 && k.idx_dim != 64) return IMEM_ERR_UNSUPPORTED;
+  if (k.hidden % 64) return IMEM_ERR_UNSUPPORTED;
+  if (k.mem_r % 16 || k.mem_r > 128) return IMEM_ERR_UNSUPPORTED;
+  if (k.idx_dim + k.n_q_heads > 128) return IMEM_ERR_UNSUPPORTED;
+  IMEM_CHECK(check_ptr(w->W_idx_q));
+  IMEM_CHECK(check_ptr(w->W_idx_k));
+  IMEM_CHECK(check_ptr(w->w_idx_g));
+  IMEM_CHECK(check_ptr(w->W_phi));
+  IMEM_CHECK(check_ptr(w->w_gate));
+
+  imem_ctx* h = (imem_ctx*)calloc(1, sizeof(imem_ctx));
+  if (!h) return IMEM_ERR_CUDA;
+  Ctx& c = h->c;
+  c.cfg = k;
+  c.group = group;
+  if (cudaGetDevice(&c.device) != cudaSuccess) { free(h); return IMEM_ERR_CUDA; }
+  const size_t es = dtype_size(k.dtype);
+  const size_t n_iq = (size_t)k.n_q_heads * k.head_dim * k.idx_dim;
+  const size_t n_ik = (size_t)k.hidden * k.idx_dim;
+  const size_t n_ig = (size_t)k.hidden * k.n_q_heads;
+  const size_t n_phi = (size_t)k.mem_r * k.head_dim;
+  const size_t n_g = (size_t)k.n_q_heads * k.head_dim;
+  cudaError_t e = cudaSuccess;
+  if (e == cudaSuccess) e = cudaMalloc(&c.W_iq, n_iq * es);
+  if (e == cudaSuccess) e = cudaMalloc(&c.W_ik, n_ik * es);
+  if (e == cudaSuccess) e = cudaMalloc(&c.w_ig, n_ig * es);
+  if (e == cudaSuccess) e = cudaMalloc((void**)&c.W_phi, n_phi * sizeof(float));
+  if (e == cudaSuccess) e = cudaMalloc((void**)&c.w_gate, n_g * sizeof(float));
+  if (e == cudaSuccess) e = cudaMalloc((void**)&c.err, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemcpy(c.W_iq, w->W_idx_q, n_iq * es, cudaMemcpyDeviceToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(c.W_ik, w->W_idx_k, n_ik * es, cudaMemcpyDeviceToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(c.w_ig, w->w_idx_g, n_ig * es, cudaMemcpyDeviceToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(c.W_phi, w->W_phi, n_phi * sizeof(float), cudaMemcpyDeviceToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(c.w_gate, w->w_gate, n_g * sizeof(float), cudaMemcpyDeviceToDevice);
+  if (e == cudaSuccess) e = cudaMemset(c.err, 0, sizeof(int));
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    imem_destroy(h);
+    return IMEM_ERR_CUDA;
+  }
+  *out = h;
+  return IMEM_OK;
+}
+
+void imem_destroy(imem_ctx* h) {
+  if (!h) return;
+  Ctx& c = h->c;
+  cudaDeviceSynchronize();
+  cudaFree(c.W_iq);
+  cudaFree(c.W_ik);
+  cudaFree(c.w_ig);
+  cudaFree(c.W_phi);
+  cudaFree(c.w_gate);
+  cudaFree(c.err);
+  free(h);
+}
+
+imem_status imem_workspace_size(imem_ctx* h, int batch, int L, int B, size_t* bytes) {
+  if (!h || !bytes) return IMEM_ERR_INVALID_ARG;
+  if (batch < 1 || L < 1) return IMEM_ERR_SHAPE;
+  if (B < 1 || B > L) return IMEM_ERR_SHAPE;
+  *bytes = imem::workspace_layout(h->c, batch, L).total;
+  return IMEM_OK;
+}
+
+imem_status imem_score_and_evict(imem_ctx* h, int batch, int L, int B, const void* X,
+                                 const void* Q, const void* K, const void* V, float* running_max,
+                                 int q_begin, int q_end, int finalize, int32_t* idx_retained,
+                                 int32_t* idx_evicted, void* K_ret, void* V_ret, int cap,
+                                 void* workspace, void* stream) {
+  if (!h) return IMEM_ERR_INVALID_ARG;
+  const Ctx& c = h->c;
+  if (finalize != 0 && finalize != 1) return IMEM_ERR_INVALID_ARG;
+  if (batch < 1 || L < 1) return IMEM_ERR_SHAPE;
+  if (q_begin < 0 || q_end <= q_begin || q_end > L) return IMEM_ERR_SHAPE;
+  IMEM_CHECK(check_ptr(X));
+  IMEM_CHECK(check_ptr(Q));
+  IMEM_CHECK(check_ptr(running_max));
+  IMEM_CHECK(check_ptr(workspace));
+  if (finalize) {
+    if (q_end != L) return IMEM_ERR_SHAPE;
+    if (B < 1 || B > L || cap < B) return IMEM_ERR_SHAPE;
+    IMEM_CHECK(check_ptr(K));
+    IMEM_CHECK(check_ptr(V));
+    IMEM_CHECK(check_ptr(idx_retained));
+    if (B < L) IMEM_CHECK(check_ptr(idx_evicted));
+    IMEM_CHECK(check_ptr(K_ret));
+    IMEM_CHECK(check_ptr(V_ret));
+  }
+  IMEM_CHECK(check_device(c));
+  cudaStream_t st = (cudaStream_t)stream;
+  const imem::Workspace ws = imem::workspace_layout(c, batch, L);
+  char* wsb = (char*)workspace;
+  float* qt = (float*)(wsb + ws.qt_off);
+  float* kh = (float*)(wsb + ws.kh_off);
+  IMEM_CHECK(cuda_status(imem::launch_prologue(c, batch, L, X, Q, q_begin, q_end, qt, kh,
+                                               running_max, st)));
+  IMEM_CHECK(cuda_status(imem::launch_scoring(c, batch, L, qt, kh, running_max, q_begin, q_end, st)));
+  if (finalize)
+    IMEM_CHECK(cuda_status(imem::launch_select_compact(c, batch, L, B, running_max, K, V,
+                                                       idx_retained, idx_evicted, K_ret, V_ret,
+                                                       cap, wsb + ws.sel_off, st)));
+  return IMEM_OK;
+}
+
+imem_status imem_update_memory(imem_ctx* h, int batch, int L, const void* K, const void* V,
+                               const int32_t* idx_evicted, int n_evicted, int chunk, float* M,
+                               float* bstab, void* workspace, void* stream) {
+  if (!h) return IMEM_ERR_INVALID_ARG;
+  const Ctx& c = h->c;
+  if (batch < 1 || L < 1) return IMEM_ERR_SHAPE;
+  if (n_evicted < 0 || n_evicted > L) return IMEM_ERR_SHAPE;
+  if (chunk < 64 || chunk % 64) return IMEM_ERR_SHAPE;
+  IMEM_CHECK(check_ptr(K));
+  IMEM_CHECK(check_ptr(V));
+  if (n_evicted > 0) IMEM_CHECK(check_ptr(idx_evicted));
+  IMEM_CHECK(check_ptr(M));
+  IMEM_CHECK(check_ptr(bstab));
+  IMEM_CHECK(check_ptr(workspace));
+  IMEM_CHECK(check_device(c));
+  const imem::Workspace ws = imem::workspace_layout(c, batch, L);
+  float* part = (float*)((char*)workspace + ws.mem_part_off);
+  return cuda_status(imem::launch_memory_update(c, batch, L, K, V, idx_evicted, n_evicted, chunk,
+                                                M, bstab, part, (cudaStream_t)stream));
+}
+
+imem_status imem_decode(imem_ctx* h, int batch, const void* q, const void* k_new,
+                        const void* v_new, void* K_ret, void* V_ret, int32_t* cache_len, int cap,
+                        const float* M, const float* bstab, void* out, void* workspace,
+                        void* stream) {
+  if (!h) return IMEM_ERR_INVALID_ARG;
+  const Ctx& c = h->c;
+  if (batch < 1 || cap < 1) return IMEM_ERR_SHAPE;
+  IMEM_CHECK(check_ptr(q));
+  IMEM_CHECK(check_ptr(k_new));
+  IMEM_CHECK(check_ptr(v_new));
+  IMEM_CHECK(check_ptr(K_ret));
+  IMEM_CHECK(check_ptr(V_ret));
+  IMEM_CHECK(check_ptr(cache_len));
+  IMEM_CHECK(check_ptr(M));
+  IMEM_CHECK(check_ptr(bstab));
+  IMEM_CHECK(check_ptr(out));
+  IMEM_CHECK(check_ptr(workspace));
+  IMEM_CHECK(check_device(c));
+  // the decode regions of the workspace do not depend on L
+  const imem::Workspace ws = imem::workspace_layout(c, batch, 1);
+  char* wsb = (char*)workspace;
+  return cuda_status(imem::launch_decode(c, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap,
+                                         M, bstab, out, (float*)(wsb + ws.dec_part_off),
+                                         (int*)(wsb + ws.dec_cnt_off), (cudaStream_t)stream));
+}
+
+imem_status imem_sync(imem_ctx* h, void* stream) {
+  if (!h) return IMEM_ERR_INVALID_ARG;
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return IMEM_ERR_CUDA;
+  int code = 0;
+  e = cudaMemcpy(&code, h->c.err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return IMEM_ERR_CUDA;
+  if (code != 0) {
+    const int zero = 0;
+    cudaMemcpy(h->c.err, &zero, sizeof(int), cudaMemcpyHostToDevice);
+  }
+  if (code == imem::DEV_TIMEOUT) return IMEM_ERR_TIMEOUT;
+  if (code == imem::DEV_CACHE_FULL) return IMEM_ERR_SHAPE;
+  return IMEM_OK;
+}
+
+}  // extern "C"

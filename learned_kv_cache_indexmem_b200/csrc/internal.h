@@ -1,0 +1,66 @@
+// internal.h -- host-side declarations shared by the C-ABI layer and the
+// kernel translation units. Not part of the public interface.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/indexmem.h"
+
+namespace imem {
+
+// Context of one layer: configuration, weights repacked for the kernels, and
+// a device error word.
+struct Ctx {
+  imem_config cfg;
+  int device;
+  int group;            // Hq / Hkv
+  // repacked weights (device, owned)
+  void* W_iq;           // [Hq, d, dI] model dtype (as given)
+  void* W_ik;           // [H, dI] model dtype (as given)
+  void* w_ig;           // [H, Hq] model dtype (as given)
+  float* W_phi;         // [r, d]
+  float* w_gate;        // [Hq, d]
+  int* err;             // device error word
+};
+
+// Layout of the caller's workspace for (batch, L).
+struct Workspace {
+  size_t qt_off, kh_off;        // indexer q~ and k^ (fp32 [b, L, dI])
+  size_t sel_off;               // selection scratch
+  size_t dec_part_off;          // decode split partials
+  size_t dec_cnt_off;           // decode counters (int), zero between calls
+  size_t mem_part_off;          // memory-update partials
+  size_t total;
+};
+
+constexpr int kDecodeMaxSplits = 64;
+constexpr int kMemMaxGroups = 64;
+
+Workspace workspace_layout(const Ctx& c, int batch, int L);
+
+// ---- launchers (return cudaGetLastError()) ----------------------------------
+
+cudaError_t launch_prologue(const Ctx& c, int batch, int L, const void* X, const void* Q,
+                            int q_begin, int q_end, float* qt, float* kh, float* running_max,
+                            cudaStream_t st);
+
+cudaError_t launch_scoring(const Ctx& c, int batch, int L, const float* qt, const float* kh,
+                           float* running_max, int q_begin, int q_end, cudaStream_t st);
+
+cudaError_t launch_select_compact(const Ctx& c, int batch, int L, int B, const float* running_max,
+                                  const void* K, const void* V, int32_t* idx_r, int32_t* idx_e,
+                                  void* K_ret, void* V_ret, int cap, void* scratch,
+                                  cudaStream_t st);
+
+cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, const void* V,
+                                 const int32_t* idx_e, int n_e, int chunk, float* M, float* bstab,
+                                 float* partials, cudaStream_t st);
+
+cudaError_t launch_decode(const Ctx& c, int batch, const void* q, const void* k_new,
+                          const void* v_new, void* K_ret, void* V_ret, int32_t* cache_len,
+                          int cap, const float* M, const float* bstab, void* out,
+                          float* partials, int* counters, cudaStream_t st);
+
+}  // namespace imem

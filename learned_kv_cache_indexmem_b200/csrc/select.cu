@@ -1,0 +1,181 @@
+// select.cu -- top-B retention and KV-cache compaction.
+//
+// Source: "IndexMem: learned KV-cache eviction with latent memory" technical
+// summary, §1 (token eviction keeps the important tokens within a bounded
+// budget and discards the rest) and §4 (experiments at 90% eviction); the
+// retained set is one per (sequence, layer) because the indexer has a single
+// shared key (§2.A).
+//
+// Selection: R = the B largest importances, ties to the lower position, with
+// -0 and +0 equal. Each importance is mapped to an unsigned key that orders
+// like the float; a 4-pass 8-bit radix select finds the B-th largest key T and
+// how many keys equal to T are taken (the lowest positions). One ordered pass
+// then writes R and its complement E, both ascending.
+//
+// Compaction: K_ret[:, j] = K[:, R[j]] and V_ret likewise, all KV heads at
+// once (one contiguous row of Hkv*d elements per token), 16-byte vectors.
+#include "common.cuh"
+#include "internal.h"
+
+namespace imem {
+namespace {
+
+constexpr int kSelThreads = 1024;
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;                  // -0 -> +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Inclusive block scan of one int per thread (1024 threads); returns the
+// inclusive prefix and writes the block total to *total.
+__device__ __forceinline__ int block_inclusive_scan(int v, int* s_warp, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) s_warp[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int w = s_warp[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += n;
+    }
+    s_warp[lane] = w;
+  }
+  __syncthreads();
+  const int res = v + (warp > 0 ? s_warp[warp - 1] : 0);
+  *total = s_warp[31];
+  __syncthreads();
+  return res;
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+select_kernel(const float* __restrict__ I, int L, int B, int32_t* __restrict__ idx_r,
+              int32_t* __restrict__ idx_e) {
+  const int bi = blockIdx.x;
+  const int tid = threadIdx.x;
+  const float* Ib = I + (size_t)bi * L;
+  __shared__ int s_hist[256];
+  __shared__ int s_warp[32];
+  __shared__ uint32_t s_prefix, s_mask;
+  __shared__ int s_k;
+
+  if (tid == 0) { s_prefix = 0; s_mask = 0; s_k = B; }
+  __syncthreads();
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    if (tid < 256) s_hist[tid] = 0;
+    __syncthreads();
+    const uint32_t prefix = s_prefix, mask = s_mask;
+    for (int t = tid; t < L; t += kSelThreads) {
+      const uint32_t key = order_key(Ib[t]);
+      if ((key & mask) == prefix) atomicAdd(&s_hist[(key >> shift) & 0xffu], 1);
+    }
+    __syncthreads();
+    if (tid < 32) {
+      // find digit d (scanning from the top) where the running count reaches k
+      const int k = s_k;
+      // each lane sums 8 bins, top lanes first
+      int local[8];
+      int sum = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { local[i] = s_hist[255 - (tid * 8 + i)]; sum += local[i]; }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (tid >= o) incl += n;
+      }
+      const int excl = incl - sum;
+      if (excl < k && k <= incl) {  // exactly one lane
+        int run = excl;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (run < k && k <= run + local[i]) {
+            const uint32_t digit = 255u - (uint32_t)(tid * 8 + i);
+            s_k = k - run;
+            s_prefix = prefix | (digit << shift);
+            s_mask = mask | (0xffu << shift);
+          }
+          run += local[i];
+        }
+      }
+    }
+    __syncthreads();
+  }
+  const uint32_t T = s_prefix;   // the B-th largest key
+  const int take_eq = s_k;       // keys equal to T to retain (lowest positions)
+
+  int eq_carry = 0, take_carry = 0;
+  for (int t0 = 0; t0 < L; t0 += kSelThreads) {
+    const int t = t0 + tid;
+    uint32_t key = 0;
+    const bool in = t < L;
+    if (in) key = order_key(Ib[t]);
+    const int is_eq = (in && key == T) ? 1 : 0;
+    int tot;
+    const int eq_incl = block_inclusive_scan(is_eq, s_warp, &tot);
+    const int eq_rank = eq_carry + eq_incl - is_eq;
+    eq_carry += tot;
+    const int take = in && (key > T || (is_eq && eq_rank < take_eq)) ? 1 : 0;
+    const int take_incl = block_inclusive_scan(take, s_warp, &tot);
+    const int before = take_carry + take_incl - take;
+    take_carry += tot;
+    if (in) {
+      if (take) idx_r[(size_t)bi * B + before] = t;
+      else idx_e[(size_t)bi * (L - B) + (t - before)] = t;
+    }
+  }
+}
+
+// One warp group per retained row: copies Hkv*d elements of K and V.
+template <typename T>
+__global__ void gather_kernel(const T* __restrict__ K, const T* __restrict__ V,
+                              const int32_t* __restrict__ idx_r, T* __restrict__ K_ret,
+                              T* __restrict__ V_ret, int L, int B, int cap, int row_elems,
+                              int rows_per_cta) {
+  const int bi = blockIdx.y;
+  const int vec = 16 / sizeof(T);
+  const int nvec = row_elems / vec;
+  for (int j = blockIdx.x * rows_per_cta; j < min(B, (blockIdx.x + 1) * rows_per_cta); ++j) {
+    const int src = idx_r[(size_t)bi * B + j];
+    const uint4* ks = reinterpret_cast<const uint4*>(K + ((size_t)bi * L + src) * row_elems);
+    const uint4* vs = reinterpret_cast<const uint4*>(V + ((size_t)bi * L + src) * row_elems);
+    uint4* kd = reinterpret_cast<uint4*>(K_ret + ((size_t)bi * cap + j) * row_elems);
+    uint4* vd = reinterpret_cast<uint4*>(V_ret + ((size_t)bi * cap + j) * row_elems);
+    for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
+      kd[i] = __ldcs(ks + i);
+      vd[i] = __ldcs(vs + i);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_select_compact(const Ctx& c, int batch, int L, int B, const float* running_max,
+                                  const void* K, const void* V, int32_t* idx_r, int32_t* idx_e,
+                                  void* K_ret, void* V_ret, int cap, void* /*scratch*/,
+                                  cudaStream_t st) {
+  select_kernel<<<batch, kSelThreads, 0, st>>>(running_max, L, B, idx_r, idx_e);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int row_elems = c.cfg.n_kv_heads * c.cfg.head_dim;
+  const int rows_per_cta = 4;
+  dim3 grid((B + rows_per_cta - 1) / rows_per_cta, batch);
+  if (c.cfg.dtype == IMEM_BF16)
+    gather_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(
+        (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, idx_r, (__nv_bfloat16*)K_ret,
+        (__nv_bfloat16*)V_ret, L, B, cap, row_elems, rows_per_cta);
+  else
+    gather_kernel<float><<<grid, 128, 0, st>>>((const float*)K, (const float*)V, idx_r,
+                                               (float*)K_ret, (float*)V_ret, L, B, cap,
+                                               row_elems, rows_per_cta);
+  return cudaGetLastError();
+}
+
+}  // namespace imem

@@ -1,0 +1,115 @@
+"""One IndexMem layer on the GPU: owns the library context and the caller-side
+buffers (allocated with torch), and calls the C ABI through ``binding``.
+
+Plumbing only -- every step of the path runs in libindexmem.so's kernels.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import torch
+
+from . import binding as B_
+
+
+@dataclasses.dataclass
+class PrefillState:
+    running_max: torch.Tensor     # [b, L] fp32
+    idx_retained: torch.Tensor    # [b, B] int32
+    idx_evicted: torch.Tensor     # [b, L-B] int32
+    K_ret: torch.Tensor           # [b, cap, Hkv, d]
+    V_ret: torch.Tensor
+    cache_len: torch.Tensor       # [b] int32
+    M: torch.Tensor               # [b, Hkv, r, d] fp32
+    bstab: torch.Tensor           # [b, Hkv, r] fp32
+
+
+class IndexMemLayer:
+    """Context for one layer. ``weights`` holds device tensors W_iq [Hq,d,dI],
+    W_ik [H,dI], w_ig [H,Hq] (model dtype), W_phi [r,d], w_gate [Hq,d] (fp32)."""
+
+    def __init__(self, hidden, n_q_heads, n_kv_heads, head_dim, idx_dim, mem_r, lam, dtype,
+                 weights, gate_override: Optional[float] = None, eps: float = 1e-6):
+        self.dims = dict(hidden=hidden, n_q_heads=n_q_heads, n_kv_heads=n_kv_heads,
+                         head_dim=head_dim, idx_dim=idx_dim, mem_r=mem_r)
+        self.lam = lam
+        self.torch_dtype = dtype
+        self.code = B_.BF16 if dtype == torch.bfloat16 else B_.FP32
+        cfg = B_.make_config(hidden, n_q_heads, n_kv_heads, head_dim, idx_dim, mem_r, lam,
+                             self.code, eps=eps, gate_override=gate_override)
+        self.ctx = B_.init(cfg, weights["W_iq"], weights["W_ik"], weights["w_ig"],
+                           weights["W_phi"], weights["w_gate"])
+        self._ws = None
+        self._ws_key = None
+
+    @classmethod
+    def from_shape(cls, shape, weights, gate_override=None):
+        return cls(shape.hidden, shape.n_q_heads, shape.n_kv_heads, shape.head_dim,
+                   shape.idx_dim, shape.mem_r, shape.lam, shape.torch_dtype, weights,
+                   gate_override=gate_override)
+
+    def close(self):
+        if self.ctx:
+            B_.destroy(self.ctx)
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # -- buffers ---------------------------------------------------------------
+    def workspace(self, batch: int, L: int, B: int, device) -> torch.Tensor:
+        key = (batch, L, B)
+        if self._ws is None or self._ws_key != key:
+            n = B_.workspace_size(self.ctx, batch, L, B)
+            self._ws = torch.zeros(n, dtype=torch.uint8, device=device)   # zero-filled once
+            self._ws_key = key
+        return self._ws
+
+    def new_state(self, batch: int, L: int, B: int, cap: int, device) -> PrefillState:
+        d, Hkv, r = self.dims["head_dim"], self.dims["n_kv_heads"], self.dims["mem_r"]
+        return PrefillState(
+            running_max=torch.empty(batch, L, dtype=torch.float32, device=device),
+            idx_retained=torch.empty(batch, B, dtype=torch.int32, device=device),
+            idx_evicted=torch.empty(batch, max(L - B, 1), dtype=torch.int32, device=device),
+            K_ret=torch.zeros(batch, cap, Hkv, d, dtype=self.torch_dtype, device=device),
+            V_ret=torch.zeros(batch, cap, Hkv, d, dtype=self.torch_dtype, device=device),
+            cache_len=torch.full((batch,), B, dtype=torch.int32, device=device),
+            M=torch.zeros(batch, Hkv, r, d, dtype=torch.float32, device=device),
+            bstab=torch.zeros(batch, Hkv, r, dtype=torch.float32, device=device))
+
+    # -- the path --------------------------------------------------------------
+    def score_and_evict(self, X, Q, K, V, st: PrefillState, B: int, q_ranges=None,
+                        stream=None):
+        batch, L = X.shape[0], X.shape[1]
+        ws = self.workspace(batch, L, B, X.device)
+        ranges = q_ranges or [(0, L)]
+        for i, (q0, q1) in enumerate(ranges):
+            last = i == len(ranges) - 1
+            B_.score_and_evict(self.ctx, batch, L, B, X, Q, K, V, st.running_max, q0, q1,
+                               1 if last else 0, st.idx_retained,
+                               st.idx_evicted if B < L else None, st.K_ret, st.V_ret,
+                               st.K_ret.shape[1], ws, stream)
+
+    def update_memory(self, K, V, st: PrefillState, B: int, chunk: int = 512, stream=None):
+        batch, L = K.shape[0], K.shape[1]
+        ws = self.workspace(batch, L, B, K.device)
+        B_.update_memory(self.ctx, batch, L, K, V, st.idx_evicted if B < L else None, L - B,
+                         chunk, st.M, st.bstab, ws, stream)
+
+    def decode(self, q, k_new, v_new, st: PrefillState, out=None, B: Optional[int] = None,
+               L: Optional[int] = None, stream=None):
+        batch = q.shape[0]
+        if self._ws is None:
+            raise RuntimeError("decode needs the workspace of a prefill (or call workspace())")
+        if out is None:
+            out = torch.empty_like(q)
+        B_.decode(self.ctx, batch, q, k_new, v_new, st.K_ret, st.V_ret, st.cache_len,
+                  st.K_ret.shape[1], st.M, st.bstab, out, self._ws, stream)
+        return out
+
+    def sync(self, stream=None):
+        B_.sync(self.ctx, stream)

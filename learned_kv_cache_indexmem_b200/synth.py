@@ -218,3 +218,24 @@ def plant_needles(wl: Workload, K: torch.Tensor, q_dec: torch.Tensor, n_needles:
                 K[bi, p, kv] = (kn * (cosine * qd + sin * u)).to(K.dtype)
     order = torch.argsort(pos)
     return pos[order], steps[order]
+
+
+def make_index_subset(batch: int, L: int, n: int, seed: int, device="cpu") -> torch.Tensor:
+    """Per sequence, n distinct positions of [0, L) drawn uniformly, ascending
+    (int32 [batch, n]) -- a synthetic evicted set."""
+    g = _gen(device, 5_000_011 * (seed + 1))
+    rows = []
+    for _ in range(batch):
+        p = torch.randperm(L, generator=g, device=device)[:n]
+        rows.append(torch.sort(p).values)
+    return torch.stack(rows).to(torch.int32).contiguous()
+
+
+def make_memory_state(shape: LayerShape, batch: int, seed: int, device="cpu"):
+    """A synthetic memory state: M [b,Hkv,r,d] and b [b,Hkv,r], fp32, N(0,1)."""
+    g = _gen(device, 6_000_023 * (seed + 1))
+    M = torch.randn(batch, shape.n_kv_heads, shape.mem_r, shape.head_dim, generator=g,
+                    device=device, dtype=torch.float32)
+    b = torch.randn(batch, shape.n_kv_heads, shape.mem_r, generator=g, device=device,
+                    dtype=torch.float32)
+    return M.contiguous(), b.contiguous()
