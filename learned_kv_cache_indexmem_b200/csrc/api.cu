@@ -30,21 +30,42 @@ Workspace workspace_layout(const Ctx& c, int batch, int L) {
   const size_t units = (size_t)batch * c.cfg.n_kv_heads;
   w.dec_cnt_off = off;
   off = align_up(off + (units + batch) * sizeof(int), 256);
-  // decode partials: at most (2*148 + units) split states of a GQA group
+  // decode: per unit up to kDecodeMaxSplits softmax states of the GQA group
+  // plus the readout
   w.dec_part_off = off;
-  off = align_up(off + (2 * 148 + units) * c.group * (size_t)(c.cfg.head_dim + 4) * sizeof(float), 256);
-  // memory partials: at most (2*148 + units) runs of an r x d (+ r) state
+  off = align_up(off + units * (kDecodeMaxSplits + 1) * c.group *
+                           (size_t)(c.cfg.head_dim + 4) * sizeof(float), 256);
+  // memory partials: at most (2*148 + units) runs of a d x (d+1) sum [S | s]
   w.mem_part_off = off;
-  off = align_up(off + (2 * 148 + units) * ((size_t)c.cfg.mem_r * c.cfg.head_dim + c.cfg.mem_r) *
+  off = align_up(off + (2 * 148 + units) * (size_t)c.cfg.head_dim * (c.cfg.head_dim + 1) *
                            sizeof(float), 256);
   w.sel_off = off;
   off = align_up(off + 256, 256);
   w.qt_off = off;
-  off = align_up(off + (size_t)batch * L * c.cfg.idx_dim * sizeof(float), 256);
+  off = align_up(off + (size_t)batch * L * kIdxPad * 2, 1024);
   w.kh_off = off;
-  off = align_up(off + (size_t)batch * L * c.cfg.idx_dim * sizeof(float), 256);
+  off = align_up(off + (size_t)batch * L * kIdxPad * 2, 1024);
   w.total = off;
   return w;
+}
+
+bool make_tmap_rows64(const Ctx& c, CUtensorMap* map, const void* base, uint64_t rows,
+                      uint32_t box_rows) {
+  using Fn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                          const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                          CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                          CUtensorMapFloatOOBfill);
+  if (!c.encode_tiled) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)kIdxPad, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)kIdxPad * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kIdxPad, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = ((Fn)c.encode_tiled)(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                                          const_cast<void*>(base), dims, strides, box, estr,
+                                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 }  // namespace imem
@@ -128,6 +149,19 @@ imem_status imem_init(const imem_config* cfg, const imem_weights* w, imem_ctx** 
   c.cfg = k;
   c.group = group;
   if (cudaGetDevice(&c.device) != cudaSuccess) { free(h); return IMEM_ERR_CUDA; }
+  if (cudaDeviceGetAttribute(&c.num_sms, cudaDevAttrMultiProcessorCount, c.device) != cudaSuccess) {
+    free(h);
+    return IMEM_ERR_CUDA;
+  }
+  {
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &c.encode_tiled, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !c.encode_tiled) {
+      free(h);
+      return IMEM_ERR_CUDA;
+    }
+  }
   const size_t es = dtype_size(k.dtype);
   const size_t n_iq = (size_t)k.n_q_heads * k.head_dim * k.idx_dim;
   const size_t n_ik = (size_t)k.hidden * k.idx_dim;
@@ -205,8 +239,8 @@ imem_status imem_score_and_evict(imem_ctx* h, int batch, int L, int B, const voi
   cudaStream_t st = (cudaStream_t)stream;
   const imem::Workspace ws = imem::workspace_layout(c, batch, L);
   char* wsb = (char*)workspace;
-  float* qt = (float*)(wsb + ws.qt_off);
-  float* kh = (float*)(wsb + ws.kh_off);
+  __nv_bfloat16* qt = (__nv_bfloat16*)(wsb + ws.qt_off);
+  __nv_bfloat16* kh = (__nv_bfloat16*)(wsb + ws.kh_off);
   IMEM_CHECK(cuda_status(imem::launch_prologue(c, batch, L, X, Q, q_begin, q_end, qt, kh,
                                                running_max, st)));
   IMEM_CHECK(cuda_status(imem::launch_scoring(c, batch, L, qt, kh, running_max, q_begin, q_end, st)));

@@ -1,136 +1,270 @@
 // decode.cu -- one decode step over the retained (compacted) KV cache with the
-// gated latent-memory readout fused into the combine.
+// gated latent-memory readout.
 //
 // Source: "IndexMem: learned KV-cache eviction with latent memory" technical
 // summary, §2.B Output: o = o_attn + g(q) * m(q), where o_attn is standard
 // attention over the retained tokens and m(q) the readout of the memory M
-// (with the stabiliser b); the readout weights are a projection phi and a gate
-// g(q). The split-K combine uses the exact merge of softmax partial states
-// (max, normaliser, unnormalised output) over disjoint key blocks, the
-// online-softmax identity stated in "Context Memorization for Efficient Long
-// Context Generation" (technical summary, Method).
+// (normalised with the stabiliser b); the readout weights are a projection
+// phi and a gate g(q). The split-K combine uses the exact merge of softmax
+// partial states (max, normaliser, unnormalised output) over disjoint key
+// blocks -- the online-softmax identity stated in "Context Memorization for
+// Efficient Long Context Generation" (technical summary, Method).
 //
-// Grid (splits, Hkv, batch). Each CTA streams the rows of one split of one
-// (sequence, KV head) and keeps a softmax state for every query head of the
-// GQA group. The last CTA of a (sequence, KV head) -- found with a counter in
-// the workspace, no waiting -- merges the partial states, adds the memory
-// readout and writes the output; the last CTA of a sequence advances
-// cache_len. Split 0 writes the new key/value row into the cache; the CTA that
-// covers row cache_len reads it from k_new/v_new instead.
+// Grid (S + 1, Hkv, batch). For each (sequence, KV head) -- a "unit" -- CTAs
+// 0..S-1 each stream a contiguous block of cache rows and keep one softmax
+// state per query head of the GQA group; CTA S computes the memory readout
+//   u = W_phi q,  m = M^T u / (b . u + eps),  g = sigmoid(w_gate . q)
+// concurrently. Every CTA publishes its result to the workspace and counts
+// itself on the unit's counter (no waiting); the last one to arrive merges
+// the S softmax states, adds g*m and writes the output, and the last unit of
+// a sequence advances cache_len. Split 0 appends the new key/value row to the
+// cache; the CTA whose block covers row cache_len reads it from k_new/v_new.
+//
+// bf16 attention: rows are staged in shared memory with cp.async (two 64-row
+// stages, XOR-swizzled 16-byte chunks) and contracted with warp-level
+// tensor-core MMA (m16n8k16, fp32 accumulation): S^T = q K^T with the GQA
+// heads as the M dimension, then O += P V reusing the score fragments as the
+// A operand. fp32 attention: the same structure on CUDA cores.
 #include "common.cuh"
 #include "internal.h"
 
 #include <math.h>
+#include <type_traits>
 
 namespace imem {
 namespace {
 
 constexpr int kThreads = 128;
+constexpr int kStageRows = 64;
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int D, int G>
-struct Partial {  // one query head's softmax state in a split
-  float m;        // running max of the log2-scaled logits
-  float l;        // sum of 2^(s - m)
+template <int D>
+struct Partial {   // one query head's softmax state over a block of rows
+  float m;         // max of the log2-scaled logits
+  float l;         // sum of 2^(s - m)
   float pad[2];
-  float o[D];     // sum of 2^(s - m) v
+  float o[D];      // sum of 2^(s - m) v
 };
 
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads)
-decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __restrict__ v_new,
-              T* __restrict__ K_ret, T* __restrict__ V_ret, int32_t* __restrict__ cache_len,
-              int cap, int Hkv, int rows_per_split, const float* __restrict__ M,
-              const float* __restrict__ bstab, const float* __restrict__ W_phi,
-              const float* __restrict__ w_gate, int r, float eps, float gate_override,
-              int use_override, T* __restrict__ out, float* __restrict__ partials,
-              int* __restrict__ counters, int* __restrict__ err) {
-  constexpr int LPR = D / 8;          // lanes per row (8 elements per lane)
-  constexpr int RPW = 32 / LPR;       // rows per warp iteration
-  const int sp = blockIdx.x, kh = blockIdx.y, bi = blockIdx.z;
-  const int S = gridDim.x;
+// ---- warp-level tensor-core helpers (bf16) -----------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  const int n = valid ? 16 : 0;   // 0: zero-fill the destination
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+// D = A(16x16, rows 8..15 zero) * B(16x8) + C
+__device__ __forceinline__ void mma_bf16(float* c, uint32_t a0, uint32_t a2, uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// byte offset of 16-byte chunk `c` of row `row` in a staged tile of D-element
+// bf16 rows (XOR swizzle keeps ldmatrix conflict-free)
+template <int D>
+__device__ __forceinline__ uint32_t tile_off(int row, int c) {
+  return (uint32_t)(row * (D * 2) + ((c ^ (row & 7)) << 4));
+}
+
+// ---- attention over rows [r0, r1) for one unit, bf16 tensor-core path --------
+// Leaves the per-warp states in s_part[warp][g].
+template <int D, int G>
+__device__ void attend_bf16(const __nv_bfloat16* __restrict__ Kb, const __nv_bfloat16* __restrict__ Vb,
+                            size_t row_stride, const __nv_bfloat16* kn, const __nv_bfloat16* vn,
+                            int len, int r0, int r1, const float (*s_q)[D],
+                            Partial<D> (*s_part)[G], unsigned char* stage_mem) {
+  constexpr int CH = D / 8;                 // 16-byte chunks per row
+  constexpr int STAGE_BYTES = kStageRows * D * 2;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int Hq = Hkv * G;
+  const int g = lane >> 2, t = lane & 3;
+  const float sscale = kLog2e * rsqrtf((float)D);
 
-  __shared__ int s_flag;
-  __shared__ float s_q[G][D];
-  __shared__ Partial<D, G> s_part[4][G];   // per-warp states, then the merged state
-
-  const int len = cache_len[bi];
-  if (len >= cap) {  // full cache: the whole sequence is skipped by every CTA
-    if (sp == 0 && kh == 0 && tid == 0) record_error(err, DEV_CACHE_FULL);
-    return;
-  }
-  const int n = len + 1;  // rows including the new one
-  const size_t row_stride = (size_t)Hkv * D;
-  const T* Kb = K_ret + (size_t)bi * cap * row_stride + (size_t)kh * D;
-  const T* Vb = V_ret + (size_t)bi * cap * row_stride + (size_t)kh * D;
-  const T* kn = k_new + ((size_t)bi * Hkv + kh) * D;
-  const T* vn = v_new + ((size_t)bi * Hkv + kh) * D;
-
-  // query heads of the group, pre-scaled so that exp2 gives the softmax
-  const float qscale = kLog2e * rsqrtf((float)D);
-  for (int i = tid; i < G * D; i += kThreads) {
-    const int g = i / D, c = i % D;
-    s_q[g][c] = Elem<T>::to_f(q[((size_t)bi * Hq + kh * G + g) * D + c]);
-  }
-  __syncthreads();
-
-  // split 0 appends the new row to the cache
-  if (sp == 0) {
-    for (int c = tid; c < D; c += kThreads) {
-      K_ret[((size_t)bi * cap + len) * row_stride + (size_t)kh * D + c] = kn[c];
-      V_ret[((size_t)bi * cap + len) * row_stride + (size_t)kh * D + c] = vn[c];
+  // q as A fragments (heads on M, rows >= G zero): a0 = dims 16s+2t.., a2 = +8
+  uint32_t qa0[D / 16], qa2[D / 16];
+#pragma unroll
+  for (int s = 0; s < D / 16; ++s) {
+    if (g < G) {
+      qa0[s] = pack_bf16(s_q[g][16 * s + 2 * t], s_q[g][16 * s + 2 * t + 1]);
+      qa2[s] = pack_bf16(s_q[g][16 * s + 8 + 2 * t], s_q[g][16 * s + 8 + 2 * t + 1]);
+    } else {
+      qa0[s] = 0u; qa2[s] = 0u;
     }
   }
+  float o[D / 8][4];
+#pragma unroll
+  for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
 
+  const uint32_t sbase = smem_u32(stage_mem);
+  auto issue = [&](int stage, int buf) {
+    const int base = r0 + stage * kStageRows;
+    const uint32_t kdst = sbase + buf * 2 * STAGE_BYTES;
+    const uint32_t vdst = kdst + STAGE_BYTES;
+    for (int i = tid; i < kStageRows * CH; i += kThreads) {
+      const int rr = i / CH, c = i % CH;
+      const int row = base + rr;
+      const bool ok = row < r1;
+      const __nv_bfloat16* ks = (row == len) ? kn : Kb + (size_t)(ok ? row : r0) * row_stride;
+      const __nv_bfloat16* vs = (row == len) ? vn : Vb + (size_t)(ok ? row : r0) * row_stride;
+      cp_async16(kdst + tile_off<D>(rr, c), ks + c * 8, ok);
+      cp_async16(vdst + tile_off<D>(rr, c), vs + c * 8, ok);
+    }
+    cp_async_commit();
+  };
+
+  const int n_stages = (r1 - r0 + kStageRows - 1) / kStageRows;
+  if (n_stages > 0) issue(0, 0);
+  for (int st = 0; st < n_stages; ++st) {
+    if (st + 1 < n_stages) {
+      issue(st + 1, (st + 1) & 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const uint32_t kt = sbase + (st & 1) * 2 * STAGE_BYTES;
+    const uint32_t vt = kt + STAGE_BYTES;
+    const int kb = r0 + st * kStageRows + warp * 16;   // this warp's 16 rows
+    if (kb < r1) {
+      // scores S^T[head][row] for rows kb..kb+15 as two 8-row n-tiles
+      float sc[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+        const int rr = warp * 16 + nt * 8 + (lane & 7);
+#pragma unroll
+        for (int p = 0; p < D / 32; ++p) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(kt + tile_off<D>(rr, 4 * p + (lane >> 3)), b0, b1, b2, b3);
+          mma_bf16(sc[nt], qa0[2 * p], qa2[2 * p], b0, b1);
+          mma_bf16(sc[nt], qa0[2 * p + 1], qa2[2 * p + 1], b2, b3);
+        }
+      }
+      // mask, scale, block max per head (lanes of a head: xor 1, 2)
+      float mx = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int row = kb + nt * 8 + 2 * t + e;
+          const float v = (row < r1) ? sc[nt][e] * sscale : -INFINITY;
+          sc[nt][e] = v;
+          mx = fmaxf(mx, v);
+        }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float m_new = fmaxf(m_run, mx);
+      const float corr = (m_run == -INFINITY) ? 0.f : exp2f(m_run - m_new);
+      float p[2][2], psum = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          p[nt][e] = (sc[nt][e] == -INFINITY) ? 0.f : exp2f(sc[nt][e] - m_new);
+          psum += p[nt][e];
+        }
+      l_run = l_run * corr + psum;
+      m_run = m_new;
+#pragma unroll
+      for (int j = 0; j < D / 8; ++j) { o[j][0] *= corr; o[j][1] *= corr; }
+      const uint32_t pa0 = pack_bf16(p[0][0], p[0][1]);
+      const uint32_t pa2 = pack_bf16(p[1][0], p[1][1]);
+      // O[head][dims] += P V over the 16 rows
+      const int rr = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int q2 = 0; q2 < D / 16; ++q2) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(vt + tile_off<D>(rr, 2 * q2 + (lane >> 4)), b0, b1, b2, b3);
+        mma_bf16(o[2 * q2], pa0, pa2, b0, b1);
+        mma_bf16(o[2 * q2 + 1], pa0, pa2, b2, b3);
+      }
+    }
+    __syncthreads();
+  }
+  // per-lane partial sums of the head's normaliser -> full sum over the quad
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  if (g < G) {
+    if (t == 0) { s_part[warp][g].m = m_run; s_part[warp][g].l = l_run; }
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) {
+      s_part[warp][g].o[8 * j + 2 * t] = o[j][0];
+      s_part[warp][g].o[8 * j + 2 * t + 1] = o[j][1];
+    }
+  }
+}
+
+// ---- attention, fp32 CUDA-core path --------------------------------------------
+template <int D, int G>
+__device__ void attend_f32(const float* __restrict__ Kb, const float* __restrict__ Vb,
+                           size_t row_stride, const float* kn, const float* vn, int len, int r0,
+                           int r1, const float (*s_q)[D], Partial<D> (*s_part)[G]) {
+  constexpr int LPR = D / 8;
+  constexpr int RPW = 32 / LPR;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int team = lane / LPR, tl = lane % LPR;
+  const float qscale = kLog2e * rsqrtf((float)D);
   float qf[G][8];
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
     for (int e = 0; e < 8; ++e) qf[g][e] = s_q[g][tl * 8 + e] * qscale;
-
   float m_run[G], l_run[G], o_acc[G][8];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    m_run[g] = -INFINITY;
-    l_run[g] = 0.f;
+    m_run[g] = -INFINITY; l_run[g] = 0.f;
 #pragma unroll
     for (int e = 0; e < 8; ++e) o_acc[g][e] = 0.f;
   }
-
-  const int r0 = sp * rows_per_split;
-  const int r1 = min(n, r0 + rows_per_split);
   for (int base = r0 + warp * RPW; base < r1; base += 4 * RPW) {
     const int row = base + team;
     const bool valid = row < r1;
     float kf[8], vf[8];
     if (valid) {
-      const T* kp = (row == len) ? kn : Kb + (size_t)row * row_stride;
-      const T* vp = (row == len) ? vn : Vb + (size_t)row * row_stride;
-      load8<T>(kp + tl * 8, kf);
-      load8<T>(vp + tl * 8, vf);
+      const float* kp = (row == len) ? kn : Kb + (size_t)row * row_stride;
+      const float* vp = (row == len) ? vn : Vb + (size_t)row * row_stride;
+      load8<float>(kp + tl * 8, kf);
+      load8<float>(vp + tl * 8, vf);
     } else {
 #pragma unroll
       for (int e = 0; e < 8; ++e) { kf[e] = 0.f; vf[e] = 0.f; }
     }
-    float s[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       float a = 0.f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) a = fmaf(qf[g][e], kf[e], a);
 #pragma unroll
-      for (int o = LPR / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-      s[g] = a;
-    }
-    if (valid) {
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float mn = fmaxf(m_run[g], s[g]);
-        const float sc = exp2f(m_run[g] - mn);
-        const float p = exp2f(s[g] - mn);
+      for (int off = LPR / 2; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+      if (valid) {
+        const float mn = fmaxf(m_run[g], a);
+        const float sc = (m_run[g] == -INFINITY) ? 0.f : exp2f(m_run[g] - mn);
+        const float p = exp2f(a - mn);
         l_run[g] = l_run[g] * sc + p;
 #pragma unroll
         for (int e = 0; e < 8; ++e) o_acc[g][e] = fmaf(o_acc[g][e], sc, p * vf[e]);
@@ -138,8 +272,6 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
       }
     }
   }
-
-  // merge the row teams of the warp (lanes tl, tl+LPR, ...) into team 0
 #pragma unroll
   for (int off = LPR; off < 32; off <<= 1) {
 #pragma unroll
@@ -166,8 +298,14 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
       for (int e = 0; e < 8; ++e) s_part[warp][g].o[tl * 8 + e] = o_acc[g][e];
     }
   }
+}
+
+// Merge the per-warp states s_part[0..3][g] into s_part[0][g] (needs the
+// block's threads; ends with a barrier).
+template <int D, int G>
+__device__ void merge_warps(Partial<D> (*s_part)[G]) {
+  const int tid = threadIdx.x;
   __syncthreads();
-  // merge the 4 warps into s_part[0]
   for (int i = tid; i < G * D; i += kThreads) {
     const int g = i / D, c = i % D;
     float mx = -INFINITY;
@@ -175,100 +313,176 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     float o = 0.f;
     for (int w = 0; w < 4; ++w)
       if (s_part[w][g].m != -INFINITY) o += s_part[w][g].o[c] * exp2f(s_part[w][g].m - mx);
-    s_part[0][g].o[c] = o;  // each (g,c) read/written by one thread only
+    s_part[0][g].o[c] = o;
   }
   __syncthreads();
   if (tid < G) {
-    const int g = tid;
     float mx = -INFINITY;
-    for (int w = 0; w < 4; ++w) mx = fmaxf(mx, s_part[w][g].m);
+    for (int w = 0; w < 4; ++w) mx = fmaxf(mx, s_part[w][tid].m);
     float l = 0.f;
     for (int w = 0; w < 4; ++w)
-      if (s_part[w][g].m != -INFINITY) l += s_part[w][g].l * exp2f(s_part[w][g].m - mx);
-    s_part[0][g].m = mx;
-    s_part[0][g].l = l;
+      if (s_part[w][tid].m != -INFINITY) l += s_part[w][tid].l * exp2f(s_part[w][tid].m - mx);
+    s_part[0][tid].m = mx;
+    s_part[0][tid].l = l;
   }
   __syncthreads();
+}
 
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kThreads)
+decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __restrict__ v_new,
+              T* __restrict__ K_ret, T* __restrict__ V_ret, int32_t* __restrict__ cache_len,
+              int cap, int Hkv, const float* __restrict__ M, const float* __restrict__ bstab,
+              const float* __restrict__ W_phi, const float* __restrict__ w_gate, int r, float eps,
+              float gate_override, int use_override, T* __restrict__ out,
+              float* __restrict__ partials, int* __restrict__ counters, int* __restrict__ err) {
+  extern __shared__ __align__(128) unsigned char dyn_smem[];
+  const int S = gridDim.x - 1;             // attention splits; CTA S = readout
+  const int sp = blockIdx.x, kh = blockIdx.y, bi = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int Hq = Hkv * G;
   const int unit = bi * Hkv + kh;
-  if (S > 1) {
-    // publish this split's state; the last CTA of the unit merges
-    Partial<D, G>* gp = reinterpret_cast<Partial<D, G>*>(partials) + ((size_t)unit * S + sp) * G;
-    for (int i = tid; i < G * D; i += kThreads) gp[i / D].o[i % D] = s_part[0][i / D].o[i % D];
-    if (tid < G) { gp[tid].m = s_part[0][tid].m; gp[tid].l = s_part[0][tid].l; }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_flag = (atomicAdd(&counters[unit], 1) == S - 1);
-    __syncthreads();
-    if (!s_flag) return;
-    __threadfence();
-    if (tid == 0) counters[unit] = 0;
-    // merge all splits (read through L2: written by other SMs)
-    for (int i = tid; i < G * D; i += kThreads) {
-      const int g = i / D, c = i % D;
-      float mx = -INFINITY;
-      for (int t = 0; t < S; ++t) mx = fmaxf(mx, __ldcg(&gp[(t - sp) * G + g].m));
-      float o = 0.f;
-      for (int t = 0; t < S; ++t) {
-        const float mt = __ldcg(&gp[(t - sp) * G + g].m);
-        if (mt != -INFINITY) o += __ldcg(&gp[(t - sp) * G + g].o[c]) * exp2f(mt - mx);
-      }
-      s_part[1][g].o[c] = o;
+
+  __shared__ float s_q[G][D];
+  __shared__ Partial<D> s_part[4][G];
+  __shared__ int s_flag;
+
+  const int len = cache_len[bi];
+  if (len >= cap) {   // full cache: every CTA of the sequence skips it
+    if (sp == 0 && kh == 0 && tid == 0) record_error(err, DEV_CACHE_FULL);
+    return;
+  }
+  const int n = len + 1;
+  for (int i = tid; i < G * D; i += kThreads)
+    s_q[i / D][i % D] = Elem<T>::to_f(q[((size_t)bi * Hq + kh * G) * D + i]);
+  __syncthreads();
+
+  // workspace of the unit: S softmax states of the group, then the readout
+  Partial<D>* up = reinterpret_cast<Partial<D>*>(partials) + (size_t)unit * (S + 1) * G;
+  float* ro = reinterpret_cast<float*>(up + (size_t)S * G);      // [G][D] g*m
+
+  const size_t row_stride = (size_t)Hkv * D;
+  if (sp < S) {
+    const T* Kb = K_ret + (size_t)bi * cap * row_stride + (size_t)kh * D;
+    const T* Vb = V_ret + (size_t)bi * cap * row_stride + (size_t)kh * D;
+    const T* kn = k_new + ((size_t)bi * Hkv + kh) * D;
+    const T* vn = v_new + ((size_t)bi * Hkv + kh) * D;
+    if (sp == 0) {   // append the new row
+      T* kd = K_ret + ((size_t)bi * cap + len) * row_stride + (size_t)kh * D;
+      T* vd = V_ret + ((size_t)bi * cap + len) * row_stride + (size_t)kh * D;
+      for (int c = tid; c < D; c += kThreads) { kd[c] = kn[c]; vd[c] = vn[c]; }
     }
-    if (tid < G) {
-      float mx = -INFINITY;
-      for (int t = 0; t < S; ++t) mx = fmaxf(mx, __ldcg(&gp[(t - sp) * G + tid].m));
-      float l = 0.f;
-      for (int t = 0; t < S; ++t) {
-        const float mt = __ldcg(&gp[(t - sp) * G + tid].m);
-        if (mt != -INFINITY) l += __ldcg(&gp[(t - sp) * G + tid].l) * exp2f(mt - mx);
-      }
-      s_part[1][tid].l = l;
+    const int per = (n + S - 1) / S;
+    const int r0 = min(n, sp * per), r1 = min(n, r0 + per);
+    if constexpr (std::is_same<T, __nv_bfloat16>::value)
+      attend_bf16<D, G>(Kb, Vb, row_stride, kn, vn, len, r0, r1, s_q, s_part, dyn_smem);
+    else
+      attend_f32<D, G>(Kb, Vb, row_stride, kn, vn, len, r0, r1, s_q, s_part);
+    merge_warps<D, G>(s_part);
+    Partial<D>* mine = up + (size_t)sp * G;
+    for (int i = tid; i < G * D; i += kThreads) mine[i / D].o[i % D] = s_part[0][i / D].o[i % D];
+    if (tid < G) { mine[tid].m = s_part[0][tid].m; mine[tid].l = s_part[0][tid].l; }
+  } else {
+    // memory readout for the group's query heads
+    float* sWT = reinterpret_cast<float*>(dyn_smem);        // [D][r+1] = W_phi^T
+    float* su = sWT + D * (r + 1);                           // [G][r]
+    float* sden = su + G * r;                                // [G]
+    float* sgate = sden + G;                                 // [G]
+    const float4* W4 = reinterpret_cast<const float4*>(W_phi);
+#pragma unroll 8
+    for (int i = tid; i < r * D / 4; i += kThreads) {
+      const float4 v = __ldg(W4 + i);
+      const int j = (4 * i) / D, c = (4 * i) % D;
+      sWT[(c + 0) * (r + 1) + j] = v.x;
+      sWT[(c + 1) * (r + 1) + j] = v.y;
+      sWT[(c + 2) * (r + 1) + j] = v.z;
+      sWT[(c + 3) * (r + 1) + j] = v.w;
     }
     __syncthreads();
-    for (int i = tid; i < G * D; i += kThreads) s_part[0][i / D].o[i % D] = s_part[1][i / D].o[i % D];
-    if (tid < G) s_part[0][tid].l = s_part[1][tid].l;
+    for (int i = tid; i < G * r; i += kThreads) {
+      const int g = i / r, j = i % r;
+      float a = 0.f;
+#pragma unroll 8
+      for (int c = 0; c < D; ++c) a = fmaf(sWT[c * (r + 1) + j], s_q[g][c], a);
+      su[i] = a;
+    }
     __syncthreads();
+    const float* bk = bstab + (size_t)unit * r;
+    for (int g = warp; g < G; g += kThreads / 32) {
+      float a = 0.f;
+      for (int j = lane; j < r; j += 32) a = fmaf(bk[j], su[g * r + j], a);
+      a = warp_sum(a);
+      float z = 0.f;
+      const float* wg = w_gate + (size_t)(kh * G + g) * D;
+      for (int c = lane; c < D; c += 32) z = fmaf(wg[c], s_q[g][c], z);
+      z = warp_sum(z);
+      if (lane == 0) {
+        sden[g] = a + eps;
+        sgate[g] = use_override ? gate_override : sigmoidf_(z);
+      }
+    }
+    __syncthreads();
+    // stage M (r x D) with 16-byte loads in one parallel round, then reduce
+    float* sM = sWT;                                         // W_phi^T no longer needed
+    __syncthreads();
+    const float4* Mk4 = reinterpret_cast<const float4*>(M + (size_t)unit * r * D);
+#pragma unroll 8
+    for (int i = tid; i < r * D / 4; i += kThreads) reinterpret_cast<float4*>(sM)[i] = __ldcg(Mk4 + i);
+    __syncthreads();
+    for (int c = tid; c < D; c += kThreads) {
+      float num[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) num[g] = 0.f;
+#pragma unroll 4
+      for (int j = 0; j < r; ++j) {
+        const float mv = sM[j * D + c];
+#pragma unroll
+        for (int g = 0; g < G; ++g) num[g] = fmaf(mv, su[g * r + j], num[g]);
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) ro[g * D + c] = sgate[g] * (num[g] / sden[g]);
+    }
   }
 
-  // ---- memory readout: u = W_phi q, m = M^T u / (b . u + eps), g = sigmoid(w_gate . q)
-  __shared__ float s_u[G][128];
-  __shared__ float s_den[G], s_gate[G];
-  const float* Mk = M + (size_t)unit * r * D;
-  const float* bk = bstab + (size_t)unit * r;
-  for (int i = tid; i < G * r; i += kThreads) {
-    const int g = i / r, j = i % r;
-    const float* wrow = W_phi + (size_t)j * D;
-    float a = 0.f;
-    for (int c = 0; c < D; ++c) a = fmaf(wrow[c], s_q[g][c], a);
-    s_u[g][j] = a;
+  // count this CTA on the unit; the last arrival merges
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_flag = (atomicAdd(&counters[unit], 1) == S);
+  __syncthreads();
+  if (!s_flag) return;
+  __threadfence();
+  if (tid == 0) counters[unit] = 0;
+  // weights of the S partial states (read through L2: written by other SMs);
+  // all (split, head) maxima and normalisers are fetched in one parallel round
+  __shared__ float s_w[kDecodeMaxSplits][G];
+  __shared__ float s_lp[kDecodeMaxSplits][G];
+  __shared__ float s_l[G];
+  for (int i = tid; i < S * G; i += kThreads) {
+    s_w[i / G][i % G] = __ldcg(&up[i].m);
+    s_lp[i / G][i % G] = __ldcg(&up[i].l);
   }
   __syncthreads();
-  if (warp < G) {
-    const int g = warp;
-    float a = 0.f;
-    for (int j = lane; j < r; j += 32) a = fmaf(bk[j], s_u[g][j], a);
-    a = warp_sum(a);
-    float z = 0.f;
-    const float* wg = w_gate + (size_t)(kh * G + g) * D;
-    for (int c = lane; c < D; c += 32) z = fmaf(wg[c], s_q[g][c], z);
-    z = warp_sum(z);
-    if (lane == 0) {
-      s_den[g] = a + eps;
-      s_gate[g] = use_override ? gate_override : sigmoidf_(z);
+  if (tid < G) {
+    float mx = -INFINITY;
+    for (int t2 = 0; t2 < S; ++t2) mx = fmaxf(mx, s_w[t2][tid]);
+    float l = 0.f;
+    for (int t2 = 0; t2 < S; ++t2) {
+      const float mt = s_w[t2][tid];
+      const float w = (mt == -INFINITY) ? 0.f : exp2f(mt - mx);
+      s_w[t2][tid] = w;
+      l += w * s_lp[t2][tid];
     }
+    s_l[tid] = l;
   }
   __syncthreads();
   for (int i = tid; i < G * D; i += kThreads) {
     const int g = i / D, c = i % D;
-    float num = 0.f;
-    for (int j = 0; j < r; ++j) num = fmaf(Mk[(size_t)j * D + c], s_u[g][j], num);
-    const float oattn = s_part[0][g].o[c] / s_part[0][g].l;
-    const float o = oattn + s_gate[g] * (num / s_den[g]);
-    out[((size_t)bi * Hq + kh * G + g) * D + c] = Elem<T>::from_f(o);
+    float o = 0.f;
+#pragma unroll 8
+    for (int t2 = 0; t2 < S; ++t2) o = fmaf(s_w[t2][g], __ldcg(&up[t2 * G + g].o[c]), o);
+    const float val = o / s_l[g] + __ldcg(&ro[g * D + c]);
+    out[((size_t)bi * Hq + kh * G + g) * D + c] = Elem<T>::from_f(val);
   }
-
-  // the last finished unit of the sequence advances cache_len
   __syncthreads();
   if (tid == 0) {
     __threadfence();
@@ -280,35 +494,54 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   }
 }
 
-template <typename T, int D>
-cudaError_t launch_g(const Ctx& c, int G, dim3 grid, const void* q, const void* kn, const void* vn,
-                     void* K_ret, void* V_ret, int32_t* cache_len, int cap, int rps,
-                     const float* M, const float* bstab, void* out, float* partials,
-                     int* counters, cudaStream_t st) {
-  const int use_ov = !isnan(c.cfg.gate_override);
-#define IMEM_DEC(GG)                                                                         \
-  decode_kernel<T, D, GG><<<grid, kThreads, 0, st>>>(                                        \
-      (const T*)q, (const T*)kn, (const T*)vn, (T*)K_ret, (T*)V_ret, cache_len, cap,         \
-      c.cfg.n_kv_heads, rps, M, bstab, c.W_phi, c.w_gate, c.cfg.mem_r, c.cfg.eps,            \
-      c.cfg.gate_override, use_ov, (T*)out, partials, counters, c.err)
-  switch (G) {
-    case 1: IMEM_DEC(1); break;
-    case 2: IMEM_DEC(2); break;
-    case 4: IMEM_DEC(4); break;
-    case 8: IMEM_DEC(8); break;
-    default: return cudaErrorInvalidValue;
+template <typename T, int D, int G>
+cudaError_t launch_tg(const Ctx& c, dim3 grid, const void* q, const void* kn, const void* vn,
+                      void* K_ret, void* V_ret, int32_t* cache_len, int cap, const float* M,
+                      const float* bstab, void* out, float* partials, int* counters,
+                      cudaStream_t st) {
+  const int r = c.cfg.mem_r;
+  size_t smem_att = std::is_same<T, __nv_bfloat16>::value ? (size_t)2 * 2 * kStageRows * D * 2 : 0;
+  size_t smem_ro = ((size_t)D * (r + 1) + G * r + 2 * G) * sizeof(float);
+  size_t smem = smem_att > smem_ro ? smem_att : smem_ro;
+  auto k = decode_kernel<T, D, G>;
+  static bool attr_set[64] = {};   // per instantiation and device
+  const int dv = c.device & 63;
+  if (!attr_set[dv]) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set[dv] = true;
   }
-#undef IMEM_DEC
+  const int use_ov = !isnan(c.cfg.gate_override);
+  k<<<grid, kThreads, smem, st>>>((const T*)q, (const T*)kn, (const T*)vn, (T*)K_ret, (T*)V_ret,
+                                  cache_len, cap, c.cfg.n_kv_heads, M, bstab, c.W_phi, c.w_gate, r,
+                                  c.cfg.eps, c.cfg.gate_override, use_ov, (T*)out, partials,
+                                  counters, c.err);
   return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_t(const Ctx& c, dim3 grid, const void* q, const void* kn, const void* vn,
+                     void* K_ret, void* V_ret, int32_t* cache_len, int cap, const float* M,
+                     const float* bstab, void* out, float* partials, int* counters,
+                     cudaStream_t st) {
+  switch (c.group) {
+    case 1: return launch_tg<T, D, 1>(c, grid, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, partials, counters, st);
+    case 2: return launch_tg<T, D, 2>(c, grid, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, partials, counters, st);
+    case 4: return launch_tg<T, D, 4>(c, grid, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, partials, counters, st);
+    case 8: return launch_tg<T, D, 8>(c, grid, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, partials, counters, st);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
+// Splits per (sequence, KV head): blocks of about 192 cache rows, at least
+// enough CTAs to cover every SM twice, at most kDecodeMaxSplits.
 int decode_splits(int batch, int n_kv_heads, int cap) {
   const int units = batch * n_kv_heads;
-  int S = (2 * 148 + units - 1) / units;
-  const int max_by_rows = (cap + 63) / 64;
-  if (S > max_by_rows) S = max_by_rows;
+  int S = (cap + kDecodeRowsPerSplit - 1) / kDecodeRowsPerSplit;
+  const int for_sms = (2 * 148 + units - 1) / units;
+  if (S < for_sms) S = for_sms;
   if (S > kDecodeMaxSplits) S = kDecodeMaxSplits;
   if (S < 1) S = 1;
   return S;
@@ -319,15 +552,14 @@ cudaError_t launch_decode(const Ctx& c, int batch, const void* q, const void* k_
                           int cap, const float* M, const float* bstab, void* out,
                           float* partials, int* counters, cudaStream_t st) {
   const int S = decode_splits(batch, c.cfg.n_kv_heads, cap);
-  const int rps = (cap + S - 1) / S;
-  dim3 grid(S, c.cfg.n_kv_heads, batch);
+  dim3 grid(S + 1, c.cfg.n_kv_heads, batch);
   const int D = c.cfg.head_dim;
   if (c.cfg.dtype == IMEM_BF16) {
-    if (D == 128) return launch_g<__nv_bfloat16, 128>(c, c.group, grid, q, k_new, v_new, K_ret, V_ret, cache_len, cap, rps, M, bstab, out, partials, counters, st);
-    if (D == 64) return launch_g<__nv_bfloat16, 64>(c, c.group, grid, q, k_new, v_new, K_ret, V_ret, cache_len, cap, rps, M, bstab, out, partials, counters, st);
+    if (D == 128) return launch_t<__nv_bfloat16, 128>(c, grid, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, partials, counters, st);
+    if (D == 64) return launch_t<__nv_bfloat16, 64>(c, grid, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, partials, counters, st);
   } else {
-    if (D == 128) return launch_g<float, 128>(c, c.group, grid, q, k_new, v_new, K_ret, V_ret, cache_len, cap, rps, M, bstab, out, partials, counters, st);
-    if (D == 64) return launch_g<float, 64>(c, c.group, grid, q, k_new, v_new, K_ret, V_ret, cache_len, cap, rps, M, bstab, out, partials, counters, st);
+    if (D == 128) return launch_t<float, 128>(c, grid, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, partials, counters, st);
+    if (D == 64) return launch_t<float, 64>(c, grid, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, partials, counters, st);
   }
   return cudaErrorInvalidValue;
 }

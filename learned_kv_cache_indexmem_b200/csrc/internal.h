@@ -2,6 +2,8 @@
 // kernel translation units. Not part of the public interface.
 #pragma once
 
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -23,11 +25,21 @@ struct Ctx {
   float* W_phi;         // [r, d]
   float* w_gate;        // [Hq, d]
   int* err;             // device error word
+  int num_sms;          // streaming multiprocessors of the device
+  void* encode_tiled;   // driver entry point cuTensorMapEncodeTiled
 };
+
+// Indexer rows in the workspace: d_I features padded to 64 bf16 (128 bytes).
+constexpr int kIdxPad = 64;
+
+// 2-D TMA map over `rows` rows of 64 bf16 (128 bytes), box {64, box_rows},
+// 128-byte swizzle, zero fill out of bounds. False if encoding fails.
+bool make_tmap_rows64(const Ctx& c, CUtensorMap* map, const void* base, uint64_t rows,
+                      uint32_t box_rows);
 
 // Layout of the caller's workspace for (batch, L).
 struct Workspace {
-  size_t qt_off, kh_off;        // indexer q~ and k^ (fp32 [b, L, dI])
+  size_t qt_off, kh_off;        // indexer q~ and k^ (bf16 [b, L, kIdxPad])
   size_t sel_off;               // selection scratch
   size_t dec_part_off;          // decode split partials
   size_t dec_cnt_off;           // decode counters (int), zero between calls
@@ -36,6 +48,7 @@ struct Workspace {
 };
 
 constexpr int kDecodeMaxSplits = 64;
+constexpr int kDecodeRowsPerSplit = 192;   // cache rows per decode CTA (target)
 constexpr int kMemMaxGroups = 64;
 
 Workspace workspace_layout(const Ctx& c, int batch, int L);
@@ -43,11 +56,12 @@ Workspace workspace_layout(const Ctx& c, int batch, int L);
 // ---- launchers (return cudaGetLastError()) ----------------------------------
 
 cudaError_t launch_prologue(const Ctx& c, int batch, int L, const void* X, const void* Q,
-                            int q_begin, int q_end, float* qt, float* kh, float* running_max,
-                            cudaStream_t st);
+                            int q_begin, int q_end, __nv_bfloat16* qt, __nv_bfloat16* kh,
+                            float* running_max, cudaStream_t st);
 
-cudaError_t launch_scoring(const Ctx& c, int batch, int L, const float* qt, const float* kh,
-                           float* running_max, int q_begin, int q_end, cudaStream_t st);
+cudaError_t launch_scoring(const Ctx& c, int batch, int L, const __nv_bfloat16* qt,
+                           const __nv_bfloat16* kh, float* running_max, int q_begin, int q_end,
+                           cudaStream_t st);
 
 cudaError_t launch_select_compact(const Ctx& c, int batch, int L, int B, const float* running_max,
                                   const void* K, const void* V, int32_t* idx_r, int32_t* idx_e,

@@ -6,141 +6,277 @@
 // accumulation with decay. With phi(k) = W_phi k and decay lambda per evicted
 // token, in ascending position order:
 //   M <- lambda M + phi(k) v^T,   b <- lambda b + phi(k)
-// Over n tokens this equals
-//   M = lambda^n M0 + sum_i lambda^(n-1-i) phi(k_i) v_i^T   (same for b),
-// so disjoint runs of evicted tokens can be accumulated independently with
-// their absolute weights lambda^(n-1-i) and summed.
+// Over the n evicted tokens this equals
+//   M = lambda^n M0 + W_phi S,  S = sum_i w_i k_i v_i^T,  w_i = lambda^(n-1-i)
+//   b = lambda^n b0 + W_phi s,  s = sum_i w_i k_i
+// (phi is linear), so disjoint runs of evicted tokens accumulate
+// independently and W_phi is applied once at the end.
 //
-// Pass 1: grid (groups, Hkv, batch); a CTA accumulates the weighted sum of
-// one run of evicted tokens for one (sequence, KV head) into fp32 partials.
-// Pass 2: one CTA per (sequence, KV head) folds the partials in a fixed order
-// into lambda^n M0 (deterministic).
+// Pass 1 (tensor cores): grid (groups, Hkv, batch); a CTA gathers the rows of
+// one run of evicted tokens for one (sequence, KV head) and accumulates
+//   [S | s] (d x (d+1)) += K_c^T [w*V_c | w]
+// in tensor memory with tcgen05.mma over 64-token chunks. Operands are fp16
+// (bf16 keys convert exactly; w*v is rounded once to fp16) with fp32
+// accumulation; both are MN-major in shared memory (a token is one 128-byte
+// row per 64 features, so gathered rows are written as they arrive). Eight
+// loader warps gather, convert and write the chunks; one thread issues the
+// MMAs; a double-buffered mbarrier ring keeps them in step.
+// Pass 2 (CUDA cores): per (sequence, KV head, 16 columns) sums the runs in a
+// fixed order (deterministic) and applies M = lambda^n M0 + W_phi S.
 #include "common.cuh"
 #include "internal.h"
+#include "tc.cuh"
 
+#include <cuda_fp16.h>
 #include <math.h>
 
 namespace imem {
 namespace {
 
-constexpr int kMemThreads = 256;
-constexpr int kSub = 32;  // tokens per inner step
+constexpr int kLoaders = 256;            // 8 loader warps
+constexpr int kMemThreads = kLoaders + 32;
+constexpr int kChunk = 64;               // tokens per MMA chunk
+constexpr int kStages = 2;
+
+template <int D>
+struct MemTile {
+  static constexpr int A_ATOMS = 2;                    // M = 128 rows (d = 64 zero-padded)
+  static constexpr int B_ATOMS = D / 64 + 1;           // d value columns + weight column
+  static constexpr int N = D + 16;                     // MMA N
+  static constexpr int A_BYTES = A_ATOMS * 8 * 1024;   // 8 K-groups of 8 tokens per atom column
+  static constexpr int B_BYTES = B_ATOMS * 8 * 1024;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int SMEM = kStages * STAGE + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+// MN-major offset of (token jj in the chunk, 16-byte chunk cc of a feature row)
+__device__ __forceinline__ uint32_t mn_off(int jj, int cc) {
+  return (uint32_t)((cc >> 3) * 8192 + (jj >> 3) * 1024 + (jj & 7) * 128 +
+                    ((((cc & 7) ^ (jj & 7))) << 4));
+}
+
+template <typename T>
+__device__ __forceinline__ void load8h(const T* p, float* f);
+template <>
+__device__ __forceinline__ void load8h<__nv_bfloat16>(const __nv_bfloat16* p, float* f) {
+  bf16x8_to_f32(__ldcs(reinterpret_cast<const uint4*>(p)), f);
+}
+template <>
+__device__ __forceinline__ void load8h<float>(const float* p, float* f) {
+  const float4 a = __ldcs(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+__device__ __forceinline__ uint4 to_half8(const float* f) {
+  uint4 r;
+  uint32_t* w = reinterpret_cast<uint32_t*>(&r);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __half2 h = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
+    w[i] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  return r;
+}
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kMemThreads)
-memory_partial_kernel(const T* __restrict__ K, const T* __restrict__ V,
-                      const int32_t* __restrict__ idx_e, int n_e, int L, int Hkv,
-                      const float* __restrict__ W_phi, int r, float lam, int tokens_per_group,
-                      float* __restrict__ partials) {
-  extern __shared__ float smem[];
-  float* sW = smem;                 // [r][D]
-  float* sK = sW + r * D;           // [kSub][D]
-  float* sV = sK + kSub * D;        // [kSub][D]
-  float* sP = sV + kSub * D;        // [kSub][r]  weighted phi
+memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t* __restrict__ idx_e,
+                 int n_e, int L, int Hkv, float log2lam, int tokens_per_group,
+                 float* __restrict__ partials, int* __restrict__ err) {
+  using TL = MemTile<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * TL::STAGE);
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+
   const int g = blockIdx.x, kh = blockIdx.y, bi = blockIdx.z;
   const int G = gridDim.x;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int j0 = g * tokens_per_group;
   const int j1 = min(n_e, j0 + tokens_per_group);
+  const int nchunks = j1 > j0 ? (j1 - j0 + kChunk - 1) / kChunk : 0;
+  const uint32_t sbase = tc::smem_addr(smem);
+  const uint32_t full0 = tc::smem_addr(bars), empty0 = full0 + 8 * kStages,
+                 done = full0 + 16 * kStages;
 
-  for (int i = tid; i < r * D; i += kMemThreads) sW[i] = W_phi[i];
+  // zero both stages once: padded rows of A and the unused weight columns stay 0
+  for (int i = tid; i < kStages * TL::STAGE / 16; i += kMemThreads)
+    reinterpret_cast<uint4*>(smem)[i] = make_uint4(0, 0, 0, 0);
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      tc::mbar_init(full0 + 8 * s, kLoaders);
+      tc::mbar_init(empty0 + 8 * s, 1);
+    }
+    tc::mbar_init(done, 1);
+    tc::fence_mbar_init();
+    s_abort = 0;
+  }
+  if (warp == 8) {
+    tc::tmem_alloc(tc::smem_addr(&s_tmem), 256);
+    tc::tmem_relinquish();
+  }
+  tc::fence_proxy_async();
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = s_tmem;
 
-  // this thread's block of the r x D accumulator: RB rows x 8 columns
-  const int cols8 = D / 8;                      // column blocks of 8
-  const int nblk = (r * D) / 8;                 // blocks of 8 entries
-  constexpr int kMaxBlk = 128 * 128 / 8 / kMemThreads;  // <= 8 blocks per thread
-  float acc[kMaxBlk][8];
-#pragma unroll
-  for (int a = 0; a < kMaxBlk; ++a)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[a][e] = 0.f;
-  float bacc = 0.f;  // threads < r accumulate b
+  float* out = partials + (((size_t)bi * Hkv + kh) * G + g) * (size_t)D * (D + 1);
 
-  const size_t row_stride = (size_t)Hkv * D;
-  const T* Kb = K + (size_t)bi * L * row_stride + (size_t)kh * D;
-  const T* Vb = V + (size_t)bi * L * row_stride + (size_t)kh * D;
-  const int32_t* E = idx_e + (size_t)bi * n_e;
-
-  for (int s0 = j0; s0 < j1; s0 += kSub) {
-    __syncthreads();
-    // gather kSub evicted rows of this head (D/8 vectors per row)
-    for (int i = tid; i < kSub * cols8; i += kMemThreads) {
-      const int jj = i / cols8, cb = i % cols8;
-      float kf[8], vf[8];
-      if (s0 + jj < j1) {
-        const int pos = E[s0 + jj];
-        load8<T>(Kb + (size_t)pos * row_stride + cb * 8, kf);
-        load8<T>(Vb + (size_t)pos * row_stride + cb * 8, vf);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) { kf[e] = 0.f; vf[e] = 0.f; }
+  if (warp < 8) {
+    // ---------------- loaders: gather, convert, write MN-major fp16 rows
+    constexpr int CH = D / 8;                       // 16-byte chunks per feature row
+    constexpr int ITEMS = kChunk * CH / kLoaders;   // per thread per chunk
+    const size_t row_stride = (size_t)Hkv * D;
+    const T* Kb = K + (size_t)bi * L * row_stride + (size_t)kh * D;
+    const T* Vb = V + (size_t)bi * L * row_stride + (size_t)kh * D;
+    const int32_t* E = idx_e + (size_t)bi * n_e;
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c % kStages;
+      if (c >= kStages && !tc::mbar_wait(empty0 + 8 * s, ((c / kStages) - 1) & 1)) {
+        record_error(err, DEV_TIMEOUT);
+        s_abort = 1;
+        break;
       }
+      const uint32_t a_t = sbase + s * TL::STAGE, b_t = a_t + TL::A_BYTES;
+      unsigned char* a_p = smem + s * TL::STAGE;
+      unsigned char* b_p = a_p + TL::A_BYTES;
+      const int base = j0 + c * kChunk;
+      float kf[ITEMS][8], vf[ITEMS][8], wv[ITEMS];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) { sK[jj * D + cb * 8 + e] = kf[e]; sV[jj * D + cb * 8 + e] = vf[e]; }
-    }
-    __syncthreads();
-    // weighted features: P[j][i] = lam^(n-1-j) * (W_phi k_j)[i]
-    for (int i = tid; i < kSub * r; i += kMemThreads) {
-      const int jj = i / r, ri = i % r;
-      float a = 0.f;
-      for (int c = 0; c < D; ++c) a = fmaf(sW[ri * D + c], sK[jj * D + c], a);
-      const int j = s0 + jj;
-      const float w = (j < j1) ? powf(lam, (float)(n_e - 1 - j)) : 0.f;
-      sP[jj * r + ri] = a * w;
-    }
-    __syncthreads();
-    // accumulate P^T V into this thread's blocks
+      for (int it = 0; it < ITEMS; ++it) {
+        const int i = tid + it * kLoaders;
+        const int jj = i / CH, cc = i % CH;
+        const int j = base + jj;
+        if (j < j1) {
+          const int pos = E[j];
+          load8h<T>(Kb + (size_t)pos * row_stride + cc * 8, kf[it]);
+          load8h<T>(Vb + (size_t)pos * row_stride + cc * 8, vf[it]);
+          wv[it] = exp2f((float)(n_e - 1 - j) * log2lam);
+        } else {
 #pragma unroll
-    for (int a = 0; a < kMaxBlk; ++a) {
-      const int blk = tid + a * kMemThreads;
-      if (blk < nblk) {
-        const int ri = blk / cols8, cb = blk % cols8;
-        for (int jj = 0; jj < kSub; ++jj) {
-          const float p = sP[jj * r + ri];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[a][e] = fmaf(p, sV[jj * D + cb * 8 + e], acc[a][e]);
+          for (int e = 0; e < 8; ++e) { kf[it][e] = 0.f; vf[it][e] = 0.f; }
+          wv[it] = 0.f;
         }
       }
+#pragma unroll
+      for (int it = 0; it < ITEMS; ++it) {
+        const int i = tid + it * kLoaders;
+        const int jj = i / CH, cc = i % CH;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) vf[it][e] *= wv[it];
+        *reinterpret_cast<uint4*>(a_p + mn_off(jj, cc)) = to_half8(kf[it]);
+        *reinterpret_cast<uint4*>(b_p + mn_off(jj, cc)) = to_half8(vf[it]);
+        if (cc == 0)   // weight column: element 0 of the row in the last B atom
+          *reinterpret_cast<__half*>(b_p + mn_off(jj, (D / 64) * 8)) = __float2half_rn(wv[it]);
+      }
+      (void)a_t; (void)b_t;
+      tc::fence_proxy_async();
+      tc::mbar_arrive(full0 + 8 * s);
     }
-    if (tid < r)
-      for (int jj = 0; jj < kSub; ++jj) bacc += sP[jj * r + tid];
+  } else if (lane == 0) {
+    // ---------------- MMA issuer
+    constexpr uint32_t IDESC = tc::idesc(tc::kFmtF16, 128, TL::N, true, true);
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c % kStages;
+      if (!tc::mbar_wait(full0 + 8 * s, (c / kStages) & 1)) {
+        record_error(err, DEV_TIMEOUT);
+        s_abort = 1;
+        break;
+      }
+      tc::fence_after();
+      const uint32_t a_t = sbase + s * TL::STAGE, b_t = a_t + TL::A_BYTES;
+#pragma unroll
+      for (int k = 0; k < kChunk / 16; ++k) {   // 16 tokens = 2 K-groups per MMA
+        const uint64_t ad = tc::sdesc_sw128(a_t + k * 2048, 8192, 1024);
+        const uint64_t bd = tc::sdesc_sw128(b_t + k * 2048, 8192, 1024);
+        tc::mma_f16(tmem, ad, bd, IDESC, (c > 0 || k > 0) ? 1u : 0u);
+      }
+      tc::mma_commit(empty0 + 8 * s);
+    }
+    tc::mma_commit(done);
   }
 
-  float* out = partials + (((size_t)bi * Hkv + kh) * G + g) * (size_t)(r * D + r);
+  // ---------------- epilogue: warps 0-3 read [S | s] rows from TMEM
+  if (warp < 4) {
+    const int row = warp * 32 + lane;   // feature index of k (TMEM lane)
+    bool ok = true;
+    if (nchunks > 0) ok = tc::mbar_wait(done, 0);
+    if (!ok) record_error(err, DEV_TIMEOUT);
+    tc::fence_after();
+    if (nchunks > 0 && ok && !s_abort) {
+      constexpr int NCOL = TL::N;   // multiple of 16
+#pragma unroll 1
+      for (int c0 = 0; c0 < NCOL; c0 += 16) {
+        float v[16];
+        tc::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + c0, v);
+        if (row < D) {
 #pragma unroll
-  for (int a = 0; a < kMaxBlk; ++a) {
-    const int blk = tid + a * kMemThreads;
-    if (blk < nblk) {
-      const int ri = blk / cols8, cb = blk % cols8;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) out[ri * D + cb * 8 + e] = acc[a][e];
+          for (int e = 0; e < 16; ++e) {
+            const int col = c0 + e;
+            if (col <= D) out[(size_t)row * (D + 1) + col] = v[e];
+          }
+        }
+      }
+    } else if (row < D) {
+      for (int col = 0; col <= D; ++col) out[(size_t)row * (D + 1) + col] = 0.f;
     }
   }
-  if (tid < r) out[r * D + tid] = bacc;
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 8) tc::tmem_dealloc(tmem, 256);
 }
 
-__global__ void memory_finalize_kernel(const float* __restrict__ partials, int G, int r, int D,
-                                       float decay_n, float* __restrict__ M,
-                                       float* __restrict__ bstab) {
-  const int unit = blockIdx.x;
-  const size_t psz = (size_t)r * D + r;
-  const float* p = partials + (size_t)unit * G * psz;
-  float* Mu = M + (size_t)unit * r * D;
-  float* bu = bstab + (size_t)unit * r;
-  for (int i = threadIdx.x; i < r * D + r; i += blockDim.x) {
-    float a = (i < r * D) ? Mu[i] * decay_n : bu[i - r * D] * decay_n;
-    for (int g = 0; g < G; ++g) a += p[g * psz + i];
-    if (i < r * D) Mu[i] = a;
-    else bu[i - r * D] = a;
+// M[:, cols] = decay * M[:, cols] + W_phi * sum_g S_g[:, cols]; the extra
+// column slice (blockIdx.x == D/16) does b from the s column.
+template <int D>
+__global__ void __launch_bounds__(256)
+memory_finalize_kernel(const float* __restrict__ partials, int G, const float* __restrict__ W_phi,
+                       int r, float decay_n, float* __restrict__ M, float* __restrict__ bstab) {
+  extern __shared__ float fsm[];
+  float* sW = fsm;                 // [r][D]
+  float* sS = sW + r * D;          // [D][16]
+  const int unit = blockIdx.y, sl = blockIdx.x;
+  const int tid = threadIdx.x;
+  const bool bcol = (sl == D / 16);
+  const int ncols = bcol ? 1 : 16;
+  const int col0 = bcol ? D : sl * 16;
+  for (int i = tid; i < r * D / 4; i += 256)
+    reinterpret_cast<float4*>(sW)[i] = __ldg(reinterpret_cast<const float4*>(W_phi) + i);
+  const float* p = partials + (size_t)unit * G * D * (D + 1);
+  for (int i = tid; i < D * ncols; i += 256) {
+    const int dk = i / ncols, cc = i % ncols;
+    float a = 0.f;
+    for (int gg = 0; gg < G; ++gg) a += __ldcg(&p[((size_t)gg * D + dk) * (D + 1) + col0 + cc]);
+    sS[dk * 16 + cc] = a;
+  }
+  __syncthreads();
+  for (int i = tid; i < r * ncols; i += 256) {
+    const int ri = i / ncols, cc = i % ncols;
+    float a = 0.f;
+#pragma unroll 8
+    for (int dk = 0; dk < D; ++dk) a = fmaf(sW[ri * D + dk], sS[dk * 16 + cc], a);
+    if (bcol) {
+      float* bp = bstab + (size_t)unit * r + ri;
+      *bp = fmaf(*bp, decay_n, a);
+    } else {
+      float* mp = M + ((size_t)unit * r + ri) * D + col0 + cc;
+      *mp = fmaf(*mp, decay_n, a);
+    }
   }
 }
 
 }  // namespace
 
+// Number of runs the evicted tokens are split into per (sequence, KV head):
+// about two CTAs per SM, each run a whole number of `chunk` tokens.
 int memory_groups(int batch, int n_kv_heads, int n_e, int chunk) {
   const int units = batch * n_kv_heads;
   const int chunks = (n_e + chunk - 1) / chunk;
-  int G = (2 * 148 + units - 1) / units;
+  int G = (2 * 148 + units / 2) / units;
   if (G > chunks) G = chunks;
   if (G > kMemMaxGroups) G = kMemMaxGroups;
   if (G < 1) G = 1;
@@ -155,16 +291,19 @@ cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, 
   const int G = memory_groups(batch, Hkv, n_e, chunk);
   const int chunks = (n_e + chunk - 1) / chunk;
   const int tokens_per_group = ((chunks + G - 1) / G) * chunk;
-  dim3 grid(G, Hkv, batch);
-  const size_t smem = ((size_t)r * D + 2 * kSub * D + kSub * r) * sizeof(float);
+  const int Gused = (n_e + tokens_per_group - 1) / tokens_per_group;   // no empty runs
+  dim3 grid(Gused, Hkv, batch);
+  const float log2lam = (float)log2((double)c.cfg.lambda);
   cudaError_t e = cudaSuccess;
 #define IMEM_MEM(TT, DD)                                                                       \
   do {                                                                                         \
-    auto kfn = memory_partial_kernel<TT, DD>;                                                  \
-    e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);     \
+    auto kfn = memory_tc_kernel<TT, DD>;                                                       \
+    e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,                 \
+                             MemTile<DD>::SMEM);                                               \
     if (e != cudaSuccess) return e;                                                            \
-    kfn<<<grid, kMemThreads, smem, st>>>((const TT*)K, (const TT*)V, idx_e, n_e, L, Hkv,       \
-                                         c.W_phi, r, c.cfg.lambda, tokens_per_group, partials); \
+    kfn<<<grid, kMemThreads, MemTile<DD>::SMEM, st>>>((const TT*)K, (const TT*)V, idx_e, n_e,  \
+                                                      L, Hkv, log2lam, tokens_per_group,       \
+                                                      partials, c.err);                        \
   } while (0)
   if (c.cfg.dtype == IMEM_BF16) {
     if (D == 128) IMEM_MEM(__nv_bfloat16, 128); else IMEM_MEM(__nv_bfloat16, 64);
@@ -175,7 +314,17 @@ cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, 
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const float decay_n = (float)pow((double)c.cfg.lambda, (double)n_e);
-  memory_finalize_kernel<<<batch * Hkv, 256, 0, st>>>(partials, G, r, D, decay_n, M, bstab);
+  dim3 fgrid(D / 16 + 1, batch * Hkv);
+  const size_t fsmem = ((size_t)r * D + (size_t)D * 16) * sizeof(float);
+  if (D == 128) {
+    e = cudaFuncSetAttribute(memory_finalize_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem);
+    if (e != cudaSuccess) return e;
+    memory_finalize_kernel<128><<<fgrid, 256, fsmem, st>>>(partials, Gused, c.W_phi, r, decay_n, M, bstab);
+  } else {
+    e = cudaFuncSetAttribute(memory_finalize_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem);
+    if (e != cudaSuccess) return e;
+    memory_finalize_kernel<64><<<fgrid, 256, fsmem, st>>>(partials, Gused, c.W_phi, r, decay_n, M, bstab);
+  }
   return cudaGetLastError();
 }
 

@@ -30,8 +30,8 @@ template <typename T>
 __global__ void __launch_bounds__(kPThreads)
 prologue_kernel(const T* __restrict__ X, const T* __restrict__ Q, const T* __restrict__ W_iq,
                 const T* __restrict__ W_ik, const T* __restrict__ w_ig, int L, int H, int Hq,
-                int D, int dI, int q_begin, int q_end, float* __restrict__ qt,
-                float* __restrict__ kh, float* __restrict__ running_max) {
+                int D, int dI, int q_begin, int q_end, __nv_bfloat16* __restrict__ qt,
+                __nv_bfloat16* __restrict__ kh, float* __restrict__ running_max) {
   extern __shared__ float sm[];
   const int NC = dI + Hq;                 // key features + gate logits
   float* sX = sm;                         // [kTok][kHChunk]
@@ -81,7 +81,8 @@ prologue_kernel(const T* __restrict__ X, const T* __restrict__ Q, const T* __res
     ss = warp_sum(ss);
     const float inv = rsqrtf(ss / dI + 1e-6f);
     if (t < q_end)
-      for (int j = lane; j < dI; j += 32) kh[((size_t)bi * L + t) * dI + j] = sKG[tt * NC + j] * inv;
+      for (int j = lane; j < kIdxPad; j += 32)
+        kh[((size_t)bi * L + t) * kIdxPad + j] = __float2bfloat16_rn(j < dI ? sKG[tt * NC + j] * inv : 0.f);
   }
 
   // ---- qtilde: per head projection, RMS norm, gate, sum
@@ -125,7 +126,11 @@ prologue_kernel(const T* __restrict__ X, const T* __restrict__ Q, const T* __res
   for (int a = 0; a * kPThreads + tid < n_q; ++a) {
     const int o = a * kPThreads + tid, tt = o / dI, j = o % dI;
     const int t = t0 + tt;
-    if (t < q_end) qt[((size_t)bi * L + t) * dI + j] = qacc[a];
+    if (t < q_end) qt[((size_t)bi * L + t) * kIdxPad + j] = __float2bfloat16_rn(qacc[a]);
+  }
+  for (int i = tid; i < kTok * (kIdxPad - dI); i += kPThreads) {   // zero padding
+    const int tt = i / (kIdxPad - dI), j = dI + i % (kIdxPad - dI);
+    if (t0 + tt < q_end) qt[((size_t)bi * L + t0 + tt) * kIdxPad + j] = __float2bfloat16_rn(0.f);
   }
   if (tid < kTok && t0 + tid < q_end) running_max[(size_t)bi * L + t0 + tid] = -INFINITY;
 }
@@ -133,8 +138,8 @@ prologue_kernel(const T* __restrict__ X, const T* __restrict__ Q, const T* __res
 }  // namespace
 
 cudaError_t launch_prologue(const Ctx& c, int batch, int L, const void* X, const void* Q,
-                            int q_begin, int q_end, float* qt, float* kh, float* running_max,
-                            cudaStream_t st) {
+                            int q_begin, int q_end, __nv_bfloat16* qt, __nv_bfloat16* kh,
+                            float* running_max, cudaStream_t st) {
   const int H = c.cfg.hidden, Hq = c.cfg.n_q_heads, D = c.cfg.head_dim, dI = c.cfg.idx_dim;
   const int NC = dI + Hq;
   const size_t smem = ((size_t)kTok * kHChunk + kHChunk * NC + kTok * NC + D * dI + kTok * D +

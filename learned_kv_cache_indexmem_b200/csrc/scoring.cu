@@ -8,89 +8,272 @@
 // the O(L^2) matrix); §2.A pre-eviction (queries arrive in ranges).
 //
 //   I[t] = max(I[t], max_{s in [max(t, q_begin), q_end)} qtilde_s . khat_t)
+//
+// With the gated head sum folded into qtilde (exact, see prologue.cu) the
+// contraction is over d_I = 64. Keys sit on the MMA M dimension (TMEM lanes)
+// and queries on N, so each epilogue thread owns one key and the pooling is a
+// register max over its TMEM row.
+//
+// Persistent kernel, one CTA per SM. Work item = (sequence, block of 256
+// keys, tile of 128 queries); the causal items of all sequences are
+// enumerated in closed form and split evenly over the CTAs. Per item the MMA
+// thread issues 2 x 4 tcgen05.mma (M=128 keys, N=128 queries, K=16) from
+// TMA-loaded, 128B-swizzled K-major tiles into one of two 256-column TMEM
+// accumulators; eight epilogue warps drain the other one with tcgen05.ld
+// and masked maxima, and flush a key's maximum with an atomic float max when
+// its key block ends (several CTAs may share a key block).
 #include "common.cuh"
 #include "internal.h"
+#include "tc.cuh"
 
 namespace imem {
 namespace {
 
-constexpr int kKT = 64;   // keys per CTA
-constexpr int kQT = 64;   // queries per step
-constexpr int kSThreads = 256;
+constexpr int kKB = 256;        // keys per key block
+constexpr int kQT = 128;        // queries per tile
+constexpr int kBStages = 4;     // query-tile ring
+constexpr int kEpiWarps = 8;
+constexpr int kScThreads = 64 + kEpiWarps * 32;
+constexpr int kABytes = kKB * 128;    // 256 rows x 128 B
+constexpr int kBBytes = kQT * 128;    // 128 rows x 128 B
+constexpr int kScSmem = 2 * kABytes + kBStages * kBBytes + 1024 + 256;
 
-__global__ void __launch_bounds__(kSThreads)
-scoring_kernel(const float* __restrict__ qt, const float* __restrict__ kh, int L, int dI,
-               int q_begin, int q_end, float* __restrict__ running_max) {
-  extern __shared__ float sm[];
-  float* sK = sm;                    // [dI][kKT]
-  float* sQ = sK + dI * kKT;         // [dI][kQT]
-  float* sRed = sQ + dI * kQT;       // [16][kKT]
-  const int bi = blockIdx.y;
-  const int k0 = blockIdx.x * kKT;
-  const int tid = threadIdx.x;
-  const int tk = tid % 16, tq = tid / 16;
+// Closed-form enumeration of the causal work items of one sequence.
+struct Sched {
+  int q_begin, q_end, nkb, kb0, N0, Qc;
+  long long per_seq;
 
-  for (int i = tid; i < kKT * dI; i += kSThreads) {
-    const int kk = i / dI, j = i % dI;
-    const int t = k0 + kk;
-    sK[j * kKT + kk] = (t < q_end) ? kh[((size_t)bi * L + t) * dI + j] : 0.f;
+  __host__ __device__ void init(int qb, int qe) {
+    q_begin = qb; q_end = qe;
+    nkb = (qe + kKB - 1) / kKB;
+    kb0 = qb / kKB;
+    N0 = (qe - qb + kQT - 1) / kQT;
+    Qc = (qe + kQT - 1) / kQT;
+    per_seq = prefix(nkb);
   }
-  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-  const int s_first = max(q_begin, k0);
-  for (int s0 = s_first; s0 < q_end; s0 += kQT) {
-    __syncthreads();
-    for (int i = tid; i < kQT * dI; i += kSThreads) {
-      const int qq = i / dI, j = i % dI;
-      const int s = s0 + qq;
-      sQ[j * kQT + qq] = (s < q_end) ? qt[((size_t)bi * L + s) * dI + j] : 0.f;
+  // query tiles of key block kb
+  __host__ __device__ int nq(int kb) const { return kb <= kb0 ? N0 : Qc - 2 * kb; }
+  // items of key blocks [0, kb)
+  __host__ __device__ long long prefix(int kb) const {
+    if (kb <= kb0 + 1) return (long long)kb * N0;
+    const long long k1 = kb0 + 1, k2 = kb - 1, cnt = k2 - k1 + 1;
+    return (long long)(kb0 + 1) * N0 + cnt * Qc - (k1 + k2) * cnt;
+  }
+  __host__ __device__ int qstart(int kb) const { return kb * kKB > q_begin ? kb * kKB : q_begin; }
+};
+
+struct Cursor {
+  int seq, kb, j;
+  __device__ void locate(const Sched& sc, long long item) {
+    seq = (int)(item / sc.per_seq);
+    const long long rem = item - (long long)seq * sc.per_seq;
+    int lo = 0, hi = sc.nkb - 1;   // largest kb with prefix(kb) <= rem
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (sc.prefix(mid) <= rem) lo = mid; else hi = mid - 1;
     }
-    __syncthreads();
-    float acc[4][4] = {};
-    for (int j = 0; j < dI; ++j) {
-      const float4 kv = *reinterpret_cast<const float4*>(&sK[j * kKT + tk * 4]);
-      const float4 qv = *reinterpret_cast<const float4*>(&sQ[j * kQT + tq * 4]);
-      const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
-      const float qq[4] = {qv.x, qv.y, qv.z, qv.w};
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(kk[a], qq[b], acc[a][b]);
+    kb = lo;
+    j = (int)(rem - sc.prefix(kb));
+  }
+  __device__ void next(const Sched& sc) {
+    if (++j == sc.nq(kb)) {
+      j = 0;
+      if (++kb == sc.nkb) { kb = 0; ++seq; }
     }
-#pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const int t = k0 + tk * 4 + a;
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const int s = s0 + tq * 4 + b;
-        if (s >= t && s < q_end) mx[a] = fmaxf(mx[a], acc[a][b]);
+  }
+};
+
+__global__ void __launch_bounds__(kScThreads, 1)
+scoring_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                  int L, int q_begin, int q_end, long long total_items,
+                  float* __restrict__ running_max, int* __restrict__ err) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sA = tc::smem_addr(smem);                 // 2 key blocks
+  const uint32_t sB = sA + 2 * kABytes;                     // kBStages query tiles
+  const uint32_t bar = sB + kBStages * kBBytes;
+  const uint32_t a_full = bar, a_empty = bar + 16, b_full = bar + 32,
+                 b_empty = b_full + 8 * kBStages, t_full = b_empty + 8 * kBStages,
+                 t_empty = t_full + 16;
+  __shared__ uint32_t s_tmem;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  Sched sc;
+  sc.init(q_begin, q_end);
+  const long long per_cta = (total_items + gridDim.x - 1) / gridDim.x;
+  const long long i_begin = (long long)blockIdx.x * per_cta;
+  const long long i_end = min(total_items, i_begin + per_cta);
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(a_full + 8 * i, 1);
+      tc::mbar_init(a_empty + 8 * i, 1);
+      tc::mbar_init(t_full + 8 * i, 1);
+      tc::mbar_init(t_empty + 8 * i, kEpiWarps);
+    }
+    for (int i = 0; i < kBStages; ++i) {
+      tc::mbar_init(b_full + 8 * i, 1);
+      tc::mbar_init(b_empty + 8 * i, 1);
+    }
+    tc::fence_mbar_init();
+    tc::prefetch_tmap(&map_q);
+    tc::prefetch_tmap(&map_k);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tc::smem_addr(&s_tmem), 512);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = s_tmem;
+
+  if (i_begin < i_end) {
+    if (warp == 0 && lane == 0) {
+      // ---------------- TMA producer
+      Cursor cu;
+      cu.locate(sc, i_begin);
+      long long prev = -1;
+      int kbi = -1;
+      for (long long i = i_begin; i < i_end; ++i) {
+        const long long kid = (long long)cu.seq * sc.nkb + cu.kb;
+        if (kid != prev) {
+          ++kbi;
+          const int ab = kbi & 1;
+          if (kbi >= 2 && !tc::mbar_wait(a_empty + 8 * ab, ((kbi >> 1) - 1) & 1)) {
+            record_error(err, DEV_TIMEOUT);
+            break;
+          }
+          tc::mbar_expect_tx(a_full + 8 * ab, kABytes);
+          tc::tma_load_2d(sA + ab * kABytes, &map_k, a_full + 8 * ab, 0, cu.seq * L + cu.kb * kKB);
+          prev = kid;
+        }
+        const int n = (int)(i - i_begin);
+        const int st = n % kBStages;
+        if (n >= kBStages && !tc::mbar_wait(b_empty + 8 * st, ((n / kBStages) - 1) & 1)) {
+          record_error(err, DEV_TIMEOUT);
+          break;
+        }
+        tc::mbar_expect_tx(b_full + 8 * st, kBBytes);
+        tc::tma_load_2d(sB + st * kBBytes, &map_q, b_full + 8 * st, 0,
+                        cu.seq * L + sc.qstart(cu.kb) + cu.j * kQT);
+        cu.next(sc);
       }
-    }
-  }
-  __syncthreads();
+    } else if (warp == 1 && lane == 0) {
+      // ---------------- MMA issuer
+      constexpr uint32_t IDESC = tc::idesc(tc::kFmtBF16, 128, kQT, false, false);
+      Cursor cu;
+      cu.locate(sc, i_begin);
+      long long prev = -1;
+      int kbi = -1;
+      for (long long i = i_begin; i < i_end; ++i) {
+        const long long kid = (long long)cu.seq * sc.nkb + cu.kb;
+        const int n = (int)(i - i_begin);
+        if (kid != prev) {
+          ++kbi;
+          if (!tc::mbar_wait(a_full + 8 * (kbi & 1), (kbi >> 1) & 1)) { record_error(err, DEV_TIMEOUT); break; }
+          prev = kid;
+        }
+        const int ab = kbi & 1;
+        const int st = n % kBStages, tb = n & 1;
+        if (!tc::mbar_wait(b_full + 8 * st, (n / kBStages) & 1)) { record_error(err, DEV_TIMEOUT); break; }
+        if (n >= 2 && !tc::mbar_wait(t_empty + 8 * tb, ((n >> 1) - 1) & 1)) { record_error(err, DEV_TIMEOUT); break; }
+        tc::fence_after();
 #pragma unroll
-  for (int a = 0; a < 4; ++a) sRed[tq * kKT + tk * 4 + a] = mx[a];
-  __syncthreads();
-  if (tid < kKT) {
-    const int t = k0 + tid;
-    if (t < q_end) {
-      float m = running_max[(size_t)bi * L + t];
-      for (int i = 0; i < 16; ++i) m = fmaxf(m, sRed[i * kKT + tid]);
-      running_max[(size_t)bi * L + t] = m;
+        for (int kt = 0; kt < 2; ++kt) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad = tc::sdesc_sw128(sA + ab * kABytes + kt * (kABytes / 2) + k * 32, 16, 1024);
+            const uint64_t bd = tc::sdesc_sw128(sB + st * kBBytes + k * 32, 16, 1024);
+            tc::mma_f16(tmem + tb * 256 + kt * 128, ad, bd, IDESC, k > 0 ? 1u : 0u);
+          }
+        }
+        tc::mma_commit(b_empty + 8 * st);
+        tc::mma_commit(t_full + 8 * tb);
+        cu.next(sc);
+        const long long nkid = (long long)cu.seq * sc.nkb + cu.kb;
+        if (i + 1 == i_end || nkid != kid) tc::mma_commit(a_empty + 8 * ab);
+      }
+    } else if (warp >= 2) {
+      // ---------------- epilogue: masked row maxima, flushed per key block
+      const int e = warp - 2;
+      const int quarter = warp & 3;        // TMEM lanes this warp may read
+      const int kt = e >> 2;               // key tile of the block (TMEM columns)
+      Cursor cu;
+      cu.locate(sc, i_begin);
+      long long prev = -1;
+      int pseq = 0, pkb = 0;
+      float runmax = -INFINITY;
+      auto flush = [&](int seq, int kb) {
+        const int t = kb * kKB + kt * 128 + quarter * 32 + lane;
+        if (t < q_end && runmax != -INFINITY) atomic_max_float(&running_max[(size_t)seq * L + t], runmax);
+      };
+      for (long long i = i_begin; i < i_end; ++i) {
+        const long long kid = (long long)cu.seq * sc.nkb + cu.kb;
+        if (kid != prev) {
+          if (prev >= 0) flush(pseq, pkb);
+          runmax = -INFINITY;
+          prev = kid; pseq = cu.seq; pkb = cu.kb;
+        }
+        const int n = (int)(i - i_begin);
+        const int tb = n & 1;
+        if (!tc::mbar_wait(t_full + 8 * tb, (n >> 1) & 1)) { record_error(err, DEV_TIMEOUT); break; }
+        tc::fence_after();
+        const int t = cu.kb * kKB + kt * 128 + quarter * 32 + lane;
+        const int s0 = sc.qstart(cu.kb) + cu.j * kQT;
+        const bool full = (s0 >= t) && (s0 + kQT <= q_end);
+        const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + tb * 256 + kt * 128;
+#pragma unroll
+        for (int c = 0; c < kQT / 32; ++c) {
+          float v[32];
+          tc::tmem_ld32(base + c * 32, v);
+          if (full) {
+#pragma unroll
+            for (int x = 0; x < 32; x += 2) runmax = fmaxf(runmax, fmaxf(v[x], v[x + 1]));
+          } else {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) {
+              const int s = s0 + c * 32 + x;
+              if (s >= t && s < q_end) runmax = fmaxf(runmax, v[x]);
+            }
+          }
+        }
+        tc::fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(t_empty + 8 * tb);
+        cu.next(sc);
+      }
+      if (prev >= 0) flush(pseq, pkb);
     }
   }
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 1) tc::tmem_dealloc(tmem, 512);
 }
 
 }  // namespace
 
-cudaError_t launch_scoring(const Ctx& c, int batch, int L, const float* qt, const float* kh,
-                           float* running_max, int q_begin, int q_end, cudaStream_t st) {
-  const int dI = c.cfg.idx_dim;
-  const size_t smem = ((size_t)dI * kKT + dI * kQT + 16 * kKT) * sizeof(float);
-  dim3 grid((q_end + kKT - 1) / kKT, batch);
-  cudaError_t e = cudaFuncSetAttribute(scoring_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
-  if (e != cudaSuccess) return e;
-  scoring_kernel<<<grid, kSThreads, smem, st>>>(qt, kh, L, dI, q_begin, q_end, running_max);
+cudaError_t launch_scoring(const Ctx& c, int batch, int L, const __nv_bfloat16* qt,
+                           const __nv_bfloat16* kh, float* running_max, int q_begin, int q_end,
+                           cudaStream_t st) {
+  CUtensorMap mq, mk;
+  if (!make_tmap_rows64(c, &mq, qt, (uint64_t)batch * L, kQT)) return cudaErrorInvalidValue;
+  if (!make_tmap_rows64(c, &mk, kh, (uint64_t)batch * L, kKB)) return cudaErrorInvalidValue;
+  Sched sc;
+  sc.init(q_begin, q_end);
+  const long long total = sc.per_seq * batch;
+  int grid = c.num_sms;
+  if (total < grid) grid = (int)total;
+  static bool attr_set[64] = {};
+  if (!attr_set[c.device & 63]) {
+    cudaError_t e = cudaFuncSetAttribute(scoring_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kScSmem);
+    if (e != cudaSuccess) return e;
+    attr_set[c.device & 63] = true;
+  }
+  scoring_tc_kernel<<<grid, kScThreads, kScSmem, st>>>(mq, mk, L, q_begin, q_end, total,
+                                                       running_max, c.err);
   return cudaGetLastError();
 }
 

@@ -15,7 +15,7 @@ from learned_kv_cache_indexmem_b200 import binding, synth
 from oracle import indexmem_oracle as om
 
 from .parity import (Case, check_decode, check_memory, check_scores, ill_conditioned, to_np,
-                     SCORE_TOL)
+                     propagated_allowance, SCORE_TOL)
 
 pytestmark = pytest.mark.gpu
 
@@ -229,7 +229,8 @@ def test_end_to_end_parity(cuda_device, name, B, steps):
     KR, VR = om.compact(to_np(case.in_cpu["K"]), to_np(case.in_cpu["V"]), R, cap)
     M_ref, b_ref = om.memory_update(case.in_cpu["K"], case.in_cpu["V"], E, case.w_cpu["W_phi"],
                                     case.shape.lam)
-    check_memory(to_np(st.M), to_np(st.bstab), M_ref, b_ref, name)
+    M_gpu, b_gpu = to_np(st.M), to_np(st.bstab)
+    check_memory(M_gpu, b_gpu, M_ref, b_ref, name)
     W_phi = case.w_cpu["W_phi"].numpy().astype(np.float64)
     w_gate = case.w_cpu["w_gate"].numpy().astype(np.float64)
     group = case.shape.n_q_heads // case.shape.n_kv_heads
@@ -242,5 +243,10 @@ def test_end_to_end_parity(cuda_device, name, B, steps):
             KR[bi, clen[bi]] = knc[bi]
             VR[bi, clen[bi]] = vnc[bi]
         clen = new_len
-        check_decode(outs[s], o_ref, ill_conditioned(b_ref, qc, W_phi, group), "%s step %d" % (name, s))
+        # the memory state is checked above to its own tolerance; its admissible
+        # error reaches the output through the readout's conditioning
+        extra = propagated_allowance(qc, M_ref, b_ref, M_gpu - M_ref, b_gpu - b_ref, W_phi,
+                                     w_gate, group)
+        check_decode(outs[s], o_ref, ill_conditioned(b_ref, qc, W_phi, group),
+                     "%s step %d" % (name, s), extra=extra)
     lay.close()
