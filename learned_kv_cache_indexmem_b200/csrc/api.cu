@@ -28,13 +28,9 @@ Workspace workspace_layout(const Ctx& c, int batch, int L) {
   Workspace w;
   size_t off = 0;
   const size_t units = (size_t)batch * c.cfg.n_kv_heads;
-  w.dec_cnt_off = off;
-  off = align_up(off + (units + batch) * sizeof(int), 256);
-  // decode: per unit up to kDecodeMaxSplits softmax states of the GQA group
-  // plus the readout
-  w.dec_part_off = off;
-  off = align_up(off + units * (kDecodeMaxSplits + 1) * c.group *
-                           (size_t)(c.cfg.head_dim + 4) * sizeof(float), 256);
+  w.dec_cnt_off = off;                        // one counter per sequence
+  off = align_up(off + (size_t)batch * sizeof(int), 256);
+  w.dec_part_off = off;                       // (unused: decode merges in shared memory)
   // memory partials: at most (2*148 + units) runs of a d x (d+1) sum [S | s]
   w.mem_part_off = off;
   off = align_up(off + (2 * 148 + units) * (size_t)c.cfg.head_dim * (c.cfg.head_dim + 1) *
@@ -98,8 +94,6 @@ imem_status check_device(const Ctx& c) {
   return dev == c.device ? IMEM_OK : IMEM_ERR_INVALID_ARG;
 }
 
-size_t dtype_size(int dt) { return dt == IMEM_BF16 ? 2 : 4; }
-
 }  // namespace
 
 extern "C" {
@@ -162,22 +156,12 @@ imem_status imem_init(const imem_config* cfg, const imem_weights* w, imem_ctx** 
       return IMEM_ERR_CUDA;
     }
   }
-  const size_t es = dtype_size(k.dtype);
-  const size_t n_iq = (size_t)k.n_q_heads * k.head_dim * k.idx_dim;
-  const size_t n_ik = (size_t)k.hidden * k.idx_dim;
-  const size_t n_ig = (size_t)k.hidden * k.n_q_heads;
   const size_t n_phi = (size_t)k.mem_r * k.head_dim;
   const size_t n_g = (size_t)k.n_q_heads * k.head_dim;
-  cudaError_t e = cudaSuccess;
-  if (e == cudaSuccess) e = cudaMalloc(&c.W_iq, n_iq * es);
-  if (e == cudaSuccess) e = cudaMalloc(&c.W_ik, n_ik * es);
-  if (e == cudaSuccess) e = cudaMalloc(&c.w_ig, n_ig * es);
+  cudaError_t e = imem::pack_indexer_weights(c, w->W_idx_q, w->W_idx_k, w->w_idx_g);
   if (e == cudaSuccess) e = cudaMalloc((void**)&c.W_phi, n_phi * sizeof(float));
   if (e == cudaSuccess) e = cudaMalloc((void**)&c.w_gate, n_g * sizeof(float));
   if (e == cudaSuccess) e = cudaMalloc((void**)&c.err, sizeof(int));
-  if (e == cudaSuccess) e = cudaMemcpy(c.W_iq, w->W_idx_q, n_iq * es, cudaMemcpyDeviceToDevice);
-  if (e == cudaSuccess) e = cudaMemcpy(c.W_ik, w->W_idx_k, n_ik * es, cudaMemcpyDeviceToDevice);
-  if (e == cudaSuccess) e = cudaMemcpy(c.w_ig, w->w_idx_g, n_ig * es, cudaMemcpyDeviceToDevice);
   if (e == cudaSuccess) e = cudaMemcpy(c.W_phi, w->W_phi, n_phi * sizeof(float), cudaMemcpyDeviceToDevice);
   if (e == cudaSuccess) e = cudaMemcpy(c.w_gate, w->w_gate, n_g * sizeof(float), cudaMemcpyDeviceToDevice);
   if (e == cudaSuccess) e = cudaMemset(c.err, 0, sizeof(int));
@@ -194,9 +178,8 @@ void imem_destroy(imem_ctx* h) {
   if (!h) return;
   Ctx& c = h->c;
   cudaDeviceSynchronize();
-  cudaFree(c.W_iq);
-  cudaFree(c.W_ik);
-  cudaFree(c.w_ig);
+  cudaFree(c.WcT);
+  cudaFree(c.WqT);
   cudaFree(c.W_phi);
   cudaFree(c.w_gate);
   cudaFree(c.err);

@@ -28,6 +28,7 @@
 #include "common.cuh"
 #include "internal.h"
 
+#include <cooperative_groups.h>
 #include <math.h>
 #include <type_traits>
 
@@ -300,33 +301,57 @@ __device__ void attend_f32(const float* __restrict__ Kb, const float* __restrict
   }
 }
 
-// Merge the per-warp states s_part[0..3][g] into s_part[0][g] (needs the
-// block's threads; ends with a barrier).
+// Merge the per-warp states w_part[0..3][g] into dst[g] (all threads of the
+// block; ends with a barrier).
 template <int D, int G>
-__device__ void merge_warps(Partial<D> (*s_part)[G]) {
+__device__ void merge_warps(const Partial<D> (*w_part)[G], Partial<D>* dst) {
   const int tid = threadIdx.x;
   __syncthreads();
   for (int i = tid; i < G * D; i += kThreads) {
     const int g = i / D, c = i % D;
     float mx = -INFINITY;
-    for (int w = 0; w < 4; ++w) mx = fmaxf(mx, s_part[w][g].m);
+    for (int w = 0; w < 4; ++w) mx = fmaxf(mx, w_part[w][g].m);
     float o = 0.f;
     for (int w = 0; w < 4; ++w)
-      if (s_part[w][g].m != -INFINITY) o += s_part[w][g].o[c] * exp2f(s_part[w][g].m - mx);
-    s_part[0][g].o[c] = o;
+      if (w_part[w][g].m != -INFINITY) o += w_part[w][g].o[c] * exp2f(w_part[w][g].m - mx);
+    dst[g].o[c] = o;
   }
-  __syncthreads();
   if (tid < G) {
     float mx = -INFINITY;
-    for (int w = 0; w < 4; ++w) mx = fmaxf(mx, s_part[w][tid].m);
+    for (int w = 0; w < 4; ++w) mx = fmaxf(mx, w_part[w][tid].m);
     float l = 0.f;
     for (int w = 0; w < 4; ++w)
-      if (s_part[w][tid].m != -INFINITY) l += s_part[w][tid].l * exp2f(s_part[w][tid].m - mx);
-    s_part[0][tid].m = mx;
-    s_part[0][tid].l = l;
+      if (w_part[w][tid].m != -INFINITY) l += w_part[w][tid].l * exp2f(w_part[w][tid].m - mx);
+    dst[tid].m = mx;
+    dst[tid].l = l;
   }
   __syncthreads();
 }
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
+// Dynamic shared memory of one decode CTA (offsets in bytes):
+//   [0, work)        attention stages | per-warp states | readout buffers
+//   [part, part + G * sizeof(Partial<D>))   this CTA's published result,
+//                    read by the other CTAs of the cluster
+template <int D, int G>
+struct DecSmem {
+  static constexpr size_t att(bool bf16) { return bf16 ? (size_t)2 * 2 * kStageRows * D * 2 : 0; }
+  static constexpr size_t warps() { return (size_t)4 * G * sizeof(Partial<D>); }
+  static size_t readout(int r) {
+    return ((size_t)2 * r * D + (size_t)G * r + 2 * G + (size_t)G * D + r) * sizeof(float);
+  }
+  static size_t part_off(bool bf16, int r) {
+    size_t w = att(bf16);
+    if (warps() > w) w = warps();
+    if (readout(r) > w) w = readout(r);
+    return (w + 127) / 128 * 128;
+  }
+  static size_t total(bool bf16, int r) { return part_off(bf16, r) + (size_t)G * sizeof(Partial<D>); }
+};
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads)
@@ -335,86 +360,106 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
               int cap, int Hkv, const float* __restrict__ M, const float* __restrict__ bstab,
               const float* __restrict__ W_phi, const float* __restrict__ w_gate, int r, float eps,
               float gate_override, int use_override, T* __restrict__ out,
-              float* __restrict__ partials, int* __restrict__ counters, int* __restrict__ err) {
+              int* __restrict__ seq_counters, int* __restrict__ err, uint32_t part_off) {
+  namespace cg = cooperative_groups;
   extern __shared__ __align__(128) unsigned char dyn_smem[];
-  const int S = gridDim.x - 1;             // attention splits; CTA S = readout
-  const int sp = blockIdx.x, kh = blockIdx.y, bi = blockIdx.z;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int S = gridDim.x - 1;              // attention CTAs; CTA S = readout
+  const int rank = blockIdx.x;              // the cluster spans blockIdx.x
+  const int kh = blockIdx.y, bi = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int Hq = Hkv * G;
   const int unit = bi * Hkv + kh;
 
-  __shared__ float s_q[G][D];
-  __shared__ Partial<D> s_part[4][G];
-  __shared__ int s_flag;
+  __shared__ __align__(16) float s_q[G][D];
+  __shared__ float s_w[kDecodeMaxSplits][G];
+  __shared__ float s_l[G];
+  Partial<D>* mine = reinterpret_cast<Partial<D>*>(dyn_smem + part_off);
 
-  const int len = cache_len[bi];
-  if (len >= cap) {   // full cache: every CTA of the sequence skips it
-    if (sp == 0 && kh == 0 && tid == 0) record_error(err, DEV_CACHE_FULL);
-    return;
-  }
-  const int n = len + 1;
+  // With programmatic dependent launch this kernel may start while the
+  // previous kernel of the stream is still running: wait for it before
+  // reading anything another kernel may write (q, the cache, cache_len, M, b).
+  griddep_wait();
   for (int i = tid; i < G * D; i += kThreads)
     s_q[i / D][i % D] = Elem<T>::to_f(q[((size_t)bi * Hq + kh * G) * D + i]);
+  const int len = cache_len[bi];
+  if (len >= cap) {   // full cache: the whole cluster (same sequence) skips it
+    if (rank == 0 && kh == 0 && tid == 0) record_error(err, DEV_CACHE_FULL);
+    return;
+  }
+  griddep_launch();
+  const int n = len + 1;
   __syncthreads();
 
-  // workspace of the unit: S softmax states of the group, then the readout
-  Partial<D>* up = reinterpret_cast<Partial<D>*>(partials) + (size_t)unit * (S + 1) * G;
-  float* ro = reinterpret_cast<float*>(up + (size_t)S * G);      // [G][D] g*m
-
   const size_t row_stride = (size_t)Hkv * D;
-  if (sp < S) {
+  if (rank < S) {
     const T* Kb = K_ret + (size_t)bi * cap * row_stride + (size_t)kh * D;
     const T* Vb = V_ret + (size_t)bi * cap * row_stride + (size_t)kh * D;
     const T* kn = k_new + ((size_t)bi * Hkv + kh) * D;
     const T* vn = v_new + ((size_t)bi * Hkv + kh) * D;
-    if (sp == 0) {   // append the new row
+    if (rank == 0) {   // append the new row
       T* kd = K_ret + ((size_t)bi * cap + len) * row_stride + (size_t)kh * D;
       T* vd = V_ret + ((size_t)bi * cap + len) * row_stride + (size_t)kh * D;
       for (int c = tid; c < D; c += kThreads) { kd[c] = kn[c]; vd[c] = vn[c]; }
     }
     const int per = (n + S - 1) / S;
-    const int r0 = min(n, sp * per), r1 = min(n, r0 + per);
+    const int r0 = min(n, rank * per), r1 = min(n, r0 + per);
+    auto* w_part = reinterpret_cast<Partial<D>(*)[G]>(dyn_smem);   // aliases the stages
     if constexpr (std::is_same<T, __nv_bfloat16>::value)
-      attend_bf16<D, G>(Kb, Vb, row_stride, kn, vn, len, r0, r1, s_q, s_part, dyn_smem);
+      attend_bf16<D, G>(Kb, Vb, row_stride, kn, vn, len, r0, r1, s_q, w_part, dyn_smem);
     else
-      attend_f32<D, G>(Kb, Vb, row_stride, kn, vn, len, r0, r1, s_q, s_part);
-    merge_warps<D, G>(s_part);
-    Partial<D>* mine = up + (size_t)sp * G;
-    for (int i = tid; i < G * D; i += kThreads) mine[i / D].o[i % D] = s_part[0][i / D].o[i % D];
-    if (tid < G) { mine[tid].m = s_part[0][tid].m; mine[tid].l = s_part[0][tid].l; }
+      attend_f32<D, G>(Kb, Vb, row_stride, kn, vn, len, r0, r1, s_q, w_part);
+    merge_warps<D, G>(w_part, mine);
   } else {
-    // memory readout for the group's query heads
-    float* sWT = reinterpret_cast<float*>(dyn_smem);        // [D][r+1] = W_phi^T
-    float* su = sWT + D * (r + 1);                           // [G][r]
-    float* sden = su + G * r;                                // [G]
-    float* sgate = sden + G;                                 // [G]
-    const float4* W4 = reinterpret_cast<const float4*>(W_phi);
-#pragma unroll 8
-    for (int i = tid; i < r * D / 4; i += kThreads) {
-      const float4 v = __ldg(W4 + i);
-      const int j = (4 * i) / D, c = (4 * i) % D;
-      sWT[(c + 0) * (r + 1) + j] = v.x;
-      sWT[(c + 1) * (r + 1) + j] = v.y;
-      sWT[(c + 2) * (r + 1) + j] = v.z;
-      sWT[(c + 3) * (r + 1) + j] = v.w;
+    // memory readout: u = W_phi q, m = M^T u / (b.u + eps), g = sigmoid(w_gate . q)
+    float* sW = reinterpret_cast<float*>(dyn_smem);          // [r][D], 16-byte chunks XOR-swizzled
+    float* sM = sW + (size_t)r * D;                           // [r][D]
+    float* swg = sM + (size_t)r * D;                          // [G][D] gate vectors
+    float* sb = swg + G * D;                                  // [r]
+    float* su = sb + r;                                       // [G][r]
+    float* sden = su + G * r;                                 // [G]
+    float* sgate = sden + G;                                  // [G]
+    // one round of asynchronous copies: W_phi, this unit's M and b, the gate rows
+    {
+      const uint32_t wdst = smem_u32(sW), mdst = smem_u32(sM);
+      const float* Mu = M + (size_t)unit * r * D;
+      for (int i = tid; i < r * D / 4; i += kThreads) {
+        const int j = (4 * i) / D, cc = ((4 * i) % D) / 4;
+        cp_async16(wdst + (uint32_t)(j * D + ((cc ^ (j & 7)) * 4)) * 4u, W_phi + 4 * i, true);
+        cp_async16(mdst + (uint32_t)i * 16u, Mu + 4 * i, true);
+      }
+      for (int i = tid; i < G * D / 4; i += kThreads)
+        cp_async16(smem_u32(swg) + (uint32_t)i * 16u, w_gate + (size_t)kh * G * D + 4 * i, true);
+      for (int i = tid; i < r / 4; i += kThreads)
+        cp_async16(smem_u32(sb) + (uint32_t)i * 16u, bstab + (size_t)unit * r + 4 * i, true);
+      cp_async_commit();
+      cp_async_wait<0>();
     }
     __syncthreads();
-    for (int i = tid; i < G * r; i += kThreads) {
-      const int g = i / r, j = i % r;
-      float a = 0.f;
+    // u[g][j] = W_phi[j] . q[g]: one output per thread, four partial sums
+    for (int o = tid; o < G * r; o += kThreads) {
+      const int g = o / r, j = o % r;
+      const float4* wr = reinterpret_cast<const float4*>(sW + (size_t)j * D);
+      const float4* q4 = reinterpret_cast<const float4*>(&s_q[g][0]);
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll 8
-      for (int c = 0; c < D; ++c) a = fmaf(sWT[c * (r + 1) + j], s_q[g][c], a);
-      su[i] = a;
+      for (int cc = 0; cc < D / 4; ++cc) {
+        const float4 w = wr[cc ^ (j & 7)];
+        const float4 x = q4[cc];
+        a0 = fmaf(w.x, x.x, a0);
+        a1 = fmaf(w.y, x.y, a1);
+        a2 = fmaf(w.z, x.z, a2);
+        a3 = fmaf(w.w, x.w, a3);
+      }
+      su[o] = (a0 + a1) + (a2 + a3);
     }
     __syncthreads();
-    const float* bk = bstab + (size_t)unit * r;
     for (int g = warp; g < G; g += kThreads / 32) {
       float a = 0.f;
-      for (int j = lane; j < r; j += 32) a = fmaf(bk[j], su[g * r + j], a);
+      for (int j = lane; j < r; j += 32) a = fmaf(sb[j], su[g * r + j], a);
       a = warp_sum(a);
       float z = 0.f;
-      const float* wg = w_gate + (size_t)(kh * G + g) * D;
-      for (int c = lane; c < D; c += 32) z = fmaf(wg[c], s_q[g][c], z);
+      for (int c = lane; c < D; c += 32) z = fmaf(swg[g * D + c], s_q[g][c], z);
       z = warp_sum(z);
       if (lane == 0) {
         sden[g] = a + eps;
@@ -422,13 +467,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
       }
     }
     __syncthreads();
-    // stage M (r x D) with 16-byte loads in one parallel round, then reduce
-    float* sM = sWT;                                         // W_phi^T no longer needed
-    __syncthreads();
-    const float4* Mk4 = reinterpret_cast<const float4*>(M + (size_t)unit * r * D);
-#pragma unroll 8
-    for (int i = tid; i < r * D / 4; i += kThreads) reinterpret_cast<float4*>(sM)[i] = __ldcg(Mk4 + i);
-    __syncthreads();
+    float* ro = reinterpret_cast<float*>(mine);               // [G][D] = g * m
     for (int c = tid; c < D; c += kThreads) {
       float num[G];
 #pragma unroll
@@ -444,22 +483,13 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     }
   }
 
-  // count this CTA on the unit; the last arrival merges
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_flag = (atomicAdd(&counters[unit], 1) == S);
-  __syncthreads();
-  if (!s_flag) return;
-  __threadfence();
-  if (tid == 0) counters[unit] = 0;
-  // weights of the S partial states (read through L2: written by other SMs);
-  // all (split, head) maxima and normalisers are fetched in one parallel round
-  __shared__ float s_w[kDecodeMaxSplits][G];
+  // every CTA's result is in its shared memory; merge through the cluster
+  cluster.sync();
   __shared__ float s_lp[kDecodeMaxSplits][G];
-  __shared__ float s_l[G];
-  for (int i = tid; i < S * G; i += kThreads) {
-    s_w[i / G][i % G] = __ldcg(&up[i].m);
-    s_lp[i / G][i % G] = __ldcg(&up[i].l);
+  for (int i = tid; i < S * G; i += kThreads) {   // one parallel round of remote reads
+    const Partial<D>* rp = cluster.map_shared_rank(mine, i / G);
+    s_w[i / G][i % G] = rp[i % G].m;
+    s_lp[i / G][i % G] = rp[i % G].l;
   }
   __syncthreads();
   if (tid < G) {
@@ -470,79 +500,106 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
       const float mt = s_w[t2][tid];
       const float w = (mt == -INFINITY) ? 0.f : exp2f(mt - mx);
       s_w[t2][tid] = w;
-      l += w * s_lp[t2][tid];
+      l = fmaf(w, s_lp[t2][tid], l);
     }
     s_l[tid] = l;
   }
   __syncthreads();
-  for (int i = tid; i < G * D; i += kThreads) {
+  // this CTA's share of the G * D outputs; all S remote values are requested
+  // before any is used
+  const int per_out = (G * D + S) / (S + 1);
+  const int o0 = rank * per_out, o1 = min(G * D, o0 + per_out);
+  const float* ro_remote = reinterpret_cast<const float*>(cluster.map_shared_rank(mine, S));
+  for (int i = o0 + tid; i < o1; i += kThreads) {
     const int g = i / D, c = i % D;
+    float vals[kDecodeMaxSplits];
+#pragma unroll
+    for (int t2 = 0; t2 < kDecodeMaxSplits; ++t2)
+      vals[t2] = (t2 < S) ? cluster.map_shared_rank(mine, t2)[g].o[c] : 0.f;
+    const float rv = ro_remote[g * D + c];
     float o = 0.f;
-#pragma unroll 8
-    for (int t2 = 0; t2 < S; ++t2) o = fmaf(s_w[t2][g], __ldcg(&up[t2 * G + g].o[c]), o);
-    const float val = o / s_l[g] + __ldcg(&ro[g * D + c]);
-    out[((size_t)bi * Hq + kh * G + g) * D + c] = Elem<T>::from_f(val);
+#pragma unroll
+    for (int t2 = 0; t2 < kDecodeMaxSplits; ++t2)
+      if (t2 < S) o = fmaf(s_w[t2][g], vals[t2], o);
+    out[((size_t)bi * Hq + kh * G + g) * D + c] = Elem<T>::from_f(o / s_l[g] + rv);
   }
-  __syncthreads();
-  if (tid == 0) {
+  cluster.sync();   // shared memory of every CTA stays alive until all reads are done
+  // the last unit of the sequence advances cache_len (all its CTAs have read it)
+  if (rank == S && tid == 0) {
     __threadfence();
-    int* seq_cnt = counters + (size_t)gridDim.z * Hkv;
-    if (atomicAdd(&seq_cnt[bi], 1) == Hkv - 1) {
-      seq_cnt[bi] = 0;
+    if (atomicAdd(&seq_counters[bi], 1) == Hkv - 1) {
+      seq_counters[bi] = 0;
       cache_len[bi] = len + 1;
     }
   }
 }
 
 template <typename T, int D, int G>
-cudaError_t launch_tg(const Ctx& c, dim3 grid, const void* q, const void* kn, const void* vn,
-                      void* K_ret, void* V_ret, int32_t* cache_len, int cap, const float* M,
-                      const float* bstab, void* out, float* partials, int* counters,
+cudaError_t launch_tg(const Ctx& c, int S, int batch, const void* q, const void* kn,
+                      const void* vn, void* K_ret, void* V_ret, int32_t* cache_len, int cap,
+                      const float* M, const float* bstab, void* out, int* counters,
                       cudaStream_t st) {
+  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   const int r = c.cfg.mem_r;
-  size_t smem_att = std::is_same<T, __nv_bfloat16>::value ? (size_t)2 * 2 * kStageRows * D * 2 : 0;
-  size_t smem_ro = ((size_t)D * (r + 1) + G * r + 2 * G) * sizeof(float);
-  size_t smem = smem_att > smem_ro ? smem_att : smem_ro;
+  const size_t smem = DecSmem<D, G>::total(kBf16, r);
+  const uint32_t part_off = (uint32_t)DecSmem<D, G>::part_off(kBf16, r);
   auto k = decode_kernel<T, D, G>;
   static bool attr_set[64] = {};   // per instantiation and device
   const int dv = c.device & 63;
   if (!attr_set[dv]) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
     attr_set[dv] = true;
   }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(S + 1, c.cfg.n_kv_heads, batch);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S + 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
   const int use_ov = !isnan(c.cfg.gate_override);
-  k<<<grid, kThreads, smem, st>>>((const T*)q, (const T*)kn, (const T*)vn, (T*)K_ret, (T*)V_ret,
-                                  cache_len, cap, c.cfg.n_kv_heads, M, bstab, c.W_phi, c.w_gate, r,
-                                  c.cfg.eps, c.cfg.gate_override, use_ov, (T*)out, partials,
-                                  counters, c.err);
-  return cudaGetLastError();
+  return cudaLaunchKernelEx(&cfg, k, (const T*)q, (const T*)kn, (const T*)vn, (T*)K_ret,
+                            (T*)V_ret, cache_len, cap, c.cfg.n_kv_heads, M, bstab,
+                            (const float*)c.W_phi, (const float*)c.w_gate, r, c.cfg.eps,
+                            c.cfg.gate_override, use_ov, (T*)out, counters, c.err, part_off);
 }
 
 template <typename T, int D>
-cudaError_t launch_t(const Ctx& c, dim3 grid, const void* q, const void* kn, const void* vn,
-                     void* K_ret, void* V_ret, int32_t* cache_len, int cap, const float* M,
-                     const float* bstab, void* out, float* partials, int* counters,
+cudaError_t launch_t(const Ctx& c, int S, int batch, const void* q, const void* kn,
+                     const void* vn, void* K_ret, void* V_ret, int32_t* cache_len, int cap,
+                     const float* M, const float* bstab, void* out, int* counters,
                      cudaStream_t st) {
   switch (c.group) {
-    case 1: return launch_tg<T, D, 1>(c, grid, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, partials, counters, st);
-    case 2: return launch_tg<T, D, 2>(c, grid, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, partials, counters, st);
-    case 4: return launch_tg<T, D, 4>(c, grid, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, partials, counters, st);
-    case 8: return launch_tg<T, D, 8>(c, grid, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, partials, counters, st);
+    case 1: return launch_tg<T, D, 1>(c, S, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
+    case 2: return launch_tg<T, D, 2>(c, S, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
+    case 4: return launch_tg<T, D, 4>(c, S, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
+    case 8: return launch_tg<T, D, 8>(c, S, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
   }
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-// Splits per (sequence, KV head): blocks of about 192 cache rows, at least
-// enough CTAs to cover every SM twice, at most kDecodeMaxSplits.
+// Attention CTAs per (sequence, KV head) = the cluster size minus one: enough
+// CTAs to cover every SM twice, no CTA streaming more than 1024 rows, at least
+// 64 rows per CTA, and a cluster of at most 16 CTAs.
 int decode_splits(int batch, int n_kv_heads, int cap) {
   const int units = batch * n_kv_heads;
-  int S = (cap + kDecodeRowsPerSplit - 1) / kDecodeRowsPerSplit;
-  const int for_sms = (2 * 148 + units - 1) / units;
-  if (S < for_sms) S = for_sms;
-  if (S > kDecodeMaxSplits) S = kDecodeMaxSplits;
+  int S = (2 * 148 + units - 1) / units - 1;
+  const int by_len = (cap + 1023) / 1024;
+  if (S < by_len) S = by_len;
+  const int by_rows = (cap + kStageRows - 1) / kStageRows;
+  if (S > by_rows) S = by_rows;
+  if (S > kDecodeMaxSplits - 1) S = kDecodeMaxSplits - 1;
   if (S < 1) S = 1;
   return S;
 }
@@ -550,16 +607,15 @@ int decode_splits(int batch, int n_kv_heads, int cap) {
 cudaError_t launch_decode(const Ctx& c, int batch, const void* q, const void* k_new,
                           const void* v_new, void* K_ret, void* V_ret, int32_t* cache_len,
                           int cap, const float* M, const float* bstab, void* out,
-                          float* partials, int* counters, cudaStream_t st) {
+                          float* /*partials*/, int* counters, cudaStream_t st) {
   const int S = decode_splits(batch, c.cfg.n_kv_heads, cap);
-  dim3 grid(S + 1, c.cfg.n_kv_heads, batch);
   const int D = c.cfg.head_dim;
   if (c.cfg.dtype == IMEM_BF16) {
-    if (D == 128) return launch_t<__nv_bfloat16, 128>(c, grid, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, partials, counters, st);
-    if (D == 64) return launch_t<__nv_bfloat16, 64>(c, grid, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, partials, counters, st);
+    if (D == 128) return launch_t<__nv_bfloat16, 128>(c, S, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
+    if (D == 64) return launch_t<__nv_bfloat16, 64>(c, S, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
   } else {
-    if (D == 128) return launch_t<float, 128>(c, grid, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, partials, counters, st);
-    if (D == 64) return launch_t<float, 64>(c, grid, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, partials, counters, st);
+    if (D == 128) return launch_t<float, 128>(c, S, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
+    if (D == 64) return launch_t<float, 64>(c, S, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -19,9 +19,9 @@ struct Ctx {
   int device;
   int group;            // Hq / Hkv
   // repacked weights (device, owned)
-  void* W_iq;           // [Hq, d, dI] model dtype (as given)
-  void* W_ik;           // [H, dI] model dtype (as given)
-  void* w_ig;           // [H, Hq] model dtype (as given)
+  void* WcT;            // [N1, H] model dtype: [W_ik | w_ig]^T, zero rows up to N1
+  void* WqT;            // [Hq * dI, d] model dtype: W_iq[h]^T stacked by head
+  int N1;               // dI + Hq rounded up to 16
   float* W_phi;         // [r, d]
   float* w_gate;        // [Hq, d]
   int* err;             // device error word
@@ -47,11 +47,14 @@ struct Workspace {
   size_t total;
 };
 
-constexpr int kDecodeMaxSplits = 64;
+constexpr int kDecodeMaxSplits = 16;          // CTAs per decode cluster (max)
 constexpr int kDecodeRowsPerSplit = 192;   // cache rows per decode CTA (target)
 constexpr int kMemMaxGroups = 64;
 
 Workspace workspace_layout(const Ctx& c, int batch, int L);
+
+// Repacks the indexer weights K-major into c.WcT / c.WqT (allocates them).
+cudaError_t pack_indexer_weights(Ctx& c, const void* W_iq, const void* W_ik, const void* w_ig);
 
 // ---- launchers (return cudaGetLastError()) ----------------------------------
 

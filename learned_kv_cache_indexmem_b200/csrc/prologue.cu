@@ -14,155 +14,343 @@
 // A[s,t] = sum_h gamma_sh (qhat_sh . khat_t)/sqrt(dI) = qtilde_s . khat_t exactly,
 // so the scoring pass contracts over dI only.
 //
+// Tensor-core kernel, persistent over 128-token tiles. Per tile:
+//   GEMM1 (tcgen05, K = hidden): [kI | gate logits] = X_tile [W_ik | w_ig]
+//   GEMM2 (tcgen05, K = d) per head h: qI_h = Q_tile[:, h] W_iq[h]
+// X and Q tiles and the repacked K-major weights arrive by TMA through a
+// 6-stage ring; GEMM1 accumulates in TMEM columns [0, 128), the per-head
+// GEMM2 results cycle through a ring of TMEM buffers in [128, 512). Four
+// epilogue warps (one token row per thread) normalise the key, then fold each
+// head into qtilde in registers (RMS norm, gate, 1/sqrt(dI)) as soon as its
+// buffer is ready, and write bf16 rows of kIdxPad features.
+// bf16 inputs use kind::f16, fp32 inputs kind::tf32 (same 128-byte rows).
 // Also resets the running maximum of the tokens in the range to -inf (those
 // keys get their first queries in this range).
 #include "common.cuh"
 #include "internal.h"
+#include "tc.cuh"
+
+#include <type_traits>
 
 namespace imem {
 namespace {
 
-constexpr int kTok = 32;
-constexpr int kPThreads = 256;
-constexpr int kHChunk = 64;
+constexpr int kTileM = 128;
+constexpr int kNSt = 6;
+constexpr int kStageA = 128 * 128;   // 128 rows x 128 bytes
+constexpr int kStageB = 128 * 128;
+constexpr int kPThreads = 192;       // producer, MMA, 4 epilogue warps
+constexpr int kProSmem = kNSt * (kStageA + kStageB) + 1024 + 512;
+constexpr int kD1Cols = 128;         // TMEM columns reserved for GEMM1
+
+__device__ __forceinline__ uint32_t tmem_ld1(uint32_t taddr) {
+  uint32_t r;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\ntcgen05.wait::ld.sync.aligned;\n"
+               : "=r"(r) : "r"(taddr) : "memory");
+  return r;
+}
 
 template <typename T>
-__global__ void __launch_bounds__(kPThreads)
-prologue_kernel(const T* __restrict__ X, const T* __restrict__ Q, const T* __restrict__ W_iq,
-                const T* __restrict__ W_ik, const T* __restrict__ w_ig, int L, int H, int Hq,
-                int D, int dI, int q_begin, int q_end, __nv_bfloat16* __restrict__ qt,
-                __nv_bfloat16* __restrict__ kh, float* __restrict__ running_max) {
-  extern __shared__ float sm[];
-  const int NC = dI + Hq;                 // key features + gate logits
-  float* sX = sm;                         // [kTok][kHChunk]
-  float* sWc = sX + kTok * kHChunk;       // [kHChunk][NC]
-  float* sKG = sWc + kHChunk * NC;        // [kTok][NC] key features | gate logits
-  float* sWq = sKG + kTok * NC;           // [D][dI]
-  float* sQ = sWq + D * dI;               // [kTok][D]
-  float* sQI = sQ + kTok * D;             // [kTok][dI]
-  float* sRms = sQI + kTok * dI;          // [kTok]
-  const int bi = blockIdx.y;
-  const int t0 = q_begin + blockIdx.x * kTok;
-  const int tid = threadIdx.x;
+__global__ void __launch_bounds__(kPThreads, 1)
+prologue_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_q,
+                   const __grid_constant__ CUtensorMap map_wc, const __grid_constant__ CUtensorMap map_wq,
+                   int L, int H, int Hq, int D, int dI, int N1, int q_begin, int q_end, int batch,
+                   __nv_bfloat16* __restrict__ qt, __nv_bfloat16* __restrict__ kh,
+                   float* __restrict__ running_max, int* __restrict__ err) {
+  constexpr int EPB = 128 / (int)sizeof(T);                  // elements per 128-byte row
+  constexpr uint32_t FMT = std::is_same<T, float>::value ? tc::kFmtTF32 : tc::kFmtBF16;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sA = tc::smem_addr(smem);
+  const uint32_t sB = sA + kNSt * kStageA;
+  const uint32_t bar = sB + kNSt * kStageB;
+  const uint32_t full0 = bar, empty0 = bar + 8 * kNSt, d1_full = bar + 16 * kNSt,
+                 d1_empty = d1_full + 8, h_full0 = d1_empty + 8;
+  const int NB = (512 - kD1Cols) / dI;                        // head buffers in TMEM
+  const uint32_t h_empty0 = h_full0 + 8 * NB;
+  __shared__ uint32_t s_tmem;
 
-  // ---- key features and gate logits: [kTok, H] x [H, dI + Hq]
-  const int n_out = kTok * NC;
-  float acc[(kTok * 128) / kPThreads];    // NC <= 128
-  for (int a = 0; a < (kTok * 128) / kPThreads; ++a) acc[a] = 0.f;
-  for (int h0 = 0; h0 < H; h0 += kHChunk) {
-    __syncthreads();
-    for (int i = tid; i < kTok * kHChunk; i += kPThreads) {
-      const int tt = i / kHChunk, c = i % kHChunk;
-      const int t = t0 + tt;
-      sX[i] = (t < q_end) ? Elem<T>::to_f(X[((size_t)bi * L + t) * H + h0 + c]) : 0.f;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tiles_per_seq = (q_end - q_begin + kTileM - 1) / kTileM;
+  const int n_tiles = tiles_per_seq * batch;
+  const int nk1 = H / EPB, nk2 = D / EPB;
+  const uint32_t tx1 = kStageA + N1 * 128, tx2 = kStageA + dI * 128;
+
+  if (tid == 0) {
+    for (int i = 0; i < kNSt; ++i) {
+      tc::mbar_init(full0 + 8 * i, 1);
+      tc::mbar_init(empty0 + 8 * i, 1);
     }
-    for (int i = tid; i < kHChunk * NC; i += kPThreads) {
-      const int c = i / NC, j = i % NC;
-      sWc[i] = (j < dI) ? Elem<T>::to_f(W_ik[(size_t)(h0 + c) * dI + j])
-                        : Elem<T>::to_f(w_ig[(size_t)(h0 + c) * Hq + (j - dI)]);
+    tc::mbar_init(d1_full, 1);
+    tc::mbar_init(d1_empty, 4);
+    for (int i = 0; i < NB; ++i) {
+      tc::mbar_init(h_full0 + 8 * i, 1);
+      tc::mbar_init(h_empty0 + 8 * i, 4);
     }
-    __syncthreads();
-    for (int a = 0; a * kPThreads + tid < n_out; ++a) {
-      const int o = a * kPThreads + tid, tt = o / NC, j = o % NC;
-      float s = acc[a];
-      for (int c = 0; c < kHChunk; ++c) s = fmaf(sX[tt * kHChunk + c], sWc[c * NC + j], s);
-      acc[a] = s;
-    }
+    tc::fence_mbar_init();
+    tc::prefetch_tmap(&map_x);
+    tc::prefetch_tmap(&map_q);
+    tc::prefetch_tmap(&map_wc);
+    tc::prefetch_tmap(&map_wq);
   }
-  for (int a = 0; a * kPThreads + tid < n_out; ++a) sKG[a * kPThreads + tid] = acc[a];
+  if (warp == 1) {
+    tc::tmem_alloc(tc::smem_addr(&s_tmem), 512);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before();
   __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = s_tmem;
 
-  // ---- khat: RMS-normalised shared key (warp per token)
-  const int lane = tid & 31, warp = tid >> 5;
-  for (int tt = warp; tt < kTok; tt += kPThreads / 32) {
-    const int t = t0 + tt;
-    float ss = 0.f;
-    for (int j = lane; j < dI; j += 32) ss += sKG[tt * NC + j] * sKG[tt * NC + j];
-    ss = warp_sum(ss);
-    const float inv = rsqrtf(ss / dI + 1e-6f);
-    if (t < q_end)
-      for (int j = lane; j < kIdxPad; j += 32)
-        kh[((size_t)bi * L + t) * kIdxPad + j] = __float2bfloat16_rn(j < dI ? sKG[tt * NC + j] * inv : 0.f);
-  }
-
-  // ---- qtilde: per head projection, RMS norm, gate, sum
-  const float inv_sqrt_dI = rsqrtf((float)dI);
-  float qacc[(kTok * 64) / kPThreads];     // dI <= 64
-  for (int a = 0; a < (kTok * 64) / kPThreads; ++a) qacc[a] = 0.f;
-  const int n_q = kTok * dI;
-  for (int h = 0; h < Hq; ++h) {
-    __syncthreads();
-    for (int i = tid; i < D * dI; i += kPThreads) sWq[i] = Elem<T>::to_f(W_iq[(size_t)h * D * dI + i]);
-    for (int i = tid; i < kTok * D; i += kPThreads) {
-      const int tt = i / D, c = i % D;
-      const int t = t0 + tt;
-      sQ[i] = (t < q_end) ? Elem<T>::to_f(Q[(((size_t)bi * L + t) * Hq + h) * D + c]) : 0.f;
-    }
-    __syncthreads();
-    float qi[(kTok * 64) / kPThreads];
-    for (int a = 0; a * kPThreads + tid < n_q; ++a) {
-      const int o = a * kPThreads + tid, tt = o / dI, j = o % dI;
-      float s = 0.f;
-      for (int c = 0; c < D; ++c) s = fmaf(sQ[tt * D + c], sWq[c * dI + j], s);
-      qi[a] = s;
-      sQI[o] = s;
-    }
-    __syncthreads();
-    for (int tt = warp; tt < kTok; tt += kPThreads / 32) {
-      float ss = 0.f;
-      for (int j = lane; j < dI; j += 32) ss += sQI[tt * dI + j] * sQI[tt * dI + j];
-      ss = warp_sum(ss);
-      if (lane == 0) {
-        const float gamma = sigmoidf_(sKG[tt * NC + dI + h]);
-        sRms[tt] = gamma * rsqrtf(ss / dI + 1e-6f) * inv_sqrt_dI;
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    int st = 0, ph = 0, used = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+      const int seq = tile / tiles_per_seq;
+      const int row = seq * L + q_begin + (tile % tiles_per_seq) * kTileM;
+      for (int it = 0; it < nk1 + Hq * nk2 && ok; ++it) {
+        if (used >= kNSt && !tc::mbar_wait(empty0 + 8 * st, ph ^ 1)) { ok = false; break; }
+        const uint32_t full = full0 + 8 * st;
+        if (it < nk1) {
+          tc::mbar_expect_tx(full, tx1);
+          tc::tma_load_2d(sA + st * kStageA, &map_x, full, it * EPB, row);
+          tc::tma_load_2d(sB + st * kStageB, &map_wc, full, it * EPB, 0);
+        } else {
+          const int h = (it - nk1) / nk2, kb = (it - nk1) % nk2;
+          tc::mbar_expect_tx(full, tx2);
+          tc::tma_load_2d(sA + st * kStageA, &map_q, full, h * D + kb * EPB, row);
+          tc::tma_load_2d(sB + st * kStageB, &map_wq, full, kb * EPB, h * dI);
+        }
+        ++used;
+        if (++st == kNSt) { st = 0; ph ^= 1; }
       }
     }
-    __syncthreads();
-    for (int a = 0; a * kPThreads + tid < n_q; ++a) {
-      const int o = a * kPThreads + tid, tt = o / dI;
-      qacc[a] = fmaf(sRms[tt], qi[a], qacc[a]);
+    if (!ok) record_error(err, DEV_TIMEOUT);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    const uint32_t id1 = tc::idesc(FMT, 128, N1, false, false);
+    const uint32_t id2 = tc::idesc(FMT, 128, dI, false, false);
+    int st = 0, ph = 0, tcount = 0, hcount = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++tcount) {
+      if (tcount >= 1 && !tc::mbar_wait(d1_empty, (tcount - 1) & 1)) { ok = false; break; }
+      tc::fence_after();
+      for (int it = 0; it < nk1 + Hq * nk2 && ok; ++it) {
+        const bool g2 = it >= nk1;
+        const int kb = g2 ? (it - nk1) % nk2 : it;
+        int hb = 0;
+        if (g2) {
+          hb = hcount % NB;
+          if (kb == 0 && hcount >= NB && !tc::mbar_wait(h_empty0 + 8 * hb, ((hcount / NB) - 1) & 1)) {
+            ok = false;
+            break;
+          }
+        }
+        if (!tc::mbar_wait(full0 + 8 * st, ph)) { ok = false; break; }
+        tc::fence_after();
+        const uint32_t d = g2 ? tmem + kD1Cols + hb * dI : tmem;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {   // four 32-byte K steps per 128-byte row
+          const uint64_t ad = tc::sdesc_sw128(sA + st * kStageA + k * 32, 16, 1024);
+          const uint64_t bd = tc::sdesc_sw128(sB + st * kStageB + k * 32, 16, 1024);
+          tc::mma_f16(d, ad, bd, g2 ? id2 : id1, (kb > 0 || k > 0) ? 1u : 0u);
+        }
+        tc::mma_commit(empty0 + 8 * st);
+        if (!g2 && it == nk1 - 1) tc::mma_commit(d1_full);
+        if (g2 && kb == nk2 - 1) {
+          tc::mma_commit(h_full0 + 8 * hb);
+          ++hcount;
+        }
+        if (++st == kNSt) { st = 0; ph ^= 1; }
+      }
+    }
+    if (!ok) record_error(err, DEV_TIMEOUT);
+  } else if (warp >= 2) {
+    // ---------------- epilogue: one token row per thread
+    const int quarter = warp & 3;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const float inv_sqrt_dI = rsqrtf((float)dI);
+    int tcount = 0, hcount = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++tcount) {
+      const int seq = tile / tiles_per_seq;
+      const int t = q_begin + (tile % tiles_per_seq) * kTileM + quarter * 32 + lane;
+      const bool valid = t < q_end;
+      const size_t row = (size_t)seq * L + t;
+      if (!tc::mbar_wait(d1_full, tcount & 1)) { ok = false; break; }
+      tc::fence_after();
+      // shared key: RMS-normalised kI
+      float acc[64];
+      float ss = 0.f;
+#pragma unroll
+      for (int c = 0; c < 64; c += 16) {
+        if (c < dI) {
+          tc::tmem_ld16(tmem + lane_base + c, acc + c);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) ss = fmaf(acc[c + e], acc[c + e], ss);
+        }
+      }
+      const float kinv = rsqrtf(ss / dI + 1e-6f);
+      if (valid) {
+#pragma unroll
+        for (int c = 0; c < 64; c += 8) {
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = (c + e < dI) ? acc[c + e] * kinv : 0.f;
+          store8<__nv_bfloat16>(kh + row * kIdxPad + c, f);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 64; ++c) acc[c] = 0.f;
+      // heads: qtilde += gamma_h / (rms_h sqrt(dI)) * qI_h
+      for (int h = 0; h < Hq; ++h) {
+        const float logit = __uint_as_float(tmem_ld1(tmem + lane_base + dI + h));
+        const float gamma = sigmoidf_(logit);
+        const int hb = hcount % NB;
+        if (!tc::mbar_wait(h_full0 + 8 * hb, (hcount / NB) & 1)) { ok = false; break; }
+        tc::fence_after();
+        float v[64];
+        float qs = 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; c += 16) {
+          if (c < dI) {
+            tc::tmem_ld16(tmem + lane_base + kD1Cols + hb * dI + c, v + c);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) qs = fmaf(v[c + e], v[c + e], qs);
+          }
+        }
+        tc::fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(h_empty0 + 8 * hb);
+        ++hcount;
+        const float coef = gamma * rsqrtf(qs / dI + 1e-6f) * inv_sqrt_dI;
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (c < dI) acc[c] = fmaf(coef, v[c], acc[c]);
+      }
+      if (!ok) break;
+      // GEMM1's columns (gate logits) are no longer needed
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(d1_empty);
+      if (valid) {
+#pragma unroll
+        for (int c = 0; c < 64; c += 8) {
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = (c + e < dI) ? acc[c + e] : 0.f;
+          store8<__nv_bfloat16>(qt + row * kIdxPad + c, f);
+        }
+        running_max[row] = -INFINITY;
+      }
+    }
+    if (!ok) record_error(err, DEV_TIMEOUT);
+  }
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 1) tc::tmem_dealloc(tmem, 512);
+}
+
+// Weight repacking at init: WcT [N1][H] = [W_ik | w_ig]^T zero-padded to N1
+// rows; WqT [Hq * dI][D] with row h*dI + j = W_iq[h][:, j].
+template <typename T>
+__global__ void pack_weights_kernel(const T* __restrict__ W_iq, const T* __restrict__ W_ik,
+                                    const T* __restrict__ w_ig, int H, int Hq, int D, int dI,
+                                    int N1, T* __restrict__ WcT, T* __restrict__ WqT) {
+  const size_t nwc = (size_t)N1 * H, nwq = (size_t)Hq * dI * D;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nwc + nwq;
+       i += (size_t)gridDim.x * blockDim.x) {
+    if (i < nwc) {
+      const int n = (int)(i / H), k = (int)(i % H);
+      T v = Elem<T>::from_f(0.f);
+      if (n < dI) v = W_ik[(size_t)k * dI + n];
+      else if (n < dI + Hq) v = w_ig[(size_t)k * Hq + (n - dI)];
+      WcT[i] = v;
+    } else {
+      const size_t j = i - nwc;
+      const int rowi = (int)(j / D), c = (int)(j % D);
+      const int h = rowi / dI, jj = rowi % dI;
+      WqT[j] = W_iq[((size_t)h * D + c) * dI + jj];
     }
   }
-  for (int a = 0; a * kPThreads + tid < n_q; ++a) {
-    const int o = a * kPThreads + tid, tt = o / dI, j = o % dI;
-    const int t = t0 + tt;
-    if (t < q_end) qt[((size_t)bi * L + t) * kIdxPad + j] = __float2bfloat16_rn(qacc[a]);
+}
+
+template <typename T>
+bool make_tmap(const Ctx& c, CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+               uint32_t box_rows) {
+  using Fn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                          const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                          CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                          CUtensorMapFloatOOBfill);
+  if (!c.encode_tiled) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * sizeof(T)};
+  const cuuint32_t box[2] = {(cuuint32_t)(128 / sizeof(T)), box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt =
+      std::is_same<T, float>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return ((Fn)c.encode_tiled)(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T>
+cudaError_t launch_pro(const Ctx& c, int batch, int L, const void* X, const void* Q, int q_begin,
+                       int q_end, __nv_bfloat16* qt, __nv_bfloat16* kh, float* running_max,
+                       cudaStream_t st) {
+  const int H = c.cfg.hidden, Hq = c.cfg.n_q_heads, D = c.cfg.head_dim, dI = c.cfg.idx_dim;
+  CUtensorMap mx, mq, mwc, mwq;
+  if (!make_tmap<T>(c, &mx, X, (uint64_t)batch * L, H, kTileM) ||
+      !make_tmap<T>(c, &mq, Q, (uint64_t)batch * L, (uint64_t)Hq * D, kTileM) ||
+      !make_tmap<T>(c, &mwc, c.WcT, c.N1, H, c.N1) ||
+      !make_tmap<T>(c, &mwq, c.WqT, (uint64_t)Hq * dI, D, dI))
+    return cudaErrorInvalidValue;
+  const int tiles = ((q_end - q_begin + kTileM - 1) / kTileM) * batch;
+  int grid = c.num_sms;
+  if (tiles < grid) grid = tiles;
+  auto k = prologue_tc_kernel<T>;
+  static bool attr_set[64] = {};
+  if (!attr_set[c.device & 63]) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kProSmem);
+    if (e != cudaSuccess) return e;
+    attr_set[c.device & 63] = true;
   }
-  for (int i = tid; i < kTok * (kIdxPad - dI); i += kPThreads) {   // zero padding
-    const int tt = i / (kIdxPad - dI), j = dI + i % (kIdxPad - dI);
-    if (t0 + tt < q_end) qt[((size_t)bi * L + t0 + tt) * kIdxPad + j] = __float2bfloat16_rn(0.f);
-  }
-  if (tid < kTok && t0 + tid < q_end) running_max[(size_t)bi * L + t0 + tid] = -INFINITY;
+  k<<<grid, kPThreads, kProSmem, st>>>(mx, mq, mwc, mwq, L, H, Hq, D, dI, c.N1, q_begin, q_end,
+                                       batch, qt, kh, running_max, c.err);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
+cudaError_t pack_indexer_weights(Ctx& c, const void* W_iq, const void* W_ik, const void* w_ig) {
+  const int H = c.cfg.hidden, Hq = c.cfg.n_q_heads, D = c.cfg.head_dim, dI = c.cfg.idx_dim;
+  c.N1 = (dI + Hq + 15) / 16 * 16;
+  const size_t es = c.cfg.dtype == IMEM_BF16 ? 2 : 4;
+  cudaError_t e = cudaMalloc(&c.WcT, (size_t)c.N1 * H * es);
+  if (e == cudaSuccess) e = cudaMalloc(&c.WqT, (size_t)Hq * dI * D * es);
+  if (e != cudaSuccess) return e;
+  if (c.cfg.dtype == IMEM_BF16)
+    pack_weights_kernel<__nv_bfloat16><<<256, 256>>>(
+        (const __nv_bfloat16*)W_iq, (const __nv_bfloat16*)W_ik, (const __nv_bfloat16*)w_ig, H, Hq,
+        D, dI, c.N1, (__nv_bfloat16*)c.WcT, (__nv_bfloat16*)c.WqT);
+  else
+    pack_weights_kernel<float><<<256, 256>>>((const float*)W_iq, (const float*)W_ik,
+                                             (const float*)w_ig, H, Hq, D, dI, c.N1,
+                                             (float*)c.WcT, (float*)c.WqT);
+  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  return e;
+}
+
 cudaError_t launch_prologue(const Ctx& c, int batch, int L, const void* X, const void* Q,
                             int q_begin, int q_end, __nv_bfloat16* qt, __nv_bfloat16* kh,
                             float* running_max, cudaStream_t st) {
-  const int H = c.cfg.hidden, Hq = c.cfg.n_q_heads, D = c.cfg.head_dim, dI = c.cfg.idx_dim;
-  const int NC = dI + Hq;
-  const size_t smem = ((size_t)kTok * kHChunk + kHChunk * NC + kTok * NC + D * dI + kTok * D +
-                       kTok * dI + kTok) * sizeof(float);
-  dim3 grid((q_end - q_begin + kTok - 1) / kTok, batch);
-  cudaError_t e;
-  if (c.cfg.dtype == IMEM_BF16) {
-    auto k = prologue_kernel<__nv_bfloat16>;
-    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k<<<grid, kPThreads, smem, st>>>((const __nv_bfloat16*)X, (const __nv_bfloat16*)Q,
-                                     (const __nv_bfloat16*)c.W_iq, (const __nv_bfloat16*)c.W_ik,
-                                     (const __nv_bfloat16*)c.w_ig, L, H, Hq, D, dI, q_begin, q_end,
-                                     qt, kh, running_max);
-  } else {
-    auto k = prologue_kernel<float>;
-    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k<<<grid, kPThreads, smem, st>>>((const float*)X, (const float*)Q, (const float*)c.W_iq,
-                                     (const float*)c.W_ik, (const float*)c.w_ig, L, H, Hq, D, dI,
-                                     q_begin, q_end, qt, kh, running_max);
-  }
-  return cudaGetLastError();
+  if (c.cfg.dtype == IMEM_BF16)
+    return launch_pro<__nv_bfloat16>(c, batch, L, X, Q, q_begin, q_end, qt, kh, running_max, st);
+  return launch_pro<float>(c, batch, L, X, Q, q_begin, q_end, qt, kh, running_max, st);
 }
 
 }  // namespace imem
