@@ -166,6 +166,30 @@ imem_status imem_decode(imem_ctx* ctx, int batch, const void* q, const void* k_n
                         int cap, const float* M, const float* bstab, void* out,
                         void* workspace, void* stream);
 
+/* Latent-memory update that allocates nothing (no counterpart in the paper: an
+ * interface for callers that cannot allocate device memory, e.g. code running
+ * inside a host framework's pre-planned memory arena or where cudaMalloc is not
+ * allowed; imem_init and a workspace both need allocations such callers cannot
+ * make). Same result as imem_update_memory, with no context: the caller passes
+ * the dimensions, the decay lambda and W_phi [mem_r, head_dim] (fp32, device)
+ * directly; K, V, idx_evicted, n_evicted, chunk, M and bstab as there.
+ * Scratch: a fixed 8 MiB array in the library's device memory, held by every
+ * GPU that loads the library until the process exits. batch * n_kv_heads *
+ * head_dim * (head_dim + 1) * 4 bytes must fit in it (batch <= 15 at 8 KV heads
+ * of dimension 128), otherwise IMEM_ERR_UNSUPPORTED and nothing is launched.
+ * The first call on a device looks up the array's device address (set-up, no
+ * allocation); make that first call before any stream capture. Every call
+ * writes the whole scratch region it uses before reading it, so nothing must
+ * start at zero; calls that overlap on the GPU (any streams, any callers) race
+ * on the shared array and must be serialised by the caller. A bounded device
+ * wait that runs out is not reported by this entry point (no context); the
+ * outputs are then unspecified.
+ * Errors: INVALID_ARG, SHAPE, ALIGN, UNSUPPORTED, CUDA. */
+imem_status imem_update_memory_static(int batch, int L, int n_kv_heads, int head_dim, int mem_r,
+                                      float lambda, int dtype, const void* K, const void* V,
+                                      const int32_t* idx_evicted, int n_evicted, int chunk,
+                                      const float* W_phi, float* M, float* bstab, void* stream);
+
 /* Waits for the stream, then reports the first error the device recorded for
  * this context since the last imem_sync (TIMEOUT for a bounded wait that ran
  * out, SHAPE for a decode into a full cache) or a CUDA error, and clears it. */

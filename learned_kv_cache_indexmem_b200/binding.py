@@ -72,6 +72,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.imem_decode.argtypes = [vp, i, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp]
     lib.imem_sync.restype = i
     lib.imem_sync.argtypes = [vp, vp]
+    lib.imem_update_memory_static.restype = i
+    lib.imem_update_memory_static.argtypes = [i, i, i, i, i, f, i, vp, vp, vp, i, i, vp, vp, vp, vp]
     _lib = lib
     return lib
 
@@ -148,6 +150,17 @@ def decode(ctx, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, 
     _check(load().imem_decode(
         ctx, batch, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(K_ret), _ptr(V_ret), _ptr(cache_len),
         cap, _ptr(M), _ptr(bstab), _ptr(out), _ptr(workspace), _stream(stream)), "imem_decode")
+
+
+def update_memory_static(batch, L, n_kv_heads, head_dim, mem_r, lam, dtype, K, V, idx_evicted,
+                         n_evicted, chunk, W_phi, M, bstab, stream=None):
+    """imem_update_memory_static: the memory update without a context or a
+    workspace, for callers that cannot allocate device memory (its scratch is a
+    fixed array inside the library; see include/indexmem.h)."""
+    _check(load().imem_update_memory_static(
+        batch, L, n_kv_heads, head_dim, mem_r, lam, dtype, _ptr(K), _ptr(V), _ptr(idx_evicted),
+        n_evicted, chunk, _ptr(W_phi), _ptr(M), _ptr(bstab), _stream(stream)),
+        "imem_update_memory_static")
 
 
 def sync(ctx, stream=None) -> None:

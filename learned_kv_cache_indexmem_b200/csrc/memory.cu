@@ -329,3 +329,124 @@ cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, 
 }
 
 }  // namespace imem
+
+// ---------------------------------------------------------------------------
+// Memory update without any allocation.
+//
+// For callers that cannot allocate device memory at all -- for example code
+// running where cudaMalloc is forbidden or would break the memory plan of a
+// host framework (inside a pre-planned arena, or in a process whose device
+// memory is owned by another allocator) -- imem_update_memory_static runs the
+// same two kernels as imem_update_memory, but its scratch (the per-run partial
+// sums [S | s]) lives in the fixed-size array below instead of a caller
+// workspace, and it needs no context: the caller passes the dimensions, the
+// decay and W_phi directly.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace imem {
+namespace {
+
+constexpr size_t kStaticScratchBytes = (size_t)8 << 20;   // 8 MiB per device
+static __device__ __align__(256) float g_static_scratch[kStaticScratchBytes / sizeof(float)];
+static __device__ int g_static_err;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mtx;
+float* g_static_ptr[kMaxDevices] = {};
+int* g_static_err_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array for the current device (host code must
+// not use the symbol itself: it is a host-side stand-in, not a device address).
+cudaError_t static_scratch(int dev, float** scratch, int** err) {
+  std::lock_guard<std::mutex> lock(g_static_mtx);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    void* e = nullptr;
+    cudaError_t r = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (r != cudaSuccess) return r;
+    r = cudaGetSymbolAddress(&e, g_static_err);
+    if (r != cudaSuccess) return r;
+    g_static_ptr[dev] = static_cast<float*>(p);
+    g_static_err_ptr[dev] = static_cast<int*>(e);
+  }
+  *scratch = g_static_ptr[dev];
+  *err = g_static_err_ptr[dev];
+  return cudaSuccess;
+}
+
+template <typename T, int D>
+cudaError_t launch_memory_static(int batch, int L, int Hkv, int r, float lambda, const void* K,
+                                 const void* V, const int32_t* idx_e, int n_e, int chunk,
+                                 const float* W_phi, float* M, float* bstab, float* scratch,
+                                 int* err, cudaStream_t st) {
+  const int units = batch * Hkv;
+  const size_t psize = (size_t)D * (D + 1) * sizeof(float);
+  int G = memory_groups(batch, Hkv, n_e, chunk);
+  while (G > 1 && (size_t)units * G * psize > kStaticScratchBytes) --G;
+  const int chunks = (n_e + chunk - 1) / chunk;
+  const int tokens_per_group = ((chunks + G - 1) / G) * chunk;
+  const int Gused = (n_e + tokens_per_group - 1) / tokens_per_group;
+  const float log2lam = (float)log2((double)lambda);
+  auto kfn = memory_tc_kernel<T, D>;
+  cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       MemTile<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  kfn<<<dim3(Gused, Hkv, batch), kMemThreads, MemTile<D>::SMEM, st>>>(
+      (const T*)K, (const T*)V, idx_e, n_e, L, Hkv, log2lam, tokens_per_group, scratch, err);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const float decay_n = (float)pow((double)lambda, (double)n_e);
+  const size_t fsmem = ((size_t)r * D + (size_t)D * 16) * sizeof(float);
+  e = cudaFuncSetAttribute(memory_finalize_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)fsmem);
+  if (e != cudaSuccess) return e;
+  memory_finalize_kernel<D><<<dim3(D / 16 + 1, units), 256, fsmem, st>>>(scratch, Gused, W_phi, r,
+                                                                        decay_n, M, bstab);
+  return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace imem
+
+extern "C" imem_status imem_update_memory_static(int batch, int L, int n_kv_heads, int head_dim,
+                                                 int mem_r, float lambda, int dtype, const void* K,
+                                                 const void* V, const int32_t* idx_evicted,
+                                                 int n_evicted, int chunk, const float* W_phi,
+                                                 float* M, float* bstab, void* stream) {
+  using namespace imem;
+  if (dtype != IMEM_FP32 && dtype != IMEM_BF16) return IMEM_ERR_INVALID_ARG;
+  if (batch < 1 || L < 1 || n_kv_heads < 1) return IMEM_ERR_SHAPE;
+  if (n_evicted < 0 || n_evicted > L) return IMEM_ERR_SHAPE;
+  if (chunk < 64 || chunk % 64) return IMEM_ERR_SHAPE;
+  if (!(lambda > 0.f && lambda <= 1.f)) return IMEM_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return IMEM_ERR_UNSUPPORTED;
+  if (mem_r < 16 || mem_r % 16 || mem_r > 128) return IMEM_ERR_UNSUPPORTED;
+  // the smallest split (one run per sequence and KV head) must fit the scratch
+  if ((size_t)batch * n_kv_heads * head_dim * (head_dim + 1) * sizeof(float) > kStaticScratchBytes)
+    return IMEM_ERR_UNSUPPORTED;
+  const void* ptrs[] = {K, V, W_phi, M, bstab};
+  for (const void* p : ptrs) {
+    if (!p) return IMEM_ERR_INVALID_ARG;
+    if ((uintptr_t)p & 15u) return IMEM_ERR_ALIGN;
+  }
+  if (n_evicted > 0) {
+    if (!idx_evicted) return IMEM_ERR_INVALID_ARG;
+    if ((uintptr_t)idx_evicted & 15u) return IMEM_ERR_ALIGN;
+  }
+  if (n_evicted == 0) return IMEM_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return IMEM_ERR_CUDA;
+  float* scratch = nullptr;
+  int* err = nullptr;
+  if (static_scratch(dev, &scratch, &err) != cudaSuccess) return IMEM_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  if (dtype == IMEM_BF16)
+    e = head_dim == 128 ? launch_memory_static<__nv_bfloat16, 128>(batch, L, n_kv_heads, mem_r, lambda, K, V, idx_evicted, n_evicted, chunk, W_phi, M, bstab, scratch, err, st)
+                        : launch_memory_static<__nv_bfloat16, 64>(batch, L, n_kv_heads, mem_r, lambda, K, V, idx_evicted, n_evicted, chunk, W_phi, M, bstab, scratch, err, st);
+  else
+    e = head_dim == 128 ? launch_memory_static<float, 128>(batch, L, n_kv_heads, mem_r, lambda, K, V, idx_evicted, n_evicted, chunk, W_phi, M, bstab, scratch, err, st)
+                        : launch_memory_static<float, 64>(batch, L, n_kv_heads, mem_r, lambda, K, V, idx_evicted, n_evicted, chunk, W_phi, M, bstab, scratch, err, st);
+  return e == cudaSuccess ? IMEM_OK : IMEM_ERR_CUDA;
+}
