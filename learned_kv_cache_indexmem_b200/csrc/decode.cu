@@ -60,6 +60,14 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+// waits until at most n of this thread's cp.async groups are pending
+__device__ __forceinline__ void cp_async_wait_dyn(int n) {
+  if (n <= 0) cp_async_wait<0>();
+  else if (n == 1) cp_async_wait<1>();
+  else if (n == 2) cp_async_wait<2>();
+  else if (n == 3) cp_async_wait<3>();
+  else cp_async_wait<4>();
+}
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
                                         uint32_t& r3) {
@@ -98,7 +106,7 @@ template <int D, int G>
 __device__ void attend_bf16(const __nv_bfloat16* __restrict__ Kb, const __nv_bfloat16* __restrict__ Vb,
                             size_t row_stride, const __nv_bfloat16* kn, const __nv_bfloat16* vn,
                             int len, int r0, int r1, const float (*s_q)[D],
-                            Partial<D> (*s_part)[G], unsigned char* stage_mem) {
+                            Partial<D> (*s_part)[G], unsigned char* stage_mem, int nst) {
   constexpr int CH = D / 8;                 // 16-byte chunks per row
   constexpr int STAGE_BYTES = kStageRows * D * 2;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -138,17 +146,14 @@ __device__ void attend_bf16(const __nv_bfloat16* __restrict__ Kb, const __nv_bfl
     cp_async_commit();
   };
 
+  // ring of nst stages, all issued up front as far as the ring allows
   const int n_stages = (r1 - r0 + kStageRows - 1) / kStageRows;
-  if (n_stages > 0) issue(0, 0);
+  int issued = 0;
+  for (; issued < n_stages && issued < nst; ++issued) issue(issued, issued);
   for (int st = 0; st < n_stages; ++st) {
-    if (st + 1 < n_stages) {
-      issue(st + 1, (st + 1) & 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
+    cp_async_wait_dyn(issued - (st + 1));   // groups younger than stage st may stay pending
     __syncthreads();
-    const uint32_t kt = sbase + (st & 1) * 2 * STAGE_BYTES;
+    const uint32_t kt = sbase + (st % nst) * 2 * STAGE_BYTES;
     const uint32_t vt = kt + STAGE_BYTES;
     const int kb = r0 + st * kStageRows + warp * 16;   // this warp's 16 rows
     if (kb < r1) {
@@ -206,6 +211,10 @@ __device__ void attend_bf16(const __nv_bfloat16* __restrict__ Kb, const __nv_bfl
       }
     }
     __syncthreads();
+    if (issued < n_stages) {   // refill the buffer just consumed
+      issue(issued, issued % nst);
+      ++issued;
+    }
   }
   // per-lane partial sums of the head's normaliser -> full sum over the quad
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
@@ -333,24 +342,35 @@ __device__ __forceinline__ void griddep_launch() {
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 }
 
-// Dynamic shared memory of one decode CTA (offsets in bytes):
-//   [0, work)        attention stages | per-warp states | readout buffers
-//   [part, part + G * sizeof(Partial<D>))   this CTA's published result,
-//                    read by the other CTAs of the cluster
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+
+// Dynamic shared memory of one decode CTA (bytes). Attention CTAs use
+// [0, att) for their row stages (then for the per-warp states); the readout
+// CTA uses [0, readout) for its operands and result and receives the S
+// attention states in [slot_off, slot_off + S * G * sizeof(Partial<D>)).
 template <int D, int G>
 struct DecSmem {
-  static constexpr size_t att(bool bf16) { return bf16 ? (size_t)2 * 2 * kStageRows * D * 2 : 0; }
+  static size_t att(bool bf16, int nst) { return bf16 ? (size_t)nst * 2 * kStageRows * D * 2 : 0; }
   static constexpr size_t warps() { return (size_t)4 * G * sizeof(Partial<D>); }
   static size_t readout(int r) {
-    return ((size_t)2 * r * D + (size_t)G * r + 2 * G + (size_t)G * D + r) * sizeof(float);
+    return ((size_t)r * D + r + (size_t)G * r + 2 * G + (size_t)4 * kThreads * G + (size_t)G * D) *
+           sizeof(float);
   }
-  static size_t part_off(bool bf16, int r) {
-    size_t w = att(bf16);
+  static size_t slot_off(int r) { return (readout(r) + 127) / 128 * 128; }
+  static size_t total(bool bf16, int nst, int r, int S) {
+    size_t w = att(bf16, nst);
     if (warps() > w) w = warps();
-    if (readout(r) > w) w = readout(r);
-    return (w + 127) / 128 * 128;
+    const size_t rs = slot_off(r) + (size_t)S * G * sizeof(Partial<D>);
+    return rs > w ? rs : w;
   }
-  static size_t total(bool bf16, int r) { return part_off(bf16, r) + (size_t)G * sizeof(Partial<D>); }
 };
 
 template <typename T, int D, int G>
@@ -360,11 +380,11 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
               int cap, int Hkv, const float* __restrict__ M, const float* __restrict__ bstab,
               const float* __restrict__ W_phi, const float* __restrict__ w_gate, int r, float eps,
               float gate_override, int use_override, T* __restrict__ out,
-              int* __restrict__ seq_counters, int* __restrict__ err, uint32_t part_off) {
+              int* __restrict__ seq_counters, int* __restrict__ err, uint32_t slot_off, int nst) {
   namespace cg = cooperative_groups;
   extern __shared__ __align__(128) unsigned char dyn_smem[];
   cg::cluster_group cluster = cg::this_cluster();
-  const int S = gridDim.x - 1;              // attention CTAs; CTA S = readout
+  const int S = gridDim.x - 1;              // attention CTAs; CTA S = readout and merge
   const int rank = blockIdx.x;              // the cluster spans blockIdx.x
   const int kh = blockIdx.y, bi = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -374,8 +394,11 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   __shared__ __align__(16) float s_q[G][D];
   __shared__ float s_w[kDecodeMaxSplits][G];
   __shared__ float s_l[G];
-  Partial<D>* mine = reinterpret_cast<Partial<D>*>(dyn_smem + part_off);
+  Partial<D>* slots = reinterpret_cast<Partial<D>*>(dyn_smem + slot_off);   // readout CTA only
 
+  // phase 0 of the cluster barrier: "this CTA is running" (remote shared
+  // memory is written only after every CTA of the cluster has arrived)
+  cluster_arrive_relaxed();
   // With programmatic dependent launch this kernel may start while the
   // previous kernel of the stream is still running: wait for it before
   // reading anything another kernel may write (q, the cache, cache_len, M, b).
@@ -406,126 +429,157 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     const int r0 = min(n, rank * per), r1 = min(n, r0 + per);
     auto* w_part = reinterpret_cast<Partial<D>(*)[G]>(dyn_smem);   // aliases the stages
     if constexpr (std::is_same<T, __nv_bfloat16>::value)
-      attend_bf16<D, G>(Kb, Vb, row_stride, kn, vn, len, r0, r1, s_q, w_part, dyn_smem);
+      attend_bf16<D, G>(Kb, Vb, row_stride, kn, vn, len, r0, r1, s_q, w_part, dyn_smem, nst);
     else
       attend_f32<D, G>(Kb, Vb, row_stride, kn, vn, len, r0, r1, s_q, w_part);
-    merge_warps<D, G>(w_part, mine);
-  } else {
-    // memory readout: u = W_phi q, m = M^T u / (b.u + eps), g = sigmoid(w_gate . q)
-    float* sW = reinterpret_cast<float*>(dyn_smem);          // [r][D], 16-byte chunks XOR-swizzled
-    float* sM = sW + (size_t)r * D;                           // [r][D]
-    float* swg = sM + (size_t)r * D;                          // [G][D] gate vectors
-    float* sb = swg + G * D;                                  // [r]
-    float* su = sb + r;                                       // [G][r]
-    float* sden = su + G * r;                                 // [G]
-    float* sgate = sden + G;                                  // [G]
-    // one round of asynchronous copies: W_phi, this unit's M and b, the gate rows
-    {
-      const uint32_t wdst = smem_u32(sW), mdst = smem_u32(sM);
-      const float* Mu = M + (size_t)unit * r * D;
-      for (int i = tid; i < r * D / 4; i += kThreads) {
-        const int j = (4 * i) / D, cc = ((4 * i) % D) / 4;
-        cp_async16(wdst + (uint32_t)(j * D + ((cc ^ (j & 7)) * 4)) * 4u, W_phi + 4 * i, true);
-        cp_async16(mdst + (uint32_t)i * 16u, Mu + 4 * i, true);
-      }
-      for (int i = tid; i < G * D / 4; i += kThreads)
-        cp_async16(smem_u32(swg) + (uint32_t)i * 16u, w_gate + (size_t)kh * G * D + 4 * i, true);
-      for (int i = tid; i < r / 4; i += kThreads)
-        cp_async16(smem_u32(sb) + (uint32_t)i * 16u, bstab + (size_t)unit * r + 4 * i, true);
-      cp_async_commit();
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    // u[g][j] = W_phi[j] . q[g]: one output per thread, four partial sums
-    for (int o = tid; o < G * r; o += kThreads) {
-      const int g = o / r, j = o % r;
-      const float4* wr = reinterpret_cast<const float4*>(sW + (size_t)j * D);
-      const float4* q4 = reinterpret_cast<const float4*>(&s_q[g][0]);
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 8
-      for (int cc = 0; cc < D / 4; ++cc) {
-        const float4 w = wr[cc ^ (j & 7)];
-        const float4 x = q4[cc];
-        a0 = fmaf(w.x, x.x, a0);
-        a1 = fmaf(w.y, x.y, a1);
-        a2 = fmaf(w.z, x.z, a2);
-        a3 = fmaf(w.w, x.w, a3);
-      }
-      su[o] = (a0 + a1) + (a2 + a3);
-    }
-    __syncthreads();
-    for (int g = warp; g < G; g += kThreads / 32) {
-      float a = 0.f;
-      for (int j = lane; j < r; j += 32) a = fmaf(sb[j], su[g * r + j], a);
-      a = warp_sum(a);
-      float z = 0.f;
-      for (int c = lane; c < D; c += 32) z = fmaf(swg[g * D + c], s_q[g][c], z);
-      z = warp_sum(z);
-      if (lane == 0) {
-        sden[g] = a + eps;
-        sgate[g] = use_override ? gate_override : sigmoidf_(z);
-      }
-    }
-    __syncthreads();
-    float* ro = reinterpret_cast<float*>(mine);               // [G][D] = g * m
-    for (int c = tid; c < D; c += kThreads) {
-      float num[G];
-#pragma unroll
-      for (int g = 0; g < G; ++g) num[g] = 0.f;
-#pragma unroll 4
-      for (int j = 0; j < r; ++j) {
-        const float mv = sM[j * D + c];
-#pragma unroll
-        for (int g = 0; g < G; ++g) num[g] = fmaf(mv, su[g * r + j], num[g]);
-      }
-#pragma unroll
-      for (int g = 0; g < G; ++g) ro[g * D + c] = sgate[g] * (num[g] / sden[g]);
-    }
+    cluster_wait();   // phase 0 complete: every CTA of the cluster is running
+    // push this CTA's merged state into the readout CTA's slot, then arrive
+    Partial<D>* slot = cluster.map_shared_rank(slots, S) + (size_t)rank * G;
+    merge_warps<D, G>(w_part, slot);
+    cluster_arrive_release();
+    return;
   }
 
-  // every CTA's result is in its shared memory; merge through the cluster
-  cluster.sync();
-  __shared__ float s_lp[kDecodeMaxSplits][G];
-  for (int i = tid; i < S * G; i += kThreads) {   // one parallel round of remote reads
-    const Partial<D>* rp = cluster.map_shared_rank(mine, i / G);
-    s_w[i / G][i % G] = rp[i % G].m;
-    s_lp[i / G][i % G] = rp[i % G].l;
-  }
-  __syncthreads();
-  if (tid < G) {
-    float mx = -INFINITY;
-    for (int t2 = 0; t2 < S; ++t2) mx = fmaxf(mx, s_w[t2][tid]);
-    float l = 0.f;
-    for (int t2 = 0; t2 < S; ++t2) {
-      const float mt = s_w[t2][tid];
-      const float w = (mt == -INFINITY) ? 0.f : exp2f(mt - mx);
-      s_w[t2][tid] = w;
-      l = fmaf(w, s_lp[t2][tid], l);
+  // ---- readout CTA: u = W_phi q, m = M^T u / (b.u + eps), g = sigmoid(w_gate . q)
+  float* sW = reinterpret_cast<float*>(dyn_smem);          // [r][D], 16-byte chunks XOR-swizzled
+  float* sb = sW + (size_t)r * D;                           // [r]
+  float* su = sb + r;                                       // [G][r]
+  float* sden = su + G * r;                                 // [G]
+  float* sgate = sden + G;                                  // [G]
+  float* snum = sgate + G;                                  // [4][G][D] partial M^T u
+  float* ro = snum + 4 * G * D;                             // [G][D] = g * m
+  {
+    const uint32_t wdst = smem_u32(sW);
+    for (int i = tid; i < r * D / 4; i += kThreads) {
+      const int j = (4 * i) / D, cc = ((4 * i) % D) / 4;
+      cp_async16(wdst + (uint32_t)(j * D + ((cc ^ (j & 7)) * 4)) * 4u, W_phi + 4 * i, true);
     }
-    s_l[tid] = l;
+    for (int i = tid; i < r / 4; i += kThreads)
+      cp_async16(smem_u32(sb) + (uint32_t)i * 16u, bstab + (size_t)unit * r + 4 * i, true);
+    cp_async_commit();
+  }
+  // M: thread (row group rg, column quad cq) holds rows rg, rg+4, ... of
+  // columns 4cq..4cq+3 (first 64 rows), loaded now so they arrive while u is
+  // computed (volatile: the loads are issued here, not at their first use)
+  constexpr int kREarly = 64;
+  const int cq = tid % (D / 4), rg = tid / (D / 4);         // D/4 column quads, kThreads/(D/4) row groups
+  constexpr int RG = kThreads / (D / 4);
+  float4 mreg[kREarly / RG];
+  const float* Mu = M + (size_t)unit * r * D;
+#pragma unroll
+  for (int k = 0; k < kREarly / RG; ++k) {
+    const int j = rg + k * RG;
+    if (j < r) {
+      asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];\n"
+                   : "=f"(mreg[k].x), "=f"(mreg[k].y), "=f"(mreg[k].z), "=f"(mreg[k].w)
+                   : "l"(Mu + (size_t)j * D + 4 * cq));
+    } else {
+      mreg[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  // gate: z = w_gate[h] . q (independent of the memory)
+  for (int g = warp; g < G; g += kThreads / 32) {
+    const float* wg = w_gate + ((size_t)kh * G + g) * D;
+    float z = 0.f;
+    for (int c = lane; c < D; c += 32) z = fmaf(__ldg(wg + c), s_q[g][c], z);
+    z = warp_sum(z);
+    if (lane == 0) sgate[g] = use_override ? gate_override : sigmoidf_(z);
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  for (int o = tid; o < G * r; o += kThreads) {
+    const int g = o / r, j = o % r;
+    const float4* wr = reinterpret_cast<const float4*>(sW + (size_t)j * D);
+    const float4* q4 = reinterpret_cast<const float4*>(&s_q[g][0]);
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 8
+    for (int cc = 0; cc < D / 4; ++cc) {
+      const float4 w = wr[cc ^ (j & 7)];
+      const float4 x = q4[cc];
+      a0 = fmaf(w.x, x.x, a0);
+      a1 = fmaf(w.y, x.y, a1);
+      a2 = fmaf(w.z, x.z, a2);
+      a3 = fmaf(w.w, x.w, a3);
+    }
+    su[o] = (a0 + a1) + (a2 + a3);
   }
   __syncthreads();
-  // this CTA's share of the G * D outputs; all S remote values are requested
-  // before any is used
-  const int per_out = (G * D + S) / (S + 1);
-  const int o0 = rank * per_out, o1 = min(G * D, o0 + per_out);
-  const float* ro_remote = reinterpret_cast<const float*>(cluster.map_shared_rank(mine, S));
-  for (int i = o0 + tid; i < o1; i += kThreads) {
+  for (int g = warp; g < G; g += kThreads / 32) {
+    float a = 0.f;
+    for (int j = lane; j < r; j += 32) a = fmaf(sb[j], su[g * r + j], a);
+    a = warp_sum(a);
+    if (lane == 0) sden[g] = a + eps;
+  }
+  {
+    // partial num over this thread's rows, for its 4 columns and every head
+    float4 acc[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) acc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < kREarly / RG; ++k) {
+      const int j = rg + k * RG;
+      if (j < r) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float uu = su[g * r + j];
+          acc[g].x = fmaf(mreg[k].x, uu, acc[g].x);
+          acc[g].y = fmaf(mreg[k].y, uu, acc[g].y);
+          acc[g].z = fmaf(mreg[k].z, uu, acc[g].z);
+          acc[g].w = fmaf(mreg[k].w, uu, acc[g].w);
+        }
+      }
+    }
+    for (int j = kREarly + rg; j < r; j += RG) {   // r > 64: remaining rows
+      const float4 mv = __ldcg(reinterpret_cast<const float4*>(Mu + (size_t)j * D + 4 * cq));
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float uu = su[g * r + j];
+        acc[g].x = fmaf(mv.x, uu, acc[g].x);
+        acc[g].y = fmaf(mv.y, uu, acc[g].y);
+        acc[g].z = fmaf(mv.z, uu, acc[g].z);
+        acc[g].w = fmaf(mv.w, uu, acc[g].w);
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+      reinterpret_cast<float4*>(snum + ((size_t)rg * G + g) * D)[cq] = acc[g];
+  }
+  __syncthreads();
+  for (int i = tid; i < G * D; i += kThreads) {
+    const int g = i / D, c = i % D;
+    float num = 0.f;
+#pragma unroll
+    for (int k = 0; k < RG; ++k) num += snum[((size_t)k * G + g) * D + c];
+    ro[i] = sgate[g] * (num / sden[g]);
+  }
+  __syncthreads();
+
+  // ---- merge the S attention states that the other CTAs pushed into the slots
+  cluster_wait();             // phase 0
+  cluster_arrive_release();   // phase 1: own arrival
+  cluster_wait();             // phase 1: every attention CTA has written its slot
+  // merge weights: a warp per head, a lane per slot (S <= 15 < 32)
+  for (int g = warp; g < G; g += kThreads / 32) {
+    const float mt = lane < S ? slots[lane * G + g].m : -INFINITY;
+    const float mx = warp_max(mt);
+    const float w = (mt == -INFINITY) ? 0.f : exp2f(mt - mx);
+    const float l = warp_sum(lane < S ? w * slots[lane * G + g].l : 0.f);
+    if (lane < S) s_w[lane][g] = w;
+    if (lane == 0) s_l[g] = l;
+  }
+  __syncthreads();
+  for (int i = tid; i < G * D; i += kThreads) {
     const int g = i / D, c = i % D;
     float vals[kDecodeMaxSplits];
 #pragma unroll
-    for (int t2 = 0; t2 < kDecodeMaxSplits; ++t2)
-      vals[t2] = (t2 < S) ? cluster.map_shared_rank(mine, t2)[g].o[c] : 0.f;
-    const float rv = ro_remote[g * D + c];
+    for (int t2 = 0; t2 < kDecodeMaxSplits; ++t2) vals[t2] = t2 < S ? slots[t2 * G + g].o[c] : 0.f;
     float o = 0.f;
 #pragma unroll
-    for (int t2 = 0; t2 < kDecodeMaxSplits; ++t2)
-      if (t2 < S) o = fmaf(s_w[t2][g], vals[t2], o);
-    out[((size_t)bi * Hq + kh * G + g) * D + c] = Elem<T>::from_f(o / s_l[g] + rv);
+    for (int t2 = 0; t2 < kDecodeMaxSplits; ++t2) o = fmaf(t2 < S ? s_w[t2][g] : 0.f, vals[t2], o);
+    out[((size_t)bi * Hq + kh * G + g) * D + c] = Elem<T>::from_f(o / s_l[g] + ro[g * D + c]);
   }
-  cluster.sync();   // shared memory of every CTA stays alive until all reads are done
   // the last unit of the sequence advances cache_len (all its CTAs have read it)
-  if (rank == S && tid == 0) {
+  if (tid == 0) {
     __threadfence();
     if (atomicAdd(&seq_counters[bi], 1) == Hkv - 1) {
       seq_counters[bi] = 0;
@@ -535,22 +589,22 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
 }
 
 template <typename T, int D, int G>
-cudaError_t launch_tg(const Ctx& c, int S, int batch, const void* q, const void* kn,
+cudaError_t launch_tg(const Ctx& c, int S, int nst, int batch, const void* q, const void* kn,
                       const void* vn, void* K_ret, void* V_ret, int32_t* cache_len, int cap,
                       const float* M, const float* bstab, void* out, int* counters,
                       cudaStream_t st) {
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   const int r = c.cfg.mem_r;
-  const size_t smem = DecSmem<D, G>::total(kBf16, r);
-  const uint32_t part_off = (uint32_t)DecSmem<D, G>::part_off(kBf16, r);
+  const size_t smem = DecSmem<D, G>::total(kBf16, nst, r, S);
+  const uint32_t slot_off = (uint32_t)DecSmem<D, G>::slot_off(r);
   auto k = decode_kernel<T, D, G>;
-  static bool attr_set[64] = {};   // per instantiation and device
+  static size_t attr_smem[64] = {};   // per instantiation and device: largest size set so far
   const int dv = c.device & 63;
-  if (!attr_set[dv]) {
+  if (attr_smem[dv] < smem) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
-    attr_set[dv] = true;
+    attr_smem[dv] = smem;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(S + 1, c.cfg.n_kv_heads, batch);
@@ -570,38 +624,52 @@ cudaError_t launch_tg(const Ctx& c, int S, int batch, const void* q, const void*
   return cudaLaunchKernelEx(&cfg, k, (const T*)q, (const T*)kn, (const T*)vn, (T*)K_ret,
                             (T*)V_ret, cache_len, cap, c.cfg.n_kv_heads, M, bstab,
                             (const float*)c.W_phi, (const float*)c.w_gate, r, c.cfg.eps,
-                            c.cfg.gate_override, use_ov, (T*)out, counters, c.err, part_off);
+                            c.cfg.gate_override, use_ov, (T*)out, counters, c.err, slot_off, nst);
 }
 
 template <typename T, int D>
-cudaError_t launch_t(const Ctx& c, int S, int batch, const void* q, const void* kn,
+cudaError_t launch_t(const Ctx& c, int S, int nst, int batch, const void* q, const void* kn,
                      const void* vn, void* K_ret, void* V_ret, int32_t* cache_len, int cap,
                      const float* M, const float* bstab, void* out, int* counters,
                      cudaStream_t st) {
   switch (c.group) {
-    case 1: return launch_tg<T, D, 1>(c, S, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
-    case 2: return launch_tg<T, D, 2>(c, S, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
-    case 4: return launch_tg<T, D, 4>(c, S, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
-    case 8: return launch_tg<T, D, 8>(c, S, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
+    case 1: return launch_tg<T, D, 1>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
+    case 2: return launch_tg<T, D, 2>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
+    case 4: return launch_tg<T, D, 4>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
+    case 8: return launch_tg<T, D, 8>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
   }
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-// Attention CTAs per (sequence, KV head) = the cluster size minus one: enough
-// CTAs to cover every SM twice, no CTA streaming more than 1024 rows, at least
-// 64 rows per CTA, and a cluster of at most 16 CTAs.
+// Attention CTAs per (sequence, KV head) = the cluster size minus one: about
+// 1.5 CTAs per SM in one wave, at most 160 cache rows per CTA while that keeps
+// the wave, no CTA streaming more than 1024 rows, clusters of at most 16.
 int decode_splits(int batch, int n_kv_heads, int cap) {
   const int units = batch * n_kv_heads;
-  int S = (2 * 148 + units - 1) / units - 1;
+  int S = (222 + units / 2) / units - 1;
+  const int by_rows = (cap + 159) / 160;
+  if (S > by_rows) S = by_rows;
   const int by_len = (cap + 1023) / 1024;
   if (S < by_len) S = by_len;
-  const int by_rows = (cap + kStageRows - 1) / kStageRows;
-  if (S > by_rows) S = by_rows;
   if (S > kDecodeMaxSplits - 1) S = kDecodeMaxSplits - 1;
   if (S < 1) S = 1;
   return S;
+}
+
+// Stages of 64 rows in an attention CTA's ring. When the whole grid fits in
+// one wave at two CTAs per SM, the ring holds every stage of a CTA's block
+// (all row loads in flight at once, up to 3); otherwise two, which keeps three
+// CTAs per SM resident for the streaming case.
+int decode_stages(int batch, int n_kv_heads, int cap, int S) {
+  const int ctas = batch * n_kv_heads * (S + 1);
+  if (ctas > 2 * 148) return 2;
+  const int per = (cap + S - 1) / S;
+  int nst = (per + kStageRows - 1) / kStageRows;
+  if (nst > 3) nst = 3;   // 3 x 32 KB keeps two CTAs per SM
+  if (nst < 2) nst = 2;
+  return nst;
 }
 
 cudaError_t launch_decode(const Ctx& c, int batch, const void* q, const void* k_new,
@@ -609,13 +677,14 @@ cudaError_t launch_decode(const Ctx& c, int batch, const void* q, const void* k_
                           int cap, const float* M, const float* bstab, void* out,
                           float* /*partials*/, int* counters, cudaStream_t st) {
   const int S = decode_splits(batch, c.cfg.n_kv_heads, cap);
+  const int nst = decode_stages(batch, c.cfg.n_kv_heads, cap, S);
   const int D = c.cfg.head_dim;
   if (c.cfg.dtype == IMEM_BF16) {
-    if (D == 128) return launch_t<__nv_bfloat16, 128>(c, S, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
-    if (D == 64) return launch_t<__nv_bfloat16, 64>(c, S, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
+    if (D == 128) return launch_t<__nv_bfloat16, 128>(c, S, nst, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
+    if (D == 64) return launch_t<__nv_bfloat16, 64>(c, S, nst, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
   } else {
-    if (D == 128) return launch_t<float, 128>(c, S, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
-    if (D == 64) return launch_t<float, 64>(c, S, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
+    if (D == 128) return launch_t<float, 128>(c, S, nst, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
+    if (D == 64) return launch_t<float, 64>(c, S, nst, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -8,7 +8,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
-#include "../../include/indexmem.h"
+#include "indexmem.h"
 
 namespace imem {
 
