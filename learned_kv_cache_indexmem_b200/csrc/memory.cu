@@ -55,19 +55,6 @@ __device__ __forceinline__ uint32_t mn_off(int jj, int cc) {
                     ((((cc & 7) ^ (jj & 7))) << 4));
 }
 
-template <typename T>
-__device__ __forceinline__ void load8h(const T* p, float* f);
-template <>
-__device__ __forceinline__ void load8h<__nv_bfloat16>(const __nv_bfloat16* p, float* f) {
-  bf16x8_to_f32(__ldcs(reinterpret_cast<const uint4*>(p)), f);
-}
-template <>
-__device__ __forceinline__ void load8h<float>(const float* p, float* f) {
-  const float4 a = __ldcs(reinterpret_cast<const float4*>(p));
-  const float4 b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
-  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-}
-
 __device__ __forceinline__ uint4 to_half8(const float* f) {
   uint4 r;
   uint32_t* w = reinterpret_cast<uint32_t*>(&r);
@@ -79,8 +66,33 @@ __device__ __forceinline__ uint4 to_half8(const float* f) {
   return r;
 }
 
+// Eight consecutive elements of a row, kept raw in registers until converted.
+template <typename T> struct RawRow;
+template <> struct RawRow<__nv_bfloat16> {
+  using type = uint4;
+  static __device__ __forceinline__ uint4 load(const __nv_bfloat16* p) {
+    return __ldcs(reinterpret_cast<const uint4*>(p));
+  }
+  static __device__ __forceinline__ uint4 zero() { return make_uint4(0, 0, 0, 0); }
+  static __device__ __forceinline__ void to_f32(const uint4& v, float* f) { bf16x8_to_f32(v, f); }
+};
+struct F8 { float4 a, b; };
+template <> struct RawRow<float> {
+  using type = F8;
+  static __device__ __forceinline__ F8 load(const float* p) {
+    return F8{__ldcs(reinterpret_cast<const float4*>(p)), __ldcs(reinterpret_cast<const float4*>(p) + 1)};
+  }
+  static __device__ __forceinline__ F8 zero() {
+    return F8{make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+  }
+  static __device__ __forceinline__ void to_f32(const F8& v, float* f) {
+    f[0] = v.a.x; f[1] = v.a.y; f[2] = v.a.z; f[3] = v.a.w;
+    f[4] = v.b.x; f[5] = v.b.y; f[6] = v.b.z; f[7] = v.b.w;
+  }
+};
+
 template <typename T, int D>
-__global__ void __launch_bounds__(kMemThreads)
+__global__ void __launch_bounds__(kMemThreads, 2)
 memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t* __restrict__ idx_e,
                  int n_e, int L, int Hkv, float log2lam, int tokens_per_group,
                  float* __restrict__ partials, int* __restrict__ err) {
@@ -134,48 +146,73 @@ memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t
     const T* Kb = K + (size_t)bi * L * row_stride + (size_t)kh * D;
     const T* Vb = V + (size_t)bi * L * row_stride + (size_t)kh * D;
     const int32_t* E = idx_e + (size_t)bi * n_e;
+    // Software pipeline: the rows of chunk c+1 are in flight while chunk c is
+    // converted and written; the evicted positions run one chunk further ahead.
+    using Raw = RawRow<T>;
+    typename Raw::type cur_k[ITEMS], cur_v[ITEMS], nxt_k[ITEMS], nxt_v[ITEMS];
+    int pos_next[ITEMS];
+    auto load_pos = [&](int c, int* pos) {
+#pragma unroll
+      for (int it = 0; it < ITEMS; ++it) {
+        const int j = j0 + c * kChunk + (tid + it * kLoaders) / CH;
+        pos[it] = (c < nchunks && j < j1) ? __ldg(E + j) : -1;
+      }
+    };
+    auto load_rows = [&](const int* pos, typename Raw::type* kr, typename Raw::type* vr) {
+#pragma unroll
+      for (int it = 0; it < ITEMS; ++it) {
+        const int cc = (tid + it * kLoaders) % CH;
+        if (pos[it] >= 0) {
+          kr[it] = Raw::load(Kb + (size_t)pos[it] * row_stride + cc * 8);
+          vr[it] = Raw::load(Vb + (size_t)pos[it] * row_stride + cc * 8);
+        } else {
+          kr[it] = Raw::zero();
+          vr[it] = Raw::zero();
+        }
+      }
+    };
+    int pos_cur[ITEMS];
+    load_pos(0, pos_cur);
+    load_pos(1, pos_next);
+    load_rows(pos_cur, cur_k, cur_v);
     for (int c = 0; c < nchunks; ++c) {
       const int s = c % kStages;
+      if (c + 1 < nchunks) {
+        load_rows(pos_next, nxt_k, nxt_v);
+#pragma unroll
+        for (int it = 0; it < ITEMS; ++it) pos_cur[it] = pos_next[it];
+        load_pos(c + 2, pos_next);
+      }
       if (c >= kStages && !tc::mbar_wait(empty0 + 8 * s, ((c / kStages) - 1) & 1)) {
         record_error(err, DEV_TIMEOUT);
         s_abort = 1;
         break;
       }
-      const uint32_t a_t = sbase + s * TL::STAGE, b_t = a_t + TL::A_BYTES;
       unsigned char* a_p = smem + s * TL::STAGE;
       unsigned char* b_p = a_p + TL::A_BYTES;
       const int base = j0 + c * kChunk;
-      float kf[ITEMS][8], vf[ITEMS][8], wv[ITEMS];
 #pragma unroll
       for (int it = 0; it < ITEMS; ++it) {
         const int i = tid + it * kLoaders;
         const int jj = i / CH, cc = i % CH;
         const int j = base + jj;
-        if (j < j1) {
-          const int pos = E[j];
-          load8h<T>(Kb + (size_t)pos * row_stride + cc * 8, kf[it]);
-          load8h<T>(Vb + (size_t)pos * row_stride + cc * 8, vf[it]);
-          wv[it] = exp2f((float)(n_e - 1 - j) * log2lam);
-        } else {
+        const float wv = (j < j1) ? exp2f((float)(n_e - 1 - j) * log2lam) : 0.f;
+        float kf[8], vf[8];
+        Raw::to_f32(cur_k[it], kf);
+        Raw::to_f32(cur_v[it], vf);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) { kf[it][e] = 0.f; vf[it][e] = 0.f; }
-          wv[it] = 0.f;
-        }
-      }
-#pragma unroll
-      for (int it = 0; it < ITEMS; ++it) {
-        const int i = tid + it * kLoaders;
-        const int jj = i / CH, cc = i % CH;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) vf[it][e] *= wv[it];
-        *reinterpret_cast<uint4*>(a_p + mn_off(jj, cc)) = to_half8(kf[it]);
-        *reinterpret_cast<uint4*>(b_p + mn_off(jj, cc)) = to_half8(vf[it]);
+        for (int e = 0; e < 8; ++e) vf[e] *= wv;
+        *reinterpret_cast<uint4*>(a_p + mn_off(jj, cc)) = to_half8(kf);
+        *reinterpret_cast<uint4*>(b_p + mn_off(jj, cc)) = to_half8(vf);
         if (cc == 0)   // weight column: element 0 of the row in the last B atom
-          *reinterpret_cast<__half*>(b_p + mn_off(jj, (D / 64) * 8)) = __float2half_rn(wv[it]);
+          *reinterpret_cast<__half*>(b_p + mn_off(jj, (D / 64) * 8)) = __float2half_rn(wv);
       }
-      (void)a_t; (void)b_t;
       tc::fence_proxy_async();
       tc::mbar_arrive(full0 + 8 * s);
+      if (c + 1 < nchunks) {
+#pragma unroll
+        for (int it = 0; it < ITEMS; ++it) { cur_k[it] = nxt_k[it]; cur_v[it] = nxt_v[it]; }
+      }
     }
   } else if (lane == 0) {
     // ---------------- MMA issuer

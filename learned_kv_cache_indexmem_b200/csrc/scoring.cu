@@ -15,13 +15,17 @@
 // register max over its TMEM row.
 //
 // Persistent kernel, one CTA per SM. Work item = (sequence, block of 256
-// keys, tile of 128 queries); the causal items of all sequences are
+// keys, tile of 256 queries); the causal items of all sequences are
 // enumerated in closed form and split evenly over the CTAs. Per item the MMA
-// thread issues 2 x 4 tcgen05.mma (M=128 keys, N=128 queries, K=16) from
-// TMA-loaded, 128B-swizzled K-major tiles into one of two 256-column TMEM
-// accumulators; eight epilogue warps drain the other one with tcgen05.ld
-// and masked maxima, and flush a key's maximum with an atomic float max when
-// its key block ends (several CTAs may share a key block).
+// thread issues, for each of the block's two 128-key tiles, 4 tcgen05.mma
+// (M=128 keys, N=256 queries, K=16) from TMA-loaded, 128B-swizzled K-major
+// tiles into that tile's 256-column TMEM accumulator. N=256 halves the
+// shared-memory operand traffic per flop of an N=128 shape, and the two key
+// tiles sharing one query tile halve the L2 traffic of one. Eight epilogue
+// warps drain one accumulator while the other is being computed (tcgen05.ld,
+// masked three-input maxima, a warp per 32 keys x 128 queries) and flush a
+// key's maximum with an atomic float max when its key block ends (several
+// CTAs may share a key block).
 #include "common.cuh"
 #include "internal.h"
 #include "tc.cuh"
@@ -29,16 +33,19 @@
 namespace imem {
 namespace {
 
-constexpr int kKB = 256;        // keys per key block
-constexpr int kQT = 128;        // queries per tile
+constexpr int kKB = 256;        // keys per key block (two M = 128 tiles)
+constexpr int kQT = 256;        // queries per tile (N = 256)
 constexpr int kBStages = 4;     // query-tile ring
 constexpr int kEpiWarps = 8;
 constexpr int kScThreads = 64 + kEpiWarps * 32;
 constexpr int kABytes = kKB * 128;    // 256 rows x 128 B
-constexpr int kBBytes = kQT * 128;    // 128 rows x 128 B
+constexpr int kBBytes = kQT * 128;    // 256 rows x 128 B
 constexpr int kScSmem = 2 * kABytes + kBStages * kBBytes + 1024 + 256;
 
-// Closed-form enumeration of the causal work items of one sequence.
+// Closed-form enumeration of the causal work items of one sequence: key
+// block kb (keys [256 kb, 256 kb + 256)) takes the query tiles of 256 from
+// qs = max(q_begin, 256 kb) to q_end; past q_begin that is Qc - kb tiles with
+// Qc = ceil(q_end / 256), so the prefix sums are arithmetic series.
 struct Sched {
   int q_begin, q_end, nkb, kb0, N0, Qc;
   long long per_seq;
@@ -52,12 +59,12 @@ struct Sched {
     per_seq = prefix(nkb);
   }
   // query tiles of key block kb
-  __host__ __device__ int nq(int kb) const { return kb <= kb0 ? N0 : Qc - 2 * kb; }
+  __host__ __device__ int nq(int kb) const { return kb <= kb0 ? N0 : Qc - kb; }
   // items of key blocks [0, kb)
   __host__ __device__ long long prefix(int kb) const {
     if (kb <= kb0 + 1) return (long long)kb * N0;
     const long long k1 = kb0 + 1, k2 = kb - 1, cnt = k2 - k1 + 1;
-    return (long long)(kb0 + 1) * N0 + cnt * Qc - (k1 + k2) * cnt;
+    return (long long)(kb0 + 1) * N0 + cnt * Qc - (k1 + k2) * cnt / 2;
   }
   __host__ __device__ int qstart(int kb) const { return kb * kKB > q_begin ? kb * kKB : q_begin; }
 };
@@ -176,21 +183,24 @@ scoring_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
           prev = kid;
         }
         const int ab = kbi & 1;
-        const int st = n % kBStages, tb = n & 1;
+        const int st = n % kBStages;
         if (!tc::mbar_wait(b_full + 8 * st, (n / kBStages) & 1)) { record_error(err, DEV_TIMEOUT); break; }
-        if (n >= 2 && !tc::mbar_wait(t_empty + 8 * tb, ((n >> 1) - 1) & 1)) { record_error(err, DEV_TIMEOUT); break; }
-        tc::fence_after();
-#pragma unroll
-        for (int kt = 0; kt < 2; ++kt) {
+        bool ok = true;
+#pragma unroll 1
+        for (int kt = 0; kt < 2; ++kt) {   // the two key tiles share the query tile
+          const int sub = 2 * n + kt, tb = sub & 1;
+          if (sub >= 2 && !tc::mbar_wait(t_empty + 8 * tb, ((sub >> 1) - 1) & 1)) { ok = false; break; }
+          tc::fence_after();
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const uint64_t ad = tc::sdesc_sw128(sA + ab * kABytes + kt * (kABytes / 2) + k * 32, 16, 1024);
             const uint64_t bd = tc::sdesc_sw128(sB + st * kBBytes + k * 32, 16, 1024);
-            tc::mma_f16(tmem + tb * 256 + kt * 128, ad, bd, IDESC, k > 0 ? 1u : 0u);
+            tc::mma_f16(tmem + tb * 256, ad, bd, IDESC, k > 0 ? 1u : 0u);
           }
+          tc::mma_commit(t_full + 8 * tb);
         }
+        if (!ok) { record_error(err, DEV_TIMEOUT); break; }
         tc::mma_commit(b_empty + 8 * st);
-        tc::mma_commit(t_full + 8 * tb);
         cu.next(sc);
         const long long nkid = (long long)cu.seq * sc.nkb + cu.kb;
         if (i + 1 == i_end || nkid != kid) tc::mma_commit(a_empty + 8 * ab);
@@ -199,51 +209,77 @@ scoring_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
       // ---------------- epilogue: masked row maxima, flushed per key block
       const int e = warp - 2;
       const int quarter = warp & 3;        // TMEM lanes this warp may read
-      const int kt = e >> 2;               // key tile of the block (TMEM columns)
+      const int half = e >> 2;             // which 128 of the 256 query columns
       Cursor cu;
       cu.locate(sc, i_begin);
       long long prev = -1;
       int pseq = 0, pkb = 0;
-      float runmax = -INFINITY;
+      float runmax[2] = {-INFINITY, -INFINITY};   // one key in each of the block's two tiles
       auto flush = [&](int seq, int kb) {
-        const int t = kb * kKB + kt * 128 + quarter * 32 + lane;
-        if (t < q_end && runmax != -INFINITY) atomic_max_float(&running_max[(size_t)seq * L + t], runmax);
+#pragma unroll
+        for (int kt = 0; kt < 2; ++kt) {
+          const int t = kb * kKB + kt * 128 + quarter * 32 + lane;
+          if (t < q_end && runmax[kt] != -INFINITY)
+            atomic_max_float(&running_max[(size_t)seq * L + t], runmax[kt]);
+        }
       };
-      for (long long i = i_begin; i < i_end; ++i) {
+      bool ok = true;
+      for (long long i = i_begin; i < i_end && ok; ++i) {
         const long long kid = (long long)cu.seq * sc.nkb + cu.kb;
         if (kid != prev) {
           if (prev >= 0) flush(pseq, pkb);
-          runmax = -INFINITY;
+          runmax[0] = runmax[1] = -INFINITY;
           prev = kid; pseq = cu.seq; pkb = cu.kb;
         }
         const int n = (int)(i - i_begin);
-        const int tb = n & 1;
-        if (!tc::mbar_wait(t_full + 8 * tb, (n >> 1) & 1)) { record_error(err, DEV_TIMEOUT); break; }
-        tc::fence_after();
-        const int t = cu.kb * kKB + kt * 128 + quarter * 32 + lane;
-        const int s0 = sc.qstart(cu.kb) + cu.j * kQT;
-        const bool full = (s0 >= t) && (s0 + kQT <= q_end);
-        const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + tb * 256 + kt * 128;
+        const int s0 = sc.qstart(cu.kb) + cu.j * kQT + half * 128;   // first query of these columns
 #pragma unroll
-        for (int c = 0; c < kQT / 32; ++c) {
-          float v[32];
-          tc::tmem_ld32(base + c * 32, v);
+        for (int kt = 0; kt < 2; ++kt) {
+          if (!tc::mbar_wait(t_full + 8 * kt, n & 1)) { ok = false; break; }
+          tc::fence_after();
+          const int t = cu.kb * kKB + kt * 128 + quarter * 32 + lane;
+          const bool full = (s0 >= t) && (s0 + 128 <= q_end);
+          const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + kt * 256 + half * 128;
+          // all four 32-column loads in flight, one wait
+          uint32_t v0[32], v1[32], v2[32], v3[32];
+          tc::tmem_ld32_async(base + 0, v0);
+          tc::tmem_ld32_async(base + 32, v1);
+          tc::tmem_ld32_async(base + 64, v2);
+          tc::tmem_ld32_async(base + 96, v3);
+          tc::tmem_wait_ld_dep<true>(v0);
+          tc::tmem_wait_ld_dep<false>(v1);
+          tc::tmem_wait_ld_dep<false>(v2);
+          tc::tmem_wait_ld_dep<false>(v3);
+          float m = runmax[kt];
           if (full) {
 #pragma unroll
-            for (int x = 0; x < 32; x += 2) runmax = fmaxf(runmax, fmaxf(v[x], v[x + 1]));
+            for (int x = 0; x < 32; x += 2) {
+              m = tc::max3f(m, __uint_as_float(v0[x]), __uint_as_float(v0[x + 1]));
+              m = tc::max3f(m, __uint_as_float(v1[x]), __uint_as_float(v1[x + 1]));
+              m = tc::max3f(m, __uint_as_float(v2[x]), __uint_as_float(v2[x + 1]));
+              m = tc::max3f(m, __uint_as_float(v3[x]), __uint_as_float(v3[x + 1]));
+            }
           } else {
+            // query s = s0 + column; valid when t <= s < q_end
+            const int lo = t - s0, hi = q_end - s0;   // valid columns: [lo, hi)
 #pragma unroll
             for (int x = 0; x < 32; ++x) {
-              const int s = s0 + c * 32 + x;
-              if (s >= t && s < q_end) runmax = fmaxf(runmax, v[x]);
+              const float a0 = (x >= lo && x < hi) ? __uint_as_float(v0[x]) : -INFINITY;
+              const float a1 = (x + 32 >= lo && x + 32 < hi) ? __uint_as_float(v1[x]) : -INFINITY;
+              const float a2 = (x + 64 >= lo && x + 64 < hi) ? __uint_as_float(v2[x]) : -INFINITY;
+              const float a3 = (x + 96 >= lo && x + 96 < hi) ? __uint_as_float(v3[x]) : -INFINITY;
+              m = tc::max3f(m, a0, a1);
+              m = tc::max3f(m, a2, a3);
             }
           }
+          runmax[kt] = m;
+          tc::fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(t_empty + 8 * kt);
         }
-        tc::fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(t_empty + 8 * tb);
         cu.next(sc);
       }
+      if (!ok) record_error(err, DEV_TIMEOUT);
       if (prev >= 0) flush(pseq, pkb);
     }
   }
