@@ -51,57 +51,89 @@ def load_peaks():
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """Samples nvidia-smi during the timed region."""
-    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    """Samples the GPU's SM clock and clock-event reasons through NVML every
+    10 ms while the timed region runs (thread); nvidia-smi as a fallback."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, gpu_index: int):
-        self.idx = gpu_index
-        self.proc = None
-        self.lines = []
+    def __init__(self, device: torch.device):
+        self.device = device
+        self.samples, self.maxes, self.reasons = [], [], set()
+        self._stop = threading.Event()
+        self._t = None
+        self.h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            props = torch.cuda.get_device_properties(device)
+            uuid = getattr(props, "uuid", None)
+            if uuid is not None:
+                try:
+                    self.h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + str(uuid)).encode())
+                except Exception:
+                    self.h = None
+            if self.h is None:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device.index or 0)
+        except Exception:
+            self.h = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.maxes.append(nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(0.01)
 
     def start(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except Exception:
-            self.proc = None
-
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+        if self.h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.t.join(timeout=2)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 6:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[2:6]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if self._t is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"], "samples": 0}
+        self._stop.set()
+        self._t.join(timeout=2)
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": max(self.maxes) if self.maxes else None,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def reduce_over_ranks(value: float, device, op: str = "max") -> float:
+    """Max (or sum) of a float over the ranks of the default process group;
+    the value itself without one."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX if op == "max"
+                                 else torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+def decode_traffic_from_profile(workload: str):
+    """dram bytes per decode launch from the committed ncu summary, if it was
+    taken on the current decode kernel source (else None)."""
+    import hashlib
+    src = os.path.join(ROOT, "learned_kv_cache_indexmem_b200", "csrc", "decode.cu")
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    sha = hashlib.sha1(open(src, "rb").read()).hexdigest()
+    for line in open(path):
+        parts = line.split()
+        if len(parts) >= 4 and parts[0] == "decode_kernel" and parts[1] == workload:
+            kv = dict(p.split("=", 1) for p in parts[2:] if "=" in p)
+            if kv.get("src_sha1") == sha:
+                return float(kv["bytes_per_launch"])
+    return None
 
 
 # ------------------------------------------------------------------ workload
@@ -328,7 +360,7 @@ def oracle_threads():
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="c2", choices=sorted(synth.WORKLOADS))
@@ -394,8 +426,7 @@ def main():
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(a.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                          else local)
+    clocks = ClockSampler(dev)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -414,10 +445,7 @@ def main():
         "memory": statistics.mean(e[1].elapsed_time(e[2]) for e in ev),
         "decode": statistics.mean(e[2].elapsed_time(e[3]) for e in ev),
     }
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_over_ranks(ms, dev, "max")
     layer_sync_ok = True
     try:
         job.layer.sync(job.stream)
@@ -447,10 +475,7 @@ def main():
     e2e = None
     if not a.no_e2e:
         e2e_ms, h2d, d2h = run_e2e(job, max(2, a.steps // 2), 1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = reduce_over_ranks(e2e_ms, dev, "max")
         e2e = {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
     cpu = None
@@ -468,7 +493,9 @@ def main():
             "dtype": "bf16" if wl.shape.dtype == "bf16" else "f32", "data": "synthetic",
             "config": config,
             "roofline": {"kernel": "decode", "bound": "hbm", "achieved": achieved, "peak": peak,
-                         "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                         "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": decode_traffic_from_profile(wl.name),
+                         "algorithmic_bytes_per_launch": dec_bytes,
                          "peak_source": peaks["source"]},
             "stages": stages,
             "clocks": clk,

@@ -71,7 +71,8 @@ def indexer_features(X, Q, W_iq, W_ik, w_ig):
       gate [b,L,Hq]     sigmoid head gate of each query token
     """
     X, Q, W_iq, W_ik, w_ig = map(f64, (X, Q, W_iq, W_ik, w_ig))
-    qI = np.einsum("blhd,hdj->blhj", Q, W_iq)
+    # per head h: qI[b, l, h, :] = Q[b, l, h, :] @ W_iq[h]  (batched matmul over heads)
+    qI = np.matmul(Q.transpose(0, 2, 1, 3), W_iq[None]).transpose(0, 2, 1, 3)
     kI = X @ W_ik
     gate = sigmoid(X @ w_ig)
     return rms_normalize(qI), rms_normalize(kI), gate
@@ -276,3 +277,31 @@ def prefill_layer(X, Q, K, V, W_iq, W_ik, w_ig, W_phi, lam: float, B: int,
     M, bs = memory_update(K, V, E, W_phi, lam)
     return {"qhat": qhat, "khat": khat, "gate": gate, "I": I, "R": R, "E": E,
             "K_R": KR, "V_R": VR, "M": M, "b": bs}
+
+
+def importance_at_keys(X, Q, W_iq, W_ik, w_ig, keys, q_end: Optional[int] = None,
+                       s_block: int = 4096) -> np.ndarray:
+    """Pooled importance I[t] = max_{s in [t, q_end)} A[s,t] for a few keys t of
+    ONE sequence, streaming the queries in blocks so that long contexts fit in
+    host memory (each A[s,t] is still computed per head by the definition of
+    ``score_block``). X [L,H], Q [L,Hq,d] (one sequence); keys ascending or not.
+    Equals ``pooled_importance`` over the full query range at those keys."""
+    X = np.asarray(X) if not hasattr(X, "detach") else X
+    L = X.shape[0]
+    q_end = L if q_end is None else q_end
+    keys = np.asarray(keys)
+    W_iq, W_ik, w_ig = f64(W_iq), f64(W_ik), f64(w_ig)
+    dI = W_ik.shape[1]
+    # keys' own features
+    _, khat_all, _ = indexer_features(X[None, keys], Q[None, keys], W_iq, W_ik, w_ig)
+    khat = khat_all[0]
+    out = np.full(len(keys), -np.inf)
+    s_min = int(keys.min())
+    for s0 in range(s_min, q_end, s_block):
+        s1 = min(q_end, s0 + s_block)
+        qhat, _, gate = indexer_features(X[None, s0:s1], Q[None, s0:s1], W_iq, W_ik, w_ig)
+        A = score_block(qhat[0], gate[0], khat, dI)                 # [S, T]
+        s_idx = np.arange(s0, s1)[:, None]
+        A = np.where(s_idx >= keys[None, :], A, -np.inf)
+        out = np.maximum(out, A.max(axis=0))
+    return out
