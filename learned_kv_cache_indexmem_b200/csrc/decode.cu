@@ -311,19 +311,28 @@ __device__ void attend_f32(const float* __restrict__ Kb, const float* __restrict
 }
 
 // Merge the per-warp states w_part[0..3][g] into dst[g] (all threads of the
-// block; ends with a barrier).
+// block; ends with a barrier). dst may be another CTA's shared memory: each
+// thread writes 4 consecutive columns with one 16-byte store.
 template <int D, int G>
 __device__ void merge_warps(const Partial<D> (*w_part)[G], Partial<D>* dst) {
   const int tid = threadIdx.x;
   __syncthreads();
-  for (int i = tid; i < G * D; i += kThreads) {
-    const int g = i / D, c = i % D;
+  for (int i = tid; i < G * D / 4; i += kThreads) {
+    const int g = (4 * i) / D, c = (4 * i) % D;
     float mx = -INFINITY;
+#pragma unroll
     for (int w = 0; w < 4; ++w) mx = fmaxf(mx, w_part[w][g].m);
-    float o = 0.f;
-    for (int w = 0; w < 4; ++w)
-      if (w_part[w][g].m != -INFINITY) o += w_part[w][g].o[c] * exp2f(w_part[w][g].m - mx);
-    dst[g].o[c] = o;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      if (w_part[w][g].m != -INFINITY) {
+        const float sc = exp2f(w_part[w][g].m - mx);
+        const float4 v = *reinterpret_cast<const float4*>(&w_part[w][g].o[c]);
+        o.x = fmaf(v.x, sc, o.x); o.y = fmaf(v.y, sc, o.y);
+        o.z = fmaf(v.z, sc, o.z); o.w = fmaf(v.w, sc, o.w);
+      }
+    }
+    *reinterpret_cast<float4*>(&dst[g].o[c]) = o;
   }
   if (tid < G) {
     float mx = -INFINITY;
@@ -568,15 +577,26 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     if (lane == 0) s_l[g] = l;
   }
   __syncthreads();
-  for (int i = tid; i < G * D; i += kThreads) {
-    const int g = i / D, c = i % D;
-    float vals[kDecodeMaxSplits];
+  for (int i = tid; i < G * D / 4; i += kThreads) {   // 4 consecutive columns per thread
+    const int g = (4 * i) / D, c = (4 * i) % D;
+    float4 vals[kDecodeMaxSplits];
 #pragma unroll
-    for (int t2 = 0; t2 < kDecodeMaxSplits; ++t2) vals[t2] = t2 < S ? slots[t2 * G + g].o[c] : 0.f;
-    float o = 0.f;
+    for (int t2 = 0; t2 < kDecodeMaxSplits; ++t2)
+      vals[t2] = t2 < S ? *reinterpret_cast<const float4*>(&slots[t2 * G + g].o[c])
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int t2 = 0; t2 < kDecodeMaxSplits; ++t2) o = fmaf(t2 < S ? s_w[t2][g] : 0.f, vals[t2], o);
-    out[((size_t)bi * Hq + kh * G + g) * D + c] = Elem<T>::from_f(o / s_l[g] + ro[g * D + c]);
+    for (int t2 = 0; t2 < kDecodeMaxSplits; ++t2) {
+      const float w = t2 < S ? s_w[t2][g] : 0.f;
+      o.x = fmaf(w, vals[t2].x, o.x); o.y = fmaf(w, vals[t2].y, o.y);
+      o.z = fmaf(w, vals[t2].z, o.z); o.w = fmaf(w, vals[t2].w, o.w);
+    }
+    const float inv_l = 1.f / s_l[g];
+    float res[4] = {o.x * inv_l + ro[g * D + c], o.y * inv_l + ro[g * D + c + 1],
+                    o.z * inv_l + ro[g * D + c + 2], o.w * inv_l + ro[g * D + c + 3]};
+    T* op = out + ((size_t)bi * Hq + kh * G + g) * D + c;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) op[e] = Elem<T>::from_f(res[e]);
   }
   // the last unit of the sequence advances cache_len (all its CTAs have read it)
   if (tid == 0) {

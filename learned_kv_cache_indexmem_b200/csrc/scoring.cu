@@ -69,30 +69,34 @@ struct Sched {
   __host__ __device__ int qstart(int kb) const { return kb * kKB > q_begin ? kb * kKB : q_begin; }
 };
 
+// Key blocks are visited in folded order 0, nkb-1, 1, nkb-2, ... so that every
+// CTA's contiguous range of items mixes long blocks (few key-tile switches)
+// and short ones (a switch and a diagonal tile every item or two).
+__host__ __device__ inline int fold_kb(int p, int nkb) { return (p & 1) ? nkb - 1 - (p >> 1) : (p >> 1); }
+
+constexpr int kMaxScCtas = 160;
+// Where each CTA's range of items starts (computed on the host per launch).
+struct ScStarts {
+  int seq[kMaxScCtas], p[kMaxScCtas], j[kMaxScCtas], count[kMaxScCtas];
+};
+
 struct Cursor {
-  int seq, kb, j;
-  __device__ void locate(const Sched& sc, long long item) {
-    seq = (int)(item / sc.per_seq);
-    const long long rem = item - (long long)seq * sc.per_seq;
-    int lo = 0, hi = sc.nkb - 1;   // largest kb with prefix(kb) <= rem
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (sc.prefix(mid) <= rem) lo = mid; else hi = mid - 1;
-    }
-    kb = lo;
-    j = (int)(rem - sc.prefix(kb));
+  int seq, p, kb, j;
+  __device__ void init(const Sched& sc, int s0, int p0, int j0) {
+    seq = s0; p = p0; j = j0; kb = fold_kb(p, sc.nkb);
   }
   __device__ void next(const Sched& sc) {
     if (++j == sc.nq(kb)) {
       j = 0;
-      if (++kb == sc.nkb) { kb = 0; ++seq; }
+      if (++p == sc.nkb) { p = 0; ++seq; }
+      kb = fold_kb(p, sc.nkb);
     }
   }
 };
 
 __global__ void __launch_bounds__(kScThreads, 1)
 scoring_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                  int L, int q_begin, int q_end, long long total_items,
+                  int L, int q_begin, int q_end, const __grid_constant__ ScStarts starts,
                   float* __restrict__ running_max, int* __restrict__ err) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -108,9 +112,8 @@ scoring_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   Sched sc;
   sc.init(q_begin, q_end);
-  const long long per_cta = (total_items + gridDim.x - 1) / gridDim.x;
-  const long long i_begin = (long long)blockIdx.x * per_cta;
-  const long long i_end = min(total_items, i_begin + per_cta);
+  const long long i_begin = 0;
+  const long long i_end = starts.count[blockIdx.x];
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -140,7 +143,7 @@ scoring_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     if (warp == 0 && lane == 0) {
       // ---------------- TMA producer
       Cursor cu;
-      cu.locate(sc, i_begin);
+      cu.init(sc, starts.seq[blockIdx.x], starts.p[blockIdx.x], starts.j[blockIdx.x]);
       long long prev = -1;
       int kbi = -1;
       for (long long i = i_begin; i < i_end; ++i) {
@@ -171,7 +174,7 @@ scoring_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
       // ---------------- MMA issuer
       constexpr uint32_t IDESC = tc::idesc(tc::kFmtBF16, 128, kQT, false, false);
       Cursor cu;
-      cu.locate(sc, i_begin);
+      cu.init(sc, starts.seq[blockIdx.x], starts.p[blockIdx.x], starts.j[blockIdx.x]);
       long long prev = -1;
       int kbi = -1;
       for (long long i = i_begin; i < i_end; ++i) {
@@ -211,7 +214,7 @@ scoring_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
       const int quarter = warp & 3;        // TMEM lanes this warp may read
       const int half = e >> 2;             // which 128 of the 256 query columns
       Cursor cu;
-      cu.locate(sc, i_begin);
+      cu.init(sc, starts.seq[blockIdx.x], starts.p[blockIdx.x], starts.j[blockIdx.x]);
       long long prev = -1;
       int pseq = 0, pkb = 0;
       float runmax[2] = {-INFINITY, -INFINITY};   // one key in each of the block's two tiles
@@ -299,8 +302,30 @@ cudaError_t launch_scoring(const Ctx& c, int batch, int L, const __nv_bfloat16* 
   Sched sc;
   sc.init(q_begin, q_end);
   const long long total = sc.per_seq * batch;
-  int grid = c.num_sms;
+  int grid = c.num_sms < kMaxScCtas ? c.num_sms : kMaxScCtas;
   if (total < grid) grid = (int)total;
+  // split the folded item sequence evenly; record each CTA's starting position
+  ScStarts starts;
+  {
+    const long long per = (total + grid - 1) / grid;
+    int seq = 0, p = 0, j = 0;
+    long long done = 0;
+    for (int b = 0; b < grid; ++b) {
+      const long long cnt = (total - done) < per ? (total - done) : per;
+      starts.seq[b] = seq; starts.p[b] = p; starts.j[b] = j; starts.count[b] = (int)cnt;
+      long long left = cnt;   // advance by cnt items, a key block at a time
+      while (left > 0) {
+        const int kb = fold_kb(p, sc.nkb);
+        const int rest = sc.nq(kb) - j;
+        if (left < rest) { j += (int)left; left = 0; }
+        else {
+          left -= rest; j = 0;
+          if (++p == sc.nkb) { p = 0; ++seq; }
+        }
+      }
+      done += cnt;
+    }
+  }
   static bool attr_set[64] = {};
   if (!attr_set[c.device & 63]) {
     cudaError_t e = cudaFuncSetAttribute(scoring_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -308,7 +333,7 @@ cudaError_t launch_scoring(const Ctx& c, int batch, int L, const __nv_bfloat16* 
     if (e != cudaSuccess) return e;
     attr_set[c.device & 63] = true;
   }
-  scoring_tc_kernel<<<grid, kScThreads, kScSmem, st>>>(mq, mk, L, q_begin, q_end, total,
+  scoring_tc_kernel<<<grid, kScThreads, kScSmem, st>>>(mq, mk, L, q_begin, q_end, starts,
                                                        running_max, c.err);
   return cudaGetLastError();
 }
