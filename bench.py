@@ -260,6 +260,63 @@ class Job:
         return self.batch * (self.L + self.n_dec)
 
 
+# ------------------------------------------------------------------ full-cache decode
+
+def full_cache_decode(job, steps=64, reps=3):
+    """The same decode kernel over the full context (budget B = L: nothing
+    evicted, memory state empty) next to the evicted cache, per decode step:
+    the pages' claim that decoding with eviction and memory stays competitive
+    with the full cache ("IndexMem" technical summary §4, Efficiency)."""
+    s = job.wl.shape
+    b, L = job.batch, job.L
+    cap = L + steps
+    full = job.layer.new_state(b, L, L, cap, job.dev)
+    full.K_ret[:, :L] = job.inp["K"]
+    full.V_ret[:, :L] = job.inp["V"]
+    full.cache_len.fill_(L)
+    len0 = full.cache_len.clone()
+    evicted = job.layer.new_state(b, L, job.B, job.B + steps, job.dev)
+    evicted.K_ret[:, :job.B] = job.st.K_ret[:, :job.B]
+    evicted.V_ret[:, :job.B] = job.st.V_ret[:, :job.B]
+    evicted.M.copy_(job.st.M)
+    evicted.bstab.copy_(job.st.bstab)
+    evicted.cache_len.fill_(job.B)
+    elen0 = evicted.cache_len.clone()
+    out = torch.empty_like(job.decin["q"][0])
+    res = {}
+    for name, st, l0 in (("full", full, len0), ("evicted", evicted, elen0)):
+        with torch.cuda.stream(job.stream):
+            st.cache_len.copy_(l0)
+            job.layer.decode(job.decin["q"][0], job.decin["k_new"][0], job.decin["v_new"][0], st,
+                             out=out, stream=job.stream)
+            torch.cuda.synchronize()
+            st.cache_len.copy_(l0)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=job.stream):
+                for i in range(steps):
+                    job.layer.decode(job.decin["q"][i], job.decin["k_new"][i], job.decin["v_new"][i],
+                                     st, out=out, stream=job.stream)
+            best = None
+            for _ in range(reps):
+                st.cache_len.copy_(l0)
+                torch.cuda.synchronize()
+                a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(job.stream)
+                g.replay()
+                e.record(job.stream)
+                torch.cuda.synchronize()
+                t = a.elapsed_time(e) / steps * 1e3
+                best = t if best is None else min(best, t)
+            del g
+        res[name] = best
+    job.layer.sync(job.stream)
+    row = s.n_kv_heads * s.head_dim * (2 if s.dtype == "bf16" else 4) * 2
+    return {"steps": steps, "us_per_step_full_cache": res["full"],
+            "us_per_step_evicted": res["evicted"], "speedup": res["full"] / res["evicted"],
+            "full_cache_GBps": b * (L + steps / 2) * row / (res["full"] * 1e-6) / 1e9}
+
+
 # ------------------------------------------------------------------ e2e
 
 def run_e2e(job, steps, warmup):
@@ -367,6 +424,8 @@ def main():
     ap.add_argument("--budget", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-full-cache", action="store_true",
+                    help="skip the full-cache decode comparison")
     a = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -478,6 +537,9 @@ def main():
         e2e_ms = reduce_over_ranks(e2e_ms, dev, "max")
         e2e = {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    full_cmp = None
+    if not a.no_full_cache:
+        full_cmp = full_cache_decode(job)
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         t_full, desc = cpu_oracle_sample(wl, B)
@@ -501,6 +563,7 @@ def main():
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "full_cache_decode": full_cmp,
             "gpu_launches": job.launches_per_step() * a.steps,
             "device_errors": not layer_sync_ok,
         }))

@@ -408,6 +408,17 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   // phase 0 of the cluster barrier: "this CTA is running" (remote shared
   // memory is written only after every CTA of the cluster has arrived)
   cluster_arrive_relaxed();
+  if (rank == S) {
+    // W_phi belongs to the context and is written only at imem_init, so the
+    // readout CTA may stage it before waiting for the previous kernel
+    float* sW = reinterpret_cast<float*>(dyn_smem);          // [r][D], chunks XOR-swizzled
+    const uint32_t wdst = smem_u32(sW);
+    for (int i = tid; i < r * D / 4; i += kThreads) {
+      const int j = (4 * i) / D, cc = ((4 * i) % D) / 4;
+      cp_async16(wdst + (uint32_t)(j * D + ((cc ^ (j & 7)) * 4)) * 4u, W_phi + 4 * i, true);
+    }
+    cp_async_commit();
+  }
   // With programmatic dependent launch this kernel may start while the
   // previous kernel of the stream is still running: wait for it before
   // reading anything another kernel may write (q, the cache, cache_len, M, b).
@@ -458,11 +469,6 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   float* snum = sgate + G;                                  // [4][G][D] partial M^T u
   float* ro = snum + 4 * G * D;                             // [G][D] = g * m
   {
-    const uint32_t wdst = smem_u32(sW);
-    for (int i = tid; i < r * D / 4; i += kThreads) {
-      const int j = (4 * i) / D, cc = ((4 * i) % D) / 4;
-      cp_async16(wdst + (uint32_t)(j * D + ((cc ^ (j & 7)) * 4)) * 4u, W_phi + 4 * i, true);
-    }
     for (int i = tid; i < r / 4; i += kThreads)
       cp_async16(smem_u32(sb) + (uint32_t)i * 16u, bstab + (size_t)unit * r + 4 * i, true);
     cp_async_commit();
