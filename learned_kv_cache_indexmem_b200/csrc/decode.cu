@@ -10,21 +10,30 @@
 // blocks -- the online-softmax identity stated in "Context Memorization for
 // Efficient Long Context Generation" (technical summary, Method).
 //
-// Grid (S + 1, Hkv, batch). For each (sequence, KV head) -- a "unit" -- CTAs
-// 0..S-1 each stream a contiguous block of cache rows and keep one softmax
-// state per query head of the GQA group; CTA S computes the memory readout
+// Grid (S + 1, Hkv, batch), one thread-block cluster of S + 1 CTAs per
+// (sequence, KV head) -- a "unit". CTAs 0..S-1 each stream a contiguous block
+// of cache rows and keep one softmax state per query head of the GQA group;
+// CTA S computes the memory readout
 //   u = W_phi q,  m = M^T u / (b . u + eps),  g = sigmoid(w_gate . q)
-// concurrently. Every CTA publishes its result to the workspace and counts
-// itself on the unit's counter (no waiting); the last one to arrive merges
-// the S softmax states, adds g*m and writes the output, and the last unit of
-// a sequence advances cache_len. Split 0 appends the new key/value row to the
-// cache; the CTA whose block covers row cache_len reads it from k_new/v_new.
+// meanwhile. Each attention CTA merges its warps' states straight into a slot
+// of CTA S's shared memory (distributed shared memory), then arrives on the
+// cluster barrier; CTA S merges the S states, adds g*m and writes the output.
+// The last unit of a sequence advances cache_len. CTA 0 appends the new
+// key/value row to the cache; the CTA whose block covers row cache_len reads
+// it from k_new/v_new.
 //
-// bf16 attention: rows are staged in shared memory with cp.async (two 64-row
-// stages, XOR-swizzled 16-byte chunks) and contracted with warp-level
-// tensor-core MMA (m16n8k16, fp32 accumulation): S^T = q K^T with the GQA
-// heads as the M dimension, then O += P V reusing the score fragments as the
-// A operand. fp32 attention: the same structure on CUDA cores.
+// Latency: the kernel is launched with programmatic stream serialization, so
+// its CTAs are resident before the previous kernel ends. CTA S stages W_phi
+// (owned by the context) before the wait; an attention CTA reads a hint of
+// cache_len before it and, right after it, issues the loads of the rows that
+// lie below the hint in its block, so they travel alongside the reads of q
+// and the true length (a wrong hint only costs those loads).
+//
+// bf16 attention: rows are staged in shared memory with cp.async (a ring of
+// two or three 64-row stages, XOR-swizzled 16-byte chunks) and contracted
+// with warp-level tensor-core MMA (m16n8k16, fp32 accumulation): S^T = q K^T
+// with the GQA heads as the M dimension, then O += P V reusing the score
+// fragments as the A operand. fp32 attention: CUDA cores.
 #include "common.cuh"
 #include "internal.h"
 
@@ -102,11 +111,40 @@ __device__ __forceinline__ uint32_t tile_off(int row, int c) {
 
 // ---- attention over rows [r0, r1) for one unit, bf16 tensor-core path --------
 // Leaves the per-warp states in s_part[warp][g].
+// Issues the loads of cache rows [r0 + 64 s, min(r0 + 64 s + 64, hi)) into
+// ring buffer s for s < n_st, one cp.async group per stage; the other rows of
+// those buffers are not touched.
+template <int D>
+__device__ void issue_rows(unsigned char* stage_mem, const __nv_bfloat16* __restrict__ Kb,
+                           const __nv_bfloat16* __restrict__ Vb, size_t row_stride, int r0, int hi,
+                           int n_st) {
+  constexpr int CH = D / 8;
+  constexpr int STAGE_BYTES = kStageRows * D * 2;
+  const uint32_t sbase = smem_u32(stage_mem);
+  for (int s = 0; s < n_st; ++s) {
+    const int base = r0 + s * kStageRows;
+    const int rows = min(kStageRows, hi - base);
+    const uint32_t kdst = sbase + s * 2 * STAGE_BYTES;
+    const uint32_t vdst = kdst + STAGE_BYTES;
+    for (int i = threadIdx.x; i < rows * CH; i += kThreads) {
+      const int rr = i / CH, c = i % CH;
+      const size_t off = (size_t)(base + rr) * row_stride + c * 8;
+      cp_async16(kdst + tile_off<D>(rr, c), Kb + off, true);
+      cp_async16(vdst + tile_off<D>(rr, c), Vb + off, true);
+    }
+    cp_async_commit();
+  }
+}
+
+// Stage buffers 0..n_spec-1 may already hold rows [r0, spec_end) (issued by
+// issue_rows before the row range was known); the rest of those stages is
+// filled here and the ring continues from stage n_spec.
 template <int D, int G>
 __device__ void attend_bf16(const __nv_bfloat16* __restrict__ Kb, const __nv_bfloat16* __restrict__ Vb,
                             size_t row_stride, const __nv_bfloat16* kn, const __nv_bfloat16* vn,
                             int len, int r0, int r1, const float (*s_q)[D],
-                            Partial<D> (*s_part)[G], unsigned char* stage_mem, int nst) {
+                            Partial<D> (*s_part)[G], unsigned char* stage_mem, int nst,
+                            int spec_end, int n_spec) {
   constexpr int CH = D / 8;                 // 16-byte chunks per row
   constexpr int STAGE_BYTES = kStageRows * D * 2;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -146,9 +184,33 @@ __device__ void attend_bf16(const __nv_bfloat16* __restrict__ Kb, const __nv_bfl
     cp_async_commit();
   };
 
+  // rows of the stages issued ahead that those loads did not cover: the cache
+  // rows in [spec_end, r1) (at most two, the new row among them) and zeros
+  // past r1, written with plain loads and stores
+  for (int st = 0; st < n_spec; ++st) {
+    const int base = r0 + st * kStageRows;
+    const int lo = max(base, spec_end);
+    const int cnt = base + kStageRows - lo;
+    const uint32_t kdst = sbase + st * 2 * STAGE_BYTES;
+    const uint32_t vdst = kdst + STAGE_BYTES;
+    for (int i = tid; i < cnt * CH; i += kThreads) {
+      const int row = lo + i / CH, c = i % CH, rr = row - base;
+      uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = kv;
+      if (row < r1) {
+        const __nv_bfloat16* ks = (row == len) ? kn : Kb + (size_t)row * row_stride;
+        const __nv_bfloat16* vs = (row == len) ? vn : Vb + (size_t)row * row_stride;
+        kv = __ldcg(reinterpret_cast<const uint4*>(ks + c * 8));
+        vv = __ldcg(reinterpret_cast<const uint4*>(vs + c * 8));
+      }
+      asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(kdst + tile_off<D>(rr, c)),
+                   "r"(kv.x), "r"(kv.y), "r"(kv.z), "r"(kv.w));
+      asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(vdst + tile_off<D>(rr, c)),
+                   "r"(vv.x), "r"(vv.y), "r"(vv.z), "r"(vv.w));
+    }
+  }
   // ring of nst stages, all issued up front as far as the ring allows
   const int n_stages = (r1 - r0 + kStageRows - 1) / kStageRows;
-  int issued = 0;
+  int issued = n_spec;
   for (; issued < n_stages && issued < nst; ++issued) issue(issued, issued);
   for (int st = 0; st < n_stages; ++st) {
     cp_async_wait_dyn(issued - (st + 1));   // groups younger than stage st may stay pending
@@ -361,6 +423,22 @@ __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }
 
+// Cache rows per attention CTA for n rows over S CTAs: ceil(n / S) rounded up
+// to 16 (one warp's rows of a stage), so that the split changes only every
+// 16 S rows and a split chosen from a slightly stale length is usually right.
+__device__ __forceinline__ int split_rows(int n, int S) { return ((n + S - 1) / S + 15) & ~15; }
+
+__device__ __forceinline__ int ld_relaxed(const int32_t* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ int atomic_add_acq_rel(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 // Dynamic shared memory of one decode CTA (bytes). Attention CTAs use
 // [0, att) for their row stages (then for the per-warp states); the readout
 // CTA uses [0, readout) for its operands and result and receives the S
@@ -403,6 +481,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   __shared__ __align__(16) float s_q[G][D];
   __shared__ float s_w[kDecodeMaxSplits][G];
   __shared__ float s_l[G];
+  __shared__ int s_len_hint;
   Partial<D>* slots = reinterpret_cast<Partial<D>*>(dyn_smem + slot_off);   // readout CTA only
 
   // phase 0 of the cluster barrier: "this CTA is running" (remote shared
@@ -419,25 +498,59 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     }
     cp_async_commit();
   }
+  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+  const size_t row_stride = (size_t)Hkv * D;
+  const T* Kb = K_ret + (size_t)bi * cap * row_stride + (size_t)kh * D;
+  const T* Vb = V_ret + (size_t)bi * cap * row_stride + (size_t)kh * D;
+  // A hint of cache_len, read before the wait (relaxed: the previous kernel
+  // may be advancing it). It only picks the rows whose loads are issued
+  // straight after the wait; the true length read after the wait decides.
+  if (kBf16 && rank < S) {
+    if (tid == 0) s_len_hint = max(0, min(ld_relaxed(cache_len + bi), cap - 1));
+    __syncthreads();
+  }
   // With programmatic dependent launch this kernel may start while the
   // previous kernel of the stream is still running: wait for it before
   // reading anything another kernel may write (q, the cache, cache_len, M, b).
   griddep_wait();
-  for (int i = tid; i < G * D; i += kThreads)
-    s_q[i / D][i % D] = Elem<T>::to_f(q[((size_t)bi * Hq + kh * G) * D + i]);
+  int len_h = 0, per_h = 0, spec_end = 0, n_spec = 0;
+  if constexpr (kBf16) {
+    if (rank < S) {
+      // rows [r0, spec_end) lie below the hinted length: if the true length is
+      // at least the hint and gives the same split, they are cache rows of
+      // this CTA's block that nothing in this step writes
+      len_h = s_len_hint;
+      per_h = split_rows(len_h + 1, S);
+      const int r0h = rank * per_h;
+      spec_end = min(min(r0h + per_h, r0h + nst * kStageRows), len_h);
+      if (spec_end > r0h) {
+        n_spec = (spec_end - r0h + kStageRows - 1) / kStageRows;
+        issue_rows<D>(dyn_smem, Kb, Vb, row_stride, r0h, spec_end, n_spec);
+      }
+    }
+  }
+  static_assert(D % 8 == 0, "q is read in groups of 8 elements");
+  for (int i = tid; i < G * D / 8; i += kThreads) {
+    float f[8];
+    load8<T>(q + ((size_t)bi * Hq + kh * G) * D + 8 * i, f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s_q[(8 * i + e) / D][(8 * i + e) % D] = f[e];
+  }
   const int len = cache_len[bi];
   if (len >= cap) {   // full cache: the whole cluster (same sequence) skips it
     if (rank == 0 && kh == 0 && tid == 0) record_error(err, DEV_CACHE_FULL);
+    cp_async_wait<0>();
     return;
   }
   griddep_launch();
   const int n = len + 1;
+  if (n_spec > 0 && !(len >= len_h && split_rows(n, S) == per_h)) {
+    cp_async_wait<0>();   // wrong guess: drop the early loads (barrier below)
+    n_spec = 0;
+  }
   __syncthreads();
 
-  const size_t row_stride = (size_t)Hkv * D;
   if (rank < S) {
-    const T* Kb = K_ret + (size_t)bi * cap * row_stride + (size_t)kh * D;
-    const T* Vb = V_ret + (size_t)bi * cap * row_stride + (size_t)kh * D;
     const T* kn = k_new + ((size_t)bi * Hkv + kh) * D;
     const T* vn = v_new + ((size_t)bi * Hkv + kh) * D;
     if (rank == 0) {   // append the new row
@@ -445,11 +558,12 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
       T* vd = V_ret + ((size_t)bi * cap + len) * row_stride + (size_t)kh * D;
       for (int c = tid; c < D; c += kThreads) { kd[c] = kn[c]; vd[c] = vn[c]; }
     }
-    const int per = (n + S - 1) / S;
+    const int per = split_rows(n, S);
     const int r0 = min(n, rank * per), r1 = min(n, r0 + per);
     auto* w_part = reinterpret_cast<Partial<D>(*)[G]>(dyn_smem);   // aliases the stages
-    if constexpr (std::is_same<T, __nv_bfloat16>::value)
-      attend_bf16<D, G>(Kb, Vb, row_stride, kn, vn, len, r0, r1, s_q, w_part, dyn_smem, nst);
+    if constexpr (kBf16)
+      attend_bf16<D, G>(Kb, Vb, row_stride, kn, vn, len, r0, r1, s_q, w_part, dyn_smem, nst,
+                        spec_end, n_spec);
     else
       attend_f32<D, G>(Kb, Vb, row_stride, kn, vn, len, r0, r1, s_q, w_part);
     cluster_wait();   // phase 0 complete: every CTA of the cluster is running
@@ -573,6 +687,12 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   cluster_wait();             // phase 0
   cluster_arrive_release();   // phase 1: own arrival
   cluster_wait();             // phase 1: every attention CTA has written its slot
+  // Every CTA of this unit has read cache_len by now; count the unit on its
+  // sequence's counter (the result is used at the end, so the atomic's round
+  // trip overlaps the merge). acq_rel: the last unit's update of cache_len is
+  // ordered after every other unit's reads.
+  int arrived = 0;
+  if (tid == 0) arrived = atomic_add_acq_rel(&seq_counters[bi], 1);
   // merge weights: a warp per head, a lane per slot (S <= 15 < 32)
   for (int g = warp; g < G; g += kThreads / 32) {
     const float mt = lane < S ? slots[lane * G + g].m : -INFINITY;
@@ -605,12 +725,9 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     for (int e = 0; e < 4; ++e) op[e] = Elem<T>::from_f(res[e]);
   }
   // the last unit of the sequence advances cache_len (all its CTAs have read it)
-  if (tid == 0) {
-    __threadfence();
-    if (atomicAdd(&seq_counters[bi], 1) == Hkv - 1) {
-      seq_counters[bi] = 0;
-      cache_len[bi] = len + 1;
-    }
+  if (tid == 0 && arrived == Hkv - 1) {
+    seq_counters[bi] = 0;
+    cache_len[bi] = len + 1;
   }
 }
 
