@@ -45,16 +45,16 @@ Workspace workspace_layout(const Ctx& c, int batch, int L) {
   return w;
 }
 
-bool make_tmap_rows64(const Ctx& c, CUtensorMap* map, const void* base, uint64_t rows,
-                      uint32_t box_rows) {
+bool make_tmap_bf16(const Ctx& c, CUtensorMap* map, const void* base, uint64_t width,
+                    uint64_t rows, uint32_t box_rows) {
   using Fn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                           const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
                           CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
                           CUtensorMapFloatOOBfill);
   if (!c.encode_tiled) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)kIdxPad, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)kIdxPad * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)kIdxPad, box_rows};
+  const cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)width * 2};
+  const cuuint32_t box[2] = {64u, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = ((Fn)c.encode_tiled)(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                                           const_cast<void*>(base), dims, strides, box, estr,
@@ -62,6 +62,11 @@ bool make_tmap_rows64(const Ctx& c, CUtensorMap* map, const void* base, uint64_t
                                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_rows64(const Ctx& c, CUtensorMap* map, const void* base, uint64_t rows,
+                      uint32_t box_rows) {
+  return make_tmap_bf16(c, map, base, kIdxPad, rows, box_rows);
 }
 
 }  // namespace imem

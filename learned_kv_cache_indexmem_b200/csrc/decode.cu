@@ -36,6 +36,7 @@
 // fragments as the A operand. fp32 attention: CUDA cores.
 #include "common.cuh"
 #include "internal.h"
+#include "tc.cuh"
 
 #include <cooperative_groups.h>
 #include <math.h>
@@ -74,8 +75,7 @@ __device__ __forceinline__ void cp_async_wait_dyn(int n) {
   if (n <= 0) cp_async_wait<0>();
   else if (n == 1) cp_async_wait<1>();
   else if (n == 2) cp_async_wait<2>();
-  else if (n == 3) cp_async_wait<3>();
-  else cp_async_wait<4>();
+  else cp_async_wait<3>();
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -102,54 +102,103 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// byte offset of 16-byte chunk `c` of row `row` in a staged tile of D-element
-// bf16 rows (XOR swizzle keeps ldmatrix conflict-free)
+// Stage buffers hold K then V, each as D/64 column halves of [64 rows][128 B]
+// written by TMA with the 128-byte swizzle: 16-byte chunk cc of row rr of a
+// half sits at rr * 128 + ((cc ^ (rr & 7)) << 4), which keeps ldmatrix
+// conflict-free. tile_off gives the byte offset of chunk c (0..D/8) of a row.
 template <int D>
 __device__ __forceinline__ uint32_t tile_off(int row, int c) {
-  return (uint32_t)(row * (D * 2) + ((c ^ (row & 7)) << 4));
+  return (uint32_t)((c >> 3) * (kStageRows * 128) + row * 128 + (((c & 7) ^ (row & 7)) << 4));
 }
-
-// ---- attention over rows [r0, r1) for one unit, bf16 tensor-core path --------
-// Leaves the per-warp states in s_part[warp][g].
-// Issues the loads of cache rows [r0 + 64 s, min(r0 + 64 s + 64, hi)) into
-// ring buffer s for s < n_st, one cp.async group per stage; the other rows of
-// those buffers are not touched.
 template <int D>
-__device__ void issue_rows(unsigned char* stage_mem, const __nv_bfloat16* __restrict__ Kb,
-                           const __nv_bfloat16* __restrict__ Vb, size_t row_stride, int r0, int hi,
-                           int n_st) {
-  constexpr int CH = D / 8;
-  constexpr int STAGE_BYTES = kStageRows * D * 2;
-  const uint32_t sbase = smem_u32(stage_mem);
-  for (int s = 0; s < n_st; ++s) {
-    const int base = r0 + s * kStageRows;
-    const int rows = min(kStageRows, hi - base);
-    const uint32_t kdst = sbase + s * 2 * STAGE_BYTES;
-    const uint32_t vdst = kdst + STAGE_BYTES;
-    for (int i = threadIdx.x; i < rows * CH; i += kThreads) {
-      const int rr = i / CH, c = i % CH;
-      const size_t off = (size_t)(base + rr) * row_stride + c * 8;
-      cp_async16(kdst + tile_off<D>(rr, c), Kb + off, true);
-      cp_async16(vdst + tile_off<D>(rr, c), Vb + off, true);
-    }
-    cp_async_commit();
+constexpr uint32_t kTileBytes = kStageRows * D * 2;   // one of K, V in a stage
+
+// Ring of nst stage buffers, each with a transaction barrier. Global stage
+// index gi uses buffer gi % nst in phase (gi / nst) & 1. Thread 0 issues the
+// loads; last[b] (thread 0 only) is the last index issued into buffer b.
+struct Ring {
+  uint32_t buf0;   // shared address of buffer 0 (1024-byte aligned)
+  uint32_t bar0;   // shared address of barrier 0 (barriers 8 bytes apart)
+  int nst;
+  int last[kDecodeMaxStages];
+};
+
+// Thread 0: loads the 64 cache rows starting at 2-D row y (of the [batch*cap,
+// Hkv*D] view) into buffer gi % nst, columns x0..x0+D-1. A buffer is reused
+// only once the load issued into it before has landed.
+template <int D>
+__device__ void ring_issue(Ring& rg, const CUtensorMap* tmK, const CUtensorMap* tmV, int gi,
+                           int x0, int y, int* err) {
+  const int b = gi % rg.nst;
+  const uint32_t bar = rg.bar0 + 8u * b;
+  if (rg.last[b] >= 0 && !tc::mbar_wait(bar, (uint32_t)(rg.last[b] / rg.nst) & 1u))
+    record_error(err, DEV_TIMEOUT);
+  rg.last[b] = gi;
+  const uint32_t dst = rg.buf0 + (uint32_t)b * 2u * kTileBytes<D>;
+  tc::mbar_expect_tx(bar, 2u * kTileBytes<D>);
+#pragma unroll
+  for (int h = 0; h < D / 64; ++h) {
+    tc::tma_load_2d(dst + h * (kStageRows * 128), tmK, bar, x0 + 64 * h, y);
+    tc::tma_load_2d(dst + kTileBytes<D> + h * (kStageRows * 128), tmV, bar, x0 + 64 * h, y);
   }
 }
 
-// Stage buffers 0..n_spec-1 may already hold rows [r0, spec_end) (issued by
-// issue_rows before the row range was known); the rest of those stages is
-// filled here and the ring continues from stage n_spec.
-template <int D, int G>
-__device__ void attend_bf16(const __nv_bfloat16* __restrict__ Kb, const __nv_bfloat16* __restrict__ Vb,
-                            size_t row_stride, const __nv_bfloat16* kn, const __nv_bfloat16* vn,
-                            int len, int r0, int r1, const float (*s_q)[D],
-                            Partial<D> (*s_part)[G], unsigned char* stage_mem, int nst,
-                            int spec_end, int n_spec) {
+// Thread 0: waits until the last load issued into every buffer has landed
+// (before the buffers are reused for something else or the CTA exits).
+template <int D>
+__device__ void ring_drain(const Ring& rg, int* err) {
+  for (int b = 0; b < rg.nst; ++b)
+    if (rg.last[b] >= 0 && !tc::mbar_wait(rg.bar0 + 8u * b, (uint32_t)(rg.last[b] / rg.nst) & 1u))
+      record_error(err, DEV_TIMEOUT);
+}
+
+// All threads: the cp.async form of ring_issue for rows [y_row, y_row + 64)
+// of this unit's cache (Kb/Vb point at row 0, rows `row_stride` apart). Rows
+// at or past `hi` are not loaded (zero-filled); one commit group per stage.
+template <int D>
+__device__ void ring_issue_lsu(const Ring& rg, const __nv_bfloat16* __restrict__ Kb,
+                               const __nv_bfloat16* __restrict__ Vb, size_t row_stride, int gi,
+                               int base, int hi) {
+  constexpr int CH = D / 8;
+  const uint32_t kdst = rg.buf0 + (uint32_t)(gi % rg.nst) * 2u * kTileBytes<D>;
+  const uint32_t vdst = kdst + kTileBytes<D>;
+  // thread -> (row rr = tid / CH + k * kThreads / CH, chunk c = tid % CH): the
+  // chunk and the swizzle term (rr & 7) stay fixed over k
+  const int c = threadIdx.x % CH, rr0 = threadIdx.x / CH;
+  constexpr int RSTEP = kThreads / CH;
+#pragma unroll
+  for (int k = 0; k < kStageRows / RSTEP; ++k) {
+    const int rr = rr0 + k * RSTEP, row = base + rr;
+    const bool ok = row < hi;
+    const size_t off = (size_t)(ok ? row : 0) * row_stride + c * 8;
+    cp_async16(kdst + tile_off<D>(rr, c), Kb + off, ok);
+    cp_async16(vdst + tile_off<D>(rr, c), Vb + off, ok);
+  }
+  cp_async_commit();
+}
+
+// ---- attention over rows [r0, r1) for one unit, bf16 tensor-core path --------
+// Stage st (rows r0 + 64 st ..) has global index g0 + st; stages below n_pre
+// were issued before the row range was known. Rows past r1 in a stage are
+// zeroed in shared memory, row len (the new token) is taken from kn/vn.
+// Leaves the per-warp states in s_part[warp][g].
+//
+// kTma: stages are loaded by TMA (thread 0 issues, transaction barriers);
+// otherwise by cp.async from every thread (rows below `hi` only). TMA frees
+// the SM's issue slots and wins when CTAs stream in several waves; cp.async
+// delivers the first rows sooner and wins when the grid is one wave.
+template <int D, int G, bool kTma>
+__device__ void attend_bf16(Ring& rg, const CUtensorMap* tmK, const CUtensorMap* tmV, int x0,
+                            int y0, const __nv_bfloat16* __restrict__ Kb,
+                            const __nv_bfloat16* __restrict__ Vb, size_t row_stride, int hi,
+                            const __nv_bfloat16* kn, const __nv_bfloat16* vn, int len,
+                            int r0, int r1, int g0, int n_pre, const float (*s_q)[D],
+                            Partial<D> (*s_part)[G], int* err) {
   constexpr int CH = D / 8;                 // 16-byte chunks per row
-  constexpr int STAGE_BYTES = kStageRows * D * 2;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   const float sscale = kLog2e * rsqrtf((float)D);
+  const int nst = rg.nst;
 
   // q as A fragments (heads on M, rows >= G zero): a0 = dims 16s+2t.., a2 = +8
   uint32_t qa0[D / 16], qa2[D / 16];
@@ -167,58 +216,49 @@ __device__ void attend_bf16(const __nv_bfloat16* __restrict__ Kb, const __nv_bfl
   for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
   float m_run = -INFINITY, l_run = 0.f;
 
-  const uint32_t sbase = smem_u32(stage_mem);
-  auto issue = [&](int stage, int buf) {
-    const int base = r0 + stage * kStageRows;
-    const uint32_t kdst = sbase + buf * 2 * STAGE_BYTES;
-    const uint32_t vdst = kdst + STAGE_BYTES;
-    for (int i = tid; i < kStageRows * CH; i += kThreads) {
-      const int rr = i / CH, c = i % CH;
-      const int row = base + rr;
-      const bool ok = row < r1;
-      const __nv_bfloat16* ks = (row == len) ? kn : Kb + (size_t)(ok ? row : r0) * row_stride;
-      const __nv_bfloat16* vs = (row == len) ? vn : Vb + (size_t)(ok ? row : r0) * row_stride;
-      cp_async16(kdst + tile_off<D>(rr, c), ks + c * 8, ok);
-      cp_async16(vdst + tile_off<D>(rr, c), vs + c * 8, ok);
-    }
-    cp_async_commit();
-  };
-
-  // rows of the stages issued ahead that those loads did not cover: the cache
-  // rows in [spec_end, r1) (at most two, the new row among them) and zeros
-  // past r1, written with plain loads and stores
-  for (int st = 0; st < n_spec; ++st) {
-    const int base = r0 + st * kStageRows;
-    const int lo = max(base, spec_end);
-    const int cnt = base + kStageRows - lo;
-    const uint32_t kdst = sbase + st * 2 * STAGE_BYTES;
-    const uint32_t vdst = kdst + STAGE_BYTES;
-    for (int i = tid; i < cnt * CH; i += kThreads) {
-      const int row = lo + i / CH, c = i % CH, rr = row - base;
-      uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = kv;
-      if (row < r1) {
-        const __nv_bfloat16* ks = (row == len) ? kn : Kb + (size_t)row * row_stride;
-        const __nv_bfloat16* vs = (row == len) ? vn : Vb + (size_t)row * row_stride;
-        kv = __ldcg(reinterpret_cast<const uint4*>(ks + c * 8));
-        vv = __ldcg(reinterpret_cast<const uint4*>(vs + c * 8));
-      }
-      asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(kdst + tile_off<D>(rr, c)),
-                   "r"(kv.x), "r"(kv.y), "r"(kv.z), "r"(kv.w));
-      asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(vdst + tile_off<D>(rr, c)),
-                   "r"(vv.x), "r"(vv.y), "r"(vv.z), "r"(vv.w));
-    }
-  }
-  // ring of nst stages, all issued up front as far as the ring allows
   const int n_stages = (r1 - r0 + kStageRows - 1) / kStageRows;
-  int issued = n_spec;
-  for (; issued < n_stages && issued < nst; ++issued) issue(issued, issued);
+  int issued = max(n_pre, min(n_stages, nst));   // stages issued so far (cp.async groups)
+  if constexpr (kTma) {
+    if (tid == 0)
+      for (int st = n_pre; st < n_stages && st < nst; ++st)
+        ring_issue<D>(rg, tmK, tmV, g0 + st, x0, y0 + r0 + st * kStageRows, err);
+  } else {
+    for (int st = n_pre; st < n_stages && st < nst; ++st)
+      ring_issue_lsu<D>(rg, Kb, Vb, row_stride, g0 + st, r0 + st * kStageRows, hi);
+  }
   for (int st = 0; st < n_stages; ++st) {
-    cp_async_wait_dyn(issued - (st + 1));   // groups younger than stage st may stay pending
-    __syncthreads();
-    const uint32_t kt = sbase + (st % nst) * 2 * STAGE_BYTES;
-    const uint32_t vt = kt + STAGE_BYTES;
+    const int gi = g0 + st, b = gi % nst;
+    if constexpr (kTma) {
+      if (!tc::mbar_wait(rg.bar0 + 8u * b, (uint32_t)(gi / nst) & 1u) && lane == 0)
+        record_error(err, DEV_TIMEOUT);
+    } else {
+      cp_async_wait_dyn(issued - (st + 1));   // groups younger than stage st may stay pending
+      __syncthreads();
+    }
+    const uint32_t kt = rg.buf0 + (uint32_t)b * 2u * kTileBytes<D>;
+    const uint32_t vt = kt + kTileBytes<D>;
     const int kb = r0 + st * kStageRows + warp * 16;   // this warp's 16 rows
     if (kb < r1) {
+      // this warp's rows past r1 (V zeroed: 0 * garbage must not reach O) and
+      // the new row, which CTA 0 is writing to the cache meanwhile
+      if (kb + 16 > r1 || (len >= kb && len < kb + 16)) {
+        for (int i = lane; i < 16 * CH; i += 32) {
+          const int rr = warp * 16 + i / CH, c = i % CH, row = kb + i / CH;
+          if (row >= r1) {
+            asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};\n" ::"r"(vt + tile_off<D>(rr, c)),
+                         "r"(0u));
+          } else if (row == len) {
+            const uint4 kv = __ldcg(reinterpret_cast<const uint4*>(kn) + c);
+            const uint4 vv = __ldcg(reinterpret_cast<const uint4*>(vn) + c);
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(kt + tile_off<D>(rr, c)),
+                         "r"(kv.x), "r"(kv.y), "r"(kv.z), "r"(kv.w));
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(vt + tile_off<D>(rr, c)),
+                         "r"(vv.x), "r"(vv.y), "r"(vv.z), "r"(vv.w));
+          }
+        }
+        if constexpr (kTma) tc::fence_proxy_async();   // generic writes before the next TMA load
+        __syncwarp();
+      }
       // scores S^T[head][row] for rows kb..kb+15 as two 8-row n-tiles
       float sc[2][4];
 #pragma unroll
@@ -272,12 +312,25 @@ __device__ void attend_bf16(const __nv_bfloat16* __restrict__ Kb, const __nv_bfl
         mma_bf16(o[2 * q2 + 1], pa0, pa2, b2, b3);
       }
     }
-    __syncthreads();
-    if (issued < n_stages) {   // refill the buffer just consumed
-      issue(issued, issued % nst);
-      ++issued;
+    __syncthreads();   // buffer b consumed by every warp
+    if (st + nst < n_stages) {
+      if constexpr (kTma) {
+        if (tid == 0)
+          ring_issue<D>(rg, tmK, tmV, g0 + st + nst, x0, y0 + r0 + (st + nst) * kStageRows, err);
+      } else {
+        ring_issue_lsu<D>(rg, Kb, Vb, row_stride, g0 + st + nst, r0 + (st + nst) * kStageRows, hi);
+        ++issued;
+      }
     }
   }
+  // loads issued ahead that this block did not use must land before the
+  // buffers are reused (s_part aliases them) or the CTA exits
+  if constexpr (kTma) {
+    if (tid == 0) ring_drain<D>(rg, err);
+  } else {
+    cp_async_wait<0>();
+  }
+  __syncthreads();
   // per-lane partial sums of the head's normaliser -> full sum over the quad
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
@@ -445,7 +498,9 @@ __device__ __forceinline__ int atomic_add_acq_rel(int* p, int v) {
 // attention states in [slot_off, slot_off + S * G * sizeof(Partial<D>)).
 template <int D, int G>
 struct DecSmem {
-  static size_t att(bool bf16, int nst) { return bf16 ? (size_t)nst * 2 * kStageRows * D * 2 : 0; }
+  static size_t att(bool bf16, int nst) {   // stage ring + slack for its 1024-byte alignment
+    return bf16 ? (size_t)nst * 2 * kStageRows * D * 2 + 1024 : 0;
+  }
   static constexpr size_t warps() { return (size_t)4 * G * sizeof(Partial<D>); }
   static size_t readout(int r) {
     return ((size_t)r * D + r + (size_t)G * r + 2 * G + (size_t)4 * kThreads * G + (size_t)G * D) *
@@ -460,14 +515,15 @@ struct DecSmem {
   }
 };
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, bool kTma>
 __global__ void __launch_bounds__(kThreads)
 decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __restrict__ v_new,
               T* __restrict__ K_ret, T* __restrict__ V_ret, int32_t* __restrict__ cache_len,
               int cap, int Hkv, const float* __restrict__ M, const float* __restrict__ bstab,
               const float* __restrict__ W_phi, const float* __restrict__ w_gate, int r, float eps,
               float gate_override, int use_override, T* __restrict__ out,
-              int* __restrict__ seq_counters, int* __restrict__ err, uint32_t slot_off, int nst) {
+              int* __restrict__ seq_counters, int* __restrict__ err, uint32_t slot_off, int nst,
+              const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
   namespace cg = cooperative_groups;
   extern __shared__ __align__(128) unsigned char dyn_smem[];
   cg::cluster_group cluster = cg::this_cluster();
@@ -482,6 +538,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   __shared__ float s_w[kDecodeMaxSplits][G];
   __shared__ float s_l[G];
   __shared__ int s_len_hint;
+  __shared__ __align__(8) uint64_t s_bar[kDecodeMaxStages];
   Partial<D>* slots = reinterpret_cast<Partial<D>*>(dyn_smem + slot_off);   // readout CTA only
 
   // phase 0 of the cluster barrier: "this CTA is running" (remote shared
@@ -502,30 +559,48 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   const size_t row_stride = (size_t)Hkv * D;
   const T* Kb = K_ret + (size_t)bi * cap * row_stride + (size_t)kh * D;
   const T* Vb = V_ret + (size_t)bi * cap * row_stride + (size_t)kh * D;
+  Ring ring;
+  ring.buf0 = (smem_u32(dyn_smem) + 1023u) & ~1023u;
+  ring.bar0 = smem_u32(s_bar);
+  ring.nst = nst;
+#pragma unroll
+  for (int b = 0; b < kDecodeMaxStages; ++b) ring.last[b] = -1;
   // A hint of cache_len, read before the wait (relaxed: the previous kernel
   // may be advancing it). It only picks the rows whose loads are issued
   // straight after the wait; the true length read after the wait decides.
   if (kBf16 && rank < S) {
-    if (tid == 0) s_len_hint = max(0, min(ld_relaxed(cache_len + bi), cap - 1));
+    if (tid == 0) {
+      if (kTma) {
+        for (int b = 0; b < nst; ++b) tc::mbar_init(ring.bar0 + 8u * b, 1);
+        tc::fence_mbar_init();
+        tc::prefetch_tmap(&tmK);
+        tc::prefetch_tmap(&tmV);
+      }
+      s_len_hint = max(0, min(ld_relaxed(cache_len + bi), cap - 1));
+    }
     __syncthreads();
   }
   // With programmatic dependent launch this kernel may start while the
   // previous kernel of the stream is still running: wait for it before
   // reading anything another kernel may write (q, the cache, cache_len, M, b).
   griddep_wait();
-  int len_h = 0, per_h = 0, spec_end = 0, n_spec = 0;
+  int len_h = 0, per_h = 0, n_spec = 0;
   if constexpr (kBf16) {
     if (rank < S) {
-      // rows [r0, spec_end) lie below the hinted length: if the true length is
-      // at least the hint and gives the same split, they are cache rows of
-      // this CTA's block that nothing in this step writes
+      // the first stages of this CTA's block under the split of the hinted
+      // length (n = hint + 1 or + 2), issued before the true length is known
       len_h = s_len_hint;
       per_h = split_rows(len_h + 1, S);
       const int r0h = rank * per_h;
-      spec_end = min(min(r0h + per_h, r0h + nst * kStageRows), len_h);
-      if (spec_end > r0h) {
-        n_spec = (spec_end - r0h + kStageRows - 1) / kStageRows;
-        issue_rows<D>(dyn_smem, Kb, Vb, row_stride, r0h, spec_end, n_spec);
+      const int hi_h = min(min(r0h + per_h, len_h + 2), cap);
+      n_spec = hi_h > r0h ? min(nst, (hi_h - r0h + kStageRows - 1) / kStageRows) : 0;
+      for (int st = 0; st < n_spec; ++st) {
+        if constexpr (kTma) {
+          if (tid == 0)
+            ring_issue<D>(ring, &tmK, &tmV, st, kh * D, bi * cap + r0h + st * kStageRows, err);
+        } else {
+          ring_issue_lsu<D>(ring, Kb, Vb, row_stride, st, r0h + st * kStageRows, hi_h);
+        }
       }
     }
   }
@@ -539,13 +614,17 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   const int len = cache_len[bi];
   if (len >= cap) {   // full cache: the whole cluster (same sequence) skips it
     if (rank == 0 && kh == 0 && tid == 0) record_error(err, DEV_CACHE_FULL);
-    cp_async_wait<0>();
+    if (kTma && tid == 0) ring_drain<D>(ring, err);
+    if (!kTma) cp_async_wait<0>();
     return;
   }
   griddep_launch();
   const int n = len + 1;
-  if (n_spec > 0 && !(len >= len_h && split_rows(n, S) == per_h)) {
-    cp_async_wait<0>();   // wrong guess: drop the early loads (barrier below)
+  // the early stages are this CTA's first stages if the true length gives
+  // the same split (and, for cp.async, needs no row past the ones loaded)
+  const bool hit = split_rows(n, S) == per_h && (kTma || len <= len_h + 1);
+  if (!kTma && !hit && n_spec > 0) {
+    cp_async_wait<0>();   // drop them; the barrier below frees the buffers
     n_spec = 0;
   }
   __syncthreads();
@@ -561,9 +640,11 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     const int per = split_rows(n, S);
     const int r0 = min(n, rank * per), r1 = min(n, r0 + per);
     auto* w_part = reinterpret_cast<Partial<D>(*)[G]>(dyn_smem);   // aliases the stages
-    if constexpr (kBf16)
-      attend_bf16<D, G>(Kb, Vb, row_stride, kn, vn, len, r0, r1, s_q, w_part, dyn_smem, nst,
-                        spec_end, n_spec);
+    if constexpr (kBf16) {
+      // a miss leaves TMA stages 0..n_spec-1 spent: the block starts after them
+      attend_bf16<D, G, kTma>(ring, &tmK, &tmV, kh * D, bi * cap, Kb, Vb, row_stride, r1, kn, vn,
+                              len, r0, r1, hit ? 0 : n_spec, hit ? n_spec : 0, s_q, w_part, err);
+    }
     else
       attend_f32<D, G>(Kb, Vb, row_stride, kn, vn, len, r0, r1, s_q, w_part);
     cluster_wait();   // phase 0 complete: every CTA of the cluster is running
@@ -731,8 +812,8 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   }
 }
 
-template <typename T, int D, int G>
-cudaError_t launch_tg(const Ctx& c, int S, int nst, int batch, const void* q, const void* kn,
+template <typename T, int D, int G, bool kTma>
+cudaError_t launch_tgs(const Ctx& c, int S, int nst, int batch, const void* q, const void* kn,
                       const void* vn, void* K_ret, void* V_ret, int32_t* cache_len, int cap,
                       const float* M, const float* bstab, void* out, int* counters,
                       cudaStream_t st) {
@@ -740,7 +821,7 @@ cudaError_t launch_tg(const Ctx& c, int S, int nst, int batch, const void* q, co
   const int r = c.cfg.mem_r;
   const size_t smem = DecSmem<D, G>::total(kBf16, nst, r, S);
   const uint32_t slot_off = (uint32_t)DecSmem<D, G>::slot_off(r);
-  auto k = decode_kernel<T, D, G>;
+  auto k = decode_kernel<T, D, G, kTma>;
   static size_t attr_smem[64] = {};   // per instantiation and device: largest size set so far
   const int dv = c.device & 63;
   if (attr_smem[dv] < smem) {
@@ -764,10 +845,37 @@ cudaError_t launch_tg(const Ctx& c, int S, int nst, int batch, const void* q, co
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   const int use_ov = !isnan(c.cfg.gate_override);
+  // bf16: the retained cache as a [batch * cap, Hkv * D] matrix, 64-row boxes
+  CUtensorMap mk, mv;
+  memset(&mk, 0, sizeof(mk));
+  memset(&mv, 0, sizeof(mv));
+  if (kTma) {
+    const uint64_t width = (uint64_t)c.cfg.n_kv_heads * D, rows = (uint64_t)batch * cap;
+    if (!make_tmap_bf16(c, &mk, K_ret, width, rows, kStageRows) ||
+        !make_tmap_bf16(c, &mv, V_ret, width, rows, kStageRows))
+      return cudaErrorInvalidValue;
+  }
   return cudaLaunchKernelEx(&cfg, k, (const T*)q, (const T*)kn, (const T*)vn, (T*)K_ret,
                             (T*)V_ret, cache_len, cap, c.cfg.n_kv_heads, M, bstab,
                             (const float*)c.W_phi, (const float*)c.w_gate, r, c.cfg.eps,
-                            c.cfg.gate_override, use_ov, (T*)out, counters, c.err, slot_off, nst);
+                            c.cfg.gate_override, use_ov, (T*)out, counters, c.err, slot_off, nst,
+                            mk, mv);
+}
+
+// TMA staging when the attention CTAs stream in more than one wave (two
+// CTAs per SM), cp.async staging otherwise; fp32 has no staging.
+template <typename T, int D, int G>
+cudaError_t launch_tg(const Ctx& c, int S, int nst, int batch, const void* q, const void* kn,
+                      const void* vn, void* K_ret, void* V_ret, int32_t* cache_len, int cap,
+                      const float* M, const float* bstab, void* out, int* counters,
+                      cudaStream_t st) {
+  const bool tma = std::is_same<T, __nv_bfloat16>::value &&
+                   batch * c.cfg.n_kv_heads * (S + 1) > 2 * c.num_sms;
+  if (tma && std::is_same<T, __nv_bfloat16>::value)
+    return launch_tgs<T, D, G, std::is_same<T, __nv_bfloat16>::value>(
+        c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
+  return launch_tgs<T, D, G, false>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M,
+                                    bstab, out, counters, st);
 }
 
 template <typename T, int D>
@@ -810,7 +918,7 @@ int decode_stages(int batch, int n_kv_heads, int cap, int S) {
   if (ctas > 2 * 148) return 2;
   const int per = (cap + S - 1) / S;
   int nst = (per + kStageRows - 1) / kStageRows;
-  if (nst > 3) nst = 3;   // 3 x 32 KB keeps two CTAs per SM
+  if (nst > kDecodeMaxStages) nst = kDecodeMaxStages;   // 3 x 32 KB keeps two CTAs per SM
   if (nst < 2) nst = 2;
   return nst;
 }

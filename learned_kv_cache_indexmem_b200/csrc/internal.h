@@ -37,6 +37,12 @@ constexpr int kIdxPad = 64;
 bool make_tmap_rows64(const Ctx& c, CUtensorMap* map, const void* base, uint64_t rows,
                       uint32_t box_rows);
 
+// 2-D TMA map over a row-major bf16 matrix [rows, width] (width * 2 bytes a
+// multiple of 16), box {64, box_rows}, 128-byte swizzle, zero fill out of
+// bounds. False if encoding fails.
+bool make_tmap_bf16(const Ctx& c, CUtensorMap* map, const void* base, uint64_t width,
+                    uint64_t rows, uint32_t box_rows);
+
 // Layout of the caller's workspace for (batch, L).
 struct Workspace {
   size_t qt_off, kh_off;        // indexer q~ and k^ (bf16 [b, L, kIdxPad])
@@ -48,6 +54,7 @@ struct Workspace {
 };
 
 constexpr int kDecodeMaxSplits = 16;          // CTAs per decode cluster (max)
+constexpr int kDecodeMaxStages = 3;           // 64-row stages in a decode CTA's ring (max)
 constexpr int kDecodeRowsPerSplit = 192;   // cache rows per decode CTA (target)
 constexpr int kMemMaxGroups = 64;
 
