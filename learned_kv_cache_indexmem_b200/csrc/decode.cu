@@ -18,7 +18,7 @@
 // meanwhile. Each attention CTA merges its warps' states straight into a slot
 // of CTA S's shared memory (distributed shared memory), then arrives on the
 // cluster barrier; CTA S merges the S states, adds g*m and writes the output.
-// The last unit of a sequence advances cache_len. CTA 0 appends the new
+// CTA 0 of the last unit of a sequence advances cache_len. CTA 0 appends the new
 // key/value row to the cache; the CTA whose block covers row cache_len reads
 // it from k_new/v_new.
 //
@@ -541,9 +541,6 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   __shared__ __align__(8) uint64_t s_bar[kDecodeMaxStages];
   Partial<D>* slots = reinterpret_cast<Partial<D>*>(dyn_smem + slot_off);   // readout CTA only
 
-  // phase 0 of the cluster barrier: "this CTA is running" (remote shared
-  // memory is written only after every CTA of the cluster has arrived)
-  cluster_arrive_relaxed();
   if (rank == S) {
     // W_phi belongs to the context and is written only at imem_init, so the
     // readout CTA may stage it before waiting for the previous kernel
@@ -584,6 +581,17 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   // previous kernel of the stream is still running: wait for it before
   // reading anything another kernel may write (q, the cache, cache_len, M, b).
   griddep_wait();
+  // this step's own inputs first (q, cache_len), so that their loads do not
+  // queue behind the row loads issued next
+  static_assert(D % 8 == 0 && G * D / 8 <= kThreads, "q is read in groups of 8, one per thread");
+  uint4 qraw[sizeof(T) / 2];   // 8 elements of q
+  const bool qv = tid < G * D / 8;
+  if (qv) {
+    const uint4* qs = reinterpret_cast<const uint4*>(q + ((size_t)bi * Hq + kh * G) * D + 8 * tid);
+#pragma unroll
+    for (int e = 0; e < (int)(sizeof(T) / 2); ++e) qraw[e] = __ldcg(qs + e);
+  }
+  const int len = __ldcg(cache_len + bi);
   int len_h = 0, per_h = 0, n_spec = 0;
   if constexpr (kBf16) {
     if (rank < S) {
@@ -604,20 +612,25 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
       }
     }
   }
-  static_assert(D % 8 == 0, "q is read in groups of 8 elements");
-  for (int i = tid; i < G * D / 8; i += kThreads) {
+  if (qv) {
     float f[8];
-    load8<T>(q + ((size_t)bi * Hq + kh * G) * D + 8 * i, f);
+    load8<T>(reinterpret_cast<const T*>(qraw), f);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) s_q[(8 * i + e) / D][(8 * i + e) % D] = f[e];
+    for (int e = 0; e < 8; ++e) s_q[(8 * tid + e) / D][(8 * tid + e) % D] = f[e];
   }
-  const int len = cache_len[bi];
   if (len >= cap) {   // full cache: the whole cluster (same sequence) skips it
     if (rank == 0 && kh == 0 && tid == 0) record_error(err, DEV_CACHE_FULL);
     if (kTma && tid == 0) ring_drain<D>(ring, err);
     if (!kTma) cp_async_wait<0>();
     return;
   }
+  // phase 0 of the cluster barrier: "this CTA is running and has read
+  // cache_len" (remote shared memory is written only after every CTA of the
+  // cluster has arrived; cache_len is advanced only after every unit's CTAs
+  // have arrived). Relaxed: a release arrive would also wait for this CTA's
+  // loads in flight; every thread has branched on the length it loaded, so
+  // that read has returned its value before the arrive.
+  cluster_arrive_relaxed();
   griddep_launch();
   const int n = len + 1;
   // the early stages are this CTA's first stages if the true length gives
@@ -648,10 +661,20 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     else
       attend_f32<D, G>(Kb, Vb, row_stride, kn, vn, len, r0, r1, s_q, w_part);
     cluster_wait();   // phase 0 complete: every CTA of the cluster is running
+    // CTA 0 counts the unit on its sequence's counter (every CTA of the unit
+    // has read cache_len); the last unit of the sequence advances cache_len.
+    // acq_rel: that update is ordered after every other unit's reads. The
+    // result is used last, so the atomic's round trip overlaps the push.
+    int arrived = 0;
+    if (rank == 0 && tid == 0) arrived = atomic_add_acq_rel(&seq_counters[bi], 1);
     // push this CTA's merged state into the readout CTA's slot, then arrive
     Partial<D>* slot = cluster.map_shared_rank(slots, S) + (size_t)rank * G;
     merge_warps<D, G>(w_part, slot);
     cluster_arrive_release();
+    if (rank == 0 && tid == 0 && arrived == Hkv - 1) {
+      seq_counters[bi] = 0;
+      cache_len[bi] = len + 1;
+    }
     return;
   }
 
@@ -768,12 +791,6 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   cluster_wait();             // phase 0
   cluster_arrive_release();   // phase 1: own arrival
   cluster_wait();             // phase 1: every attention CTA has written its slot
-  // Every CTA of this unit has read cache_len by now; count the unit on its
-  // sequence's counter (the result is used at the end, so the atomic's round
-  // trip overlaps the merge). acq_rel: the last unit's update of cache_len is
-  // ordered after every other unit's reads.
-  int arrived = 0;
-  if (tid == 0) arrived = atomic_add_acq_rel(&seq_counters[bi], 1);
   // merge weights: a warp per head, a lane per slot (S <= 15 < 32)
   for (int g = warp; g < G; g += kThreads / 32) {
     const float mt = lane < S ? slots[lane * G + g].m : -INFINITY;
@@ -802,13 +819,12 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     float res[4] = {o.x * inv_l + ro[g * D + c], o.y * inv_l + ro[g * D + c + 1],
                     o.z * inv_l + ro[g * D + c + 2], o.w * inv_l + ro[g * D + c + 3]};
     T* op = out + ((size_t)bi * Hq + kh * G + g) * D + c;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) op[e] = Elem<T>::from_f(res[e]);
-  }
-  // the last unit of the sequence advances cache_len (all its CTAs have read it)
-  if (tid == 0 && arrived == Hkv - 1) {
-    seq_counters[bi] = 0;
-    cache_len[bi] = len + 1;
+    if constexpr (kBf16) {
+      const uint32_t lo = pack_bf16(res[0], res[1]), hi = pack_bf16(res[2], res[3]);
+      *reinterpret_cast<uint2*>(op) = make_uint2(lo, hi);
+    } else {
+      *reinterpret_cast<float4*>(op) = make_float4(res[0], res[1], res[2], res[3]);
+    }
   }
 }
 
