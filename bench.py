@@ -317,6 +317,89 @@ def full_cache_decode(job, steps=64, reps=3):
             "full_cache_GBps": b * (L + steps / 2) * row / (res["full"] * 1e-6) / 1e9}
 
 
+# ------------------------------------------------------------------ whole-model decode
+
+def model_decode(dev, peak_gbs, steps=8, reps=3):
+    """Decode through the retained caches of a whole model: the 36-layer
+    workload (batch 64, 2048 retained rows per sequence and layer, memory state
+    resident), independent random-init layers, caches filled with N(0,1)
+    values (values do not change the work; parity at this shape is a test).
+    The caches (about 20 GB) are far beyond L2, so every step streams them
+    from HBM. One CUDA graph holds `steps` decode steps through all layers."""
+    wl = synth.WORKLOADS["c4"]
+    s = wl.shape
+    b, B = wl.batch, wl.budget
+    cap = B + steps
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(wl.seed)
+    dec = synth.make_decode_inputs(wl, synth.make_weights(s, wl.seed, dev), steps, wl.seed, dev)
+    layers = []
+    for li in range(wl.n_layers):
+        w = synth.make_weights(s, wl.seed + li, dev)
+        lay = IndexMemLayer.from_shape(s, w)
+        st = lay.new_state(b, B + 1, B, cap, dev)
+        st.K_ret.normal_(generator=gen)
+        st.V_ret.normal_(generator=gen)
+        M0, b0 = synth.make_memory_state(s, b, wl.seed + li, dev)
+        st.M.copy_(M0)
+        st.bstab.copy_(b0)
+        lay.workspace(b, B + 1, B, dev)
+        layers.append((lay, st))
+        del w
+    out = torch.empty_like(dec["q"][0])
+    stream = torch.cuda.Stream(dev)
+
+    def run():
+        for i in range(steps):
+            for lay, st in layers:
+                lay.decode(dec["q"][i], dec["k_new"][i], dec["v_new"][i], st, out=out,
+                           stream=stream)
+
+    def reset():
+        for _, st in layers:
+            st.cache_len.fill_(B)
+
+    with torch.cuda.stream(stream):
+        reset()
+        run()
+        torch.cuda.synchronize()
+        reset()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            run()
+        best = None
+        for _ in range(reps):
+            reset()
+            torch.cuda.synchronize()
+            a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            e.record(stream)
+            torch.cuda.synchronize()
+            t = a.elapsed_time(e) * 1e-3
+            best = t if best is None else min(best, t)
+        del g
+    for lay, _ in layers:
+        lay.sync(stream)
+    es = 2 if s.dtype == "bf16" else 4
+    row = s.n_kv_heads * s.head_dim * es * 2
+    per_launch = b * ((B + (steps + 1) / 2.0) * row +
+                      s.n_kv_heads * (s.mem_r * s.head_dim + s.mem_r) * 4 +
+                      2 * s.n_q_heads * s.head_dim * es + row / 2)
+    launches = steps * wl.n_layers
+    gbs = per_launch * launches / best / 1e9
+    del layers
+    torch.cuda.empty_cache()
+    return {"workload": "c4: %d independent layers, batch %d, %d retained rows per sequence and "
+                        "layer, memory r=%d, %d decode steps" % (wl.n_layers, b, B, s.mem_r, steps),
+            "us_per_layer_step": best / launches * 1e6,
+            "tokens_per_s": b * steps / best,
+            "bytes_per_launch": per_launch, "GBps": gbs, "hbm_frac": gbs / peak_gbs,
+            "note": "caches ~%.1f GB, beyond L2: HBM-bound" % (
+                wl.n_layers * 2 * b * cap * s.n_kv_heads * s.head_dim * es / 1e9)}
+
+
 # ------------------------------------------------------------------ e2e
 
 def run_e2e(job, steps, warmup):
@@ -426,6 +509,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-full-cache", action="store_true",
                     help="skip the full-cache decode comparison")
+    ap.add_argument("--no-model-decode", action="store_true",
+                    help="skip the 36-layer decode measurement")
     a = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -540,6 +625,9 @@ def main():
     full_cmp = None
     if not a.no_full_cache:
         full_cmp = full_cache_decode(job)
+    model_dec = None
+    if not a.no_model_decode:
+        model_dec = model_decode(dev, peak)
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         t_full, desc = cpu_oracle_sample(wl, B)
@@ -564,6 +652,7 @@ def main():
             "e2e": e2e,
             "cpu_baseline": cpu,
             "full_cache_decode": full_cmp,
+            "model_decode": model_dec,
             "gpu_launches": job.launches_per_step() * a.steps,
             "device_errors": not layer_sync_ok,
         }))
