@@ -317,6 +317,77 @@ def full_cache_decode(job, steps=64, reps=3):
             "full_cache_GBps": b * (L + steps / 2) * row / (res["full"] * 1e-6) / 1e9}
 
 
+# ------------------------------------------------------------------ moment readout
+
+def moment_readout(job, steps=64, reps=3):
+    """The MomentKV readout ("MomentKV" technical summary, Method §1, §2, §4) on
+    the same workload, next to IndexMem's gated memory readout: the statistics
+    update from the evicted tokens and the decode step, each timed with CUDA
+    events (the decode steps as one CUDA graph)."""
+    s = job.wl.shape
+    b, L, Bud = job.batch, job.L, job.B
+    lay = IndexMemLayer.from_shape(s, job.w, readout="moment")
+    st = lay.new_state(b, L, Bud, Bud + steps, job.dev)
+    lay.workspace(b, L, Bud, job.dev)
+    res = {}
+
+    def timed(fn, n=reps):
+        best = None
+        for _ in range(n):
+            a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            a.record(job.stream)
+            fn()
+            e.record(job.stream)
+            torch.cuda.synchronize()
+            t = a.elapsed_time(e)
+            best = t if best is None else min(best, t)
+        return best
+
+    with torch.cuda.stream(job.stream):
+        d = job.inp
+        lay.score_and_evict(d["X"], d["Q"], d["K"], d["V"], st, Bud, q_ranges=job.ranges,
+                            stream=job.stream)
+
+        def upd_m():
+            st.M.zero_(); st.bstab.zero_(); st.s_v.zero_(); st.n_e.zero_()
+            lay.update_memory(d["K"], d["V"], st, Bud, chunk=job.wl.mem_chunk, stream=job.stream)
+
+        def upd_g():
+            job.st.M.zero_(); job.st.bstab.zero_()
+            job.memory()
+
+        res["update_ms_moment"] = timed(upd_m)
+        res["update_ms_gated"] = timed(upd_g)
+        len0 = torch.full_like(st.cache_len, Bud)
+        out = torch.empty_like(job.decin["q"][0])
+        graphs = {}
+        for name, layer, state in (("moment", lay, st), ("gated", job.layer, job.st)):
+            state.cache_len.copy_(len0)
+            layer.decode(job.decin["q"][0], job.decin["k_new"][0], job.decin["v_new"][0], state,
+                         out=out, stream=job.stream)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            state.cache_len.copy_(len0)
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=job.stream):
+                for i in range(steps):
+                    layer.decode(job.decin["q"][i], job.decin["k_new"][i], job.decin["v_new"][i],
+                                 state, out=out, stream=job.stream)
+
+            def rep(g=g, state=state):
+                state.cache_len.copy_(len0)
+                g.replay()
+            res["decode_us_per_step_" + name] = timed(rep) / steps * 1e3
+            graphs[name] = g
+        del graphs
+    lay.sync(job.stream)
+    job.layer.sync(job.stream)
+    lay.close()
+    res["steps"] = steps
+    return res
+
+
 # ------------------------------------------------------------------ whole-model decode
 
 def model_decode(dev, peak_gbs, steps=8, reps=3):
@@ -511,6 +582,8 @@ def main():
                     help="skip the full-cache decode comparison")
     ap.add_argument("--no-model-decode", action="store_true",
                     help="skip the 36-layer decode measurement")
+    ap.add_argument("--no-moment", action="store_true",
+                    help="skip the MomentKV readout measurement")
     a = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -625,6 +698,9 @@ def main():
     full_cmp = None
     if not a.no_full_cache:
         full_cmp = full_cache_decode(job)
+    moment = None
+    if not a.no_moment:
+        moment = moment_readout(job)
     model_dec = None
     if not a.no_model_decode:
         model_dec = model_decode(dev, peak)
@@ -652,6 +728,7 @@ def main():
             "e2e": e2e,
             "cpu_baseline": cpu,
             "full_cache_decode": full_cmp,
+            "moment_readout": moment,
             "model_decode": model_dec,
             "gpu_launches": job.launches_per_step() * a.steps,
             "device_errors": not layer_sync_ok,

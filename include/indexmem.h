@@ -9,6 +9,10 @@
  *             indexer, §2.B Latent memory, §4 Experimental results.
  *   [IM-abs]  "IndexMem: Learned KV-Cache Eviction with Latent Memory for
  *             Long-Context LLM Inference", arXiv abstract.
+ *   [MK-sum]  "MomentKV" technical summary (gist.science), Method §1 moment
+ *             statistics, §2 first-order evicted output, §4 normalisation-
+ *             corrected inference (the second compensation of the evicted
+ *             tokens that this library computes: IMEM_READOUT_MOMENT).
  *
  * Conventions for every entry point
  *   - Tensor arguments are DEVICE pointers owned by the caller, row-major and
@@ -50,12 +54,25 @@ typedef enum {
 
 typedef enum { IMEM_FP32 = 0, IMEM_BF16 = 1 } imem_dtype;
 
+/* How the evicted tokens compensate the retained attention.
+ *   IMEM_READOUT_GATED:  IndexMem's latent memory, o = o_attn + g(q) m(q)
+ *                        ([IM-sum] §2.B).
+ *   IMEM_READOUT_MOMENT: MomentKV's moment statistics ([MK-sum]): per KV head
+ *                        the count n_e, the key and value sums s_k, s_v and
+ *                        S^T = sum k v^T; the output mixes the retained
+ *                        attention with a first-order estimate of the
+ *                        evicted one (imem_decode_moment). */
+typedef enum { IMEM_READOUT_GATED = 0, IMEM_READOUT_MOMENT = 1 } imem_readout;
+
 /* Layer configuration.
  * Supported by this build: head_dim in {64,128}; idx_dim in {32,64};
  * idx_heads == n_q_heads (one indexer head per attention query head,
  * [IM-sum] §2.A: the multi-head queries are down-projected);
  * n_q_heads % n_kv_heads == 0 with a group of at most 8; hidden % 64 == 0;
- * mem_r in {16,32,...,128}; 0 < lambda <= 1. */
+ * mem_r in {16,32,...,128}; 0 < lambda <= 1.
+ * readout = IMEM_READOUT_MOMENT requires mem_r == head_dim and lambda == 1 (the
+ * statistics are plain sums); W_phi is then the identity and w_gate, eps and
+ * gate_override are not used (imem_weights.W_phi and .w_gate may be NULL). */
 typedef struct {
   int hidden;        /* H: hidden size of the model                        */
   int n_q_heads;     /* Hq                                                  */
@@ -68,6 +85,7 @@ typedef struct {
   float eps;         /* readout denominator epsilon (1e-6 by default)       */
   int dtype;         /* imem_dtype                                          */
   float gate_override; /* NaN: learned gate g(q); otherwise g forced to it  */
+  int readout;       /* imem_readout                                        */
 } imem_config;
 
 /* Layer weights, device pointers, read once by imem_init (repacked into the
@@ -145,7 +163,8 @@ imem_status imem_score_and_evict(imem_ctx* ctx, int batch, int L, int B,
  * K, V [batch, L, Hkv, d] model dtype; M [batch, Hkv, r, d] fp32 in/out;
  * bstab [batch, Hkv, r] fp32 in/out. `chunk` = evicted tokens per work unit
  * (a multiple of 64, e.g. 512). n_evicted = 0 leaves M and b unchanged.
- * Errors: INVALID_ARG, SHAPE, ALIGN, CUDA. */
+ * Errors: INVALID_ARG, SHAPE, ALIGN, CUDA; UNSUPPORTED for a context in
+ * IMEM_READOUT_MOMENT mode (use imem_update_moments). */
 imem_status imem_update_memory(imem_ctx* ctx, int batch, int L, const void* K, const void* V,
                                const int32_t* idx_evicted, int n_evicted, int chunk,
                                float* M, float* bstab, void* workspace, void* stream);
@@ -160,7 +179,8 @@ imem_status imem_update_memory(imem_ctx* ctx, int batch, int L, const void* K, c
  *   out = o_attn + g m            (out [batch, Hq, d], model dtype)
  * M, bstab are read only. A sequence whose cache is full (cache_len >= cap)
  * is left unchanged and its output row is not written; imem_sync reports it.
- * Errors: INVALID_ARG, SHAPE, ALIGN, CUDA. */
+ * Errors: INVALID_ARG, SHAPE, ALIGN, CUDA; UNSUPPORTED for a context in
+ * IMEM_READOUT_MOMENT mode (use imem_decode_moment). */
 imem_status imem_decode(imem_ctx* ctx, int batch, const void* q, const void* k_new,
                         const void* v_new, void* K_ret, void* V_ret, int32_t* cache_len,
                         int cap, const float* M, const float* bstab, void* out,
@@ -189,6 +209,40 @@ imem_status imem_update_memory_static(int batch, int L, int n_kv_heads, int head
                                       float lambda, int dtype, const void* K, const void* V,
                                       const int32_t* idx_evicted, int n_evicted, int chunk,
                                       const float* W_phi, float* M, float* bstab, void* stream);
+
+/* Moment statistics of the evicted tokens ([MK-sum] Method §1), for a context
+ * created with readout = IMEM_READOUT_MOMENT (else IMEM_ERR_UNSUPPORTED).
+ * For every sequence and KV head h, over the evicted positions E[0..n):
+ *   S_T_h += sum_i k_{E[i],h} v_{E[i],h}^T   (S_T [batch, Hkv, d, d] fp32: row =
+ *                                            key dimension, column = value
+ *                                            dimension, i.e. S^T of [MK-sum])
+ *   s_k_h += sum_i k_{E[i],h},  s_v_h += sum_i v_{E[i],h}   ([batch, Hkv, d] fp32)
+ *   n_e[s] += n_evicted                                     ([batch] fp32)
+ * Other arguments, the workspace and the errors as imem_update_memory. The same
+ * tensor-core kernel as the memory update computes S_T and s_k (identity map,
+ * no decay); its loader warps add the value sums on the way. */
+imem_status imem_update_moments(imem_ctx* ctx, int batch, int L, const void* K, const void* V,
+                                const int32_t* idx_evicted, int n_evicted, int chunk,
+                                float* S_T, float* s_k, float* s_v, float* n_e,
+                                void* workspace, void* stream);
+
+/* One decode step with the MomentKV readout ([MK-sum] Method §2, §4), for a
+ * context created with readout = IMEM_READOUT_MOMENT (else
+ * IMEM_ERR_UNSUPPORTED). q, k_new, v_new, K_ret, V_ret, cache_len, cap, out and
+ * the workspace as imem_decode; S_T, s_k, s_v, n_e as imem_update_moments
+ * (read only). Query head h uses KV head h/(Hq/Hkv):
+ *   o_R = softmax(q K^T / sqrt(d)) V over rows [0, cache_len] (new row incl.),
+ *   Z_R = sum of exp(q k^T / sqrt(d)) over the same rows,
+ *   k_bar = s_k / n_e, v_bar = s_v / n_e, S~ = S - s_v s_k^T / n_e,
+ *   f_E = v_bar + S~ q / (n_e sqrt(d)),
+ *   Z_E = n_e exp(q . k_bar / sqrt(d))   (Jensen lower bound of the evicted
+ *                                         partition function),
+ *   w_R = Z_R / (Z_R + Z_E),  out = w_R o_R + (1 - w_R) f_E
+ * and out = o_R where n_e = 0. Errors as imem_decode. */
+imem_status imem_decode_moment(imem_ctx* ctx, int batch, const void* q, const void* k_new,
+                               const void* v_new, void* K_ret, void* V_ret, int32_t* cache_len,
+                               int cap, const float* S_T, const float* s_k, const float* s_v,
+                               const float* n_e, void* out, void* workspace, void* stream);
 
 /* Waits for the stream, then reports the first error the device recorded for
  * this context since the last imem_sync (TIMEOUT for a bounded wait that ran

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(HERE, "libindexmem.so")
 STATUS = {0: "IMEM_OK", 1: "IMEM_ERR_INVALID_ARG", 2: "IMEM_ERR_SHAPE", 3: "IMEM_ERR_ALIGN",
           4: "IMEM_ERR_UNSUPPORTED", 5: "IMEM_ERR_CUDA", 6: "IMEM_ERR_TIMEOUT"}
 FP32, BF16 = 0, 1
+READOUT_GATED, READOUT_MOMENT = 0, 1
 
 
 class IndexMemError(RuntimeError):
@@ -33,7 +34,7 @@ class Config(ctypes.Structure):
                 ("idx_heads", ctypes.c_int), ("idx_dim", ctypes.c_int),
                 ("mem_r", ctypes.c_int), ("lambda_", ctypes.c_float),
                 ("eps", ctypes.c_float), ("dtype", ctypes.c_int),
-                ("gate_override", ctypes.c_float)]
+                ("gate_override", ctypes.c_float), ("readout", ctypes.c_int)]
 
 
 class Weights(ctypes.Structure):
@@ -72,6 +73,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.imem_decode.argtypes = [vp, i, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp]
     lib.imem_sync.restype = i
     lib.imem_sync.argtypes = [vp, vp]
+    lib.imem_update_moments.restype = i
+    lib.imem_update_moments.argtypes = [vp, i, i, vp, vp, vp, i, i, vp, vp, vp, vp, vp, vp]
+    lib.imem_decode_moment.restype = i
+    lib.imem_decode_moment.argtypes = [vp, i, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp, vp,
+                                       vp]
     lib.imem_update_memory_static.restype = i
     lib.imem_update_memory_static.argtypes = [i, i, i, i, i, f, i, vp, vp, vp, i, i, vp, vp, vp, vp]
     _lib = lib
@@ -105,10 +111,11 @@ def status_string(code: int) -> str:
 
 
 def make_config(hidden, n_q_heads, n_kv_heads, head_dim, idx_dim, mem_r, lam, dtype,
-                eps=1e-6, gate_override=None, idx_heads=None) -> Config:
+                eps=1e-6, gate_override=None, idx_heads=None, readout=None) -> Config:
     return Config(hidden, n_q_heads, n_kv_heads, head_dim,
                   n_q_heads if idx_heads is None else idx_heads, idx_dim, mem_r, lam, eps, dtype,
-                  math.nan if gate_override is None else float(gate_override))
+                  math.nan if gate_override is None else float(gate_override),
+                  READOUT_GATED if readout is None else readout)
 
 
 def init(cfg: Config, W_idx_q, W_idx_k, w_idx_g, W_phi, w_gate) -> int:
@@ -150,6 +157,21 @@ def decode(ctx, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, 
     _check(load().imem_decode(
         ctx, batch, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(K_ret), _ptr(V_ret), _ptr(cache_len),
         cap, _ptr(M), _ptr(bstab), _ptr(out), _ptr(workspace), _stream(stream)), "imem_decode")
+
+
+def update_moments(ctx, batch, L, K, V, idx_evicted, n_evicted, chunk, S_T, s_k, s_v, n_e,
+                   workspace, stream=None):
+    _check(load().imem_update_moments(
+        ctx, batch, L, _ptr(K), _ptr(V), _ptr(idx_evicted), n_evicted, chunk, _ptr(S_T),
+        _ptr(s_k), _ptr(s_v), _ptr(n_e), _ptr(workspace), _stream(stream)), "imem_update_moments")
+
+
+def decode_moment(ctx, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, S_T, s_k, s_v, n_e,
+                  out, workspace, stream=None):
+    _check(load().imem_decode_moment(
+        ctx, batch, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(K_ret), _ptr(V_ret), _ptr(cache_len),
+        cap, _ptr(S_T), _ptr(s_k), _ptr(s_v), _ptr(n_e), _ptr(out), _ptr(workspace),
+        _stream(stream)), "imem_decode_moment")
 
 
 def update_memory_static(batch, L, n_kv_heads, head_dim, mem_r, lam, dtype, K, V, idx_evicted,

@@ -11,6 +11,8 @@
 #include "common.cuh"
 #include "internal.h"
 
+#include <vector>
+
 struct imem_ctx {
   imem::Ctx c;
 };
@@ -35,6 +37,9 @@ Workspace workspace_layout(const Ctx& c, int batch, int L) {
   w.mem_part_off = off;
   off = align_up(off + (2 * 148 + units) * (size_t)c.cfg.head_dim * (c.cfg.head_dim + 1) *
                            sizeof(float), 256);
+  w.sv_part_off = off;                        // moment mode: one d-vector per run
+  if (c.cfg.readout == IMEM_READOUT_MOMENT)
+    off = align_up(off + (2 * 148 + units) * (size_t)c.cfg.head_dim * sizeof(float), 256);
   w.sel_off = off;
   off = align_up(off + 256, 256);
   w.qt_off = off;
@@ -136,11 +141,18 @@ imem_status imem_init(const imem_config* cfg, const imem_weights* w, imem_ctx** 
   if (k.hidden % 64) return IMEM_ERR_UNSUPPORTED;
   if (k.mem_r % 16 || k.mem_r > 128) return IMEM_ERR_UNSUPPORTED;
   if (k.idx_dim + k.n_q_heads > 128) return IMEM_ERR_UNSUPPORTED;
+  if (k.readout != IMEM_READOUT_GATED && k.readout != IMEM_READOUT_MOMENT)
+    return IMEM_ERR_INVALID_ARG;
+  const bool moment = k.readout == IMEM_READOUT_MOMENT;
+  if (moment && k.mem_r != k.head_dim) return IMEM_ERR_UNSUPPORTED;
+  if (moment && k.lambda != 1.f) return IMEM_ERR_UNSUPPORTED;
   IMEM_CHECK(check_ptr(w->W_idx_q));
   IMEM_CHECK(check_ptr(w->W_idx_k));
   IMEM_CHECK(check_ptr(w->w_idx_g));
-  IMEM_CHECK(check_ptr(w->W_phi));
-  IMEM_CHECK(check_ptr(w->w_gate));
+  if (!moment) {
+    IMEM_CHECK(check_ptr(w->W_phi));
+    IMEM_CHECK(check_ptr(w->w_gate));
+  }
 
   imem_ctx* h = (imem_ctx*)calloc(1, sizeof(imem_ctx));
   if (!h) return IMEM_ERR_CUDA;
@@ -167,8 +179,18 @@ imem_status imem_init(const imem_config* cfg, const imem_weights* w, imem_ctx** 
   if (e == cudaSuccess) e = cudaMalloc((void**)&c.W_phi, n_phi * sizeof(float));
   if (e == cudaSuccess) e = cudaMalloc((void**)&c.w_gate, n_g * sizeof(float));
   if (e == cudaSuccess) e = cudaMalloc((void**)&c.err, sizeof(int));
-  if (e == cudaSuccess) e = cudaMemcpy(c.W_phi, w->W_phi, n_phi * sizeof(float), cudaMemcpyDeviceToDevice);
-  if (e == cudaSuccess) e = cudaMemcpy(c.w_gate, w->w_gate, n_g * sizeof(float), cudaMemcpyDeviceToDevice);
+  if (moment) {
+    // moment statistics: the identity map (S^T and s_k come out of the same
+    // kernel as M and b) and no gate
+    std::vector<float> eye(n_phi, 0.f);
+    for (int i = 0; i < k.mem_r; ++i) eye[(size_t)i * k.head_dim + i] = 1.f;
+    if (e == cudaSuccess)
+      e = cudaMemcpy(c.W_phi, eye.data(), n_phi * sizeof(float), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemset(c.w_gate, 0, n_g * sizeof(float));
+  } else {
+    if (e == cudaSuccess) e = cudaMemcpy(c.W_phi, w->W_phi, n_phi * sizeof(float), cudaMemcpyDeviceToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(c.w_gate, w->w_gate, n_g * sizeof(float), cudaMemcpyDeviceToDevice);
+  }
   if (e == cudaSuccess) e = cudaMemset(c.err, 0, sizeof(int));
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
@@ -244,6 +266,7 @@ imem_status imem_update_memory(imem_ctx* h, int batch, int L, const void* K, con
                                float* bstab, void* workspace, void* stream) {
   if (!h) return IMEM_ERR_INVALID_ARG;
   const Ctx& c = h->c;
+  if (c.cfg.readout != IMEM_READOUT_GATED) return IMEM_ERR_UNSUPPORTED;
   if (batch < 1 || L < 1) return IMEM_ERR_SHAPE;
   if (n_evicted < 0 || n_evicted > L) return IMEM_ERR_SHAPE;
   if (chunk < 64 || chunk % 64) return IMEM_ERR_SHAPE;
@@ -257,16 +280,49 @@ imem_status imem_update_memory(imem_ctx* h, int batch, int L, const void* K, con
   const imem::Workspace ws = imem::workspace_layout(c, batch, L);
   float* part = (float*)((char*)workspace + ws.mem_part_off);
   return cuda_status(imem::launch_memory_update(c, batch, L, K, V, idx_evicted, n_evicted, chunk,
-                                                M, bstab, part, (cudaStream_t)stream));
+                                                M, bstab, part, nullptr, nullptr, nullptr,
+                                                (cudaStream_t)stream));
 }
 
-imem_status imem_decode(imem_ctx* h, int batch, const void* q, const void* k_new,
-                        const void* v_new, void* K_ret, void* V_ret, int32_t* cache_len, int cap,
-                        const float* M, const float* bstab, void* out, void* workspace,
-                        void* stream) {
+imem_status imem_update_moments(imem_ctx* h, int batch, int L, const void* K, const void* V,
+                                const int32_t* idx_evicted, int n_evicted, int chunk, float* S_T,
+                                float* s_k, float* s_v, float* n_e, void* workspace,
+                                void* stream) {
   if (!h) return IMEM_ERR_INVALID_ARG;
   const Ctx& c = h->c;
+  if (c.cfg.readout != IMEM_READOUT_MOMENT) return IMEM_ERR_UNSUPPORTED;
+  if (batch < 1 || L < 1) return IMEM_ERR_SHAPE;
+  if (n_evicted < 0 || n_evicted > L) return IMEM_ERR_SHAPE;
+  if (chunk < 64 || chunk % 64) return IMEM_ERR_SHAPE;
+  IMEM_CHECK(check_ptr(K));
+  IMEM_CHECK(check_ptr(V));
+  if (n_evicted > 0) IMEM_CHECK(check_ptr(idx_evicted));
+  IMEM_CHECK(check_ptr(S_T));
+  IMEM_CHECK(check_ptr(s_k));
+  IMEM_CHECK(check_ptr(s_v));
+  IMEM_CHECK(check_ptr(n_e));
+  IMEM_CHECK(check_ptr(workspace));
+  IMEM_CHECK(check_device(c));
+  const imem::Workspace ws = imem::workspace_layout(c, batch, L);
+  float* part = (float*)((char*)workspace + ws.mem_part_off);
+  float* svp = (float*)((char*)workspace + ws.sv_part_off);
+  return cuda_status(imem::launch_memory_update(c, batch, L, K, V, idx_evicted, n_evicted, chunk,
+                                                S_T, s_k, part, svp, s_v, n_e,
+                                                (cudaStream_t)stream));
+}
+
+namespace {
+imem_status decode_common(imem_ctx* h, int batch, const void* q, const void* k_new,
+                          const void* v_new, void* K_ret, void* V_ret, int32_t* cache_len,
+                          int cap, const float* M, const float* bstab, const float* s_v,
+                          const float* n_e, void* out, void* workspace, void* stream) {
+  const Ctx& c = h->c;
+  const bool moment = c.cfg.readout == IMEM_READOUT_MOMENT;
   if (batch < 1 || cap < 1) return IMEM_ERR_SHAPE;
+  if (moment) {
+    IMEM_CHECK(check_ptr(s_v));
+    IMEM_CHECK(check_ptr(n_e));
+  }
   IMEM_CHECK(check_ptr(q));
   IMEM_CHECK(check_ptr(k_new));
   IMEM_CHECK(check_ptr(v_new));
@@ -282,8 +338,29 @@ imem_status imem_decode(imem_ctx* h, int batch, const void* q, const void* k_new
   const imem::Workspace ws = imem::workspace_layout(c, batch, 1);
   char* wsb = (char*)workspace;
   return cuda_status(imem::launch_decode(c, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap,
-                                         M, bstab, out, (float*)(wsb + ws.dec_part_off),
-                                         (int*)(wsb + ws.dec_cnt_off), (cudaStream_t)stream));
+                                         M, bstab, s_v, n_e, out, (int*)(wsb + ws.dec_cnt_off),
+                                         (cudaStream_t)stream));
+}
+}  // namespace
+
+imem_status imem_decode(imem_ctx* h, int batch, const void* q, const void* k_new,
+                        const void* v_new, void* K_ret, void* V_ret, int32_t* cache_len, int cap,
+                        const float* M, const float* bstab, void* out, void* workspace,
+                        void* stream) {
+  if (!h) return IMEM_ERR_INVALID_ARG;
+  if (h->c.cfg.readout != IMEM_READOUT_GATED) return IMEM_ERR_UNSUPPORTED;
+  return decode_common(h, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, nullptr,
+                       nullptr, out, workspace, stream);
+}
+
+imem_status imem_decode_moment(imem_ctx* h, int batch, const void* q, const void* k_new,
+                               const void* v_new, void* K_ret, void* V_ret, int32_t* cache_len,
+                               int cap, const float* S_T, const float* s_k, const float* s_v,
+                               const float* n_e, void* out, void* workspace, void* stream) {
+  if (!h) return IMEM_ERR_INVALID_ARG;
+  if (h->c.cfg.readout != IMEM_READOUT_MOMENT) return IMEM_ERR_UNSUPPORTED;
+  return decode_common(h, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, S_T, s_k, s_v,
+                       n_e, out, workspace, stream);
 }
 
 imem_status imem_sync(imem_ctx* h, void* stream) {

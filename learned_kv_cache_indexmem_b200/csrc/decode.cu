@@ -502,9 +502,10 @@ struct DecSmem {
     return bf16 ? (size_t)nst * 2 * kStageRows * D * 2 + 1024 : 0;
   }
   static constexpr size_t warps() { return (size_t)4 * G * sizeof(Partial<D>); }
+  static_assert((kThreads / (D / 4)) * D == 4 * kThreads, "M^T u partials: RG * D = 4 * kThreads");
   static size_t readout(int r) {
-    return ((size_t)r * D + r + (size_t)G * r + 2 * G + (size_t)4 * kThreads * G + (size_t)G * D) *
-           sizeof(float);
+    return ((size_t)r * D + r + (size_t)G * r + 2 * G + (size_t)4 * kThreads * G + (size_t)G * D +
+            D) * sizeof(float);
   }
   static size_t slot_off(int r) { return (readout(r) + 127) / 128 * 128; }
   static size_t total(bool bf16, int nst, int r, int S) {
@@ -520,6 +521,7 @@ __global__ void __launch_bounds__(kThreads)
 decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __restrict__ v_new,
               T* __restrict__ K_ret, T* __restrict__ V_ret, int32_t* __restrict__ cache_len,
               int cap, int Hkv, const float* __restrict__ M, const float* __restrict__ bstab,
+              const float* __restrict__ s_v, const float* __restrict__ n_e, int moment,
               const float* __restrict__ W_phi, const float* __restrict__ w_gate, int r, float eps,
               float gate_override, int use_override, T* __restrict__ out,
               int* __restrict__ seq_counters, int* __restrict__ err, uint32_t slot_off, int nst,
@@ -538,12 +540,14 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   __shared__ float s_w[kDecodeMaxSplits][G];
   __shared__ float s_l[G];
   __shared__ int s_len_hint;
+  __shared__ float s_wr[G], s_kq[G];   // moment readout: w_R and q.k_bar per head
   __shared__ __align__(8) uint64_t s_bar[kDecodeMaxStages];
   Partial<D>* slots = reinterpret_cast<Partial<D>*>(dyn_smem + slot_off);   // readout CTA only
 
-  if (rank == S) {
+  if (rank == S && !moment) {
     // W_phi belongs to the context and is written only at imem_init, so the
-    // readout CTA may stage it before waiting for the previous kernel
+    // readout CTA may stage it before waiting for the previous kernel (the
+    // moment readout's map is the identity: u = q, nothing to stage)
     float* sW = reinterpret_cast<float*>(dyn_smem);          // [r][D], chunks XOR-swizzled
     const uint32_t wdst = smem_u32(sW);
     for (int i = tid; i < r * D / 4; i += kThreads) {
@@ -684,19 +688,32 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   float* su = sb + r;                                       // [G][r]
   float* sden = su + G * r;                                 // [G]
   float* sgate = sden + G;                                  // [G]
-  float* snum = sgate + G;                                  // [4][G][D] partial M^T u
-  float* ro = snum + 4 * G * D;                             // [G][D] = g * m
+  constexpr int RG = kThreads / (D / 4);                    // row groups of the M^T u partials
+  float* snum = sgate + G;                                  // [RG][G][D] partial M^T u
+  float* ro = snum + RG * G * D;                            // [G][D] = g * m (moment: S q)
+  float* ssv = ro + G * D;                                  // [D] moment: s_v of this unit
   {
     for (int i = tid; i < r / 4; i += kThreads)
       cp_async16(smem_u32(sb) + (uint32_t)i * 16u, bstab + (size_t)unit * r + 4 * i, true);
+    if (moment)
+      for (int i = tid; i < D / 4; i += kThreads)
+        cp_async16(smem_u32(ssv) + (uint32_t)i * 16u, s_v + (size_t)unit * D + 4 * i, true);
+    cp_async_commit();
+  }
+  const float ne = moment ? __ldcg(n_e + bi) : 0.f;
+  constexpr int kREarly = 64;   // rows of M held in registers (below)
+  if (moment && r > kREarly) {
+    // moment readout: the rows of M past the register ones go to the (unused)
+    // W_phi region, so that they are in flight while u is formed
+    for (int i = tid; i < (r - kREarly) * D / 4; i += kThreads)
+      cp_async16(smem_u32(sW) + (uint32_t)i * 16u,
+                 M + ((size_t)unit * r + kREarly) * D + 4 * i, true);
     cp_async_commit();
   }
   // M: thread (row group rg, column quad cq) holds rows rg, rg+4, ... of
   // columns 4cq..4cq+3 (first 64 rows), loaded now so they arrive while u is
   // computed (volatile: the loads are issued here, not at their first use)
-  constexpr int kREarly = 64;
-  const int cq = tid % (D / 4), rg = tid / (D / 4);         // D/4 column quads, kThreads/(D/4) row groups
-  constexpr int RG = kThreads / (D / 4);
+  const int cq = tid % (D / 4), rg = tid / (D / 4);         // D/4 column quads, RG row groups
   float4 mreg[kREarly / RG];
   const float* Mu = M + (size_t)unit * r * D;
 #pragma unroll
@@ -710,8 +727,8 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
       mreg[k] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
-  // gate: z = w_gate[h] . q (independent of the memory)
-  for (int g = warp; g < G; g += kThreads / 32) {
+  // gate: z = w_gate[h] . q (independent of the memory; none in moment mode)
+  for (int g = warp; g < G && !moment; g += kThreads / 32) {
     const float* wg = w_gate + ((size_t)kh * G + g) * D;
     float z = 0.f;
     for (int c = lane; c < D; c += 32) z = fmaf(__ldg(wg + c), s_q[g][c], z);
@@ -720,7 +737,8 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   }
   cp_async_wait<0>();
   __syncthreads();
-  for (int o = tid; o < G * r; o += kThreads) {
+  for (int o = tid; o < G * r && moment; o += kThreads) su[o] = s_q[o / r][o % r];   // u = q
+  for (int o = tid; o < G * r && !moment; o += kThreads) {
     const int g = o / r, j = o % r;
     const float4* wr = reinterpret_cast<const float4*>(sW + (size_t)j * D);
     const float4* q4 = reinterpret_cast<const float4*>(&s_q[g][0]);
@@ -741,7 +759,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     float a = 0.f;
     for (int j = lane; j < r; j += 32) a = fmaf(sb[j], su[g * r + j], a);
     a = warp_sum(a);
-    if (lane == 0) sden[g] = a + eps;
+    if (lane == 0) sden[g] = moment ? a : a + eps;   // moment: s_k . q
   }
   {
     // partial num over this thread's rows, for its 4 columns and every head
@@ -763,7 +781,9 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
       }
     }
     for (int j = kREarly + rg; j < r; j += RG) {   // r > 64: remaining rows
-      const float4 mv = __ldcg(reinterpret_cast<const float4*>(Mu + (size_t)j * D + 4 * cq));
+      const float4 mv =
+          moment ? reinterpret_cast<const float4*>(sW + (size_t)(j - kREarly) * D)[cq]
+                 : __ldcg(reinterpret_cast<const float4*>(Mu + (size_t)j * D + 4 * cq));
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float uu = su[g * r + j];
@@ -783,7 +803,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     float num = 0.f;
 #pragma unroll
     for (int k = 0; k < RG; ++k) num += snum[((size_t)k * G + g) * D + c];
-    ro[i] = sgate[g] * (num / sden[g]);
+    ro[i] = moment ? num : sgate[g] * (num / sden[g]);
   }
   __syncthreads();
 
@@ -798,7 +818,21 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     const float w = (mt == -INFINITY) ? 0.f : exp2f(mt - mx);
     const float l = warp_sum(lane < S ? w * slots[lane * G + g].l : 0.f);
     if (lane < S) s_w[lane][g] = w;
-    if (lane == 0) s_l[g] = l;
+    if (lane == 0) {
+      s_l[g] = l;
+      if (moment) {
+        // Jensen: log2 Z_E = log2 n_e + (q.k_bar) log2(e) / sqrt(d);
+        // log2 Z_R = mx + log2 l (logits are kept in log2 units)
+        float wr = 1.f, kq = 0.f;
+        if (ne > 0.f) {
+          kq = sden[g] / ne;
+          const float lze = log2f(ne) + kq * (kLog2e * rsqrtf((float)D));
+          wr = 1.f / (1.f + exp2f(lze - (mx + log2f(l))));
+        }
+        s_wr[g] = wr;
+        s_kq[g] = kq;
+      }
+    }
   }
   __syncthreads();
   for (int i = tid; i < G * D / 4; i += kThreads) {   // 4 consecutive columns per thread
@@ -816,8 +850,21 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
       o.z = fmaf(w, vals[t2].z, o.z); o.w = fmaf(w, vals[t2].w, o.w);
     }
     const float inv_l = 1.f / s_l[g];
-    float res[4] = {o.x * inv_l + ro[g * D + c], o.y * inv_l + ro[g * D + c + 1],
-                    o.z * inv_l + ro[g * D + c + 2], o.w * inv_l + ro[g * D + c + 3]};
+    float res[4] = {o.x * inv_l, o.y * inv_l, o.z * inv_l, o.w * inv_l};
+    if (!moment) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) res[e] += ro[g * D + c + e];
+    } else if (s_wr[g] < 1.f) {
+      // f_E = v_bar + (S q - s_v (q.k_bar)) / (n_e sqrt(d)); mix with w_R
+      const float wr = s_wr[g], kq = s_kq[g], inv_ne = 1.f / ne;
+      const float scl = inv_ne * rsqrtf((float)D);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float sv = ssv[c + e];
+        const float fe = sv * inv_ne + (ro[g * D + c + e] - sv * kq) * scl;
+        res[e] = wr * res[e] + (1.f - wr) * fe;
+      }
+    }
     T* op = out + ((size_t)bi * Hq + kh * G + g) * D + c;
     if constexpr (kBf16) {
       const uint32_t lo = pack_bf16(res[0], res[1]), hi = pack_bf16(res[2], res[3]);
@@ -831,8 +878,8 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
 template <typename T, int D, int G, bool kTma>
 cudaError_t launch_tgs(const Ctx& c, int S, int nst, int batch, const void* q, const void* kn,
                       const void* vn, void* K_ret, void* V_ret, int32_t* cache_len, int cap,
-                      const float* M, const float* bstab, void* out, int* counters,
-                      cudaStream_t st) {
+                      const float* M, const float* bstab, const float* s_v, const float* n_e,
+                      void* out, int* counters, cudaStream_t st) {
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   const int r = c.cfg.mem_r;
   const size_t smem = DecSmem<D, G>::total(kBf16, nst, r, S);
@@ -872,8 +919,8 @@ cudaError_t launch_tgs(const Ctx& c, int S, int nst, int batch, const void* q, c
       return cudaErrorInvalidValue;
   }
   return cudaLaunchKernelEx(&cfg, k, (const T*)q, (const T*)kn, (const T*)vn, (T*)K_ret,
-                            (T*)V_ret, cache_len, cap, c.cfg.n_kv_heads, M, bstab,
-                            (const float*)c.W_phi, (const float*)c.w_gate, r, c.cfg.eps,
+                            (T*)V_ret, cache_len, cap, c.cfg.n_kv_heads, M, bstab, s_v, n_e,
+                            (int)(c.cfg.readout == IMEM_READOUT_MOMENT), (const float*)c.W_phi, (const float*)c.w_gate, r, c.cfg.eps,
                             c.cfg.gate_override, use_ov, (T*)out, counters, c.err, slot_off, nst,
                             mk, mv);
 }
@@ -883,27 +930,27 @@ cudaError_t launch_tgs(const Ctx& c, int S, int nst, int batch, const void* q, c
 template <typename T, int D, int G>
 cudaError_t launch_tg(const Ctx& c, int S, int nst, int batch, const void* q, const void* kn,
                       const void* vn, void* K_ret, void* V_ret, int32_t* cache_len, int cap,
-                      const float* M, const float* bstab, void* out, int* counters,
-                      cudaStream_t st) {
+                      const float* M, const float* bstab, const float* s_v, const float* n_e,
+                      void* out, int* counters, cudaStream_t st) {
   const bool tma = std::is_same<T, __nv_bfloat16>::value &&
                    batch * c.cfg.n_kv_heads * (S + 1) > 2 * c.num_sms;
   if (tma && std::is_same<T, __nv_bfloat16>::value)
     return launch_tgs<T, D, G, std::is_same<T, __nv_bfloat16>::value>(
-        c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
+        c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, s_v, n_e, out, counters, st);
   return launch_tgs<T, D, G, false>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M,
-                                    bstab, out, counters, st);
+                                    bstab, s_v, n_e, out, counters, st);
 }
 
 template <typename T, int D>
 cudaError_t launch_t(const Ctx& c, int S, int nst, int batch, const void* q, const void* kn,
                      const void* vn, void* K_ret, void* V_ret, int32_t* cache_len, int cap,
-                     const float* M, const float* bstab, void* out, int* counters,
-                     cudaStream_t st) {
+                     const float* M, const float* bstab, const float* s_v, const float* n_e,
+                     void* out, int* counters, cudaStream_t st) {
   switch (c.group) {
-    case 1: return launch_tg<T, D, 1>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
-    case 2: return launch_tg<T, D, 2>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
-    case 4: return launch_tg<T, D, 4>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
-    case 8: return launch_tg<T, D, 8>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
+    case 1: return launch_tg<T, D, 1>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, s_v, n_e, out, counters, st);
+    case 2: return launch_tg<T, D, 2>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, s_v, n_e, out, counters, st);
+    case 4: return launch_tg<T, D, 4>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, s_v, n_e, out, counters, st);
+    case 8: return launch_tg<T, D, 8>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, s_v, n_e, out, counters, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -941,17 +988,17 @@ int decode_stages(int batch, int n_kv_heads, int cap, int S) {
 
 cudaError_t launch_decode(const Ctx& c, int batch, const void* q, const void* k_new,
                           const void* v_new, void* K_ret, void* V_ret, int32_t* cache_len,
-                          int cap, const float* M, const float* bstab, void* out,
-                          float* /*partials*/, int* counters, cudaStream_t st) {
+                          int cap, const float* M, const float* bstab, const float* s_v,
+                          const float* n_e, void* out, int* counters, cudaStream_t st) {
   const int S = decode_splits(batch, c.cfg.n_kv_heads, cap);
   const int nst = decode_stages(batch, c.cfg.n_kv_heads, cap, S);
   const int D = c.cfg.head_dim;
   if (c.cfg.dtype == IMEM_BF16) {
-    if (D == 128) return launch_t<__nv_bfloat16, 128>(c, S, nst, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
-    if (D == 64) return launch_t<__nv_bfloat16, 64>(c, S, nst, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
+    if (D == 128) return launch_t<__nv_bfloat16, 128>(c, S, nst, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, s_v, n_e, out, counters, st);
+    if (D == 64) return launch_t<__nv_bfloat16, 64>(c, S, nst, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, s_v, n_e, out, counters, st);
   } else {
-    if (D == 128) return launch_t<float, 128>(c, S, nst, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
-    if (D == 64) return launch_t<float, 64>(c, S, nst, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, out, counters, st);
+    if (D == 128) return launch_t<float, 128>(c, S, nst, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, s_v, n_e, out, counters, st);
+    if (D == 64) return launch_t<float, 64>(c, S, nst, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, s_v, n_e, out, counters, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -50,6 +50,7 @@ struct Workspace {
   size_t dec_part_off;          // decode split partials
   size_t dec_cnt_off;           // decode counters (int), zero between calls
   size_t mem_part_off;          // memory-update partials
+  size_t sv_part_off;           // value-sum partials of the moment statistics
   size_t total;
 };
 
@@ -78,13 +79,18 @@ cudaError_t launch_select_compact(const Ctx& c, int batch, int L, int B, const f
                                   void* K_ret, void* V_ret, int cap, void* scratch,
                                   cudaStream_t st);
 
+// sv_partials, s_v, n_count: value sums and evicted count (moment statistics);
+// all three null for the plain memory update.
 cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, const void* V,
                                  const int32_t* idx_e, int n_e, int chunk, float* M, float* bstab,
-                                 float* partials, cudaStream_t st);
+                                 float* partials, float* sv_partials, float* s_v, float* n_count,
+                                 cudaStream_t st);
 
+// s_v, n_e: the moment statistics' value sums and counts (moment readout);
+// null for the gated readout.
 cudaError_t launch_decode(const Ctx& c, int batch, const void* q, const void* k_new,
                           const void* v_new, void* K_ret, void* V_ret, int32_t* cache_len,
-                          int cap, const float* M, const float* bstab, void* out,
-                          float* partials, int* counters, cudaStream_t st);
+                          int cap, const float* M, const float* bstab, const float* s_v,
+                          const float* n_e, void* out, int* counters, cudaStream_t st);
 
 }  // namespace imem

@@ -91,11 +91,12 @@ template <> struct RawRow<float> {
   }
 };
 
-template <typename T, int D>
+template <typename T, int D, bool kSV>
 __global__ void __launch_bounds__(kMemThreads, 2)
 memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t* __restrict__ idx_e,
                  int n_e, int L, int Hkv, float log2lam, int tokens_per_group,
-                 float* __restrict__ partials, int* __restrict__ err) {
+                 float* __restrict__ partials, float* __restrict__ sv_partials,
+                 int* __restrict__ err) {
   using TL = MemTile<D>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -103,6 +104,7 @@ memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * TL::STAGE);
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
+  __shared__ float s_sv[8][16][8];   // per loader warp, per 16-byte column chunk: value sums
 
   const int g = blockIdx.x, kh = blockIdx.y, bi = blockIdx.z;
   const int G = gridDim.x;
@@ -171,6 +173,12 @@ memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t
         }
       }
     };
+    // optional value sums sum_i w_i v_i: a thread's items all share the
+    // column chunk tid % CH (kLoaders is a multiple of CH)
+    static_assert(kLoaders % CH == 0, "fixed column chunk per loader thread");
+    float svacc[kSV ? 8 : 1];
+#pragma unroll
+    for (int e = 0; e < (kSV ? 8 : 1); ++e) svacc[e] = 0.f;
     int pos_cur[ITEMS];
     load_pos(0, pos_cur);
     load_pos(1, pos_next);
@@ -202,6 +210,10 @@ memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t
         Raw::to_f32(cur_v[it], vf);
 #pragma unroll
         for (int e = 0; e < 8; ++e) vf[e] *= wv;
+        if constexpr (kSV) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) svacc[e] += vf[e];
+        }
         *reinterpret_cast<uint4*>(a_p + mn_off(jj, cc)) = to_half8(kf);
         *reinterpret_cast<uint4*>(b_p + mn_off(jj, cc)) = to_half8(vf);
         if (cc == 0)   // weight column: element 0 of the row in the last B atom
@@ -212,6 +224,25 @@ memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t
       if (c + 1 < nchunks) {
 #pragma unroll
         for (int it = 0; it < ITEMS; ++it) { cur_k[it] = nxt_k[it]; cur_v[it] = nxt_v[it]; }
+      }
+    }
+    if constexpr (kSV) {
+      // lanes with equal tid % CH hold the same columns: fold them, then the
+      // 8 loader warps through shared memory (named barrier 1: loaders only)
+#pragma unroll
+      for (int off = CH; off < 32; off <<= 1)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) svacc[e] += __shfl_xor_sync(0xffffffffu, svacc[e], off);
+      if (lane < CH) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s_sv[warp][lane][e] = svacc[e];
+      }
+      asm volatile("bar.sync 1, %0;\n" ::"n"(kLoaders) : "memory");
+      if (tid < D) {
+        float a = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) a += s_sv[w][tid / 8][tid % 8];
+        sv_partials[(((size_t)bi * Hkv + kh) * G + g) * D + tid] = a;
       }
     }
   } else if (lane == 0) {
@@ -269,11 +300,26 @@ memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t
 
 // M[:, cols] = decay * M[:, cols] + W_phi * sum_g S_g[:, cols]; the extra
 // column slice (blockIdx.x == D/16) does b from the s column.
+// With sv_partials, slice D/16 + 1 does the value sums: s_v = decay * s_v +
+// sum_g, and the sequence's count n_e += n_add (KV head 0 of the sequence).
 template <int D>
 __global__ void __launch_bounds__(256)
 memory_finalize_kernel(const float* __restrict__ partials, int G, const float* __restrict__ W_phi,
-                       int r, float decay_n, float* __restrict__ M, float* __restrict__ bstab) {
+                       int r, float decay_n, float* __restrict__ M, float* __restrict__ bstab,
+                       const float* __restrict__ sv_partials, float* __restrict__ s_v,
+                       float* __restrict__ n_e, float n_add, int Hkv) {
   extern __shared__ float fsm[];
+  if (blockIdx.x == D / 16 + 1) {   // value sums (only launched with sv_partials)
+    const int unit = blockIdx.y;
+    for (int c = threadIdx.x; c < D; c += 256) {
+      float a = 0.f;
+      for (int gg = 0; gg < G; ++gg) a += __ldcg(&sv_partials[((size_t)unit * G + gg) * D + c]);
+      float* sp = s_v + (size_t)unit * D + c;
+      *sp = fmaf(*sp, decay_n, a);
+    }
+    if (threadIdx.x == 0 && unit % Hkv == 0) n_e[unit / Hkv] += n_add;
+    return;
+  }
   float* sW = fsm;                 // [r][D]
   float* sS = sW + r * D;          // [D][16]
   const int unit = blockIdx.y, sl = blockIdx.x;
@@ -281,8 +327,9 @@ memory_finalize_kernel(const float* __restrict__ partials, int G, const float* _
   const bool bcol = (sl == D / 16);
   const int ncols = bcol ? 1 : 16;
   const int col0 = bcol ? D : sl * 16;
-  for (int i = tid; i < r * D / 4; i += 256)
-    reinterpret_cast<float4*>(sW)[i] = __ldg(reinterpret_cast<const float4*>(W_phi) + i);
+  if (W_phi)   // null: the identity map (r == D)
+    for (int i = tid; i < r * D / 4; i += 256)
+      reinterpret_cast<float4*>(sW)[i] = __ldg(reinterpret_cast<const float4*>(W_phi) + i);
   const float* p = partials + (size_t)unit * G * D * (D + 1);
   for (int i = tid; i < D * ncols; i += 256) {
     const int dk = i / ncols, cc = i % ncols;
@@ -294,8 +341,12 @@ memory_finalize_kernel(const float* __restrict__ partials, int G, const float* _
   for (int i = tid; i < r * ncols; i += 256) {
     const int ri = i / ncols, cc = i % ncols;
     float a = 0.f;
+    if (W_phi) {
 #pragma unroll 8
-    for (int dk = 0; dk < D; ++dk) a = fmaf(sW[ri * D + dk], sS[dk * 16 + cc], a);
+      for (int dk = 0; dk < D; ++dk) a = fmaf(sW[ri * D + dk], sS[dk * 16 + cc], a);
+    } else {
+      a = sS[ri * 16 + cc];
+    }
     if (bcol) {
       float* bp = bstab + (size_t)unit * r + ri;
       *bp = fmaf(*bp, decay_n, a);
@@ -322,7 +373,8 @@ int memory_groups(int batch, int n_kv_heads, int n_e, int chunk) {
 
 cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, const void* V,
                                  const int32_t* idx_e, int n_e, int chunk, float* M, float* bstab,
-                                 float* partials, cudaStream_t st) {
+                                 float* partials, float* sv_partials, float* s_v, float* n_count,
+                                 cudaStream_t st) {
   if (n_e == 0) return cudaSuccess;
   const int Hkv = c.cfg.n_kv_heads, D = c.cfg.head_dim, r = c.cfg.mem_r;
   const int G = memory_groups(batch, Hkv, n_e, chunk);
@@ -334,13 +386,13 @@ cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, 
   cudaError_t e = cudaSuccess;
 #define IMEM_MEM(TT, DD)                                                                       \
   do {                                                                                         \
-    auto kfn = memory_tc_kernel<TT, DD>;                                                       \
+    auto kfn = sv_partials ? memory_tc_kernel<TT, DD, true> : memory_tc_kernel<TT, DD, false>; \
     e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,                 \
                              MemTile<DD>::SMEM);                                               \
     if (e != cudaSuccess) return e;                                                            \
     kfn<<<grid, kMemThreads, MemTile<DD>::SMEM, st>>>((const TT*)K, (const TT*)V, idx_e, n_e,  \
                                                       L, Hkv, log2lam, tokens_per_group,       \
-                                                      partials, c.err);                        \
+                                                      partials, sv_partials, c.err);           \
   } while (0)
   if (c.cfg.dtype == IMEM_BF16) {
     if (D == 128) IMEM_MEM(__nv_bfloat16, 128); else IMEM_MEM(__nv_bfloat16, 64);
@@ -351,16 +403,22 @@ cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, 
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const float decay_n = (float)pow((double)c.cfg.lambda, (double)n_e);
-  dim3 fgrid(D / 16 + 1, batch * Hkv);
+  dim3 fgrid(D / 16 + 1 + (sv_partials ? 1 : 0), batch * Hkv);
+  // moment statistics use the identity map: the finalize skips the product
+  const float* phi = c.cfg.readout == IMEM_READOUT_MOMENT ? nullptr : c.W_phi;
   const size_t fsmem = ((size_t)r * D + (size_t)D * 16) * sizeof(float);
   if (D == 128) {
     e = cudaFuncSetAttribute(memory_finalize_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem);
     if (e != cudaSuccess) return e;
-    memory_finalize_kernel<128><<<fgrid, 256, fsmem, st>>>(partials, Gused, c.W_phi, r, decay_n, M, bstab);
+    memory_finalize_kernel<128><<<fgrid, 256, fsmem, st>>>(partials, Gused, phi, r, decay_n, M,
+                                                           bstab, sv_partials, s_v, n_count,
+                                                           (float)n_e, Hkv);
   } else {
     e = cudaFuncSetAttribute(memory_finalize_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem);
     if (e != cudaSuccess) return e;
-    memory_finalize_kernel<64><<<fgrid, 256, fsmem, st>>>(partials, Gused, c.W_phi, r, decay_n, M, bstab);
+    memory_finalize_kernel<64><<<fgrid, 256, fsmem, st>>>(partials, Gused, phi, r, decay_n, M,
+                                                          bstab, sv_partials, s_v, n_count,
+                                                          (float)n_e, Hkv);
   }
   return cudaGetLastError();
 }
@@ -425,12 +483,13 @@ cudaError_t launch_memory_static(int batch, int L, int Hkv, int r, float lambda,
   const int tokens_per_group = ((chunks + G - 1) / G) * chunk;
   const int Gused = (n_e + tokens_per_group - 1) / tokens_per_group;
   const float log2lam = (float)log2((double)lambda);
-  auto kfn = memory_tc_kernel<T, D>;
+  auto kfn = memory_tc_kernel<T, D, false>;
   cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        MemTile<D>::SMEM);
   if (e != cudaSuccess) return e;
   kfn<<<dim3(Gused, Hkv, batch), kMemThreads, MemTile<D>::SMEM, st>>>(
-      (const T*)K, (const T*)V, idx_e, n_e, L, Hkv, log2lam, tokens_per_group, scratch, err);
+      (const T*)K, (const T*)V, idx_e, n_e, L, Hkv, log2lam, tokens_per_group, scratch, nullptr,
+      err);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const float decay_n = (float)pow((double)lambda, (double)n_e);
@@ -438,8 +497,8 @@ cudaError_t launch_memory_static(int batch, int L, int Hkv, int r, float lambda,
   e = cudaFuncSetAttribute(memory_finalize_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)fsmem);
   if (e != cudaSuccess) return e;
-  memory_finalize_kernel<D><<<dim3(D / 16 + 1, units), 256, fsmem, st>>>(scratch, Gused, W_phi, r,
-                                                                        decay_n, M, bstab);
+  memory_finalize_kernel<D><<<dim3(D / 16 + 1, units), 256, fsmem, st>>>(
+      scratch, Gused, W_phi, r, decay_n, M, bstab, nullptr, nullptr, nullptr, 0.f, Hkv);
   return cudaGetLastError();
 }
 

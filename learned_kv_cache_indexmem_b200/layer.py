@@ -21,33 +21,48 @@ class PrefillState:
     K_ret: torch.Tensor           # [b, cap, Hkv, d]
     V_ret: torch.Tensor
     cache_len: torch.Tensor       # [b] int32
-    M: torch.Tensor               # [b, Hkv, r, d] fp32
-    bstab: torch.Tensor           # [b, Hkv, r] fp32
+    M: torch.Tensor               # [b, Hkv, r, d] fp32 (moment readout: S^T, r = d)
+    bstab: torch.Tensor           # [b, Hkv, r] fp32 (moment readout: s_k)
+    s_v: Optional[torch.Tensor] = None   # [b, Hkv, d] fp32, moment readout only
+    n_e: Optional[torch.Tensor] = None   # [b] fp32, moment readout only
 
 
 class IndexMemLayer:
     """Context for one layer. ``weights`` holds device tensors W_iq [Hq,d,dI],
-    W_ik [H,dI], w_ig [H,Hq] (model dtype), W_phi [r,d], w_gate [Hq,d] (fp32)."""
+    W_ik [H,dI], w_ig [H,Hq] (model dtype), W_phi [r,d], w_gate [Hq,d] (fp32).
+
+    readout="gated" is IndexMem's memory readout; readout="moment" keeps
+    MomentKV's moment statistics instead (r = d, no decay; W_phi and w_gate
+    are not used): update_memory then accumulates them and decode mixes the
+    retained attention with their estimate of the evicted attention."""
 
     def __init__(self, hidden, n_q_heads, n_kv_heads, head_dim, idx_dim, mem_r, lam, dtype,
-                 weights, gate_override: Optional[float] = None, eps: float = 1e-6):
+                 weights, gate_override: Optional[float] = None, eps: float = 1e-6,
+                 readout: str = "gated"):
+        if readout not in ("gated", "moment"):
+            raise ValueError("readout must be 'gated' or 'moment'")
+        self.moment = readout == "moment"
+        if self.moment:
+            mem_r, lam = head_dim, 1.0
         self.dims = dict(hidden=hidden, n_q_heads=n_q_heads, n_kv_heads=n_kv_heads,
                          head_dim=head_dim, idx_dim=idx_dim, mem_r=mem_r)
         self.lam = lam
         self.torch_dtype = dtype
         self.code = B_.BF16 if dtype == torch.bfloat16 else B_.FP32
         cfg = B_.make_config(hidden, n_q_heads, n_kv_heads, head_dim, idx_dim, mem_r, lam,
-                             self.code, eps=eps, gate_override=gate_override)
+                             self.code, eps=eps, gate_override=gate_override,
+                             readout=B_.READOUT_MOMENT if self.moment else B_.READOUT_GATED)
         self.ctx = B_.init(cfg, weights["W_iq"], weights["W_ik"], weights["w_ig"],
-                           weights["W_phi"], weights["w_gate"])
+                           None if self.moment else weights["W_phi"],
+                           None if self.moment else weights["w_gate"])
         self._ws = None
         self._ws_key = None
 
     @classmethod
-    def from_shape(cls, shape, weights, gate_override=None):
+    def from_shape(cls, shape, weights, gate_override=None, readout: str = "gated"):
         return cls(shape.hidden, shape.n_q_heads, shape.n_kv_heads, shape.head_dim,
                    shape.idx_dim, shape.mem_r, shape.lam, shape.torch_dtype, weights,
-                   gate_override=gate_override)
+                   gate_override=gate_override, readout=readout)
 
     def close(self):
         if self.ctx:
@@ -79,7 +94,10 @@ class IndexMemLayer:
             V_ret=torch.zeros(batch, cap, Hkv, d, dtype=self.torch_dtype, device=device),
             cache_len=torch.full((batch,), B, dtype=torch.int32, device=device),
             M=torch.zeros(batch, Hkv, r, d, dtype=torch.float32, device=device),
-            bstab=torch.zeros(batch, Hkv, r, dtype=torch.float32, device=device))
+            bstab=torch.zeros(batch, Hkv, r, dtype=torch.float32, device=device),
+            s_v=(torch.zeros(batch, Hkv, d, dtype=torch.float32, device=device)
+                 if self.moment else None),
+            n_e=torch.zeros(batch, dtype=torch.float32, device=device) if self.moment else None)
 
     # -- the path --------------------------------------------------------------
     def score_and_evict(self, X, Q, K, V, st: PrefillState, B: int, q_ranges=None,
@@ -97,8 +115,13 @@ class IndexMemLayer:
     def update_memory(self, K, V, st: PrefillState, B: int, chunk: int = 512, stream=None):
         batch, L = K.shape[0], K.shape[1]
         ws = self.workspace(batch, L, B, K.device)
-        B_.update_memory(self.ctx, batch, L, K, V, st.idx_evicted if B < L else None, L - B,
-                         chunk, st.M, st.bstab, ws, stream)
+        idx = st.idx_evicted if B < L else None
+        if self.moment:
+            B_.update_moments(self.ctx, batch, L, K, V, idx, L - B, chunk, st.M, st.bstab, st.s_v,
+                              st.n_e, ws, stream)
+        else:
+            B_.update_memory(self.ctx, batch, L, K, V, idx, L - B, chunk, st.M, st.bstab, ws,
+                             stream)
 
     def decode(self, q, k_new, v_new, st: PrefillState, out=None, B: Optional[int] = None,
                L: Optional[int] = None, stream=None):
@@ -107,8 +130,13 @@ class IndexMemLayer:
             raise RuntimeError("decode needs the workspace of a prefill (or call workspace())")
         if out is None:
             out = torch.empty_like(q)
-        B_.decode(self.ctx, batch, q, k_new, v_new, st.K_ret, st.V_ret, st.cache_len,
-                  st.K_ret.shape[1], st.M, st.bstab, out, self._ws, stream)
+        if self.moment:
+            B_.decode_moment(self.ctx, batch, q, k_new, v_new, st.K_ret, st.V_ret, st.cache_len,
+                             st.K_ret.shape[1], st.M, st.bstab, st.s_v, st.n_e, out, self._ws,
+                             stream)
+        else:
+            B_.decode(self.ctx, batch, q, k_new, v_new, st.K_ret, st.V_ret, st.cache_len,
+                      st.K_ret.shape[1], st.M, st.bstab, out, self._ws, stream)
         return out
 
     def sync(self, stream=None):

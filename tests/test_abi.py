@@ -56,6 +56,9 @@ def _cfg(**kw):
     (dict(lam=1.5), "IMEM_ERR_INVALID_ARG"),
     (dict(dtype=7), "IMEM_ERR_INVALID_ARG"),
     (dict(idx_heads=4), "IMEM_ERR_UNSUPPORTED"),
+    (dict(readout=5), "IMEM_ERR_INVALID_ARG"),
+    (dict(readout=B.READOUT_MOMENT, mem_r=32, lam=1.0), "IMEM_ERR_UNSUPPORTED"),   # r != d
+    (dict(readout=B.READOUT_MOMENT, mem_r=64, lam=0.99), "IMEM_ERR_UNSUPPORTED"),  # decay
 ])
 def test_init_rejects_bad_config_before_any_device_work(kw, code):
     with pytest.raises(B.IndexMemError) as ei:
@@ -81,6 +84,9 @@ def test_null_context_is_invalid_for_every_call():
     assert lib.imem_update_memory(None, 1, 16, 16, 16, 16, 4, 64, 16, 16, 16, None) == 1
     assert lib.imem_decode(None, 1, 16, 16, 16, 16, 16, 16, 8, 16, 16, 16, 16, None) == 1
     assert lib.imem_sync(None, None) == 1
+    assert lib.imem_update_moments(None, 1, 16, 16, 16, 16, 4, 64, 16, 16, 16, 16, 16, None) == 1
+    assert lib.imem_decode_moment(None, 1, 16, 16, 16, 16, 16, 16, 8, 16, 16, 16, 16, 16, 16,
+                                  None) == 1
     lib.imem_destroy(None)   # accepted
     out = ctypes.c_void_p(123)
     assert lib.imem_init(None, None, ctypes.byref(out)) == 1 and out.value is None
