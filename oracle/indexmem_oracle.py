@@ -279,6 +279,54 @@ def prefill_layer(X, Q, K, V, W_iq, W_ik, w_ig, W_phi, lam: float, B: int,
             "K_R": KR, "V_R": VR, "M": M, "b": bs}
 
 
+def prefill_streaming(X, Q, K, V, W_iq, W_ik, w_ig, W_phi, lam: float, B: int, ranges):
+    """Pre-eviction during chunked prefill ([IM-sum] §2.A: the indexer can evict
+    before the whole prefix has been processed, keeping the cache bounded).
+
+    The query ranges are processed in order (contiguous, from 0). Before range
+    [q0, q1) the cache holds the retained set R (at most B positions) with
+    their pooled importances. The candidates are R followed by the range's own
+    keys; their importances are pooled over the range's queries (running max,
+    causal within the range: I[t] = max(I_R[t], max_{s in [q0,q1)} A[s,t]) for
+    t in R, max_{s in [t,q1)} A[s,t] for t in the range). If there are more
+    than B candidates, the B most important stay (ties to the lower position)
+    and the others are evicted into the memory in ascending position order,
+    after everything evicted by earlier ranges.
+
+    Returns a dict: R [b, min(B, L)] final retained positions (ascending), M, b
+    (the memory), and ``chunks``: per range a dict with cand [b, n] candidate
+    positions, I [b, n] their importances, R, E (positions, ascending)."""
+    qhat, khat, gate = indexer_features(X, Q, W_iq, W_ik, w_ig)
+    b, L = khat.shape[:2]
+    R = [np.zeros(0, dtype=np.int64) for _ in range(b)]
+    IR = [np.zeros(0) for _ in range(b)]
+    M = bs = None
+    chunks = []
+    for (q0, q1) in ranges:
+        rec = {"cand": [], "I": [], "R": [], "E": []}
+        for bi in range(b):
+            cand = np.concatenate([R[bi], np.arange(q0, q1)])
+            prev = np.full((1, L), -np.inf)
+            prev[0, R[bi]] = IR[bi]
+            Ic = pooled_importance(qhat[bi:bi + 1], khat[bi:bi + 1], gate[bi:bi + 1],
+                                   q_begin=q0, q_end=q1, prev=prev, keys=cand)[0]
+            if len(cand) > B:
+                ri, ei = select_budget(Ic[None], B)   # candidate order = position order
+                R[bi], E, IR[bi] = cand[ri[0]], cand[ei[0]], Ic[ri[0]]
+            else:
+                R[bi], E, IR[bi] = cand, np.zeros(0, dtype=np.int64), Ic
+            for k, v in (("cand", cand), ("I", Ic), ("R", R[bi]), ("E", E)):
+                rec[k].append(v)
+        for k in rec:
+            rec[k] = np.stack(rec[k])
+        if rec["E"].shape[1] > 0:
+            M, bs = memory_update(K, V, rec["E"], W_phi, lam, M0=M, b0=bs)
+        chunks.append(rec)
+    if M is None:
+        M, bs = memory_update(K, V, np.zeros((b, 0), dtype=np.int64), W_phi, lam)
+    return {"R": np.stack(R), "M": M, "b": bs, "chunks": chunks}
+
+
 def importance_at_keys(X, Q, W_iq, W_ik, w_ig, keys, q_end: Optional[int] = None,
                        s_block: int = 4096) -> np.ndarray:
     """Pooled importance I[t] = max_{s in [t, q_end)} A[s,t] for a few keys t of
