@@ -244,6 +244,45 @@ imem_status imem_decode_moment(imem_ctx* ctx, int batch, const void* q, const vo
                                int cap, const float* S_T, const float* s_k, const float* s_v,
                                const float* n_e, void* out, void* workspace, void* stream);
 
+/* Pre-eviction during chunked prefill ([IM-sum] §2.A: the indexer can evict
+ * before the whole prefix has been processed, so the cache never holds more
+ * than B tokens). Called once per query range, in order, the ranges contiguous
+ * from 0: [q_begin, q_end) with q_end - q_begin <= chunk_max. Before a range the
+ * cache holds n_R = min(B, q_begin) retained tokens; the candidates are those,
+ * then the range's tokens. Their importance is pooled over the range's
+ * queries by the streaming running max (retained keys keep the maximum of
+ * earlier ranges; the range's keys are causal within it). If there are more
+ * than B candidates, the B most important stay (ties to the lower position)
+ * and the other n_ev = n_R + (q_end - q_begin) - B leave, in ascending
+ * position order, into the memory: M, bstab updated as imem_update_memory does
+ * with them (after all tokens evicted by earlier ranges).
+ *   X, Q, K, V         as imem_score_and_evict ([batch, L, ...], model dtype).
+ *   retained [batch, B] int32, in/out: the retained positions, ascending (the
+ *                      first n_R of each row valid before the call, the first
+ *                      min(B, q_end) after it). Caller-owned state.
+ *   evicted [batch * chunk_max] int32, out: [batch, n_ev] packed, ascending.
+ *   cand_importance    NULL or [batch, B + chunk_max] fp32, out: the candidates'
+ *                      pooled importance before selection (row: n_R retained,
+ *                      then the range's tokens; the rest of the row undefined).
+ *   M, bstab           the memory, in/out (as imem_update_memory); mem_chunk as
+ *                      its `chunk`.
+ *   finalize = 1       (requires q_end == L): K_ret/V_ret[:, :min(B, L)] =
+ *                      K/V[retained] as imem_score_and_evict does.
+ *   workspace          imem_workspace_size_evict bytes, zero-filled once, the
+ *                      same buffer for every range of one prefill (it keeps the
+ *                      retained tokens' indexer keys and importances); it also
+ *                      serves imem_decode.
+ * Errors: INVALID_ARG, SHAPE (ranges, cap), ALIGN, CUDA; UNSUPPORTED for a
+ * context in IMEM_READOUT_MOMENT mode. */
+imem_status imem_workspace_size_evict(imem_ctx* ctx, int batch, int L, int B, int chunk_max,
+                                      size_t* bytes);
+imem_status imem_prefill_evict_chunk(imem_ctx* ctx, int batch, int L, int B, int chunk_max,
+                                     const void* X, const void* Q, const void* K, const void* V,
+                                     int q_begin, int q_end, int32_t* retained, int32_t* evicted,
+                                     float* cand_importance, float* M, float* bstab,
+                                     int mem_chunk, int finalize, void* K_ret, void* V_ret,
+                                     int cap, void* workspace, void* stream);
+
 /* Waits for the stream, then reports the first error the device recorded for
  * this context since the last imem_sync (TIMEOUT for a bounded wait that ran
  * out, SHAPE for a decode into a full cache) or a CUDA error, and clears it. */

@@ -73,6 +73,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.imem_decode.argtypes = [vp, i, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp]
     lib.imem_sync.restype = i
     lib.imem_sync.argtypes = [vp, vp]
+    lib.imem_workspace_size_evict.restype = i
+    lib.imem_workspace_size_evict.argtypes = [vp, i, i, i, i, ctypes.POINTER(ctypes.c_size_t)]
+    lib.imem_prefill_evict_chunk.restype = i
+    lib.imem_prefill_evict_chunk.argtypes = [vp, i, i, i, i, vp, vp, vp, vp, i, i, vp, vp, vp,
+                                             vp, vp, i, i, vp, vp, i, vp, vp]
     lib.imem_update_moments.restype = i
     lib.imem_update_moments.argtypes = [vp, i, i, vp, vp, vp, i, i, vp, vp, vp, vp, vp, vp]
     lib.imem_decode_moment.restype = i
@@ -157,6 +162,23 @@ def decode(ctx, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab, 
     _check(load().imem_decode(
         ctx, batch, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(K_ret), _ptr(V_ret), _ptr(cache_len),
         cap, _ptr(M), _ptr(bstab), _ptr(out), _ptr(workspace), _stream(stream)), "imem_decode")
+
+
+def workspace_size_evict(ctx: int, batch: int, L: int, B: int, chunk_max: int) -> int:
+    n = ctypes.c_size_t()
+    _check(load().imem_workspace_size_evict(ctx, batch, L, B, chunk_max, ctypes.byref(n)),
+           "imem_workspace_size_evict")
+    return n.value
+
+
+def prefill_evict_chunk(ctx, batch, L, B, chunk_max, X, Q, K, V, q_begin, q_end, retained,
+                        evicted, cand_importance, M, bstab, mem_chunk, finalize, K_ret, V_ret,
+                        cap, workspace, stream=None):
+    _check(load().imem_prefill_evict_chunk(
+        ctx, batch, L, B, chunk_max, _ptr(X), _ptr(Q), _ptr(K), _ptr(V), q_begin, q_end,
+        _ptr(retained), _ptr(evicted), _ptr(cand_importance), _ptr(M), _ptr(bstab), mem_chunk,
+        int(finalize), _ptr(K_ret), _ptr(V_ret), cap, _ptr(workspace), _stream(stream)),
+        "imem_prefill_evict_chunk")
 
 
 def update_moments(ctx, batch, L, K, V, idx_evicted, n_evicted, chunk, S_T, s_k, s_v, n_e,

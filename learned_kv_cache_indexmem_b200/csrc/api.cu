@@ -50,6 +50,29 @@ Workspace workspace_layout(const Ctx& c, int batch, int L) {
   return w;
 }
 
+// Pre-eviction workspace: the plain layout over Lc = B + chunk_max candidate
+// rows (its q~ and k^ regions become the candidate buffers), then the
+// candidates' importances and the compaction temporaries.
+struct EvictWorkspace {
+  Workspace base;
+  size_t I_c_off, kh_tmp_off, I_tmp_off, pos_tmp_off, idx_r_off, idx_e_off, total;
+};
+
+EvictWorkspace evict_workspace_layout(const Ctx& c, int batch, int B, int chunk_max) {
+  const size_t Lc = (size_t)B + chunk_max;
+  EvictWorkspace w;
+  w.base = workspace_layout(c, batch, (int)Lc);
+  size_t off = w.base.total;
+  w.I_c_off = off;     off = align_up(off + (size_t)batch * Lc * sizeof(float), 256);
+  w.kh_tmp_off = off;  off = align_up(off + (size_t)batch * B * kIdxPad * 2, 1024);
+  w.I_tmp_off = off;   off = align_up(off + (size_t)batch * B * sizeof(float), 256);
+  w.pos_tmp_off = off; off = align_up(off + (size_t)batch * B * sizeof(int32_t), 256);
+  w.idx_r_off = off;   off = align_up(off + (size_t)batch * B * sizeof(int32_t), 256);
+  w.idx_e_off = off;   off = align_up(off + (size_t)batch * Lc * sizeof(int32_t), 256);
+  w.total = off;
+  return w;
+}
+
 bool make_tmap_bf16(const Ctx& c, CUtensorMap* map, const void* base, uint64_t width,
                     uint64_t rows, uint32_t box_rows) {
   using Fn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -361,6 +384,88 @@ imem_status imem_decode_moment(imem_ctx* h, int batch, const void* q, const void
   if (h->c.cfg.readout != IMEM_READOUT_MOMENT) return IMEM_ERR_UNSUPPORTED;
   return decode_common(h, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, S_T, s_k, s_v,
                        n_e, out, workspace, stream);
+}
+
+imem_status imem_workspace_size_evict(imem_ctx* h, int batch, int L, int B, int chunk_max,
+                                     size_t* bytes) {
+  if (!h || !bytes) return IMEM_ERR_INVALID_ARG;
+  if (batch < 1 || L < 1 || B < 1 || chunk_max < 1) return IMEM_ERR_SHAPE;
+  if ((size_t)B + chunk_max > (size_t)INT32_MAX / imem::kIdxPad) return IMEM_ERR_SHAPE;
+  *bytes = imem::evict_workspace_layout(h->c, batch, B, chunk_max).total;
+  return IMEM_OK;
+}
+
+imem_status imem_prefill_evict_chunk(imem_ctx* h, int batch, int L, int B, int chunk_max,
+                                     const void* X, const void* Q, const void* K, const void* V,
+                                     int q_begin, int q_end, int32_t* retained, int32_t* evicted,
+                                     float* cand_importance, float* M, float* bstab,
+                                     int mem_chunk, int finalize, void* K_ret, void* V_ret,
+                                     int cap, void* workspace, void* stream) {
+  if (!h) return IMEM_ERR_INVALID_ARG;
+  const Ctx& c = h->c;
+  if (c.cfg.readout != IMEM_READOUT_GATED) return IMEM_ERR_UNSUPPORTED;
+  if (finalize != 0 && finalize != 1) return IMEM_ERR_INVALID_ARG;
+  if (batch < 1 || L < 1 || B < 1 || chunk_max < 1) return IMEM_ERR_SHAPE;
+  if (q_begin < 0 || q_end <= q_begin || q_end > L || q_end - q_begin > chunk_max)
+    return IMEM_ERR_SHAPE;
+  if (mem_chunk < 64 || mem_chunk % 64) return IMEM_ERR_SHAPE;
+  const int n_R = B < q_begin ? B : q_begin;          // retained before this range
+  const int C = q_end - q_begin, n = n_R + C, n_ev = n > B ? n - B : 0;
+  IMEM_CHECK(check_ptr(X));
+  IMEM_CHECK(check_ptr(Q));
+  IMEM_CHECK(check_ptr(retained));
+  IMEM_CHECK(check_ptr(workspace));
+  if (cand_importance) IMEM_CHECK(check_ptr(cand_importance));
+  if (n_ev > 0) {
+    IMEM_CHECK(check_ptr(K));
+    IMEM_CHECK(check_ptr(V));
+    IMEM_CHECK(check_ptr(evicted));
+    IMEM_CHECK(check_ptr(M));
+    IMEM_CHECK(check_ptr(bstab));
+  }
+  if (finalize) {
+    if (q_end != L) return IMEM_ERR_SHAPE;
+    if (cap < (B < L ? B : L)) return IMEM_ERR_SHAPE;
+    IMEM_CHECK(check_ptr(K));
+    IMEM_CHECK(check_ptr(V));
+    IMEM_CHECK(check_ptr(K_ret));
+    IMEM_CHECK(check_ptr(V_ret));
+  }
+  IMEM_CHECK(check_device(c));
+  cudaStream_t st = (cudaStream_t)stream;
+  const int Lc = B + chunk_max;
+  const imem::EvictWorkspace ws = imem::evict_workspace_layout(c, batch, B, chunk_max);
+  char* wsb = (char*)workspace;
+  imem::EvictBuffers eb;
+  __nv_bfloat16* qt = (__nv_bfloat16*)(wsb + ws.base.qt_off);
+  eb.kh_c = (__nv_bfloat16*)(wsb + ws.base.kh_off);
+  eb.I_c = (float*)(wsb + ws.I_c_off);
+  eb.kh_tmp = (__nv_bfloat16*)(wsb + ws.kh_tmp_off);
+  eb.I_tmp = (float*)(wsb + ws.I_tmp_off);
+  eb.pos_tmp = (int32_t*)(wsb + ws.pos_tmp_off);
+  eb.idx_r = (int32_t*)(wsb + ws.idx_r_off);
+  eb.idx_e = (int32_t*)(wsb + ws.idx_e_off);
+  // the range's indexer features go to candidate rows [n_R, n)
+  IMEM_CHECK(cuda_status(imem::launch_prologue(c, batch, L, X, Q, q_begin, q_end, qt, eb.kh_c,
+                                               eb.I_c, st, Lc, n_R - q_begin)));
+  IMEM_CHECK(cuda_status(imem::launch_scoring(c, batch, Lc, qt, eb.kh_c, eb.I_c, n_R, n, st)));
+  if (cand_importance)
+    IMEM_CHECK(cuda_status(cudaMemcpyAsync(cand_importance, eb.I_c, (size_t)batch * Lc * sizeof(float),
+                                           cudaMemcpyDeviceToDevice, st)));
+  if (n_ev > 0) {
+    IMEM_CHECK(cuda_status(imem::launch_evict_chunk(c, batch, B, Lc, n_R, q_begin, C, eb, retained,
+                                                    evicted, st)));
+    float* part = (float*)(wsb + ws.base.mem_part_off);
+    IMEM_CHECK(cuda_status(imem::launch_memory_update(c, batch, L, K, V, evicted, n_ev, mem_chunk,
+                                                      M, bstab, part, nullptr, nullptr, nullptr,
+                                                      st)));
+  } else {
+    IMEM_CHECK(cuda_status(imem::launch_append_positions(batch, B, n_R, q_begin, C, retained, st)));
+  }
+  if (finalize)
+    IMEM_CHECK(cuda_status(imem::launch_gather(c, batch, L, B < L ? B : L, retained, B, K, V,
+                                               K_ret, V_ret, cap, st)));
+  return IMEM_OK;
 }
 
 imem_status imem_sync(imem_ctx* h, void* stream) {

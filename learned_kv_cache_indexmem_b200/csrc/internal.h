@@ -66,9 +66,12 @@ cudaError_t pack_indexer_weights(Ctx& c, const void* W_iq, const void* W_ik, con
 
 // ---- launchers (return cudaGetLastError()) ----------------------------------
 
+// Token t of sequence s (q_begin <= t < q_end) is written to output row
+// s * out_stride + t + out_shift of qt, kh and running_max (out_stride 0: L).
 cudaError_t launch_prologue(const Ctx& c, int batch, int L, const void* X, const void* Q,
                             int q_begin, int q_end, __nv_bfloat16* qt, __nv_bfloat16* kh,
-                            float* running_max, cudaStream_t st);
+                            float* running_max, cudaStream_t st, int out_stride = 0,
+                            int out_shift = 0);
 
 cudaError_t launch_scoring(const Ctx& c, int batch, int L, const __nv_bfloat16* qt,
                            const __nv_bfloat16* kh, float* running_max, int q_begin, int q_end,
@@ -78,6 +81,32 @@ cudaError_t launch_select_compact(const Ctx& c, int batch, int L, int B, const f
                                   const void* K, const void* V, int32_t* idx_r, int32_t* idx_e,
                                   void* K_ret, void* V_ret, int cap, void* scratch,
                                   cudaStream_t st);
+
+// Pre-eviction during chunked prefill: one query range [q0, q0 + C) over the
+// candidates = n_R retained tokens + the range's C tokens, laid out with a
+// row stride Lc in the candidate buffers (indexer keys kh_c [b, Lc, 64],
+// importances I_c [b, Lc]). Selects the B most important candidates,
+// compacts them to rows [0, B) (positions to `retained` [b, B]) and writes the
+// evicted positions, ascending, to `evicted` [b, n - B] (n = n_R + C > B).
+struct EvictBuffers {
+  __nv_bfloat16* kh_c;   // [b, Lc, kIdxPad]
+  float* I_c;            // [b, Lc]
+  __nv_bfloat16* kh_tmp; // [b, B, kIdxPad]
+  float* I_tmp;          // [b, B]
+  int32_t* pos_tmp;      // [b, B]
+  int32_t* idx_r;        // [b, B]
+  int32_t* idx_e;        // [b, Lc]
+};
+cudaError_t launch_evict_chunk(const Ctx& c, int batch, int B, int Lc, int n_R, int q0, int C,
+                               const EvictBuffers& w, int32_t* retained, int32_t* evicted,
+                               cudaStream_t st);
+// Appends positions q0..q0+C-1 at rows [n_R, n_R + C) of `retained` (stride B).
+cudaError_t launch_append_positions(int batch, int B, int n_R, int q0, int C, int32_t* retained,
+                                    cudaStream_t st);
+// K_ret/V_ret[:, :n] = K/V[idx[:, :n]] (idx stride `idx_stride`).
+cudaError_t launch_gather(const Ctx& c, int batch, int L, int n, const int32_t* idx,
+                          int idx_stride, const void* K, const void* V, void* K_ret, void* V_ret,
+                          int cap, cudaStream_t st);
 
 // sv_partials, s_v, n_count: value sums and evicted count (moment statistics);
 // all three null for the plain memory update.

@@ -56,7 +56,8 @@ prologue_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
                    const __grid_constant__ CUtensorMap map_wc, const __grid_constant__ CUtensorMap map_wq,
                    int L, int H, int Hq, int D, int dI, int N1, int q_begin, int q_end, int batch,
                    __nv_bfloat16* __restrict__ qt, __nv_bfloat16* __restrict__ kh,
-                   float* __restrict__ running_max, int* __restrict__ err) {
+                   float* __restrict__ running_max, int out_stride, int out_shift,
+                   int* __restrict__ err) {
   constexpr int EPB = 128 / (int)sizeof(T);                  // elements per 128-byte row
   constexpr uint32_t FMT = std::is_same<T, float>::value ? tc::kFmtTF32 : tc::kFmtBF16;
   extern __shared__ unsigned char smem_raw[];
@@ -178,7 +179,7 @@ prologue_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
       const int seq = tile / tiles_per_seq;
       const int t = q_begin + (tile % tiles_per_seq) * kTileM + quarter * 32 + lane;
       const bool valid = t < q_end;
-      const size_t row = (size_t)seq * L + t;
+      const size_t row = (size_t)seq * out_stride + t + out_shift;   // output row of token t
       if (!tc::mbar_wait(d1_full, tcount & 1)) { ok = false; break; }
       tc::fence_after();
       // shared key: RMS-normalised kI
@@ -300,7 +301,7 @@ bool make_tmap(const Ctx& c, CUtensorMap* map, const void* base, uint64_t rows, 
 template <typename T>
 cudaError_t launch_pro(const Ctx& c, int batch, int L, const void* X, const void* Q, int q_begin,
                        int q_end, __nv_bfloat16* qt, __nv_bfloat16* kh, float* running_max,
-                       cudaStream_t st) {
+                       int out_stride, int out_shift, cudaStream_t st) {
   const int H = c.cfg.hidden, Hq = c.cfg.n_q_heads, D = c.cfg.head_dim, dI = c.cfg.idx_dim;
   CUtensorMap mx, mq, mwc, mwq;
   if (!make_tmap<T>(c, &mx, X, (uint64_t)batch * L, H, kTileM) ||
@@ -319,7 +320,7 @@ cudaError_t launch_pro(const Ctx& c, int batch, int L, const void* X, const void
     attr_set[c.device & 63] = true;
   }
   k<<<grid, kPThreads, kProSmem, st>>>(mx, mq, mwc, mwq, L, H, Hq, D, dI, c.N1, q_begin, q_end,
-                                       batch, qt, kh, running_max, c.err);
+                                       batch, qt, kh, running_max, out_stride, out_shift, c.err);
   return cudaGetLastError();
 }
 
@@ -347,10 +348,13 @@ cudaError_t pack_indexer_weights(Ctx& c, const void* W_iq, const void* W_ik, con
 
 cudaError_t launch_prologue(const Ctx& c, int batch, int L, const void* X, const void* Q,
                             int q_begin, int q_end, __nv_bfloat16* qt, __nv_bfloat16* kh,
-                            float* running_max, cudaStream_t st) {
+                            float* running_max, cudaStream_t st, int out_stride, int out_shift) {
+  if (out_stride <= 0) out_stride = L;
   if (c.cfg.dtype == IMEM_BF16)
-    return launch_pro<__nv_bfloat16>(c, batch, L, X, Q, q_begin, q_end, qt, kh, running_max, st);
-  return launch_pro<float>(c, batch, L, X, Q, q_begin, q_end, qt, kh, running_max, st);
+    return launch_pro<__nv_bfloat16>(c, batch, L, X, Q, q_begin, q_end, qt, kh, running_max,
+                                     out_stride, out_shift, st);
+  return launch_pro<float>(c, batch, L, X, Q, q_begin, q_end, qt, kh, running_max, out_stride,
+                           out_shift, st);
 }
 
 }  // namespace imem

@@ -14,6 +14,12 @@
 //
 // Compaction: K_ret[:, j] = K[:, R[j]] and V_ret likewise, all KV heads at
 // once (one contiguous row of Hkv*d elements per token), 16-byte vectors.
+//
+// Pre-eviction during chunked prefill (§2.A: eviction before the whole
+// prefix is processed): the same selection over the candidates of a query
+// range (the retained tokens, then the range's tokens), then the retained
+// candidates' indexer keys, importances and positions are compacted to the
+// front of the candidate buffers and the evicted positions listed in order.
 #include "common.cuh"
 #include "internal.h"
 
@@ -56,11 +62,11 @@ __device__ __forceinline__ int block_inclusive_scan(int v, int* s_warp, int* tot
 }
 
 __global__ void __launch_bounds__(kSelThreads)
-select_kernel(const float* __restrict__ I, int L, int B, int32_t* __restrict__ idx_r,
+select_kernel(const float* __restrict__ I, int L, int stride, int B, int32_t* __restrict__ idx_r,
               int32_t* __restrict__ idx_e) {
   const int bi = blockIdx.x;
   const int tid = threadIdx.x;
-  const float* Ib = I + (size_t)bi * L;
+  const float* Ib = I + (size_t)bi * stride;
   __shared__ int s_hist[256];
   __shared__ int s_warp[32];
   __shared__ uint32_t s_prefix, s_mask;
@@ -133,17 +139,18 @@ select_kernel(const float* __restrict__ I, int L, int B, int32_t* __restrict__ i
   }
 }
 
-// One warp group per retained row: copies Hkv*d elements of K and V.
+// One warp group per retained row: copies Hkv*d elements of K and V. Rows
+// [0, n) of sequence bi come from positions idx_r[bi * idx_stride + j].
 template <typename T>
 __global__ void gather_kernel(const T* __restrict__ K, const T* __restrict__ V,
                               const int32_t* __restrict__ idx_r, T* __restrict__ K_ret,
-                              T* __restrict__ V_ret, int L, int B, int cap, int row_elems,
-                              int rows_per_cta) {
+                              T* __restrict__ V_ret, int L, int n, int idx_stride, int cap,
+                              int row_elems, int rows_per_cta) {
   const int bi = blockIdx.y;
   const int vec = 16 / sizeof(T);
   const int nvec = row_elems / vec;
-  for (int j = blockIdx.x * rows_per_cta; j < min(B, (blockIdx.x + 1) * rows_per_cta); ++j) {
-    const int src = idx_r[(size_t)bi * B + j];
+  for (int j = blockIdx.x * rows_per_cta; j < min(n, (blockIdx.x + 1) * rows_per_cta); ++j) {
+    const int src = idx_r[(size_t)bi * idx_stride + j];
     const uint4* ks = reinterpret_cast<const uint4*>(K + ((size_t)bi * L + src) * row_elems);
     const uint4* vs = reinterpret_cast<const uint4*>(V + ((size_t)bi * L + src) * row_elems);
     uint4* kd = reinterpret_cast<uint4*>(K_ret + ((size_t)bi * cap + j) * row_elems);
@@ -155,27 +162,119 @@ __global__ void gather_kernel(const T* __restrict__ K, const T* __restrict__ V,
   }
 }
 
+// ---- pre-eviction during chunked prefill ----------------------------------
+// Candidate ci of a range is retained row ci (ci < n_R) or the range's token
+// q0 + ci - n_R; candidate order is position order.
+__device__ __forceinline__ int cand_pos(int ci, int n_R, int q0, const int32_t* ret_b) {
+  return ci < n_R ? ret_b[ci] : q0 + ci - n_R;
+}
+
+constexpr int kRowsPerCompactCta = 32;   // 8 threads (16-byte chunks of a 128-byte key) per row
+
+// Gathers the selected candidates (idx_r) into the temporaries and writes the
+// evicted candidates' positions (idx_e, ascending) to `evicted`.
+__global__ void __launch_bounds__(256)
+evict_compact_kernel(const int32_t* __restrict__ idx_r, const int32_t* __restrict__ idx_e, int B,
+                     int n_ev, int n_R, int q0, int Lc, const int32_t* __restrict__ retained,
+                     const __nv_bfloat16* __restrict__ kh_c, const float* __restrict__ I_c,
+                     int32_t* __restrict__ pos_tmp, __nv_bfloat16* __restrict__ kh_tmp,
+                     float* __restrict__ I_tmp, int32_t* __restrict__ evicted) {
+  const int bi = blockIdx.y;
+  const int j = blockIdx.x * kRowsPerCompactCta + threadIdx.x / 8, c = threadIdx.x % 8;
+  const int32_t* ret_b = retained + (size_t)bi * B;
+  if (j < B) {
+    const int ci = idx_r[(size_t)bi * B + j];
+    const uint4* src = reinterpret_cast<const uint4*>(kh_c + ((size_t)bi * Lc + ci) * kIdxPad);
+    reinterpret_cast<uint4*>(kh_tmp + ((size_t)bi * B + j) * kIdxPad)[c] = src[c];
+    if (c == 0) {
+      pos_tmp[(size_t)bi * B + j] = cand_pos(ci, n_R, q0, ret_b);
+      I_tmp[(size_t)bi * B + j] = I_c[(size_t)bi * Lc + ci];
+    }
+  } else if (j < B + n_ev && c == 0) {
+    const int e = j - B;
+    evicted[(size_t)bi * n_ev + e] = cand_pos(idx_e[(size_t)bi * n_ev + e], n_R, q0, ret_b);
+  }
+}
+
+// Rows [0, B) of the candidate buffers and `retained` from the temporaries.
+__global__ void __launch_bounds__(256)
+evict_copyback_kernel(int B, int Lc, const int32_t* __restrict__ pos_tmp,
+                      const __nv_bfloat16* __restrict__ kh_tmp, const float* __restrict__ I_tmp,
+                      int32_t* __restrict__ retained, __nv_bfloat16* __restrict__ kh_c,
+                      float* __restrict__ I_c) {
+  const int bi = blockIdx.y;
+  const int j = blockIdx.x * kRowsPerCompactCta + threadIdx.x / 8, c = threadIdx.x % 8;
+  if (j >= B) return;
+  reinterpret_cast<uint4*>(kh_c + ((size_t)bi * Lc + j) * kIdxPad)[c] =
+      reinterpret_cast<const uint4*>(kh_tmp + ((size_t)bi * B + j) * kIdxPad)[c];
+  if (c == 0) {
+    retained[(size_t)bi * B + j] = pos_tmp[(size_t)bi * B + j];
+    I_c[(size_t)bi * Lc + j] = I_tmp[(size_t)bi * B + j];
+  }
+}
+
+__global__ void append_positions_kernel(int B, int n_R, int q0, int C, int32_t* __restrict__ retained) {
+  const int bi = blockIdx.y;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < C) retained[(size_t)bi * B + n_R + i] = q0 + i;
+}
+
 }  // namespace
+
+cudaError_t launch_evict_chunk(const Ctx& c, int batch, int B, int Lc, int n_R, int q0, int C,
+                               const EvictBuffers& w, int32_t* retained, int32_t* evicted,
+                               cudaStream_t st) {
+  (void)c;
+  const int n = n_R + C, n_ev = n - B;
+  if (n_ev <= 0) return cudaErrorInvalidValue;
+  select_kernel<<<batch, kSelThreads, 0, st>>>(w.I_c, n, Lc, B, w.idx_r, w.idx_e);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  dim3 g1((B + n_ev + kRowsPerCompactCta - 1) / kRowsPerCompactCta, batch);
+  evict_compact_kernel<<<g1, 256, 0, st>>>(w.idx_r, w.idx_e, B, n_ev, n_R, q0, Lc, retained,
+                                           w.kh_c, w.I_c, w.pos_tmp, w.kh_tmp, w.I_tmp, evicted);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  dim3 g2((B + kRowsPerCompactCta - 1) / kRowsPerCompactCta, batch);
+  evict_copyback_kernel<<<g2, 256, 0, st>>>(B, Lc, w.pos_tmp, w.kh_tmp, w.I_tmp, retained, w.kh_c,
+                                            w.I_c);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append_positions(int batch, int B, int n_R, int q0, int C, int32_t* retained,
+                                    cudaStream_t st) {
+  if (C <= 0) return cudaSuccess;
+  dim3 g((C + 255) / 256, batch);
+  append_positions_kernel<<<g, 256, 0, st>>>(B, n_R, q0, C, retained);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const Ctx& c, int batch, int L, int n, const int32_t* idx,
+                          int idx_stride, const void* K, const void* V, void* K_ret, void* V_ret,
+                          int cap, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  const int row_elems = c.cfg.n_kv_heads * c.cfg.head_dim;
+  const int rows_per_cta = 4;
+  dim3 grid((n + rows_per_cta - 1) / rows_per_cta, batch);
+  if (c.cfg.dtype == IMEM_BF16)
+    gather_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(
+        (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, idx, (__nv_bfloat16*)K_ret,
+        (__nv_bfloat16*)V_ret, L, n, idx_stride, cap, row_elems, rows_per_cta);
+  else
+    gather_kernel<float><<<grid, 128, 0, st>>>((const float*)K, (const float*)V, idx,
+                                               (float*)K_ret, (float*)V_ret, L, n, idx_stride,
+                                               cap, row_elems, rows_per_cta);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_select_compact(const Ctx& c, int batch, int L, int B, const float* running_max,
                                   const void* K, const void* V, int32_t* idx_r, int32_t* idx_e,
                                   void* K_ret, void* V_ret, int cap, void* /*scratch*/,
                                   cudaStream_t st) {
-  select_kernel<<<batch, kSelThreads, 0, st>>>(running_max, L, B, idx_r, idx_e);
+  select_kernel<<<batch, kSelThreads, 0, st>>>(running_max, L, L, B, idx_r, idx_e);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int row_elems = c.cfg.n_kv_heads * c.cfg.head_dim;
-  const int rows_per_cta = 4;
-  dim3 grid((B + rows_per_cta - 1) / rows_per_cta, batch);
-  if (c.cfg.dtype == IMEM_BF16)
-    gather_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(
-        (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, idx_r, (__nv_bfloat16*)K_ret,
-        (__nv_bfloat16*)V_ret, L, B, cap, row_elems, rows_per_cta);
-  else
-    gather_kernel<float><<<grid, 128, 0, st>>>((const float*)K, (const float*)V, idx_r,
-                                               (float*)K_ret, (float*)V_ret, L, B, cap,
-                                               row_elems, rows_per_cta);
-  return cudaGetLastError();
+  return launch_gather(c, batch, L, B, idx_r, B, K, V, K_ret, V_ret, cap, st);
 }
 
 }  // namespace imem

@@ -84,6 +84,15 @@ class IndexMemLayer:
             self._ws_key = key
         return self._ws
 
+    def workspace_evict(self, batch: int, L: int, B: int, chunk: int, device) -> torch.Tensor:
+        """Workspace for pre-eviction (also serves decode)."""
+        key = ("evict", batch, L, B, chunk)
+        if self._ws is None or self._ws_key != key:
+            n = B_.workspace_size_evict(self.ctx, batch, L, B, chunk)
+            self._ws = torch.zeros(n, dtype=torch.uint8, device=device)
+            self._ws_key = key
+        return self._ws
+
     def new_state(self, batch: int, L: int, B: int, cap: int, device) -> PrefillState:
         d, Hkv, r = self.dims["head_dim"], self.dims["n_kv_heads"], self.dims["mem_r"]
         return PrefillState(
@@ -111,6 +120,34 @@ class IndexMemLayer:
                                1 if last else 0, st.idx_retained,
                                st.idx_evicted if B < L else None, st.K_ret, st.V_ret,
                                st.K_ret.shape[1], ws, stream)
+
+    def prefill_evict(self, X, Q, K, V, st: PrefillState, B: int, chunk: int,
+                      mem_chunk: int = 512, stream=None, record: bool = False):
+        """Chunked prefill with pre-eviction after every query range of
+        ``chunk`` tokens: the cache never holds more than B tokens and the
+        evicted ones enter the memory as they leave. Fills st.idx_retained
+        (first min(B, L) entries), st.K_ret/V_ret, st.M, st.bstab.
+        record=True returns per range the candidates' importances, the
+        retained and the evicted positions (copies, for inspection)."""
+        batch, L = X.shape[0], X.shape[1]
+        ws = self.workspace_evict(batch, L, B, chunk, X.device)
+        ev = torch.empty(batch * chunk, dtype=torch.int32, device=X.device)
+        cand = (torch.empty(batch, B + chunk, dtype=torch.float32, device=X.device)
+                if record else None)
+        recs = []
+        for q0 in range(0, L, chunk):
+            q1 = min(L, q0 + chunk)
+            B_.prefill_evict_chunk(self.ctx, batch, L, B, chunk, X, Q, K, V, q0, q1,
+                                   st.idx_retained, ev, cand, st.M, st.bstab, mem_chunk,
+                                   q1 == L, st.K_ret, st.V_ret, st.K_ret.shape[1], ws, stream)
+            if record:
+                n = min(B, q0) + (q1 - q0)
+                n_ev = max(0, n - B)
+                recs.append({"range": (q0, q1), "I": cand[:, :n].clone(),
+                             "retained": st.idx_retained[:, :min(B, q1)].clone(),
+                             "evicted": ev[:batch * n_ev].view(batch, n_ev).clone()})
+        st.cache_len.fill_(min(B, L))
+        return recs
 
     def update_memory(self, K, V, st: PrefillState, B: int, chunk: int = 512, stream=None):
         batch, L = K.shape[0], K.shape[1]
