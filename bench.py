@@ -388,6 +388,67 @@ def moment_readout(job, steps=64, reps=3):
     return res
 
 
+# ------------------------------------------------------------------ pre-eviction
+
+def pre_eviction(dev, reps=3):
+    """Chunked prefill that evicts after every query range (the cache never
+    holds more than B tokens; "IndexMem" technical summary §2.A, eviction
+    before the full prefill) next to the chunked prefill that selects once at
+    the end, on the long-context workload (c3: one sequence, L = 131072,
+    ranges of 8192, B = 13107, memory update included in both). CUDA events
+    around each whole prefill."""
+    wl = synth.WORKLOADS["c3"]
+    s = wl.shape
+    b, L, B, ch = wl.batch, wl.L, wl.budget, wl.prefill_chunk
+    w = synth.make_weights(s, wl.seed, dev)
+    inp = synth.make_layer_inputs(wl, w, wl.seed, dev)
+    ranges = [(q, min(L, q + ch)) for q in range(0, L, ch)]
+    stream = torch.cuda.Stream(dev)
+    lay_e, lay_o = IndexMemLayer.from_shape(s, w), IndexMemLayer.from_shape(s, w)
+    st_e = lay_e.new_state(b, L, B, B, dev)
+    st_o = lay_o.new_state(b, L, B, B, dev)
+    d = inp
+
+    def evict():
+        st_e.M.zero_(); st_e.bstab.zero_()
+        lay_e.prefill_evict(d["X"], d["Q"], d["K"], d["V"], st_e, B, ch, mem_chunk=wl.mem_chunk,
+                            stream=stream)
+
+    def at_end():
+        st_o.M.zero_(); st_o.bstab.zero_()
+        lay_o.score_and_evict(d["X"], d["Q"], d["K"], d["V"], st_o, B, q_ranges=ranges,
+                              stream=stream)
+        lay_o.update_memory(d["K"], d["V"], st_o, B, chunk=wl.mem_chunk, stream=stream)
+
+    res = {}
+    with torch.cuda.stream(stream):
+        for name, fn in (("pre_evict", evict), ("select_at_end", at_end)):
+            fn()
+            torch.cuda.synchronize()
+            best = None
+            for _ in range(reps):
+                a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                e.record(stream)
+                torch.cuda.synchronize()
+                t = a.elapsed_time(e)
+                best = t if best is None else min(best, t)
+            res["ms_" + name] = best
+            res["keys_per_s_" + name] = b * L / (best * 1e-3)
+    lay_e.sync(stream)
+    lay_o.sync(stream)
+    res.update({"workload": "c3: batch %d, L=%d, ranges of %d, B=%d" % (b, L, ch, B),
+                "candidate_rows_pre_evict": B + ch, "indexer_rows_select_at_end": L,
+                "retained_same_set_fraction": float(np.intersect1d(
+                    st_e.idx_retained.cpu().numpy(), st_o.idx_retained.cpu().numpy()).size) / B})
+    lay_e.close()
+    lay_o.close()
+    del inp
+    torch.cuda.empty_cache()
+    return res
+
+
 # ------------------------------------------------------------------ whole-model decode
 
 def model_decode(dev, peak_gbs, steps=8, reps=3):
@@ -584,6 +645,8 @@ def main():
                     help="skip the 36-layer decode measurement")
     ap.add_argument("--no-moment", action="store_true",
                     help="skip the MomentKV readout measurement")
+    ap.add_argument("--no-pre-eviction", action="store_true",
+                    help="skip the pre-eviction (long-context chunked prefill) measurement")
     a = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -701,6 +764,9 @@ def main():
     moment = None
     if not a.no_moment:
         moment = moment_readout(job)
+    pre_ev = None
+    if not a.no_pre_eviction:
+        pre_ev = pre_eviction(dev)
     model_dec = None
     if not a.no_model_decode:
         model_dec = model_decode(dev, peak)
@@ -729,6 +795,7 @@ def main():
             "cpu_baseline": cpu,
             "full_cache_decode": full_cmp,
             "moment_readout": moment,
+            "pre_eviction": pre_ev,
             "model_decode": model_dec,
             "gpu_launches": job.launches_per_step() * a.steps,
             "device_errors": not layer_sync_ok,

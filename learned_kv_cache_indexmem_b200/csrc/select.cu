@@ -9,8 +9,11 @@
 // Selection: R = the B largest importances, ties to the lower position, with
 // -0 and +0 equal. Each importance is mapped to an unsigned key that orders
 // like the float; a 4-pass 8-bit radix select finds the B-th largest key T and
-// how many keys equal to T are taken (the lowest positions). One ordered pass
-// then writes R and its complement E, both ascending.
+// how many keys equal to T are taken (the lowest positions), one CTA per
+// sequence with eight loads in flight per thread. Then every warp
+// counts the keys above and equal to T in its contiguous slice of positions,
+// one scan over the warps gives each slice's offsets, and a second walk writes
+// R and its complement E, both ascending.
 //
 // Compaction: K_ret[:, j] = K[:, R[j]] and V_ret likewise, all KV heads at
 // once (one contiguous row of Hkv*d elements per token), 16-byte vectors.
@@ -27,6 +30,7 @@ namespace imem {
 namespace {
 
 constexpr int kSelThreads = 1024;
+constexpr int kUnroll = 8;   // keys loaded per thread before any is used
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -34,53 +38,40 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Inclusive block scan of one int per thread (1024 threads); returns the
-// inclusive prefix and writes the block total to *total.
-__device__ __forceinline__ int block_inclusive_scan(int v, int* s_warp, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int n = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += n;
-  }
-  if (lane == 31) s_warp[warp] = v;
-  __syncthreads();
-  if (warp == 0) {
-    int w = s_warp[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += n;
-    }
-    s_warp[lane] = w;
-  }
-  __syncthreads();
-  const int res = v + (warp > 0 ? s_warp[warp - 1] : 0);
-  *total = s_warp[31];
-  __syncthreads();
-  return res;
-}
-
 __global__ void __launch_bounds__(kSelThreads)
 select_kernel(const float* __restrict__ I, int L, int stride, int B, int32_t* __restrict__ idx_r,
               int32_t* __restrict__ idx_e) {
+  constexpr int kWarps = kSelThreads / 32;
   const int bi = blockIdx.x;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* Ib = I + (size_t)bi * stride;
-  __shared__ int s_hist[256];
-  __shared__ int s_warp[32];
+  __shared__ int s_tot[256];            // digit histogram of the current pass
+  __shared__ int s_cnt[2][kWarps];      // per warp: keys above T, keys equal to T
+  __shared__ int s_base[2][kWarps];     // per warp: takes before it, equal keys before it
   __shared__ uint32_t s_prefix, s_mask;
   __shared__ int s_k;
 
   if (tid == 0) { s_prefix = 0; s_mask = 0; s_k = B; }
-  __syncthreads();
+  // radix select of the B-th largest key, 8 bits a pass from the top
   for (int shift = 24; shift >= 0; shift -= 8) {
-    if (tid < 256) s_hist[tid] = 0;
+    if (tid < 256) s_tot[tid] = 0;
     __syncthreads();
     const uint32_t prefix = s_prefix, mask = s_mask;
-    for (int t = tid; t < L; t += kSelThreads) {
-      const uint32_t key = order_key(Ib[t]);
-      if ((key & mask) == prefix) atomicAdd(&s_hist[(key >> shift) & 0xffu], 1);
+    // kUnroll loads in flight per thread before any is used (one CTA streams
+    // the whole row: latency, not bandwidth, is what limits it)
+    for (int t0 = 0; t0 < L; t0 += kSelThreads * kUnroll) {
+      float v[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int t = t0 + u * kSelThreads + tid;
+        v[u] = t < L ? Ib[t] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const uint32_t key = order_key(v[u]);
+        if (t0 + u * kSelThreads + tid < L && (key & mask) == prefix)
+          atomicAdd(&s_tot[(key >> shift) & 0xffu], 1);
+      }
     }
     __syncthreads();
     if (tid < 32) {
@@ -90,7 +81,7 @@ select_kernel(const float* __restrict__ I, int L, int stride, int B, int32_t* __
       int local[8];
       int sum = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) { local[i] = s_hist[255 - (tid * 8 + i)]; sum += local[i]; }
+      for (int i = 0; i < 8; ++i) { local[i] = s_tot[255 - (tid * 8 + i)]; sum += local[i]; }
       int incl = sum;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -117,24 +108,73 @@ select_kernel(const float* __restrict__ I, int L, int stride, int B, int32_t* __
   const uint32_t T = s_prefix;   // the B-th largest key
   const int take_eq = s_k;       // keys equal to T to retain (lowest positions)
 
-  int eq_carry = 0, take_carry = 0;
-  for (int t0 = 0; t0 < L; t0 += kSelThreads) {
-    const int t = t0 + tid;
-    uint32_t key = 0;
-    const bool in = t < L;
-    if (in) key = order_key(Ib[t]);
-    const int is_eq = (in && key == T) ? 1 : 0;
-    int tot;
-    const int eq_incl = block_inclusive_scan(is_eq, s_warp, &tot);
-    const int eq_rank = eq_carry + eq_incl - is_eq;
-    eq_carry += tot;
-    const int take = in && (key > T || (is_eq && eq_rank < take_eq)) ? 1 : 0;
-    const int take_incl = block_inclusive_scan(take, s_warp, &tot);
-    const int before = take_carry + take_incl - take;
-    take_carry += tot;
-    if (in) {
-      if (take) idx_r[(size_t)bi * B + before] = t;
-      else idx_e[(size_t)bi * (L - B) + (t - before)] = t;
+  // ordered output: warp w owns the contiguous positions [w seg, (w+1) seg)
+  const int seg = ((L + kWarps - 1) / kWarps + 31) & ~31;
+  const int w0 = min(L, warp * seg), w1 = min(L, w0 + seg);
+  int gt = 0, eq = 0;
+  for (int t0 = w0; t0 < w1; t0 += 32 * kUnroll) {
+    float v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int t = t0 + u * 32 + lane;
+      v[u] = t < w1 ? Ib[t] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const bool in = t0 + u * 32 + lane < w1;
+      const uint32_t key = order_key(v[u]);
+      gt += __popc(__ballot_sync(0xffffffffu, in && key > T));
+      eq += __popc(__ballot_sync(0xffffffffu, in && key == T));
+    }
+  }
+  if (lane == 0) { s_cnt[0][warp] = gt; s_cnt[1][warp] = eq; }
+  __syncthreads();
+  if (warp == 0) {
+    // equal keys before each warp, then each warp's takes and their prefix
+    const int e = s_cnt[1][lane];
+    int e_incl = e;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, e_incl, o);
+      if (lane >= o) e_incl += n;
+    }
+    const int e_base = e_incl - e;
+    const int takes = s_cnt[0][lane] + max(0, min(e, take_eq - e_base));
+    int t_incl = takes;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, t_incl, o);
+      if (lane >= o) t_incl += n;
+    }
+    s_base[0][lane] = t_incl - takes;
+    s_base[1][lane] = e_base;
+  }
+  __syncthreads();
+  int before = s_base[0][warp], eq_seen = s_base[1][warp];
+  const unsigned lt = (1u << lane) - 1u;
+  for (int t0 = w0; t0 < w1; t0 += 32 * kUnroll) {
+    float v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int t = t0 + u * 32 + lane;
+      v[u] = t < w1 ? Ib[t] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int t = t0 + u * 32 + lane;
+      const bool in = t < w1;
+      const uint32_t key = order_key(v[u]);
+      const bool is_eq = in && key == T;
+      const unsigned eqb = __ballot_sync(0xffffffffu, is_eq);
+      const bool take = in && (key > T || (is_eq && eq_seen + __popc(eqb & lt) < take_eq));
+      const unsigned tb = __ballot_sync(0xffffffffu, take);
+      const int my = before + __popc(tb & lt);
+      if (in) {
+        if (take) idx_r[(size_t)bi * B + my] = t;
+        else idx_e[(size_t)bi * (L - B) + (t - my)] = t;
+      }
+      before += __popc(tb);
+      eq_seen += __popc(eqb);
     }
   }
 }
