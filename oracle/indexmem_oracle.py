@@ -327,6 +327,65 @@ def prefill_streaming(X, Q, K, V, W_iq, W_ik, w_ig, W_phi, lam: float, B: int, r
     return {"R": np.stack(R), "M": M, "b": bs, "chunks": chunks}
 
 
+def decode_step_online(x_new, q, k_new, v_new, K_R, V_R, khat_R, I_R, pos_R, next_pos, M, bstab,
+                       W_iq, W_ik, w_ig, W_phi, w_gate, lam: float):
+    """One decode step with online eviction at a fixed budget ([IM-sum] §2.B:
+    the memory is updated online during inference as tokens leave the cache;
+    §2.A: the indexer scores keys for the queries that arrive).
+
+    The cache holds B = K_R.shape[1] - 1 tokens in slots [0, B) (any order):
+    keys/values K_R, V_R [b, B+1, Hkv, d] (slot B free), indexer keys khat_R
+    [b, B+1, dI], importances I_R [b, B+1], positions pos_R [b, B+1].
+    x_new [b, H] is the new token's hidden state, q [b, Hq, d] its query,
+    k_new, v_new [b, Hkv, d]; next_pos [b] its position.
+
+      1. o = decode_step over slots [0, B) + the new token (memory before
+         this step's eviction);
+      2. the new token's indexer query q~ and key k^ (indexer_features of the
+         token); I_t <- max(I_t, q~ . k^_t) for the cached tokens, and the new
+         token's importance is its own score q~ . k^_new;
+      3. the least important of the B + 1 leaves (ties: the higher position
+         leaves, so that ties keep lower positions); M <- lam M + phi(k) v^T,
+         b <- lam b + phi(k) with its key and value;
+      4. the new token takes the freed slot (nothing moves if it left itself).
+
+    Returns (o, evicted position [b], new state dict with K_R, V_R, khat_R,
+    I_R, pos_R, M, b) -- float64 copies."""
+    x_new, q = f64(x_new), f64(q)
+    k_new, v_new = f64(k_new), f64(v_new)
+    KR, VR = f64(K_R).copy(), f64(V_R).copy()
+    khR, IR = f64(khat_R).copy(), f64(I_R).copy()
+    posR = np.asarray(pos_R).astype(np.int64).copy()
+    M, bs = f64(M).copy(), f64(bstab).copy()
+    W_phi = f64(W_phi)
+    b = q.shape[0]
+    B = KR.shape[1] - 1
+    o, _, _, _, _ = decode_step(q, k_new, v_new, KR[:, :B], VR[:, :B], np.full(b, B), M, bs,
+                                W_phi, w_gate)
+    qhat, khat, gate = indexer_features(x_new[:, None], q[:, None], W_iq, W_ik, w_ig)
+    dI = khat.shape[-1]
+    q_t = np.einsum("bh,bhd->bd", gate[:, 0], qhat[:, 0]) / math.sqrt(dI)   # q~ [b, dI]
+    evicted = np.zeros(b, dtype=np.int64)
+    for bi in range(b):
+        IR[bi, :B] = np.maximum(IR[bi, :B], khR[bi, :B] @ q_t[bi])
+        khR[bi, B] = khat[bi, 0]
+        IR[bi, B] = khat[bi, 0] @ q_t[bi]
+        KR[bi, B], VR[bi, B] = k_new[bi], v_new[bi]
+        posR[bi, B] = int(next_pos[bi])
+        # lowest importance leaves; among equal ones the highest position
+        e = min(range(B + 1), key=lambda j: (IR[bi, j] + 0.0, -posR[bi, j]))
+        evicted[bi] = posR[bi, e]
+        k, v = KR[bi, e], VR[bi, e]                      # [Hkv, d]
+        phi = k @ W_phi.T                                # [Hkv, r]
+        M[bi] = lam * M[bi] + phi[:, :, None] * v[:, None, :]
+        bs[bi] = lam * bs[bi] + phi
+        if e != B:
+            for arr in (KR, VR, khR, IR, posR):
+                arr[bi, e] = arr[bi, B]
+    state = {"K_R": KR, "V_R": VR, "khat_R": khR, "I_R": IR, "pos_R": posR, "M": M, "b": bs}
+    return o, evicted, state
+
+
 def importance_at_keys(X, Q, W_iq, W_ik, w_ig, keys, q_end: Optional[int] = None,
                        s_block: int = 4096) -> np.ndarray:
     """Pooled importance I[t] = max_{s in [t, q_end)} A[s,t] for a few keys t of
