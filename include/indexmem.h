@@ -283,6 +283,47 @@ imem_status imem_prefill_evict_chunk(imem_ctx* ctx, int batch, int L, int B, int
                                      int mem_chunk, int finalize, void* K_ret, void* V_ret,
                                      int cap, void* workspace, void* stream);
 
+/* Decode-time online eviction at a fixed budget ([IM-sum] §2.B: the memory
+ * is updated online during inference as tokens leave the cache; §2.A: a key's
+ * importance is the running maximum of its indexer scores over the queries
+ * that arrive). The cache keeps B tokens in slots [0, B), in any order, with
+ * per slot the indexer key khat_ret [batch, cap, 64] (bf16, d_I features then
+ * zeros), the importance I_ret [batch, cap] (fp32) and the position pos_ret
+ * [batch, cap] (int32); next_pos [batch] (int32) is the next token's position.
+ * cap >= B + 1 (slot B is the step's scratch).
+ *
+ * imem_online_init: the state after a one-shot prefill (imem_score_and_evict
+ * with finalize = 1, the same workspace, batch and L): khat_ret, I_ret,
+ * pos_ret of the retained tokens (in idx_retained order, i.e. ascending
+ * positions) and next_pos = L. running_max and idx_retained as left by that
+ * call. Errors: INVALID_ARG, SHAPE (B > L, cap < B + 1), ALIGN, CUDA,
+ * UNSUPPORTED (moment readout).
+ *
+ * imem_decode_online: one decode step. x_new [batch, H] is the new token's
+ * hidden state, q, k_new, v_new as imem_decode; cache_len must be B on entry.
+ *   1. out = imem_decode's output over slots [0, B) + the new token, with M,
+ *      bstab before this step's eviction (the new token goes to slot B);
+ *   2. the new token's indexer query q~ and key k^ are formed as in prefill
+ *      (per-head projection of q, RMS norms, gates from x_new; both rounded to
+ *      bf16); I_t = max(I_t, q~ . k^_t) for the cached tokens; the new token's
+ *      importance is q~ . k^_new;
+ *   3. the least important of the B + 1 tokens leaves (ties: the higher
+ *      position leaves); M <- lambda M + phi(k) v^T, bstab <- lambda bstab +
+ *      phi(k) with its key and value (every KV head); evicted [batch] (int32,
+ *      out) receives its position;
+ *   4. the new token takes the freed slot (nothing moves if it left itself);
+ *      cache_len returns to B; next_pos advances.
+ * Errors: as imem_decode; UNSUPPORTED for the moment readout. */
+imem_status imem_online_init(imem_ctx* ctx, int batch, int L, int B, const float* running_max,
+                             const int32_t* idx_retained, const void* workspace, void* khat_ret,
+                             float* I_ret, int32_t* pos_ret, int32_t* next_pos, int cap,
+                             void* stream);
+imem_status imem_decode_online(imem_ctx* ctx, int batch, int B, const void* x_new, const void* q,
+                               const void* k_new, const void* v_new, void* K_ret, void* V_ret,
+                               void* khat_ret, float* I_ret, int32_t* pos_ret, int32_t* next_pos,
+                               int32_t* cache_len, int cap, float* M, float* bstab, void* out,
+                               int32_t* evicted, void* workspace, void* stream);
+
 /* Waits for the stream, then reports the first error the device recorded for
  * this context since the last imem_sync (TIMEOUT for a bounded wait that ran
  * out, SHAPE for a decode into a full cache) or a CUDA error, and clears it. */

@@ -78,6 +78,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.imem_prefill_evict_chunk.restype = i
     lib.imem_prefill_evict_chunk.argtypes = [vp, i, i, i, i, vp, vp, vp, vp, i, i, vp, vp, vp,
                                              vp, vp, i, i, vp, vp, i, vp, vp]
+    lib.imem_online_init.restype = i
+    lib.imem_online_init.argtypes = [vp, i, i, i, vp, vp, vp, vp, vp, vp, vp, i, vp]
+    lib.imem_decode_online.restype = i
+    lib.imem_decode_online.argtypes = [vp, i, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i,
+                                       vp, vp, vp, vp, vp, vp]
     lib.imem_update_moments.restype = i
     lib.imem_update_moments.argtypes = [vp, i, i, vp, vp, vp, i, i, vp, vp, vp, vp, vp, vp]
     lib.imem_decode_moment.restype = i
@@ -179,6 +184,22 @@ def prefill_evict_chunk(ctx, batch, L, B, chunk_max, X, Q, K, V, q_begin, q_end,
         _ptr(retained), _ptr(evicted), _ptr(cand_importance), _ptr(M), _ptr(bstab), mem_chunk,
         int(finalize), _ptr(K_ret), _ptr(V_ret), cap, _ptr(workspace), _stream(stream)),
         "imem_prefill_evict_chunk")
+
+
+def online_init(ctx, batch, L, B, running_max, idx_retained, workspace, khat_ret, I_ret, pos_ret,
+                next_pos, cap, stream=None):
+    _check(load().imem_online_init(
+        ctx, batch, L, B, _ptr(running_max), _ptr(idx_retained), _ptr(workspace), _ptr(khat_ret),
+        _ptr(I_ret), _ptr(pos_ret), _ptr(next_pos), cap, _stream(stream)), "imem_online_init")
+
+
+def decode_online(ctx, batch, B, x_new, q, k_new, v_new, K_ret, V_ret, khat_ret, I_ret, pos_ret,
+                  next_pos, cache_len, cap, M, bstab, out, evicted, workspace, stream=None):
+    _check(load().imem_decode_online(
+        ctx, batch, B, _ptr(x_new), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(K_ret), _ptr(V_ret),
+        _ptr(khat_ret), _ptr(I_ret), _ptr(pos_ret), _ptr(next_pos), _ptr(cache_len), cap, _ptr(M),
+        _ptr(bstab), _ptr(out), _ptr(evicted), _ptr(workspace), _stream(stream)),
+        "imem_decode_online")
 
 
 def update_moments(ctx, batch, L, K, V, idx_evicted, n_evicted, chunk, S_T, s_k, s_v, n_e,

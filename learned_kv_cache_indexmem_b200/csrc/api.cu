@@ -32,6 +32,18 @@ Workspace workspace_layout(const Ctx& c, int batch, int L) {
   const size_t units = (size_t)batch * c.cfg.n_kv_heads;
   w.dec_cnt_off = off;                        // one counter per sequence
   off = align_up(off + (size_t)batch * sizeof(int), 256);
+  // online eviction: the new token's feature partials, the score CTAs'
+  // candidates (16 bytes each), a counter and the chosen slot per sequence
+  w.on_qpart_off = off;
+  off = align_up(off + (size_t)batch * c.cfg.n_q_heads * c.cfg.idx_dim * sizeof(float), 256);
+  w.on_kpart_off = off;
+  off = align_up(off + (size_t)batch * c.cfg.idx_dim * sizeof(float), 256);
+  w.on_cand_off = off;
+  off = align_up(off + (size_t)batch * kOnlineMaxCtas * 16, 256);
+  w.on_cnt_off = off;
+  off = align_up(off + (size_t)batch * sizeof(int), 256);
+  w.on_slot_off = off;
+  off = align_up(off + (size_t)batch * sizeof(int), 256);
   w.dec_part_off = off;                       // (unused: decode merges in shared memory)
   // memory partials: at most (2*148 + units) runs of a d x (d+1) sum [S | s]
   w.mem_part_off = off;
@@ -466,6 +478,64 @@ imem_status imem_prefill_evict_chunk(imem_ctx* h, int batch, int L, int B, int c
     IMEM_CHECK(cuda_status(imem::launch_gather(c, batch, L, B < L ? B : L, retained, B, K, V,
                                                K_ret, V_ret, cap, st)));
   return IMEM_OK;
+}
+
+imem_status imem_online_init(imem_ctx* h, int batch, int L, int B, const float* running_max,
+                             const int32_t* idx_retained, const void* workspace, void* khat_ret,
+                             float* I_ret, int32_t* pos_ret, int32_t* next_pos, int cap,
+                             void* stream) {
+  if (!h) return IMEM_ERR_INVALID_ARG;
+  const Ctx& c = h->c;
+  if (c.cfg.readout != IMEM_READOUT_GATED) return IMEM_ERR_UNSUPPORTED;
+  if (batch < 1 || L < 1 || B < 1 || B > L || cap < B + 1) return IMEM_ERR_SHAPE;
+  IMEM_CHECK(check_ptr(running_max));
+  IMEM_CHECK(check_ptr(idx_retained));
+  IMEM_CHECK(check_ptr(workspace));
+  IMEM_CHECK(check_ptr(khat_ret));
+  IMEM_CHECK(check_ptr(I_ret));
+  IMEM_CHECK(check_ptr(pos_ret));
+  IMEM_CHECK(check_ptr(next_pos));
+  IMEM_CHECK(check_device(c));
+  const imem::Workspace ws = imem::workspace_layout(c, batch, L);
+  const __nv_bfloat16* kh = (const __nv_bfloat16*)((const char*)workspace + ws.kh_off);
+  return cuda_status(imem::launch_online_init(c, batch, L, B, cap, running_max, idx_retained, kh,
+                                              (__nv_bfloat16*)khat_ret, I_ret, pos_ret, next_pos,
+                                              (cudaStream_t)stream));
+}
+
+imem_status imem_decode_online(imem_ctx* h, int batch, int B, const void* x_new, const void* q,
+                               const void* k_new, const void* v_new, void* K_ret, void* V_ret,
+                               void* khat_ret, float* I_ret, int32_t* pos_ret, int32_t* next_pos,
+                               int32_t* cache_len, int cap, float* M, float* bstab, void* out,
+                               int32_t* evicted, void* workspace, void* stream) {
+  if (!h) return IMEM_ERR_INVALID_ARG;
+  const Ctx& c = h->c;
+  if (c.cfg.readout != IMEM_READOUT_GATED) return IMEM_ERR_UNSUPPORTED;
+  if (batch < 1 || B < 1 || cap < B + 1) return IMEM_ERR_SHAPE;
+  IMEM_CHECK(check_ptr(x_new));
+  IMEM_CHECK(check_ptr(khat_ret));
+  IMEM_CHECK(check_ptr(I_ret));
+  IMEM_CHECK(check_ptr(pos_ret));
+  IMEM_CHECK(check_ptr(next_pos));
+  IMEM_CHECK(check_ptr(evicted));
+  // the attention step with the memory before this step's eviction (it
+  // validates the remaining arguments and appends the new token at slot B)
+  cudaStream_t st = (cudaStream_t)stream;
+  IMEM_CHECK(check_ptr(workspace));
+  const imem::Workspace ws = imem::workspace_layout(c, batch, 1);
+  char* wsb = (char*)workspace;
+  float* qpart = (float*)(wsb + ws.on_qpart_off);
+  float* kpart = (float*)(wsb + ws.on_kpart_off);
+  IMEM_CHECK(check_ptr(q));
+  IMEM_CHECK(check_device(c));
+  IMEM_CHECK(cuda_status(imem::launch_online_features(c, batch, x_new, q, qpart, kpart, st)));
+  IMEM_CHECK(decode_common(h, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab,
+                           nullptr, nullptr, out, workspace, stream));
+  return cuda_status(imem::launch_online_evict(c, batch, B, cap, qpart, kpart, khat_ret, I_ret,
+                                               pos_ret, next_pos, K_ret, V_ret, cache_len, M,
+                                               bstab, evicted, wsb + ws.on_cand_off,
+                                               (int*)(wsb + ws.on_cnt_off),
+                                               (int*)(wsb + ws.on_slot_off), st));
 }
 
 imem_status imem_sync(imem_ctx* h, void* stream) {

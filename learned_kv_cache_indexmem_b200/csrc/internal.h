@@ -44,11 +44,14 @@ bool make_tmap_bf16(const Ctx& c, CUtensorMap* map, const void* base, uint64_t w
                     uint64_t rows, uint32_t box_rows);
 
 // Layout of the caller's workspace for (batch, L).
+constexpr int kOnlineMaxCtas = 64;   // score CTAs per sequence in online eviction (max)
+
 struct Workspace {
   size_t qt_off, kh_off;        // indexer q~ and k^ (bf16 [b, L, kIdxPad])
   size_t sel_off;               // selection scratch
   size_t dec_part_off;          // decode split partials
   size_t dec_cnt_off;           // decode counters (int), zero between calls
+  size_t on_qpart_off, on_kpart_off, on_cand_off, on_cnt_off, on_slot_off;   // online eviction
   size_t mem_part_off;          // memory-update partials
   size_t sv_part_off;           // value-sum partials of the moment statistics
   size_t total;
@@ -103,6 +106,20 @@ cudaError_t launch_evict_chunk(const Ctx& c, int batch, int B, int Lc, int n_R, 
 // Appends positions q0..q0+C-1 at rows [n_R, n_R + C) of `retained` (stride B).
 cudaError_t launch_append_positions(int batch, int B, int n_R, int q0, int C, int32_t* retained,
                                     cudaStream_t st);
+// Decode-time online eviction (online.cu).
+int online_score_ctas(int B);
+cudaError_t launch_online_init(const Ctx& c, int batch, int L, int B, int cap,
+                               const float* running_max, const int32_t* idx_r,
+                               const __nv_bfloat16* kh, __nv_bfloat16* khat_ret, float* I_ret,
+                               int32_t* pos_ret, int32_t* next_pos, cudaStream_t st);
+cudaError_t launch_online_features(const Ctx& c, int batch, const void* x, const void* q,
+                                   float* qpart, float* kpart, cudaStream_t st);
+cudaError_t launch_online_evict(const Ctx& c, int batch, int B, int cap, const float* qpart,
+                                const float* kpart, void* khat_ret, float* I_ret, int32_t* pos_ret,
+                                int32_t* next_pos, void* K_ret, void* V_ret, int32_t* cache_len,
+                                float* M, float* bstab, int32_t* evicted, void* cand,
+                                int* counter, int* evict_slot, cudaStream_t st);
+
 // K_ret/V_ret[:, :n] = K/V[idx[:, :n]] (idx stride `idx_stride`).
 cudaError_t launch_gather(const Ctx& c, int batch, int L, int n, const int32_t* idx,
                           int idx_stride, const void* K, const void* V, void* K_ret, void* V_ret,

@@ -27,6 +27,18 @@ class PrefillState:
     n_e: Optional[torch.Tensor] = None   # [b] fp32, moment readout only
 
 
+@dataclasses.dataclass
+class OnlineState:
+    """Decode-time online eviction: per cache slot the indexer key, the
+    importance and the position; the next token's position; the position
+    evicted by the last step."""
+    khat_ret: torch.Tensor        # [b, cap, 64] bf16
+    I_ret: torch.Tensor           # [b, cap] fp32
+    pos_ret: torch.Tensor         # [b, cap] int32
+    next_pos: torch.Tensor        # [b] int32
+    evicted: torch.Tensor         # [b] int32
+
+
 class IndexMemLayer:
     """Context for one layer. ``weights`` holds device tensors W_iq [Hq,d,dI],
     W_ik [H,dI], w_ig [H,Hq] (model dtype), W_phi [r,d], w_gate [Hq,d] (fp32).
@@ -174,6 +186,34 @@ class IndexMemLayer:
         else:
             B_.decode(self.ctx, batch, q, k_new, v_new, st.K_ret, st.V_ret, st.cache_len,
                       st.K_ret.shape[1], st.M, st.bstab, out, self._ws, stream)
+        return out
+
+    def online_init(self, st: PrefillState, B: int, L: int, stream=None) -> OnlineState:
+        """State for decode-time online eviction after a one-shot prefill of L
+        tokens into st (same layer, same workspace); the cache has B tokens."""
+        batch, cap = st.K_ret.shape[0], st.K_ret.shape[1]
+        dev = st.K_ret.device
+        on = OnlineState(
+            khat_ret=torch.zeros(batch, cap, 64, dtype=torch.bfloat16, device=dev),
+            I_ret=torch.zeros(batch, cap, dtype=torch.float32, device=dev),
+            pos_ret=torch.zeros(batch, cap, dtype=torch.int32, device=dev),
+            next_pos=torch.zeros(batch, dtype=torch.int32, device=dev),
+            evicted=torch.zeros(batch, dtype=torch.int32, device=dev))
+        B_.online_init(self.ctx, batch, L, B, st.running_max, st.idx_retained, self._ws,
+                       on.khat_ret, on.I_ret, on.pos_ret, on.next_pos, cap, stream)
+        return on
+
+    def decode_online(self, x_new, q, k_new, v_new, st: PrefillState, on: OnlineState, B: int,
+                      out=None, stream=None):
+        """One decode step that keeps the cache at B tokens: the least
+        important of the B + 1 leaves into the memory (on.evicted: its
+        position)."""
+        batch = q.shape[0]
+        if out is None:
+            out = torch.empty_like(q)
+        B_.decode_online(self.ctx, batch, B, x_new, q, k_new, v_new, st.K_ret, st.V_ret,
+                         on.khat_ret, on.I_ret, on.pos_ret, on.next_pos, st.cache_len,
+                         st.K_ret.shape[1], st.M, st.bstab, out, on.evicted, self._ws, stream)
         return out
 
     def sync(self, stream=None):

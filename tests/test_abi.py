@@ -88,6 +88,9 @@ def test_null_context_is_invalid_for_every_call():
     assert lib.imem_workspace_size_evict(None, 1, 16, 4, 8, ctypes.byref(n2)) == 1
     assert lib.imem_prefill_evict_chunk(None, 1, 16, 4, 8, 16, 16, 16, 16, 0, 8, 16, 16, None, 16,
                                         16, 64, 0, None, None, 8, 16, None) == 1
+    assert lib.imem_online_init(None, 1, 16, 4, 16, 16, 16, 16, 16, 16, 16, 8, None) == 1
+    assert lib.imem_decode_online(None, 1, 4, 16, 16, 16, 16, 16, 16, 16, 16, 16, 16, 16, 8, 16,
+                                  16, 16, 16, 16, None) == 1
     assert lib.imem_update_moments(None, 1, 16, 16, 16, 16, 4, 64, 16, 16, 16, 16, 16, None) == 1
     assert lib.imem_decode_moment(None, 1, 16, 16, 16, 16, 16, 16, 8, 16, 16, 16, 16, 16, 16,
                                   None) == 1

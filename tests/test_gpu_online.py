@@ -1,0 +1,92 @@
+"""Decode-time online eviction ("IndexMem" technical summary §2.B, memory
+updated online during inference; §2.A, pooled importance) through the C ABI
+against the oracle, step by step from the GPU's own state before each step:
+the output, the importances carried, the evicted token (the oracle's choice
+or a near-tie within the score tolerance), the memory updated with it, and
+the cache rows after the move."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from learned_kv_cache_indexmem_b200 import synth
+from oracle import indexmem_oracle as om
+
+from .parity import SCORE_TOL, Case, check_decode, check_memory, ill_conditioned, to_np
+
+pytestmark = pytest.mark.gpu
+W = synth.WORKLOADS
+
+
+@pytest.mark.parametrize("name,L,B,steps,batch", [
+    ("c0", 512, 64, 12, 1),
+    ("c1", 1024, 128, 20, 2),
+    ("c1", 600, 300, 8, 1),      # several score CTAs per sequence
+])
+def test_online_eviction_parity(cuda_device, name, L, B, steps, batch):
+    case = Case(W[name], cuda_device, L=L + steps, batch=batch, n_decode=1)
+    s = case.shape
+    lay = case.layer()
+    cap = B + 1
+    st = lay.new_state(batch, L, B, cap, cuda_device)
+    d = {k: v[:, :L].contiguous() for k, v in case.in_dev.items()}
+    lay.score_and_evict(d["X"], d["Q"], d["K"], d["V"], st, B)
+    lay.update_memory(d["K"], d["V"], st, B, chunk=64)
+    on = lay.online_init(st, B, L)
+    lay.sync()
+    assert np.array_equal(to_np(on.pos_ret[:, :B]), to_np(st.idx_retained))
+    assert np.all(to_np(on.next_pos) == L)
+    w = case.w_cpu
+    W_phi = w["W_phi"].numpy().astype(np.float64)
+    group = s.n_q_heads // s.n_kv_heads
+    K_all, V_all = to_np(case.in_cpu["K"]), to_np(case.in_cpu["V"])
+    for i in range(steps):
+        t = L + i
+        pre = {"K": to_np(st.K_ret), "V": to_np(st.V_ret), "kh": to_np(on.khat_ret),
+               "I": to_np(on.I_ret), "pos": to_np(on.pos_ret).astype(np.int64),
+               "M": to_np(st.M), "b": to_np(st.bstab)}
+        x, q, kn, vn = (case.in_dev[k][:, t].contiguous() for k in ("X", "Q", "K", "V"))
+        out = lay.decode_online(x, q, kn, vn, st, on, B)
+        lay.sync()
+        xc, qc, knc, vnc = (to_np(case.in_cpu[k][:, t]) for k in ("X", "Q", "K", "V"))
+        o_ref, ev_ref, new = om.decode_step_online(
+            xc, qc, knc, vnc, pre["K"], pre["V"], pre["kh"][..., :s.idx_dim], pre["I"],
+            pre["pos"], np.full(batch, t), pre["M"], pre["b"], w["W_iq"], w["W_ik"], w["w_ig"],
+            W_phi, w["w_gate"], s.lam)
+        what = "%s step %d" % (name, i)
+        check_decode(to_np(out), o_ref, ill_conditioned(pre["b"], qc, W_phi, group), what)
+        ev = to_np(on.evicted).astype(np.int64)
+        pos_after = to_np(on.pos_ret).astype(np.int64)
+        I_after = to_np(on.I_ret)
+        # the oracle's importances of the B + 1 candidates from the GPU's state
+        qh, kh_new, g = om.indexer_features(xc[:, None], qc[:, None], w["W_iq"], w["W_ik"],
+                                            w["w_ig"])
+        qt = np.einsum("bh,bhd->bd", g[:, 0], qh[:, 0]) / math.sqrt(s.idx_dim)
+        for bi in range(batch):
+            cand_pos = list(pre["pos"][bi, :B]) + [t]
+            I_cand = np.concatenate([
+                np.maximum(pre["I"][bi, :B], pre["kh"][bi, :B, :s.idx_dim] @ qt[bi]),
+                [kh_new[bi, 0] @ qt[bi]]])
+            scale = max(np.abs(I_cand).max(), math.sqrt(np.mean(I_cand ** 2)))
+            # the evicted token is the least important (a near-tie may differ)
+            j_gpu = cand_pos.index(ev[bi])
+            assert I_cand[j_gpu] <= I_cand.min() + SCORE_TOL * scale, "%s: eviction" % what
+            if ev[bi] != ev_ref[bi]:
+                j_ref = cand_pos.index(ev_ref[bi])
+                assert abs(I_cand[j_gpu] - I_cand[j_ref]) <= SCORE_TOL * scale, what
+            # the cache after the move: the candidates minus the evicted one
+            assert sorted(pos_after[bi, :B]) == sorted(set(cand_pos) - {ev[bi]}), what
+            for j in range(B):
+                p = pos_after[bi, j]
+                assert np.array_equal(to_np(st.K_ret[bi, j]), K_all[bi, p]), what
+                assert np.array_equal(to_np(st.V_ret[bi, j]), V_all[bi, p]), what
+                assert abs(I_after[bi, j] - I_cand[cand_pos.index(p)]) <= SCORE_TOL * scale, what
+        # the memory: the state before the step updated with the GPU's choice
+        E = np.array([[ev[bi]] for bi in range(batch)])
+        M_ref, b_ref = om.memory_update(case.in_cpu["K"], case.in_cpu["V"], E, W_phi, s.lam,
+                                        M0=pre["M"], b0=pre["b"])
+        check_memory(to_np(st.M), to_np(st.bstab), M_ref, b_ref, what)
+        assert np.all(to_np(st.cache_len) == B)
+        assert np.all(to_np(on.next_pos) == t + 1)
+    lay.close()
