@@ -388,6 +388,53 @@ def moment_readout(job, steps=64, reps=3):
     return res
 
 
+# ------------------------------------------------------------------ online eviction
+
+def online_decode(job, steps=64, reps=3):
+    """Decode steps that keep the cache at the budget (each step's least
+    important token leaves into the memory: "IndexMem" technical summary
+    §2.B, memory updated online) next to the plain decode over the same
+    evicted cache; per step, CUDA graphs of `steps` steps."""
+    b, B, L = job.batch, job.B, job.L
+    lay = job.layer
+    st = lay.new_state(b, L, B, job.cap, job.dev)
+    for k in ("running_max", "idx_retained", "K_ret", "V_ret", "M", "bstab"):
+        getattr(st, k).copy_(getattr(job.st, k))
+    st.cache_len.fill_(B)
+    out = torch.empty_like(job.decin["q"][0])
+    res = {}
+    with torch.cuda.stream(job.stream):
+        on = lay.online_init(st, B, L, stream=job.stream)
+        dec = job.decin
+
+        def step(i):
+            lay.decode_online(dec["x"][i], dec["q"][i], dec["k_new"][i], dec["v_new"][i], st, on,
+                              B, out=out, stream=job.stream)
+        step(0)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=job.stream):
+            for i in range(steps):
+                step(i)
+        best = None
+        for _ in range(reps):
+            torch.cuda.synchronize()
+            a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(job.stream)
+            g.replay()
+            e.record(job.stream)
+            torch.cuda.synchronize()
+            t = a.elapsed_time(e) / steps * 1e3
+            best = t if best is None else min(best, t)
+        del g
+    lay.sync(job.stream)
+    res["us_per_step_online"] = best
+    res["launches_per_step_online"] = 4
+    res["steps"] = steps
+    res["cache_rows"] = B
+    return res
+
+
 # ------------------------------------------------------------------ pre-eviction
 
 def pre_eviction(dev, reps=3):
@@ -645,6 +692,8 @@ def main():
                     help="skip the 36-layer decode measurement")
     ap.add_argument("--no-moment", action="store_true",
                     help="skip the MomentKV readout measurement")
+    ap.add_argument("--no-online", action="store_true",
+                    help="skip the decode-time online eviction measurement")
     ap.add_argument("--no-pre-eviction", action="store_true",
                     help="skip the pre-eviction (long-context chunked prefill) measurement")
     a = ap.parse_args()
@@ -764,6 +813,11 @@ def main():
     moment = None
     if not a.no_moment:
         moment = moment_readout(job)
+    online = None
+    if not a.no_online:
+        online = online_decode(job)
+        if full_cmp is not None:
+            online["us_per_step_plain"] = full_cmp["us_per_step_evicted"]
     pre_ev = None
     if not a.no_pre_eviction:
         pre_ev = pre_eviction(dev)
@@ -795,6 +849,7 @@ def main():
             "cpu_baseline": cpu,
             "full_cache_decode": full_cmp,
             "moment_readout": moment,
+            "online_eviction": online,
             "pre_eviction": pre_ev,
             "model_decode": model_dec,
             "gpu_launches": job.launches_per_step() * a.steps,

@@ -31,7 +31,7 @@ namespace imem {
 namespace {
 
 constexpr int kOnThreads = 256;
-constexpr int kKSplit = 8;            // CTAs sharing the d_I key rows of a sequence
+constexpr int kKSplit = 8;            // CTAs sharing the d_I key rows of a sequence (<= 8 rows each)
 
 __device__ __forceinline__ float bf16_round(float x) {
   return __bfloat162float(__float2bfloat16_rn(x));
@@ -45,6 +45,14 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 
 template <typename T>
 __device__ __forceinline__ float ldf(const T* p) { return Elem<T>::to_f(*p); }
+
+// Programmatic dependent launch: each online kernel may start while the
+// previous kernel of the stream runs; it waits before reading anything that
+// kernel may write, and lets its own dependents start early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
 
 // block-wide sum of one float per thread (kOnThreads threads); all threads
 // receive the total
@@ -83,49 +91,88 @@ online_init_kernel(int L, int B, int cap, const float* __restrict__ running_max,
 // ---- the new token's indexer features ----------------------------------------
 // CTA h < Hq: qpart[h] = sigmoid(w_ig[:,h] . x) * rmsnorm(W_iq[h]^T q_h) / sqrt(dI)
 // CTA Hq + s: kpart[rows of slice s] = W_ik^T x
+// Every load moves 8 elements (16 bytes of bf16); H and D are multiples of 64.
 template <typename T>
 __global__ void __launch_bounds__(kOnThreads)
 online_features_kernel(const T* __restrict__ x, const T* __restrict__ q, const T* __restrict__ WcT,
                        const T* __restrict__ WqT, int H, int Hq, int D, int dI,
                        float* __restrict__ qpart, float* __restrict__ kpart) {
-  extern __shared__ float osm[];
   __shared__ float red[kOnThreads / 32];
+  __shared__ float s_red8[kOnThreads / 32][8];
   __shared__ float s_qi[64];
   const int bi = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait();
+  pdl_launch();
   const T* xb = x + (size_t)bi * H;
   if ((int)blockIdx.x < Hq) {
     const int h = blockIdx.x;
-    float* sq = osm;   // [D]
-    for (int c = tid; c < D; c += kOnThreads) sq[c] = ldf(q + ((size_t)bi * Hq + h) * D + c);
     // gate logit over the hidden state (row dI + h of WcT is w_ig[:, h])
     const T* wg = WcT + (size_t)(dI + h) * H;
     float z = 0.f;
-    for (int c = tid; c < H; c += kOnThreads) z = fmaf(ldf(wg + c), ldf(xb + c), z);
-    z = block_sum(z, red);
-    // qI_j = W_iq[h][:, j] . q_h (row h*dI + j of WqT), a warp per output
-    for (int j = warp; j < dI; j += kOnThreads / 32) {
-      const T* wr = WqT + ((size_t)h * dI + j) * D;
-      float a = 0.f;
-      for (int c = lane; c < D; c += 32) a = fmaf(ldf(wr + c), sq[c], a);
-      a = warp_sum(a);
-      if (lane == 0) s_qi[j] = a;
+    for (int c = 8 * tid; c < H; c += 8 * kOnThreads) {
+      float wf[8], xf[8];
+      load8<T>(wg + c, wf);
+      load8<T>(xb + c, xf);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) z = fmaf(wf[e], xf[e], z);
     }
+    z = block_sum(z, red);
+    // qI_j = W_iq[h][:, j] . q_h (row h*dI + j of WqT): 4 threads per row,
+    // each D/4 elements
+    const T* qh = q + ((size_t)bi * Hq + h) * D;
+    const int j = tid >> 2, part = tid & 3;
+    float a = 0.f;
+    if (j < dI) {
+      const T* wr = WqT + ((size_t)h * dI + j) * D;
+      for (int c = 8 * part; c < D; c += 32) {
+        float wf[8], qf[8];
+        load8<T>(wr + c, wf);
+        load8<T>(qh + c, qf);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) a = fmaf(wf[e], qf[e], a);
+      }
+    }
+    a += __shfl_xor_sync(0xffffffffu, a, 1);
+    a += __shfl_xor_sync(0xffffffffu, a, 2);
+    if (j < dI && part == 0) s_qi[j] = a;
     __syncthreads();
-    float ss = 0.f;
-    for (int j = tid; j < dI; j += kOnThreads) ss = fmaf(s_qi[j], s_qi[j], ss);
-    ss = block_sum(ss, red);
+    const float ss = block_sum(tid < dI ? s_qi[tid] * s_qi[tid] : 0.f, red);
     const float coef = sigmoidf_(z) * rsqrtf(ss / dI + 1e-6f) * rsqrtf((float)dI);
-    for (int j = tid; j < dI; j += kOnThreads)
-      qpart[((size_t)bi * Hq + h) * dI + j] = coef * s_qi[j];
+    for (int jj = tid; jj < dI; jj += kOnThreads)
+      qpart[((size_t)bi * Hq + h) * dI + jj] = coef * s_qi[jj];
   } else {
+    // rows [r0, r0 + nr) of W_ik^T x: every thread takes 8 hidden elements
+    // at a time for all rows of the slice
     const int s = blockIdx.x - Hq;
     const int per = (dI + kKSplit - 1) / kKSplit;
-    for (int r = s * per + warp; r < min(dI, (s + 1) * per); r += kOnThreads / 32) {
-      const T* wr = WcT + (size_t)r * H;
-      float a = 0.f;
-      for (int c = lane; c < H; c += 32) a = fmaf(ldf(wr + c), ldf(xb + c), a);
-      a = warp_sum(a);
-      if (lane == 0) kpart[(size_t)bi * dI + r] = a;
+    const int r0 = s * per, nr = min(per, dI - r0);
+    float acc[8];
+#pragma unroll
+    for (int rr = 0; rr < 8; ++rr) acc[rr] = 0.f;
+    for (int c = 8 * tid; c < H; c += 8 * kOnThreads) {
+      float xf[8];
+      load8<T>(xb + c, xf);
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        if (rr < nr) {
+          float wf[8];
+          load8<T>(WcT + (size_t)(r0 + rr) * H + c, wf);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[rr] = fmaf(wf[e], xf[e], acc[rr]);
+        }
+      }
+    }
+#pragma unroll
+    for (int rr = 0; rr < 8; ++rr) {
+      const float v = warp_sum(acc[rr]);
+      if (lane == 0) s_red8[warp][rr] = v;
+    }
+    __syncthreads();
+    if (tid < nr) {
+      float t = 0.f;
+#pragma unroll
+      for (int w = 0; w < kOnThreads / 32; ++w) t += s_red8[w][tid];
+      kpart[(size_t)bi * dI + r0 + tid] = t;
     }
   }
 }
@@ -151,15 +198,25 @@ online_score_kernel(int B, int cap, int Hq, int dI, int rows_per_cta,
   __shared__ int s_last;
   const int bi = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nct = gridDim.x;
-  // q~ (sum over heads) and the new key k^ (RMS norm), both rounded to bf16
-  float kv = 0.f;
-  if (tid < dI) {
+  pdl_wait();
+  pdl_launch();
+  // q~ (sum over heads: 4 groups of heads per feature, loads in flight
+  // together) and the new key k^ (RMS norm), both rounded to bf16
+  __shared__ float s_hsum[4][64];
+  {
+    const int j = tid & 63, grp = tid >> 6;
     float a = 0.f;
-    for (int h = 0; h < Hq; ++h) a += qpart[((size_t)bi * Hq + h) * dI + tid];
-    s_qt[tid] = bf16_round(a);
-    kv = kpart[(size_t)bi * dI + tid];
+    if (j < dI) {
+      const int h0 = grp * ((Hq + 3) / 4), h1 = min(Hq, h0 + (Hq + 3) / 4);
+#pragma unroll 8
+      for (int h = h0; h < h1; ++h) a += qpart[((size_t)bi * Hq + h) * dI + j];
+    }
+    s_hsum[grp][j] = a;
   }
-  const float ss = block_sum(tid < dI ? kv * kv : 0.f, red);
+  const float kv = tid < dI ? kpart[(size_t)bi * dI + tid] : 0.f;
+  __syncthreads();
+  if (tid < dI) s_qt[tid] = bf16_round((s_hsum[0][tid] + s_hsum[1][tid]) + (s_hsum[2][tid] + s_hsum[3][tid]));
+  const float ss = block_sum(kv * kv, red);
   if (tid < dI) s_kn[tid] = bf16_round(kv * rsqrtf(ss / dI + 1e-6f));
   for (int j = tid + dI; j < 64; j += kOnThreads) { s_qt[j] = 0.f; s_kn[j] = 0.f; }
   __syncthreads();
@@ -246,24 +303,44 @@ online_evict_kernel(int B, int cap, int Hkv, int D, int r, float lambda,
   float* sk = osm;          // [D]
   float* sv = sk + D;       // [D]
   float* sphi = sv + D;     // [r]
-  const int kh = blockIdx.x, bi = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int kh = blockIdx.x, bi = blockIdx.y, tid = threadIdx.x;
+  pdl_wait();
+  pdl_launch();
   const int e = evict_slot[bi];
   const size_t rs = (size_t)Hkv * D;
   T* ke = K_ret + ((size_t)bi * cap + e) * rs + (size_t)kh * D;
   T* ve = V_ret + ((size_t)bi * cap + e) * rs + (size_t)kh * D;
   for (int c = tid; c < D; c += kOnThreads) { sk[c] = ldf(ke + c); sv[c] = ldf(ve + c); }
   __syncthreads();
-  for (int j = warp; j < r; j += kOnThreads / 32) {
+  // phi = W_phi k: 4 threads per row, float4 loads (D/16 each, in flight together)
+  for (int j0 = 0; j0 < r; j0 += kOnThreads / 4) {
+    const int j = j0 + tid / 4, part = tid & 3;
     float a = 0.f;
-    for (int c = lane; c < D; c += 32) a = fmaf(W_phi[(size_t)j * D + c], sk[c], a);
-    a = warp_sum(a);
-    if (lane == 0) sphi[j] = a;
+    if (j < r) {
+      const float4* wr = reinterpret_cast<const float4*>(W_phi + (size_t)j * D);
+#pragma unroll 8
+      for (int c4 = part; c4 < D / 4; c4 += 4) {
+        const float4 w = __ldg(wr + c4);
+        a = fmaf(w.x, sk[4 * c4], fmaf(w.y, sk[4 * c4 + 1], fmaf(w.z, sk[4 * c4 + 2], fmaf(w.w, sk[4 * c4 + 3], a))));
+      }
+    }
+    a += __shfl_xor_sync(0xffffffffu, a, 1);
+    a += __shfl_xor_sync(0xffffffffu, a, 2);
+    if (j < r && part == 0) sphi[j] = a;
   }
   __syncthreads();
-  float* Mu = M + ((size_t)bi * Hkv + kh) * r * D;
-  for (int i = tid; i < r * D; i += kOnThreads) {
-    const int j = i / D, c = i % D;
-    Mu[i] = fmaf(lambda, Mu[i], sphi[j] * sv[c]);
+  // M <- lambda M + phi v^T, float4 read-modify-write (r*D/4 per head)
+  float4* Mu = reinterpret_cast<float4*>(M + ((size_t)bi * Hkv + kh) * r * D);
+#pragma unroll 4
+  for (int i = tid; i < r * D / 4; i += kOnThreads) {
+    const int j = (4 * i) / D, c = (4 * i) % D;
+    float4 m = Mu[i];
+    const float ph = sphi[j];
+    m.x = fmaf(lambda, m.x, ph * sv[c]);
+    m.y = fmaf(lambda, m.y, ph * sv[c + 1]);
+    m.z = fmaf(lambda, m.z, ph * sv[c + 2]);
+    m.w = fmaf(lambda, m.w, ph * sv[c + 3]);
+    Mu[i] = m;
   }
   for (int j = tid; j < r; j += kOnThreads) {
     float* bp = bstab + ((size_t)bi * Hkv + kh) * r + j;
@@ -308,20 +385,33 @@ cudaError_t launch_online_init(const Ctx& c, int batch, int L, int B, int cap,
   return cudaGetLastError();
 }
 
+// launch with programmatic stream serialization (the kernels wait for their
+// predecessor themselves)
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*k)(KArgs...), dim3 grid, size_t smem, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kOnThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, static_cast<KArgs>(args)...);
+}
+
 cudaError_t launch_online_features(const Ctx& c, int batch, const void* x, const void* q,
                                    float* qpart, float* kpart, cudaStream_t st) {
   const int H = c.cfg.hidden, Hq = c.cfg.n_q_heads, D = c.cfg.head_dim, dI = c.cfg.idx_dim;
   dim3 g(Hq + kKSplit, batch);
-  const size_t sm = (size_t)D * sizeof(float);
   if (c.cfg.dtype == IMEM_BF16)
-    online_features_kernel<__nv_bfloat16><<<g, kOnThreads, sm, st>>>(
-        (const __nv_bfloat16*)x, (const __nv_bfloat16*)q, (const __nv_bfloat16*)c.WcT,
-        (const __nv_bfloat16*)c.WqT, H, Hq, D, dI, qpart, kpart);
-  else
-    online_features_kernel<float><<<g, kOnThreads, sm, st>>>(
-        (const float*)x, (const float*)q, (const float*)c.WcT, (const float*)c.WqT, H, Hq, D, dI,
-        qpart, kpart);
-  return cudaGetLastError();
+    return launch_pdl(online_features_kernel<__nv_bfloat16>, g, 0, st, x, q, c.WcT, c.WqT, H, Hq,
+                      D, dI, qpart, kpart);
+  return launch_pdl(online_features_kernel<float>, g, 0, st, x, q, c.WcT, c.WqT, H, Hq, D, dI,
+                    qpart, kpart);
 }
 
 cudaError_t launch_online_evict(const Ctx& c, int batch, int B, int cap, const float* qpart,
@@ -331,25 +421,21 @@ cudaError_t launch_online_evict(const Ctx& c, int batch, int B, int cap, const f
                                 int* counter, int* evict_slot, cudaStream_t st) {
   const int nct = online_score_ctas(B);
   const int rows_per_cta = (B + 1 + nct - 1) / nct;
-  online_score_kernel<<<dim3(nct, batch), kOnThreads, 0, st>>>(
-      B, cap, c.cfg.n_q_heads, c.cfg.idx_dim, rows_per_cta, qpart, kpart,
-      (__nv_bfloat16*)khat_ret, I_ret, pos_ret, next_pos, (EvictCand*)cand, counter, evict_slot,
-      evicted);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(online_score_kernel, dim3(nct, batch), 0, st, B, cap,
+                             c.cfg.n_q_heads, c.cfg.idx_dim, rows_per_cta, qpart, kpart,
+                             khat_ret, I_ret, pos_ret, next_pos, cand, counter, evict_slot,
+                             evicted);
   if (e != cudaSuccess) return e;
   const int Hkv = c.cfg.n_kv_heads, D = c.cfg.head_dim, r = c.cfg.mem_r;
   const size_t sm = (size_t)(2 * D + r) * sizeof(float);
   dim3 g(Hkv, batch);
   if (c.cfg.dtype == IMEM_BF16)
-    online_evict_kernel<__nv_bfloat16><<<g, kOnThreads, sm, st>>>(
-        B, cap, Hkv, D, r, c.cfg.lambda, evict_slot, c.W_phi, (__nv_bfloat16*)K_ret,
-        (__nv_bfloat16*)V_ret, (__nv_bfloat16*)khat_ret, I_ret, pos_ret, next_pos, cache_len, M,
-        bstab);
-  else
-    online_evict_kernel<float><<<g, kOnThreads, sm, st>>>(
-        B, cap, Hkv, D, r, c.cfg.lambda, evict_slot, c.W_phi, (float*)K_ret, (float*)V_ret,
-        (__nv_bfloat16*)khat_ret, I_ret, pos_ret, next_pos, cache_len, M, bstab);
-  return cudaGetLastError();
+    return launch_pdl(online_evict_kernel<__nv_bfloat16>, g, sm, st, B, cap, Hkv, D, r,
+                      c.cfg.lambda, evict_slot, c.W_phi, K_ret, V_ret, khat_ret, I_ret, pos_ret,
+                      next_pos, cache_len, M, bstab);
+  return launch_pdl(online_evict_kernel<float>, g, sm, st, B, cap, Hkv, D, r, c.cfg.lambda,
+                    evict_slot, c.W_phi, K_ret, V_ret, khat_ret, I_ret, pos_ret, next_pos,
+                    cache_len, M, bstab);
 }
 
 }  // namespace imem

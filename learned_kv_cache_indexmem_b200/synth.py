@@ -173,7 +173,8 @@ def make_layer_inputs(wl: Workload, weights, seed: Optional[int] = None, device=
 
 def make_decode_inputs(wl: Workload, weights, n_steps: int, seed: Optional[int] = None,
                        device="cpu", batch: Optional[int] = None):
-    """Per decode step: q [n,b,Hq,d], k_new / v_new [n,b,Hkv,d] (workload dtype)."""
+    """Per decode step: the new token's hidden state x [n,b,H] and its
+    projections q [n,b,Hq,d], k_new / v_new [n,b,Hkv,d] (workload dtype)."""
     s = wl.shape
     seed = wl.seed if seed is None else seed
     batch = wl.batch if batch is None else batch
@@ -183,7 +184,8 @@ def make_decode_inputs(wl: Workload, weights, n_steps: int, seed: Optional[int] 
     q = _project(x, weights["W_q"], s.n_q_heads, s.head_dim)
     k = _project(x, weights["W_k"], s.n_kv_heads, s.head_dim)
     v = _project(x, weights["W_v"], s.n_kv_heads, s.head_dim)
-    return {"q": q.contiguous(), "k_new": k.contiguous(), "v_new": v.contiguous()}
+    return {"x": x.contiguous(), "q": q.contiguous(), "k_new": k.contiguous(),
+            "v_new": v.contiguous()}
 
 
 def plant_needles(wl: Workload, K: torch.Tensor, q_dec: torch.Tensor, n_needles: int,
