@@ -486,11 +486,6 @@ __device__ __forceinline__ int ld_relaxed(const int32_t* p) {
   asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
-__device__ __forceinline__ int atomic_add_acq_rel(int* p, int v) {
-  int old;
-  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
 
 // Dynamic shared memory of one decode CTA (bytes). Attention CTAs use
 // [0, att) for their row stages (then for the per-warp states); the readout
@@ -503,15 +498,17 @@ struct DecSmem {
   }
   static constexpr size_t warps() { return (size_t)4 * G * sizeof(Partial<D>); }
   static_assert((kThreads / (D / 4)) * D == 4 * kThreads, "M^T u partials: RG * D = 4 * kThreads");
-  static size_t readout(int r) {
+  // W_phi | b | u | den | gate | M^T u partials | g m | s_v | w_gate | M
+  // (m_in_w: M shares the W_phi region)
+  static size_t readout(int r, bool moment) {
     return ((size_t)r * D + r + (size_t)G * r + 2 * G + (size_t)4 * kThreads * G + (size_t)G * D +
-            D) * sizeof(float);
+            D + (size_t)G * D + (moment ? 0 : (size_t)r * D)) * sizeof(float);
   }
-  static size_t slot_off(int r) { return (readout(r) + 127) / 128 * 128; }
-  static size_t total(bool bf16, int nst, int r, int S) {
+  static size_t slot_off(int r, bool moment) { return (readout(r, moment) + 127) / 128 * 128; }
+  static size_t total(bool bf16, int nst, int r, int S, bool moment) {
     size_t w = att(bf16, nst);
     if (warps() > w) w = warps();
-    const size_t rs = slot_off(r) + (size_t)S * G * sizeof(Partial<D>);
+    const size_t rs = slot_off(r, moment) + (size_t)S * G * sizeof(Partial<D>);
     return rs > w ? rs : w;
   }
 };
@@ -544,16 +541,31 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   __shared__ __align__(8) uint64_t s_bar[kDecodeMaxStages];
   Partial<D>* slots = reinterpret_cast<Partial<D>*>(dyn_smem + slot_off);   // readout CTA only
 
+  // readout CTA's shared memory (see DecSmem::readout)
+  constexpr int RG = kThreads / (D / 4);                    // row groups of the M^T u partials
+  float* sW = reinterpret_cast<float*>(dyn_smem);          // [r][D] W_phi, 16-byte chunks XOR-swizzled
+  float* sb = sW + (size_t)r * D;                           // [r]
+  float* su = sb + r;                                       // [G][r]
+  float* sden = su + G * r;                                 // [G]
+  float* sgate = sden + G;                                  // [G]
+  float* snum = sgate + G;                                  // [RG][G][D] partial M^T u
+  float* ro = snum + RG * G * D;                            // [G][D] = g * m (moment: S q)
+  float* ssv = ro + G * D;                                  // [D] moment: s_v of this unit
+  float* sG = ssv + D;                                      // [G][D] w_gate rows of the group
+  // [r][D] M of this unit: its own region in a one-wave grid (staged early,
+  // latency), the W_phi region otherwise (staged after u, occupancy)
+  float* sM = (moment || kTma) ? sW : sG + G * D;
   if (rank == S && !moment) {
-    // W_phi belongs to the context and is written only at imem_init, so the
-    // readout CTA may stage it before waiting for the previous kernel (the
-    // moment readout's map is the identity: u = q, nothing to stage)
-    float* sW = reinterpret_cast<float*>(dyn_smem);          // [r][D], chunks XOR-swizzled
+    // W_phi and w_gate belong to the context and are written only at
+    // imem_init, so the readout CTA stages them before waiting for the
+    // previous kernel (the moment readout uses neither: u = q, no gate)
     const uint32_t wdst = smem_u32(sW);
     for (int i = tid; i < r * D / 4; i += kThreads) {
       const int j = (4 * i) / D, cc = ((4 * i) % D) / 4;
       cp_async16(wdst + (uint32_t)(j * D + ((cc ^ (j & 7)) * 4)) * 4u, W_phi + 4 * i, true);
     }
+    for (int i = tid; i < G * D / 4; i += kThreads)
+      cp_async16(smem_u32(sG) + (uint32_t)i * 16u, w_gate + (size_t)kh * G * D + 4 * i, true);
     cp_async_commit();
   }
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
@@ -666,11 +678,13 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
       attend_f32<D, G>(Kb, Vb, row_stride, kn, vn, len, r0, r1, s_q, w_part);
     cluster_wait();   // phase 0 complete: every CTA of the cluster is running
     // CTA 0 counts the unit on its sequence's counter (every CTA of the unit
-    // has read cache_len); the last unit of the sequence advances cache_len.
-    // acq_rel: that update is ordered after every other unit's reads. The
-    // result is used last, so the atomic's round trip overlaps the push.
+    // has read cache_len: each branched on the length it loaded before
+    // arriving on the barrier just completed, so those loads have returned
+    // their values); the last unit of the sequence advances cache_len. A
+    // relaxed atomic whose result is used last, so that its round trip
+    // overlaps the push (an acquire would stall the warp here).
     int arrived = 0;
-    if (rank == 0 && tid == 0) arrived = atomic_add_acq_rel(&seq_counters[bi], 1);
+    if (rank == 0 && tid == 0) arrived = atomicAdd(&seq_counters[bi], 1);
     // push this CTA's merged state into the readout CTA's slot, then arrive
     Partial<D>* slot = cluster.map_shared_rank(slots, S) + (size_t)rank * G;
     merge_warps<D, G>(w_part, slot);
@@ -683,76 +697,65 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   }
 
   // ---- readout CTA: u = W_phi q, m = M^T u / (b.u + eps), g = sigmoid(w_gate . q)
-  float* sW = reinterpret_cast<float*>(dyn_smem);          // [r][D], 16-byte chunks XOR-swizzled
-  float* sb = sW + (size_t)r * D;                           // [r]
-  float* su = sb + r;                                       // [G][r]
-  float* sden = su + G * r;                                 // [G]
-  float* sgate = sden + G;                                  // [G]
-  constexpr int RG = kThreads / (D / 4);                    // row groups of the M^T u partials
-  float* snum = sgate + G;                                  // [RG][G][D] partial M^T u
-  float* ro = snum + RG * G * D;                            // [G][D] = g * m (moment: S q)
-  float* ssv = ro + G * D;                                  // [D] moment: s_v of this unit
   {
+    // b (and s_v) and the whole of M, in flight together
     for (int i = tid; i < r / 4; i += kThreads)
       cp_async16(smem_u32(sb) + (uint32_t)i * 16u, bstab + (size_t)unit * r + 4 * i, true);
     if (moment)
       for (int i = tid; i < D / 4; i += kThreads)
         cp_async16(smem_u32(ssv) + (uint32_t)i * 16u, s_v + (size_t)unit * D + 4 * i, true);
+    if (moment || !kTma) {
+      const float* Mu = M + (size_t)unit * r * D;
+      for (int i = tid; i < r * D / 4; i += kThreads)
+        cp_async16(smem_u32(sM) + (uint32_t)i * 16u, Mu + 4 * i, true);
+    }
     cp_async_commit();
   }
   const float ne = moment ? __ldcg(n_e + bi) : 0.f;
-  constexpr int kREarly = 64;   // rows of M held in registers (below)
-  if (moment && r > kREarly) {
-    // moment readout: the rows of M past the register ones go to the (unused)
-    // W_phi region, so that they are in flight while u is formed
-    for (int i = tid; i < (r - kREarly) * D / 4; i += kThreads)
-      cp_async16(smem_u32(sW) + (uint32_t)i * 16u,
-                 M + ((size_t)unit * r + kREarly) * D + 4 * i, true);
-    cp_async_commit();
-  }
-  // M: thread (row group rg, column quad cq) holds rows rg, rg+4, ... of
-  // columns 4cq..4cq+3 (first 64 rows), loaded now so they arrive while u is
-  // computed (volatile: the loads are issued here, not at their first use)
-  const int cq = tid % (D / 4), rg = tid / (D / 4);         // D/4 column quads, RG row groups
-  float4 mreg[kREarly / RG];
-  const float* Mu = M + (size_t)unit * r * D;
-#pragma unroll
-  for (int k = 0; k < kREarly / RG; ++k) {
-    const int j = rg + k * RG;
-    if (j < r) {
-      asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];\n"
-                   : "=f"(mreg[k].x), "=f"(mreg[k].y), "=f"(mreg[k].z), "=f"(mreg[k].w)
-                   : "l"(Mu + (size_t)j * D + 4 * cq));
-    } else {
-      mreg[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-  }
-  // gate: z = w_gate[h] . q (independent of the memory; none in moment mode)
+  cp_async_wait<0>();
+  __syncthreads();
+  // gate: z = w_gate[h] . q (none in moment mode)
   for (int g = warp; g < G && !moment; g += kThreads / 32) {
-    const float* wg = w_gate + ((size_t)kh * G + g) * D;
     float z = 0.f;
-    for (int c = lane; c < D; c += 32) z = fmaf(__ldg(wg + c), s_q[g][c], z);
+    for (int c = lane; c < D; c += 32) z = fmaf(sG[g * D + c], s_q[g][c], z);
     z = warp_sum(z);
     if (lane == 0) sgate[g] = use_override ? gate_override : sigmoidf_(z);
   }
-  cp_async_wait<0>();
-  __syncthreads();
-  for (int o = tid; o < G * r && moment; o += kThreads) su[o] = s_q[o / r][o % r];   // u = q
-  for (int o = tid; o < G * r && !moment; o += kThreads) {
-    const int g = o / r, j = o % r;
-    const float4* wr = reinterpret_cast<const float4*>(sW + (size_t)j * D);
-    const float4* q4 = reinterpret_cast<const float4*>(&s_q[g][0]);
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 8
-    for (int cc = 0; cc < D / 4; ++cc) {
-      const float4 w = wr[cc ^ (j & 7)];
-      const float4 x = q4[cc];
-      a0 = fmaf(w.x, x.x, a0);
-      a1 = fmaf(w.y, x.y, a1);
-      a2 = fmaf(w.z, x.z, a2);
-      a3 = fmaf(w.w, x.w, a3);
+  if (moment) {
+    for (int o = tid; o < G * r; o += kThreads) su[o] = s_q[o / r][o % r];   // u = q
+  } else {
+    // u = W_phi q: a pair of threads per row of W_phi (one half each), all G
+    // heads at once, so that each row is read once (q is a broadcast read)
+    for (int o = tid; o < 2 * r; o += kThreads) {
+      const int j = o >> 1, half = o & 1;
+      const float4* wr = reinterpret_cast<const float4*>(sW + (size_t)j * D);
+      float acc[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) acc[g] = 0.f;
+#pragma unroll 4
+      for (int cc = half * (D / 8); cc < (half + 1) * (D / 8); ++cc) {
+        const float4 w = wr[cc ^ (j & 7)];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float4 x = reinterpret_cast<const float4*>(&s_q[g][0])[cc];
+          acc[g] = fmaf(w.x, x.x, fmaf(w.y, x.y, fmaf(w.z, x.z, fmaf(w.w, x.w, acc[g]))));
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 1);
+        if (half == 0) su[g * r + j] = acc[g];
+      }
     }
-    su[o] = (a0 + a1) + (a2 + a3);
+    if (kTma) {
+      // M into the W_phi region, now that every thread is done with W_phi
+      __syncthreads();
+      const float* Mu = M + (size_t)unit * r * D;
+      for (int i = tid; i < r * D / 4; i += kThreads)
+        cp_async16(smem_u32(sM) + (uint32_t)i * 16u, Mu + 4 * i, true);
+      cp_async_commit();
+      cp_async_wait<0>();
+    }
   }
   __syncthreads();
   for (int g = warp; g < G; g += kThreads / 32) {
@@ -762,28 +765,14 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     if (lane == 0) sden[g] = moment ? a : a + eps;   // moment: s_k . q
   }
   {
-    // partial num over this thread's rows, for its 4 columns and every head
+    // partial M^T u over this thread's rows, for its 4 columns and every head
+    const int cq = tid % (D / 4), rg = tid / (D / 4);       // D/4 column quads, RG row groups
     float4 acc[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) acc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int k = 0; k < kREarly / RG; ++k) {
-      const int j = rg + k * RG;
-      if (j < r) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float uu = su[g * r + j];
-          acc[g].x = fmaf(mreg[k].x, uu, acc[g].x);
-          acc[g].y = fmaf(mreg[k].y, uu, acc[g].y);
-          acc[g].z = fmaf(mreg[k].z, uu, acc[g].z);
-          acc[g].w = fmaf(mreg[k].w, uu, acc[g].w);
-        }
-      }
-    }
-    for (int j = kREarly + rg; j < r; j += RG) {   // r > 64: remaining rows
-      const float4 mv =
-          moment ? reinterpret_cast<const float4*>(sW + (size_t)(j - kREarly) * D)[cq]
-                 : __ldcg(reinterpret_cast<const float4*>(Mu + (size_t)j * D + 4 * cq));
+#pragma unroll 4
+    for (int j = rg; j < r; j += RG) {
+      const float4 mv = reinterpret_cast<const float4*>(sM + (size_t)j * D)[cq];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float uu = su[g * r + j];
@@ -882,8 +871,10 @@ cudaError_t launch_tgs(const Ctx& c, int S, int nst, int batch, const void* q, c
                       void* out, int* counters, cudaStream_t st) {
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   const int r = c.cfg.mem_r;
-  const size_t smem = DecSmem<D, G>::total(kBf16, nst, r, S);
-  const uint32_t slot_off = (uint32_t)DecSmem<D, G>::slot_off(r);
+  // M shares the W_phi region in moment mode and in multi-wave (TMA) grids
+  const bool m_in_w = c.cfg.readout == IMEM_READOUT_MOMENT || kTma;
+  const size_t smem = DecSmem<D, G>::total(kBf16, nst, r, S, m_in_w);
+  const uint32_t slot_off = (uint32_t)DecSmem<D, G>::slot_off(r, m_in_w);
   auto k = decode_kernel<T, D, G, kTma>;
   static size_t attr_smem[64] = {};   // per instantiation and device: largest size set so far
   const int dv = c.device & 63;
