@@ -656,20 +656,21 @@ def run_e2e(job, steps, warmup):
 
 # ------------------------------------------------------------------ cpu oracle
 
-def cpu_oracle_sample(wl, B, budget_s=20.0):
+def cpu_oracle_sample(wl, B, scale=1):
     """Times the CPU oracle on a bounded sample of the workload and scales each
     stage to the full step by its unit count. Returns (seconds per full step,
-    description of the sample, threads used)."""
+    description of the sample). `scale` multiplies the sample's tokens, keys,
+    evicted tokens and decode steps (1: ~2 s of CPU work, 4: ~10 s)."""
     from oracle import indexmem_oracle as om
     s = wl.shape
     torch.manual_seed(0)
-    Ls = min(wl.L, 2048)                       # one sequence, first Ls tokens
+    Ls = min(wl.L, 2048 * scale)               # one sequence, first Ls tokens
     w = synth.make_weights(s, wl.seed, "cpu")
     inp = synth.make_layer_inputs(wl, w, wl.seed, "cpu", L=Ls, batch=1)
     t0 = time.perf_counter()
     qhat, khat, gate = om.indexer_features(inp["X"], inp["Q"], w["W_iq"], w["W_ik"], w["w_ig"])
     t_feat = (time.perf_counter() - t0) / Ls                      # per token
-    keys = np.arange(0, Ls, max(1, Ls // 64))
+    keys = np.arange(0, Ls, max(1, Ls // (64 * scale)))
     t0 = time.perf_counter()
     om.pooled_importance(qhat, khat, gate, keys=keys)
     pairs_s = sum(Ls - k for k in keys)
@@ -678,12 +679,12 @@ def cpu_oracle_sample(wl, B, budget_s=20.0):
     t0 = time.perf_counter()
     R, E = om.select_budget(I, B)
     t_sel = time.perf_counter() - t0                               # per sequence
-    n_mem = min(512, Ls - 1)
+    n_mem = min(512 * scale, Ls - 1)
     Em = np.arange(n_mem)[None]
     t0 = time.perf_counter()
     M, bs = om.memory_update(inp["K"], inp["V"], Em, w["W_phi"], s.lam)
     t_mem = (time.perf_counter() - t0) / n_mem                     # per evicted token
-    n_steps = 4
+    n_steps = 4 * scale
     dec = synth.make_decode_inputs(wl, w, n_steps, wl.seed, "cpu", batch=1)
     Bs = min(B, Ls)
     KR, VR = om.compact(inp["K"].float().numpy(), inp["V"].float().numpy(), np.arange(Bs)[None],
@@ -764,7 +765,7 @@ def main():
         per_step = []
         desc = None
         for i in range(a.warmup + a.steps):
-            t, desc = cpu_oracle_sample(wl, B)
+            t, desc = cpu_oracle_sample(wl, B, scale=2)   # ~3 s a step
             if i >= a.warmup:
                 per_step.append(t)
         t = statistics.mean(per_step)
@@ -867,7 +868,7 @@ def main():
         model_dec = model_decode(dev, peak)
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        t_full, desc = cpu_oracle_sample(wl, B)
+        t_full, desc = cpu_oracle_sample(wl, B, scale=8)   # ~10-15 s of CPU work
         cpu = {"value": job.tokens_per_step() / t_full, "unit": "tokens/s",
                "cores": oracle_threads(), "kind": "oracle", "sample": desc}
     if world > 1:
