@@ -324,6 +324,16 @@ imem_status imem_decode_online(imem_ctx* ctx, int batch, int B, const void* x_ne
                                int32_t* cache_len, int cap, float* M, float* bstab, void* out,
                                int32_t* evicted, void* workspace, void* stream);
 
+/* Failure-path self-test (no counterpart in the papers): launches one CTA
+ * that waits on a transaction barrier nothing completes, through the same
+ * bounded wait every kernel of this library uses, with the given limit in SM
+ * clock cycles (1 .. 2e9; the kernels use 2e9, about one second). The wait
+ * runs out, the device records a timeout in the context's error word and the
+ * next imem_sync returns IMEM_ERR_TIMEOUT (and clears it); the context stays
+ * usable. Nothing faults and nothing waits without a limit.
+ * Errors: INVALID_ARG (limit out of range), CUDA. */
+imem_status imem_selftest_wait(imem_ctx* ctx, long long limit_cycles, void* stream);
+
 /* Waits for the stream, then reports the first error the device recorded for
  * this context since the last imem_sync (TIMEOUT for a bounded wait that ran
  * out, SHAPE for a decode into a full cache) or a CUDA error, and clears it. */

@@ -83,6 +83,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.imem_decode_online.restype = i
     lib.imem_decode_online.argtypes = [vp, i, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i,
                                        vp, vp, vp, vp, vp, vp]
+    lib.imem_selftest_wait.restype = i
+    lib.imem_selftest_wait.argtypes = [vp, ctypes.c_longlong, vp]
     lib.imem_update_moments.restype = i
     lib.imem_update_moments.argtypes = [vp, i, i, vp, vp, vp, i, i, vp, vp, vp, vp, vp, vp]
     lib.imem_decode_moment.restype = i
@@ -200,6 +202,11 @@ def decode_online(ctx, batch, B, x_new, q, k_new, v_new, K_ret, V_ret, khat_ret,
         _ptr(khat_ret), _ptr(I_ret), _ptr(pos_ret), _ptr(next_pos), _ptr(cache_len), cap, _ptr(M),
         _ptr(bstab), _ptr(out), _ptr(evicted), _ptr(workspace), _stream(stream)),
         "imem_decode_online")
+
+
+def selftest_wait(ctx, limit_cycles, stream=None):
+    """imem_selftest_wait: a bounded device wait that runs out (failure path)."""
+    _check(load().imem_selftest_wait(ctx, int(limit_cycles), _stream(stream)), "imem_selftest_wait")
 
 
 def update_moments(ctx, batch, L, K, V, idx_evicted, n_evicted, chunk, S_T, s_k, s_v, n_e,

@@ -538,6 +538,13 @@ imem_status imem_decode_online(imem_ctx* h, int batch, int B, const void* x_new,
                                                (int*)(wsb + ws.on_slot_off), st));
 }
 
+imem_status imem_selftest_wait(imem_ctx* h, long long limit_cycles, void* stream) {
+  if (!h) return IMEM_ERR_INVALID_ARG;
+  if (limit_cycles < 1 || limit_cycles > 2000000000LL) return IMEM_ERR_INVALID_ARG;
+  IMEM_CHECK(check_device(h->c));
+  return cuda_status(imem::launch_wait_selftest(h->c, limit_cycles, (cudaStream_t)stream));
+}
+
 imem_status imem_sync(imem_ctx* h, void* stream) {
   if (!h) return IMEM_ERR_INVALID_ARG;
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);

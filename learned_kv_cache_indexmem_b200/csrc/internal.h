@@ -120,6 +120,9 @@ cudaError_t launch_online_evict(const Ctx& c, int batch, int B, int cap, const f
                                 float* M, float* bstab, int32_t* evicted, void* cand,
                                 int* counter, int* evict_slot, cudaStream_t st);
 
+// A kernel whose bounded wait runs out after `limit` cycles (failure-path test).
+cudaError_t launch_wait_selftest(const Ctx& c, long long limit, cudaStream_t st);
+
 // K_ret/V_ret[:, :n] = K/V[idx[:, :n]] (idx stride `idx_stride`).
 cudaError_t launch_gather(const Ctx& c, int batch, int L, int n, const int32_t* idx,
                           int idx_stride, const void* K, const void* V, void* K_ret, void* V_ret,

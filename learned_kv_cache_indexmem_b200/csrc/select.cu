@@ -26,6 +26,8 @@
 #include "common.cuh"
 #include "internal.h"
 
+#include <cooperative_groups.h>
+
 namespace imem {
 namespace {
 
@@ -179,6 +181,178 @@ select_kernel(const float* __restrict__ I, int L, int stride, int B, int32_t* __
   }
 }
 
+// ---- the same selection over a thread-block cluster ---------------------------
+// CTA `rank` of the cluster holds keys [rank * kpt * 1024, ...) in registers
+// (warp w: the contiguous kpt * 32 positions from w * kpt * 32). Each radix
+// pass builds a per-CTA histogram; after one cluster barrier every CTA sums
+// all of them through distributed shared memory and picks the same digit
+// (histograms double-buffered: a buffer is refilled two passes later, after
+// every CTA's reads of it). Output: counts per warp and per CTA, one scan
+// over the CTAs (shared memory of the others) and one over the warps.
+constexpr int kCsMaxKpt = 16;
+constexpr int kCsMaxCluster = 16;
+
+__global__ void __launch_bounds__(kSelThreads, 1)
+select_cluster_kernel(const float* __restrict__ I, int L, int stride, int B, int kpt,
+                      int32_t* __restrict__ idx_r, int32_t* __restrict__ idx_e) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  constexpr int kWarps = kSelThreads / 32;
+  const int CS = (int)cl.num_blocks(), rank = (int)cl.block_rank();
+  const int bi = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float* Ib = I + (size_t)bi * stride;
+  __shared__ int s_hist[2][256];
+  __shared__ int s_tot[256];
+  __shared__ int s_wcnt[2][kWarps];
+  __shared__ int s_wbase[2][kWarps];
+  __shared__ int s_cnt[2];                  // this CTA: keys above T, keys equal to T
+  __shared__ int s_cbase[2];                // takes and equal keys before this CTA
+  __shared__ uint32_t s_prefix, s_mask;
+  __shared__ int s_k;
+
+  const int w0 = rank * kpt * kSelThreads + warp * kpt * 32;   // this warp's first position
+  uint32_t key[kCsMaxKpt];
+  uint32_t valid = 0;
+#pragma unroll
+  for (int k = 0; k < kCsMaxKpt; ++k) {
+    key[k] = 0u;
+    const int t = w0 + k * 32 + lane;
+    if (k < kpt && t < L) {
+      key[k] = order_key(Ib[t]);
+      valid |= 1u << k;
+    }
+  }
+  if (tid == 0) { s_prefix = 0; s_mask = 0; s_k = B; }
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass, buf = pass & 1;
+    if (tid < 256) s_hist[buf][tid] = 0;
+    __syncthreads();
+    const uint32_t prefix = s_prefix, mask = s_mask;
+#pragma unroll
+    for (int k = 0; k < kCsMaxKpt; ++k)
+      if ((valid >> k & 1u) && (key[k] & mask) == prefix)
+        atomicAdd(&s_hist[buf][(key[k] >> shift) & 0xffu], 1);
+    __syncthreads();
+    cl.sync();   // every CTA's histogram of this pass is complete
+    if (tid < 256) {
+      int c = 0;
+      for (int r = 0; r < CS; ++r) c += *cl.map_shared_rank(&s_hist[buf][tid], r);
+      s_tot[tid] = c;
+    }
+    __syncthreads();
+    if (tid < 32) {
+      const int k = s_k;
+      int local[8];
+      int sum = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { local[i] = s_tot[255 - (tid * 8 + i)]; sum += local[i]; }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int nn = __shfl_up_sync(0xffffffffu, incl, o);
+        if (tid >= o) incl += nn;
+      }
+      const int excl = incl - sum;
+      if (excl < k && k <= incl) {
+        int run = excl;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (run < k && k <= run + local[i]) {
+            const uint32_t digit = 255u - (uint32_t)(tid * 8 + i);
+            s_k = k - run;
+            s_prefix = prefix | (digit << shift);
+            s_mask = mask | (0xffu << shift);
+          }
+          run += local[i];
+        }
+      }
+    }
+    __syncthreads();
+  }
+  const uint32_t T = s_prefix;
+  const int take_eq = s_k;
+  // counts of this warp's keys above and equal to T
+  int gt = 0, eq = 0;
+#pragma unroll
+  for (int k = 0; k < kCsMaxKpt; ++k) {
+    const bool in = valid >> k & 1u;
+    gt += __popc(__ballot_sync(0xffffffffu, in && key[k] > T));
+    eq += __popc(__ballot_sync(0xffffffffu, in && key[k] == T));
+  }
+  if (lane == 0) { s_wcnt[0][warp] = gt; s_wcnt[1][warp] = eq; }
+  __syncthreads();
+  if (warp == 0) {
+    const int g = s_wcnt[0][lane], e = s_wcnt[1][lane];
+    const int gs = __reduce_add_sync(0xffffffffu, g), es = __reduce_add_sync(0xffffffffu, e);
+    if (lane == 0) { s_cnt[0] = gs; s_cnt[1] = es; }
+  }
+  __syncthreads();
+  cl.sync();   // every CTA's counts are visible
+  if (warp == 0) {
+    // equal keys and takes before this CTA, from the CTAs of lower rank
+    const int r = lane;
+    const int ge = r < CS ? *cl.map_shared_rank(&s_cnt[0], r) : 0;
+    const int ee = r < CS ? *cl.map_shared_rank(&s_cnt[1], r) : 0;
+    int e_incl = ee;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int nn = __shfl_up_sync(0xffffffffu, e_incl, o);
+      if (lane >= o) e_incl += nn;
+    }
+    const int e_base = e_incl - ee;
+    const int takes = ge + max(0, min(ee, take_eq - e_base));
+    int t_incl = takes;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int nn = __shfl_up_sync(0xffffffffu, t_incl, o);
+      if (lane >= o) t_incl += nn;
+    }
+    if (lane == rank) { s_cbase[0] = t_incl - takes; s_cbase[1] = e_base; }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // then the warps of this CTA, after the CTAs before it
+    const int e = s_wcnt[1][lane];
+    int e_incl = e;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int nn = __shfl_up_sync(0xffffffffu, e_incl, o);
+      if (lane >= o) e_incl += nn;
+    }
+    const int e_base = s_cbase[1] + e_incl - e;
+    const int takes = s_wcnt[0][lane] + max(0, min(e, take_eq - e_base));
+    int t_incl = takes;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int nn = __shfl_up_sync(0xffffffffu, t_incl, o);
+      if (lane >= o) t_incl += nn;
+    }
+    s_wbase[0][lane] = s_cbase[0] + t_incl - takes;
+    s_wbase[1][lane] = e_base;
+  }
+  __syncthreads();
+  int before = s_wbase[0][warp], eq_seen = s_wbase[1][warp];
+  const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int k = 0; k < kCsMaxKpt; ++k) {
+    const int t = w0 + k * 32 + lane;
+    const bool in = valid >> k & 1u;
+    const bool is_eq = in && key[k] == T;
+    const unsigned eqb = __ballot_sync(0xffffffffu, is_eq);
+    const bool take = in && (key[k] > T || (is_eq && eq_seen + __popc(eqb & lt) < take_eq));
+    const unsigned tb = __ballot_sync(0xffffffffu, take);
+    const int my = before + __popc(tb & lt);
+    if (in) {
+      if (take) idx_r[(size_t)bi * B + my] = t;
+      else idx_e[(size_t)bi * (L - B) + (t - my)] = t;
+    }
+    before += __popc(tb);
+    eq_seen += __popc(eqb);
+  }
+  cl.sync();   // no CTA leaves while another may read its shared memory
+}
+
 // One warp group per retained row: copies Hkv*d elements of K and V. Rows
 // [0, n) of sequence bi come from positions idx_r[bi * idx_stride + j].
 template <typename T>
@@ -259,6 +433,40 @@ __global__ void append_positions_kernel(int B, int n_R, int q0, int C, int32_t* 
   if (i < C) retained[(size_t)bi * B + n_R + i] = q0 + i;
 }
 
+// Selection of the B largest of L importances per sequence (stride between
+// sequences): a cluster per sequence when the keys fit its registers, one
+// CTA per sequence otherwise.
+cudaError_t launch_select(int batch, const float* I, int L, int stride, int B, int32_t* idx_r,
+                          int32_t* idx_e, cudaStream_t st) {
+  int CS = (L + 4095) / 4096;
+  if (CS < 1) CS = 1;
+  if (CS > kCsMaxCluster) CS = kCsMaxCluster;
+  const int kpt = (L + CS * kSelThreads - 1) / (CS * kSelThreads);
+  if (kpt > kCsMaxKpt) {
+    select_kernel<<<batch, kSelThreads, 0, st>>>(I, L, stride, B, idx_r, idx_e);
+    return cudaGetLastError();
+  }
+  static bool attr_set = false;
+  if (!attr_set) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(select_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CS, batch, 1);
+  cfg.blockDim = dim3(kSelThreads, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, select_cluster_kernel, I, L, stride, B, kpt, idx_r, idx_e);
+}
+
 }  // namespace
 
 cudaError_t launch_evict_chunk(const Ctx& c, int batch, int B, int Lc, int n_R, int q0, int C,
@@ -267,8 +475,7 @@ cudaError_t launch_evict_chunk(const Ctx& c, int batch, int B, int Lc, int n_R, 
   (void)c;
   const int n = n_R + C, n_ev = n - B;
   if (n_ev <= 0) return cudaErrorInvalidValue;
-  select_kernel<<<batch, kSelThreads, 0, st>>>(w.I_c, n, Lc, B, w.idx_r, w.idx_e);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_select(batch, w.I_c, n, Lc, B, w.idx_r, w.idx_e, st);
   if (e != cudaSuccess) return e;
   dim3 g1((B + n_ev + kRowsPerCompactCta - 1) / kRowsPerCompactCta, batch);
   evict_compact_kernel<<<g1, 256, 0, st>>>(w.idx_r, w.idx_e, B, n_ev, n_R, q0, Lc, retained,
@@ -311,8 +518,7 @@ cudaError_t launch_select_compact(const Ctx& c, int batch, int L, int B, const f
                                   const void* K, const void* V, int32_t* idx_r, int32_t* idx_e,
                                   void* K_ret, void* V_ret, int cap, void* /*scratch*/,
                                   cudaStream_t st) {
-  select_kernel<<<batch, kSelThreads, 0, st>>>(running_max, L, L, B, idx_r, idx_e);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_select(batch, running_max, L, L, B, idx_r, idx_e, st);
   if (e != cudaSuccess) return e;
   return launch_gather(c, batch, L, B, idx_r, B, K, V, K_ret, V_ret, cap, st);
 }
