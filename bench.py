@@ -390,6 +390,73 @@ def moment_readout(job, steps=64, reps=3):
     return res
 
 
+# ------------------------------------------------------------------ stage split, budgets
+
+def prefill_split(job, reps=5):
+    """The prefill split as the survey of the method reports it: the indexer
+    (prologue + scoring, the call without selection) and eviction + compaction
+    (selection and the K/V gather: the rest of the full call), CUDA events."""
+    d = job.inp
+    st = job.st
+
+    def timed(finalize):
+        best = None
+        for _ in range(reps):
+            a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            a.record(job.stream)
+            for i, (q0, q1) in enumerate(job.ranges):
+                last = i == len(job.ranges) - 1
+                binding.score_and_evict(job.layer.ctx, job.batch, job.L, job.B, d["X"], d["Q"],
+                                        d["K"], d["V"], st.running_max, q0, q1,
+                                        1 if (finalize and last) else 0, st.idx_retained,
+                                        st.idx_evicted, st.K_ret, st.V_ret, st.K_ret.shape[1],
+                                        job.layer._ws, job.stream)
+            e.record(job.stream)
+            torch.cuda.synchronize()
+            t = a.elapsed_time(e)
+            best = t if best is None else min(best, t)
+        return best
+
+    t_idx = timed(False)
+    t_all = timed(True)
+    s = job.wl.shape
+    es = 2 if s.dtype == "bf16" else 4
+    row = s.n_kv_heads * s.head_dim * es * 2
+    ev_bytes = job.batch * (4 * job.L + 4 * job.L + 2 * job.B * row)   # scores, indices, K/V rows
+    t_ev = max(t_all - t_idx, 1e-6)
+    return {"indexer_ms": t_idx, "indexer_keys_per_s": job.batch * job.L / (t_idx * 1e-3),
+            "indexer_tflops": job.scoring_flops() / (t_idx * 1e-3) / 1e12,
+            "evict_compact_ms": t_ev, "evict_compact_GBps": ev_bytes / (t_ev * 1e-3) / 1e9}
+
+
+def budget_sweep(wl, dev, seed, budgets=(128, 256, 512), steps=5, warmup=3):
+    """The whole step at the other budgets of the workload (the benchmark's own
+    budget is the main line): time per step, tokens/s and decode per launch."""
+    out = {}
+    for B in budgets:
+        j = Job(wl, B, dev, seed)
+        j.capture_decode()
+        for _ in range(warmup):
+            j.step()
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(j.stream)
+        for i in range(steps):
+            j.step(ev[i])
+        e.record(j.stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(e) / steps
+        dec = statistics.mean(x[2].elapsed_time(x[3]) for x in ev)
+        out[str(B)] = {"ms_per_step": ms, "tokens_per_s": j.tokens_per_step() / (ms * 1e-3),
+                       "decode_us_per_launch": dec / j.n_dec * 1e3}
+        j.layer.sync(j.stream)
+        del j
+        torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------------------ online eviction
 
 def online_decode(job, steps=64, reps=3):
@@ -734,6 +801,8 @@ def main():
                     help="skip the 36-layer decode measurement")
     ap.add_argument("--no-moment", action="store_true",
                     help="skip the MomentKV readout measurement")
+    ap.add_argument("--no-budget-sweep", action="store_true",
+                    help="skip the other budgets of the workload")
     ap.add_argument("--no-online", action="store_true",
                     help="skip the decode-time online eviction measurement")
     ap.add_argument("--no-pre-eviction", action="store_true",
@@ -855,6 +924,11 @@ def main():
     moment = None
     if not a.no_moment:
         moment = moment_readout(job)
+    split = prefill_split(job)
+    stages["prefill_split"] = split
+    sweep = None
+    if not a.no_budget_sweep and wl.name == "c2" and a.budget is None:
+        sweep = budget_sweep(wl, dev, wl.seed + 1000 * rank)
     online = None
     if not a.no_online:
         online = online_decode(job)
@@ -891,6 +965,7 @@ def main():
             "cpu_baseline": cpu,
             "full_cache_decode": full_cmp,
             "moment_readout": moment,
+            "budget_sweep": sweep,
             "online_eviction": online,
             "pre_eviction": pre_ev,
             "model_decode": model_dec,
