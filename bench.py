@@ -289,6 +289,7 @@ def full_cache_decode(job, steps=64, reps=3):
     for name, st, l0 in (("full", full, len0), ("evicted", evicted, elen0)):
         with torch.cuda.stream(job.stream):
             st.cache_len.copy_(l0)
+            job.layer.invalidate_decode(b, stream=job.stream)   # the state was written directly
             job.layer.decode(job.decin["q"][0], job.decin["k_new"][0], job.decin["v_new"][0], st,
                              out=out, stream=job.stream)
             torch.cuda.synchronize()
@@ -302,6 +303,7 @@ def full_cache_decode(job, steps=64, reps=3):
             best = None
             for _ in range(reps):
                 st.cache_len.copy_(l0)
+                job.layer.invalidate_decode(b, stream=job.stream)
                 torch.cuda.synchronize()
                 a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record(job.stream)
@@ -366,6 +368,7 @@ def moment_readout(job, steps=64, reps=3):
         graphs = {}
         for name, layer, state in (("moment", lay, st), ("gated", job.layer, job.st)):
             state.cache_len.copy_(len0)
+            layer.invalidate_decode(state.cache_len.shape[0], stream=job.stream)
             layer.decode(job.decin["q"][0], job.decin["k_new"][0], job.decin["v_new"][0], state,
                          out=out, stream=job.stream)
             torch.cuda.synchronize()
@@ -377,8 +380,9 @@ def moment_readout(job, steps=64, reps=3):
                     layer.decode(job.decin["q"][i], job.decin["k_new"][i], job.decin["v_new"][i],
                                  state, out=out, stream=job.stream)
 
-            def rep(g=g, state=state):
+            def rep(g=g, state=state, layer=layer):
                 state.cache_len.copy_(len0)
+                layer.invalidate_decode(state.cache_len.shape[0], stream=job.stream)
                 g.replay()
             res["decode_us_per_step_" + name] = timed(rep) / steps * 1e3
             graphs[name] = g
@@ -474,6 +478,7 @@ def online_decode(job, steps=64, reps=3):
     res = {}
     with torch.cuda.stream(job.stream):
         on = lay.online_init(st, B, L, stream=job.stream)
+        lay.invalidate_decode(b, stream=job.stream)   # the state was copied in directly
         dec = job.decin
 
         def step(i):
@@ -604,8 +609,9 @@ def model_decode(dev, peak_gbs, steps=8, reps=3):
                            stream=stream)
 
     def reset():
-        for _, st in layers:
+        for lay, st in layers:
             st.cache_len.fill_(B)
+            lay.invalidate_decode(b, stream=stream)
 
     with torch.cuda.stream(stream):
         reset()

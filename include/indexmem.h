@@ -179,12 +179,30 @@ imem_status imem_update_memory(imem_ctx* ctx, int batch, int L, const void* K, c
  *   out = o_attn + g m            (out [batch, Hq, d], model dtype)
  * M, bstab are read only. A sequence whose cache is full (cache_len >= cap)
  * is left unchanged and its output row is not written; imem_sync reports it.
+ * Ordering: the kernel is launched with programmatic dependent launch and
+ * loads cache rows below cache_len - 1, b and M before it waits for the
+ * previous kernel of the stream. It uses those copies only if the workspace's
+ * decode tag of the sequence matches cache_len after the wait: the decode
+ * steps (and imem_decode_online) set the tag from the length they leave;
+ * a zero-filled workspace, imem_score_and_evict, imem_update_memory,
+ * imem_update_moments and imem_prefill_evict_chunk clear it (0).
+ * A caller that writes K_ret, V_ret,
+ * cache_len, M or bstab by other means (its own kernels, copies,
+ * imem_update_memory_static) between two decode steps on one workspace calls
+ * imem_decode_invalidate on that workspace before the next step.
  * Errors: INVALID_ARG, SHAPE, ALIGN, CUDA; UNSUPPORTED for a context in
  * IMEM_READOUT_MOMENT mode (use imem_decode_moment). */
 imem_status imem_decode(imem_ctx* ctx, int batch, const void* q, const void* k_new,
                         const void* v_new, void* K_ret, void* V_ret, int32_t* cache_len,
                         int cap, const float* M, const float* bstab, void* out,
                         void* workspace, void* stream);
+
+/* Clears the decode tags of `batch` sequences in a workspace (stream-ordered,
+ * no other effect), so that the next decode step on it loads nothing before
+ * its launch-dependency wait. Call it after writing a retained cache, its
+ * length or the memory state other than through this library (see
+ * imem_decode, "Ordering"). Errors: INVALID_ARG, SHAPE, CUDA. */
+imem_status imem_decode_invalidate(imem_ctx* ctx, int batch, void* workspace, void* stream);
 
 /* Latent-memory update that allocates nothing (no counterpart in the paper: an
  * interface for callers that cannot allocate device memory, e.g. code running
@@ -238,7 +256,8 @@ imem_status imem_update_moments(imem_ctx* ctx, int batch, int L, const void* K, 
  *   Z_E = n_e exp(q . k_bar / sqrt(d))   (Jensen lower bound of the evicted
  *                                         partition function),
  *   w_R = Z_R / (Z_R + Z_E),  out = w_R o_R + (1 - w_R) f_E
- * and out = o_R where n_e = 0. Errors as imem_decode. */
+ * and out = o_R where n_e = 0. Ordering as imem_decode, with S_T, s_k and
+ * s_v in the place of M and bstab. Errors as imem_decode. */
 imem_status imem_decode_moment(imem_ctx* ctx, int batch, const void* q, const void* k_new,
                                const void* v_new, void* K_ret, void* V_ret, int32_t* cache_len,
                                int cap, const float* S_T, const float* s_k, const float* s_v,

@@ -83,6 +83,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.imem_decode_online.restype = i
     lib.imem_decode_online.argtypes = [vp, i, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i,
                                        vp, vp, vp, vp, vp, vp]
+    lib.imem_decode_invalidate.restype = i
+    lib.imem_decode_invalidate.argtypes = [vp, i, vp, vp]
     lib.imem_selftest_wait.restype = i
     lib.imem_selftest_wait.argtypes = [vp, ctypes.c_longlong, vp]
     lib.imem_update_moments.restype = i
@@ -202,6 +204,13 @@ def decode_online(ctx, batch, B, x_new, q, k_new, v_new, K_ret, V_ret, khat_ret,
         _ptr(khat_ret), _ptr(I_ret), _ptr(pos_ret), _ptr(next_pos), _ptr(cache_len), cap, _ptr(M),
         _ptr(bstab), _ptr(out), _ptr(evicted), _ptr(workspace), _stream(stream)),
         "imem_decode_online")
+
+
+def decode_invalidate(ctx, batch, workspace, stream=None):
+    """imem_decode_invalidate: clears the workspace's decode tags (after the
+    caller wrote a retained cache, its length or the memory by other means)."""
+    _check(load().imem_decode_invalidate(ctx, batch, _ptr(workspace), _stream(stream)),
+           "imem_decode_invalidate")
 
 
 def selftest_wait(ctx, limit_cycles, stream=None):

@@ -30,8 +30,9 @@ Workspace workspace_layout(const Ctx& c, int batch, int L) {
   Workspace w;
   size_t off = 0;
   const size_t units = (size_t)batch * c.cfg.n_kv_heads;
-  w.dec_cnt_off = off;                        // one counter per sequence
-  off = align_up(off + (size_t)batch * sizeof(int), 256);
+  w.dec_cnt_off = off;                        // one counter per sequence, then
+  w.dec_tag_off = off + (size_t)batch * sizeof(int);   // the decode tags (one per sequence)
+  off = align_up(off + (size_t)2 * batch * sizeof(int), 256);
   // online eviction: the new token's feature partials, the score CTAs'
   // candidates (16 bytes each), a counter and the chosen slot per sequence
   w.on_qpart_off = off;
@@ -60,6 +61,17 @@ Workspace workspace_layout(const Ctx& c, int batch, int L) {
   off = align_up(off + (size_t)batch * L * kIdxPad * 2, 1024);
   w.total = off;
   return w;
+}
+
+// The decode tag of a sequence is 1 + the cache length its last decode step
+// left (0: none, as in a zero-filled workspace); a decode step uses rows and
+// memory it loaded before its launch-dependency wait only when the tag is
+// 1 + the length it finds after the wait. Every call that writes a retained
+// cache, its length or the memory state by other means clears the tags of
+// the workspace it is given.
+cudaError_t clear_decode_tags(const Ctx& c, int batch, void* workspace, cudaStream_t st) {
+  const Workspace w = workspace_layout(c, batch, 1);
+  return cudaMemsetAsync((char*)workspace + w.dec_tag_off, 0, (size_t)batch * sizeof(int), st);
 }
 
 // Pre-eviction workspace: the plain layout over Lc = B + chunk_max candidate
@@ -284,6 +296,7 @@ imem_status imem_score_and_evict(imem_ctx* h, int batch, int L, int B, const voi
   cudaStream_t st = (cudaStream_t)stream;
   const imem::Workspace ws = imem::workspace_layout(c, batch, L);
   char* wsb = (char*)workspace;
+  IMEM_CHECK(cuda_status(imem::clear_decode_tags(c, batch, workspace, st)));
   __nv_bfloat16* qt = (__nv_bfloat16*)(wsb + ws.qt_off);
   __nv_bfloat16* kh = (__nv_bfloat16*)(wsb + ws.kh_off);
   IMEM_CHECK(cuda_status(imem::launch_prologue(c, batch, L, X, Q, q_begin, q_end, qt, kh,
@@ -314,6 +327,7 @@ imem_status imem_update_memory(imem_ctx* h, int batch, int L, const void* K, con
   IMEM_CHECK(check_device(c));
   const imem::Workspace ws = imem::workspace_layout(c, batch, L);
   float* part = (float*)((char*)workspace + ws.mem_part_off);
+  IMEM_CHECK(cuda_status(imem::clear_decode_tags(c, batch, workspace, (cudaStream_t)stream)));
   return cuda_status(imem::launch_memory_update(c, batch, L, K, V, idx_evicted, n_evicted, chunk,
                                                 M, bstab, part, nullptr, nullptr, nullptr,
                                                 (cudaStream_t)stream));
@@ -341,6 +355,7 @@ imem_status imem_update_moments(imem_ctx* h, int batch, int L, const void* K, co
   const imem::Workspace ws = imem::workspace_layout(c, batch, L);
   float* part = (float*)((char*)workspace + ws.mem_part_off);
   float* svp = (float*)((char*)workspace + ws.sv_part_off);
+  IMEM_CHECK(cuda_status(imem::clear_decode_tags(c, batch, workspace, (cudaStream_t)stream)));
   return cuda_status(imem::launch_memory_update(c, batch, L, K, V, idx_evicted, n_evicted, chunk,
                                                 S_T, s_k, part, svp, s_v, n_e,
                                                 (cudaStream_t)stream));
@@ -398,6 +413,14 @@ imem_status imem_decode_moment(imem_ctx* h, int batch, const void* q, const void
                        n_e, out, workspace, stream);
 }
 
+imem_status imem_decode_invalidate(imem_ctx* h, int batch, void* workspace, void* stream) {
+  if (!h) return IMEM_ERR_INVALID_ARG;
+  if (batch < 1) return IMEM_ERR_SHAPE;
+  IMEM_CHECK(check_ptr(workspace));
+  IMEM_CHECK(check_device(h->c));
+  return cuda_status(imem::clear_decode_tags(h->c, batch, workspace, (cudaStream_t)stream));
+}
+
 imem_status imem_workspace_size_evict(imem_ctx* h, int batch, int L, int B, int chunk_max,
                                      size_t* bytes) {
   if (!h || !bytes) return IMEM_ERR_INVALID_ARG;
@@ -448,6 +471,7 @@ imem_status imem_prefill_evict_chunk(imem_ctx* h, int batch, int L, int B, int c
   const int Lc = B + chunk_max;
   const imem::EvictWorkspace ws = imem::evict_workspace_layout(c, batch, B, chunk_max);
   char* wsb = (char*)workspace;
+  IMEM_CHECK(cuda_status(imem::clear_decode_tags(c, batch, workspace, st)));
   imem::EvictBuffers eb;
   __nv_bfloat16* qt = (__nv_bfloat16*)(wsb + ws.base.qt_off);
   eb.kh_c = (__nv_bfloat16*)(wsb + ws.base.kh_off);
@@ -535,7 +559,8 @@ imem_status imem_decode_online(imem_ctx* h, int batch, int B, const void* x_new,
                                                pos_ret, next_pos, K_ret, V_ret, cache_len, M,
                                                bstab, evicted, wsb + ws.on_cand_off,
                                                (int*)(wsb + ws.on_cnt_off),
-                                               (int*)(wsb + ws.on_slot_off), st));
+                                               (int*)(wsb + ws.on_slot_off),
+                                               (int*)(wsb + ws.dec_tag_off), st));
 }
 
 imem_status imem_selftest_wait(imem_ctx* h, long long limit_cycles, void* stream) {

@@ -24,10 +24,15 @@
 //
 // Latency: the kernel is launched with programmatic stream serialization, so
 // its CTAs are resident before the previous kernel ends. CTA S stages W_phi
-// (owned by the context) before the wait; an attention CTA reads a hint of
-// cache_len before it and, right after it, issues the loads of the rows that
-// lie below the hint in its block, so they travel alongside the reads of q
-// and the true length (a wrong hint only costs those loads).
+// (owned by the context) before the wait, and b and M too where M has a
+// region of its own; an attention CTA reads a hint of cache_len before it and
+// loads the rows of its block below the hint minus one (cp.async staging; TMA
+// staging issues them right after the wait). After the wait a per-sequence
+// tag in the workspace, 1 + the length that the last decode step left and
+// cleared by every other call that writes the cache state, decides whether
+// those early copies stand: they do when the tag matches the true length
+// (the rows then predate the previous kernel, and b and M are unchanged);
+// otherwise they are dropped and loaded again.
 //
 // bf16 attention: rows are staged in shared memory with cp.async (a ring of
 // two or three 64-row stages, XOR-swizzled 16-byte chunks) and contracted
@@ -175,6 +180,29 @@ __device__ void ring_issue_lsu(const Ring& rg, const __nv_bfloat16* __restrict__
     cp_async16(vdst + tile_off<D>(rr, c), Vb + off, ok);
   }
   cp_async_commit();
+}
+
+// All threads: cp.async loads of the rows in [lo, hi) of the stage that holds
+// rows [base, base + 64) (ring index gi); the stage's other rows are left
+// untouched and nothing is committed (the caller closes the group).
+template <int D>
+__device__ void ring_issue_rows(const Ring& rg, const __nv_bfloat16* __restrict__ Kb,
+                                const __nv_bfloat16* __restrict__ Vb, size_t row_stride, int gi,
+                                int base, int lo, int hi) {
+  constexpr int CH = D / 8;
+  const uint32_t kdst = rg.buf0 + (uint32_t)(gi % rg.nst) * 2u * kTileBytes<D>;
+  const uint32_t vdst = kdst + kTileBytes<D>;
+  const int c = threadIdx.x % CH, rr0 = threadIdx.x / CH;
+  constexpr int RSTEP = kThreads / CH;
+#pragma unroll
+  for (int k = 0; k < kStageRows / RSTEP; ++k) {
+    const int rr = rr0 + k * RSTEP, row = base + rr;
+    if (row >= lo && row < hi) {
+      const size_t off = (size_t)row * row_stride + c * 8;
+      cp_async16(kdst + tile_off<D>(rr, c), Kb + off, true);
+      cp_async16(vdst + tile_off<D>(rr, c), Vb + off, true);
+    }
+  }
 }
 
 // ---- attention over rows [r0, r1) for one unit, bf16 tensor-core path --------
@@ -461,6 +489,26 @@ __device__ void merge_warps(const Partial<D> (*w_part)[G], Partial<D>* dst) {
   __syncthreads();
 }
 
+// Readout CTA: cp.async loads of b [r], s_v [D] (moment mode) and, if with_M,
+// M [r][D] of one unit into shared memory, as one commit group.
+template <int D>
+__device__ void stage_readout_state(int unit, int r, const float* __restrict__ bstab,
+                                    const float* __restrict__ s_v, const float* __restrict__ M,
+                                    int moment, bool with_M, float* sb, float* ssv, float* sM) {
+  const int tid = threadIdx.x;
+  for (int i = tid; i < r / 4; i += kThreads)
+    cp_async16(smem_u32(sb) + (uint32_t)i * 16u, bstab + (size_t)unit * r + 4 * i, true);
+  if (moment)
+    for (int i = tid; i < D / 4; i += kThreads)
+      cp_async16(smem_u32(ssv) + (uint32_t)i * 16u, s_v + (size_t)unit * D + 4 * i, true);
+  if (with_M) {
+    const float* Mu = M + (size_t)unit * r * D;
+    for (int i = tid; i < r * D / 4; i += kThreads)
+      cp_async16(smem_u32(sM) + (uint32_t)i * 16u, Mu + 4 * i, true);
+  }
+  cp_async_commit();
+}
+
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch() {
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
@@ -532,6 +580,9 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int Hq = Hkv * G;
   const int unit = bi * Hkv + kh;
+  // per sequence: 1 + the length the last decode step left, 0 if another
+  // call wrote the cache state since (see "Early loads")
+  int* __restrict__ dec_tag = seq_counters + gridDim.z;
 
   __shared__ __align__(16) float s_q[G][D];
   __shared__ float s_w[kDecodeMaxSplits][G];
@@ -568,6 +619,10 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
       cp_async16(smem_u32(sG) + (uint32_t)i * 16u, w_gate + (size_t)kh * G * D + 4 * i, true);
     cp_async_commit();
   }
+  // early b (and s_v) and M, where M has a region of its own: kept if the
+  // check after the wait finds that no other kernel can have changed them
+  const bool ro_early = moment || !kTma;
+  if (rank == S && ro_early) stage_readout_state<D>(unit, r, bstab, s_v, M, moment, true, sb, ssv, sM);
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   const size_t row_stride = (size_t)Hkv * D;
   const T* Kb = K_ret + (size_t)bi * cap * row_stride + (size_t)kh * D;
@@ -579,8 +634,8 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
 #pragma unroll
   for (int b = 0; b < kDecodeMaxStages; ++b) ring.last[b] = -1;
   // A hint of cache_len, read before the wait (relaxed: the previous kernel
-  // may be advancing it). It only picks the rows whose loads are issued
-  // straight after the wait; the true length read after the wait decides.
+  // may be advancing it). It picks this CTA's block under the split the hint
+  // gives; the true length read after the wait decides.
   if (kBf16 && rank < S) {
     if (tid == 0) {
       if (kTma) {
@@ -593,9 +648,35 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     }
     __syncthreads();
   }
+  // Early loads. The first stages of the hinted block (n = hint + 1 or + 2)
+  // are issued before the wait, as far as row hint - 2: the previous decode
+  // step may still be appending row hint - 1 or hint. The remaining rows of
+  // those stages are issued after the wait if the check there accepts them.
+  int len_h = 0, per_h = 0, r0h = 0, blk_h = 0, pre_lim = 0, n_spec = 0, n_full = 0;
+  if constexpr (kBf16) {
+    if (rank < S) {
+      len_h = s_len_hint;
+      per_h = split_rows(len_h + 1, S);
+      r0h = rank * per_h;
+      blk_h = min(min(r0h + per_h, len_h + 2), cap);
+      n_spec = blk_h > r0h ? min(nst, (blk_h - r0h + kStageRows - 1) / kStageRows) : 0;
+      if constexpr (!kTma) {
+        pre_lim = min(blk_h, max(r0h, len_h - 1));
+        for (int st = 0; st < n_spec; ++st) {
+          const int a = r0h + st * kStageRows, e = min(a + kStageRows, blk_h);
+          if (a >= pre_lim) break;
+          ring_issue_rows<D>(ring, Kb, Vb, row_stride, st, a, a, min(e, pre_lim));
+          if (e > pre_lim) break;   // the stage holding row pre_lim stays an open group
+          cp_async_commit();
+          ++n_full;
+        }
+      }
+    }
+  }
   // With programmatic dependent launch this kernel may start while the
   // previous kernel of the stream is still running: wait for it before
-  // reading anything another kernel may write (q, the cache, cache_len, M, b).
+  // relying on anything another kernel may write (q, the cache, cache_len,
+  // M, b).
   griddep_wait();
   // this step's own inputs first (q, cache_len), so that their loads do not
   // queue behind the row loads issued next
@@ -608,25 +689,13 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     for (int e = 0; e < (int)(sizeof(T) / 2); ++e) qraw[e] = __ldcg(qs + e);
   }
   const int len = __ldcg(cache_len + bi);
-  int len_h = 0, per_h = 0, n_spec = 0;
-  if constexpr (kBf16) {
-    if (rank < S) {
-      // the first stages of this CTA's block under the split of the hinted
-      // length (n = hint + 1 or + 2), issued before the true length is known
-      len_h = s_len_hint;
-      per_h = split_rows(len_h + 1, S);
-      const int r0h = rank * per_h;
-      const int hi_h = min(min(r0h + per_h, len_h + 2), cap);
-      n_spec = hi_h > r0h ? min(nst, (hi_h - r0h + kStageRows - 1) / kStageRows) : 0;
-      for (int st = 0; st < n_spec; ++st) {
-        if constexpr (kTma) {
-          if (tid == 0)
-            ring_issue<D>(ring, &tmK, &tmV, st, kh * D, bi * cap + r0h + st * kStageRows, err);
-        } else {
-          ring_issue_lsu<D>(ring, Kb, Vb, row_stride, st, r0h + st * kStageRows, hi_h);
-        }
-      }
-    }
+  const int tag = __ldcg(dec_tag + bi);
+  if constexpr (kBf16 && kTma) {
+    // TMA staging issues its early stages only now (one thread, few
+    // instructions): the first stages of the hinted block
+    if (rank < S && tid == 0)
+      for (int st = 0; st < n_spec; ++st)
+        ring_issue<D>(ring, &tmK, &tmV, st, kh * D, bi * cap + r0h + st * kStageRows, err);
   }
   if (qv) {
     float f[8];
@@ -637,7 +706,8 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   if (len >= cap) {   // full cache: the whole cluster (same sequence) skips it
     if (rank == 0 && kh == 0 && tid == 0) record_error(err, DEV_CACHE_FULL);
     if (kTma && tid == 0) ring_drain<D>(ring, err);
-    if (!kTma) cp_async_wait<0>();
+    cp_async_commit();   // closes an open group of early rows
+    cp_async_wait<0>();
     return;
   }
   // phase 0 of the cluster barrier: "this CTA is running and has read
@@ -649,12 +719,31 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   cluster_arrive_relaxed();
   griddep_launch();
   const int n = len + 1;
-  // the early stages are this CTA's first stages if the true length gives
-  // the same split (and, for cp.async, needs no row past the ones loaded)
-  const bool hit = split_rows(n, S) == per_h && (kTma || len <= len_h + 1);
-  if (!kTma && !hit && n_spec > 0) {
-    cp_async_wait<0>();   // drop them; the barrier below frees the buffers
-    n_spec = 0;
+  // The early stages are this CTA's first stages if the true length gives the
+  // same split. Rows loaded before the wait also need that no kernel which
+  // may have been running then wrote them: tag == len + 1 says that the last
+  // writer of this sequence's cache state was a decode step that left this
+  // length (every other call of the library clears the tag), and the hint is
+  // then len or len - 1, so those rows lie below the row that step appended.
+  bool hit = split_rows(n, S) == per_h;
+  if constexpr (!kTma) {
+    hit = hit && tag == len + 1 && (len_h == len || len_h + 1 == len);
+    if constexpr (kBf16) {
+      if (rank < S && n_spec > 0) {
+        if (hit) {
+          // the rest of the early stages: from row pre_lim to the block's end
+          for (int st = n_full; st < n_spec; ++st) {
+            const int a = r0h + st * kStageRows, e = min(a + kStageRows, blk_h);
+            ring_issue_rows<D>(ring, Kb, Vb, row_stride, st, a, max(a, pre_lim), e);
+            cp_async_commit();
+          }
+        } else {
+          cp_async_commit();   // closes an open group
+          cp_async_wait<0>();  // drop them; the barrier below frees the buffers
+          n_spec = 0;
+        }
+      }
+    }
   }
   __syncthreads();
 
@@ -692,24 +781,17 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     if (rank == 0 && tid == 0 && arrived == Hkv - 1) {
       seq_counters[bi] = 0;
       cache_len[bi] = len + 1;
+      dec_tag[bi] = len + 2;
     }
     return;
   }
 
   // ---- readout CTA: u = W_phi q, m = M^T u / (b.u + eps), g = sigmoid(w_gate . q)
-  {
-    // b (and s_v) and the whole of M, in flight together
-    for (int i = tid; i < r / 4; i += kThreads)
-      cp_async16(smem_u32(sb) + (uint32_t)i * 16u, bstab + (size_t)unit * r + 4 * i, true);
-    if (moment)
-      for (int i = tid; i < D / 4; i += kThreads)
-        cp_async16(smem_u32(ssv) + (uint32_t)i * 16u, s_v + (size_t)unit * D + 4 * i, true);
-    if (moment || !kTma) {
-      const float* Mu = M + (size_t)unit * r * D;
-      for (int i = tid; i < r * D / 4; i += kThreads)
-        cp_async16(smem_u32(sM) + (uint32_t)i * 16u, Mu + 4 * i, true);
-    }
-    cp_async_commit();
+  if (!ro_early || tag != len + 1) {
+    // b (and s_v) and, where it has its own region, M: loaded now (the early
+    // copies, if any, land first and are overwritten)
+    if (ro_early) cp_async_wait<0>();
+    stage_readout_state<D>(unit, r, bstab, s_v, M, moment, ro_early, sb, ssv, sM);
   }
   const float ne = moment ? __ldcg(n_e + bi) : 0.f;
   cp_async_wait<0>();

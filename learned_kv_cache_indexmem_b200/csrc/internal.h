@@ -51,6 +51,7 @@ struct Workspace {
   size_t sel_off;               // selection scratch
   size_t dec_part_off;          // decode split partials
   size_t dec_cnt_off;           // decode counters (int), zero between calls
+  size_t dec_tag_off;           // decode tags (int): right after the counters
   size_t on_qpart_off, on_kpart_off, on_cand_off, on_cnt_off, on_slot_off;   // online eviction
   size_t mem_part_off;          // memory-update partials
   size_t sv_part_off;           // value-sum partials of the moment statistics
@@ -118,7 +119,7 @@ cudaError_t launch_online_evict(const Ctx& c, int batch, int B, int cap, const f
                                 const float* kpart, void* khat_ret, float* I_ret, int32_t* pos_ret,
                                 int32_t* next_pos, void* K_ret, void* V_ret, int32_t* cache_len,
                                 float* M, float* bstab, int32_t* evicted, void* cand,
-                                int* counter, int* evict_slot, cudaStream_t st);
+                                int* counter, int* evict_slot, int* dec_tag, cudaStream_t st);
 
 // A kernel whose bounded wait runs out after `limit` cycles (failure-path test).
 cudaError_t launch_wait_selftest(const Ctx& c, long long limit, cudaStream_t st);

@@ -20,7 +20,9 @@
 //             last-CTA reduction;
 //   evict     per KV head: phi = W_phi k_e, M <- lambda M + phi v_e^T,
 //             b <- lambda b + phi; the new token's row moves into the freed
-//             slot; cache_len returns to B.
+//             slot; cache_len returns to B and the workspace's decode tag
+//             of the sequence to B + 1 (the next decode step may then use
+//             the rows it loads before its launch-dependency wait).
 // q~ and k^ are rounded to bf16 before their dot products, as in prefill.
 #include "common.cuh"
 #include "internal.h"
@@ -298,7 +300,7 @@ online_evict_kernel(int B, int cap, int Hkv, int D, int r, float lambda,
                     __nv_bfloat16* __restrict__ khat_ret, float* __restrict__ I_ret,
                     int32_t* __restrict__ pos_ret, int32_t* __restrict__ next_pos,
                     int32_t* __restrict__ cache_len, float* __restrict__ M,
-                    float* __restrict__ bstab) {
+                    float* __restrict__ bstab, int* __restrict__ dec_tag) {
   extern __shared__ float osm[];
   float* sk = osm;          // [D]
   float* sv = sk + D;       // [D]
@@ -362,6 +364,7 @@ online_evict_kernel(int B, int cap, int Hkv, int D, int r, float lambda,
         pos_ret[(size_t)bi * cap + e] = pos_ret[(size_t)bi * cap + B];
       }
       cache_len[bi] = B;
+      dec_tag[bi] = B + 1;   // the next decode step may use rows it loads before its wait
       next_pos[bi] += 1;
     }
   }
@@ -418,7 +421,7 @@ cudaError_t launch_online_evict(const Ctx& c, int batch, int B, int cap, const f
                                 const float* kpart, void* khat_ret, float* I_ret, int32_t* pos_ret,
                                 int32_t* next_pos, void* K_ret, void* V_ret, int32_t* cache_len,
                                 float* M, float* bstab, int32_t* evicted, void* cand,
-                                int* counter, int* evict_slot, cudaStream_t st) {
+                                int* counter, int* evict_slot, int* dec_tag, cudaStream_t st) {
   const int nct = online_score_ctas(B);
   const int rows_per_cta = (B + 1 + nct - 1) / nct;
   cudaError_t e = launch_pdl(online_score_kernel, dim3(nct, batch), 0, st, B, cap,
@@ -432,10 +435,10 @@ cudaError_t launch_online_evict(const Ctx& c, int batch, int B, int cap, const f
   if (c.cfg.dtype == IMEM_BF16)
     return launch_pdl(online_evict_kernel<__nv_bfloat16>, g, sm, st, B, cap, Hkv, D, r,
                       c.cfg.lambda, evict_slot, c.W_phi, K_ret, V_ret, khat_ret, I_ret, pos_ret,
-                      next_pos, cache_len, M, bstab);
+                      next_pos, cache_len, M, bstab, dec_tag);
   return launch_pdl(online_evict_kernel<float>, g, sm, st, B, cap, Hkv, D, r, c.cfg.lambda,
                     evict_slot, c.W_phi, K_ret, V_ret, khat_ret, I_ret, pos_ret, next_pos,
-                    cache_len, M, bstab);
+                    cache_len, M, bstab, dec_tag);
 }
 
 }  // namespace imem

@@ -172,6 +172,13 @@ class IndexMemLayer:
             B_.update_memory(self.ctx, batch, L, K, V, idx, L - B, chunk, st.M, st.bstab, ws,
                              stream)
 
+    def invalidate_decode(self, batch: int, stream=None):
+        """After writing a retained cache, its length or the memory state
+        other than through this layer: the next decode step then loads
+        nothing before its launch-dependency wait."""
+        if self._ws is not None:
+            B_.decode_invalidate(self.ctx, batch, self._ws, stream)
+
     def decode(self, q, k_new, v_new, st: PrefillState, out=None, B: Optional[int] = None,
                L: Optional[int] = None, stream=None):
         batch = q.shape[0]

@@ -92,6 +92,7 @@ def test_null_context_is_invalid_for_every_call():
     assert lib.imem_decode_online(None, 1, 4, 16, 16, 16, 16, 16, 16, 16, 16, 16, 16, 16, 8, 16,
                                   16, 16, 16, 16, None) == 1
     assert lib.imem_selftest_wait(None, 1000, None) == 1
+    assert lib.imem_decode_invalidate(None, 1, 16, None) == 1
     assert lib.imem_update_moments(None, 1, 16, 16, 16, 16, 4, 64, 16, 16, 16, 16, 16, None) == 1
     assert lib.imem_decode_moment(None, 1, 16, 16, 16, 16, 16, 16, 8, 16, 16, 16, 16, 16, 16,
                                   None) == 1
