@@ -34,11 +34,12 @@
 // (the rows then predate the previous kernel, and b and M are unchanged);
 // otherwise they are dropped and loaded again.
 //
-// bf16 attention: rows are staged in shared memory with cp.async (a ring of
-// two or three 64-row stages, XOR-swizzled 16-byte chunks) and contracted
-// with warp-level tensor-core MMA (m16n8k16, fp32 accumulation): S^T = q K^T
-// with the GQA heads as the M dimension, then O += P V reusing the score
-// fragments as the A operand. fp32 attention: CUDA cores.
+// bf16 attention: rows are staged in shared memory (a ring of two or three
+// 64-row stages, XOR-swizzled 16-byte chunks) and contracted with warp-level
+// tensor-core MMA (m16n8k16, fp32 accumulation) with the cache rows on M and
+// the GQA heads on N: S = K q^T, then O^T += V^T P, V^T read with transposing
+// shared-memory loads and P turned into the B operand by an in-register 8x8
+// transpose. A warp's 16 rows cost 2 x D/16 MMAs. fp32 attention: CUDA cores.
 #include "common.cuh"
 #include "internal.h"
 #include "tc.cuh"
@@ -93,14 +94,20 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
 }
-// D = A(16x16, rows 8..15 zero) * B(16x8) + C
-__device__ __forceinline__ void mma_bf16(float* c, uint32_t a0, uint32_t a2, uint32_t b0,
-                                         uint32_t b1) {
+// D = A(16x16) * B(16x8) + C with all four A registers
+__device__ __forceinline__ void mma_bf16_a4(float* c, uint32_t a0, uint32_t a1, uint32_t a2,
+                                            uint32_t a3, uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};\n"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// transpose of an 8x8 matrix of 16-bit pairs held one pair per lane
+__device__ __forceinline__ uint32_t movm_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
 }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -228,21 +235,25 @@ __device__ void attend_bf16(Ring& rg, const CUtensorMap* tmK, const CUtensorMap*
   const float sscale = kLog2e * rsqrtf((float)D);
   const int nst = rg.nst;
 
-  // q as A fragments (heads on M, rows >= G zero): a0 = dims 16s+2t.., a2 = +8
-  uint32_t qa0[D / 16], qa2[D / 16];
+  // Cache rows on the MMA's M dimension, the GQA heads on N (8 columns,
+  // heads >= G zero): S[row][head] = K q^T, then O^T[dim][head] += V^T P.
+  // q as B fragments: b0 = dims 16s+2t.., b1 = +8, column g = head g
+  uint32_t qb0[D / 16], qb1[D / 16];
 #pragma unroll
   for (int s = 0; s < D / 16; ++s) {
     if (g < G) {
-      qa0[s] = pack_bf16(s_q[g][16 * s + 2 * t], s_q[g][16 * s + 2 * t + 1]);
-      qa2[s] = pack_bf16(s_q[g][16 * s + 8 + 2 * t], s_q[g][16 * s + 8 + 2 * t + 1]);
+      qb0[s] = pack_bf16(s_q[g][16 * s + 2 * t], s_q[g][16 * s + 2 * t + 1]);
+      qb1[s] = pack_bf16(s_q[g][16 * s + 8 + 2 * t], s_q[g][16 * s + 8 + 2 * t + 1]);
     } else {
-      qa0[s] = 0u; qa2[s] = 0u;
+      qb0[s] = 0u; qb1[s] = 0u;
     }
   }
-  float o[D / 8][4];
+  // O^T accumulators: o[mt] = dims 16mt+g (0, 1) and +8 (2, 3), heads 2t, 2t+1
+  float o[D / 16][4];
 #pragma unroll
-  for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-  float m_run = -INFINITY, l_run = 0.f;
+  for (int j = 0; j < D / 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  // running max and this lane's share of the normaliser, heads 2t and 2t+1
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
 
   const int n_stages = (r1 - r0 + kStageRows - 1) / kStageRows;
   int issued = max(n_pre, min(n_stages, nst));   // stages issued so far (cp.async groups)
@@ -287,57 +298,62 @@ __device__ void attend_bf16(Ring& rg, const CUtensorMap* tmK, const CUtensorMap*
         if constexpr (kTma) tc::fence_proxy_async();   // generic writes before the next TMA load
         __syncwarp();
       }
-      // scores S^T[head][row] for rows kb..kb+15 as two 8-row n-tiles
-      float sc[2][4];
+      // scores S[row][head] for rows kb..kb+15: one 16-row A tile per 16
+      // dims (two accumulators, even and odd steps, for independent chains)
+      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        const int rr = warp * 16 + (lane & 15);
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-        const int rr = warp * 16 + nt * 8 + (lane & 7);
-#pragma unroll
-        for (int p = 0; p < D / 32; ++p) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(kt + tile_off<D>(rr, 4 * p + (lane >> 3)), b0, b1, b2, b3);
-          mma_bf16(sc[nt], qa0[2 * p], qa2[2 * p], b0, b1);
-          mma_bf16(sc[nt], qa0[2 * p + 1], qa2[2 * p + 1], b2, b3);
+        for (int s2 = 0; s2 < D / 16; ++s2) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(kt + tile_off<D>(rr, 2 * s2 + (lane >> 4)), a0, a1, a2, a3);
+          if (s2 & 1) mma_bf16_a4(sb, a0, a1, a2, a3, qb0[s2], qb1[s2]);
+          else mma_bf16_a4(sa, a0, a1, a2, a3, qb0[s2], qb1[s2]);
         }
       }
-      // mask, scale, block max per head (lanes of a head: xor 1, 2)
-      float mx = -INFINITY;
+      // mask rows past r1, scale; sc[0..1]: row kb+g, sc[2..3]: row kb+g+8
+      float sc[4];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int e = 0; e < 4; ++e) {
+        const int row = kb + g + ((e >> 1) << 3);
+        sc[e] = (row < r1) ? (sa[e] + sb[e]) * sscale : -INFINITY;
+      }
+      // block max per head over the 16 rows (lanes of a head: same t)
+      float mx[2] = {fmaxf(sc[0], sc[2]), fmaxf(sc[1], sc[3])};
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int row = kb + nt * 8 + 2 * t + e;
-          const float v = (row < r1) ? sc[nt][e] * sscale : -INFINITY;
-          sc[nt][e] = v;
-          mx = fmaxf(mx, v);
-        }
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      const float m_new = fmaxf(m_run, mx);
-      const float corr = (m_run == -INFINITY) ? 0.f : exp2f(m_run - m_new);
-      float p[2][2], psum = 0.f;
+      for (int off = 4; off < 32; off <<= 1) {
+        mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], off));
+        mx[1] = fmaxf(mx[1], __shfl_xor_sync(0xffffffffu, mx[1], off));
+      }
+      float corr[2];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int h = 0; h < 2; ++h) {
+        const float m_new = fmaxf(m_run[h], mx[h]);
+        corr[h] = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - m_new);
+        m_run[h] = m_new;
+      }
+      float p[4];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          p[nt][e] = (sc[nt][e] == -INFINITY) ? 0.f : exp2f(sc[nt][e] - m_new);
-          psum += p[nt][e];
-        }
-      l_run = l_run * corr + psum;
-      m_run = m_new;
+      for (int e = 0; e < 4; ++e) p[e] = (sc[e] == -INFINITY) ? 0.f : exp2f(sc[e] - m_run[e & 1]);
+      l_run[0] = l_run[0] * corr[0] + (p[0] + p[2]);
+      l_run[1] = l_run[1] * corr[1] + (p[1] + p[3]);
 #pragma unroll
-      for (int j = 0; j < D / 8; ++j) { o[j][0] *= corr; o[j][1] *= corr; }
-      const uint32_t pa0 = pack_bf16(p[0][0], p[0][1]);
-      const uint32_t pa2 = pack_bf16(p[1][0], p[1][1]);
-      // O[head][dims] += P V over the 16 rows
-      const int rr = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+      for (int j = 0; j < D / 16; ++j) {
+        o[j][0] *= corr[0]; o[j][1] *= corr[1];
+        o[j][2] *= corr[0]; o[j][3] *= corr[1];
+      }
+      // P as the B operand (rows on K, heads on N): transpose the two 8x8
+      // blocks of the score fragment (rows 0-7, rows 8-15)
+      const uint32_t pb0 = movm_trans(pack_bf16(p[0], p[1]));
+      const uint32_t pb1 = movm_trans(pack_bf16(p[2], p[3]));
+      // O^T[dims][head] += V^T P: V^T as A tiles (16 dims x 16 rows) from the
+      // row-major V stage with transposing loads
+      const int rv = warp * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
 #pragma unroll
-      for (int q2 = 0; q2 < D / 16; ++q2) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(vt + tile_off<D>(rr, 2 * q2 + (lane >> 4)), b0, b1, b2, b3);
-        mma_bf16(o[2 * q2], pa0, pa2, b0, b1);
-        mma_bf16(o[2 * q2 + 1], pa0, pa2, b2, b3);
+      for (int mt = 0; mt < D / 16; ++mt) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_t(vt + tile_off<D>(rv, 2 * mt + ((lane >> 3) & 1)), a0, a1, a2, a3);
+        mma_bf16_a4(o[mt], a0, a1, a2, a3, pb0, pb1);
       }
     }
     __syncthreads();   // buffer b consumed by every warp
@@ -359,15 +375,22 @@ __device__ void attend_bf16(Ring& rg, const CUtensorMap* tmK, const CUtensorMap*
     cp_async_wait<0>();
   }
   __syncthreads();
-  // per-lane partial sums of the head's normaliser -> full sum over the quad
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
-  if (g < G) {
-    if (t == 0) { s_part[warp][g].m = m_run; s_part[warp][g].l = l_run; }
+  // per-lane shares of each head's normaliser -> the sum over its 8 lanes
 #pragma unroll
-    for (int j = 0; j < D / 8; ++j) {
-      s_part[warp][g].o[8 * j + 2 * t] = o[j][0];
-      s_part[warp][g].o[8 * j + 2 * t + 1] = o[j][1];
+  for (int off = 4; off < 32; off <<= 1) {
+    l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
+    l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int head = 2 * t + h;
+    if (head < G) {
+      if (g == 0) { s_part[warp][head].m = m_run[h]; s_part[warp][head].l = l_run[h]; }
+#pragma unroll
+      for (int j = 0; j < D / 16; ++j) {
+        s_part[warp][head].o[16 * j + g] = o[j][h];
+        s_part[warp][head].o[16 * j + g + 8] = o[j][2 + h];
+      }
     }
   }
 }
