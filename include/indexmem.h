@@ -332,6 +332,10 @@ imem_status imem_prefill_evict_chunk(imem_ctx* ctx, int batch, int L, int B, int
  *      out) receives its position;
  *   4. the new token takes the freed slot (nothing moves if it left itself);
  *      cache_len returns to B; next_pos advances.
+ * Ordering as imem_decode: step 4 also sets the workspace's decode tag for
+ * cache length B, so the next step's attention may use the rows it loads
+ * before its launch-dependency wait. imem_online_init does not write the
+ * cache state and leaves the tag as it is.
  * Errors: as imem_decode; UNSUPPORTED for the moment readout. */
 imem_status imem_online_init(imem_ctx* ctx, int batch, int L, int B, const float* running_max,
                              const int32_t* idx_retained, const void* workspace, void* khat_ret,
