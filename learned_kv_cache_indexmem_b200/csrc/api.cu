@@ -19,7 +19,6 @@ struct imem_ctx {
 
 namespace imem {
 
-int decode_splits(int batch, int n_kv_heads, int cap);
 int memory_groups(int batch, int n_kv_heads, int n_e, int chunk);
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }

@@ -153,6 +153,7 @@ def _decode_case(case, cap, lens, gate_override=None):
     ("c1", 1, [410], 410 + 256, 256),
     ("c1", 3, [410, 37, 1], 420, 8),        # ragged cache lengths
     ("c1", 2, [2000, 1500], 2100, 4),       # several splits
+    ("c1", 4, [128, 100, 60, 1], 640, 8),   # short ragged caches, 4 splits
 ])
 def test_decode_parity(cuda_device, name, batch, lens, cap, steps):
     L = max(max(lens), 64)
