@@ -19,8 +19,10 @@
 //             packed (ordered importance, inverted position) key and a
 //             last-CTA reduction;
 //   evict     per KV head: phi = W_phi k_e, M <- lambda M + phi v_e^T,
-//             b <- lambda b + phi; the new token's row moves into the freed
-//             slot; cache_len returns to B and the workspace's decode tag
+//             b <- lambda b + phi; the new token and the evicted one swap
+//             slots (row, indexer key, importance, position), so slot B keeps
+//             the token that left with the importance it was chosen by;
+//             cache_len returns to B and the workspace's decode tag
 //             of the sequence to B + 1 (the next decode step may then use
 //             the rows it loads before its launch-dependency wait).
 // q~ and k^ are rounded to bf16 before their dot products, as in prefill.
@@ -348,20 +350,33 @@ online_evict_kernel(int B, int cap, int Hkv, int D, int r, float lambda,
     float* bp = bstab + ((size_t)bi * Hkv + kh) * r + j;
     *bp = fmaf(lambda, *bp, sphi[j]);
   }
-  if (e != B) {   // the new token (slot B) takes the freed slot
-    const T* kn = K_ret + ((size_t)bi * cap + B) * rs + (size_t)kh * D;
-    const T* vn = V_ret + ((size_t)bi * cap + B) * rs + (size_t)kh * D;
-    for (int c = tid; c < D; c += kOnThreads) { ke[c] = kn[c]; ve[c] = vn[c]; }
+  if (e != B) {   // the new token (slot B) and the evicted one swap slots
+    T* kn = K_ret + ((size_t)bi * cap + B) * rs + (size_t)kh * D;
+    T* vn = V_ret + ((size_t)bi * cap + B) * rs + (size_t)kh * D;
+    for (int c = tid; c < D; c += kOnThreads) {
+      const T k0 = ke[c], v0 = ve[c];
+      ke[c] = kn[c]; ve[c] = vn[c];
+      kn[c] = k0; vn[c] = v0;
+    }
   }
   if (kh == 0 && tid < kIdxPad / 8) {
     if (e != B) {
-      reinterpret_cast<uint4*>(khat_ret + ((size_t)bi * cap + e) * kIdxPad)[tid] =
-          reinterpret_cast<const uint4*>(khat_ret + ((size_t)bi * cap + B) * kIdxPad)[tid];
+      uint4* he = reinterpret_cast<uint4*>(khat_ret + ((size_t)bi * cap + e) * kIdxPad) + tid;
+      uint4* hn = reinterpret_cast<uint4*>(khat_ret + ((size_t)bi * cap + B) * kIdxPad) + tid;
+      const uint4 h0 = *he;
+      *he = *hn;
+      *hn = h0;
     }
     if (tid == 0) {
       if (e != B) {
-        I_ret[(size_t)bi * cap + e] = I_ret[(size_t)bi * cap + B];
-        pos_ret[(size_t)bi * cap + e] = pos_ret[(size_t)bi * cap + B];
+        float* Ie = I_ret + (size_t)bi * cap + e;
+        float* In = I_ret + (size_t)bi * cap + B;
+        int32_t* pe = pos_ret + (size_t)bi * cap + e;
+        int32_t* pn = pos_ret + (size_t)bi * cap + B;
+        const float I0 = *Ie;
+        const int32_t p0 = *pe;
+        *Ie = *In; *pe = *pn;
+        *In = I0; *pn = p0;
       }
       cache_len[bi] = B;
       dec_tag[bi] = B + 1;   // the next decode step may use rows it loads before its wait

@@ -9,6 +9,11 @@ the correctness criteria state:
   decode   |do| <= 1e-2 + 2e-2 |o_ref| elementwise; readouts whose denominator
            is ill-conditioned (|b.u| < 1e-4 ||b|| ||u||) are excluded (at most
            0.1% of them), their attention part is checked by a gate-0 run.
+
+Where the GPU path takes a decision or produces a state that a later stage
+consumes (the retained set from its scores, the memory state M, b that decode
+reads), the oracle's later stage is run on the GPU's own decision or state,
+and that decision or state is checked separately at its own tolerance.
 """
 from __future__ import annotations
 
@@ -61,31 +66,9 @@ def ill_conditioned(bstab, q, W_phi, group):
     return dot < ILL_COND * np.linalg.norm(bk, axis=-1) * np.linalg.norm(u, axis=-1)
 
 
-def propagated_allowance(q, M_ref, b_ref, dM, db, W_phi, w_gate, group, gate_override=None):
-    """Per-readout bound on how far an admissible memory state moves the output.
-    The readout m = M^T u / (b.u + eps) is first-order sensitive to a state error
-    (dM, db) as |dm| <= (||dM||_F ||u|| + ||m|| ||db|| ||u||) / |b.u + eps|; with
-    the gate g in [0, 1] the output moves by at most g times that. Returned as
-    2x the bound (second-order slack), shape [b, Hq, 1]."""
-    u = np.einsum("rd,bhd->bhr", W_phi, q)
-    Mk = np.repeat(M_ref, group, axis=1)
-    bk = np.repeat(b_ref, group, axis=1)
-    den = np.sum(bk * u, -1) + 1e-6
-    m = np.einsum("bhrd,bhr->bhd", Mk, u) / den[..., None]
-    nu = np.linalg.norm(u, axis=-1)
-    ndM = np.repeat(np.sqrt(np.sum(dM ** 2, axis=(-1, -2))), group, axis=1)
-    ndb = np.repeat(np.linalg.norm(db, axis=-1), group, axis=1)
-    bound = (ndM * nu + np.linalg.norm(m, axis=-1) * ndb * nu) / np.abs(den)
-    g = 1.0 / (1.0 + np.exp(-np.einsum("hd,bhd->bh", w_gate, q))) if gate_override is None \
-        else np.full(bound.shape, gate_override)
-    return (2.0 * g * bound)[..., None]
-
-
-def check_decode(o_gpu, o_ref, mask_ill=None, what="", extra=None):
+def check_decode(o_gpu, o_ref, mask_ill=None, what=""):
     o_gpu = np.asarray(o_gpu, np.float64)
     tol = DEC_ATOL + DEC_RTOL * np.abs(o_ref)
-    if extra is not None:
-        tol = tol + extra
     bad = np.abs(o_gpu - o_ref) > tol
     if mask_ill is not None:
         frac = mask_ill.mean()

@@ -1,9 +1,11 @@
 """Decode-time online eviction ("IndexMem" technical summary §2.B, memory
 updated online during inference; §2.A, pooled importance) through the C ABI
 against the oracle, step by step from the GPU's own state before each step:
-the output, the importances carried, the evicted token (the oracle's choice
-or a near-tie within the score tolerance), the memory updated with it, and
-the cache rows after the move."""
+the output; the B + 1 candidates' importances the GPU used (slot B keeps the
+token that left) against the oracle's within the score tolerance; the evicted
+token bit-exactly as the least important of those importances (ties: the
+higher position leaves); the memory updated with it; and the cache rows after
+the move."""
 import math
 
 import numpy as np
@@ -57,8 +59,8 @@ def test_online_eviction_parity(cuda_device, name, L, B, steps, batch):
         what = "%s step %d" % (name, i)
         check_decode(to_np(out), o_ref, ill_conditioned(pre["b"], qc, W_phi, group), what)
         ev = to_np(on.evicted).astype(np.int64)
-        pos_after = to_np(on.pos_ret).astype(np.int64)
-        I_after = to_np(on.I_ret)
+        pos_after = on.pos_ret.cpu().numpy().astype(np.int64)
+        I_after = on.I_ret.cpu().numpy()                 # float32, as the GPU compared them
         # the oracle's importances of the B + 1 candidates from the GPU's state
         qh, kh_new, g = om.indexer_features(xc[:, None], qc[:, None], w["W_iq"], w["W_ik"],
                                             w["w_ig"])
@@ -69,19 +71,24 @@ def test_online_eviction_parity(cuda_device, name, L, B, steps, batch):
                 np.maximum(pre["I"][bi, :B], pre["kh"][bi, :B, :s.idx_dim] @ qt[bi]),
                 [kh_new[bi, 0] @ qt[bi]]])
             scale = max(np.abs(I_cand).max(), math.sqrt(np.mean(I_cand ** 2)))
-            # the evicted token is the least important (a near-tie may differ)
-            j_gpu = cand_pos.index(ev[bi])
-            assert I_cand[j_gpu] <= I_cand.min() + SCORE_TOL * scale, "%s: eviction" % what
-            if ev[bi] != ev_ref[bi]:
-                j_ref = cand_pos.index(ev_ref[bi])
-                assert abs(I_cand[j_gpu] - I_cand[j_ref]) <= SCORE_TOL * scale, what
-            # the cache after the move: the candidates minus the evicted one
-            assert sorted(pos_after[bi, :B]) == sorted(set(cand_pos) - {ev[bi]}), what
-            for j in range(B):
+            # slots [0, B] after the step are the step's B + 1 candidates, slot B
+            # the one that left
+            assert sorted(pos_after[bi, :B + 1]) == sorted(cand_pos), what
+            assert pos_after[bi, B] == ev[bi], what
+            for j in range(B + 1):
+                p = pos_after[bi, j]
+                assert abs(float(I_after[bi, j]) - I_cand[cand_pos.index(p)]) <= \
+                    SCORE_TOL * scale, "%s: importance of %d" % (what, p)
+            # the eviction, bit-exact on the GPU's importances: the least
+            # important leaves, ties to the higher position (-0 == +0)
+            Ig = I_after[bi, :B + 1].astype(np.float32) + np.float32(0.0)
+            low = np.flatnonzero(Ig == Ig.min())
+            assert ev[bi] == pos_after[bi, low].max(), "%s: eviction" % what
+            # the cache after the move: rows by position, slot B the evicted row
+            for j in range(B + 1):
                 p = pos_after[bi, j]
                 assert np.array_equal(to_np(st.K_ret[bi, j]), K_all[bi, p]), what
                 assert np.array_equal(to_np(st.V_ret[bi, j]), V_all[bi, p]), what
-                assert abs(I_after[bi, j] - I_cand[cand_pos.index(p)]) <= SCORE_TOL * scale, what
         # the memory: the state before the step updated with the GPU's choice
         E = np.array([[ev[bi]] for bi in range(batch)])
         M_ref, b_ref = om.memory_update(case.in_cpu["K"], case.in_cpu["V"], E, W_phi, s.lam,
