@@ -12,6 +12,9 @@ enum DeviceError : int {
   DEV_OK = 0,
   DEV_TIMEOUT = 1,     // a bounded wait on an mbarrier ran out
   DEV_CACHE_FULL = 2,  // decode into a cache whose cache_len >= cap
+  DEV_RANGE = 3,       // an input value outside what the kernel computes with:
+                       // an evicted index outside [0, L), or a key or weighted
+                       // value beyond the fp16 range of the memory operands
 };
 
 __device__ __forceinline__ void record_error(int* err, int code) {

@@ -13,16 +13,23 @@
 // independently and W_phi is applied once at the end.
 //
 // Pass 1 (tensor cores): grid (groups, Hkv, batch); a CTA gathers the rows of
-// one run of evicted tokens for one (sequence, KV head) and accumulates
-//   [S | s] (d x (d+1)) += K_c^T [w*V_c | w]
-// in tensor memory with tcgen05.mma over 64-token chunks. Operands are fp16
-// (bf16 keys convert exactly; w*v is rounded once to fp16) with fp32
-// accumulation; both are MN-major in shared memory (a token is one 128-byte
-// row per 64 features, so gathered rows are written as they arrive). Eight
-// loader warps gather, convert and write the chunks; one thread issues the
-// MMAs; a double-buffered mbarrier ring keeps them in step.
+// one run [j0, j1) of evicted tokens for one (sequence, KV head) and
+// accumulates
+//   [S_g | s_g] (d x (d+1)) = K_c^T [w*V_c | w],  w_i = lambda^(j1-1-i)
+// in tensor memory with tcgen05.mma over 64-token chunks. The weights are
+// relative to the end of the run (the run's factor lambda^(n-j1) is applied
+// in fp32 by pass 2), so they stay far from fp16's subnormal range for runs
+// of moderate length. Operands are fp16 (bf16 keys convert exactly within
+// fp16's range; w*v is rounded once to fp16) with fp32 accumulation; a key or
+// weighted value beyond that range (|x| > 65504) is reported as DEV_RANGE.
+// Both operands are MN-major in shared memory (a token is one 128-byte row per
+// 64 features, so gathered rows are written as they arrive). Eight loader
+// warps gather, convert and write the chunks; one thread issues the MMAs; a
+// double-buffered mbarrier ring keeps them in step. An evicted index outside
+// [0, L) reads no row and is reported as DEV_RANGE.
 // Pass 2 (CUDA cores): per (sequence, KV head, 16 columns) sums the runs in a
-// fixed order (deterministic) and applies M = lambda^n M0 + W_phi S.
+// fixed order (deterministic), each scaled by its factor, and applies
+// M = lambda^n M0 + W_phi S.
 #include "common.cuh"
 #include "internal.h"
 #include "tc.cuh"
@@ -157,7 +164,12 @@ memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t
 #pragma unroll
       for (int it = 0; it < ITEMS; ++it) {
         const int j = j0 + c * kChunk + (tid + it * kLoaders) / CH;
-        pos[it] = (c < nchunks && j < j1) ? __ldg(E + j) : -1;
+        int p = (c < nchunks && j < j1) ? __ldg(E + j) : -1;
+        if (p >= L || (p < 0 && c < nchunks && j < j1)) {   // no row to read
+          record_error(err, DEV_RANGE);
+          p = -1;
+        }
+        pos[it] = p;
       }
     };
     auto load_rows = [&](const int* pos, typename Raw::type* kr, typename Raw::type* vr) {
@@ -204,12 +216,17 @@ memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t
         const int i = tid + it * kLoaders;
         const int jj = i / CH, cc = i % CH;
         const int j = base + jj;
-        const float wv = (j < j1) ? exp2f((float)(n_e - 1 - j) * log2lam) : 0.f;
+        const float wv = (j < j1) ? exp2f((float)(j1 - 1 - j) * log2lam) : 0.f;
         float kf[8], vf[8];
         Raw::to_f32(cur_k[it], kf);
         Raw::to_f32(cur_v[it], vf);
+        float big = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) vf[e] *= wv;
+        for (int e = 0; e < 8; ++e) {
+          vf[e] *= wv;
+          big = fmaxf(big, fmaxf(fabsf(kf[e]), fabsf(vf[e])));
+        }
+        if (big > 65504.f) record_error(err, DEV_RANGE);   // beyond fp16's range
         if constexpr (kSV) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) svacc[e] += vf[e];
@@ -302,18 +319,30 @@ memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t
 // column slice (blockIdx.x == D/16) does b from the s column.
 // With sv_partials, slice D/16 + 1 does the value sums: s_v = decay * s_v +
 // sum_g, and the sequence's count n_e += n_add (KV head 0 of the sequence).
+// Run g covers evicted tokens [g*tpg, min(n, (g+1)*tpg)); its partial sums are
+// weighted relative to its end, so it enters with the factor lambda^(n - end).
+__device__ __forceinline__ float run_factor(int g, int tpg, int n, float log2lam) {
+  const int end = min(n, (g + 1) * tpg);
+  return exp2f((float)(n - end) * log2lam);
+}
+
 template <int D>
 __global__ void __launch_bounds__(256)
-memory_finalize_kernel(const float* __restrict__ partials, int G, const float* __restrict__ W_phi,
+memory_finalize_kernel(const float* __restrict__ partials, int G, int tpg, int n_tok,
+                       float log2lam, const float* __restrict__ W_phi,
                        int r, float decay_n, float* __restrict__ M, float* __restrict__ bstab,
                        const float* __restrict__ sv_partials, float* __restrict__ s_v,
                        float* __restrict__ n_e, float n_add, int Hkv) {
   extern __shared__ float fsm[];
+  __shared__ float s_fac[kMemMaxGroups];
+  for (int gg = threadIdx.x; gg < G; gg += 256) s_fac[gg] = run_factor(gg, tpg, n_tok, log2lam);
+  __syncthreads();
   if (blockIdx.x == D / 16 + 1) {   // value sums (only launched with sv_partials)
     const int unit = blockIdx.y;
     for (int c = threadIdx.x; c < D; c += 256) {
       float a = 0.f;
-      for (int gg = 0; gg < G; ++gg) a += __ldcg(&sv_partials[((size_t)unit * G + gg) * D + c]);
+      for (int gg = 0; gg < G; ++gg)
+        a = fmaf(s_fac[gg], __ldcg(&sv_partials[((size_t)unit * G + gg) * D + c]), a);
       float* sp = s_v + (size_t)unit * D + c;
       *sp = fmaf(*sp, decay_n, a);
     }
@@ -334,7 +363,8 @@ memory_finalize_kernel(const float* __restrict__ partials, int G, const float* _
   for (int i = tid; i < D * ncols; i += 256) {
     const int dk = i / ncols, cc = i % ncols;
     float a = 0.f;
-    for (int gg = 0; gg < G; ++gg) a += __ldcg(&p[((size_t)gg * D + dk) * (D + 1) + col0 + cc]);
+    for (int gg = 0; gg < G; ++gg)
+      a = fmaf(s_fac[gg], __ldcg(&p[((size_t)gg * D + dk) * (D + 1) + col0 + cc]), a);
     sS[dk * 16 + cc] = a;
   }
   __syncthreads();
@@ -410,13 +440,15 @@ cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, 
   if (D == 128) {
     e = cudaFuncSetAttribute(memory_finalize_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem);
     if (e != cudaSuccess) return e;
-    memory_finalize_kernel<128><<<fgrid, 256, fsmem, st>>>(partials, Gused, phi, r, decay_n, M,
+    memory_finalize_kernel<128><<<fgrid, 256, fsmem, st>>>(partials, Gused, tokens_per_group,
+                                                           n_e, log2lam, phi, r, decay_n, M,
                                                            bstab, sv_partials, s_v, n_count,
                                                            (float)n_e, Hkv);
   } else {
     e = cudaFuncSetAttribute(memory_finalize_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem);
     if (e != cudaSuccess) return e;
-    memory_finalize_kernel<64><<<fgrid, 256, fsmem, st>>>(partials, Gused, phi, r, decay_n, M,
+    memory_finalize_kernel<64><<<fgrid, 256, fsmem, st>>>(partials, Gused, tokens_per_group,
+                                                          n_e, log2lam, phi, r, decay_n, M,
                                                           bstab, sv_partials, s_v, n_count,
                                                           (float)n_e, Hkv);
   }
@@ -437,8 +469,6 @@ cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, 
 // workspace, and it needs no context: the caller passes the dimensions, the
 // decay and W_phi directly.
 // ---------------------------------------------------------------------------
-#include <mutex>
-
 namespace imem {
 namespace {
 
@@ -446,27 +476,22 @@ constexpr size_t kStaticScratchBytes = (size_t)8 << 20;   // 8 MiB per device
 static __device__ __align__(256) float g_static_scratch[kStaticScratchBytes / sizeof(float)];
 static __device__ int g_static_err;
 
-constexpr int kMaxDevices = 64;
-std::mutex g_static_mtx;
-float* g_static_ptr[kMaxDevices] = {};
-int* g_static_err_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array for the current device (host code must
-// not use the symbol itself: it is a host-side stand-in, not a device address).
-cudaError_t static_scratch(int dev, float** scratch, int** err) {
-  std::lock_guard<std::mutex> lock(g_static_mtx);
-  if (!g_static_ptr[dev]) {
-    void* p = nullptr;
-    void* e = nullptr;
-    cudaError_t r = cudaGetSymbolAddress(&p, g_static_scratch);
-    if (r != cudaSuccess) return r;
-    r = cudaGetSymbolAddress(&e, g_static_err);
-    if (r != cudaSuccess) return r;
-    g_static_ptr[dev] = static_cast<float*>(p);
-    g_static_err_ptr[dev] = static_cast<int*>(e);
-  }
-  *scratch = g_static_ptr[dev];
-  *err = g_static_err_ptr[dev];
+// Device addresses of the scratch array and its error word in the context
+// that is current now. Host code must not use the symbols themselves: they are
+// host-side stand-ins, not device addresses. The lookup is repeated on every
+// call (it allocates nothing): an address kept from an earlier call would be
+// stale after cudaDeviceReset or in another context. The first lookup on a
+// device loads the library's device code there if that has not happened yet,
+// which is why the first call on a device belongs before any stream capture.
+cudaError_t static_scratch(float** scratch, int** err) {
+  void* p = nullptr;
+  void* e = nullptr;
+  cudaError_t r = cudaGetSymbolAddress(&p, g_static_scratch);
+  if (r != cudaSuccess) return r;
+  r = cudaGetSymbolAddress(&e, g_static_err);
+  if (r != cudaSuccess) return r;
+  *scratch = static_cast<float*>(p);
+  *err = static_cast<int*>(e);
   return cudaSuccess;
 }
 
@@ -498,7 +523,8 @@ cudaError_t launch_memory_static(int batch, int L, int Hkv, int r, float lambda,
                            (int)fsmem);
   if (e != cudaSuccess) return e;
   memory_finalize_kernel<D><<<dim3(D / 16 + 1, units), 256, fsmem, st>>>(
-      scratch, Gused, W_phi, r, decay_n, M, bstab, nullptr, nullptr, nullptr, 0.f, Hkv);
+      scratch, Gused, tokens_per_group, n_e, log2lam, W_phi, r, decay_n, M, bstab, nullptr,
+      nullptr, nullptr, 0.f, Hkv);
   return cudaGetLastError();
 }
 
@@ -531,11 +557,9 @@ extern "C" imem_status imem_update_memory_static(int batch, int L, int n_kv_head
     if ((uintptr_t)idx_evicted & 15u) return IMEM_ERR_ALIGN;
   }
   if (n_evicted == 0) return IMEM_OK;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return IMEM_ERR_CUDA;
   float* scratch = nullptr;
   int* err = nullptr;
-  if (static_scratch(dev, &scratch, &err) != cudaSuccess) return IMEM_ERR_CUDA;
+  if (static_scratch(&scratch, &err) != cudaSuccess) return IMEM_ERR_CUDA;
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
   if (dtype == IMEM_BF16)
@@ -545,4 +569,23 @@ extern "C" imem_status imem_update_memory_static(int batch, int L, int n_kv_head
     e = head_dim == 128 ? launch_memory_static<float, 128>(batch, L, n_kv_heads, mem_r, lambda, K, V, idx_evicted, n_evicted, chunk, W_phi, M, bstab, scratch, err, st)
                         : launch_memory_static<float, 64>(batch, L, n_kv_heads, mem_r, lambda, K, V, idx_evicted, n_evicted, chunk, W_phi, M, bstab, scratch, err, st);
   return e == cudaSuccess ? IMEM_OK : IMEM_ERR_CUDA;
+}
+
+extern "C" imem_status imem_static_status(void* stream) {
+  using namespace imem;
+  float* scratch = nullptr;
+  int* err = nullptr;
+  if (static_scratch(&scratch, &err) != cudaSuccess) return IMEM_ERR_CUDA;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return IMEM_ERR_CUDA;
+  int code = 0;
+  if (cudaMemcpy(&code, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return IMEM_ERR_CUDA;
+  if (code != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return IMEM_ERR_CUDA;
+  }
+  if (code == DEV_TIMEOUT) return IMEM_ERR_TIMEOUT;
+  if (code == DEV_RANGE) return IMEM_ERR_RANGE;
+  return IMEM_OK;
 }

@@ -1,8 +1,12 @@
 """Failure handling on the GPU without a fault: a bounded device wait that
 runs out is reported by imem_sync as IMEM_ERR_TIMEOUT, cleared by it, and the
-context keeps working (a decode step then matches the oracle)."""
+context keeps working (a decode step then matches the oracle). Inputs outside
+what the memory update computes with (a key beyond fp16's range, an evicted
+index outside [0, L)) are caught by the kernel's own checks, reported as
+IMEM_ERR_RANGE, and the context keeps working."""
 import numpy as np
 import pytest
+import torch
 
 from learned_kv_cache_indexmem_b200 import binding as B
 from learned_kv_cache_indexmem_b200 import synth
@@ -44,4 +48,46 @@ def test_bounded_wait_timeout_is_reported_and_cleared(cuda_device):
     with pytest.raises(B.IndexMemError) as ei:
         B.selftest_wait(lay.ctx, 0)
     assert ei.value.name == "IMEM_ERR_INVALID_ARG"
+    lay.close()
+
+
+def test_memory_update_out_of_range_inputs_are_reported(cuda_device):
+    wl = synth.WORKLOADS["c1"]
+    s = wl.shape
+    case = Case(wl, cuda_device, L=256, batch=2, n_decode=1)
+    lay = case.layer()
+    ws = lay.workspace(2, 256, 1, cuda_device)
+    K, V = case.in_dev["K"].clone(), case.in_dev["V"].clone()
+    E = synth.make_index_subset(2, 256, 100, 3, cuda_device)
+    M = torch.zeros(2, s.n_kv_heads, s.mem_r, s.head_dim, device=cuda_device)
+    b = torch.zeros(2, s.n_kv_heads, s.mem_r, device=cuda_device)
+    # a key beyond fp16's largest finite value (bf16 holds it)
+    K[1, int(E[1, 40]), 3, 17] = 1.0e5
+    B.update_memory(lay.ctx, 2, 256, K, V, E, 100, 64, M, b, ws)
+    with pytest.raises(B.IndexMemError) as ei:
+        lay.sync()
+    assert ei.value.name == "IMEM_ERR_RANGE"
+    # an evicted index at L: no row is read, the error is reported
+    E2 = E.clone()
+    E2[0, 99] = 256
+    B.update_memory(lay.ctx, 2, 256, case.in_dev["K"], case.in_dev["V"], E2, 100, 64, M, b, ws)
+    with pytest.raises(B.IndexMemError) as ei:
+        lay.sync()
+    assert ei.value.name == "IMEM_ERR_RANGE"
+    # the same index through the allocation-free entry point and its status word
+    B.update_memory_static(2, 256, s.n_kv_heads, s.head_dim, s.mem_r, s.lam, B.BF16,
+                           case.in_dev["K"], case.in_dev["V"], E2, 100, 64, case.w_dev["W_phi"],
+                           M, b)
+    with pytest.raises(B.IndexMemError) as ei:
+        B.static_status()
+    assert ei.value.name == "IMEM_ERR_RANGE"
+    B.static_status()                            # cleared
+    # in-range inputs afterwards: no error, result as the oracle's
+    M.zero_(); b.zero_()
+    B.update_memory(lay.ctx, 2, 256, case.in_dev["K"], case.in_dev["V"], E, 100, 64, M, b, ws)
+    lay.sync()
+    M_ref, b_ref = om.memory_update(case.in_cpu["K"], case.in_cpu["V"], E.cpu().numpy(),
+                                    case.w_cpu["W_phi"], s.lam)
+    from .parity import check_memory
+    check_memory(to_np(M), to_np(b), M_ref, b_ref, "after range errors")
     lay.close()

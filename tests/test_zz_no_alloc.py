@@ -8,7 +8,11 @@ keeps its scratch in a fixed array inside the library instead. This test calls
 it through the C ABI twice in a row (the second call on the state the first
 left, with a different evicted set, so stale scratch contents would show) and
 checks each result against the existing entry point within the memory-state
-tolerance of the other parity tests. It lives in a file of its own that pytest
+tolerance of the other parity tests. Two more cases check it against the CPU
+oracle directly: the tiny fp32 layer (head dimension 64, r = 32) and the
+largest batch its scratch holds (15 sequences x 8 KV heads of dimension 128,
+one run per sequence and head). After every call the shared device error word
+(imem_static_status) must be clear. It lives in a file of its own that pytest
 collects last, and needs nothing from the tests before it.
 """
 import numpy as np
@@ -17,6 +21,7 @@ import torch
 
 from learned_kv_cache_indexmem_b200 import binding, synth
 from learned_kv_cache_indexmem_b200.layer import IndexMemLayer
+from oracle import indexmem_oracle as om
 
 pytestmark = pytest.mark.gpu
 
@@ -50,10 +55,34 @@ def test_static_update_matches_workspace_update_twice(cuda_device):
                                      w["W_phi"], M_st, b_st)
         torch.cuda.synchronize()
         lay.sync()
+        binding.static_status()                 # no device error recorded
         assert _rel_err(M_st, M_ref) <= MEM_TOL, "call %d: M" % call
         assert _rel_err(b_st, b_ref) <= MEM_TOL, "call %d: b" % call
         assert not torch.equal(M_st, M0)
     lay.close()
+
+
+@pytest.mark.parametrize("name,batch,L,n_e,chunk", [
+    ("c0", 1, 1024, 896, 512),      # fp32, head dimension 64, r = 32
+    ("c1", 15, 640, 520, 64),       # the capacity edge: 15 x 8 x 128 x 129 floats
+])
+def test_static_update_against_oracle(cuda_device, name, batch, L, n_e, chunk):
+    wl = synth.WORKLOADS[name]
+    s = wl.shape
+    dev = cuda_device
+    w = synth.make_weights(s, 5, dev)
+    inp = synth.make_layer_inputs(wl, w, 5, dev, L=L, batch=batch)
+    M0, b0 = synth.make_memory_state(s, batch, 5, dev)
+    E = synth.make_index_subset(batch, L, n_e, 9, dev)
+    M, b = M0.clone(), b0.clone()
+    binding.update_memory_static(batch, L, s.n_kv_heads, s.head_dim, s.mem_r, s.lam,
+                                 binding.BF16 if s.dtype == "bf16" else binding.FP32,
+                                 inp["K"], inp["V"], E, n_e, chunk, w["W_phi"], M, b)
+    binding.static_status()
+    M_ref, b_ref = om.memory_update(inp["K"].cpu(), inp["V"].cpu(), E.cpu().numpy(),
+                                    w["W_phi"].cpu(), s.lam, M0=M0.cpu(), b0=b0.cpu())
+    assert _rel_err(M, torch.from_numpy(M_ref)) <= MEM_TOL, "M"
+    assert _rel_err(b, torch.from_numpy(b_ref)) <= MEM_TOL, "b"
 
 
 def test_static_update_rejects_sizes_beyond_its_scratch(cuda_device):
