@@ -396,42 +396,130 @@ def moment_readout(job, steps=64, reps=3):
 
 # ------------------------------------------------------------------ stage split, budgets
 
-def prefill_split(job, reps=5):
-    """The prefill split as the survey of the method reports it: the indexer
-    (prologue + scoring, the call without selection) and eviction + compaction
-    (selection and the K/V gather: the rest of the full call), CUDA events."""
+def prefill_split(job, peaks, reps=5):
+    """The prefill by kernel, each through its own C-ABI call and timed alone
+    with CUDA events on the launching stream (best of `reps`): the indexer
+    prologue (imem_indexer_features: read X and Q, write q~ and k^), the
+    scoring with the streaming per-key max (imem_indexer_score: 128 flop per
+    causal pair) and the selection + compaction (imem_select_compact). Each
+    gets its roofline: the prologue against HBM, the scoring against the
+    burst bf16 tensor peak (a kernel timed alone), the selection + compaction
+    against HBM."""
     d = job.inp
     st = job.st
+    ws = job.layer._ws
+    ctx = job.layer.ctx
+    b, L, B = job.batch, job.L, job.B
 
-    def timed(finalize):
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
         best = None
         for _ in range(reps):
             a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             torch.cuda.synchronize()
             a.record(job.stream)
-            for i, (q0, q1) in enumerate(job.ranges):
-                last = i == len(job.ranges) - 1
-                binding.score_and_evict(job.layer.ctx, job.batch, job.L, job.B, d["X"], d["Q"],
-                                        d["K"], d["V"], st.running_max, q0, q1,
-                                        1 if (finalize and last) else 0, st.idx_retained,
-                                        st.idx_evicted, st.K_ret, st.V_ret, st.K_ret.shape[1],
-                                        job.layer._ws, job.stream)
+            fn()
             e.record(job.stream)
             torch.cuda.synchronize()
             t = a.elapsed_time(e)
             best = t if best is None else min(best, t)
         return best
 
-    t_idx = timed(False)
-    t_all = timed(True)
+    def features():
+        for q0, q1 in job.ranges:
+            binding.indexer_features(ctx, b, L, d["X"], d["Q"], st.running_max, q0, q1, ws,
+                                     job.stream)
+
+    def score():
+        # the prologue's features are in the workspace; the scoring re-runs
+        # over them (running_max only rises, so repeats give the same result)
+        for q0, q1 in job.ranges:
+            binding.indexer_score(ctx, b, L, st.running_max, q0, q1, ws, job.stream)
+
+    def select():
+        binding.select_compact(ctx, b, L, B, st.running_max, d["K"], d["V"], st.idx_retained,
+                               st.idx_evicted, st.K_ret, st.V_ret, st.K_ret.shape[1], ws,
+                               job.stream)
+
+    def whole():
+        for i, (q0, q1) in enumerate(job.ranges):
+            last = i == len(job.ranges) - 1
+            binding.score_and_evict(ctx, b, L, B, d["X"], d["Q"], d["K"], d["V"],
+                                    st.running_max, q0, q1, 1 if last else 0, st.idx_retained,
+                                    st.idx_evicted, st.K_ret, st.V_ret, st.K_ret.shape[1], ws,
+                                    job.stream)
+
+    features()                       # features in place for the score-only timing
+    t_pro = timed(features)
+    t_sco = timed(score)
+    t_sel = timed(select)
+    t_all = timed(whole)
     s = job.wl.shape
     es = 2 if s.dtype == "bf16" else 4
     row = s.n_kv_heads * s.head_dim * es * 2
-    ev_bytes = job.batch * (4 * job.L + 4 * job.L + 2 * job.B * row)   # scores, indices, K/V rows
-    t_ev = max(t_all - t_idx, 1e-6)
-    return {"indexer_ms": t_idx, "indexer_keys_per_s": job.batch * job.L / (t_idx * 1e-3),
-            "indexer_tflops": job.scoring_flops() / (t_idx * 1e-3) / 1e12,
-            "evict_compact_ms": t_ev, "evict_compact_GBps": ev_bytes / (t_ev * 1e-3) / 1e9}
+    pro_bytes = job.prefill_bytes() - 2 * b * B * row + b * L * 2 * 64 * 2   # X, Q in; q~, k^ out
+    sel_bytes = b * (4 * L + 4 * L + 2 * B * row)      # scores in, indices out, K/V rows in+out
+    flops = job.scoring_flops()
+    pro_gbs = pro_bytes / (t_pro * 1e-3) / 1e9
+    sco_tf = flops / (t_sco * 1e-3) / 1e12
+    sel_gbs = sel_bytes / (t_sel * 1e-3) / 1e9
+    return {
+        "prologue": {"ms": t_pro, "keys_per_s": b * L / (t_pro * 1e-3), "bytes": pro_bytes,
+                     "GBps": pro_gbs, "roofline": {"bound": "hbm", "peak": peaks["hbm_gbs"],
+                                                   "unit": "GB/s",
+                                                   "frac": pro_gbs / peaks["hbm_gbs"]}},
+        "scoring": {"ms": t_sco, "keys_per_s": b * L / (t_sco * 1e-3), "flop": flops,
+                    "TFLOPs": sco_tf, "roofline": {"bound": "tensor", "peak": peaks["bf16_tflops"],
+                                                   "unit": "TFLOP/s",
+                                                   "frac": sco_tf / peaks["bf16_tflops"],
+                                                   "peak_kind": "burst (kernel timed alone)"}},
+        "select_compact": {"ms": t_sel, "bytes": sel_bytes, "GBps": sel_gbs,
+                           "roofline": {"bound": "hbm", "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                        "frac": sel_gbs / peaks["hbm_gbs"]}},
+        "indexer_ms": t_pro + t_sco,
+        "indexer_keys_per_s": b * L / ((t_pro + t_sco) * 1e-3),
+        "score_and_evict_ms": t_all,
+        "note": "each kernel timed alone (CUDA events on its stream, best of %d); "
+                "score_and_evict_ms is the one-call prefill" % reps}
+
+
+def other_workload_step(name, dev, seed, steps=5, warmup=3):
+    """The whole step (prefill, memory update, decode steps in a CUDA graph) on
+    another single-layer workload, timed like the main line: ms per step,
+    tokens/s, decode tokens/s and decode per launch."""
+    wl = synth.WORKLOADS[name]
+    j = Job(wl, wl.budget, dev, seed)
+    j.capture_decode()
+    for _ in range(warmup):
+        j.step()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(j.stream)
+    for i in range(steps):
+        j.step(ev[i])
+    e.record(j.stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(e) / steps
+    dec = statistics.mean(x[2].elapsed_time(x[3]) for x in ev)
+    pre = statistics.mean(x[0].elapsed_time(x[1]) for x in ev)
+    mem = statistics.mean(x[1].elapsed_time(x[2]) for x in ev)
+    dec_launch_ms = dec / j.n_dec
+    dec_bytes = j.decode_bytes_per_launch()
+    j.layer.sync(j.stream)
+    out = {"workload": "%s: batch %d, L=%d, B=%d, %d decode steps" % (
+               name, wl.batch, wl.L, wl.budget, wl.n_decode),
+           "ms_per_step": ms, "tokens_per_s": j.tokens_per_step() / (ms * 1e-3),
+           "prefill_ms": pre, "indexer_keys_per_s": j.batch * j.L / (pre * 1e-3),
+           "memory_ms": mem, "decode_ms": dec,
+           "decode_tokens_per_s": j.batch * j.n_dec / (dec * 1e-3),
+           "decode_us_per_launch": dec_launch_ms * 1e3,
+           "decode_bytes_per_launch": dec_bytes,
+           "decode_GBps": dec_bytes / (dec_launch_ms * 1e-3) / 1e9}
+    del j
+    torch.cuda.empty_cache()
+    return out
 
 
 def budget_sweep(wl, dev, seed, budgets=(128, 256, 512), steps=5, warmup=3):
@@ -813,6 +901,8 @@ def main():
                     help="skip the decode-time online eviction measurement")
     ap.add_argument("--no-pre-eviction", action="store_true",
                     help="skip the pre-eviction (long-context chunked prefill) measurement")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the whole-step lines of the 4K (c1) and 128K (c3) workloads")
     a = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -930,8 +1020,13 @@ def main():
     moment = None
     if not a.no_moment:
         moment = moment_readout(job)
-    split = prefill_split(job)
+    split = prefill_split(job, peaks)
     stages["prefill_split"] = split
+    others = {}
+    if not a.no_other_workloads and wl.name == "c2":
+        for name in ("c1", "c3"):
+            others[name] = other_workload_step(name, dev, synth.WORKLOADS[name].seed + 1000 * rank)
+            others[name]["decode_hbm_frac"] = others[name]["decode_GBps"] / peak
     sweep = None
     if not a.no_budget_sweep and wl.name == "c2" and a.budget is None:
         sweep = budget_sweep(wl, dev, wl.seed + 1000 * rank)
@@ -956,6 +1051,11 @@ def main():
     if rank == 0:
         print(json.dumps({
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "decode_tokens_per_s": stages["decode"]["tokens_per_s"] * world,
+            "indexer_keys_per_s": split["indexer_keys_per_s"] * world,
+            "value_counts": "b*L context keys + b*n_decode decoded tokens per whole step; "
+                            "decode_tokens_per_s and indexer_keys_per_s are the metric's two "
+                            "quantities on their own",
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if wl.shape.dtype == "bf16" else "f32", "data": "synthetic",
@@ -975,6 +1075,11 @@ def main():
             "online_eviction": online,
             "pre_eviction": pre_ev,
             "model_decode": model_dec,
+            "other_workloads": others or None,
+            "roofline_scoring": dict(split["scoring"]["roofline"],
+                                     achieved=split["scoring"]["TFLOPs"], kernel="scoring"),
+            "roofline_prologue": dict(split["prologue"]["roofline"],
+                                      achieved=split["prologue"]["GBps"], kernel="prologue"),
             "gpu_launches": job.launches_per_step() * a.steps,
             "device_errors": not layer_sync_ok,
         }))

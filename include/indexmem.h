@@ -22,8 +22,9 @@
  *     void* so this header needs no CUDA include; 0 = legacy default stream).
  *   - Arguments are validated on the host before anything is launched; an
  *     invalid call returns an error status and enqueues nothing.
- *   - Errors raised on the device (a bounded wait that ran out) are recorded
- *     in the context and reported by imem_sync(). No entry point throws.
+ *   - Errors raised on the device (a bounded wait that ran out, an input
+ *     value out of range) are recorded in the context and reported by
+ *     imem_sync(). No entry point throws.
  *   - A context is bound to the device that was current at imem_init; calls
  *     must be made with that device current. Calls that share a context or a
  *     workspace must be ordered on one stream.
@@ -49,7 +50,11 @@ typedef enum {
   IMEM_ERR_ALIGN = 3,        /* a pointer is not 16-byte aligned             */
   IMEM_ERR_UNSUPPORTED = 4,  /* a dimension this build has no kernel for    */
   IMEM_ERR_CUDA = 5,         /* a CUDA runtime call failed                  */
-  IMEM_ERR_TIMEOUT = 6       /* a bounded device-side wait ran out          */
+  IMEM_ERR_TIMEOUT = 6,      /* a bounded device-side wait ran out          */
+  IMEM_ERR_RANGE = 7         /* an input value out of the supported range:  */
+                             /* an evicted index outside [0, L), or a key   */
+                             /* or decay-weighted value of the memory       */
+                             /* update with |x| > 65504 (fp16 operands)     */
 } imem_status;
 
 typedef enum { IMEM_FP32 = 0, IMEM_BF16 = 1 } imem_dtype;
@@ -153,6 +158,33 @@ imem_status imem_score_and_evict(imem_ctx* ctx, int batch, int L, int B,
                                  void* K_ret, void* V_ret, int cap,
                                  void* workspace, void* stream);
 
+/* The three steps of imem_score_and_evict as separate calls, for callers
+ * that schedule or time them on their own (same arguments, workspace and
+ * errors as there; imem_score_and_evict(..., finalize) equals
+ * imem_indexer_features + imem_indexer_score (+ imem_select_compact)):
+ *
+ * imem_indexer_features ([IM-sum] §2.A Architecture): the indexer query
+ *   q~_s = sum_h g_{s,h} RMSNorm(W_idx_q[h]^T q_{s,h}) / sqrt(d_I) and key
+ *   k^_s = RMSNorm(W_idx_k^T x_s) of the tokens s in [q_begin, q_end), stored
+ *   (bf16) in the workspace; running_max[:, q_begin:q_end] is reset to -inf.
+ * imem_indexer_score ([IM-sum] §2.A Function/Training): for all keys t < q_end
+ *   running_max[t] = max(running_max[t], max_{s in [max(t,q_begin), q_end)}
+ *   q~_s . k^_t) over the features in the workspace (the features of keys
+ *   t < q_begin from earlier ranges).
+ * imem_select_compact ([IM-sum] §1, §4): the finalize step: selection of the B
+ *   largest importances (ties to the lower position), idx_retained,
+ *   idx_evicted and the gather into K_ret, V_ret; clears the workspace's
+ *   decode tags. */
+imem_status imem_indexer_features(imem_ctx* ctx, int batch, int L, const void* X, const void* Q,
+                                  float* running_max, int q_begin, int q_end, void* workspace,
+                                  void* stream);
+imem_status imem_indexer_score(imem_ctx* ctx, int batch, int L, float* running_max, int q_begin,
+                               int q_end, void* workspace, void* stream);
+imem_status imem_select_compact(imem_ctx* ctx, int batch, int L, int B, const float* running_max,
+                                const void* K, const void* V, int32_t* idx_retained,
+                                int32_t* idx_evicted, void* K_ret, void* V_ret, int cap,
+                                void* workspace, void* stream);
+
 /* Latent-memory update from the evicted tokens ([IM-sum] §2.B Mechanism,
  * fast weights: decayed outer-product accumulation into M and stabiliser b).
  * For every sequence and KV head h, with phi(x) = W_phi x and the evicted
@@ -163,8 +195,14 @@ imem_status imem_score_and_evict(imem_ctx* ctx, int batch, int L, int B,
  * K, V [batch, L, Hkv, d] model dtype; M [batch, Hkv, r, d] fp32 in/out;
  * bstab [batch, Hkv, r] fp32 in/out. `chunk` = evicted tokens per work unit
  * (a multiple of 64, e.g. 512). n_evicted = 0 leaves M and b unchanged.
+ * Precision and range: the tensor-core sums take fp16 operands with fp32
+ * accumulation. Keys must satisfy |k| <= 65504 and values |v| <= 65504 (every
+ * bf16 key inside that range converts to fp16 exactly; decay-weighted values
+ * are rounded once to fp16); every evicted index must lie in [0, L). A value or
+ * index outside that is reported by imem_sync as IMEM_ERR_RANGE (the row of an
+ * out-of-range index is not read; M and bstab are then unspecified).
  * Errors: INVALID_ARG, SHAPE, ALIGN, CUDA; UNSUPPORTED for a context in
- * IMEM_READOUT_MOMENT mode (use imem_update_moments). */
+ * IMEM_READOUT_MOMENT mode (use imem_update_moments); RANGE via imem_sync. */
 imem_status imem_update_memory(imem_ctx* ctx, int batch, int L, const void* K, const void* V,
                                const int32_t* idx_evicted, int n_evicted, int chunk,
                                float* M, float* bstab, void* workspace, void* stream);
@@ -219,14 +257,23 @@ imem_status imem_decode_invalidate(imem_ctx* ctx, int batch, void* workspace, vo
  * allocation); make that first call before any stream capture. Every call
  * writes the whole scratch region it uses before reading it, so nothing must
  * start at zero; calls that overlap on the GPU (any streams, any callers) race
- * on the shared array and must be serialised by the caller. A bounded device
- * wait that runs out is not reported by this entry point (no context); the
- * outputs are then unspecified.
+ * on the shared array and must be serialised by the caller. The array's
+ * device address is looked up on every call (no allocation), so a call stays
+ * valid after cudaDeviceReset or in another context. Errors raised on the
+ * device (a bounded wait that ran out, the range conditions of
+ * imem_update_memory) go to one error word shared by all calls on the device;
+ * imem_static_status reports and clears it. M and bstab are then unspecified.
  * Errors: INVALID_ARG, SHAPE, ALIGN, UNSUPPORTED, CUDA. */
 imem_status imem_update_memory_static(int batch, int L, int n_kv_heads, int head_dim, int mem_r,
                                       float lambda, int dtype, const void* K, const void* V,
                                       const int32_t* idx_evicted, int n_evicted, int chunk,
                                       const float* W_phi, float* M, float* bstab, void* stream);
+
+/* Waits for `stream`, then reports and clears the device error word that the
+ * calls of imem_update_memory_static on the current device share (no
+ * counterpart in the paper; allocates nothing): IMEM_OK, IMEM_ERR_TIMEOUT or
+ * IMEM_ERR_RANGE, or IMEM_ERR_CUDA if a CUDA call fails. */
+imem_status imem_static_status(void* stream);
 
 /* Moment statistics of the evicted tokens ([MK-sum] Method §1), for a context
  * created with readout = IMEM_READOUT_MOMENT (else IMEM_ERR_UNSUPPORTED).
@@ -330,8 +377,13 @@ imem_status imem_prefill_evict_chunk(imem_ctx* ctx, int batch, int L, int B, int
  *      position leaves); M <- lambda M + phi(k) v^T, bstab <- lambda bstab +
  *      phi(k) with its key and value (every KV head); evicted [batch] (int32,
  *      out) receives its position;
- *   4. the new token takes the freed slot (nothing moves if it left itself);
- *      cache_len returns to B; next_pos advances.
+ *   4. the new token takes the freed slot and the evicted token moves to
+ *      slot B (nothing moves if the new token left itself): after the step
+ *      slots [0, B) hold the retained tokens and slot B the one that left,
+ *      with its row, indexer key, position and the importance it was chosen
+ *      by, so that K_ret/V_ret/khat_ret/I_ret/pos_ret[:, :B + 1] are the
+ *      B + 1 candidates of the step; cache_len returns to B; next_pos
+ *      advances.
  * Ordering as imem_decode: step 4 also sets the workspace's decode tag for
  * cache length B, so the next step's attention may use the rows it loads
  * before its launch-dependency wait. imem_online_init does not write the
@@ -359,7 +411,8 @@ imem_status imem_selftest_wait(imem_ctx* ctx, long long limit_cycles, void* stre
 
 /* Waits for the stream, then reports the first error the device recorded for
  * this context since the last imem_sync (TIMEOUT for a bounded wait that ran
- * out, SHAPE for a decode into a full cache) or a CUDA error, and clears it. */
+ * out, SHAPE for a decode into a full cache, RANGE for an input value out of
+ * range) or a CUDA error, and clears it. */
 imem_status imem_sync(imem_ctx* ctx, void* stream);
 
 #ifdef __cplusplus

@@ -16,7 +16,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libindexmem.so")
 
 STATUS = {0: "IMEM_OK", 1: "IMEM_ERR_INVALID_ARG", 2: "IMEM_ERR_SHAPE", 3: "IMEM_ERR_ALIGN",
-          4: "IMEM_ERR_UNSUPPORTED", 5: "IMEM_ERR_CUDA", 6: "IMEM_ERR_TIMEOUT"}
+          4: "IMEM_ERR_UNSUPPORTED", 5: "IMEM_ERR_CUDA", 6: "IMEM_ERR_TIMEOUT",
+          7: "IMEM_ERR_RANGE"}
 FP32, BF16 = 0, 1
 READOUT_GATED, READOUT_MOMENT = 0, 1
 
@@ -94,6 +95,14 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                        vp]
     lib.imem_update_memory_static.restype = i
     lib.imem_update_memory_static.argtypes = [i, i, i, i, i, f, i, vp, vp, vp, i, i, vp, vp, vp, vp]
+    lib.imem_static_status.restype = i
+    lib.imem_static_status.argtypes = [vp]
+    lib.imem_indexer_features.restype = i
+    lib.imem_indexer_features.argtypes = [vp, i, i, vp, vp, vp, i, i, vp, vp]
+    lib.imem_indexer_score.restype = i
+    lib.imem_indexer_score.argtypes = [vp, i, i, vp, i, i, vp, vp]
+    lib.imem_select_compact.restype = i
+    lib.imem_select_compact.argtypes = [vp, i, i, i, vp, vp, vp, vp, vp, vp, vp, i, vp, vp]
     _lib = lib
     return lib
 
@@ -242,6 +251,31 @@ def update_memory_static(batch, L, n_kv_heads, head_dim, mem_r, lam, dtype, K, V
         batch, L, n_kv_heads, head_dim, mem_r, lam, dtype, _ptr(K), _ptr(V), _ptr(idx_evicted),
         n_evicted, chunk, _ptr(W_phi), _ptr(M), _ptr(bstab), _stream(stream)),
         "imem_update_memory_static")
+
+
+def indexer_features(ctx, batch, L, X, Q, running_max, q_begin, q_end, workspace, stream=None):
+    _check(load().imem_indexer_features(ctx, batch, L, _ptr(X), _ptr(Q), _ptr(running_max),
+                                        q_begin, q_end, _ptr(workspace), _stream(stream)),
+           "imem_indexer_features")
+
+
+def indexer_score(ctx, batch, L, running_max, q_begin, q_end, workspace, stream=None):
+    _check(load().imem_indexer_score(ctx, batch, L, _ptr(running_max), q_begin, q_end,
+                                     _ptr(workspace), _stream(stream)), "imem_indexer_score")
+
+
+def select_compact(ctx, batch, L, B, running_max, K, V, idx_retained, idx_evicted, K_ret, V_ret,
+                   cap, workspace, stream=None):
+    _check(load().imem_select_compact(ctx, batch, L, B, _ptr(running_max), _ptr(K), _ptr(V),
+                                      _ptr(idx_retained), _ptr(idx_evicted), _ptr(K_ret),
+                                      _ptr(V_ret), cap, _ptr(workspace), _stream(stream)),
+           "imem_select_compact")
+
+
+def static_status(stream=None) -> None:
+    """imem_static_status: raises if a call of update_memory_static on this
+    device recorded a device error since the last query (and clears it)."""
+    _check(load().imem_static_status(_stream(stream)), "imem_static_status")
 
 
 def sync(ctx, stream=None) -> None:

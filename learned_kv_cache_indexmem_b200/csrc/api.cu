@@ -163,6 +163,7 @@ const char* imem_status_string(imem_status s) {
     case IMEM_ERR_UNSUPPORTED: return "IMEM_ERR_UNSUPPORTED";
     case IMEM_ERR_CUDA: return "IMEM_ERR_CUDA";
     case IMEM_ERR_TIMEOUT: return "IMEM_ERR_TIMEOUT";
+    case IMEM_ERR_RANGE: return "IMEM_ERR_RANGE";
   }
   return "IMEM_ERR_UNKNOWN";
 }
@@ -306,6 +307,67 @@ imem_status imem_score_and_evict(imem_ctx* h, int batch, int L, int B, const voi
                                                        idx_retained, idx_evicted, K_ret, V_ret,
                                                        cap, wsb + ws.sel_off, st)));
   return IMEM_OK;
+}
+
+imem_status imem_indexer_features(imem_ctx* h, int batch, int L, const void* X, const void* Q,
+                                  float* running_max, int q_begin, int q_end, void* workspace,
+                                  void* stream) {
+  if (!h) return IMEM_ERR_INVALID_ARG;
+  const Ctx& c = h->c;
+  if (batch < 1 || L < 1) return IMEM_ERR_SHAPE;
+  if (q_begin < 0 || q_end <= q_begin || q_end > L) return IMEM_ERR_SHAPE;
+  IMEM_CHECK(check_ptr(X));
+  IMEM_CHECK(check_ptr(Q));
+  IMEM_CHECK(check_ptr(running_max));
+  IMEM_CHECK(check_ptr(workspace));
+  IMEM_CHECK(check_device(c));
+  const imem::Workspace ws = imem::workspace_layout(c, batch, L);
+  char* wsb = (char*)workspace;
+  return cuda_status(imem::launch_prologue(c, batch, L, X, Q, q_begin, q_end,
+                                           (__nv_bfloat16*)(wsb + ws.qt_off),
+                                           (__nv_bfloat16*)(wsb + ws.kh_off), running_max,
+                                           (cudaStream_t)stream));
+}
+
+imem_status imem_indexer_score(imem_ctx* h, int batch, int L, float* running_max, int q_begin,
+                               int q_end, void* workspace, void* stream) {
+  if (!h) return IMEM_ERR_INVALID_ARG;
+  const Ctx& c = h->c;
+  if (batch < 1 || L < 1) return IMEM_ERR_SHAPE;
+  if (q_begin < 0 || q_end <= q_begin || q_end > L) return IMEM_ERR_SHAPE;
+  IMEM_CHECK(check_ptr(running_max));
+  IMEM_CHECK(check_ptr(workspace));
+  IMEM_CHECK(check_device(c));
+  const imem::Workspace ws = imem::workspace_layout(c, batch, L);
+  char* wsb = (char*)workspace;
+  return cuda_status(imem::launch_scoring(c, batch, L, (const __nv_bfloat16*)(wsb + ws.qt_off),
+                                          (const __nv_bfloat16*)(wsb + ws.kh_off), running_max,
+                                          q_begin, q_end, (cudaStream_t)stream));
+}
+
+imem_status imem_select_compact(imem_ctx* h, int batch, int L, int B, const float* running_max,
+                                const void* K, const void* V, int32_t* idx_retained,
+                                int32_t* idx_evicted, void* K_ret, void* V_ret, int cap,
+                                void* workspace, void* stream) {
+  if (!h) return IMEM_ERR_INVALID_ARG;
+  const Ctx& c = h->c;
+  if (batch < 1 || L < 1) return IMEM_ERR_SHAPE;
+  if (B < 1 || B > L || cap < B) return IMEM_ERR_SHAPE;
+  IMEM_CHECK(check_ptr(running_max));
+  IMEM_CHECK(check_ptr(K));
+  IMEM_CHECK(check_ptr(V));
+  IMEM_CHECK(check_ptr(idx_retained));
+  if (B < L) IMEM_CHECK(check_ptr(idx_evicted));
+  IMEM_CHECK(check_ptr(K_ret));
+  IMEM_CHECK(check_ptr(V_ret));
+  IMEM_CHECK(check_ptr(workspace));
+  IMEM_CHECK(check_device(c));
+  cudaStream_t st = (cudaStream_t)stream;
+  const imem::Workspace ws = imem::workspace_layout(c, batch, L);
+  IMEM_CHECK(cuda_status(imem::clear_decode_tags(c, batch, workspace, st)));
+  return cuda_status(imem::launch_select_compact(c, batch, L, B, running_max, K, V, idx_retained,
+                                                 idx_evicted, K_ret, V_ret, cap,
+                                                 (char*)workspace + ws.sel_off, st));
 }
 
 imem_status imem_update_memory(imem_ctx* h, int batch, int L, const void* K, const void* V,
@@ -582,6 +644,7 @@ imem_status imem_sync(imem_ctx* h, void* stream) {
   }
   if (code == imem::DEV_TIMEOUT) return IMEM_ERR_TIMEOUT;
   if (code == imem::DEV_CACHE_FULL) return IMEM_ERR_SHAPE;
+  if (code == imem::DEV_RANGE) return IMEM_ERR_RANGE;
   return IMEM_OK;
 }
 

@@ -96,6 +96,10 @@ def test_null_context_is_invalid_for_every_call():
     assert lib.imem_update_moments(None, 1, 16, 16, 16, 16, 4, 64, 16, 16, 16, 16, 16, None) == 1
     assert lib.imem_decode_moment(None, 1, 16, 16, 16, 16, 16, 16, 8, 16, 16, 16, 16, 16, 16,
                                   None) == 1
+    assert lib.imem_indexer_features(None, 1, 16, 16, 16, 16, 0, 16, 16, None) == 1
+    assert lib.imem_indexer_score(None, 1, 16, 16, 0, 16, 16, None) == 1
+    assert lib.imem_select_compact(None, 1, 16, 4, 16, 16, 16, 16, 16, 16, 16, 8, 16,
+                                   None) == 1
     lib.imem_destroy(None)   # accepted
     out = ctypes.c_void_p(123)
     assert lib.imem_init(None, None, ctypes.byref(out)) == 1 and out.value is None
