@@ -396,9 +396,13 @@ def moment_readout(job, steps=64, reps=3):
 
 # ------------------------------------------------------------------ stage split, budgets
 
-def prefill_split(job, peaks, reps=5):
+def prefill_split(job, peaks, reps=5, inner=10):
     """The prefill by kernel, each through its own C-ABI call and timed alone
-    with CUDA events on the launching stream (best of `reps`): the indexer
+    with CUDA events on the launching stream: `inner` back-to-back calls
+    between two events (each call is idempotent: the prologue rewrites the
+    same features, the scoring's running maxima are already the maxima, the
+    selection rewrites the same outputs), the average per call, best of
+    `reps`; this takes the host's launch latency out of the figure: the indexer
     prologue (imem_indexer_features: read X and Q, write q~ and k^), the
     scoring with the streaming per-key max (imem_indexer_score: 128 flop per
     causal pair) and the selection + compaction (imem_select_compact). Each
@@ -411,7 +415,7 @@ def prefill_split(job, peaks, reps=5):
     ctx = job.layer.ctx
     b, L, B = job.batch, job.L, job.B
 
-    def timed(fn):
+    def timed(fn, n=inner):
         fn()
         torch.cuda.synchronize()
         best = None
@@ -419,10 +423,11 @@ def prefill_split(job, peaks, reps=5):
             a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             torch.cuda.synchronize()
             a.record(job.stream)
-            fn()
+            for _ in range(n):
+                fn()
             e.record(job.stream)
             torch.cuda.synchronize()
-            t = a.elapsed_time(e)
+            t = a.elapsed_time(e) / n
             best = t if best is None else min(best, t)
         return best
 
@@ -480,8 +485,9 @@ def prefill_split(job, peaks, reps=5):
         "indexer_ms": t_pro + t_sco,
         "indexer_keys_per_s": b * L / ((t_pro + t_sco) * 1e-3),
         "score_and_evict_ms": t_all,
-        "note": "each kernel timed alone (CUDA events on its stream, best of %d); "
-                "score_and_evict_ms is the one-call prefill" % reps}
+        "note": "each kernel alone: CUDA events on its stream around %d back-to-back calls, "
+                "average per call, best of %d; score_and_evict_ms is the one-call prefill "
+                "timed the same way" % (inner, reps)}
 
 
 def other_workload_step(name, dev, seed, steps=5, warmup=3):
@@ -591,7 +597,7 @@ def online_decode(job, steps=64, reps=3):
         del g
     lay.sync(job.stream)
     res["us_per_step_online"] = best
-    res["launches_per_step_online"] = 4
+    res["launches_per_step_online"] = 3   # features (second stream), attention, score + evict
     res["steps"] = steps
     res["cache_rows"] = B
     return res

@@ -52,9 +52,9 @@ typedef enum {
   IMEM_ERR_CUDA = 5,         /* a CUDA runtime call failed                  */
   IMEM_ERR_TIMEOUT = 6,      /* a bounded device-side wait ran out          */
   IMEM_ERR_RANGE = 7         /* an input value out of the supported range:  */
-                             /* an evicted index outside [0, L), or a key   */
-                             /* or decay-weighted value of the memory       */
-                             /* update with |x| > 65504 (fp16 operands)     */
+                             /* an evicted index outside [0, L), or (fp32   */
+                             /* inputs) a key or decay-weighted value of    */
+                             /* the memory update beyond fp16's range       */
 } imem_status;
 
 typedef enum { IMEM_FP32 = 0, IMEM_BF16 = 1 } imem_dtype;
@@ -195,11 +195,13 @@ imem_status imem_select_compact(imem_ctx* ctx, int batch, int L, int B, const fl
  * K, V [batch, L, Hkv, d] model dtype; M [batch, Hkv, r, d] fp32 in/out;
  * bstab [batch, Hkv, r] fp32 in/out. `chunk` = evicted tokens per work unit
  * (a multiple of 64, e.g. 512). n_evicted = 0 leaves M and b unchanged.
- * Precision and range: the tensor-core sums take fp16 operands with fp32
- * accumulation. Keys must satisfy |k| <= 65504 and values |v| <= 65504 (every
- * bf16 key inside that range converts to fp16 exactly; decay-weighted values
- * are rounded once to fp16); every evicted index must lie in [0, L). A value or
- * index outside that is reported by imem_sync as IMEM_ERR_RANGE (the row of an
+ * Precision and range: fp32 accumulation on the tensor cores. bf16 inputs:
+ * the values enter as they are and each decay-weighted key as two bf16 halves
+ * (hi + lo, about 16 significant bits, fp32's range). fp32 inputs: fp16
+ * operands (keys converted, decay-weighted values rounded once), so keys and
+ * values must stay below 65520 in magnitude (fp16 rounds larger ones to
+ * infinity). Every evicted index must lie in [0, L). A value or index outside
+ * that is reported by imem_sync as IMEM_ERR_RANGE (the row of an
  * out-of-range index is not read; M and bstab are then unspecified).
  * Errors: INVALID_ARG, SHAPE, ALIGN, CUDA; UNSUPPORTED for a context in
  * IMEM_READOUT_MOMENT mode (use imem_update_moments); RANGE via imem_sync. */
@@ -248,13 +250,17 @@ imem_status imem_decode_invalidate(imem_ctx* ctx, int batch, void* workspace, vo
  * allowed; imem_init and a workspace both need allocations such callers cannot
  * make). Same result as imem_update_memory, with no context: the caller passes
  * the dimensions, the decay lambda and W_phi [mem_r, head_dim] (fp32, device)
- * directly; K, V, idx_evicted, n_evicted, chunk, M and bstab as there.
+ * directly; K, V, idx_evicted, n_evicted, chunk, M and bstab as there. Its
+ * tensor-core sums take fp16 operands for both dtypes (the register-pipelined
+ * kernel, which needs no shared-memory position list), so keys and
+ * decay-weighted values must stay below 65520 in magnitude.
  * Scratch: a fixed 8 MiB array in the library's device memory, held by every
  * GPU that loads the library until the process exits. batch * n_kv_heads *
  * head_dim * (head_dim + 1) * 4 bytes must fit in it (batch <= 15 at 8 KV heads
  * of dimension 128), otherwise IMEM_ERR_UNSUPPORTED and nothing is launched.
- * The first call on a device looks up the array's device address (set-up, no
- * allocation); make that first call before any stream capture. Every call
+ * The first call on a device may load the library's device code there
+ * (set-up, no allocation); make that first call before any stream capture.
+ * Every call
  * writes the whole scratch region it uses before reading it, so nothing must
  * start at zero; calls that overlap on the GPU (any streams, any callers) race
  * on the shared array and must be serialised by the caller. The array's
@@ -384,11 +390,18 @@ imem_status imem_prefill_evict_chunk(imem_ctx* ctx, int batch, int L, int B, int
  *      by, so that K_ret/V_ret/khat_ret/I_ret/pos_ret[:, :B + 1] are the
  *      B + 1 candidates of the step; cache_len returns to B; next_pos
  *      advances.
- * Ordering as imem_decode: step 4 also sets the workspace's decode tag for
- * cache length B, so the next step's attention may use the rows it loads
- * before its launch-dependency wait. imem_online_init does not write the
- * cache state and leaves the tag as it is.
- * Errors: as imem_decode; UNSUPPORTED for the moment readout. */
+ * Streams: step 2's indexer query and key need neither the cache nor the
+ * memory, so they are computed on a second stream owned by the context
+ * (created by imem_online_init or the first step, which therefore belong
+ * before any stream capture; no device memory),
+ * forked from `stream` and joined back into it by events before step 3;
+ * under stream capture this becomes two parallel branches of the graph.
+ * Ordering: step 4 clears the workspace's decode tag of the sequence (slot e
+ * and the memory changed after the attention step), so the next decode step
+ * uses nothing it loaded before its launch-dependency wait.
+ * imem_online_init does not write the cache state and leaves the tag as it is.
+ * Errors: as imem_decode; UNSUPPORTED for the moment readout; nothing is
+ * enqueued if an argument is invalid. */
 imem_status imem_online_init(imem_ctx* ctx, int batch, int L, int B, const float* running_max,
                              const int32_t* idx_retained, const void* workspace, void* khat_ret,
                              float* I_ret, int32_t* pos_ret, int32_t* next_pos, int cap,

@@ -19,8 +19,6 @@ struct imem_ctx {
 
 namespace imem {
 
-int memory_groups(int batch, int n_kv_heads, int n_e, int chunk);
-
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 Workspace workspace_layout(const Ctx& c, int batch, int L) {
@@ -32,26 +30,19 @@ Workspace workspace_layout(const Ctx& c, int batch, int L) {
   w.dec_cnt_off = off;                        // one counter per sequence, then
   w.dec_tag_off = off + (size_t)batch * sizeof(int);   // the decode tags (one per sequence)
   off = align_up(off + (size_t)2 * batch * sizeof(int), 256);
-  // online eviction: the new token's feature partials, the score CTAs'
-  // candidates (16 bytes each), a counter and the chosen slot per sequence
+  // online eviction: the new token's feature partials
   w.on_qpart_off = off;
   off = align_up(off + (size_t)batch * c.cfg.n_q_heads * c.cfg.idx_dim * sizeof(float), 256);
   w.on_kpart_off = off;
   off = align_up(off + (size_t)batch * c.cfg.idx_dim * sizeof(float), 256);
-  w.on_cand_off = off;
-  off = align_up(off + (size_t)batch * kOnlineMaxCtas * 16, 256);
-  w.on_cnt_off = off;
-  off = align_up(off + (size_t)batch * sizeof(int), 256);
-  w.on_slot_off = off;
-  off = align_up(off + (size_t)batch * sizeof(int), 256);
   w.dec_part_off = off;                       // (unused: decode merges in shared memory)
-  // memory partials: at most (2*148 + units) runs of a d x (d+1) sum [S | s]
+  // memory partials: one d x (d+1) sum [S | s] per run of evicted tokens
+  const size_t runs = memory_runs_bound((int)units, L, c.num_sms);
   w.mem_part_off = off;
-  off = align_up(off + (2 * 148 + units) * (size_t)c.cfg.head_dim * (c.cfg.head_dim + 1) *
-                           sizeof(float), 256);
+  off = align_up(off + runs * (size_t)c.cfg.head_dim * (c.cfg.head_dim + 1) * sizeof(float), 256);
   w.sv_part_off = off;                        // moment mode: one d-vector per run
   if (c.cfg.readout == IMEM_READOUT_MOMENT)
-    off = align_up(off + (2 * 148 + units) * (size_t)c.cfg.head_dim * sizeof(float), 256);
+    off = align_up(off + runs * (size_t)c.cfg.head_dim * sizeof(float), 256);
   w.sel_off = off;
   off = align_up(off + 256, 256);
   w.qt_off = off;
@@ -148,6 +139,19 @@ imem_status check_device(const Ctx& c) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return IMEM_ERR_CUDA;
   return dev == c.device ? IMEM_OK : IMEM_ERR_INVALID_ARG;
+}
+
+// The second stream and the fork/join events of online eviction, created on
+// first use (no device memory is allocated).
+imem_status online_streams(Ctx& c) {
+  if (c.side && c.ev_fork && c.ev_join) return IMEM_OK;
+  if (!c.side && cudaStreamCreateWithFlags(&c.side, cudaStreamNonBlocking) != cudaSuccess)
+    return IMEM_ERR_CUDA;
+  if (!c.ev_fork && cudaEventCreateWithFlags(&c.ev_fork, cudaEventDisableTiming) != cudaSuccess)
+    return IMEM_ERR_CUDA;
+  if (!c.ev_join && cudaEventCreateWithFlags(&c.ev_join, cudaEventDisableTiming) != cudaSuccess)
+    return IMEM_ERR_CUDA;
+  return IMEM_OK;
 }
 
 }  // namespace
@@ -257,6 +261,9 @@ void imem_destroy(imem_ctx* h) {
   cudaFree(c.W_phi);
   cudaFree(c.w_gate);
   cudaFree(c.err);
+  if (c.ev_fork) cudaEventDestroy(c.ev_fork);
+  if (c.ev_join) cudaEventDestroy(c.ev_join);
+  if (c.side) cudaStreamDestroy(c.side);
   free(h);
 }
 
@@ -581,6 +588,7 @@ imem_status imem_online_init(imem_ctx* h, int batch, int L, int B, const float* 
   IMEM_CHECK(check_ptr(pos_ret));
   IMEM_CHECK(check_ptr(next_pos));
   IMEM_CHECK(check_device(c));
+  IMEM_CHECK(online_streams(h->c));
   const imem::Workspace ws = imem::workspace_layout(c, batch, L);
   const __nv_bfloat16* kh = (const __nv_bfloat16*)((const char*)workspace + ws.kh_off);
   return cuda_status(imem::launch_online_init(c, batch, L, B, cap, running_max, idx_retained, kh,
@@ -603,25 +611,41 @@ imem_status imem_decode_online(imem_ctx* h, int batch, int B, const void* x_new,
   IMEM_CHECK(check_ptr(pos_ret));
   IMEM_CHECK(check_ptr(next_pos));
   IMEM_CHECK(check_ptr(evicted));
-  // the attention step with the memory before this step's eviction (it
-  // validates the remaining arguments and appends the new token at slot B)
-  cudaStream_t st = (cudaStream_t)stream;
   IMEM_CHECK(check_ptr(workspace));
+  // the attention step's arguments too: nothing is enqueued unless all are valid
+  IMEM_CHECK(check_ptr(q));
+  IMEM_CHECK(check_ptr(k_new));
+  IMEM_CHECK(check_ptr(v_new));
+  IMEM_CHECK(check_ptr(K_ret));
+  IMEM_CHECK(check_ptr(V_ret));
+  IMEM_CHECK(check_ptr(cache_len));
+  IMEM_CHECK(check_ptr(M));
+  IMEM_CHECK(check_ptr(bstab));
+  IMEM_CHECK(check_ptr(out));
+  IMEM_CHECK(check_device(c));
+  IMEM_CHECK(online_streams(h->c));
+  cudaStream_t st = (cudaStream_t)stream;
   const imem::Workspace ws = imem::workspace_layout(c, batch, 1);
   char* wsb = (char*)workspace;
   float* qpart = (float*)(wsb + ws.on_qpart_off);
   float* kpart = (float*)(wsb + ws.on_kpart_off);
-  IMEM_CHECK(check_ptr(q));
-  IMEM_CHECK(check_device(c));
-  IMEM_CHECK(cuda_status(imem::launch_online_features(c, batch, x_new, q, qpart, kpart, st)));
-  IMEM_CHECK(decode_common(h, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M, bstab,
-                           nullptr, nullptr, out, workspace, stream));
-  return cuda_status(imem::launch_online_evict(c, batch, B, cap, qpart, kpart, khat_ret, I_ret,
-                                               pos_ret, next_pos, K_ret, V_ret, cache_len, M,
-                                               bstab, evicted, wsb + ws.on_cand_off,
-                                               (int*)(wsb + ws.on_cnt_off),
-                                               (int*)(wsb + ws.on_slot_off),
-                                               (int*)(wsb + ws.dec_tag_off), st));
+  // the new token's indexer features need neither the cache nor the memory:
+  // they run on the context's second stream beside the attention step
+  IMEM_CHECK(cuda_status(cudaEventRecord(c.ev_fork, st)));
+  IMEM_CHECK(cuda_status(cudaStreamWaitEvent(c.side, c.ev_fork, 0)));
+  IMEM_CHECK(cuda_status(imem::launch_online_features(c, batch, x_new, q, qpart, kpart, c.side)));
+  IMEM_CHECK(cuda_status(cudaEventRecord(c.ev_join, c.side)));
+  // the attention step with the memory before this step's eviction (it
+  // validates the remaining arguments and appends the new token at slot B)
+  const imem_status ds = decode_common(h, batch, q, k_new, v_new, K_ret, V_ret, cache_len, cap, M,
+                                       bstab, nullptr, nullptr, out, workspace, stream);
+  // join first, so that the second stream's work is always waited for
+  IMEM_CHECK(cuda_status(cudaStreamWaitEvent(st, c.ev_join, 0)));
+  IMEM_CHECK(ds);
+  return cuda_status(imem::launch_online_score_evict(c, batch, B, cap, qpart, kpart, khat_ret,
+                                                     I_ret, pos_ret, next_pos, K_ret, V_ret,
+                                                     cache_len, M, bstab, evicted,
+                                                     (int*)(wsb + ws.dec_tag_off), st));
 }
 
 imem_status imem_selftest_wait(imem_ctx* h, long long limit_cycles, void* stream) {

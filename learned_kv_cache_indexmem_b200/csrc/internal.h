@@ -27,6 +27,10 @@ struct Ctx {
   int* err;             // device error word
   int num_sms;          // streaming multiprocessors of the device
   void* encode_tiled;   // driver entry point cuTensorMapEncodeTiled
+  // online eviction: a second stream for the new token's indexer features
+  // (forked from and joined back into the caller's stream by events)
+  cudaStream_t side;
+  cudaEvent_t ev_fork, ev_join;
 };
 
 // Indexer rows in the workspace: d_I features padded to 64 bf16 (128 bytes).
@@ -44,7 +48,7 @@ bool make_tmap_bf16(const Ctx& c, CUtensorMap* map, const void* base, uint64_t w
                     uint64_t rows, uint32_t box_rows);
 
 // Layout of the caller's workspace for (batch, L).
-constexpr int kOnlineMaxCtas = 64;   // score CTAs per sequence in online eviction (max)
+constexpr int kOnlineMaxCluster = 8;   // CTAs per sequence of the online score-and-evict cluster
 
 struct Workspace {
   size_t qt_off, kh_off;        // indexer q~ and k^ (bf16 [b, L, kIdxPad])
@@ -52,7 +56,7 @@ struct Workspace {
   size_t dec_part_off;          // decode split partials
   size_t dec_cnt_off;           // decode counters (int), zero between calls
   size_t dec_tag_off;           // decode tags (int): right after the counters
-  size_t on_qpart_off, on_kpart_off, on_cand_off, on_cnt_off, on_slot_off;   // online eviction
+  size_t on_qpart_off, on_kpart_off;   // online eviction: the new token's feature partials
   size_t mem_part_off;          // memory-update partials
   size_t sv_part_off;           // value-sum partials of the moment statistics
   size_t total;
@@ -61,9 +65,13 @@ struct Workspace {
 constexpr int kDecodeMaxSplits = 16;          // CTAs per decode cluster (max)
 constexpr int kDecodeMaxStages = 3;           // 64-row stages in a decode CTA's ring (max)
 constexpr int kDecodeRowsPerSplit = 192;   // cache rows per decode CTA (target)
-constexpr int kMemMaxGroups = 64;
+constexpr int kMemMaxGroups = 512;   // runs per (sequence, KV head) of the memory update (max)
 
 Workspace workspace_layout(const Ctx& c, int batch, int L);
+
+// Upper bound of (sequence, KV head) units x runs of the memory update for up
+// to L evicted tokens per unit (the partial sums in the workspace).
+size_t memory_runs_bound(int units, int L, int num_sms);
 
 // Repacks the indexer weights K-major into c.WcT / c.WqT (allocates them).
 cudaError_t pack_indexer_weights(Ctx& c, const void* W_iq, const void* W_ik, const void* w_ig);
@@ -108,18 +116,18 @@ cudaError_t launch_evict_chunk(const Ctx& c, int batch, int B, int Lc, int n_R, 
 cudaError_t launch_append_positions(int batch, int B, int n_R, int q0, int C, int32_t* retained,
                                     cudaStream_t st);
 // Decode-time online eviction (online.cu).
-int online_score_ctas(int B);
+int online_cluster_ctas(int B);
 cudaError_t launch_online_init(const Ctx& c, int batch, int L, int B, int cap,
                                const float* running_max, const int32_t* idx_r,
                                const __nv_bfloat16* kh, __nv_bfloat16* khat_ret, float* I_ret,
                                int32_t* pos_ret, int32_t* next_pos, cudaStream_t st);
 cudaError_t launch_online_features(const Ctx& c, int batch, const void* x, const void* q,
                                    float* qpart, float* kpart, cudaStream_t st);
-cudaError_t launch_online_evict(const Ctx& c, int batch, int B, int cap, const float* qpart,
-                                const float* kpart, void* khat_ret, float* I_ret, int32_t* pos_ret,
-                                int32_t* next_pos, void* K_ret, void* V_ret, int32_t* cache_len,
-                                float* M, float* bstab, int32_t* evicted, void* cand,
-                                int* counter, int* evict_slot, int* dec_tag, cudaStream_t st);
+cudaError_t launch_online_score_evict(const Ctx& c, int batch, int B, int cap, const float* qpart,
+                                      const float* kpart, void* khat_ret, float* I_ret,
+                                      int32_t* pos_ret, int32_t* next_pos, void* K_ret,
+                                      void* V_ret, int32_t* cache_len, float* M, float* bstab,
+                                      int32_t* evicted, int* dec_tag, cudaStream_t st);
 
 // A kernel whose bounded wait runs out after `limit` cycles (failure-path test).
 cudaError_t launch_wait_selftest(const Ctx& c, long long limit, cudaStream_t st);

@@ -21,7 +21,8 @@
 // in fp32 by pass 2), so they stay far from fp16's subnormal range for runs
 // of moderate length. Operands are fp16 (bf16 keys convert exactly within
 // fp16's range; w*v is rounded once to fp16) with fp32 accumulation; a key or
-// weighted value beyond that range (|x| > 65504) is reported as DEV_RANGE.
+// weighted value beyond that range (|x| >= 65520, which rounds to infinity)
+// is reported as DEV_RANGE.
 // Both operands are MN-major in shared memory (a token is one 128-byte row per
 // 64 features, so gathered rows are written as they arrive). Eight loader
 // warps gather, convert and write the chunks; one thread issues the MMAs; a
@@ -56,6 +57,13 @@ struct MemTile {
   static constexpr int SMEM = kStages * STAGE + 1024 /*align*/ + 256 /*barriers*/;
 };
 
+// Programmatic dependent launch: the finalize is launched while the
+// tensor-core pass finishes; it stages W_phi, then waits for that pass.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 // MN-major offset of (token jj in the chunk, 16-byte chunk cc of a feature row)
 __device__ __forceinline__ uint32_t mn_off(int jj, int cc) {
   return (uint32_t)((cc >> 3) * 8192 + (jj >> 3) * 1024 + (jj & 7) * 128 +
@@ -70,6 +78,16 @@ __device__ __forceinline__ uint4 to_half8(const float* f) {
     __half2 h = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
     w[i] = *reinterpret_cast<uint32_t*>(&h);
   }
+  return r;
+}
+
+// Nonzero if one of the eight fp16 values is an infinity (a finite input that
+// rounded beyond fp16's largest finite value, 65504).
+__device__ __forceinline__ uint32_t half8_has_inf(const uint4& h) {
+  const uint32_t w[4] = {h.x, h.y, h.z, h.w};
+  uint32_t r = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) r |= __vcmpeq2(w[i] & 0x7fff7fffu, 0x7c007c00u);
   return r;
 }
 
@@ -99,7 +117,7 @@ template <> struct RawRow<float> {
 };
 
 template <typename T, int D, bool kSV>
-__global__ void __launch_bounds__(kMemThreads, 2)
+__global__ void __maxnreg__(112)
 memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t* __restrict__ idx_e,
                  int n_e, int L, int Hkv, float log2lam, int tokens_per_group,
                  float* __restrict__ partials, float* __restrict__ sv_partials,
@@ -160,14 +178,17 @@ memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t
     using Raw = RawRow<T>;
     typename Raw::type cur_k[ITEMS], cur_v[ITEMS], nxt_k[ITEMS], nxt_v[ITEMS];
     int pos_next[ITEMS];
+    // bad: an evicted index outside [0, L) (its row is not read) or an
+    // operand fp16 cannot hold was met; reported once after the loop
+    uint32_t bad = 0;
     auto load_pos = [&](int c, int* pos) {
 #pragma unroll
       for (int it = 0; it < ITEMS; ++it) {
         const int j = j0 + c * kChunk + (tid + it * kLoaders) / CH;
-        int p = (c < nchunks && j < j1) ? __ldg(E + j) : -1;
-        if (p >= L || (p < 0 && c < nchunks && j < j1)) {   // no row to read
-          record_error(err, DEV_RANGE);
-          p = -1;
+        int p = -1;
+        if (c < nchunks && j < j1) {
+          p = __ldg(E + j);
+          if ((unsigned)p >= (unsigned)L) { bad = 1u; p = -1; }
         }
         pos[it] = p;
       }
@@ -220,19 +241,16 @@ memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t
         float kf[8], vf[8];
         Raw::to_f32(cur_k[it], kf);
         Raw::to_f32(cur_v[it], vf);
-        float big = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          vf[e] *= wv;
-          big = fmaxf(big, fmaxf(fabsf(kf[e]), fabsf(vf[e])));
-        }
-        if (big > 65504.f) record_error(err, DEV_RANGE);   // beyond fp16's range
+        for (int e = 0; e < 8; ++e) vf[e] *= wv;
         if constexpr (kSV) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) svacc[e] += vf[e];
         }
-        *reinterpret_cast<uint4*>(a_p + mn_off(jj, cc)) = to_half8(kf);
-        *reinterpret_cast<uint4*>(b_p + mn_off(jj, cc)) = to_half8(vf);
+        const uint4 hk = to_half8(kf), hv = to_half8(vf);
+        bad |= half8_has_inf(hk) | half8_has_inf(hv);   // |x| >= 65520: beyond fp16
+        *reinterpret_cast<uint4*>(a_p + mn_off(jj, cc)) = hk;
+        *reinterpret_cast<uint4*>(b_p + mn_off(jj, cc)) = hv;
         if (cc == 0)   // weight column: element 0 of the row in the last B atom
           *reinterpret_cast<__half*>(b_p + mn_off(jj, (D / 64) * 8)) = __float2half_rn(wv);
       }
@@ -243,6 +261,7 @@ memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t
         for (int it = 0; it < ITEMS; ++it) { cur_k[it] = nxt_k[it]; cur_v[it] = nxt_v[it]; }
       }
     }
+    if (bad) record_error(err, DEV_RANGE);
     if constexpr (kSV) {
       // lanes with equal tid % CH hold the same columns: fold them, then the
       // 8 loader warps through shared memory (named barrier 1: loaders only)
@@ -286,6 +305,7 @@ memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t
   }
 
   // ---------------- epilogue: warps 0-3 read [S | s] rows from TMEM
+  pdl_launch();   // the finalize may start staging W_phi (it waits for this grid)
   if (warp < 4) {
     const int row = warp * 32 + lane;   // feature index of k (TMEM lane)
     bool ok = true;
@@ -339,6 +359,7 @@ memory_finalize_kernel(const float* __restrict__ partials, int G, int tpg, int n
   __syncthreads();
   if (blockIdx.x == D / 16 + 1) {   // value sums (only launched with sv_partials)
     const int unit = blockIdx.y;
+    pdl_wait();
     for (int c = threadIdx.x; c < D; c += 256) {
       float a = 0.f;
       for (int gg = 0; gg < G; ++gg)
@@ -359,13 +380,33 @@ memory_finalize_kernel(const float* __restrict__ partials, int G, int tpg, int n
   if (W_phi)   // null: the identity map (r == D)
     for (int i = tid; i < r * D / 4; i += 256)
       reinterpret_cast<float4*>(sW)[i] = __ldg(reinterpret_cast<const float4*>(W_phi) + i);
+  // sum of the runs: every thread owns IPT (row, column) items and loads all
+  // of them for one run before the next run, so that its loads are
+  // independent (a loop over the runs per item would chain G round trips
+  // to L2 per item)
+  pdl_wait();
   const float* p = partials + (size_t)unit * G * D * (D + 1);
-  for (int i = tid; i < D * ncols; i += 256) {
-    const int dk = i / ncols, cc = i % ncols;
-    float a = 0.f;
-    for (int gg = 0; gg < G; ++gg)
-      a = fmaf(s_fac[gg], __ldcg(&p[((size_t)gg * D + dk) * (D + 1) + col0 + cc]), a);
-    sS[dk * 16 + cc] = a;
+  constexpr int IPT = D * 16 / 256;
+  float acc[IPT];
+#pragma unroll
+  for (int k = 0; k < IPT; ++k) acc[k] = 0.f;
+#pragma unroll 2
+  for (int gg = 0; gg < G; ++gg) {
+    const float f = s_fac[gg];
+    const float* pg = p + (size_t)gg * D * (D + 1) + col0;
+    float v[IPT];
+#pragma unroll
+    for (int k = 0; k < IPT; ++k) {
+      const int i = tid + k * 256;
+      v[k] = i < D * ncols ? __ldcg(&pg[(i / ncols) * (D + 1) + i % ncols]) : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < IPT; ++k) acc[k] = fmaf(f, v[k], acc[k]);
+  }
+#pragma unroll
+  for (int k = 0; k < IPT; ++k) {
+    const int i = tid + k * 256;
+    if (i < D * ncols) sS[(i / ncols) * 16 + i % ncols] = acc[k];
   }
   __syncthreads();
   for (int i = tid; i < r * ncols; i += 256) {
@@ -387,18 +428,324 @@ memory_finalize_kernel(const float* __restrict__ partials, int G, int tpg, int n
   }
 }
 
+// ---------------------------------------------------------------------------
+// bf16 inputs: the same run sums [S_g | s_g] = (w K_c)^T [V_c | 1] with the
+// rows gathered by cp.async straight into the operand layouts of the MMA, so
+// that many chunks of rows are in flight per SM without registers:
+//   A = (w k)^T, the decay weight applied to the key and split into two bf16
+//       halves hi = bf16(w k), lo = bf16(w k - hi) (two MMAs into the same
+//       accumulator; about 16 mantissa bits, fp32's range: no fp16 limit);
+//       a key row lands in the A_hi buffer and is rewritten there in place;
+//   B = [v | 1], the value row as loaded (bf16 is exact) and a column of
+//       ones written once, which makes s = sum w k fall out of the same MMA.
+// Chunks of 32 tokens; a ring of kBfStages stages; the loaders keep
+// kBfStages - 2 chunks in flight ahead of the one they convert. The run's
+// evicted positions are read into shared memory once (runs of at most
+// kRunMax tokens). One CTA per SM.
+constexpr int kBfChunk = 32;
+constexpr int kBfStages = 7;
+constexpr int kBfAhead = kBfStages - 2;
+constexpr int kRunMax = 4096;
+
+template <int D>
+struct BfTile {
+  static constexpr int KG = kBfChunk / 8;                // 8-token K groups per chunk
+  static constexpr int ATOM_COL = KG * 1024;             // one 64-element MN block
+  static constexpr int A_BYTES = 2 * ATOM_COL;           // M = 128 (d = 64 zero-padded)
+  static constexpr int B_ATOMS = D / 64 + 1;             // value columns + the ones column
+  static constexpr int B_BYTES = B_ATOMS * ATOM_COL;
+  static constexpr int N = D + 16;
+  static constexpr int STAGE = 2 * A_BYTES + B_BYTES;    // A_hi | A_lo | B
+  static constexpr int SMEM = kBfStages * STAGE + kRunMax * 4 + 1024 + 256;
+};
+
+__device__ __forceinline__ uint32_t bf_off(int jj, int cc, int atom_col) {
+  return (uint32_t)((cc >> 3) * atom_col + (jj >> 3) * 1024 + (jj & 7) * 128 +
+                    (((cc & 7) ^ (jj & 7)) << 4));
+}
+
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid) {
+  const int n = valid ? 16 : 0;   // 0: zero-fill the destination
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_group() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kMemThreads, 1)
+memory_bf16_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V,
+                   const int32_t* __restrict__ idx_e, int n_e, int L, int Hkv, float log2lam,
+                   int tokens_per_run, float* __restrict__ partials, int* __restrict__ err) {
+  using TL = BfTile<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  int* s_pos = reinterpret_cast<int*>(smem + kBfStages * TL::STAGE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_pos + kRunMax);
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+
+  const int g = blockIdx.x, kh = blockIdx.y, bi = blockIdx.z;
+  const int G = gridDim.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int j0 = g * tokens_per_run;
+  const int j1 = min(n_e, j0 + tokens_per_run);
+  const int ntok = max(0, j1 - j0);
+  const int nchunks = (ntok + kBfChunk - 1) / kBfChunk;
+  const uint32_t sbase = tc::smem_addr(smem);
+  const uint32_t full0 = tc::smem_addr(bars), empty0 = full0 + 8 * kBfStages,
+                 done = full0 + 16 * kBfStages;
+
+  // zero every stage (padding rows of A, unused columns of B), then the ones
+  // column of B: element 0 of the first 16-byte chunk of the last atom column
+  for (int i = tid; i < kBfStages * TL::STAGE / 16; i += kMemThreads)
+    reinterpret_cast<uint4*>(smem)[i] = make_uint4(0, 0, 0, 0);
+  __syncthreads();
+  for (int i = tid; i < kBfStages * kBfChunk; i += kMemThreads) {
+    const int st = i / kBfChunk, jj = i % kBfChunk;
+    *reinterpret_cast<__nv_bfloat16*>(smem + st * TL::STAGE + 2 * TL::A_BYTES +
+                                      bf_off(jj, (D / 64) * 8, TL::ATOM_COL)) =
+        __float2bfloat16_rn(1.f);
+  }
+  // the run's evicted positions (-1: no row: past the run, or out of range)
+  uint32_t bad = 0;
+  const int32_t* E = idx_e + (size_t)bi * n_e + j0;
+  for (int i = tid; i < nchunks * kBfChunk; i += kMemThreads) {
+    int p = -1;
+    if (i < ntok) {
+      p = __ldg(E + i);
+      if ((unsigned)p >= (unsigned)L) { bad = 1u; p = -1; }
+    }
+    s_pos[i] = p;
+  }
+  if (tid == 0) {
+    for (int st = 0; st < kBfStages; ++st) {
+      tc::mbar_init(full0 + 8 * st, kLoaders);
+      tc::mbar_init(empty0 + 8 * st, 1);
+    }
+    tc::mbar_init(done, 1);
+    tc::fence_mbar_init();
+    s_abort = 0;
+  }
+  if (warp == 8) {
+    tc::tmem_alloc(tc::smem_addr(&s_tmem), 256);
+    tc::tmem_relinquish();
+  }
+  tc::fence_proxy_async();
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = s_tmem;
+  float* out = partials + (((size_t)bi * Hkv + kh) * G + g) * (size_t)D * (D + 1);
+
+  if (warp < 8) {
+    // ---------------- loaders
+    constexpr int CH = D / 8;                          // 16-byte chunks per row
+    constexpr int ITEMS = kBfChunk * CH / kLoaders;    // per thread per chunk (K and V each)
+    static_assert(ITEMS >= 1 && kBfChunk * CH % kLoaders == 0, "whole items per thread");
+    const size_t row_stride = (size_t)Hkv * D;
+    const __nv_bfloat16* Kb = K + (size_t)bi * L * row_stride + (size_t)kh * D;
+    const __nv_bfloat16* Vb = V + (size_t)bi * L * row_stride + (size_t)kh * D;
+    auto issue = [&](int c) {
+      const uint32_t a = sbase + (uint32_t)((c % kBfStages) * TL::STAGE);
+      const uint32_t b = a + 2 * TL::A_BYTES;
+#pragma unroll
+      for (int it = 0; it < ITEMS; ++it) {
+        const int i = tid + it * kLoaders, jj = i / CH, cc = i % CH;
+        const int p = s_pos[c * kBfChunk + jj];
+        const size_t off = (size_t)(p < 0 ? 0 : p) * row_stride + cc * 8;
+        const uint32_t o = bf_off(jj, cc, TL::ATOM_COL);
+        cp_async16_zfill(a + o, Kb + off, p >= 0);
+        cp_async16_zfill(b + o, Vb + off, p >= 0);
+      }
+    };
+    // exactly kBfAhead groups first (empty past the run's end), one per
+    // iteration after: group k then holds chunk k, and waiting until at most
+    // kBfAhead groups are pending at iteration c means chunk c has landed
+    for (int c = 0; c < kBfAhead; ++c) {
+      if (c < nchunks) issue(c);
+      cp_async_commit_group();
+    }
+    for (int c = 0; c < nchunks; ++c) {
+      const int cn = c + kBfAhead;
+      if (cn < nchunks) {
+        // its stage last held chunk cn - kBfStages (= c - 2): wait for that MMA
+        if (cn >= kBfStages &&
+            !tc::mbar_wait(empty0 + 8 * (cn % kBfStages), ((cn / kBfStages) - 1) & 1)) {
+          record_error(err, DEV_TIMEOUT);
+          s_abort = 1;
+          break;
+        }
+        issue(cn);
+      }
+      cp_async_commit_group();          // (possibly empty) keeps the group count uniform
+      cp_async_wait_group<kBfAhead>();  // this thread's copies of chunk c have landed
+      // A: the key rows this thread copied, scaled by the decay weight and
+      // split into hi (in place) and lo
+      unsigned char* a_p = smem + (c % kBfStages) * TL::STAGE;
+#pragma unroll
+      for (int it = 0; it < ITEMS; ++it) {
+        const int i = tid + it * kLoaders, jj = i / CH, cc = i % CH;
+        const int j = j0 + c * kBfChunk + jj;
+        const float w = j < j1 ? exp2f((float)(j1 - 1 - j) * log2lam) : 0.f;
+        const uint32_t o = bf_off(jj, cc, TL::ATOM_COL);
+        const uint4 raw = *reinterpret_cast<const uint4*>(a_p + o);
+        float kf[8];
+        bf16x8_to_f32(raw, kf);
+        uint4 hi, lo;
+        uint32_t* hw = reinterpret_cast<uint32_t*>(&hi);
+        uint32_t* lw = reinterpret_cast<uint32_t*>(&lo);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float x0 = w * kf[2 * e], x1 = w * kf[2 * e + 1];
+          const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+          const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - __low2float(h), x1 - __high2float(h));
+          hw[e] = *reinterpret_cast<const uint32_t*>(&h);
+          lw[e] = *reinterpret_cast<const uint32_t*>(&l);
+        }
+        *reinterpret_cast<uint4*>(a_p + o) = hi;
+        *reinterpret_cast<uint4*>(a_p + TL::A_BYTES + o) = lo;
+      }
+      tc::fence_proxy_async();   // generic-proxy shared writes (and landed copies) -> MMA
+      tc::mbar_arrive(full0 + 8 * (c % kBfStages));
+    }
+    cp_async_wait_group<0>();   // nothing of this thread in flight past here
+    if (bad) record_error(err, DEV_RANGE);
+  } else if (lane == 0) {
+    // ---------------- MMA issuer: 2 x (16-token steps) x (hi, lo) per chunk
+    constexpr uint32_t IDESC = tc::idesc(tc::kFmtBF16, 128, TL::N, true, true);
+    for (int c = 0; c < nchunks; ++c) {
+      const int st = c % kBfStages;
+      if (!tc::mbar_wait(full0 + 8 * st, (c / kBfStages) & 1)) {
+        record_error(err, DEV_TIMEOUT);
+        s_abort = 1;
+        break;
+      }
+      tc::fence_after();
+      const uint32_t a_t = sbase + st * TL::STAGE, b_t = a_t + 2 * TL::A_BYTES;
+#pragma unroll
+      for (int k = 0; k < kBfChunk / 16; ++k) {
+        const uint64_t bd = tc::sdesc_sw128(b_t + k * 2048, TL::ATOM_COL, 1024);
+        const uint64_t ah = tc::sdesc_sw128(a_t + k * 2048, TL::ATOM_COL, 1024);
+        const uint64_t al = tc::sdesc_sw128(a_t + TL::A_BYTES + k * 2048, TL::ATOM_COL, 1024);
+        tc::mma_f16(tmem, ah, bd, IDESC, (c > 0 || k > 0) ? 1u : 0u);
+        tc::mma_f16(tmem, al, bd, IDESC, 1u);
+      }
+      tc::mma_commit(empty0 + 8 * st);
+    }
+    tc::mma_commit(done);
+  }
+
+  // ---------------- epilogue: warps 0-3 read [S | s] rows from TMEM
+  pdl_launch();
+  if (warp < 4) {
+    const int row = warp * 32 + lane;   // feature index of k (TMEM lane)
+    bool ok = true;
+    if (nchunks > 0) ok = tc::mbar_wait(done, 0);
+    if (!ok) record_error(err, DEV_TIMEOUT);
+    tc::fence_after();
+    if (nchunks > 0 && ok && !s_abort) {
+#pragma unroll 1
+      for (int c0 = 0; c0 < TL::N; c0 += 16) {
+        float v[16];
+        tc::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + c0, v);
+        if (row < D) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int col = c0 + e;
+            if (col <= D) out[(size_t)row * (D + 1) + col] = v[e];
+          }
+        }
+      }
+    } else if (row < D) {
+      for (int col = 0; col <= D; ++col) out[(size_t)row * (D + 1) + col] = 0.f;
+    }
+  }
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 8) tc::tmem_dealloc(tmem, 256);
+}
+
+// Launches the finalize with programmatic stream serialization (it waits for
+// the tensor-core pass itself, after staging W_phi).
+template <int D>
+cudaError_t launch_finalize(dim3 grid, size_t smem, cudaStream_t st, const float* partials, int G,
+                            int tpg, int n_tok, float log2lam, const float* W_phi, int r,
+                            float decay_n, float* M, float* bstab, const float* sv_partials,
+                            float* s_v, float* n_count, float n_add, int Hkv) {
+  cudaError_t e = cudaFuncSetAttribute(memory_finalize_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, memory_finalize_kernel<D>, partials, G, tpg, n_tok, log2lam,
+                            W_phi, r, decay_n, M, bstab, sv_partials, s_v, n_count, n_add, Hkv);
+}
+
 }  // namespace
 
-// Number of runs the evicted tokens are split into per (sequence, KV head):
-// about two CTAs per SM, each run a whole number of `chunk` tokens.
-int memory_groups(int batch, int n_kv_heads, int n_e, int chunk) {
+// Split of the evicted tokens of every (sequence, KV head) into runs: a whole
+// number of 64-token chunks per run, about two CTAs per SM in one wave
+// (units * runs <= 2 * num_sms where the tokens allow). tokens_per_run is the
+// run length; the last run of a unit may be shorter. The result does not
+// depend on the split (the finalize applies each run's decay factor).
+struct MemSplit { int runs, tokens_per_run; };
+MemSplit memory_split(int batch, int n_kv_heads, int n_e, int num_sms, size_t max_runs_total) {
   const int units = batch * n_kv_heads;
-  const int chunks = (n_e + chunk - 1) / chunk;
-  int G = (2 * 148 + units / 2) / units;
+  const int chunks = (n_e + kChunk - 1) / kChunk;
+  int G = (2 * num_sms) / units;
   if (G > chunks) G = chunks;
   if (G > kMemMaxGroups) G = kMemMaxGroups;
+  while (G > 1 && (size_t)units * G > max_runs_total) --G;
   if (G < 1) G = 1;
-  return G;
+  const int tpr = ((chunks + G - 1) / G) * kChunk;
+  return MemSplit{(n_e + tpr - 1) / tpr, tpr};
+}
+
+// Runs of the bf16 kernel (one CTA per SM): at least ceil(n / kRunMax) runs
+// per unit (the run's positions sit in shared memory), a whole number of
+// 32-token chunks each; among the run counts up to four waves, the one whose
+// last wave is fullest (the fewest runs within 3% of the best), so that SMs do
+// not idle in a partial wave.
+MemSplit memory_split_bf16(int batch, int n_kv_heads, int n_e, int num_sms) {
+  const int units = batch * n_kv_heads;
+  const int chunks = (n_e + kBfChunk - 1) / kBfChunk;
+  int lo = (n_e + kRunMax - 1) / kRunMax;
+  if (lo < 1) lo = 1;
+  int hi = (4 * num_sms) / units;
+  if (hi > chunks) hi = chunks;
+  if (hi > kMemMaxGroups) hi = kMemMaxGroups;
+  if (hi < lo) hi = lo;
+  double best = -1.0;
+  int G = lo;
+  for (int g = lo; g <= hi; ++g) {
+    const long ctas = (long)units * g;
+    const long waves = (ctas + num_sms - 1) / num_sms;
+    const double eff = (double)ctas / (double)(waves * num_sms);
+    if (eff > best + 0.03) { best = eff; G = g; }
+  }
+  const int tpr = ((chunks + G - 1) / G) * kBfChunk;
+  return MemSplit{(n_e + tpr - 1) / tpr, tpr};
+}
+
+// Upper bound of units * runs over both kernels for up to L evicted tokens
+// per unit (sizes the partial sums in the workspace).
+size_t memory_runs_bound(int units, int L, int num_sms) {
+  return (size_t)units * ((L + kRunMax - 1) / kRunMax + 1) + 4 * (size_t)num_sms + units;
 }
 
 cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, const void* V,
@@ -407,13 +754,31 @@ cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, 
                                  cudaStream_t st) {
   if (n_e == 0) return cudaSuccess;
   const int Hkv = c.cfg.n_kv_heads, D = c.cfg.head_dim, r = c.cfg.mem_r;
-  const int G = memory_groups(batch, Hkv, n_e, chunk);
-  const int chunks = (n_e + chunk - 1) / chunk;
-  const int tokens_per_group = ((chunks + G - 1) / G) * chunk;
-  const int Gused = (n_e + tokens_per_group - 1) / tokens_per_group;   // no empty runs
+  (void)chunk;   // the split below does not change the result
+  // bf16 gated memory: the cp.async-fed kernel, unless a run would exceed the
+  // run count the finalize handles (n_e beyond kMemMaxGroups * kRunMax)
+  const bool bf16_path = c.cfg.dtype == IMEM_BF16 && !sv_partials &&
+                         (n_e + kRunMax - 1) / kRunMax <= kMemMaxGroups;
+  const MemSplit sp = bf16_path ? memory_split_bf16(batch, Hkv, n_e, c.num_sms)
+                                : memory_split(batch, Hkv, n_e, c.num_sms,
+                                               (size_t)batch * Hkv + 2 * 148);
+  const int tokens_per_group = sp.tokens_per_run;
+  const int Gused = sp.runs;
   dim3 grid(Gused, Hkv, batch);
   const float log2lam = (float)log2((double)c.cfg.lambda);
   cudaError_t e = cudaSuccess;
+#define IMEM_MEMBF(DD)                                                                        \
+  do {                                                                                        \
+    e = cudaFuncSetAttribute(memory_bf16_kernel<DD>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             BfTile<DD>::SMEM);                                               \
+    if (e != cudaSuccess) return e;                                                           \
+    memory_bf16_kernel<DD><<<grid, kMemThreads, BfTile<DD>::SMEM, st>>>(                      \
+        (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, idx_e, n_e, L, Hkv, log2lam,        \
+        tokens_per_group, partials, c.err);                                                   \
+  } while (0)
+  if (bf16_path) {
+    if (D == 128) IMEM_MEMBF(128); else IMEM_MEMBF(64);
+  } else {
 #define IMEM_MEM(TT, DD)                                                                       \
   do {                                                                                         \
     auto kfn = sv_partials ? memory_tc_kernel<TT, DD, true> : memory_tc_kernel<TT, DD, false>; \
@@ -429,7 +794,9 @@ cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, 
   } else {
     if (D == 128) IMEM_MEM(float, 128); else IMEM_MEM(float, 64);
   }
+  }
 #undef IMEM_MEM
+#undef IMEM_MEMBF
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const float decay_n = (float)pow((double)c.cfg.lambda, (double)n_e);
@@ -437,21 +804,13 @@ cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, 
   // moment statistics use the identity map: the finalize skips the product
   const float* phi = c.cfg.readout == IMEM_READOUT_MOMENT ? nullptr : c.W_phi;
   const size_t fsmem = ((size_t)r * D + (size_t)D * 16) * sizeof(float);
-  if (D == 128) {
-    e = cudaFuncSetAttribute(memory_finalize_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem);
-    if (e != cudaSuccess) return e;
-    memory_finalize_kernel<128><<<fgrid, 256, fsmem, st>>>(partials, Gused, tokens_per_group,
-                                                           n_e, log2lam, phi, r, decay_n, M,
-                                                           bstab, sv_partials, s_v, n_count,
-                                                           (float)n_e, Hkv);
-  } else {
-    e = cudaFuncSetAttribute(memory_finalize_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem);
-    if (e != cudaSuccess) return e;
-    memory_finalize_kernel<64><<<fgrid, 256, fsmem, st>>>(partials, Gused, tokens_per_group,
-                                                          n_e, log2lam, phi, r, decay_n, M,
-                                                          bstab, sv_partials, s_v, n_count,
-                                                          (float)n_e, Hkv);
-  }
+  if (D == 128)
+    e = launch_finalize<128>(fgrid, fsmem, st, partials, Gused, tokens_per_group, n_e, log2lam,
+                             phi, r, decay_n, M, bstab, sv_partials, s_v, n_count, (float)n_e, Hkv);
+  else
+    e = launch_finalize<64>(fgrid, fsmem, st, partials, Gused, tokens_per_group, n_e, log2lam,
+                            phi, r, decay_n, M, bstab, sv_partials, s_v, n_count, (float)n_e, Hkv);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -502,11 +861,13 @@ cudaError_t launch_memory_static(int batch, int L, int Hkv, int r, float lambda,
                                  int* err, cudaStream_t st) {
   const int units = batch * Hkv;
   const size_t psize = (size_t)D * (D + 1) * sizeof(float);
-  int G = memory_groups(batch, Hkv, n_e, chunk);
-  while (G > 1 && (size_t)units * G * psize > kStaticScratchBytes) --G;
-  const int chunks = (n_e + chunk - 1) / chunk;
-  const int tokens_per_group = ((chunks + G - 1) / G) * chunk;
-  const int Gused = (n_e + tokens_per_group - 1) / tokens_per_group;
+  (void)chunk;
+  int num_sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+  const MemSplit sp = memory_split(batch, Hkv, n_e, num_sms, kStaticScratchBytes / psize);
+  const int tokens_per_group = sp.tokens_per_run;
+  const int Gused = sp.runs;
   const float log2lam = (float)log2((double)lambda);
   auto kfn = memory_tc_kernel<T, D, false>;
   cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -519,12 +880,9 @@ cudaError_t launch_memory_static(int batch, int L, int Hkv, int r, float lambda,
   if (e != cudaSuccess) return e;
   const float decay_n = (float)pow((double)lambda, (double)n_e);
   const size_t fsmem = ((size_t)r * D + (size_t)D * 16) * sizeof(float);
-  e = cudaFuncSetAttribute(memory_finalize_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)fsmem);
+  e = launch_finalize<D>(dim3(D / 16 + 1, units), fsmem, st, scratch, Gused, tokens_per_group, n_e,
+                         log2lam, W_phi, r, decay_n, M, bstab, nullptr, nullptr, nullptr, 0.f, Hkv);
   if (e != cudaSuccess) return e;
-  memory_finalize_kernel<D><<<dim3(D / 16 + 1, units), 256, fsmem, st>>>(
-      scratch, Gused, tokens_per_group, n_e, log2lam, W_phi, r, decay_n, M, bstab, nullptr,
-      nullptr, nullptr, 0.f, Hkv);
   return cudaGetLastError();
 }
 

@@ -7,28 +7,31 @@
 // queries that arrive).
 //
 // The cache holds B tokens in slots [0, B) in any order, each with its
-// indexer key k^ (bf16), importance I and position. Per decode step, after
-// the attention step (which appends the new token at slot B):
+// indexer key k^ (bf16), importance I and position. Per decode step:
 //   features  the new token's indexer query q~ = sum_h g_h q^_h / sqrt(dI)
 //             and key k^ (per-head projections of the attention query, gate
 //             logits and key from the hidden state, RMS norms): Hq + 8 CTAs
-//             per sequence, one GEMV each, partials in the workspace;
-//   score     I_t <- max(I_t, q~ . k^_t) for the cached tokens, the new
+//             per sequence, one GEMV each, partials in the workspace. It
+//             needs neither the cache nor the memory, so the C ABI runs it
+//             on a second stream next to the attention step (which appends
+//             the new token at slot B);
+//   score + evict  (after both) one thread-block cluster per sequence:
+//             I_t <- max(I_t, q~ . k^_t) for the cached tokens, the new
 //             token's I = q~ . k^_new; the least important of the B + 1
-//             (ties: the higher position) is found by a per-CTA minimum of a
-//             packed (ordered importance, inverted position) key and a
-//             last-CTA reduction;
-//   evict     per KV head: phi = W_phi k_e, M <- lambda M + phi v_e^T,
-//             b <- lambda b + phi; the new token and the evicted one swap
-//             slots (row, indexer key, importance, position), so slot B keeps
-//             the token that left with the importance it was chosen by;
-//             cache_len returns to B and the workspace's decode tag
-//             of the sequence to B + 1 (the next decode step may then use
-//             the rows it loads before its launch-dependency wait).
+//             (ties: the higher position) by per-CTA minima of a packed
+//             (ordered importance, inverted position) key exchanged over
+//             distributed shared memory; per KV head phi = W_phi k_e,
+//             M <- lambda M + phi v_e^T, b <- lambda b + phi; the new token
+//             and the evicted one swap slots (row, indexer key, importance,
+//             position), so slot B keeps the token that left with the
+//             importance it was chosen by; cache_len returns to B and the
+//             workspace's decode tag of the sequence is cleared (rows of
+//             slot e and the memory changed after the attention step).
 // q~ and k^ are rounded to bf16 before their dot products, as in prefill.
 #include "common.cuh"
 #include "internal.h"
 
+#include <cooperative_groups.h>
 #include <math.h>
 
 namespace imem {
@@ -181,27 +184,52 @@ online_features_kernel(const T* __restrict__ x, const T* __restrict__ q, const T
   }
 }
 
-// ---- importances and the token to evict --------------------------------------
-struct EvictCand {
-  unsigned long long key;   // ordered importance << 32 | ~position (min wins)
-  int slot;
-  int pad;
-};
+// ---- importances, the token to evict and the memory update -----------------
+// One thread-block cluster of nct CTAs per sequence. Each CTA takes a
+// contiguous block of the B + 1 candidate rows (slot B: the new token):
+// I_t <- max(I_t, q~ . k^_t) for the cached tokens, the new token's I =
+// q~ . k^_new, and its block's least important candidate as a packed key
+// (ordered importance << 32 | ~position: the minimum is the least important,
+// ties to the higher position). The CTAs exchange their keys through
+// distributed shared memory and, after one cluster barrier, all know the
+// token e to evict. Then CTA r updates the memory of the KV heads h = r,
+// r + nct, ...: M <- lambda M + phi(k_e) v_e^T, b <- lambda b + phi(k_e),
+// and swaps the rows of e and B of those heads (the new token takes slot e,
+// the evicted token slot B); the CTA owning row e swaps the indexer keys,
+// importances and positions of the two slots.
+__device__ __forceinline__ float order_key_inv(uint32_t o) {
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
 
+template <typename T>
 __global__ void __launch_bounds__(kOnThreads)
-online_score_kernel(int B, int cap, int Hq, int dI, int rows_per_cta,
-                    const float* __restrict__ qpart, const float* __restrict__ kpart,
-                    __nv_bfloat16* __restrict__ khat_ret, float* __restrict__ I_ret,
-                    int32_t* __restrict__ pos_ret, const int32_t* __restrict__ next_pos,
-                    EvictCand* __restrict__ cand, int* __restrict__ counter,
-                    int* __restrict__ evict_slot, int32_t* __restrict__ evicted) {
+online_score_evict_kernel(int B, int cap, int Hq, int Hkv, int D, int dI, int r, float lambda,
+                          int rows_per_cta, const float* __restrict__ qpart,
+                          const float* __restrict__ kpart, const float* __restrict__ W_phi,
+                          T* __restrict__ K_ret, T* __restrict__ V_ret,
+                          __nv_bfloat16* __restrict__ khat_ret, float* __restrict__ I_ret,
+                          int32_t* __restrict__ pos_ret, int32_t* __restrict__ next_pos,
+                          int32_t* __restrict__ cache_len, float* __restrict__ M,
+                          float* __restrict__ bstab, int32_t* __restrict__ evicted,
+                          int* __restrict__ dec_tag) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ float osm[];
+  float* sk = osm;          // [D]
+  float* sv = sk + D;       // [D]
+  float* sphi = sv + D;     // [r]
   __shared__ float s_qt[64], s_kn[64];
   __shared__ float red[kOnThreads / 32];
   __shared__ unsigned long long s_key[kOnThreads / 32];
   __shared__ int s_slot[kOnThreads / 32];
-  __shared__ int s_last;
+  __shared__ unsigned long long s_ckey[kOnlineMaxCluster];   // one per CTA of the cluster
+  __shared__ int s_cslot[kOnlineMaxCluster];
+  __shared__ float s_Inew;
   const int bi = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nct = gridDim.x;
+  const int nct = gridDim.x, rank = blockIdx.x;
+  // phase 0 of the cluster barrier: "this CTA is running" (its shared memory
+  // may be written by the others only after every CTA has arrived)
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory");
   pdl_wait();
   pdl_launch();
   // q~ (sum over heads: 4 groups of heads per feature, loads in flight
@@ -224,10 +252,17 @@ online_score_kernel(int B, int cap, int Hq, int dI, int rows_per_cta,
   if (tid < dI) s_kn[tid] = bf16_round(kv * rsqrtf(ss / dI + 1e-6f));
   for (int j = tid + dI; j < 64; j += kOnThreads) { s_qt[j] = 0.f; s_kn[j] = 0.f; }
   __syncthreads();
+  if (warp == 0) {   // the new token's importance: its own score
+    float a = fmaf(s_kn[lane], s_qt[lane], s_kn[lane + 32] * s_qt[lane + 32]);
+    a = warp_sum(a);
+    if (lane == 0) s_Inew = a;
+  }
+  __syncthreads();
+  const int npos = next_pos[bi];
 
   unsigned long long best = ~0ull;
   int best_slot = -1;
-  const int t0 = blockIdx.x * rows_per_cta, t1 = min(B + 1, t0 + rows_per_cta);
+  const int t0 = rank * rows_per_cta, t1 = min(B + 1, t0 + rows_per_cta);
   for (int t = t0 + tid; t < t1; t += kOnThreads) {
     float I;
     int pos;
@@ -245,23 +280,13 @@ online_score_kernel(int B, int cap, int Hq, int dI, int rows_per_cta,
       I_ret[(size_t)bi * cap + t] = I;
       pos = pos_ret[(size_t)bi * cap + t];
     } else {   // slot B: the new token, scored by its own query
-      float a = 0.f;
-      for (int c = 0; c < 64; ++c) a = fmaf(s_kn[c], s_qt[c], a);
-      I = a;
-      pos = next_pos[bi];
-      I_ret[(size_t)bi * cap + B] = I;
-      pos_ret[(size_t)bi * cap + B] = pos;
-      float f[8];
-      for (int c = 0; c < kIdxPad / 8; ++c) {
-        for (int e = 0; e < 8; ++e) f[e] = s_kn[8 * c + e];
-        store8<__nv_bfloat16>(khat_ret + ((size_t)bi * cap + B) * kIdxPad + 8 * c, f);
-      }
+      I = s_Inew;
+      pos = npos;
     }
     const unsigned long long key =
         ((unsigned long long)order_key(I) << 32) | (unsigned long long)(~(uint32_t)pos);
     if (key < best) { best = key; best_slot = t; }
   }
-  // CTA minimum
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const unsigned long long k2 = __shfl_xor_sync(0xffffffffu, best, o);
@@ -270,126 +295,116 @@ online_score_kernel(int B, int cap, int Hq, int dI, int rows_per_cta,
   }
   if (lane == 0) { s_key[warp] = best; s_slot[warp] = best_slot; }
   __syncthreads();
-  if (tid == 0) {
+  asm volatile("barrier.cluster.wait.aligned;\n" ::: "memory");   // phase 0: all running
+  if (tid < nct) {
+    // this CTA's candidate into slot `rank` of CTA tid's exchange arrays
+    unsigned long long k = s_key[0];
+    int sl = s_slot[0];
     for (int w = 1; w < kOnThreads / 32; ++w)
-      if (s_key[w] < best) { best = s_key[w]; best_slot = s_slot[w]; }
-    cand[(size_t)bi * nct + blockIdx.x] = EvictCand{best, best_slot, 0};
-    __threadfence();
-    s_last = atomicAdd(&counter[bi], 1) == nct - 1;
+      if (s_key[w] < k) { k = s_key[w]; sl = s_slot[w]; }
+    cluster.map_shared_rank(s_ckey, tid)[rank] = k;
+    cluster.map_shared_rank(s_cslot, tid)[rank] = sl;
   }
-  __syncthreads();
-  if (s_last && tid == 0) {
-    // the last CTA of the sequence reduces the candidates
-    __threadfence();
-    unsigned long long k = ~0ull;
-    int slot = -1;
-    for (int i = 0; i < nct; ++i) {
-      const EvictCand ci = cand[(size_t)bi * nct + i];
-      if (ci.key < k) { k = ci.key; slot = ci.slot; }
-    }
-    evict_slot[bi] = slot;
-    evicted[bi] = (int32_t)(~(uint32_t)(k & 0xffffffffull));
-    counter[bi] = 0;
+  cluster.sync();   // every CTA has written its candidate into every CTA
+  unsigned long long k = ~0ull;
+  int e = -1;
+  for (int i = 0; i < nct; ++i)
+    if (s_ckey[i] < k) { k = s_ckey[i]; e = s_cslot[i]; }
+  int pos_e = (int32_t)(~(uint32_t)(k & 0xffffffffull));
+  float I_e = order_key_inv((uint32_t)(k >> 32));
+  if (e < 0) {   // no ordered candidate (NaN importances): the new token leaves
+    e = B; pos_e = npos; I_e = s_Inew;
   }
-}
 
-// ---- memory update with the evicted token, slot refill ------------------------
-template <typename T>
-__global__ void __launch_bounds__(kOnThreads)
-online_evict_kernel(int B, int cap, int Hkv, int D, int r, float lambda,
-                    const int* __restrict__ evict_slot, const float* __restrict__ W_phi,
-                    T* __restrict__ K_ret, T* __restrict__ V_ret,
-                    __nv_bfloat16* __restrict__ khat_ret, float* __restrict__ I_ret,
-                    int32_t* __restrict__ pos_ret, int32_t* __restrict__ next_pos,
-                    int32_t* __restrict__ cache_len, float* __restrict__ M,
-                    float* __restrict__ bstab, int* __restrict__ dec_tag) {
-  extern __shared__ float osm[];
-  float* sk = osm;          // [D]
-  float* sv = sk + D;       // [D]
-  float* sphi = sv + D;     // [r]
-  const int kh = blockIdx.x, bi = blockIdx.y, tid = threadIdx.x;
-  pdl_wait();
-  pdl_launch();
-  const int e = evict_slot[bi];
+  // memory update and row swap for this CTA's KV heads
   const size_t rs = (size_t)Hkv * D;
-  T* ke = K_ret + ((size_t)bi * cap + e) * rs + (size_t)kh * D;
-  T* ve = V_ret + ((size_t)bi * cap + e) * rs + (size_t)kh * D;
-  for (int c = tid; c < D; c += kOnThreads) { sk[c] = ldf(ke + c); sv[c] = ldf(ve + c); }
-  __syncthreads();
-  // phi = W_phi k: 4 threads per row, float4 loads (D/16 each, in flight together)
-  for (int j0 = 0; j0 < r; j0 += kOnThreads / 4) {
-    const int j = j0 + tid / 4, part = tid & 3;
-    float a = 0.f;
-    if (j < r) {
-      const float4* wr = reinterpret_cast<const float4*>(W_phi + (size_t)j * D);
+  for (int kh = rank; kh < Hkv; kh += nct) {
+    T* ke = K_ret + ((size_t)bi * cap + e) * rs + (size_t)kh * D;
+    T* ve = V_ret + ((size_t)bi * cap + e) * rs + (size_t)kh * D;
+    for (int c = tid; c < D; c += kOnThreads) { sk[c] = ldf(ke + c); sv[c] = ldf(ve + c); }
+    __syncthreads();
+    // phi = W_phi k: 4 threads per row, float4 loads
+    for (int j0 = 0; j0 < r; j0 += kOnThreads / 4) {
+      const int j = j0 + tid / 4, part = tid & 3;
+      float a = 0.f;
+      if (j < r) {
+        const float4* wr = reinterpret_cast<const float4*>(W_phi + (size_t)j * D);
 #pragma unroll 8
-      for (int c4 = part; c4 < D / 4; c4 += 4) {
-        const float4 w = __ldg(wr + c4);
-        a = fmaf(w.x, sk[4 * c4], fmaf(w.y, sk[4 * c4 + 1], fmaf(w.z, sk[4 * c4 + 2], fmaf(w.w, sk[4 * c4 + 3], a))));
+        for (int c4 = part; c4 < D / 4; c4 += 4) {
+          const float4 w = __ldg(wr + c4);
+          a = fmaf(w.x, sk[4 * c4], fmaf(w.y, sk[4 * c4 + 1], fmaf(w.z, sk[4 * c4 + 2], fmaf(w.w, sk[4 * c4 + 3], a))));
+        }
+      }
+      a += __shfl_xor_sync(0xffffffffu, a, 1);
+      a += __shfl_xor_sync(0xffffffffu, a, 2);
+      if (j < r && part == 0) sphi[j] = a;
+    }
+    __syncthreads();
+    float4* Mu = reinterpret_cast<float4*>(M + ((size_t)bi * Hkv + kh) * r * D);
+#pragma unroll 4
+    for (int i = tid; i < r * D / 4; i += kOnThreads) {
+      const int j = (4 * i) / D, c = (4 * i) % D;
+      float4 m = Mu[i];
+      const float ph = sphi[j];
+      m.x = fmaf(lambda, m.x, ph * sv[c]);
+      m.y = fmaf(lambda, m.y, ph * sv[c + 1]);
+      m.z = fmaf(lambda, m.z, ph * sv[c + 2]);
+      m.w = fmaf(lambda, m.w, ph * sv[c + 3]);
+      Mu[i] = m;
+    }
+    for (int j = tid; j < r; j += kOnThreads) {
+      float* bp = bstab + ((size_t)bi * Hkv + kh) * r + j;
+      *bp = fmaf(lambda, *bp, sphi[j]);
+    }
+    if (e != B) {   // the new token (slot B) and the evicted one swap rows
+      T* kn = K_ret + ((size_t)bi * cap + B) * rs + (size_t)kh * D;
+      T* vn = V_ret + ((size_t)bi * cap + B) * rs + (size_t)kh * D;
+      for (int c = tid; c < D; c += kOnThreads) {
+        const T k0 = ke[c], v0 = ve[c];
+        ke[c] = kn[c]; ve[c] = vn[c];
+        kn[c] = k0; vn[c] = v0;
       }
     }
-    a += __shfl_xor_sync(0xffffffffu, a, 1);
-    a += __shfl_xor_sync(0xffffffffu, a, 2);
-    if (j < r && part == 0) sphi[j] = a;
+    __syncthreads();   // sk, sv, sphi reused by the next head
   }
-  __syncthreads();
-  // M <- lambda M + phi v^T, float4 read-modify-write (r*D/4 per head)
-  float4* Mu = reinterpret_cast<float4*>(M + ((size_t)bi * Hkv + kh) * r * D);
-#pragma unroll 4
-  for (int i = tid; i < r * D / 4; i += kOnThreads) {
-    const int j = (4 * i) / D, c = (4 * i) % D;
-    float4 m = Mu[i];
-    const float ph = sphi[j];
-    m.x = fmaf(lambda, m.x, ph * sv[c]);
-    m.y = fmaf(lambda, m.y, ph * sv[c + 1]);
-    m.z = fmaf(lambda, m.z, ph * sv[c + 2]);
-    m.w = fmaf(lambda, m.w, ph * sv[c + 3]);
-    Mu[i] = m;
-  }
-  for (int j = tid; j < r; j += kOnThreads) {
-    float* bp = bstab + ((size_t)bi * Hkv + kh) * r + j;
-    *bp = fmaf(lambda, *bp, sphi[j]);
-  }
-  if (e != B) {   // the new token (slot B) and the evicted one swap slots
-    T* kn = K_ret + ((size_t)bi * cap + B) * rs + (size_t)kh * D;
-    T* vn = V_ret + ((size_t)bi * cap + B) * rs + (size_t)kh * D;
-    for (int c = tid; c < D; c += kOnThreads) {
-      const T k0 = ke[c], v0 = ve[c];
-      ke[c] = kn[c]; ve[c] = vn[c];
-      kn[c] = k0; vn[c] = v0;
-    }
-  }
-  if (kh == 0 && tid < kIdxPad / 8) {
-    if (e != B) {
+  // indexer key, importance and position: slot e takes the new token, slot B
+  // keeps the evicted one (the CTA whose block holds row e)
+  if (e >= t0 && e < t1) {
+    if (tid < kIdxPad / 8) {
+      uint4* hb = reinterpret_cast<uint4*>(khat_ret + ((size_t)bi * cap + B) * kIdxPad) + tid;
       uint4* he = reinterpret_cast<uint4*>(khat_ret + ((size_t)bi * cap + e) * kIdxPad) + tid;
-      uint4* hn = reinterpret_cast<uint4*>(khat_ret + ((size_t)bi * cap + B) * kIdxPad) + tid;
-      const uint4 h0 = *he;
-      *he = *hn;
-      *hn = h0;
+      float f[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) f[c] = s_kn[8 * tid + c];
+      uint4 knew;
+      store8<__nv_bfloat16>(reinterpret_cast<__nv_bfloat16*>(&knew), f);
+      if (e != B) *hb = *he;
+      *he = knew;
     }
     if (tid == 0) {
-      if (e != B) {
-        float* Ie = I_ret + (size_t)bi * cap + e;
-        float* In = I_ret + (size_t)bi * cap + B;
-        int32_t* pe = pos_ret + (size_t)bi * cap + e;
-        int32_t* pn = pos_ret + (size_t)bi * cap + B;
-        const float I0 = *Ie;
-        const int32_t p0 = *pe;
-        *Ie = *In; *pe = *pn;
-        *In = I0; *pn = p0;
-      }
-      cache_len[bi] = B;
-      dec_tag[bi] = B + 1;   // the next decode step may use rows it loads before its wait
-      next_pos[bi] += 1;
+      I_ret[(size_t)bi * cap + e] = s_Inew;
+      pos_ret[(size_t)bi * cap + e] = npos;
+      I_ret[(size_t)bi * cap + B] = I_e;
+      pos_ret[(size_t)bi * cap + B] = pos_e;
     }
+  }
+  if (rank == 0 && tid == 0) {
+    evicted[bi] = pos_e;
+    cache_len[bi] = B;
+    // the rows of slot e and the memory changed after the decode step: the
+    // next decode step must not use rows or memory it loaded before its wait
+    dec_tag[bi] = 0;
+    next_pos[bi] = npos + 1;
   }
 }
 
 }  // namespace
 
-int online_score_ctas(int B) {
+// CTAs per sequence of the score-and-evict cluster: one per 256 candidate rows,
+// at most kOnlineMaxCluster.
+int online_cluster_ctas(int B) {
   int n = (B + 1 + kOnThreads - 1) / kOnThreads;
-  return n > kOnlineMaxCtas ? kOnlineMaxCtas : n;
+  return n > kOnlineMaxCluster ? kOnlineMaxCluster : (n < 1 ? 1 : n);
 }
 
 cudaError_t launch_online_init(const Ctx& c, int batch, int L, int B, int cap,
@@ -432,28 +447,41 @@ cudaError_t launch_online_features(const Ctx& c, int batch, const void* x, const
                     qpart, kpart);
 }
 
-cudaError_t launch_online_evict(const Ctx& c, int batch, int B, int cap, const float* qpart,
-                                const float* kpart, void* khat_ret, float* I_ret, int32_t* pos_ret,
-                                int32_t* next_pos, void* K_ret, void* V_ret, int32_t* cache_len,
-                                float* M, float* bstab, int32_t* evicted, void* cand,
-                                int* counter, int* evict_slot, int* dec_tag, cudaStream_t st) {
-  const int nct = online_score_ctas(B);
+cudaError_t launch_online_score_evict(const Ctx& c, int batch, int B, int cap, const float* qpart,
+                                      const float* kpart, void* khat_ret, float* I_ret,
+                                      int32_t* pos_ret, int32_t* next_pos, void* K_ret,
+                                      void* V_ret, int32_t* cache_len, float* M, float* bstab,
+                                      int32_t* evicted, int* dec_tag, cudaStream_t st) {
+  const int nct = online_cluster_ctas(B);
   const int rows_per_cta = (B + 1 + nct - 1) / nct;
-  cudaError_t e = launch_pdl(online_score_kernel, dim3(nct, batch), 0, st, B, cap,
-                             c.cfg.n_q_heads, c.cfg.idx_dim, rows_per_cta, qpart, kpart,
-                             khat_ret, I_ret, pos_ret, next_pos, cand, counter, evict_slot,
-                             evicted);
-  if (e != cudaSuccess) return e;
   const int Hkv = c.cfg.n_kv_heads, D = c.cfg.head_dim, r = c.cfg.mem_r;
   const size_t sm = (size_t)(2 * D + r) * sizeof(float);
-  dim3 g(Hkv, batch);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nct, batch, 1);
+  cfg.blockDim = dim3(kOnThreads, 1, 1);
+  cfg.dynamicSmemBytes = sm;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = nct;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
   if (c.cfg.dtype == IMEM_BF16)
-    return launch_pdl(online_evict_kernel<__nv_bfloat16>, g, sm, st, B, cap, Hkv, D, r,
-                      c.cfg.lambda, evict_slot, c.W_phi, K_ret, V_ret, khat_ret, I_ret, pos_ret,
-                      next_pos, cache_len, M, bstab, dec_tag);
-  return launch_pdl(online_evict_kernel<float>, g, sm, st, B, cap, Hkv, D, r, c.cfg.lambda,
-                    evict_slot, c.W_phi, K_ret, V_ret, khat_ret, I_ret, pos_ret, next_pos,
-                    cache_len, M, bstab, dec_tag);
+    return cudaLaunchKernelEx(&cfg, online_score_evict_kernel<__nv_bfloat16>, B, cap,
+                              c.cfg.n_q_heads, Hkv, D, c.cfg.idx_dim, r, c.cfg.lambda,
+                              rows_per_cta, qpart, kpart, (const float*)c.W_phi,
+                              (__nv_bfloat16*)K_ret, (__nv_bfloat16*)V_ret,
+                              (__nv_bfloat16*)khat_ret, I_ret, pos_ret, next_pos, cache_len, M,
+                              bstab, evicted, dec_tag);
+  return cudaLaunchKernelEx(&cfg, online_score_evict_kernel<float>, B, cap, c.cfg.n_q_heads, Hkv,
+                            D, c.cfg.idx_dim, r, c.cfg.lambda, rows_per_cta, qpart, kpart,
+                            (const float*)c.W_phi, (float*)K_ret, (float*)V_ret,
+                            (__nv_bfloat16*)khat_ret, I_ret, pos_ret, next_pos, cache_len, M,
+                            bstab, evicted, dec_tag);
 }
 
 }  // namespace imem

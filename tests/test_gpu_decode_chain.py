@@ -18,7 +18,7 @@ from learned_kv_cache_indexmem_b200 import synth
 from oracle import indexmem_oracle as om
 from oracle import momentkv_oracle as mk
 
-from .parity import Case, check_decode, ill_conditioned, to_np
+from .parity import Case, check_decode, check_memory, ill_conditioned, to_np
 from .test_gpu_parity import _decode_case
 
 pytestmark = pytest.mark.gpu
@@ -153,11 +153,15 @@ def test_library_call_between_chains_clears_the_tag(cuda_device):
     KR, VR = om.compact(to_np(inp_b["K"]), to_np(inp_b["V"]), R, B + steps)
     M_ref, b_ref = om.memory_update(inp_b["K"], inp_b["V"], E, case_a.w_cpu["W_phi"],
                                     wl.shape.lam, M0=to_np(M_before), b0=to_np(b_before))
+    # the memory the step read: the GPU's, checked against the oracle's here;
+    # the oracle's decode then reads the GPU's state
+    M_gpu, b_gpu = to_np(st.M), to_np(st.bstab)
+    check_memory(M_gpu, b_gpu, M_ref, b_ref, "after prefill")
     qc, knc, vnc = (to_np(case_b.dec_cpu[k][0]) for k in ("q", "k_new", "v_new"))
-    o_ref, _, _, _, _ = om.decode_step(qc, knc, vnc, KR, VR, np.full(batch, B), M_ref, b_ref,
+    o_ref, _, _, _, _ = om.decode_step(qc, knc, vnc, KR, VR, np.full(batch, B), M_gpu, b_gpu,
                                        W_phi, w_gate)
     group = wl.shape.n_q_heads // wl.shape.n_kv_heads
-    check_decode(to_np(out), o_ref, ill_conditioned(b_ref, qc, W_phi, group), "after prefill")
+    check_decode(to_np(out), o_ref, ill_conditioned(b_gpu, qc, W_phi, group), "after prefill")
     lay.close()
 
 

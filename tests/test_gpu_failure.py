@@ -1,9 +1,10 @@
 """Failure handling on the GPU without a fault: a bounded device wait that
 runs out is reported by imem_sync as IMEM_ERR_TIMEOUT, cleared by it, and the
 context keeps working (a decode step then matches the oracle). Inputs outside
-what the memory update computes with (a key beyond fp16's range, an evicted
-index outside [0, L)) are caught by the kernel's own checks, reported as
-IMEM_ERR_RANGE, and the context keeps working."""
+what the memory update computes with (an evicted index outside [0, L); with
+fp32 inputs a key beyond fp16's range) are caught by the kernel's own checks,
+reported as IMEM_ERR_RANGE, and the context keeps working; with bf16 inputs a
+key beyond fp16's range is computed correctly."""
 import numpy as np
 import pytest
 import torch
@@ -52,21 +53,24 @@ def test_bounded_wait_timeout_is_reported_and_cleared(cuda_device):
 
 
 def test_memory_update_out_of_range_inputs_are_reported(cuda_device):
+    # bf16 inputs: the keys enter the tensor-core sums as bf16 hi + lo halves
+    # (fp32's range), so a key far beyond fp16's range is computed, not refused
     wl = synth.WORKLOADS["c1"]
     s = wl.shape
     case = Case(wl, cuda_device, L=256, batch=2, n_decode=1)
     lay = case.layer()
     ws = lay.workspace(2, 256, 1, cuda_device)
-    K, V = case.in_dev["K"].clone(), case.in_dev["V"].clone()
+    K = case.in_dev["K"].clone()
     E = synth.make_index_subset(2, 256, 100, 3, cuda_device)
     M = torch.zeros(2, s.n_kv_heads, s.mem_r, s.head_dim, device=cuda_device)
     b = torch.zeros(2, s.n_kv_heads, s.mem_r, device=cuda_device)
-    # a key beyond fp16's largest finite value (bf16 holds it)
     K[1, int(E[1, 40]), 3, 17] = 1.0e5
-    B.update_memory(lay.ctx, 2, 256, K, V, E, 100, 64, M, b, ws)
-    with pytest.raises(B.IndexMemError) as ei:
-        lay.sync()
-    assert ei.value.name == "IMEM_ERR_RANGE"
+    B.update_memory(lay.ctx, 2, 256, K, case.in_dev["V"], E, 100, 64, M, b, ws)
+    lay.sync()
+    M_ref, b_ref = om.memory_update(K.cpu(), case.in_cpu["V"], E.cpu().numpy(),
+                                    case.w_cpu["W_phi"], s.lam)
+    from .parity import check_memory
+    check_memory(to_np(M), to_np(b), M_ref, b_ref, "bf16 key 1e5")
     # an evicted index at L: no row is read, the error is reported
     E2 = E.clone()
     E2[0, 99] = 256
@@ -88,6 +92,22 @@ def test_memory_update_out_of_range_inputs_are_reported(cuda_device):
     lay.sync()
     M_ref, b_ref = om.memory_update(case.in_cpu["K"], case.in_cpu["V"], E.cpu().numpy(),
                                     case.w_cpu["W_phi"], s.lam)
-    from .parity import check_memory
     check_memory(to_np(M), to_np(b), M_ref, b_ref, "after range errors")
     lay.close()
+    # fp32 inputs keep fp16 tensor-core operands: a key beyond fp16's range is
+    # reported as IMEM_ERR_RANGE
+    wl0 = synth.WORKLOADS["c0"]
+    s0 = wl0.shape
+    case0 = Case(wl0, cuda_device, L=256, batch=1, n_decode=1)
+    lay0 = case0.layer()
+    ws0 = lay0.workspace(1, 256, 1, cuda_device)
+    K0 = case0.in_dev["K"].clone()
+    E0 = synth.make_index_subset(1, 256, 100, 4, cuda_device)
+    K0[0, int(E0[0, 7]), 1, 5] = 1.0e5
+    M0 = torch.zeros(1, s0.n_kv_heads, s0.mem_r, s0.head_dim, device=cuda_device)
+    b0 = torch.zeros(1, s0.n_kv_heads, s0.mem_r, device=cuda_device)
+    B.update_memory(lay0.ctx, 1, 256, K0, case0.in_dev["V"], E0, 100, 64, M0, b0, ws0)
+    with pytest.raises(B.IndexMemError) as ei:
+        lay0.sync()
+    assert ei.value.name == "IMEM_ERR_RANGE"
+    lay0.close()

@@ -97,3 +97,75 @@ def test_online_eviction_parity(cuda_device, name, L, B, steps, batch):
         assert np.all(to_np(st.cache_len) == B)
         assert np.all(to_np(on.next_pos) == t + 1)
     lay.close()
+
+
+def test_online_steps_back_to_back_equal_synchronised_steps(cuda_device):
+    """The same online steps from the same state, (a) with a host
+    synchronisation after every step, (b) enqueued back to back, (c) replayed
+    as one CUDA graph: the kernels are deterministic, so outputs, evicted
+    positions, cache rows, importances and memory must agree bitwise. A missed
+    ordering between the steps (the features on the second stream, the next
+    attention step's early loads after the eviction) would show here."""
+    B, L, steps, batch = 128, 1024, 12, 2
+    case = Case(W["c1"], cuda_device, L=L + steps, batch=batch, n_decode=1)
+    lay = case.layer()
+    cap = B + 1
+    st = lay.new_state(batch, L, B, cap, cuda_device)
+    d = {k: v[:, :L].contiguous() for k, v in case.in_dev.items()}
+    lay.score_and_evict(d["X"], d["Q"], d["K"], d["V"], st, B)
+    lay.update_memory(d["K"], d["V"], st, B, chunk=64)
+    on = lay.online_init(st, B, L)
+    lay.sync()
+    names = ("K_ret", "V_ret", "M", "bstab", "cache_len")
+    onames = ("khat_ret", "I_ret", "pos_ret", "next_pos", "evicted")
+    init = ({k: getattr(st, k).clone() for k in names}, {k: getattr(on, k).clone() for k in onames})
+
+    def restore():
+        for k in names:
+            getattr(st, k).copy_(init[0][k])
+        for k in onames:
+            getattr(on, k).copy_(init[1][k])
+        lay.invalidate_decode(batch)
+
+    toks = [tuple(case.in_dev[k][:, L + i].contiguous() for k in ("X", "Q", "K", "V"))
+            for i in range(steps)]
+    outs = [torch.empty_like(toks[0][1]) for _ in range(steps)]
+    evs = [torch.empty_like(on.evicted) for _ in range(steps)]
+
+    def run(sync):
+        for i, (x, q, kn, vn) in enumerate(toks):
+            lay.decode_online(x, q, kn, vn, st, on, B, out=outs[i])
+            evs[i].copy_(on.evicted)
+            if sync:
+                lay.sync()
+
+    def snapshot():
+        torch.cuda.synchronize()
+        return ([o.clone() for o in outs], [e.clone() for e in evs],
+                {k: getattr(st, k).clone() for k in names},
+                {k: getattr(on, k).clone() for k in onames})
+
+    restore(); run(True); ref = snapshot()
+    restore(); run(False); lay.sync(); b2b = snapshot()
+    s = torch.cuda.Stream(cuda_device)
+    restore(); torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for i, (x, q, kn, vn) in enumerate(toks):
+                lay.decode_online(x, q, kn, vn, st, on, B, out=outs[i], stream=s)
+                evs[i].copy_(on.evicted)
+    torch.cuda.synchronize()
+    restore(); torch.cuda.synchronize()
+    g.replay(); torch.cuda.synchronize(); lay.sync()
+    gr = snapshot()
+    for what, got in (("back to back", b2b), ("graph", gr)):
+        for i in range(steps):
+            assert torch.equal(got[0][i], ref[0][i]), "%s: output of step %d" % (what, i)
+            assert torch.equal(got[1][i], ref[1][i]), "%s: eviction of step %d" % (what, i)
+        for k in names:
+            assert torch.equal(got[2][k], ref[2][k]), "%s: %s" % (what, k)
+        for k in onames:
+            assert torch.equal(got[3][k], ref[3][k]), "%s: %s" % (what, k)
+    del g
+    lay.close()
