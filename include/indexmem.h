@@ -390,11 +390,12 @@ imem_status imem_prefill_evict_chunk(imem_ctx* ctx, int batch, int L, int B, int
  *      by, so that K_ret/V_ret/khat_ret/I_ret/pos_ret[:, :B + 1] are the
  *      B + 1 candidates of the step; cache_len returns to B; next_pos
  *      advances.
- * Streams: step 2's indexer query and key need neither the cache nor the
- * memory, so they are computed on a second stream owned by the context
+ * Streams: step 2 and the choice of step 3 need neither the cache rows nor
+ * the memory, so they are computed on a second stream owned by the context
  * (created by imem_online_init or the first step, which therefore belong
  * before any stream capture; no device memory),
- * forked from `stream` and joined back into it by events before step 3;
+ * forked from `stream` and joined back into it by events before the memory
+ * update of step 3;
  * under stream capture this becomes two parallel branches of the graph.
  * Ordering: step 4 clears the workspace's decode tag of the sequence (slot e
  * and the memory changed after the attention step), so the next decode step

@@ -35,6 +35,8 @@ Workspace workspace_layout(const Ctx& c, int batch, int L) {
   off = align_up(off + (size_t)batch * c.cfg.n_q_heads * c.cfg.idx_dim * sizeof(float), 256);
   w.on_kpart_off = off;
   off = align_up(off + (size_t)batch * c.cfg.idx_dim * sizeof(float), 256);
+  w.on_choice_off = off;
+  off = align_up(off + (size_t)batch * sizeof(OnlineChoice), 256);
   w.dec_part_off = off;                       // (unused: decode merges in shared memory)
   // memory partials: one d x (d+1) sum [S | s] per run of evicted tokens
   const size_t runs = memory_runs_bound((int)units, L, c.num_sms);
@@ -629,11 +631,15 @@ imem_status imem_decode_online(imem_ctx* h, int batch, int B, const void* x_new,
   char* wsb = (char*)workspace;
   float* qpart = (float*)(wsb + ws.on_qpart_off);
   float* kpart = (float*)(wsb + ws.on_kpart_off);
-  // the new token's indexer features need neither the cache nor the memory:
+  void* choice = wsb + ws.on_choice_off;
+  // the new token's indexer features and the importance update with the
+  // choice of the token to evict need neither the cache rows nor the memory:
   // they run on the context's second stream beside the attention step
   IMEM_CHECK(cuda_status(cudaEventRecord(c.ev_fork, st)));
   IMEM_CHECK(cuda_status(cudaStreamWaitEvent(c.side, c.ev_fork, 0)));
   IMEM_CHECK(cuda_status(imem::launch_online_features(c, batch, x_new, q, qpart, kpart, c.side)));
+  IMEM_CHECK(cuda_status(imem::launch_online_score(c, batch, B, cap, qpart, kpart, khat_ret, I_ret,
+                                                   pos_ret, next_pos, choice, c.side)));
   IMEM_CHECK(cuda_status(cudaEventRecord(c.ev_join, c.side)));
   // the attention step with the memory before this step's eviction (it
   // validates the remaining arguments and appends the new token at slot B)
@@ -642,10 +648,9 @@ imem_status imem_decode_online(imem_ctx* h, int batch, int B, const void* x_new,
   // join first, so that the second stream's work is always waited for
   IMEM_CHECK(cuda_status(cudaStreamWaitEvent(st, c.ev_join, 0)));
   IMEM_CHECK(ds);
-  return cuda_status(imem::launch_online_score_evict(c, batch, B, cap, qpart, kpart, khat_ret,
-                                                     I_ret, pos_ret, next_pos, K_ret, V_ret,
-                                                     cache_len, M, bstab, evicted,
-                                                     (int*)(wsb + ws.dec_tag_off), st));
+  return cuda_status(imem::launch_online_evict(c, batch, B, cap, choice, khat_ret, I_ret, pos_ret,
+                                               next_pos, K_ret, V_ret, cache_len, M, bstab,
+                                               evicted, (int*)(wsb + ws.dec_tag_off), st));
 }
 
 imem_status imem_selftest_wait(imem_ctx* h, long long limit_cycles, void* stream) {

@@ -228,7 +228,7 @@ __device__ void attend_bf16(Ring& rg, const CUtensorMap* tmK, const CUtensorMap*
                             const __nv_bfloat16* __restrict__ Vb, size_t row_stride, int hi,
                             const __nv_bfloat16* kn, const __nv_bfloat16* vn, int len,
                             int r0, int r1, int g0, int n_pre, const float (*s_q)[D],
-                            Partial<D> (*s_part)[G], int* err) {
+                            Partial<D> (*s_part)[G], int* err, const uint4* s_new) {
   constexpr int CH = D / 8;                 // 16-byte chunks per row
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
@@ -265,6 +265,104 @@ __device__ void attend_bf16(Ring& rg, const CUtensorMap* tmK, const CUtensorMap*
     for (int st = n_pre; st < n_stages && st < nst; ++st)
       ring_issue_lsu<D>(rg, Kb, Vb, row_stride, g0 + st, r0 + st * kStageRows, hi);
   }
+  if (!kTma && n_stages <= nst) {
+    // Every stage of this block is in the ring at once (one-wave grids): the
+    // scores of all of a warp's row tiles first (independent MMA chains,
+    // interleaved), one softmax over them, then all the P V products; the
+    // stage-by-stage loop below would chain the tiles one after another.
+    cp_async_wait<0>();
+    __syncthreads();
+#pragma unroll
+    for (int st = 0; st < kDecodeMaxStages; ++st) {
+      const int kb = r0 + st * kStageRows + warp * 16;
+      if (st < n_stages && kb < r1 && (kb + 16 > r1 || (len >= kb && len < kb + 16))) {
+        const uint32_t kt = rg.buf0 + (uint32_t)((g0 + st) % nst) * 2u * kTileBytes<D>;
+        const uint32_t vt = kt + kTileBytes<D>;
+        for (int i = lane; i < 16 * CH; i += 32) {
+          const int rr = warp * 16 + i / CH, c = i % CH, row = kb + i / CH;
+          if (row >= r1) {
+            asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};\n" ::"r"(vt + tile_off<D>(rr, c)),
+                         "r"(0u));
+          } else if (row == len) {
+            const uint4 kv = s_new[c];
+            const uint4 vv = s_new[CH + c];
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(kt + tile_off<D>(rr, c)),
+                         "r"(kv.x), "r"(kv.y), "r"(kv.z), "r"(kv.w));
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(vt + tile_off<D>(rr, c)),
+                         "r"(vv.x), "r"(vv.y), "r"(vv.z), "r"(vv.w));
+          }
+        }
+      }
+    }
+    __syncwarp();
+    // scores: tiles past the block compute on whatever the buffer holds and
+    // are masked by selection (never by arithmetic, so nothing there leaks)
+    float sa[kDecodeMaxStages][4], sb[kDecodeMaxStages][4];
+    uint32_t kts[kDecodeMaxStages];
+#pragma unroll
+    for (int st = 0; st < kDecodeMaxStages; ++st) {
+      kts[st] = rg.buf0 + (uint32_t)((g0 + st) % nst) * 2u * kTileBytes<D>;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sa[st][e] = sb[st][e] = 0.f;
+    }
+    {
+      const int rr = warp * 16 + (lane & 15);
+#pragma unroll
+      for (int s2 = 0; s2 < D / 16; ++s2) {
+#pragma unroll
+        for (int st = 0; st < kDecodeMaxStages; ++st) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(kts[st] + tile_off<D>(rr, 2 * s2 + (lane >> 4)), a0, a1, a2, a3);
+          if (s2 & 1) mma_bf16_a4(sb[st], a0, a1, a2, a3, qb0[s2], qb1[s2]);
+          else mma_bf16_a4(sa[st], a0, a1, a2, a3, qb0[s2], qb1[s2]);
+        }
+      }
+    }
+    float sc[kDecodeMaxStages][4];
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int st = 0; st < kDecodeMaxStages; ++st) {
+      const int kb = r0 + st * kStageRows + warp * 16;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int row = kb + g + ((e >> 1) << 3);
+        sc[st][e] = (st < n_stages && row < r1) ? (sa[st][e] + sb[st][e]) * sscale : -INFINITY;
+      }
+      mx[0] = fmaxf(mx[0], fmaxf(sc[st][0], sc[st][2]));
+      mx[1] = fmaxf(mx[1], fmaxf(sc[st][1], sc[st][3]));
+    }
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], off));
+      mx[1] = fmaxf(mx[1], __shfl_xor_sync(0xffffffffu, mx[1], off));
+    }
+    m_run[0] = mx[0];
+    m_run[1] = mx[1];
+#pragma unroll
+    for (int st = 0; st < kDecodeMaxStages; ++st) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        sc[st][e] = (sc[st][e] == -INFINITY) ? 0.f : exp2f(sc[st][e] - m_run[e & 1]);
+      l_run[0] += sc[st][0] + sc[st][2];
+      l_run[1] += sc[st][1] + sc[st][3];
+    }
+    const int rv = warp * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+#pragma unroll
+    for (int st = 0; st < kDecodeMaxStages; ++st) {
+      const int kb = r0 + st * kStageRows + warp * 16;
+      if (st < n_stages && kb < r1) {   // warp-uniform
+        const uint32_t pb0 = movm_trans(pack_bf16(sc[st][0], sc[st][1]));
+        const uint32_t pb1 = movm_trans(pack_bf16(sc[st][2], sc[st][3]));
+        const uint32_t vt = kts[st] + kTileBytes<D>;
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(vt + tile_off<D>(rv, 2 * mt + ((lane >> 3) & 1)), a0, a1, a2, a3);
+          mma_bf16_a4(o[mt], a0, a1, a2, a3, pb0, pb1);
+        }
+      }
+    }
+  } else
   for (int st = 0; st < n_stages; ++st) {
     const int gi = g0 + st, b = gi % nst;
     if constexpr (kTma) {
@@ -287,8 +385,8 @@ __device__ void attend_bf16(Ring& rg, const CUtensorMap* tmK, const CUtensorMap*
             asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};\n" ::"r"(vt + tile_off<D>(rr, c)),
                          "r"(0u));
           } else if (row == len) {
-            const uint4 kv = __ldcg(reinterpret_cast<const uint4*>(kn) + c);
-            const uint4 vv = __ldcg(reinterpret_cast<const uint4*>(vn) + c);
+            const uint4 kv = s_new[c];
+            const uint4 vv = s_new[CH + c];
             asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(kt + tile_off<D>(rr, c)),
                          "r"(kv.x), "r"(kv.y), "r"(kv.z), "r"(kv.w));
             asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(vt + tile_off<D>(rr, c)),
@@ -608,6 +706,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   int* __restrict__ dec_tag = seq_counters + gridDim.z;
 
   __shared__ __align__(16) float s_q[G][D];
+  __shared__ __align__(16) uint4 s_newrow[2 * D / 8];   // the new row: k_new | v_new (bf16)
   __shared__ float s_w[kDecodeMaxSplits][G];
   __shared__ float s_l[G];
   __shared__ int s_len_hint;
@@ -711,6 +810,12 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
 #pragma unroll
     for (int e = 0; e < (int)(sizeof(T) / 2); ++e) qraw[e] = __ldcg(qs + e);
   }
+  if (kBf16 && rank < S && tid < 2 * D / 8) {
+    // the new row, read with q: the attention loop then patches it in from
+    // shared memory instead of a round trip to L2 inside the loop
+    const T* src = (tid < D / 8 ? k_new : v_new) + ((size_t)bi * Hkv + kh) * D;
+    s_newrow[tid] = __ldcg(reinterpret_cast<const uint4*>(src) + (tid % (D / 8)));
+  }
   const int len = __ldcg(cache_len + bi);
   const int tag = __ldcg(dec_tag + bi);
   if constexpr (kBf16 && kTma) {
@@ -784,7 +889,8 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     if constexpr (kBf16) {
       // a miss leaves TMA stages 0..n_spec-1 spent: the block starts after them
       attend_bf16<D, G, kTma>(ring, &tmK, &tmV, kh * D, bi * cap, Kb, Vb, row_stride, r1, kn, vn,
-                              len, r0, r1, hit ? 0 : n_spec, hit ? n_spec : 0, s_q, w_part, err);
+                              len, r0, r1, hit ? 0 : n_spec, hit ? n_spec : 0, s_q, w_part, err,
+                              s_newrow);
     }
     else
       attend_f32<D, G>(Kb, Vb, row_stride, kn, vn, len, r0, r1, s_q, w_part);

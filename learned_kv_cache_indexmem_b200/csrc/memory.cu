@@ -131,8 +131,10 @@ memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t
   __shared__ int s_abort;
   __shared__ float s_sv[8][16][8];   // per loader warp, per 16-byte column chunk: value sums
 
-  const int g = blockIdx.x, kh = blockIdx.y, bi = blockIdx.z;
-  const int G = gridDim.x;
+  // head-major grid: the KV heads of one run are neighbours in launch order, so
+  // they stream through the same token rows at about the same time
+  const int kh = blockIdx.x, g = blockIdx.y, bi = blockIdx.z;
+  const int G = gridDim.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int j0 = g * tokens_per_group;
   const int j1 = min(n_e, j0 + tokens_per_group);
@@ -370,16 +372,35 @@ memory_finalize_kernel(const float* __restrict__ partials, int G, int tpg, int n
     if (threadIdx.x == 0 && unit % Hkv == 0) n_e[unit / Hkv] += n_add;
     return;
   }
-  float* sW = fsm;                 // [r][D]
-  float* sS = sW + r * D;          // [D][16]
+  float* sW = fsm;                 // [r][D + 1] (padded rows: conflict-free column reads)
+  float* sS = sW + r * (D + 1);    // [D][16]
   const int unit = blockIdx.y, sl = blockIdx.x;
   const int tid = threadIdx.x;
   const bool bcol = (sl == D / 16);
   const int ncols = bcol ? 1 : 16;
   const int col0 = bcol ? D : sl * 16;
-  if (W_phi)   // null: the identity map (r == D)
-    for (int i = tid; i < r * D / 4; i += 256)
-      reinterpret_cast<float4*>(sW)[i] = __ldg(reinterpret_cast<const float4*>(W_phi) + i);
+  if (W_phi) {   // null: the identity map (r == D)
+    // a batch of 8 float4 loads per thread is issued before any of its
+    // stores (one round trip per batch; r * D / 4 <= 2048 needs one batch)
+    constexpr int WQ = 8;
+    for (int base = 0; base < r * D / 4; base += WQ * 256) {
+      float4 wv[WQ];
+#pragma unroll
+      for (int k = 0; k < WQ; ++k) {
+        const int i = base + tid + k * 256;
+        wv[k] = i < r * D / 4 ? __ldg(reinterpret_cast<const float4*>(W_phi) + i)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int k = 0; k < WQ; ++k) {
+        const int i = base + tid + k * 256;
+        if (i < r * D / 4) {
+          float* dst = sW + ((4 * i) / D) * (D + 1) + (4 * i) % D;
+          dst[0] = wv[k].x; dst[1] = wv[k].y; dst[2] = wv[k].z; dst[3] = wv[k].w;
+        }
+      }
+    }
+  }
   // sum of the runs: every thread owns IPT (row, column) items and loads all
   // of them for one run before the next run, so that its loads are
   // independent (a loop over the runs per item would chain G round trips
@@ -390,18 +411,24 @@ memory_finalize_kernel(const float* __restrict__ partials, int G, int tpg, int n
   float acc[IPT];
 #pragma unroll
   for (int k = 0; k < IPT; ++k) acc[k] = 0.f;
-#pragma unroll 2
-  for (int gg = 0; gg < G; ++gg) {
-    const float f = s_fac[gg];
-    const float* pg = p + (size_t)gg * D * (D + 1) + col0;
-    float v[IPT];
+  // four runs' loads in flight together, then their sums
+  for (int g0 = 0; g0 < G; g0 += 4) {
+    float v[4][IPT];
 #pragma unroll
-    for (int k = 0; k < IPT; ++k) {
-      const int i = tid + k * 256;
-      v[k] = i < D * ncols ? __ldcg(&pg[(i / ncols) * (D + 1) + i % ncols]) : 0.f;
+    for (int u = 0; u < 4; ++u) {
+      const float* pg = p + (size_t)(g0 + u) * D * (D + 1) + col0;
+#pragma unroll
+      for (int k = 0; k < IPT; ++k) {
+        const int i = tid + k * 256;
+        v[u][k] = (g0 + u < G && i < D * ncols) ? __ldcg(&pg[(i / ncols) * (D + 1) + i % ncols]) : 0.f;
+      }
     }
 #pragma unroll
-    for (int k = 0; k < IPT; ++k) acc[k] = fmaf(f, v[k], acc[k]);
+    for (int u = 0; u < 4; ++u) {
+      const float f = g0 + u < G ? s_fac[g0 + u] : 0.f;
+#pragma unroll
+      for (int k = 0; k < IPT; ++k) acc[k] = fmaf(f, v[u][k], acc[k]);
+    }
   }
 #pragma unroll
   for (int k = 0; k < IPT; ++k) {
@@ -409,21 +436,46 @@ memory_finalize_kernel(const float* __restrict__ partials, int G, int tpg, int n
     if (i < D * ncols) sS[(i / ncols) * 16 + i % ncols] = acc[k];
   }
   __syncthreads();
-  for (int i = tid; i < r * ncols; i += 256) {
-    const int ri = i / ncols, cc = i % ncols;
-    float a = 0.f;
+  // out[ri][c] = sum_dk W_phi[ri][dk] S[dk][c]: a thread takes two rows
+  // (ri, ri + r/2) and four columns, so that each loaded S quad serves two
+  // rows and each W_phi value four columns
+  const int nq = ncols == 16 ? 4 : 1;                 // column quads
+  for (int o = tid; o < (r / 2) * nq; o += 256) {
+    const int ri = o / nq, q = o % nq;
+    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
     if (W_phi) {
+      const float* w0 = sW + (size_t)ri * (D + 1);
+      const float* w1 = sW + (size_t)(ri + r / 2) * (D + 1);
 #pragma unroll 8
-      for (int dk = 0; dk < D; ++dk) a = fmaf(sW[ri * D + dk], sS[dk * 16 + cc], a);
+      for (int dk = 0; dk < D; ++dk) {
+        const float4 sv = *reinterpret_cast<const float4*>(sS + dk * 16 + 4 * q);
+        const float x0 = w0[dk], x1 = w1[dk];
+        a0[0] = fmaf(x0, sv.x, a0[0]); a0[1] = fmaf(x0, sv.y, a0[1]);
+        a0[2] = fmaf(x0, sv.z, a0[2]); a0[3] = fmaf(x0, sv.w, a0[3]);
+        a1[0] = fmaf(x1, sv.x, a1[0]); a1[1] = fmaf(x1, sv.y, a1[1]);
+        a1[2] = fmaf(x1, sv.z, a1[2]); a1[3] = fmaf(x1, sv.w, a1[3]);
+      }
     } else {
-      a = sS[ri * 16 + cc];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        a0[e] = sS[ri * 16 + 4 * q + e];
+        a1[e] = sS[(ri + r / 2) * 16 + 4 * q + e];
+      }
     }
-    if (bcol) {
-      float* bp = bstab + (size_t)unit * r + ri;
-      *bp = fmaf(*bp, decay_n, a);
+    if (bcol) {   // one column: b
+      float* bp = bstab + (size_t)unit * r;
+      bp[ri] = fmaf(bp[ri], decay_n, a0[0]);
+      bp[ri + r / 2] = fmaf(bp[ri + r / 2], decay_n, a1[0]);
     } else {
-      float* mp = M + ((size_t)unit * r + ri) * D + col0 + cc;
-      *mp = fmaf(*mp, decay_n, a);
+      float* m0 = M + ((size_t)unit * r + ri) * D + col0 + 4 * q;
+      float* m1 = M + ((size_t)unit * r + ri + r / 2) * D + col0 + 4 * q;
+      float4 v0 = *reinterpret_cast<float4*>(m0), v1 = *reinterpret_cast<float4*>(m1);
+      v0.x = fmaf(v0.x, decay_n, a0[0]); v0.y = fmaf(v0.y, decay_n, a0[1]);
+      v0.z = fmaf(v0.z, decay_n, a0[2]); v0.w = fmaf(v0.w, decay_n, a0[3]);
+      v1.x = fmaf(v1.x, decay_n, a1[0]); v1.y = fmaf(v1.y, decay_n, a1[1]);
+      v1.z = fmaf(v1.z, decay_n, a1[2]); v1.w = fmaf(v1.w, decay_n, a1[3]);
+      *reinterpret_cast<float4*>(m0) = v0;
+      *reinterpret_cast<float4*>(m1) = v1;
     }
   }
 }
@@ -491,8 +543,10 @@ memory_bf16_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __r
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
-  const int g = blockIdx.x, kh = blockIdx.y, bi = blockIdx.z;
-  const int G = gridDim.x;
+  // head-major grid: the KV heads of one run are neighbours in launch order, so
+  // they stream through the same token rows at about the same time
+  const int kh = blockIdx.x, g = blockIdx.y, bi = blockIdx.z;
+  const int G = gridDim.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int j0 = g * tokens_per_run;
   const int j1 = min(n_e, j0 + tokens_per_run);
@@ -513,16 +567,27 @@ memory_bf16_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __r
                                       bf_off(jj, (D / 64) * 8, TL::ATOM_COL)) =
         __float2bfloat16_rn(1.f);
   }
-  // the run's evicted positions (-1: no row: past the run, or out of range)
+  // the run's evicted positions (-1: no row: past the run, or out of range),
+  // all of a thread's loads issued before its stores (one round trip)
   uint32_t bad = 0;
   const int32_t* E = idx_e + (size_t)bi * n_e + j0;
-  for (int i = tid; i < nchunks * kBfChunk; i += kMemThreads) {
-    int p = -1;
-    if (i < ntok) {
-      p = __ldg(E + i);
-      if ((unsigned)p >= (unsigned)L) { bad = 1u; p = -1; }
+  {
+    constexpr int PP = (kRunMax + kMemThreads - 1) / kMemThreads;
+    int pv[PP];
+#pragma unroll
+    for (int k = 0; k < PP; ++k) {
+      const int i = tid + k * kMemThreads;
+      pv[k] = i < ntok ? __ldg(E + i) : -1;
     }
-    s_pos[i] = p;
+#pragma unroll
+    for (int k = 0; k < PP; ++k) {
+      const int i = tid + k * kMemThreads;
+      if (i < nchunks * kBfChunk) {
+        int p = pv[k];
+        if (i < ntok && (unsigned)p >= (unsigned)L) { bad = 1u; p = -1; }
+        s_pos[i] = p;
+      }
+    }
   }
   if (tid == 0) {
     for (int st = 0; st < kBfStages; ++st) {
@@ -764,7 +829,7 @@ cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, 
                                                (size_t)batch * Hkv + 2 * 148);
   const int tokens_per_group = sp.tokens_per_run;
   const int Gused = sp.runs;
-  dim3 grid(Gused, Hkv, batch);
+  dim3 grid(Hkv, Gused, batch);
   const float log2lam = (float)log2((double)c.cfg.lambda);
   cudaError_t e = cudaSuccess;
 #define IMEM_MEMBF(DD)                                                                        \
@@ -803,7 +868,7 @@ cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, 
   dim3 fgrid(D / 16 + 1 + (sv_partials ? 1 : 0), batch * Hkv);
   // moment statistics use the identity map: the finalize skips the product
   const float* phi = c.cfg.readout == IMEM_READOUT_MOMENT ? nullptr : c.W_phi;
-  const size_t fsmem = ((size_t)r * D + (size_t)D * 16) * sizeof(float);
+  const size_t fsmem = ((size_t)r * (D + 1) + (size_t)D * 16) * sizeof(float);
   if (D == 128)
     e = launch_finalize<128>(fgrid, fsmem, st, partials, Gused, tokens_per_group, n_e, log2lam,
                              phi, r, decay_n, M, bstab, sv_partials, s_v, n_count, (float)n_e, Hkv);
@@ -873,13 +938,13 @@ cudaError_t launch_memory_static(int batch, int L, int Hkv, int r, float lambda,
   cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        MemTile<D>::SMEM);
   if (e != cudaSuccess) return e;
-  kfn<<<dim3(Gused, Hkv, batch), kMemThreads, MemTile<D>::SMEM, st>>>(
+  kfn<<<dim3(Hkv, Gused, batch), kMemThreads, MemTile<D>::SMEM, st>>>(
       (const T*)K, (const T*)V, idx_e, n_e, L, Hkv, log2lam, tokens_per_group, scratch, nullptr,
       err);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const float decay_n = (float)pow((double)lambda, (double)n_e);
-  const size_t fsmem = ((size_t)r * D + (size_t)D * 16) * sizeof(float);
+  const size_t fsmem = ((size_t)r * (D + 1) + (size_t)D * 16) * sizeof(float);
   e = launch_finalize<D>(dim3(D / 16 + 1, units), fsmem, st, scratch, Gused, tokens_per_group, n_e,
                          log2lam, W_phi, r, decay_n, M, bstab, nullptr, nullptr, nullptr, 0.f, Hkv);
   if (e != cudaSuccess) return e;

@@ -15,12 +15,15 @@
 //             needs neither the cache nor the memory, so the C ABI runs it
 //             on a second stream next to the attention step (which appends
 //             the new token at slot B);
-//   score + evict  (after both) one thread-block cluster per sequence:
-//             I_t <- max(I_t, q~ . k^_t) for the cached tokens, the new
-//             token's I = q~ . k^_new; the least important of the B + 1
-//             (ties: the higher position) by per-CTA minima of a packed
+//   score     (second stream, after the features) one thread-block cluster
+//             per sequence: I_t <- max(I_t, q~ . k^_t) for the cached tokens,
+//             the new token's I = q~ . k^_new; the least important of the
+//             B + 1 (ties: the higher position) by per-CTA minima of a packed
 //             (ordered importance, inverted position) key exchanged over
-//             distributed shared memory; per KV head phi = W_phi k_e,
+//             distributed shared memory; the choice to the workspace. It
+//             touches neither the rows, the memory nor slot B, so it runs
+//             beside the attention step as well;
+//   evict     (after both branches) per KV head phi = W_phi k_e,
 //             M <- lambda M + phi v_e^T, b <- lambda b + phi; the new token
 //             and the evicted one swap slots (row, indexer key, importance,
 //             position), so slot B keeps the token that left with the
@@ -184,40 +187,29 @@ online_features_kernel(const T* __restrict__ x, const T* __restrict__ q, const T
   }
 }
 
-// ---- importances, the token to evict and the memory update -----------------
+// ---- importances and the token to evict (second stream) ----------------------
 // One thread-block cluster of nct CTAs per sequence. Each CTA takes a
 // contiguous block of the B + 1 candidate rows (slot B: the new token):
 // I_t <- max(I_t, q~ . k^_t) for the cached tokens, the new token's I =
 // q~ . k^_new, and its block's least important candidate as a packed key
 // (ordered importance << 32 | ~position: the minimum is the least important,
 // ties to the higher position). The CTAs exchange their keys through
-// distributed shared memory and, after one cluster barrier, all know the
-// token e to evict. Then CTA r updates the memory of the KV heads h = r,
-// r + nct, ...: M <- lambda M + phi(k_e) v_e^T, b <- lambda b + phi(k_e),
-// and swaps the rows of e and B of those heads (the new token takes slot e,
-// the evicted token slot B); the CTA owning row e swaps the indexer keys,
-// importances and positions of the two slots.
+// distributed shared memory; after one cluster barrier CTA 0 writes the
+// choice (slot, position, importance) and the new token's importance and
+// indexer key to the workspace. Nothing here reads or writes the cache rows,
+// the memory or slot B, so it runs beside the attention step.
 __device__ __forceinline__ float order_key_inv(uint32_t o) {
   return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
 }
 
-template <typename T>
 __global__ void __launch_bounds__(kOnThreads)
-online_score_evict_kernel(int B, int cap, int Hq, int Hkv, int D, int dI, int r, float lambda,
-                          int rows_per_cta, const float* __restrict__ qpart,
-                          const float* __restrict__ kpart, const float* __restrict__ W_phi,
-                          T* __restrict__ K_ret, T* __restrict__ V_ret,
-                          __nv_bfloat16* __restrict__ khat_ret, float* __restrict__ I_ret,
-                          int32_t* __restrict__ pos_ret, int32_t* __restrict__ next_pos,
-                          int32_t* __restrict__ cache_len, float* __restrict__ M,
-                          float* __restrict__ bstab, int32_t* __restrict__ evicted,
-                          int* __restrict__ dec_tag) {
+online_score_kernel(int B, int cap, int Hq, int dI, int rows_per_cta,
+                    const float* __restrict__ qpart, const float* __restrict__ kpart,
+                    const __nv_bfloat16* __restrict__ khat_ret, float* __restrict__ I_ret,
+                    const int32_t* __restrict__ pos_ret, const int32_t* __restrict__ next_pos,
+                    OnlineChoice* __restrict__ choice) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
-  extern __shared__ float osm[];
-  float* sk = osm;          // [D]
-  float* sv = sk + D;       // [D]
-  float* sphi = sv + D;     // [r]
   __shared__ float s_qt[64], s_kn[64];
   __shared__ float red[kOnThreads / 32];
   __shared__ unsigned long long s_key[kOnThreads / 32];
@@ -296,105 +288,131 @@ online_score_evict_kernel(int B, int cap, int Hq, int Hkv, int D, int dI, int r,
   if (lane == 0) { s_key[warp] = best; s_slot[warp] = best_slot; }
   __syncthreads();
   asm volatile("barrier.cluster.wait.aligned;\n" ::: "memory");   // phase 0: all running
-  if (tid < nct) {
-    // this CTA's candidate into slot `rank` of CTA tid's exchange arrays
+  if (tid == 0) {   // this CTA's candidate into slot `rank` of CTA 0
     unsigned long long k = s_key[0];
     int sl = s_slot[0];
     for (int w = 1; w < kOnThreads / 32; ++w)
       if (s_key[w] < k) { k = s_key[w]; sl = s_slot[w]; }
-    cluster.map_shared_rank(s_ckey, tid)[rank] = k;
-    cluster.map_shared_rank(s_cslot, tid)[rank] = sl;
+    cluster.map_shared_rank(s_ckey, 0)[rank] = k;
+    cluster.map_shared_rank(s_cslot, 0)[rank] = sl;
   }
-  cluster.sync();   // every CTA has written its candidate into every CTA
-  unsigned long long k = ~0ull;
-  int e = -1;
-  for (int i = 0; i < nct; ++i)
-    if (s_ckey[i] < k) { k = s_ckey[i]; e = s_cslot[i]; }
-  int pos_e = (int32_t)(~(uint32_t)(k & 0xffffffffull));
-  float I_e = order_key_inv((uint32_t)(k >> 32));
-  if (e < 0) {   // no ordered candidate (NaN importances): the new token leaves
-    e = B; pos_e = npos; I_e = s_Inew;
+  cluster.sync();   // every CTA has written its candidate into CTA 0
+  if (rank == 0 && tid == 0) {
+    unsigned long long k = ~0ull;
+    int e = -1;
+    for (int i = 0; i < nct; ++i)
+      if (s_ckey[i] < k) { k = s_ckey[i]; e = s_cslot[i]; }
+    OnlineChoice ch;
+    ch.slot = e;
+    ch.pos = (int32_t)(~(uint32_t)(k & 0xffffffffull));
+    ch.I_e = order_key_inv((uint32_t)(k >> 32));
+    if (e < 0) {   // no ordered candidate (NaN importances): the new token leaves
+      ch.slot = B; ch.pos = npos; ch.I_e = s_Inew;
+    }
+    ch.I_new = s_Inew;
+    ch.pos_new = npos;
+    choice[bi] = ch;
   }
+  if (rank == 0 && tid < kIdxPad / 8) {   // the new token's indexer key (bf16)
+    float f[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) f[c] = s_kn[8 * tid + c];
+    store8<__nv_bfloat16>(choice[bi].khat_new + 8 * tid, f);
+  }
+}
 
-  // memory update and row swap for this CTA's KV heads
+// ---- memory update with the evicted token, slot swap (after the attention) ---
+// CTA (KV head kh, sequence bi): phi = W_phi k_e, M <- lambda M + phi v_e^T,
+// b <- lambda b + phi; the rows of slot e and slot B (the new token, appended
+// by the attention step) swap for this head. CTA kh = 0 also swaps the indexer
+// keys, importances and positions (slot e takes the new token, slot B keeps
+// the evicted one with the importance it was chosen by), writes the evicted
+// position, returns cache_len to B, advances next_pos and clears the decode
+// tag (slot e and the memory changed after the attention step).
+template <typename T>
+__global__ void __launch_bounds__(kOnThreads)
+online_evict_kernel(int B, int cap, int Hkv, int D, int r, float lambda,
+                    const OnlineChoice* __restrict__ choice, const float* __restrict__ W_phi,
+                    T* __restrict__ K_ret, T* __restrict__ V_ret,
+                    __nv_bfloat16* __restrict__ khat_ret, float* __restrict__ I_ret,
+                    int32_t* __restrict__ pos_ret, int32_t* __restrict__ next_pos,
+                    int32_t* __restrict__ cache_len, float* __restrict__ M,
+                    float* __restrict__ bstab, int32_t* __restrict__ evicted,
+                    int* __restrict__ dec_tag) {
+  extern __shared__ float osm[];
+  float* sk = osm;          // [D]
+  float* sv = sk + D;       // [D]
+  float* sphi = sv + D;     // [r]
+  const int kh = blockIdx.x, bi = blockIdx.y, tid = threadIdx.x;
+  pdl_wait();
+  pdl_launch();
+  const OnlineChoice ch = choice[bi];
+  const int e = ch.slot;
   const size_t rs = (size_t)Hkv * D;
-  for (int kh = rank; kh < Hkv; kh += nct) {
-    T* ke = K_ret + ((size_t)bi * cap + e) * rs + (size_t)kh * D;
-    T* ve = V_ret + ((size_t)bi * cap + e) * rs + (size_t)kh * D;
-    for (int c = tid; c < D; c += kOnThreads) { sk[c] = ldf(ke + c); sv[c] = ldf(ve + c); }
-    __syncthreads();
-    // phi = W_phi k: 4 threads per row, float4 loads
-    for (int j0 = 0; j0 < r; j0 += kOnThreads / 4) {
-      const int j = j0 + tid / 4, part = tid & 3;
-      float a = 0.f;
-      if (j < r) {
-        const float4* wr = reinterpret_cast<const float4*>(W_phi + (size_t)j * D);
+  T* ke = K_ret + ((size_t)bi * cap + e) * rs + (size_t)kh * D;
+  T* ve = V_ret + ((size_t)bi * cap + e) * rs + (size_t)kh * D;
+  for (int c = tid; c < D; c += kOnThreads) { sk[c] = ldf(ke + c); sv[c] = ldf(ve + c); }
+  __syncthreads();
+  // phi = W_phi k: 4 threads per row, float4 loads
+  for (int j0 = 0; j0 < r; j0 += kOnThreads / 4) {
+    const int j = j0 + tid / 4, part = tid & 3;
+    float a = 0.f;
+    if (j < r) {
+      const float4* wr = reinterpret_cast<const float4*>(W_phi + (size_t)j * D);
 #pragma unroll 8
-        for (int c4 = part; c4 < D / 4; c4 += 4) {
-          const float4 w = __ldg(wr + c4);
-          a = fmaf(w.x, sk[4 * c4], fmaf(w.y, sk[4 * c4 + 1], fmaf(w.z, sk[4 * c4 + 2], fmaf(w.w, sk[4 * c4 + 3], a))));
-        }
-      }
-      a += __shfl_xor_sync(0xffffffffu, a, 1);
-      a += __shfl_xor_sync(0xffffffffu, a, 2);
-      if (j < r && part == 0) sphi[j] = a;
-    }
-    __syncthreads();
-    float4* Mu = reinterpret_cast<float4*>(M + ((size_t)bi * Hkv + kh) * r * D);
-#pragma unroll 4
-    for (int i = tid; i < r * D / 4; i += kOnThreads) {
-      const int j = (4 * i) / D, c = (4 * i) % D;
-      float4 m = Mu[i];
-      const float ph = sphi[j];
-      m.x = fmaf(lambda, m.x, ph * sv[c]);
-      m.y = fmaf(lambda, m.y, ph * sv[c + 1]);
-      m.z = fmaf(lambda, m.z, ph * sv[c + 2]);
-      m.w = fmaf(lambda, m.w, ph * sv[c + 3]);
-      Mu[i] = m;
-    }
-    for (int j = tid; j < r; j += kOnThreads) {
-      float* bp = bstab + ((size_t)bi * Hkv + kh) * r + j;
-      *bp = fmaf(lambda, *bp, sphi[j]);
-    }
-    if (e != B) {   // the new token (slot B) and the evicted one swap rows
-      T* kn = K_ret + ((size_t)bi * cap + B) * rs + (size_t)kh * D;
-      T* vn = V_ret + ((size_t)bi * cap + B) * rs + (size_t)kh * D;
-      for (int c = tid; c < D; c += kOnThreads) {
-        const T k0 = ke[c], v0 = ve[c];
-        ke[c] = kn[c]; ve[c] = vn[c];
-        kn[c] = k0; vn[c] = v0;
+      for (int c4 = part; c4 < D / 4; c4 += 4) {
+        const float4 w = __ldg(wr + c4);
+        a = fmaf(w.x, sk[4 * c4], fmaf(w.y, sk[4 * c4 + 1], fmaf(w.z, sk[4 * c4 + 2], fmaf(w.w, sk[4 * c4 + 3], a))));
       }
     }
-    __syncthreads();   // sk, sv, sphi reused by the next head
+    a += __shfl_xor_sync(0xffffffffu, a, 1);
+    a += __shfl_xor_sync(0xffffffffu, a, 2);
+    if (j < r && part == 0) sphi[j] = a;
   }
-  // indexer key, importance and position: slot e takes the new token, slot B
-  // keeps the evicted one (the CTA whose block holds row e)
-  if (e >= t0 && e < t1) {
+  __syncthreads();
+  float4* Mu = reinterpret_cast<float4*>(M + ((size_t)bi * Hkv + kh) * r * D);
+#pragma unroll 4
+  for (int i = tid; i < r * D / 4; i += kOnThreads) {
+    const int j = (4 * i) / D, c = (4 * i) % D;
+    float4 m = Mu[i];
+    const float ph = sphi[j];
+    m.x = fmaf(lambda, m.x, ph * sv[c]);
+    m.y = fmaf(lambda, m.y, ph * sv[c + 1]);
+    m.z = fmaf(lambda, m.z, ph * sv[c + 2]);
+    m.w = fmaf(lambda, m.w, ph * sv[c + 3]);
+    Mu[i] = m;
+  }
+  for (int j = tid; j < r; j += kOnThreads) {
+    float* bp = bstab + ((size_t)bi * Hkv + kh) * r + j;
+    *bp = fmaf(lambda, *bp, sphi[j]);
+  }
+  if (e != B) {   // the new token (slot B) and the evicted one swap rows
+    T* kn = K_ret + ((size_t)bi * cap + B) * rs + (size_t)kh * D;
+    T* vn = V_ret + ((size_t)bi * cap + B) * rs + (size_t)kh * D;
+    for (int c = tid; c < D; c += kOnThreads) {
+      const T k0 = ke[c], v0 = ve[c];
+      ke[c] = kn[c]; ve[c] = vn[c];
+      kn[c] = k0; vn[c] = v0;
+    }
+  }
+  if (kh == 0) {
     if (tid < kIdxPad / 8) {
       uint4* hb = reinterpret_cast<uint4*>(khat_ret + ((size_t)bi * cap + B) * kIdxPad) + tid;
       uint4* he = reinterpret_cast<uint4*>(khat_ret + ((size_t)bi * cap + e) * kIdxPad) + tid;
-      float f[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) f[c] = s_kn[8 * tid + c];
-      uint4 knew;
-      store8<__nv_bfloat16>(reinterpret_cast<__nv_bfloat16*>(&knew), f);
+      const uint4 knew = reinterpret_cast<const uint4*>(choice[bi].khat_new)[tid];
       if (e != B) *hb = *he;
       *he = knew;
     }
     if (tid == 0) {
-      I_ret[(size_t)bi * cap + e] = s_Inew;
-      pos_ret[(size_t)bi * cap + e] = npos;
-      I_ret[(size_t)bi * cap + B] = I_e;
-      pos_ret[(size_t)bi * cap + B] = pos_e;
+      I_ret[(size_t)bi * cap + e] = ch.I_new;
+      pos_ret[(size_t)bi * cap + e] = ch.pos_new;
+      I_ret[(size_t)bi * cap + B] = ch.I_e;
+      pos_ret[(size_t)bi * cap + B] = ch.pos;
+      evicted[bi] = ch.pos;
+      cache_len[bi] = B;
+      dec_tag[bi] = 0;
+      next_pos[bi] = ch.pos_new + 1;
     }
-  }
-  if (rank == 0 && tid == 0) {
-    evicted[bi] = pos_e;
-    cache_len[bi] = B;
-    // the rows of slot e and the memory changed after the decode step: the
-    // next decode step must not use rows or memory it loaded before its wait
-    dec_tag[bi] = 0;
-    next_pos[bi] = npos + 1;
   }
 }
 
@@ -447,19 +465,16 @@ cudaError_t launch_online_features(const Ctx& c, int batch, const void* x, const
                     qpart, kpart);
 }
 
-cudaError_t launch_online_score_evict(const Ctx& c, int batch, int B, int cap, const float* qpart,
-                                      const float* kpart, void* khat_ret, float* I_ret,
-                                      int32_t* pos_ret, int32_t* next_pos, void* K_ret,
-                                      void* V_ret, int32_t* cache_len, float* M, float* bstab,
-                                      int32_t* evicted, int* dec_tag, cudaStream_t st) {
+cudaError_t launch_online_score(const Ctx& c, int batch, int B, int cap, const float* qpart,
+                                const float* kpart, const void* khat_ret, float* I_ret,
+                                const int32_t* pos_ret, const int32_t* next_pos, void* choice,
+                                cudaStream_t st) {
   const int nct = online_cluster_ctas(B);
   const int rows_per_cta = (B + 1 + nct - 1) / nct;
-  const int Hkv = c.cfg.n_kv_heads, D = c.cfg.head_dim, r = c.cfg.mem_r;
-  const size_t sm = (size_t)(2 * D + r) * sizeof(float);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nct, batch, 1);
   cfg.blockDim = dim3(kOnThreads, 1, 1);
-  cfg.dynamicSmemBytes = sm;
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -470,18 +485,28 @@ cudaError_t launch_online_score_evict(const Ctx& c, int batch, int B, int cap, c
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, online_score_kernel, B, cap, c.cfg.n_q_heads, c.cfg.idx_dim,
+                            rows_per_cta, qpart, kpart, (const __nv_bfloat16*)khat_ret, I_ret,
+                            pos_ret, next_pos, (OnlineChoice*)choice);
+}
+
+cudaError_t launch_online_evict(const Ctx& c, int batch, int B, int cap, const void* choice,
+                                void* khat_ret, float* I_ret, int32_t* pos_ret, int32_t* next_pos,
+                                void* K_ret, void* V_ret, int32_t* cache_len, float* M,
+                                float* bstab, int32_t* evicted, int* dec_tag, cudaStream_t st) {
+  const int Hkv = c.cfg.n_kv_heads, D = c.cfg.head_dim, r = c.cfg.mem_r;
+  const size_t sm = (size_t)(2 * D + r) * sizeof(float);
+  const dim3 g(Hkv, batch);
+  const OnlineChoice* ch = (const OnlineChoice*)choice;
   if (c.cfg.dtype == IMEM_BF16)
-    return cudaLaunchKernelEx(&cfg, online_score_evict_kernel<__nv_bfloat16>, B, cap,
-                              c.cfg.n_q_heads, Hkv, D, c.cfg.idx_dim, r, c.cfg.lambda,
-                              rows_per_cta, qpart, kpart, (const float*)c.W_phi,
-                              (__nv_bfloat16*)K_ret, (__nv_bfloat16*)V_ret,
-                              (__nv_bfloat16*)khat_ret, I_ret, pos_ret, next_pos, cache_len, M,
-                              bstab, evicted, dec_tag);
-  return cudaLaunchKernelEx(&cfg, online_score_evict_kernel<float>, B, cap, c.cfg.n_q_heads, Hkv,
-                            D, c.cfg.idx_dim, r, c.cfg.lambda, rows_per_cta, qpart, kpart,
-                            (const float*)c.W_phi, (float*)K_ret, (float*)V_ret,
-                            (__nv_bfloat16*)khat_ret, I_ret, pos_ret, next_pos, cache_len, M,
-                            bstab, evicted, dec_tag);
+    return launch_pdl(online_evict_kernel<__nv_bfloat16>, g, sm, st, B, cap, Hkv, D, r,
+                      c.cfg.lambda, ch, (const float*)c.W_phi, (__nv_bfloat16*)K_ret,
+                      (__nv_bfloat16*)V_ret, (__nv_bfloat16*)khat_ret, I_ret, pos_ret, next_pos,
+                      cache_len, M, bstab, evicted, dec_tag);
+  return launch_pdl(online_evict_kernel<float>, g, sm, st, B, cap, Hkv, D, r, c.cfg.lambda, ch,
+                    (const float*)c.W_phi, (float*)K_ret, (float*)V_ret,
+                    (__nv_bfloat16*)khat_ret, I_ret, pos_ret, next_pos, cache_len, M, bstab,
+                    evicted, dec_tag);
 }
 
 }  // namespace imem
