@@ -682,7 +682,7 @@ struct DecSmem {
   }
 };
 
-template <typename T, int D, int G, bool kTma>
+template <typename T, int D, int G, bool kTma, int NRO>
 __global__ void __launch_bounds__(kThreads)
 decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __restrict__ v_new,
               T* __restrict__ K_ret, T* __restrict__ V_ret, int32_t* __restrict__ cache_len,
@@ -695,7 +695,14 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   namespace cg = cooperative_groups;
   extern __shared__ __align__(128) unsigned char dyn_smem[];
   cg::cluster_group cluster = cg::this_cluster();
-  const int S = gridDim.x - 1;              // attention CTAs; CTA S = readout and merge
+  // Readout CTAs per cluster (NRO): two, each for half of the query heads of
+  // the group, where the grid still fits one wave with the extra CTA (the
+  // readout's products on 128 threads are then the critical path); CTA S
+  // merges, CTA S + 1 pushes its readout to it.
+  static_assert(NRO == 1 || (NRO == 2 && !kTma && G >= 2), "two readout CTAs: one-wave grids, G >= 2");
+  constexpr int kNro = NRO;
+  constexpr int HG = G / kNro;              // query heads per readout CTA
+  const int S = gridDim.x - kNro;           // attention CTAs; CTA S = readout and merge
   const int rank = blockIdx.x;              // the cluster spans blockIdx.x
   const int kh = blockIdx.y, bi = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -728,7 +735,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   // [r][D] M of this unit: its own region in a one-wave grid (staged early,
   // latency), the W_phi region otherwise (staged after u, occupancy)
   float* sM = (moment || kTma) ? sW : sG + G * D;
-  if (rank == S && !moment) {
+  if (rank >= S && !moment) {
     // W_phi and w_gate belong to the context and are written only at
     // imem_init, so the readout CTA stages them before waiting for the
     // previous kernel (the moment readout uses neither: u = q, no gate)
@@ -744,7 +751,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   // early b (and s_v) and M, where M has a region of its own: kept if the
   // check after the wait finds that no other kernel can have changed them
   const bool ro_early = moment || !kTma;
-  if (rank == S && ro_early) stage_readout_state<D>(unit, r, bstab, s_v, M, moment, true, sb, ssv, sM);
+  if (rank >= S && ro_early) stage_readout_state<D>(unit, r, bstab, s_v, M, moment, true, sb, ssv, sM);
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   const size_t row_stride = (size_t)Hkv * D;
   const T* Kb = K_ret + (size_t)bi * cap * row_stride + (size_t)kh * D;
@@ -916,6 +923,8 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   }
 
   // ---- readout CTA: u = W_phi q, m = M^T u / (b.u + eps), g = sigmoid(w_gate . q)
+  // for the heads [hg0, hg0 + HG) of this readout CTA
+  const int hg0 = (rank - S) * HG;
   if (!ro_early || tag != len + 1) {
     // b (and s_v) and, where it has its own region, M: loaded now (the early
     // copies, if any, land first and are overwritten)
@@ -926,36 +935,38 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   cp_async_wait<0>();
   __syncthreads();
   // gate: z = w_gate[h] . q (none in moment mode)
-  for (int g = warp; g < G && !moment; g += kThreads / 32) {
+  for (int gg = warp; gg < HG && !moment; gg += kThreads / 32) {
+    const int g = hg0 + gg;
     float z = 0.f;
     for (int c = lane; c < D; c += 32) z = fmaf(sG[g * D + c], s_q[g][c], z);
     z = warp_sum(z);
     if (lane == 0) sgate[g] = use_override ? gate_override : sigmoidf_(z);
   }
   if (moment) {
-    for (int o = tid; o < G * r; o += kThreads) su[o] = s_q[o / r][o % r];   // u = q
+    for (int o = tid; o < HG * r; o += kThreads)   // u = q
+      su[(hg0 + o / r) * r + o % r] = s_q[hg0 + o / r][o % r];
   } else {
     // u = W_phi q: a pair of threads per row of W_phi (one half each), all G
     // heads at once, so that each row is read once (q is a broadcast read)
     for (int o = tid; o < 2 * r; o += kThreads) {
       const int j = o >> 1, half = o & 1;
       const float4* wr = reinterpret_cast<const float4*>(sW + (size_t)j * D);
-      float acc[G];
+      float acc[HG];
 #pragma unroll
-      for (int g = 0; g < G; ++g) acc[g] = 0.f;
+      for (int gg = 0; gg < HG; ++gg) acc[gg] = 0.f;
 #pragma unroll 4
       for (int cc = half * (D / 8); cc < (half + 1) * (D / 8); ++cc) {
         const float4 w = wr[cc ^ (j & 7)];
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float4 x = reinterpret_cast<const float4*>(&s_q[g][0])[cc];
-          acc[g] = fmaf(w.x, x.x, fmaf(w.y, x.y, fmaf(w.z, x.z, fmaf(w.w, x.w, acc[g]))));
+        for (int gg = 0; gg < HG; ++gg) {
+          const float4 x = reinterpret_cast<const float4*>(&s_q[hg0 + gg][0])[cc];
+          acc[gg] = fmaf(w.x, x.x, fmaf(w.y, x.y, fmaf(w.z, x.z, fmaf(w.w, x.w, acc[gg]))));
         }
       }
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 1);
-        if (half == 0) su[g * r + j] = acc[g];
+      for (int gg = 0; gg < HG; ++gg) {
+        acc[gg] += __shfl_xor_sync(0xffffffffu, acc[gg], 1);
+        if (half == 0) su[(hg0 + gg) * r + j] = acc[gg];
       }
     }
     if (kTma) {
@@ -969,7 +980,8 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     }
   }
   __syncthreads();
-  for (int g = warp; g < G; g += kThreads / 32) {
+  for (int gg = warp; gg < HG; gg += kThreads / 32) {
+    const int g = hg0 + gg;
     float a = 0.f;
     for (int j = lane; j < r; j += 32) a = fmaf(sb[j], su[g * r + j], a);
     a = warp_sum(a);
@@ -978,27 +990,27 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   {
     // partial M^T u over this thread's rows, for its 4 columns and every head
     const int cq = tid % (D / 4), rg = tid / (D / 4);       // D/4 column quads, RG row groups
-    float4 acc[G];
+    float4 acc[HG];
 #pragma unroll
-    for (int g = 0; g < G; ++g) acc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int gg = 0; gg < HG; ++gg) acc[gg] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
     for (int j = rg; j < r; j += RG) {
       const float4 mv = reinterpret_cast<const float4*>(sM + (size_t)j * D)[cq];
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float uu = su[g * r + j];
-        acc[g].x = fmaf(mv.x, uu, acc[g].x);
-        acc[g].y = fmaf(mv.y, uu, acc[g].y);
-        acc[g].z = fmaf(mv.z, uu, acc[g].z);
-        acc[g].w = fmaf(mv.w, uu, acc[g].w);
+      for (int gg = 0; gg < HG; ++gg) {
+        const float uu = su[(hg0 + gg) * r + j];
+        acc[gg].x = fmaf(mv.x, uu, acc[gg].x);
+        acc[gg].y = fmaf(mv.y, uu, acc[gg].y);
+        acc[gg].z = fmaf(mv.z, uu, acc[gg].z);
+        acc[gg].w = fmaf(mv.w, uu, acc[gg].w);
       }
     }
 #pragma unroll
-    for (int g = 0; g < G; ++g)
-      reinterpret_cast<float4*>(snum + ((size_t)rg * G + g) * D)[cq] = acc[g];
+    for (int gg = 0; gg < HG; ++gg)
+      reinterpret_cast<float4*>(snum + ((size_t)rg * G + hg0 + gg) * D)[cq] = acc[gg];
   }
   __syncthreads();
-  for (int i = tid; i < G * D; i += kThreads) {
+  for (int i = hg0 * D + tid; i < (hg0 + HG) * D; i += kThreads) {
     const int g = i / D, c = i % D;
     float num = 0.f;
 #pragma unroll
@@ -1006,6 +1018,16 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     ro[i] = moment ? num : sgate[g] * (num / sden[g]);
   }
   __syncthreads();
+  if (kNro > 1 && rank > S) {
+    // the second readout CTA: its heads' readout (and b . u, which the
+    // moment readout's merge needs) into the merge CTA, then arrive
+    cluster_wait();   // phase 0: the merge CTA is running
+    float* ro_m = cluster.map_shared_rank(ro, S);
+    for (int i = hg0 * D + tid; i < (hg0 + HG) * D; i += kThreads) ro_m[i] = ro[i];
+    if (tid < HG) cluster.map_shared_rank(sden, S)[hg0 + tid] = sden[hg0 + tid];
+    cluster_arrive_release();   // phase 1
+    return;
+  }
 
   // ---- merge the S attention states that the other CTAs pushed into the slots
   cluster_wait();             // phase 0
@@ -1075,7 +1097,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   }
 }
 
-template <typename T, int D, int G, bool kTma>
+template <typename T, int D, int G, bool kTma, int NRO>
 cudaError_t launch_tgs(const Ctx& c, int S, int nst, int batch, const void* q, const void* kn,
                       const void* vn, void* K_ret, void* V_ret, int32_t* cache_len, int cap,
                       const float* M, const float* bstab, const float* s_v, const float* n_e,
@@ -1086,7 +1108,7 @@ cudaError_t launch_tgs(const Ctx& c, int S, int nst, int batch, const void* q, c
   const bool m_in_w = c.cfg.readout == IMEM_READOUT_MOMENT || kTma;
   const size_t smem = DecSmem<D, G>::total(kBf16, nst, r, S, m_in_w);
   const uint32_t slot_off = (uint32_t)DecSmem<D, G>::slot_off(r, m_in_w);
-  auto k = decode_kernel<T, D, G, kTma>;
+  auto k = decode_kernel<T, D, G, kTma, NRO>;
   static size_t attr_smem[64] = {};   // per instantiation and device: largest size set so far
   const int dv = c.device & 63;
   if (attr_smem[dv] < smem) {
@@ -1096,13 +1118,14 @@ cudaError_t launch_tgs(const Ctx& c, int S, int nst, int batch, const void* q, c
     attr_smem[dv] = smem;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(S + 1, c.cfg.n_kv_heads, batch);
+  const int nro = NRO;   // readout CTAs per cluster
+  cfg.gridDim = dim3(S + nro, c.cfg.n_kv_heads, batch);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = S + 1;
+  attr[0].val.clusterDim.x = S + nro;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1134,13 +1157,20 @@ cudaError_t launch_tg(const Ctx& c, int S, int nst, int batch, const void* q, co
                       const void* vn, void* K_ret, void* V_ret, int32_t* cache_len, int cap,
                       const float* M, const float* bstab, const float* s_v, const float* n_e,
                       void* out, int* counters, cudaStream_t st) {
-  const bool tma = std::is_same<T, __nv_bfloat16>::value &&
-                   batch * c.cfg.n_kv_heads * (S + 1) > 2 * c.num_sms;
-  if (tma && std::is_same<T, __nv_bfloat16>::value)
-    return launch_tgs<T, D, G, std::is_same<T, __nv_bfloat16>::value>(
-        c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M, bstab, s_v, n_e, out, counters, st);
-  return launch_tgs<T, D, G, false>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M,
-                                    bstab, s_v, n_e, out, counters, st);
+  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+  const int units = batch * c.cfg.n_kv_heads;
+  const bool tma = kBf16 && units * (S + 1) > 2 * c.num_sms;
+  if (tma)
+    return launch_tgs<T, D, G, kBf16, 1>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M,
+                                         bstab, s_v, n_e, out, counters, st);
+  // a second readout CTA where the grid keeps about 1.5 CTAs per SM with it
+  if constexpr (G >= 2) {
+    if (S + 2 <= kDecodeMaxSplits && units * (S + 2) * 2 <= 3 * c.num_sms + 4)
+      return launch_tgs<T, D, G, false, 2>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap,
+                                           M, bstab, s_v, n_e, out, counters, st);
+  }
+  return launch_tgs<T, D, G, false, 1>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M,
+                                       bstab, s_v, n_e, out, counters, st);
 }
 
 template <typename T, int D>
