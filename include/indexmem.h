@@ -344,6 +344,18 @@ imem_status imem_decode_moment(imem_ctx* ctx, int batch, const void* q, const vo
  *                      same buffer for every range of one prefill (it keeps the
  *                      retained tokens' indexer keys and importances); it also
  *                      serves imem_decode.
+ * Ordering: the memory update of a range's evicted tokens runs on a second
+ * stream of the context, after this call's selection on `stream`, so that it
+ * overlaps the next range's prologue and scoring. Every later call on the
+ * context makes its stream wait for that update: the next range's call
+ * before its selection, every other call before it enqueues anything; and
+ * the call with finalize = 1 waits for its own update before it returns (in
+ * the order of `stream`). Between two calls a caller that reads or writes M, bstab or
+ * `evicted` with its own work calls imem_join (or imem_sync) on its stream
+ * first. The second stream and its events are created at the first call:
+ * make it before any stream capture, and capture whole sequences of calls
+ * up to the one with finalize = 1 (a capture that ends with an update still
+ * pending on the second stream is unjoined).
  * Errors: INVALID_ARG, SHAPE (ranges, cap), ALIGN, CUDA; UNSUPPORTED for a
  * context in IMEM_READOUT_MOMENT mode. */
 imem_status imem_workspace_size_evict(imem_ctx* ctx, int batch, int L, int B, int chunk_max,
@@ -423,7 +435,18 @@ imem_status imem_decode_online(imem_ctx* ctx, int batch, int B, const void* x_ne
  * Errors: INVALID_ARG (limit out of range), CUDA. */
 imem_status imem_selftest_wait(imem_ctx* ctx, long long limit_cycles, void* stream);
 
-/* Waits for the stream, then reports the first error the device recorded for
+/* Makes `stream` wait for work that the context still runs on its second
+ * stream: the memory update of the last range given to
+ * imem_prefill_evict_chunk without finalize (no counterpart in the paper;
+ * stream-ordered, no host synchronisation, nothing else enqueued). Every
+ * other call of the library on the context does the same before its own
+ * work; a caller needs it only before its own reads or writes of M, bstab or
+ * the evicted positions between two pre-eviction calls.
+ * Errors: INVALID_ARG, CUDA. */
+imem_status imem_join(imem_ctx* ctx, void* stream);
+
+/* Waits for the stream (after imem_join's wait for the context's second
+ * stream), then reports the first error the device recorded for
  * this context since the last imem_sync (TIMEOUT for a bounded wait that ran
  * out, SHAPE for a decode into a full cache, RANGE for an input value out of
  * range) or a CUDA error, and clears it. */

@@ -74,6 +74,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.imem_decode.argtypes = [vp, i, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp]
     lib.imem_sync.restype = i
     lib.imem_sync.argtypes = [vp, vp]
+    lib.imem_join.restype = i
+    lib.imem_join.argtypes = [vp, vp]
     lib.imem_workspace_size_evict.restype = i
     lib.imem_workspace_size_evict.argtypes = [vp, i, i, i, i, ctypes.POINTER(ctypes.c_size_t)]
     lib.imem_prefill_evict_chunk.restype = i
@@ -276,6 +278,12 @@ def static_status(stream=None) -> None:
     """imem_static_status: raises if a call of update_memory_static on this
     device recorded a device error since the last query (and clears it)."""
     _check(load().imem_static_status(_stream(stream)), "imem_static_status")
+
+
+def join(ctx, stream=None) -> None:
+    """imem_join: `stream` waits for a pre-eviction memory update still
+    running on the context's second stream."""
+    _check(load().imem_join(ctx, _stream(stream)), "imem_join")
 
 
 def sync(ctx, stream=None) -> None:

@@ -156,6 +156,31 @@ imem_status online_streams(Ctx& c) {
   return IMEM_OK;
 }
 
+
+// The pre-eviction's second stream and its events, created on first use.
+imem_status prefill_streams(Ctx& c) {
+  if (!c.side && cudaStreamCreateWithFlags(&c.side, cudaStreamNonBlocking) != cudaSuccess)
+    return IMEM_ERR_CUDA;
+  if (!c.ev_pe_fork &&
+      cudaEventCreateWithFlags(&c.ev_pe_fork, cudaEventDisableTiming) != cudaSuccess)
+    return IMEM_ERR_CUDA;
+  if (!c.ev_pe_done &&
+      cudaEventCreateWithFlags(&c.ev_pe_done, cudaEventDisableTiming) != cudaSuccess)
+    return IMEM_ERR_CUDA;
+  return IMEM_OK;
+}
+
+// Makes `st` wait for a pre-eviction memory update still running on the
+// second stream (see imem_prefill_evict_chunk); every call that enqueues work
+// does this first, so the update is complete before anything else of the
+// library reads or writes the memory state or the evicted positions.
+imem_status wait_pending(Ctx& c, cudaStream_t st) {
+  if (!c.pe_pending) return IMEM_OK;
+  if (cudaStreamWaitEvent(st, c.ev_pe_done, 0) != cudaSuccess) return IMEM_ERR_CUDA;
+  c.pe_pending = false;
+  return IMEM_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -265,6 +290,8 @@ void imem_destroy(imem_ctx* h) {
   cudaFree(c.err);
   if (c.ev_fork) cudaEventDestroy(c.ev_fork);
   if (c.ev_join) cudaEventDestroy(c.ev_join);
+  if (c.ev_pe_fork) cudaEventDestroy(c.ev_pe_fork);
+  if (c.ev_pe_done) cudaEventDestroy(c.ev_pe_done);
   if (c.side) cudaStreamDestroy(c.side);
   free(h);
 }
@@ -302,6 +329,7 @@ imem_status imem_score_and_evict(imem_ctx* h, int batch, int L, int B, const voi
     IMEM_CHECK(check_ptr(V_ret));
   }
   IMEM_CHECK(check_device(c));
+  IMEM_CHECK(wait_pending(h->c, (cudaStream_t)stream));
   cudaStream_t st = (cudaStream_t)stream;
   const imem::Workspace ws = imem::workspace_layout(c, batch, L);
   char* wsb = (char*)workspace;
@@ -330,6 +358,7 @@ imem_status imem_indexer_features(imem_ctx* h, int batch, int L, const void* X, 
   IMEM_CHECK(check_ptr(running_max));
   IMEM_CHECK(check_ptr(workspace));
   IMEM_CHECK(check_device(c));
+  IMEM_CHECK(wait_pending(h->c, (cudaStream_t)stream));
   const imem::Workspace ws = imem::workspace_layout(c, batch, L);
   char* wsb = (char*)workspace;
   return cuda_status(imem::launch_prologue(c, batch, L, X, Q, q_begin, q_end,
@@ -347,6 +376,7 @@ imem_status imem_indexer_score(imem_ctx* h, int batch, int L, float* running_max
   IMEM_CHECK(check_ptr(running_max));
   IMEM_CHECK(check_ptr(workspace));
   IMEM_CHECK(check_device(c));
+  IMEM_CHECK(wait_pending(h->c, (cudaStream_t)stream));
   const imem::Workspace ws = imem::workspace_layout(c, batch, L);
   char* wsb = (char*)workspace;
   return cuda_status(imem::launch_scoring(c, batch, L, (const __nv_bfloat16*)(wsb + ws.qt_off),
@@ -371,6 +401,7 @@ imem_status imem_select_compact(imem_ctx* h, int batch, int L, int B, const floa
   IMEM_CHECK(check_ptr(V_ret));
   IMEM_CHECK(check_ptr(workspace));
   IMEM_CHECK(check_device(c));
+  IMEM_CHECK(wait_pending(h->c, (cudaStream_t)stream));
   cudaStream_t st = (cudaStream_t)stream;
   const imem::Workspace ws = imem::workspace_layout(c, batch, L);
   IMEM_CHECK(cuda_status(imem::clear_decode_tags(c, batch, workspace, st)));
@@ -395,6 +426,7 @@ imem_status imem_update_memory(imem_ctx* h, int batch, int L, const void* K, con
   IMEM_CHECK(check_ptr(bstab));
   IMEM_CHECK(check_ptr(workspace));
   IMEM_CHECK(check_device(c));
+  IMEM_CHECK(wait_pending(h->c, (cudaStream_t)stream));
   const imem::Workspace ws = imem::workspace_layout(c, batch, L);
   float* part = (float*)((char*)workspace + ws.mem_part_off);
   IMEM_CHECK(cuda_status(imem::clear_decode_tags(c, batch, workspace, (cudaStream_t)stream)));
@@ -422,6 +454,7 @@ imem_status imem_update_moments(imem_ctx* h, int batch, int L, const void* K, co
   IMEM_CHECK(check_ptr(n_e));
   IMEM_CHECK(check_ptr(workspace));
   IMEM_CHECK(check_device(c));
+  IMEM_CHECK(wait_pending(h->c, (cudaStream_t)stream));
   const imem::Workspace ws = imem::workspace_layout(c, batch, L);
   float* part = (float*)((char*)workspace + ws.mem_part_off);
   float* svp = (float*)((char*)workspace + ws.sv_part_off);
@@ -454,6 +487,7 @@ imem_status decode_common(imem_ctx* h, int batch, const void* q, const void* k_n
   IMEM_CHECK(check_ptr(out));
   IMEM_CHECK(check_ptr(workspace));
   IMEM_CHECK(check_device(c));
+  IMEM_CHECK(wait_pending(h->c, (cudaStream_t)stream));
   // the decode regions of the workspace do not depend on L
   const imem::Workspace ws = imem::workspace_layout(c, batch, 1);
   char* wsb = (char*)workspace;
@@ -488,6 +522,7 @@ imem_status imem_decode_invalidate(imem_ctx* h, int batch, void* workspace, void
   if (batch < 1) return IMEM_ERR_SHAPE;
   IMEM_CHECK(check_ptr(workspace));
   IMEM_CHECK(check_device(h->c));
+  IMEM_CHECK(wait_pending(h->c, (cudaStream_t)stream));
   return cuda_status(imem::clear_decode_tags(h->c, batch, workspace, (cudaStream_t)stream));
 }
 
@@ -537,6 +572,7 @@ imem_status imem_prefill_evict_chunk(imem_ctx* h, int batch, int L, int B, int c
     IMEM_CHECK(check_ptr(V_ret));
   }
   IMEM_CHECK(check_device(c));
+  IMEM_CHECK(prefill_streams(h->c));
   cudaStream_t st = (cudaStream_t)stream;
   const int Lc = B + chunk_max;
   const imem::EvictWorkspace ws = imem::evict_workspace_layout(c, batch, B, chunk_max);
@@ -558,19 +594,35 @@ imem_status imem_prefill_evict_chunk(imem_ctx* h, int batch, int L, int B, int c
   if (cand_importance)
     IMEM_CHECK(cuda_status(cudaMemcpyAsync(cand_importance, eb.I_c, (size_t)batch * Lc * sizeof(float),
                                            cudaMemcpyDeviceToDevice, st)));
+  // the previous range's memory update, if still running, reads `evicted`
+  // and owns M, bstab: the selection below rewrites `evicted`
+  IMEM_CHECK(wait_pending(h->c, st));
   if (n_ev > 0) {
     IMEM_CHECK(cuda_status(imem::launch_evict_chunk(c, batch, B, Lc, n_R, q_begin, C, eb, retained,
                                                     evicted, st)));
+    // the range's memory update on the second stream: it needs only K, V,
+    // `evicted` and the memory, so it runs beside the next range's prologue
+    // and scoring; the next call (or the end of this one, with finalize)
+    // waits for it
     float* part = (float*)(wsb + ws.base.mem_part_off);
-    IMEM_CHECK(cuda_status(imem::launch_memory_update(c, batch, L, K, V, evicted, n_ev, mem_chunk,
+    IMEM_CHECK(cuda_status(cudaEventRecord(c.ev_pe_fork, st)));
+    IMEM_CHECK(cuda_status(cudaStreamWaitEvent(c.side, c.ev_pe_fork, 0)));
+    const cudaError_t me = imem::launch_memory_update(c, batch, L, K, V, evicted, n_ev, mem_chunk,
                                                       M, bstab, part, nullptr, nullptr, nullptr,
-                                                      st)));
+                                                      c.side);
+    // recorded even after a failed launch, so that the wait below never
+    // refers to an event of an earlier range
+    IMEM_CHECK(cuda_status(cudaEventRecord(c.ev_pe_done, c.side)));
+    h->c.pe_pending = true;
+    IMEM_CHECK(cuda_status(me));
   } else {
     IMEM_CHECK(cuda_status(imem::launch_append_positions(batch, B, n_R, q_begin, C, retained, st)));
   }
-  if (finalize)
+  if (finalize) {
     IMEM_CHECK(cuda_status(imem::launch_gather(c, batch, L, B < L ? B : L, retained, B, K, V,
                                                K_ret, V_ret, cap, st)));
+    IMEM_CHECK(wait_pending(h->c, st));
+  }
   return IMEM_OK;
 }
 
@@ -590,6 +642,7 @@ imem_status imem_online_init(imem_ctx* h, int batch, int L, int B, const float* 
   IMEM_CHECK(check_ptr(pos_ret));
   IMEM_CHECK(check_ptr(next_pos));
   IMEM_CHECK(check_device(c));
+  IMEM_CHECK(wait_pending(h->c, (cudaStream_t)stream));
   IMEM_CHECK(online_streams(h->c));
   const imem::Workspace ws = imem::workspace_layout(c, batch, L);
   const __nv_bfloat16* kh = (const __nv_bfloat16*)((const char*)workspace + ws.kh_off);
@@ -625,6 +678,7 @@ imem_status imem_decode_online(imem_ctx* h, int batch, int B, const void* x_new,
   IMEM_CHECK(check_ptr(bstab));
   IMEM_CHECK(check_ptr(out));
   IMEM_CHECK(check_device(c));
+  IMEM_CHECK(wait_pending(h->c, (cudaStream_t)stream));
   IMEM_CHECK(online_streams(h->c));
   cudaStream_t st = (cudaStream_t)stream;
   const imem::Workspace ws = imem::workspace_layout(c, batch, 1);
@@ -657,11 +711,19 @@ imem_status imem_selftest_wait(imem_ctx* h, long long limit_cycles, void* stream
   if (!h) return IMEM_ERR_INVALID_ARG;
   if (limit_cycles < 1 || limit_cycles > 2000000000LL) return IMEM_ERR_INVALID_ARG;
   IMEM_CHECK(check_device(h->c));
+  IMEM_CHECK(wait_pending(h->c, (cudaStream_t)stream));
   return cuda_status(imem::launch_wait_selftest(h->c, limit_cycles, (cudaStream_t)stream));
+}
+
+imem_status imem_join(imem_ctx* h, void* stream) {
+  if (!h) return IMEM_ERR_INVALID_ARG;
+  IMEM_CHECK(check_device(h->c));
+  return wait_pending(h->c, (cudaStream_t)stream);
 }
 
 imem_status imem_sync(imem_ctx* h, void* stream) {
   if (!h) return IMEM_ERR_INVALID_ARG;
+  IMEM_CHECK(wait_pending(h->c, (cudaStream_t)stream));
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return IMEM_ERR_CUDA;
   int code = 0;

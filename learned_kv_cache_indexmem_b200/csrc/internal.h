@@ -31,6 +31,12 @@ struct Ctx {
   // (forked from and joined back into the caller's stream by events)
   cudaStream_t side;
   cudaEvent_t ev_fork, ev_join;
+  // pre-eviction: a range's memory update runs on `side`, after ev_pe_fork
+  // of the caller's stream, beside the next range's prologue and scoring;
+  // ev_pe_done marks its end, and while pe_pending is set every call on the
+  // context makes its stream wait for ev_pe_done before it enqueues work
+  cudaEvent_t ev_pe_fork, ev_pe_done;
+  bool pe_pending;
 };
 
 // Indexer rows in the workspace: d_I features padded to 64 bf16 (128 bytes).

@@ -85,6 +85,59 @@ __device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity,
   return true;
 }
 
+// Waits, with acquire semantics at cluster scope, for the phase with the given
+// parity (for phases completed by arrivals of another CTA of the cluster,
+// whose shared-memory writes before its release-arrive must be visible);
+// bounded like mbar_wait.
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
+                                                  long long limit = kWaitLimit) {
+  auto probe = [&]() {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+  };
+  if (probe()) return true;
+  const long long t0 = clock64();
+  while (!probe()) {
+    if (clock64() - t0 > limit) return false;
+  }
+  return true;
+}
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+// Arrives on an mbarrier of another CTA of the cluster (address from mapa),
+// releasing this thread's earlier memory accesses at cluster scope.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_bar)
+               : "memory");
+}
+// 16 bytes into another CTA's shared memory (address from mapa).
+__device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, float a, float b, float c,
+                                              float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"r"(cluster_addr), "f"(a),
+               "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+  return r;
+}
+// Every thread of every CTA of the cluster: arrive (release) and wait (acquire).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\nbarrier.cluster.wait.acquire;\n" ::
+                   : "memory");
+}
+
 // Generic-proxy writes to shared memory made visible to the async proxy
 // (tensor core / TMA) -- each writing thread fences before signalling.
 __device__ __forceinline__ void fence_proxy_async() {

@@ -84,6 +84,7 @@ def test_null_context_is_invalid_for_every_call():
     assert lib.imem_update_memory(None, 1, 16, 16, 16, 16, 4, 64, 16, 16, 16, None) == 1
     assert lib.imem_decode(None, 1, 16, 16, 16, 16, 16, 16, 8, 16, 16, 16, 16, None) == 1
     assert lib.imem_sync(None, None) == 1
+    assert lib.imem_join(None, None) == 1
     n2 = ctypes.c_size_t()
     assert lib.imem_workspace_size_evict(None, 1, 16, 4, 8, ctypes.byref(n2)) == 1
     assert lib.imem_prefill_evict_chunk(None, 1, 16, 4, 8, 16, 16, 16, 16, 0, 8, 16, 16, None, 16,

@@ -6,8 +6,9 @@ their order, the memory against the sequential update in eviction order, and
 the final compaction."""
 import numpy as np
 import pytest
+import torch
 
-from learned_kv_cache_indexmem_b200 import synth
+from learned_kv_cache_indexmem_b200 import binding, synth
 from oracle import indexmem_oracle as om
 
 from .parity import Case, check_memory, check_scores, to_np
@@ -93,3 +94,37 @@ def test_single_range_equals_one_shot_prefill(cuda_device):
     np.testing.assert_array_equal(to_np(st_a.bstab), to_np(st_b.bstab))
     a.close()
     b_.close()
+
+
+def test_memory_between_ranges_after_join(cuda_device):
+    # each range's memory update runs on the context's second stream beside the
+    # next range's prologue and scoring; after imem_join the caller's stream
+    # sees M and bstab with every eviction so far, range by range
+    L, B, chunk, batch = 2100, 410, 512, 2
+    case = Case(W["c1"], cuda_device, L=L, batch=batch, n_decode=1)
+    lay = case.layer()
+    st = lay.new_state(batch, L, B, B + 4, cuda_device)
+    d = case.in_dev
+    ws = lay.workspace_evict(batch, L, B, chunk, cuda_device)
+    ev = torch.empty(batch * chunk, dtype=torch.int32, device=cuda_device)
+    evicted = [[] for _ in range(batch)]
+    checked = 0
+    for q0 in range(0, L, chunk):
+        q1 = min(L, q0 + chunk)
+        n_ev = max(0, min(B, q0) + (q1 - q0) - B)
+        binding.prefill_evict_chunk(lay.ctx, batch, L, B, chunk, d["X"], d["Q"], d["K"], d["V"],
+                                    q0, q1, st.idx_retained, ev, None, st.M, st.bstab, 64,
+                                    q1 == L, st.K_ret, st.V_ret, st.K_ret.shape[1], ws)
+        binding.join(lay.ctx)
+        e = to_np(ev[:batch * n_ev].view(batch, n_ev)).astype(np.int64)
+        for bi in range(batch):
+            evicted[bi] += list(e[bi])
+        if n_ev:
+            M_ref, b_ref = om.memory_update(case.in_cpu["K"], case.in_cpu["V"], np.array(evicted),
+                                            case.w_cpu["W_phi"], case.shape.lam)
+            check_memory(to_np(st.M), to_np(st.bstab), M_ref, b_ref,
+                         "after range %d-%d" % (q0, q1))
+            checked += 1
+    assert checked >= 3
+    lay.sync()
+    lay.close()
