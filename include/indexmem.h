@@ -329,9 +329,9 @@ imem_status imem_decode_moment(imem_ctx* ctx, int batch, const void* q, const vo
  * position order, into the memory: M, bstab updated as imem_update_memory does
  * with them (after all tokens evicted by earlier ranges).
  *   X, Q, K, V         as imem_score_and_evict ([batch, L, ...], model dtype).
- *   retained [batch, B] int32, in/out: the retained positions, ascending (the
- *                      first n_R of each row valid before the call, the first
- *                      min(B, q_end) after it). Caller-owned state.
+ *   retained [batch, B] int32, out: the retained positions, ascending (the
+ *                      first min(B, q_end) of each row valid after the call;
+ *                      the workspace keeps the library's own copy).
  *   evicted [batch * chunk_max] int32, out: [batch, n_ev] packed, ascending.
  *   cand_importance    NULL or [batch, B + chunk_max] fp32, out: the candidates'
  *                      pooled importance before selection (row: n_R retained,
@@ -344,18 +344,22 @@ imem_status imem_decode_moment(imem_ctx* ctx, int batch, const void* q, const vo
  *                      same buffer for every range of one prefill (it keeps the
  *                      retained tokens' indexer keys and importances); it also
  *                      serves imem_decode.
- * Ordering: the memory update of a range's evicted tokens runs on a second
- * stream of the context, after this call's selection on `stream`, so that it
- * overlaps the next range's prologue and scoring. Every later call on the
- * context makes its stream wait for that update: the next range's call
- * before its selection, every other call before it enqueues anything; and
- * the call with finalize = 1 waits for its own update before it returns (in
- * the order of `stream`). Between two calls a caller that reads or writes M, bstab or
- * `evicted` with its own work calls imem_join (or imem_sync) on its stream
- * first. The second stream and its events are created at the first call:
- * make it before any stream capture, and capture whole sequences of calls
- * up to the one with finalize = 1 (a capture that ends with an update still
- * pending on the second stream is unjoined).
+ * Ordering: a range's selection, compaction (retained, evicted) and memory
+ * update run on a second stream of the context, after this call's scoring
+ * on `stream`, so that they overlap the next range's prologue (and the memory
+ * update its scoring too). Every later call on the context makes its stream
+ * wait for them: the next range's call for the compaction before its
+ * scoring, every other call for all of it before it enqueues anything; the
+ * call with finalize = 1 waits for its own before its compaction of K_ret,
+ * V_ret (in the order of `stream`). Between two calls a caller that reads or
+ * writes retained, evicted, M or bstab with its own work calls imem_join (or
+ * imem_sync) on its stream first. A context runs one pre-eviction prefill at
+ * a time: the call with q_begin = 0 starts a new one (the context keeps
+ * which of the workspace's two candidate buffers the next range uses). The
+ * second stream and its events are created at the first call: make it
+ * before any stream capture, and capture whole sequences of calls up to the
+ * one with finalize = 1 (a capture that ends with work still pending on the
+ * second stream is unjoined).
  * Errors: INVALID_ARG, SHAPE (ranges, cap), ALIGN, CUDA; UNSUPPORTED for a
  * context in IMEM_READOUT_MOMENT mode. */
 imem_status imem_workspace_size_evict(imem_ctx* ctx, int batch, int L, int B, int chunk_max,
@@ -436,12 +440,12 @@ imem_status imem_decode_online(imem_ctx* ctx, int batch, int B, const void* x_ne
 imem_status imem_selftest_wait(imem_ctx* ctx, long long limit_cycles, void* stream);
 
 /* Makes `stream` wait for work that the context still runs on its second
- * stream: the memory update of the last range given to
- * imem_prefill_evict_chunk without finalize (no counterpart in the paper;
+ * stream: the selection, compaction and memory update of the last range given
+ * to imem_prefill_evict_chunk without finalize (no counterpart in the paper;
  * stream-ordered, no host synchronisation, nothing else enqueued). Every
  * other call of the library on the context does the same before its own
- * work; a caller needs it only before its own reads or writes of M, bstab or
- * the evicted positions between two pre-eviction calls.
+ * work; a caller needs it only before its own reads or writes of M, bstab,
+ * the retained or the evicted positions between two pre-eviction calls.
  * Errors: INVALID_ARG, CUDA. */
 imem_status imem_join(imem_ctx* ctx, void* stream);
 

@@ -67,11 +67,12 @@ cudaError_t clear_decode_tags(const Ctx& c, int batch, void* workspace, cudaStre
 }
 
 // Pre-eviction workspace: the plain layout over Lc = B + chunk_max candidate
-// rows (its q~ and k^ regions become the candidate buffers), then the
-// candidates' importances and the compaction temporaries.
+// rows (its q~ region holds the range's queries, its k^ region candidate
+// buffer 0's keys), then buffer 1's keys, both buffers' importances and
+// retained positions, and the selection's index lists.
 struct EvictWorkspace {
   Workspace base;
-  size_t I_c_off, kh_tmp_off, I_tmp_off, pos_tmp_off, idx_r_off, idx_e_off, total;
+  size_t kh1_off, I_off[2], pos_off[2], idx_r_off, idx_e_off, total;
 };
 
 EvictWorkspace evict_workspace_layout(const Ctx& c, int batch, int B, int chunk_max) {
@@ -79,10 +80,11 @@ EvictWorkspace evict_workspace_layout(const Ctx& c, int batch, int B, int chunk_
   EvictWorkspace w;
   w.base = workspace_layout(c, batch, (int)Lc);
   size_t off = w.base.total;
-  w.I_c_off = off;     off = align_up(off + (size_t)batch * Lc * sizeof(float), 256);
-  w.kh_tmp_off = off;  off = align_up(off + (size_t)batch * B * kIdxPad * 2, 1024);
-  w.I_tmp_off = off;   off = align_up(off + (size_t)batch * B * sizeof(float), 256);
-  w.pos_tmp_off = off; off = align_up(off + (size_t)batch * B * sizeof(int32_t), 256);
+  w.kh1_off = off;     off = align_up(off + (size_t)batch * Lc * kIdxPad * 2, 1024);
+  w.I_off[0] = off;    off = align_up(off + (size_t)batch * Lc * sizeof(float), 256);
+  w.I_off[1] = off;    off = align_up(off + (size_t)batch * Lc * sizeof(float), 256);
+  w.pos_off[0] = off;  off = align_up(off + (size_t)batch * B * sizeof(int32_t), 256);
+  w.pos_off[1] = off;  off = align_up(off + (size_t)batch * B * sizeof(int32_t), 256);
   w.idx_r_off = off;   off = align_up(off + (size_t)batch * B * sizeof(int32_t), 256);
   w.idx_e_off = off;   off = align_up(off + (size_t)batch * Lc * sizeof(int32_t), 256);
   w.total = off;
@@ -164,20 +166,31 @@ imem_status prefill_streams(Ctx& c) {
   if (!c.ev_pe_fork &&
       cudaEventCreateWithFlags(&c.ev_pe_fork, cudaEventDisableTiming) != cudaSuccess)
     return IMEM_ERR_CUDA;
+  if (!c.ev_pe_compact &&
+      cudaEventCreateWithFlags(&c.ev_pe_compact, cudaEventDisableTiming) != cudaSuccess)
+    return IMEM_ERR_CUDA;
   if (!c.ev_pe_done &&
       cudaEventCreateWithFlags(&c.ev_pe_done, cudaEventDisableTiming) != cudaSuccess)
     return IMEM_ERR_CUDA;
   return IMEM_OK;
 }
 
-// Makes `st` wait for a pre-eviction memory update still running on the
-// second stream (see imem_prefill_evict_chunk); every call that enqueues work
-// does this first, so the update is complete before anything else of the
-// library reads or writes the memory state or the evicted positions.
+// Makes `st` wait for pre-eviction work still running on the second stream
+// (see imem_prefill_evict_chunk); every call that enqueues work does this
+// first, so that work is complete before anything else of the library reads
+// or writes the memory state, the retained or the evicted positions.
 imem_status wait_pending(Ctx& c, cudaStream_t st) {
   if (!c.pe_pending) return IMEM_OK;
   if (cudaStreamWaitEvent(st, c.ev_pe_done, 0) != cudaSuccess) return IMEM_ERR_CUDA;
   c.pe_pending = false;
+  c.pe_compact_pending = false;
+  return IMEM_OK;
+}
+// The same for the last range's selection and compaction only.
+imem_status wait_compact(Ctx& c, cudaStream_t st) {
+  if (!c.pe_compact_pending) return IMEM_OK;
+  if (cudaStreamWaitEvent(st, c.ev_pe_compact, 0) != cudaSuccess) return IMEM_ERR_CUDA;
+  c.pe_compact_pending = false;
   return IMEM_OK;
 }
 
@@ -291,6 +304,7 @@ void imem_destroy(imem_ctx* h) {
   if (c.ev_fork) cudaEventDestroy(c.ev_fork);
   if (c.ev_join) cudaEventDestroy(c.ev_join);
   if (c.ev_pe_fork) cudaEventDestroy(c.ev_pe_fork);
+  if (c.ev_pe_compact) cudaEventDestroy(c.ev_pe_compact);
   if (c.ev_pe_done) cudaEventDestroy(c.ev_pe_done);
   if (c.side) cudaStreamDestroy(c.side);
   free(h);
@@ -573,55 +587,75 @@ imem_status imem_prefill_evict_chunk(imem_ctx* h, int batch, int L, int B, int c
   }
   IMEM_CHECK(check_device(c));
   IMEM_CHECK(prefill_streams(h->c));
+  Ctx& cm = h->c;
   cudaStream_t st = (cudaStream_t)stream;
+  if (q_begin == 0) {
+    // a new prefill: nothing of an earlier one may still run, buffer 0 first
+    IMEM_CHECK(wait_pending(cm, st));
+    cm.pe_parity = 0;
+  }
   const int Lc = B + chunk_max;
   const imem::EvictWorkspace ws = imem::evict_workspace_layout(c, batch, B, chunk_max);
   char* wsb = (char*)workspace;
   IMEM_CHECK(cuda_status(imem::clear_decode_tags(c, batch, workspace, st)));
+  // two candidate buffers: this range's candidates in buffer p, the rows it
+  // retains compacted into buffer 1 - p (no row is overwritten before it is
+  // read, and the next range's prologue writes its rows there while this
+  // range's selection may still read buffer p)
+  const int p = cm.pe_parity;
+  __nv_bfloat16* khb[2] = {(__nv_bfloat16*)(wsb + ws.base.kh_off),
+                           (__nv_bfloat16*)(wsb + ws.kh1_off)};
   imem::EvictBuffers eb;
   __nv_bfloat16* qt = (__nv_bfloat16*)(wsb + ws.base.qt_off);
-  eb.kh_c = (__nv_bfloat16*)(wsb + ws.base.kh_off);
-  eb.I_c = (float*)(wsb + ws.I_c_off);
-  eb.kh_tmp = (__nv_bfloat16*)(wsb + ws.kh_tmp_off);
-  eb.I_tmp = (float*)(wsb + ws.I_tmp_off);
-  eb.pos_tmp = (int32_t*)(wsb + ws.pos_tmp_off);
+  eb.kh_c = khb[p];
+  eb.I_c = (float*)(wsb + ws.I_off[p]);
+  eb.pos_c = (int32_t*)(wsb + ws.pos_off[p]);
+  eb.kh_n = khb[1 - p];
+  eb.I_n = (float*)(wsb + ws.I_off[1 - p]);
+  eb.pos_n = (int32_t*)(wsb + ws.pos_off[1 - p]);
   eb.idx_r = (int32_t*)(wsb + ws.idx_r_off);
   eb.idx_e = (int32_t*)(wsb + ws.idx_e_off);
   // the range's indexer features go to candidate rows [n_R, n)
   IMEM_CHECK(cuda_status(imem::launch_prologue(c, batch, L, X, Q, q_begin, q_end, qt, eb.kh_c,
                                                eb.I_c, st, Lc, n_R - q_begin)));
+  // rows [0, n_R) of buffer p come from the previous range's compaction
+  IMEM_CHECK(wait_compact(cm, st));
   IMEM_CHECK(cuda_status(imem::launch_scoring(c, batch, Lc, qt, eb.kh_c, eb.I_c, n_R, n, st)));
   if (cand_importance)
     IMEM_CHECK(cuda_status(cudaMemcpyAsync(cand_importance, eb.I_c, (size_t)batch * Lc * sizeof(float),
                                            cudaMemcpyDeviceToDevice, st)));
-  // the previous range's memory update, if still running, reads `evicted`
-  // and owns M, bstab: the selection below rewrites `evicted`
-  IMEM_CHECK(wait_pending(h->c, st));
   if (n_ev > 0) {
-    IMEM_CHECK(cuda_status(imem::launch_evict_chunk(c, batch, B, Lc, n_R, q_begin, C, eb, retained,
-                                                    evicted, st)));
-    // the range's memory update on the second stream: it needs only K, V,
-    // `evicted` and the memory, so it runs beside the next range's prologue
-    // and scoring; the next call (or the end of this one, with finalize)
-    // waits for it
+    // selection, compaction and the memory update on the second stream: they
+    // run beside the next range's prologue (and the memory update beside its
+    // scoring); the next call waits for the compaction before its scoring,
+    // every other call for all of it first
     float* part = (float*)(wsb + ws.base.mem_part_off);
-    IMEM_CHECK(cuda_status(cudaEventRecord(c.ev_pe_fork, st)));
-    IMEM_CHECK(cuda_status(cudaStreamWaitEvent(c.side, c.ev_pe_fork, 0)));
-    const cudaError_t me = imem::launch_memory_update(c, batch, L, K, V, evicted, n_ev, mem_chunk,
-                                                      M, bstab, part, nullptr, nullptr, nullptr,
-                                                      c.side);
-    // recorded even after a failed launch, so that the wait below never
-    // refers to an event of an earlier range
-    IMEM_CHECK(cuda_status(cudaEventRecord(c.ev_pe_done, c.side)));
-    h->c.pe_pending = true;
-    IMEM_CHECK(cuda_status(me));
+    IMEM_CHECK(cuda_status(cudaEventRecord(cm.ev_pe_fork, st)));
+    IMEM_CHECK(cuda_status(cudaStreamWaitEvent(cm.side, cm.ev_pe_fork, 0)));
+    cudaError_t se = imem::launch_evict_chunk(c, batch, B, Lc, n_R, q_begin, C, eb, retained,
+                                              evicted, cm.side);
+    // both events are recorded even after a failed launch, so that no later
+    // wait refers to an event of an earlier range
+    const cudaError_t e1 = cudaEventRecord(cm.ev_pe_compact, cm.side);
+    if (se == cudaSuccess)
+      se = imem::launch_memory_update(c, batch, L, K, V, evicted, n_ev, mem_chunk, M, bstab, part,
+                                      nullptr, nullptr, nullptr, cm.side);
+    const cudaError_t e2 = cudaEventRecord(cm.ev_pe_done, cm.side);
+    cm.pe_pending = true;
+    cm.pe_compact_pending = true;
+    cm.pe_parity = 1 - p;
+    IMEM_CHECK(cuda_status(se));
+    IMEM_CHECK(cuda_status(e1));
+    IMEM_CHECK(cuda_status(e2));
   } else {
-    IMEM_CHECK(cuda_status(imem::launch_append_positions(batch, B, n_R, q_begin, C, retained, st)));
+    IMEM_CHECK(wait_pending(cm, st));
+    IMEM_CHECK(cuda_status(imem::launch_append_positions(batch, B, n_R, q_begin, C, retained,
+                                                         eb.pos_c, st)));
   }
   if (finalize) {
+    IMEM_CHECK(wait_pending(cm, st));
     IMEM_CHECK(cuda_status(imem::launch_gather(c, batch, L, B < L ? B : L, retained, B, K, V,
                                                K_ret, V_ret, cap, st)));
-    IMEM_CHECK(wait_pending(h->c, st));
   }
   return IMEM_OK;
 }

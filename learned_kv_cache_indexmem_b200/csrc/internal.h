@@ -31,12 +31,15 @@ struct Ctx {
   // (forked from and joined back into the caller's stream by events)
   cudaStream_t side;
   cudaEvent_t ev_fork, ev_join;
-  // pre-eviction: a range's memory update runs on `side`, after ev_pe_fork
-  // of the caller's stream, beside the next range's prologue and scoring;
-  // ev_pe_done marks its end, and while pe_pending is set every call on the
+  // pre-eviction: a range's selection, compaction and memory update run on
+  // `side`, after ev_pe_fork of the caller's stream, beside the next range's
+  // prologue (and the memory update beside its scoring too); ev_pe_compact
+  // and ev_pe_done mark their ends. While pe_pending is set every call on the
   // context makes its stream wait for ev_pe_done before it enqueues work
-  cudaEvent_t ev_pe_fork, ev_pe_done;
-  bool pe_pending;
+  cudaEvent_t ev_pe_fork, ev_pe_compact, ev_pe_done;
+  bool pe_pending;           // the last range's work on `side` may still run
+  bool pe_compact_pending;   // ... and its selection and compaction too
+  int pe_parity;             // candidate buffer of the next range (0 or 1)
 };
 
 // Indexer rows in the workspace: d_I features padded to 64 bf16 (128 bytes).
@@ -101,26 +104,30 @@ cudaError_t launch_select_compact(const Ctx& c, int batch, int L, int B, const f
                                   cudaStream_t st);
 
 // Pre-eviction during chunked prefill: one query range [q0, q0 + C) over the
-// candidates = n_R retained tokens + the range's C tokens, laid out with a
-// row stride Lc in the candidate buffers (indexer keys kh_c [b, Lc, 64],
-// importances I_c [b, Lc]). Selects the B most important candidates,
-// compacts them to rows [0, B) (positions to `retained` [b, B]) and writes the
-// evicted positions, ascending, to `evicted` [b, n - B] (n = n_R + C > B).
+// candidates = n_R retained tokens + the range's C tokens, rows [0, n) of one
+// of two candidate buffers (indexer keys [b, Lc, 64], importances [b, Lc], row
+// stride Lc; positions of the retained rows [b, B]). Selects the B most
+// important candidates and writes them, in position order, to rows [0, B) of
+// the other buffer (keys, importances, positions) and their positions to
+// `retained` [b, B]; the evicted positions, ascending, to `evicted`
+// [b, n - B] (n = n_R + C > B). Reads nothing it writes.
 struct EvictBuffers {
-  __nv_bfloat16* kh_c;   // [b, Lc, kIdxPad]
-  float* I_c;            // [b, Lc]
-  __nv_bfloat16* kh_tmp; // [b, B, kIdxPad]
-  float* I_tmp;          // [b, B]
-  int32_t* pos_tmp;      // [b, B]
+  __nv_bfloat16* kh_c;   // this range's candidates: keys [b, Lc, kIdxPad]
+  float* I_c;            // importances [b, Lc]
+  int32_t* pos_c;        // positions of the retained rows [b, B]
+  __nv_bfloat16* kh_n;   // the other buffer: the rows retained after this range
+  float* I_n;
+  int32_t* pos_n;
   int32_t* idx_r;        // [b, B]
   int32_t* idx_e;        // [b, Lc]
 };
 cudaError_t launch_evict_chunk(const Ctx& c, int batch, int B, int Lc, int n_R, int q0, int C,
                                const EvictBuffers& w, int32_t* retained, int32_t* evicted,
                                cudaStream_t st);
-// Appends positions q0..q0+C-1 at rows [n_R, n_R + C) of `retained` (stride B).
+// Appends positions q0..q0+C-1 at rows [n_R, n_R + C) of `retained` and of
+// `pos` (both [b, B]).
 cudaError_t launch_append_positions(int batch, int B, int n_R, int q0, int C, int32_t* retained,
-                                    cudaStream_t st);
+                                    int32_t* pos, cudaStream_t st);
 // Decode-time online eviction (online.cu).
 int online_cluster_ctas(int B);
 cudaError_t launch_online_init(const Ctx& c, int batch, int L, int B, int cap,

@@ -385,24 +385,29 @@ __device__ __forceinline__ int cand_pos(int ci, int n_R, int q0, const int32_t* 
 
 constexpr int kRowsPerCompactCta = 32;   // 8 threads (16-byte chunks of a 128-byte key) per row
 
-// Gathers the selected candidates (idx_r) into the temporaries and writes the
-// evicted candidates' positions (idx_e, ascending) to `evicted`.
+// Writes the selected candidates (idx_r), in position order, to rows [0, B)
+// of the other candidate buffer and their positions to `retained`, and the
+// evicted candidates' positions (idx_e, ascending) to `evicted`. It reads
+// only the current buffer, so no row is overwritten before it is read.
 __global__ void __launch_bounds__(256)
 evict_compact_kernel(const int32_t* __restrict__ idx_r, const int32_t* __restrict__ idx_e, int B,
-                     int n_ev, int n_R, int q0, int Lc, const int32_t* __restrict__ retained,
+                     int n_ev, int n_R, int q0, int Lc, const int32_t* __restrict__ pos_c,
                      const __nv_bfloat16* __restrict__ kh_c, const float* __restrict__ I_c,
-                     int32_t* __restrict__ pos_tmp, __nv_bfloat16* __restrict__ kh_tmp,
-                     float* __restrict__ I_tmp, int32_t* __restrict__ evicted) {
+                     int32_t* __restrict__ pos_n, __nv_bfloat16* __restrict__ kh_n,
+                     float* __restrict__ I_n, int32_t* __restrict__ retained,
+                     int32_t* __restrict__ evicted) {
   const int bi = blockIdx.y;
   const int j = blockIdx.x * kRowsPerCompactCta + threadIdx.x / 8, c = threadIdx.x % 8;
-  const int32_t* ret_b = retained + (size_t)bi * B;
+  const int32_t* ret_b = pos_c + (size_t)bi * B;
   if (j < B) {
     const int ci = idx_r[(size_t)bi * B + j];
     const uint4* src = reinterpret_cast<const uint4*>(kh_c + ((size_t)bi * Lc + ci) * kIdxPad);
-    reinterpret_cast<uint4*>(kh_tmp + ((size_t)bi * B + j) * kIdxPad)[c] = src[c];
+    reinterpret_cast<uint4*>(kh_n + ((size_t)bi * Lc + j) * kIdxPad)[c] = src[c];
     if (c == 0) {
-      pos_tmp[(size_t)bi * B + j] = cand_pos(ci, n_R, q0, ret_b);
-      I_tmp[(size_t)bi * B + j] = I_c[(size_t)bi * Lc + ci];
+      const int p = cand_pos(ci, n_R, q0, ret_b);
+      pos_n[(size_t)bi * B + j] = p;
+      retained[(size_t)bi * B + j] = p;
+      I_n[(size_t)bi * Lc + j] = I_c[(size_t)bi * Lc + ci];
     }
   } else if (j < B + n_ev && c == 0) {
     const int e = j - B;
@@ -410,27 +415,14 @@ evict_compact_kernel(const int32_t* __restrict__ idx_r, const int32_t* __restric
   }
 }
 
-// Rows [0, B) of the candidate buffers and `retained` from the temporaries.
-__global__ void __launch_bounds__(256)
-evict_copyback_kernel(int B, int Lc, const int32_t* __restrict__ pos_tmp,
-                      const __nv_bfloat16* __restrict__ kh_tmp, const float* __restrict__ I_tmp,
-                      int32_t* __restrict__ retained, __nv_bfloat16* __restrict__ kh_c,
-                      float* __restrict__ I_c) {
-  const int bi = blockIdx.y;
-  const int j = blockIdx.x * kRowsPerCompactCta + threadIdx.x / 8, c = threadIdx.x % 8;
-  if (j >= B) return;
-  reinterpret_cast<uint4*>(kh_c + ((size_t)bi * Lc + j) * kIdxPad)[c] =
-      reinterpret_cast<const uint4*>(kh_tmp + ((size_t)bi * B + j) * kIdxPad)[c];
-  if (c == 0) {
-    retained[(size_t)bi * B + j] = pos_tmp[(size_t)bi * B + j];
-    I_c[(size_t)bi * Lc + j] = I_tmp[(size_t)bi * B + j];
-  }
-}
-
-__global__ void append_positions_kernel(int B, int n_R, int q0, int C, int32_t* __restrict__ retained) {
+__global__ void append_positions_kernel(int B, int n_R, int q0, int C, int32_t* __restrict__ retained,
+                                        int32_t* __restrict__ pos) {
   const int bi = blockIdx.y;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < C) retained[(size_t)bi * B + n_R + i] = q0 + i;
+  if (i < C) {
+    retained[(size_t)bi * B + n_R + i] = q0 + i;
+    pos[(size_t)bi * B + n_R + i] = q0 + i;
+  }
 }
 
 // Selection of the B largest of L importances per sequence (stride between
@@ -478,21 +470,17 @@ cudaError_t launch_evict_chunk(const Ctx& c, int batch, int B, int Lc, int n_R, 
   cudaError_t e = launch_select(batch, w.I_c, n, Lc, B, w.idx_r, w.idx_e, st);
   if (e != cudaSuccess) return e;
   dim3 g1((B + n_ev + kRowsPerCompactCta - 1) / kRowsPerCompactCta, batch);
-  evict_compact_kernel<<<g1, 256, 0, st>>>(w.idx_r, w.idx_e, B, n_ev, n_R, q0, Lc, retained,
-                                           w.kh_c, w.I_c, w.pos_tmp, w.kh_tmp, w.I_tmp, evicted);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  dim3 g2((B + kRowsPerCompactCta - 1) / kRowsPerCompactCta, batch);
-  evict_copyback_kernel<<<g2, 256, 0, st>>>(B, Lc, w.pos_tmp, w.kh_tmp, w.I_tmp, retained, w.kh_c,
-                                            w.I_c);
+  evict_compact_kernel<<<g1, 256, 0, st>>>(w.idx_r, w.idx_e, B, n_ev, n_R, q0, Lc, w.pos_c,
+                                           w.kh_c, w.I_c, w.pos_n, w.kh_n, w.I_n, retained,
+                                           evicted);
   return cudaGetLastError();
 }
 
 cudaError_t launch_append_positions(int batch, int B, int n_R, int q0, int C, int32_t* retained,
-                                    cudaStream_t st) {
+                                    int32_t* pos, cudaStream_t st) {
   if (C <= 0) return cudaSuccess;
   dim3 g((C + 255) / 256, batch);
-  append_positions_kernel<<<g, 256, 0, st>>>(B, n_R, q0, C, retained);
+  append_positions_kernel<<<g, 256, 0, st>>>(B, n_R, q0, C, retained, pos);
   return cudaGetLastError();
 }
 

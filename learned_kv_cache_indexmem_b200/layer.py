@@ -153,6 +153,7 @@ class IndexMemLayer:
                                    st.idx_retained, ev, cand, st.M, st.bstab, mem_chunk,
                                    q1 == L, st.K_ret, st.V_ret, st.K_ret.shape[1], ws, stream)
             if record:
+                B_.join(self.ctx, stream)   # the range's selection runs on a second stream
                 n = min(B, q0) + (q1 - q0)
                 n_ev = max(0, n - B)
                 recs.append({"range": (q0, q1), "I": cand[:, :n].clone(),
