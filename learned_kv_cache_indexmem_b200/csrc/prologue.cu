@@ -56,6 +56,10 @@ struct ProSmem {
   static constexpr int TOTAL = NST * (kStageA + kStageB) + BARS + SLOT + GAM + 1024;
 };
 
+__device__ __forceinline__ void add4(float* a, float4 v) {
+  a[0] += v.x; a[1] += v.y; a[2] += v.z; a[3] += v.w;
+}
+
 __device__ __forceinline__ uint32_t tmem_ld1(uint32_t taddr) {
   uint32_t r;
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\ntcgen05.wait::ld.sync.aligned;\n"
@@ -260,15 +264,18 @@ prologue_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
         if (lane == 0) tc::mbar_arrive(d1_empty);
         // 3. the other CTA's partial sums
         if (!tc::mbar_wait_cluster(rx_full, n_rx & 1)) { ok = false; break; }
+        // 16-byte reads: a row stride of 4 mod 8 floats keeps a quarter warp's
+        // 16-byte accesses on distinct banks
+        const float4* s4 = reinterpret_cast<const float4*>(srow);
         if (rank == 0) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c < dI) acc[c] += srow[c];
+          for (int c = 0; c < 64; c += 4)
+            if (c < dI) add4(acc + c, s4[c / 4]);
 #pragma unroll
-          for (int h = 0; h < kPairHeads; ++h) lg[h] += srow[dI + h];
+          for (int h = 0; h < kPairHeads; h += 4) add4(lg + h, s4[(dI + h) / 4]);
         } else {
 #pragma unroll
-          for (int h = 0; h < kPairHeads; ++h) lg[h] += srow[h];
+          for (int h = 0; h < kPairHeads; h += 4) add4(lg + h, s4[h / 4]);
         }
         tc::mbar_arrive_remote(tx_rem);
         ++n_rx;
@@ -339,9 +346,10 @@ prologue_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_const
           write_q = false;
         } else {
           if (!tc::mbar_wait_cluster(rx_full, n_rx & 1)) { ok = false; break; }
+          const float4* s4 = reinterpret_cast<const float4*>(srow);
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c < dI) acc[c] += srow[c];
+          for (int c = 0; c < 64; c += 4)
+            if (c < dI) add4(acc + c, s4[c / 4]);
           tc::mbar_arrive_remote(tx_rem);
           ++n_rx;
         }
