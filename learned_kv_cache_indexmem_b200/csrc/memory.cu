@@ -306,7 +306,9 @@ memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t
     tc::mma_commit(done);
   }
 
-  // ---------------- epilogue: warps 0-3 read [S | s] rows from TMEM
+  // ---------------- epilogue: warps 0-3 read [S | s] rows from TMEM and store
+  // them transposed (column c of the run's sum = D consecutive floats), so
+  // that a warp's stores cover 128 contiguous bytes
   pdl_launch();   // the finalize may start staging W_phi (it waits for this grid)
   if (warp < 4) {
     const int row = warp * 32 + lane;   // feature index of k (TMEM lane)
@@ -324,12 +326,12 @@ memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int col = c0 + e;
-            if (col <= D) out[(size_t)row * (D + 1) + col] = v[e];
+            if (col <= D) out[(size_t)col * D + row] = v[e];
           }
         }
       }
     } else if (row < D) {
-      for (int col = 0; col <= D; ++col) out[(size_t)row * (D + 1) + col] = 0.f;
+      for (int col = 0; col <= D; ++col) out[(size_t)col * D + row] = 0.f;
     }
   }
   tc::fence_before();
@@ -416,11 +418,11 @@ memory_finalize_kernel(const float* __restrict__ partials, int G, int tpg, int n
     float v[4][IPT];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const float* pg = p + (size_t)(g0 + u) * D * (D + 1) + col0;
+      const float* pg = p + (size_t)(g0 + u) * D * (D + 1) + (size_t)col0 * D;
 #pragma unroll
       for (int k = 0; k < IPT; ++k) {
-        const int i = tid + k * 256;
-        v[u][k] = (g0 + u < G && i < D * ncols) ? __ldcg(&pg[(i / ncols) * (D + 1) + i % ncols]) : 0.f;
+        const int i = tid + k * 256;   // column i / D, row i % D: a warp reads 128 bytes
+        v[u][k] = (g0 + u < G && i < D * ncols) ? __ldcg(&pg[i]) : 0.f;
       }
     }
 #pragma unroll
@@ -433,7 +435,7 @@ memory_finalize_kernel(const float* __restrict__ partials, int G, int tpg, int n
 #pragma unroll
   for (int k = 0; k < IPT; ++k) {
     const int i = tid + k * 256;
-    if (i < D * ncols) sS[(i / ncols) * 16 + i % ncols] = acc[k];
+    if (i < D * ncols) sS[(i % D) * 16 + i / D] = acc[k];
   }
   __syncthreads();
   // out[ri][c] = sum_dk W_phi[ri][dk] S[dk][c]: a thread takes two rows
@@ -707,7 +709,9 @@ memory_bf16_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __r
     tc::mma_commit(done);
   }
 
-  // ---------------- epilogue: warps 0-3 read [S | s] rows from TMEM
+  // ---------------- epilogue: warps 0-3 read [S | s] rows from TMEM and store
+  // them transposed (column c of the run's sum = D consecutive floats), so
+  // that a warp's stores cover 128 contiguous bytes
   pdl_launch();
   if (warp < 4) {
     const int row = warp * 32 + lane;   // feature index of k (TMEM lane)
@@ -724,12 +728,12 @@ memory_bf16_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __r
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int col = c0 + e;
-            if (col <= D) out[(size_t)row * (D + 1) + col] = v[e];
+            if (col <= D) out[(size_t)col * D + row] = v[e];
           }
         }
       }
     } else if (row < D) {
-      for (int col = 0; col <= D; ++col) out[(size_t)row * (D + 1) + col] = 0.f;
+      for (int col = 0; col <= D; ++col) out[(size_t)col * D + row] = 0.f;
     }
   }
   tc::fence_before();
