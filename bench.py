@@ -597,7 +597,7 @@ def online_decode(job, steps=64, reps=3):
         del g
     lay.sync(job.stream)
     res["us_per_step_online"] = best
-    res["launches_per_step_online"] = 4   # features, score (second stream); attention, evict
+    res["launches_per_step_online"] = 3   # features (second stream); attention, score and evict
     res["steps"] = steps
     res["cache_rows"] = B
     return res

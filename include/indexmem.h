@@ -406,19 +406,19 @@ imem_status imem_prefill_evict_chunk(imem_ctx* ctx, int batch, int L, int B, int
  *      by, so that K_ret/V_ret/khat_ret/I_ret/pos_ret[:, :B + 1] are the
  *      B + 1 candidates of the step; cache_len returns to B; next_pos
  *      advances.
- * Streams: step 2 and the choice of step 3 need neither the cache rows nor
- * the memory, so they are computed on a second stream owned by the context
- * (created by imem_online_init or the first step, which therefore belong
- * before any stream capture; no device memory),
- * forked from `stream` and joined back into it by events before the memory
- * update of step 3;
- * under stream capture this becomes two parallel branches of the graph.
+ * Streams: the new token's features (step 2 before the importances) need
+ * neither the cache rows nor the memory, so they are computed on a second
+ * stream owned by the context (created by imem_online_init or the first
+ * step, which therefore belong before any stream capture; no device
+ * memory), forked from `stream` and joined back into it by events before
+ * the importances, the choice and the memory update (one kernel); under
+ * stream capture this becomes two parallel branches of the graph.
  * Ordering: step 4 clears the workspace's decode tag of the sequence (slot e
  * and the memory changed after the attention step), so the next decode step
  * uses nothing it loaded before its launch-dependency wait.
  * imem_online_init does not write the cache state and leaves the tag as it is.
- * Errors: as imem_decode; UNSUPPORTED for the moment readout; nothing is
- * enqueued if an argument is invalid. */
+ * Errors: as imem_decode; UNSUPPORTED for the moment readout or more than
+ * 16 KV heads; nothing is enqueued if an argument is invalid. */
 imem_status imem_online_init(imem_ctx* ctx, int batch, int L, int B, const float* running_max,
                              const int32_t* idx_retained, const void* workspace, void* khat_ret,
                              float* I_ret, int32_t* pos_ret, int32_t* next_pos, int cap,

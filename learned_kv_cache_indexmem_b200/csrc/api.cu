@@ -35,8 +35,6 @@ Workspace workspace_layout(const Ctx& c, int batch, int L) {
   off = align_up(off + (size_t)batch * c.cfg.n_q_heads * c.cfg.idx_dim * sizeof(float), 256);
   w.on_kpart_off = off;
   off = align_up(off + (size_t)batch * c.cfg.idx_dim * sizeof(float), 256);
-  w.on_choice_off = off;
-  off = align_up(off + (size_t)batch * sizeof(OnlineChoice), 256);
   w.dec_part_off = off;                       // (unused: decode merges in shared memory)
   // memory partials: one d x (d+1) sum [S | s] per run of evicted tokens
   const size_t runs = memory_runs_bound((int)units, L, c.num_sms);
@@ -157,7 +155,6 @@ imem_status online_streams(Ctx& c) {
     return IMEM_ERR_CUDA;
   return IMEM_OK;
 }
-
 
 // The pre-eviction's second stream and its events, created on first use.
 imem_status prefill_streams(Ctx& c) {
@@ -373,6 +370,7 @@ imem_status imem_indexer_features(imem_ctx* h, int batch, int L, const void* X, 
   IMEM_CHECK(check_ptr(workspace));
   IMEM_CHECK(check_device(c));
   IMEM_CHECK(wait_pending(h->c, (cudaStream_t)stream));
+  IMEM_CHECK(online_streams(h->c));
   const imem::Workspace ws = imem::workspace_layout(c, batch, L);
   char* wsb = (char*)workspace;
   return cuda_status(imem::launch_prologue(c, batch, L, X, Q, q_begin, q_end,
@@ -391,6 +389,7 @@ imem_status imem_indexer_score(imem_ctx* h, int batch, int L, float* running_max
   IMEM_CHECK(check_ptr(workspace));
   IMEM_CHECK(check_device(c));
   IMEM_CHECK(wait_pending(h->c, (cudaStream_t)stream));
+  IMEM_CHECK(online_streams(h->c));
   const imem::Workspace ws = imem::workspace_layout(c, batch, L);
   char* wsb = (char*)workspace;
   return cuda_status(imem::launch_scoring(c, batch, L, (const __nv_bfloat16*)(wsb + ws.qt_off),
@@ -441,6 +440,7 @@ imem_status imem_update_memory(imem_ctx* h, int batch, int L, const void* K, con
   IMEM_CHECK(check_ptr(workspace));
   IMEM_CHECK(check_device(c));
   IMEM_CHECK(wait_pending(h->c, (cudaStream_t)stream));
+  IMEM_CHECK(online_streams(h->c));
   const imem::Workspace ws = imem::workspace_layout(c, batch, L);
   float* part = (float*)((char*)workspace + ws.mem_part_off);
   IMEM_CHECK(cuda_status(imem::clear_decode_tags(c, batch, workspace, (cudaStream_t)stream)));
@@ -469,6 +469,7 @@ imem_status imem_update_moments(imem_ctx* h, int batch, int L, const void* K, co
   IMEM_CHECK(check_ptr(workspace));
   IMEM_CHECK(check_device(c));
   IMEM_CHECK(wait_pending(h->c, (cudaStream_t)stream));
+  IMEM_CHECK(online_streams(h->c));
   const imem::Workspace ws = imem::workspace_layout(c, batch, L);
   float* part = (float*)((char*)workspace + ws.mem_part_off);
   float* svp = (float*)((char*)workspace + ws.sv_part_off);
@@ -693,6 +694,7 @@ imem_status imem_decode_online(imem_ctx* h, int batch, int B, const void* x_new,
   if (!h) return IMEM_ERR_INVALID_ARG;
   const Ctx& c = h->c;
   if (c.cfg.readout != IMEM_READOUT_GATED) return IMEM_ERR_UNSUPPORTED;
+  if (c.cfg.n_kv_heads > imem::kOnlineMaxCluster) return IMEM_ERR_UNSUPPORTED;
   if (batch < 1 || B < 1 || cap < B + 1) return IMEM_ERR_SHAPE;
   IMEM_CHECK(check_ptr(x_new));
   IMEM_CHECK(check_ptr(khat_ret));
@@ -719,15 +721,11 @@ imem_status imem_decode_online(imem_ctx* h, int batch, int B, const void* x_new,
   char* wsb = (char*)workspace;
   float* qpart = (float*)(wsb + ws.on_qpart_off);
   float* kpart = (float*)(wsb + ws.on_kpart_off);
-  void* choice = wsb + ws.on_choice_off;
-  // the new token's indexer features and the importance update with the
-  // choice of the token to evict need neither the cache rows nor the memory:
+  // the new token's indexer features need neither the cache nor the memory:
   // they run on the context's second stream beside the attention step
   IMEM_CHECK(cuda_status(cudaEventRecord(c.ev_fork, st)));
   IMEM_CHECK(cuda_status(cudaStreamWaitEvent(c.side, c.ev_fork, 0)));
   IMEM_CHECK(cuda_status(imem::launch_online_features(c, batch, x_new, q, qpart, kpart, c.side)));
-  IMEM_CHECK(cuda_status(imem::launch_online_score(c, batch, B, cap, qpart, kpart, khat_ret, I_ret,
-                                                   pos_ret, next_pos, choice, c.side)));
   IMEM_CHECK(cuda_status(cudaEventRecord(c.ev_join, c.side)));
   // the attention step with the memory before this step's eviction (it
   // validates the remaining arguments and appends the new token at slot B)
@@ -736,9 +734,12 @@ imem_status imem_decode_online(imem_ctx* h, int batch, int B, const void* x_new,
   // join first, so that the second stream's work is always waited for
   IMEM_CHECK(cuda_status(cudaStreamWaitEvent(st, c.ev_join, 0)));
   IMEM_CHECK(ds);
-  return cuda_status(imem::launch_online_evict(c, batch, B, cap, choice, khat_ret, I_ret, pos_ret,
-                                               next_pos, K_ret, V_ret, cache_len, M, bstab,
-                                               evicted, (int*)(wsb + ws.dec_tag_off), st));
+  // the importances, the token that leaves, the memory update and the slot
+  // swap: one kernel after both branches
+  return cuda_status(imem::launch_online_score_evict(c, batch, B, cap, qpart, kpart, khat_ret,
+                                                     I_ret, pos_ret, next_pos, K_ret, V_ret,
+                                                     cache_len, M, bstab, evicted,
+                                                     (int*)(wsb + ws.dec_tag_off), st));
 }
 
 imem_status imem_selftest_wait(imem_ctx* h, long long limit_cycles, void* stream) {

@@ -27,8 +27,9 @@ struct Ctx {
   int* err;             // device error word
   int num_sms;          // streaming multiprocessors of the device
   void* encode_tiled;   // driver entry point cuTensorMapEncodeTiled
-  // online eviction: a second stream for the new token's indexer features
-  // (forked from and joined back into the caller's stream by events)
+  // a second stream (created on first use): online eviction's new-token
+  // features (forked from and joined back into the caller's stream by
+  // events) and the pre-eviction's range work
   cudaStream_t side;
   cudaEvent_t ev_fork, ev_join;
   // pre-eviction: a range's selection, compaction and memory update run on
@@ -57,7 +58,7 @@ bool make_tmap_bf16(const Ctx& c, CUtensorMap* map, const void* base, uint64_t w
                     uint64_t rows, uint32_t box_rows);
 
 // Layout of the caller's workspace for (batch, L).
-constexpr int kOnlineMaxCluster = 8;   // CTAs per sequence of the online score-and-evict cluster
+constexpr int kOnlineMaxCluster = 16;  // KV heads (= CTAs of the online score-and-evict cluster), max
 
 struct Workspace {
   size_t qt_off, kh_off;        // indexer q~ and k^ (bf16 [b, L, kIdxPad])
@@ -65,7 +66,7 @@ struct Workspace {
   size_t dec_part_off;          // decode split partials
   size_t dec_cnt_off;           // decode counters (int), zero between calls
   size_t dec_tag_off;           // decode tags (int): right after the counters
-  size_t on_qpart_off, on_kpart_off, on_choice_off;   // online eviction: feature partials, choice
+  size_t on_qpart_off, on_kpart_off;   // online eviction: the new token's feature partials
   size_t mem_part_off;          // memory-update partials
   size_t sv_part_off;           // value-sum partials of the moment statistics
   size_t total;
@@ -129,31 +130,17 @@ cudaError_t launch_evict_chunk(const Ctx& c, int batch, int B, int Lc, int n_R, 
 cudaError_t launch_append_positions(int batch, int B, int n_R, int q0, int C, int32_t* retained,
                                     int32_t* pos, cudaStream_t st);
 // Decode-time online eviction (online.cu).
-int online_cluster_ctas(int B);
 cudaError_t launch_online_init(const Ctx& c, int batch, int L, int B, int cap,
                                const float* running_max, const int32_t* idx_r,
                                const __nv_bfloat16* kh, __nv_bfloat16* khat_ret, float* I_ret,
                                int32_t* pos_ret, int32_t* next_pos, cudaStream_t st);
 cudaError_t launch_online_features(const Ctx& c, int batch, const void* x, const void* q,
                                    float* qpart, float* kpart, cudaStream_t st);
-// The token chosen by the online score kernel, per sequence (workspace).
-struct __align__(16) OnlineChoice {
-  int slot;            // cache slot of the token that leaves (B: the new token)
-  int pos;             // its position
-  float I_e;           // its importance (the one it was chosen by)
-  float I_new;         // the new token's importance
-  int pos_new;         // the new token's position
-  int pad[3];
-  __nv_bfloat16 khat_new[kIdxPad];   // the new token's indexer key
-};
-cudaError_t launch_online_score(const Ctx& c, int batch, int B, int cap, const float* qpart,
-                                const float* kpart, const void* khat_ret, float* I_ret,
-                                const int32_t* pos_ret, const int32_t* next_pos, void* choice,
-                                cudaStream_t st);
-cudaError_t launch_online_evict(const Ctx& c, int batch, int B, int cap, const void* choice,
-                                void* khat_ret, float* I_ret, int32_t* pos_ret, int32_t* next_pos,
-                                void* K_ret, void* V_ret, int32_t* cache_len, float* M,
-                                float* bstab, int32_t* evicted, int* dec_tag, cudaStream_t st);
+cudaError_t launch_online_score_evict(const Ctx& c, int batch, int B, int cap, const float* qpart,
+                                      const float* kpart, void* khat_ret, float* I_ret,
+                                      int32_t* pos_ret, int32_t* next_pos, void* K_ret, void* V_ret,
+                                      int32_t* cache_len, float* M, float* bstab, int32_t* evicted,
+                                      int* dec_tag, cudaStream_t st);
 
 // A kernel whose bounded wait runs out after `limit` cycles (failure-path test).
 cudaError_t launch_wait_selftest(const Ctx& c, long long limit, cudaStream_t st);

@@ -8,28 +8,25 @@
 //
 // The cache holds B tokens in slots [0, B) in any order, each with its
 // indexer key k^ (bf16), importance I and position. Per decode step:
-//   features  the new token's indexer query q~ = sum_h g_h q^_h / sqrt(dI)
-//             and key k^ (per-head projections of the attention query, gate
-//             logits and key from the hidden state, RMS norms): Hq + 8 CTAs
-//             per sequence, one GEMV each, partials in the workspace. It
-//             needs neither the cache nor the memory, so the C ABI runs it
-//             on a second stream next to the attention step (which appends
-//             the new token at slot B);
-//   score     (second stream, after the features) one thread-block cluster
-//             per sequence: I_t <- max(I_t, q~ . k^_t) for the cached tokens,
-//             the new token's I = q~ . k^_new; the least important of the
-//             B + 1 (ties: the higher position) by per-CTA minima of a packed
-//             (ordered importance, inverted position) key exchanged over
-//             distributed shared memory; the choice to the workspace. It
-//             touches neither the rows, the memory nor slot B, so it runs
-//             beside the attention step as well;
-//   evict     (after both branches) per KV head phi = W_phi k_e,
-//             M <- lambda M + phi v_e^T, b <- lambda b + phi; the new token
-//             and the evicted one swap slots (row, indexer key, importance,
-//             position), so slot B keeps the token that left with the
-//             importance it was chosen by; cache_len returns to B and the
-//             workspace's decode tag of the sequence is cleared (rows of
-//             slot e and the memory changed after the attention step).
+//   features     the new token's indexer query shares and key rows (per-head
+//                projections of the attention query, gate logits and key
+//                from the hidden state): Hq + 8 CTAs per sequence, one GEMV
+//                each, partials in the workspace. It needs neither the cache
+//                nor the memory, so the C ABI runs it on a second stream next
+//                to the attention step (which appends the new token at slot B);
+//   score+evict  (after both branches) one thread-block cluster per sequence,
+//                a CTA per KV head: q~ and k^ from the partials (RMS norm),
+//                I_t <- max(I_t, q~ . k^_t) for the cached tokens, the new
+//                token's I = q~ . k^_new; the least important of the B + 1
+//                (ties: the higher position) by per-CTA minima of a packed
+//                (ordered importance, inverted position) key exchanged over
+//                distributed shared memory; then per KV head phi = W_phi k_e,
+//                M <- lambda M + phi v_e^T, b <- lambda b + phi; the new token
+//                and the evicted one swap slots (row, indexer key,
+//                importance, position), so slot B keeps the token that left
+//                with the importance it was chosen by; cache_len returns to B
+//                and the workspace's decode tag of the sequence is cleared
+//                (rows of slot e and the memory changed after the attention).
 // q~ and k^ are rounded to bf16 before their dot products, as in prefill.
 #include "common.cuh"
 #include "internal.h"
@@ -187,36 +184,56 @@ online_features_kernel(const T* __restrict__ x, const T* __restrict__ q, const T
   }
 }
 
-// ---- importances and the token to evict (second stream) ----------------------
-// One thread-block cluster of nct CTAs per sequence. Each CTA takes a
-// contiguous block of the B + 1 candidate rows (slot B: the new token):
-// I_t <- max(I_t, q~ . k^_t) for the cached tokens, the new token's I =
-// q~ . k^_new, and its block's least important candidate as a packed key
-// (ordered importance << 32 | ~position: the minimum is the least important,
-// ties to the higher position). The CTAs exchange their keys through
-// distributed shared memory; after one cluster barrier CTA 0 writes the
-// choice (slot, position, importance) and the new token's importance and
-// indexer key to the workspace. Nothing here reads or writes the cache rows,
-// the memory or slot B, so it runs beside the attention step.
+// ---- importances, the token to evict, memory update and slot swap ------------
+// After the attention step and the features (the join of the two streams):
+// one thread-block cluster of Hkv CTAs per sequence.
+// Phase 1 (every CTA): q~ (the sum of the heads' shares) and k^ (RMS norm),
+// both rounded to bf16; for its block of the B + 1 candidate rows (slot B:
+// the new token, scored by its own query) I_t <- max(I_t, q~ . k^_t), and the
+// block's least important candidate as a packed key (ordered importance << 32
+// | ~position: the minimum is the least important, ties to the higher
+// position). Every CTA writes its candidate into every CTA's table
+// (distributed shared memory); after a cluster barrier each takes the same
+// minimum: the token e that leaves (the new token if no importance is
+// ordered, e.g. NaN).
+// Phase 2 (CTA = KV head kh): phi = W_phi k_e, M <- lambda M + phi v_e^T,
+// b <- lambda b + phi, and the rows of slot e and slot B (the new token,
+// appended by the attention step) swap for this head; CTA 0 also swaps the
+// indexer keys, importances and positions (slot e takes the new token, slot
+// B keeps the evicted one with the importance it was chosen by), writes the
+// evicted position, returns cache_len to B, advances next_pos and clears the
+// decode tag (slot e and the memory changed after the attention step).
 __device__ __forceinline__ float order_key_inv(uint32_t o) {
   return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
 }
 
+template <typename T>
 __global__ void __launch_bounds__(kOnThreads)
-online_score_kernel(int B, int cap, int Hq, int dI, int rows_per_cta,
-                    const float* __restrict__ qpart, const float* __restrict__ kpart,
-                    const __nv_bfloat16* __restrict__ khat_ret, float* __restrict__ I_ret,
-                    const int32_t* __restrict__ pos_ret, const int32_t* __restrict__ next_pos,
-                    OnlineChoice* __restrict__ choice) {
+online_score_evict_kernel(int B, int cap, int Hq, int Hkv, int D, int r, int dI, int rows_per_cta,
+                          float lambda, const float* __restrict__ qpart,
+                          const float* __restrict__ kpart, const float* __restrict__ W_phi,
+                          T* __restrict__ K_ret, T* __restrict__ V_ret,
+                          __nv_bfloat16* __restrict__ khat_ret, float* __restrict__ I_ret,
+                          int32_t* __restrict__ pos_ret, int32_t* __restrict__ next_pos,
+                          int32_t* __restrict__ cache_len, float* __restrict__ M,
+                          float* __restrict__ bstab, int32_t* __restrict__ evicted,
+                          int* __restrict__ dec_tag) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ float osm[];
+  float* sk = osm;          // [D] the evicted token's key, this CTA's head
+  float* sv = sk + D;       // [D] its value
+  float* sphi = sv + D;     // [r]
   __shared__ float s_qt[64], s_kn[64];
+  __shared__ float s_hsum[4][64];
   __shared__ float red[kOnThreads / 32];
   __shared__ unsigned long long s_key[kOnThreads / 32];
   __shared__ int s_slot[kOnThreads / 32];
   __shared__ unsigned long long s_ckey[kOnlineMaxCluster];   // one per CTA of the cluster
   __shared__ int s_cslot[kOnlineMaxCluster];
   __shared__ float s_Inew;
+  __shared__ int s_e, s_epos;
+  __shared__ float s_Ie;
   const int bi = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nct = gridDim.x, rank = blockIdx.x;
   // phase 0 of the cluster barrier: "this CTA is running" (its shared memory
@@ -226,7 +243,6 @@ online_score_kernel(int B, int cap, int Hq, int dI, int rows_per_cta,
   pdl_launch();
   // q~ (sum over heads: 4 groups of heads per feature, loads in flight
   // together) and the new key k^ (RMS norm), both rounded to bf16
-  __shared__ float s_hsum[4][64];
   {
     const int j = tid & 63, grp = tid >> 6;
     float a = 0.f;
@@ -288,142 +304,108 @@ online_score_kernel(int B, int cap, int Hq, int dI, int rows_per_cta,
   if (lane == 0) { s_key[warp] = best; s_slot[warp] = best_slot; }
   __syncthreads();
   asm volatile("barrier.cluster.wait.aligned;\n" ::: "memory");   // phase 0: all running
-  if (tid == 0) {   // this CTA's candidate into slot `rank` of CTA 0
+  if (tid == 0) {   // this CTA's candidate into slot `rank` of every CTA's table
     unsigned long long k = s_key[0];
     int sl = s_slot[0];
     for (int w = 1; w < kOnThreads / 32; ++w)
       if (s_key[w] < k) { k = s_key[w]; sl = s_slot[w]; }
-    cluster.map_shared_rank(s_ckey, 0)[rank] = k;
-    cluster.map_shared_rank(s_cslot, 0)[rank] = sl;
+    for (int d = 0; d < nct; ++d) {
+      cluster.map_shared_rank(s_ckey, d)[rank] = k;
+      cluster.map_shared_rank(s_cslot, d)[rank] = sl;
+    }
   }
-  cluster.sync();   // every CTA has written its candidate into CTA 0
-  if (rank == 0 && tid == 0) {
+  cluster.sync();   // every candidate is in every table; every CTA's reads of
+                    // the indexer keys and importances are done
+  if (tid == 0) {
     unsigned long long k = ~0ull;
     int e = -1;
     for (int i = 0; i < nct; ++i)
       if (s_ckey[i] < k) { k = s_ckey[i]; e = s_cslot[i]; }
-    OnlineChoice ch;
-    ch.slot = e;
-    ch.pos = (int32_t)(~(uint32_t)(k & 0xffffffffull));
-    ch.I_e = order_key_inv((uint32_t)(k >> 32));
     if (e < 0) {   // no ordered candidate (NaN importances): the new token leaves
-      ch.slot = B; ch.pos = npos; ch.I_e = s_Inew;
+      s_e = B; s_epos = npos; s_Ie = s_Inew;
+    } else {
+      s_e = e;
+      s_epos = (int32_t)(~(uint32_t)(k & 0xffffffffull));
+      s_Ie = order_key_inv((uint32_t)(k >> 32));
     }
-    ch.I_new = s_Inew;
-    ch.pos_new = npos;
-    choice[bi] = ch;
   }
-  if (rank == 0 && tid < kIdxPad / 8) {   // the new token's indexer key (bf16)
-    float f[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) f[c] = s_kn[8 * tid + c];
-    store8<__nv_bfloat16>(choice[bi].khat_new + 8 * tid, f);
-  }
-}
-
-// ---- memory update with the evicted token, slot swap (after the attention) ---
-// CTA (KV head kh, sequence bi): phi = W_phi k_e, M <- lambda M + phi v_e^T,
-// b <- lambda b + phi; the rows of slot e and slot B (the new token, appended
-// by the attention step) swap for this head. CTA kh = 0 also swaps the indexer
-// keys, importances and positions (slot e takes the new token, slot B keeps
-// the evicted one with the importance it was chosen by), writes the evicted
-// position, returns cache_len to B, advances next_pos and clears the decode
-// tag (slot e and the memory changed after the attention step).
-template <typename T>
-__global__ void __launch_bounds__(kOnThreads)
-online_evict_kernel(int B, int cap, int Hkv, int D, int r, float lambda,
-                    const OnlineChoice* __restrict__ choice, const float* __restrict__ W_phi,
-                    T* __restrict__ K_ret, T* __restrict__ V_ret,
-                    __nv_bfloat16* __restrict__ khat_ret, float* __restrict__ I_ret,
-                    int32_t* __restrict__ pos_ret, int32_t* __restrict__ next_pos,
-                    int32_t* __restrict__ cache_len, float* __restrict__ M,
-                    float* __restrict__ bstab, int32_t* __restrict__ evicted,
-                    int* __restrict__ dec_tag) {
-  extern __shared__ float osm[];
-  float* sk = osm;          // [D]
-  float* sv = sk + D;       // [D]
-  float* sphi = sv + D;     // [r]
-  const int kh = blockIdx.x, bi = blockIdx.y, tid = threadIdx.x;
-  pdl_wait();
-  pdl_launch();
-  const OnlineChoice ch = choice[bi];
-  const int e = ch.slot;
-  const size_t rs = (size_t)Hkv * D;
-  T* ke = K_ret + ((size_t)bi * cap + e) * rs + (size_t)kh * D;
-  T* ve = V_ret + ((size_t)bi * cap + e) * rs + (size_t)kh * D;
-  for (int c = tid; c < D; c += kOnThreads) { sk[c] = ldf(ke + c); sv[c] = ldf(ve + c); }
   __syncthreads();
-  // phi = W_phi k: 4 threads per row, float4 loads
-  for (int j0 = 0; j0 < r; j0 += kOnThreads / 4) {
-    const int j = j0 + tid / 4, part = tid & 3;
-    float a = 0.f;
-    if (j < r) {
-      const float4* wr = reinterpret_cast<const float4*>(W_phi + (size_t)j * D);
+  const int e = s_e;
+  // ---- phase 2: this CTA's KV head
+  const int kh = rank;
+  if (kh < Hkv) {
+    const size_t rs = (size_t)Hkv * D;
+    T* ke = K_ret + ((size_t)bi * cap + e) * rs + (size_t)kh * D;
+    T* ve = V_ret + ((size_t)bi * cap + e) * rs + (size_t)kh * D;
+    for (int c = tid; c < D; c += kOnThreads) { sk[c] = ldf(ke + c); sv[c] = ldf(ve + c); }
+    __syncthreads();
+    // phi = W_phi k: 4 threads per row, float4 loads
+    for (int j0 = 0; j0 < r; j0 += kOnThreads / 4) {
+      const int j = j0 + tid / 4, part = tid & 3;
+      float a = 0.f;
+      if (j < r) {
+        const float4* wr = reinterpret_cast<const float4*>(W_phi + (size_t)j * D);
 #pragma unroll 8
-      for (int c4 = part; c4 < D / 4; c4 += 4) {
-        const float4 w = __ldg(wr + c4);
-        a = fmaf(w.x, sk[4 * c4], fmaf(w.y, sk[4 * c4 + 1], fmaf(w.z, sk[4 * c4 + 2], fmaf(w.w, sk[4 * c4 + 3], a))));
+        for (int c4 = part; c4 < D / 4; c4 += 4) {
+          const float4 w = __ldg(wr + c4);
+          a = fmaf(w.x, sk[4 * c4], fmaf(w.y, sk[4 * c4 + 1], fmaf(w.z, sk[4 * c4 + 2], fmaf(w.w, sk[4 * c4 + 3], a))));
+        }
+      }
+      a += __shfl_xor_sync(0xffffffffu, a, 1);
+      a += __shfl_xor_sync(0xffffffffu, a, 2);
+      if (j < r && part == 0) sphi[j] = a;
+    }
+    __syncthreads();
+    float4* Mu = reinterpret_cast<float4*>(M + ((size_t)bi * Hkv + kh) * r * D);
+#pragma unroll 4
+    for (int i = tid; i < r * D / 4; i += kOnThreads) {
+      const int j = (4 * i) / D, c = (4 * i) % D;
+      float4 m = Mu[i];
+      const float ph = sphi[j];
+      m.x = fmaf(lambda, m.x, ph * sv[c]);
+      m.y = fmaf(lambda, m.y, ph * sv[c + 1]);
+      m.z = fmaf(lambda, m.z, ph * sv[c + 2]);
+      m.w = fmaf(lambda, m.w, ph * sv[c + 3]);
+      Mu[i] = m;
+    }
+    for (int j = tid; j < r; j += kOnThreads) {
+      float* bp = bstab + ((size_t)bi * Hkv + kh) * r + j;
+      *bp = fmaf(lambda, *bp, sphi[j]);
+    }
+    if (e != B) {   // the new token (slot B) and the evicted one swap rows
+      T* kn = K_ret + ((size_t)bi * cap + B) * rs + (size_t)kh * D;
+      T* vn = V_ret + ((size_t)bi * cap + B) * rs + (size_t)kh * D;
+      for (int c = tid; c < D; c += kOnThreads) {
+        const T k0 = ke[c], v0 = ve[c];
+        ke[c] = kn[c]; ve[c] = vn[c];
+        kn[c] = k0; vn[c] = v0;
       }
     }
-    a += __shfl_xor_sync(0xffffffffu, a, 1);
-    a += __shfl_xor_sync(0xffffffffu, a, 2);
-    if (j < r && part == 0) sphi[j] = a;
   }
-  __syncthreads();
-  float4* Mu = reinterpret_cast<float4*>(M + ((size_t)bi * Hkv + kh) * r * D);
-#pragma unroll 4
-  for (int i = tid; i < r * D / 4; i += kOnThreads) {
-    const int j = (4 * i) / D, c = (4 * i) % D;
-    float4 m = Mu[i];
-    const float ph = sphi[j];
-    m.x = fmaf(lambda, m.x, ph * sv[c]);
-    m.y = fmaf(lambda, m.y, ph * sv[c + 1]);
-    m.z = fmaf(lambda, m.z, ph * sv[c + 2]);
-    m.w = fmaf(lambda, m.w, ph * sv[c + 3]);
-    Mu[i] = m;
-  }
-  for (int j = tid; j < r; j += kOnThreads) {
-    float* bp = bstab + ((size_t)bi * Hkv + kh) * r + j;
-    *bp = fmaf(lambda, *bp, sphi[j]);
-  }
-  if (e != B) {   // the new token (slot B) and the evicted one swap rows
-    T* kn = K_ret + ((size_t)bi * cap + B) * rs + (size_t)kh * D;
-    T* vn = V_ret + ((size_t)bi * cap + B) * rs + (size_t)kh * D;
-    for (int c = tid; c < D; c += kOnThreads) {
-      const T k0 = ke[c], v0 = ve[c];
-      ke[c] = kn[c]; ve[c] = vn[c];
-      kn[c] = k0; vn[c] = v0;
-    }
-  }
-  if (kh == 0) {
+  if (rank == 0) {
     if (tid < kIdxPad / 8) {
       uint4* hb = reinterpret_cast<uint4*>(khat_ret + ((size_t)bi * cap + B) * kIdxPad) + tid;
       uint4* he = reinterpret_cast<uint4*>(khat_ret + ((size_t)bi * cap + e) * kIdxPad) + tid;
-      const uint4 knew = reinterpret_cast<const uint4*>(choice[bi].khat_new)[tid];
+      float f[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) f[c] = s_kn[8 * tid + c];
       if (e != B) *hb = *he;
-      *he = knew;
+      store8<__nv_bfloat16>(reinterpret_cast<__nv_bfloat16*>(he), f);
     }
     if (tid == 0) {
-      I_ret[(size_t)bi * cap + e] = ch.I_new;
-      pos_ret[(size_t)bi * cap + e] = ch.pos_new;
-      I_ret[(size_t)bi * cap + B] = ch.I_e;
-      pos_ret[(size_t)bi * cap + B] = ch.pos;
-      evicted[bi] = ch.pos;
+      I_ret[(size_t)bi * cap + e] = s_Inew;
+      pos_ret[(size_t)bi * cap + e] = npos;
+      I_ret[(size_t)bi * cap + B] = s_Ie;
+      pos_ret[(size_t)bi * cap + B] = s_epos;
+      evicted[bi] = s_epos;
       cache_len[bi] = B;
       dec_tag[bi] = 0;
-      next_pos[bi] = ch.pos_new + 1;
+      next_pos[bi] = npos + 1;
     }
   }
 }
 
 }  // namespace
-
-// CTAs per sequence of the score-and-evict cluster: one per 256 candidate rows,
-// at most kOnlineMaxCluster.
-int online_cluster_ctas(int B) {
-  int n = (B + 1 + kOnThreads - 1) / kOnThreads;
-  return n > kOnlineMaxCluster ? kOnlineMaxCluster : (n < 1 ? 1 : n);
-}
 
 cudaError_t launch_online_init(const Ctx& c, int batch, int L, int B, int cap,
                                const float* running_max, const int32_t* idx_r,
@@ -465,16 +447,20 @@ cudaError_t launch_online_features(const Ctx& c, int batch, const void* x, const
                     qpart, kpart);
 }
 
-cudaError_t launch_online_score(const Ctx& c, int batch, int B, int cap, const float* qpart,
-                                const float* kpart, const void* khat_ret, float* I_ret,
-                                const int32_t* pos_ret, const int32_t* next_pos, void* choice,
-                                cudaStream_t st) {
-  const int nct = online_cluster_ctas(B);
+cudaError_t launch_online_score_evict(const Ctx& c, int batch, int B, int cap, const float* qpart,
+                                      const float* kpart, void* khat_ret, float* I_ret,
+                                      int32_t* pos_ret, int32_t* next_pos, void* K_ret, void* V_ret,
+                                      int32_t* cache_len, float* M, float* bstab, int32_t* evicted,
+                                      int* dec_tag, cudaStream_t st) {
+  const int Hkv = c.cfg.n_kv_heads, D = c.cfg.head_dim, r = c.cfg.mem_r;
+  const int nct = Hkv;   // one CTA per KV head
+  if (nct > kOnlineMaxCluster) return cudaErrorInvalidValue;
   const int rows_per_cta = (B + 1 + nct - 1) / nct;
+  const size_t sm = (size_t)(2 * D + r) * sizeof(float);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nct, batch, 1);
   cfg.blockDim = dim3(kOnThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = sm;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -485,28 +471,23 @@ cudaError_t launch_online_score(const Ctx& c, int batch, int B, int cap, const f
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, online_score_kernel, B, cap, c.cfg.n_q_heads, c.cfg.idx_dim,
-                            rows_per_cta, qpart, kpart, (const __nv_bfloat16*)khat_ret, I_ret,
-                            pos_ret, next_pos, (OnlineChoice*)choice);
-}
-
-cudaError_t launch_online_evict(const Ctx& c, int batch, int B, int cap, const void* choice,
-                                void* khat_ret, float* I_ret, int32_t* pos_ret, int32_t* next_pos,
-                                void* K_ret, void* V_ret, int32_t* cache_len, float* M,
-                                float* bstab, int32_t* evicted, int* dec_tag, cudaStream_t st) {
-  const int Hkv = c.cfg.n_kv_heads, D = c.cfg.head_dim, r = c.cfg.mem_r;
-  const size_t sm = (size_t)(2 * D + r) * sizeof(float);
-  const dim3 g(Hkv, batch);
-  const OnlineChoice* ch = (const OnlineChoice*)choice;
-  if (c.cfg.dtype == IMEM_BF16)
-    return launch_pdl(online_evict_kernel<__nv_bfloat16>, g, sm, st, B, cap, Hkv, D, r,
-                      c.cfg.lambda, ch, (const float*)c.W_phi, (__nv_bfloat16*)K_ret,
-                      (__nv_bfloat16*)V_ret, (__nv_bfloat16*)khat_ret, I_ret, pos_ret, next_pos,
-                      cache_len, M, bstab, evicted, dec_tag);
-  return launch_pdl(online_evict_kernel<float>, g, sm, st, B, cap, Hkv, D, r, c.cfg.lambda, ch,
-                    (const float*)c.W_phi, (float*)K_ret, (float*)V_ret,
-                    (__nv_bfloat16*)khat_ret, I_ret, pos_ret, next_pos, cache_len, M, bstab,
-                    evicted, dec_tag);
+  if (c.cfg.dtype == IMEM_BF16) {
+    auto k = online_score_evict_kernel<__nv_bfloat16>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    return cudaLaunchKernelEx(&cfg, k, B, cap, c.cfg.n_q_heads, Hkv, D, r, c.cfg.idx_dim,
+                              rows_per_cta, c.cfg.lambda, qpart, kpart, (const float*)c.W_phi,
+                              (__nv_bfloat16*)K_ret, (__nv_bfloat16*)V_ret,
+                              (__nv_bfloat16*)khat_ret, I_ret, pos_ret, next_pos, cache_len, M,
+                              bstab, evicted, dec_tag);
+  }
+  auto k = online_score_evict_kernel<float>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernelEx(&cfg, k, B, cap, c.cfg.n_q_heads, Hkv, D, r, c.cfg.idx_dim,
+                            rows_per_cta, c.cfg.lambda, qpart, kpart, (const float*)c.W_phi,
+                            (float*)K_ret, (float*)V_ret, (__nv_bfloat16*)khat_ret, I_ret, pos_ret,
+                            next_pos, cache_len, M, bstab, evicted, dec_tag);
 }
 
 }  // namespace imem
