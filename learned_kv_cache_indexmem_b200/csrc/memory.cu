@@ -558,10 +558,21 @@ memory_bf16_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __r
   const uint32_t full0 = tc::smem_addr(bars), empty0 = full0 + 8 * kBfStages,
                  done = full0 + 16 * kBfStages;
 
-  // zero every stage (padding rows of A, unused columns of B), then the ones
-  // column of B: element 0 of the first 16-byte chunk of the last atom column
-  for (int i = tid; i < kBfStages * TL::STAGE / 16; i += kMemThreads)
-    reinterpret_cast<uint4*>(smem)[i] = make_uint4(0, 0, 0, 0);
+  // zero what no copy or conversion writes: the last atom column of B (the
+  // ones column and the padding columns) and, for d = 64, the upper half of
+  // A's rows in both key buffers; then the ones column of B (element 0 of the
+  // first 16-byte chunk of that atom column)
+  {
+    constexpr int ATOM16 = TL::ATOM_COL / 16;             // 16-byte chunks per atom column
+    constexpr int REGIONS = 1 + (D == 64 ? 2 : 0);
+    for (int i = tid; i < kBfStages * REGIONS * ATOM16; i += kMemThreads) {
+      const int st = i / (REGIONS * ATOM16), k = i % (REGIONS * ATOM16);
+      const int region = k / ATOM16, o = k % ATOM16;
+      const uint32_t off = region == 0 ? 2 * TL::A_BYTES + (TL::B_ATOMS - 1) * TL::ATOM_COL
+                                       : (region - 1) * TL::A_BYTES + TL::ATOM_COL;
+      reinterpret_cast<uint4*>(smem + st * TL::STAGE + off)[o] = make_uint4(0, 0, 0, 0);
+    }
+  }
   __syncthreads();
   for (int i = tid; i < kBfStages * kBfChunk; i += kMemThreads) {
     const int st = i / kBfChunk, jj = i % kBfChunk;
