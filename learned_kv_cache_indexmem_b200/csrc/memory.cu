@@ -492,13 +492,19 @@ memory_finalize_kernel(const float* __restrict__ partials, int G, int tpg, int n
 //       a key row lands in the A_hi buffer and is rewritten there in place;
 //   B = [v | 1], the value row as loaded (bf16 is exact) and a column of
 //       ones written once, which makes s = sum w k fall out of the same MMA.
-// Chunks of 32 tokens; a ring of kBfStages stages; the loaders keep
-// kBfStages - 2 chunks in flight ahead of the one they convert. The run's
-// evicted positions are read into shared memory once (runs of at most
-// kRunMax tokens). One CTA per SM.
+// Chunks of 32 tokens; a ring of kBfStages stages; each loader thread keeps
+// kBfAhead chunks in flight ahead of the one it converts, so that a stage is
+// refilled kBfStages - kBfAhead chunks after its conversion (the MMAs of that
+// chunk have long finished: the loaders rarely wait for them). Two CTAs per
+// SM (each with its own ring and accumulator): at c2 shapes a 3-stage ring with
+// one chunk ahead measured faster than a 7-stage ring with five ahead at one
+// CTA per SM (75.9 vs 94.2 us for the stage). The run's evicted positions are
+// read into shared memory once (runs of at most kRunMax tokens).
 constexpr int kBfChunk = 32;
-constexpr int kBfStages = 7;
-constexpr int kBfAhead = kBfStages - 2;
+constexpr int kBfStages = 3;
+constexpr int kBfAhead = 1;
+constexpr int kBfLoaders = 256;   // loader threads (at most one 16-byte item each per chunk)
+constexpr int kBfCtasPerSm = 2;
 constexpr int kRunMax = 4096;
 
 template <int D>
@@ -512,6 +518,12 @@ struct BfTile {
   static constexpr int STAGE = 2 * A_BYTES + B_BYTES;    // A_hi | A_lo | B
   static constexpr int SMEM = kBfStages * STAGE + kRunMax * 4 + 1024 + 256;
 };
+
+// loader threads and the block size (+ the MMA warp) of the bf16 kernel
+template <int D> constexpr int bf_loaders() {
+  return kBfChunk * (D / 8) < kBfLoaders ? kBfChunk * (D / 8) : kBfLoaders;
+}
+template <int D> constexpr int bf_threads() { return bf_loaders<D>() + 32; }
 
 __device__ __forceinline__ uint32_t bf_off(int jj, int cc, int atom_col) {
   return (uint32_t)((cc >> 3) * atom_col + (jj >> 3) * 1024 + (jj & 7) * 128 +
@@ -532,11 +544,12 @@ __device__ __forceinline__ void cp_async_wait_group() {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kMemThreads, 1)
+__global__ void __launch_bounds__(bf_threads<D>(), kBfCtasPerSm)
 memory_bf16_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V,
                    const int32_t* __restrict__ idx_e, int n_e, int L, int Hkv, float log2lam,
                    int tokens_per_run, float* __restrict__ partials, int* __restrict__ err) {
   using TL = BfTile<D>;
+  constexpr int NL = bf_loaders<D>(), NT = NL + 32;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -565,7 +578,7 @@ memory_bf16_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __r
   {
     constexpr int ATOM16 = TL::ATOM_COL / 16;             // 16-byte chunks per atom column
     constexpr int REGIONS = 1 + (D == 64 ? 2 : 0);
-    for (int i = tid; i < kBfStages * REGIONS * ATOM16; i += kMemThreads) {
+    for (int i = tid; i < kBfStages * REGIONS * ATOM16; i += NT) {
       const int st = i / (REGIONS * ATOM16), k = i % (REGIONS * ATOM16);
       const int region = k / ATOM16, o = k % ATOM16;
       const uint32_t off = region == 0 ? 2 * TL::A_BYTES + (TL::B_ATOMS - 1) * TL::ATOM_COL
@@ -574,7 +587,7 @@ memory_bf16_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __r
     }
   }
   __syncthreads();
-  for (int i = tid; i < kBfStages * kBfChunk; i += kMemThreads) {
+  for (int i = tid; i < kBfStages * kBfChunk; i += NT) {
     const int st = i / kBfChunk, jj = i % kBfChunk;
     *reinterpret_cast<__nv_bfloat16*>(smem + st * TL::STAGE + 2 * TL::A_BYTES +
                                       bf_off(jj, (D / 64) * 8, TL::ATOM_COL)) =
@@ -585,16 +598,16 @@ memory_bf16_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __r
   uint32_t bad = 0;
   const int32_t* E = idx_e + (size_t)bi * n_e + j0;
   {
-    constexpr int PP = (kRunMax + kMemThreads - 1) / kMemThreads;
+    constexpr int PP = (kRunMax + NT - 1) / NT;
     int pv[PP];
 #pragma unroll
     for (int k = 0; k < PP; ++k) {
-      const int i = tid + k * kMemThreads;
+      const int i = tid + k * NT;
       pv[k] = i < ntok ? __ldg(E + i) : -1;
     }
 #pragma unroll
     for (int k = 0; k < PP; ++k) {
-      const int i = tid + k * kMemThreads;
+      const int i = tid + k * NT;
       if (i < nchunks * kBfChunk) {
         int p = pv[k];
         if (i < ntok && (unsigned)p >= (unsigned)L) { bad = 1u; p = -1; }
@@ -604,14 +617,14 @@ memory_bf16_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __r
   }
   if (tid == 0) {
     for (int st = 0; st < kBfStages; ++st) {
-      tc::mbar_init(full0 + 8 * st, kLoaders);
+      tc::mbar_init(full0 + 8 * st, NL);
       tc::mbar_init(empty0 + 8 * st, 1);
     }
     tc::mbar_init(done, 1);
     tc::fence_mbar_init();
     s_abort = 0;
   }
-  if (warp == 8) {
+  if (warp == NL / 32) {
     tc::tmem_alloc(tc::smem_addr(&s_tmem), 256);
     tc::tmem_relinquish();
   }
@@ -622,11 +635,11 @@ memory_bf16_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __r
   const uint32_t tmem = s_tmem;
   float* out = partials + (((size_t)bi * Hkv + kh) * G + g) * (size_t)D * (D + 1);
 
-  if (warp < 8) {
+  if (warp < NL / 32) {
     // ---------------- loaders
     constexpr int CH = D / 8;                          // 16-byte chunks per row
-    constexpr int ITEMS = kBfChunk * CH / kLoaders;    // per thread per chunk (K and V each)
-    static_assert(ITEMS >= 1 && kBfChunk * CH % kLoaders == 0, "whole items per thread");
+    constexpr int ITEMS = kBfChunk * CH / NL;    // per thread per chunk (K and V each)
+    static_assert(ITEMS >= 1 && kBfChunk * CH % NL == 0, "whole items per thread");
     const size_t row_stride = (size_t)Hkv * D;
     const __nv_bfloat16* Kb = K + (size_t)bi * L * row_stride + (size_t)kh * D;
     const __nv_bfloat16* Vb = V + (size_t)bi * L * row_stride + (size_t)kh * D;
@@ -635,7 +648,7 @@ memory_bf16_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __r
       const uint32_t b = a + 2 * TL::A_BYTES;
 #pragma unroll
       for (int it = 0; it < ITEMS; ++it) {
-        const int i = tid + it * kLoaders, jj = i / CH, cc = i % CH;
+        const int i = tid + it * NL, jj = i / CH, cc = i % CH;
         const int p = s_pos[c * kBfChunk + jj];
         const size_t off = (size_t)(p < 0 ? 0 : p) * row_stride + cc * 8;
         const uint32_t o = bf_off(jj, cc, TL::ATOM_COL);
@@ -653,7 +666,7 @@ memory_bf16_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __r
     for (int c = 0; c < nchunks; ++c) {
       const int cn = c + kBfAhead;
       if (cn < nchunks) {
-        // its stage last held chunk cn - kBfStages (= c - 2): wait for that MMA
+        // its stage last held chunk cn - kBfStages: wait for that chunk's MMAs
         if (cn >= kBfStages &&
             !tc::mbar_wait(empty0 + 8 * (cn % kBfStages), ((cn / kBfStages) - 1) & 1)) {
           record_error(err, DEV_TIMEOUT);
@@ -669,7 +682,7 @@ memory_bf16_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __r
       unsigned char* a_p = smem + (c % kBfStages) * TL::STAGE;
 #pragma unroll
       for (int it = 0; it < ITEMS; ++it) {
-        const int i = tid + it * kLoaders, jj = i / CH, cc = i % CH;
+        const int i = tid + it * NL, jj = i / CH, cc = i % CH;
         const int j = j0 + c * kBfChunk + jj;
         const float w = j < j1 ? exp2f((float)(j1 - 1 - j) * log2lam) : 0.f;
         const uint32_t o = bf_off(jj, cc, TL::ATOM_COL);
@@ -749,7 +762,7 @@ memory_bf16_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __r
   }
   tc::fence_before();
   __syncthreads();
-  if (warp == 8) tc::tmem_dealloc(tmem, 256);
+  if (warp == NL / 32) tc::tmem_dealloc(tmem, 256);
 }
 
 // Launches the finalize with programmatic stream serialization (it waits for
@@ -796,7 +809,7 @@ MemSplit memory_split(int batch, int n_kv_heads, int n_e, int num_sms, size_t ma
   return MemSplit{(n_e + tpr - 1) / tpr, tpr};
 }
 
-// Runs of the bf16 kernel (one CTA per SM): at least ceil(n / kRunMax) runs
+// Runs of the bf16 kernel (kBfCtasPerSm CTAs per SM): at least ceil(n / kRunMax) runs
 // per unit (the run's positions sit in shared memory), a whole number of
 // 32-token chunks each; among the run counts up to four waves, the one whose
 // last wave is fullest (the fewest runs within 3% of the best), so that SMs do
@@ -806,7 +819,8 @@ MemSplit memory_split_bf16(int batch, int n_kv_heads, int n_e, int num_sms) {
   const int chunks = (n_e + kBfChunk - 1) / kBfChunk;
   int lo = (n_e + kRunMax - 1) / kRunMax;
   if (lo < 1) lo = 1;
-  int hi = (4 * num_sms) / units;
+  const int slots = num_sms * kBfCtasPerSm;
+  int hi = (4 * slots) / units;
   if (hi > chunks) hi = chunks;
   if (hi > kMemMaxGroups) hi = kMemMaxGroups;
   if (hi < lo) hi = lo;
@@ -814,8 +828,8 @@ MemSplit memory_split_bf16(int batch, int n_kv_heads, int n_e, int num_sms) {
   int G = lo;
   for (int g = lo; g <= hi; ++g) {
     const long ctas = (long)units * g;
-    const long waves = (ctas + num_sms - 1) / num_sms;
-    const double eff = (double)ctas / (double)(waves * num_sms);
+    const long waves = (ctas + slots - 1) / slots;
+    const double eff = (double)ctas / (double)(waves * slots);
     if (eff > best + 0.03) { best = eff; G = g; }
   }
   const int tpr = ((chunks + G - 1) / G) * kBfChunk;
@@ -825,7 +839,8 @@ MemSplit memory_split_bf16(int batch, int n_kv_heads, int n_e, int num_sms) {
 // Upper bound of units * runs over both kernels for up to L evicted tokens
 // per unit (sizes the partial sums in the workspace).
 size_t memory_runs_bound(int units, int L, int num_sms) {
-  return (size_t)units * ((L + kRunMax - 1) / kRunMax + 1) + 4 * (size_t)num_sms + units;
+  return (size_t)units * ((L + kRunMax - 1) / kRunMax + 1) + 4 * (size_t)num_sms * kBfCtasPerSm +
+         units;
 }
 
 cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, const void* V,
@@ -852,7 +867,7 @@ cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, 
     e = cudaFuncSetAttribute(memory_bf16_kernel<DD>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              BfTile<DD>::SMEM);                                               \
     if (e != cudaSuccess) return e;                                                           \
-    memory_bf16_kernel<DD><<<grid, kMemThreads, BfTile<DD>::SMEM, st>>>(                      \
+    memory_bf16_kernel<DD><<<grid, bf_threads<DD>(), BfTile<DD>::SMEM, st>>>(                      \
         (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, idx_e, n_e, L, Hkv, log2lam,        \
         tokens_per_group, partials, c.err);                                                   \
   } while (0)
