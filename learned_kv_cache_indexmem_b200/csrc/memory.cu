@@ -339,19 +339,30 @@ memory_tc_kernel(const T* __restrict__ K, const T* __restrict__ V, const int32_t
   if (warp == 8) tc::tmem_dealloc(tmem, 256);
 }
 
-// M[:, cols] = decay * M[:, cols] + W_phi * sum_g S_g[:, cols]; the extra
-// column slice (blockIdx.x == D/16) does b from the s column.
-// With sv_partials, slice D/16 + 1 does the value sums: s_v = decay * s_v +
+// M[:, cols] = decay * M[:, cols] + W_phi * sum_g S_g[:, cols] for 16
+// columns a CTA; the extra column slice (blockIdx.x == D / 16) does b from
+// the s column. With sv_partials, slice D / 16 + 1 does the value sums: s_v = decay * s_v +
 // sum_g, and the sequence's count n_e += n_add (KV head 0 of the sequence).
 // Run g covers evicted tokens [g*tpg, min(n, (g+1)*tpg)); its partial sums are
 // weighted relative to its end, so it enters with the factor lambda^(n - end).
+constexpr int kFinRuns = 12;   // runs' column slices a finalize CTA holds in shared memory at once
+
+// dynamic shared memory of the finalize: S's padded columns and the run slices
+inline size_t fin_smem(int D, int G) {
+  return ((size_t)16 * (D + 16) + (size_t)(G < kFinRuns ? G : kFinRuns) * 16 * D) * sizeof(float);
+}
+
+__device__ __forceinline__ void fin_cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+}
+
 __device__ __forceinline__ float run_factor(int g, int tpg, int n, float log2lam) {
   const int end = min(n, (g + 1) * tpg);
   return exp2f((float)(n - end) * log2lam);
 }
 
 template <int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
 memory_finalize_kernel(const float* __restrict__ partials, int G, int tpg, int n_tok,
                        float log2lam, const float* __restrict__ W_phi,
                        int r, float decay_n, float* __restrict__ M, float* __restrict__ bstab,
@@ -374,110 +385,118 @@ memory_finalize_kernel(const float* __restrict__ partials, int G, int tpg, int n
     if (threadIdx.x == 0 && unit % Hkv == 0) n_e[unit / Hkv] += n_add;
     return;
   }
-  float* sW = fsm;                 // [r][D + 1] (padded rows: conflict-free column reads)
-  float* sS = sW + r * (D + 1);    // [D][16]
+  constexpr int BD = D / 4;        // a thread's block of d_k
+  constexpr int SST = D + 16;      // padded column stride of sS: the four d_k blocks of a
+                                   // column start in different banks
+  float* sS = fsm;                 // [16][SST]: column c of S, d_k block b at b * (BD + 4)
+  float* sP = fsm + 16 * SST;      // [kFinRuns][16 * D]: the runs' column slices as stored
   const int unit = blockIdx.y, sl = blockIdx.x;
   const int tid = threadIdx.x;
   const bool bcol = (sl == D / 16);
   const int ncols = bcol ? 1 : 16;
   const int col0 = bcol ? D : sl * 16;
-  if (W_phi) {   // null: the identity map (r == D)
-    // a batch of 8 float4 loads per thread is issued before any of its
-    // stores (one round trip per batch; r * D / 4 <= 2048 needs one batch)
-    constexpr int WQ = 8;
-    for (int base = 0; base < r * D / 4; base += WQ * 256) {
-      float4 wv[WQ];
+  // product: thread (row rl of a pass of 64 rows, d_k block b) keeps its
+  // W_phi block in registers; the four blocks of a row are neighbouring lanes
+  // and meet by shuffles; lane b then writes columns 4b..4b+3 of the row
+  const int b = tid & 3, rl = tid >> 2;
+  float w[BD];
+  float4 old = make_float4(0.f, 0.f, 0.f, 0.f);
+  // the pass's W_phi blocks and old values (M and b are not written by the
+  // tensor-core pass, and every earlier write to them has completed, so pass
+  // 0 reads them before the wait)
+  auto load_pass = [&](int pass) {
+    const int ri = pass * 64 + rl;
+    if (ri >= r) return;
+    if (W_phi) {
 #pragma unroll
-      for (int k = 0; k < WQ; ++k) {
-        const int i = base + tid + k * 256;
-        wv[k] = i < r * D / 4 ? __ldg(reinterpret_cast<const float4*>(W_phi) + i)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int k = 0; k < WQ; ++k) {
-        const int i = base + tid + k * 256;
-        if (i < r * D / 4) {
-          float* dst = sW + ((4 * i) / D) * (D + 1) + (4 * i) % D;
-          dst[0] = wv[k].x; dst[1] = wv[k].y; dst[2] = wv[k].z; dst[3] = wv[k].w;
-        }
+      for (int j = 0; j < BD / 4; ++j) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(W_phi + (size_t)ri * D + b * BD) + j);
+        w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
       }
     }
-  }
-  // sum of the runs: every thread owns IPT (row, column) items and loads all
-  // of them for one run before the next run, so that its loads are
-  // independent (a loop over the runs per item would chain G round trips
-  // to L2 per item)
+    if (bcol) old.x = bstab[(size_t)unit * r + ri];
+    else old = *reinterpret_cast<const float4*>(M + ((size_t)unit * r + ri) * D + col0 + 4 * b);
+  };
+  load_pass(0);
   pdl_wait();
-  const float* p = partials + (size_t)unit * G * D * (D + 1);
-  constexpr int IPT = D * 16 / 256;
+  // sum of the runs: up to kFinRuns runs' slices at once into shared memory
+  // (cp.async: one round trip), then each item summed in run order
+  const float* p = partials + (size_t)unit * G * D * (D + 1) + (size_t)col0 * D;
+  const int pieces = ncols * D / 4;   // 16-byte pieces of a run's slice
+  constexpr int IPT = 16 * D / 256;
   float acc[IPT];
 #pragma unroll
   for (int k = 0; k < IPT; ++k) acc[k] = 0.f;
-  // four runs' loads in flight together, then their sums
-  for (int g0 = 0; g0 < G; g0 += 4) {
-    float v[4][IPT];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float* pg = p + (size_t)(g0 + u) * D * (D + 1) + (size_t)col0 * D;
+  for (int g0 = 0; g0 < G; g0 += kFinRuns) {
+    const int nb = min(kFinRuns, G - g0);
+    for (int k = tid; k < nb * pieces; k += 256) {
+      const int u = k / pieces, pc = k % pieces;
+      fin_cp_async16(tc::smem_addr(sP + (size_t)u * 16 * D + 4 * pc),
+                     p + (size_t)(g0 + u) * D * (D + 1) + 4 * pc);
+    }
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+    __syncthreads();
+    for (int u = 0; u < nb; ++u) {
+      const float f = s_fac[g0 + u];
 #pragma unroll
       for (int k = 0; k < IPT; ++k) {
-        const int i = tid + k * 256;   // column i / D, row i % D: a warp reads 128 bytes
-        v[u][k] = (g0 + u < G && i < D * ncols) ? __ldcg(&pg[i]) : 0.f;
+        const int i = tid + k * 256;   // column i / D, row i % D
+        if (i < ncols * D) acc[k] = fmaf(f, sP[(size_t)u * 16 * D + i], acc[k]);
       }
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float f = g0 + u < G ? s_fac[g0 + u] : 0.f;
-#pragma unroll
-      for (int k = 0; k < IPT; ++k) acc[k] = fmaf(f, v[u][k], acc[k]);
-    }
+    __syncthreads();   // the next batch rewrites sP
   }
 #pragma unroll
   for (int k = 0; k < IPT; ++k) {
     const int i = tid + k * 256;
-    if (i < D * ncols) sS[(i % D) * 16 + i / D] = acc[k];
+    if (i < ncols * D) {
+      const int c = i / D, dk = i % D;
+      sS[c * SST + dk + 4 * (dk / BD)] = acc[k];
+    }
   }
   __syncthreads();
-  // out[ri][c] = sum_dk W_phi[ri][dk] S[dk][c]: a thread takes two rows
-  // (ri, ri + r/2) and four columns, so that each loaded S quad serves two
-  // rows and each W_phi value four columns
-  const int nq = ncols == 16 ? 4 : 1;                 // column quads
-  for (int o = tid; o < (r / 2) * nq; o += 256) {
-    const int ri = o / nq, q = o % nq;
-    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-    if (W_phi) {
-      const float* w0 = sW + (size_t)ri * (D + 1);
-      const float* w1 = sW + (size_t)(ri + r / 2) * (D + 1);
-#pragma unroll 8
-      for (int dk = 0; dk < D; ++dk) {
-        const float4 sv = *reinterpret_cast<const float4*>(sS + dk * 16 + 4 * q);
-        const float x0 = w0[dk], x1 = w1[dk];
-        a0[0] = fmaf(x0, sv.x, a0[0]); a0[1] = fmaf(x0, sv.y, a0[1]);
-        a0[2] = fmaf(x0, sv.z, a0[2]); a0[3] = fmaf(x0, sv.w, a0[3]);
-        a1[0] = fmaf(x1, sv.x, a1[0]); a1[1] = fmaf(x1, sv.y, a1[1]);
-        a1[2] = fmaf(x1, sv.z, a1[2]); a1[3] = fmaf(x1, sv.w, a1[3]);
-      }
-    } else {
+  const int npass = (r + 63) / 64;
+  for (int pass = 0; pass < npass; ++pass) {
+    if (pass > 0) load_pass(pass);
+    const int ri = pass * 64 + rl;
+    if (ri >= r) break;   // r is a multiple of 16: whole warps
+    float a[16];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        a0[e] = sS[ri * 16 + 4 * q + e];
-        a1[e] = sS[(ri + r / 2) * 16 + 4 * q + e];
+    for (int c = 0; c < 16; ++c) a[c] = 0.f;
+    if (W_phi) {
+      const float* s0 = sS + b * (BD + 4);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        if (c < ncols) {
+#pragma unroll
+          for (int j = 0; j < BD / 4; ++j) {
+            const float4 s4 = *reinterpret_cast<const float4*>(s0 + c * SST + 4 * j);
+            a[c] = fmaf(w[4 * j], s4.x, a[c]);
+            a[c] = fmaf(w[4 * j + 1], s4.y, a[c]);
+            a[c] = fmaf(w[4 * j + 2], s4.z, a[c]);
+            a[c] = fmaf(w[4 * j + 3], s4.w, a[c]);
+          }
+          a[c] += __shfl_xor_sync(0xffffffffu, a[c], 1);
+          a[c] += __shfl_xor_sync(0xffffffffu, a[c], 2);
+        }
       }
+    } else {   // identity map: row ri of M takes row ri of S
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        if (c < ncols) a[c] = sS[c * SST + ri + 4 * (ri / BD)];
     }
-    if (bcol) {   // one column: b
-      float* bp = bstab + (size_t)unit * r;
-      bp[ri] = fmaf(bp[ri], decay_n, a0[0]);
-      bp[ri + r / 2] = fmaf(bp[ri + r / 2], decay_n, a1[0]);
+    if (bcol) {
+      if (b == 0) bstab[(size_t)unit * r + ri] = fmaf(old.x, decay_n, a[0]);
     } else {
-      float* m0 = M + ((size_t)unit * r + ri) * D + col0 + 4 * q;
-      float* m1 = M + ((size_t)unit * r + ri + r / 2) * D + col0 + 4 * q;
-      float4 v0 = *reinterpret_cast<float4*>(m0), v1 = *reinterpret_cast<float4*>(m1);
-      v0.x = fmaf(v0.x, decay_n, a0[0]); v0.y = fmaf(v0.y, decay_n, a0[1]);
-      v0.z = fmaf(v0.z, decay_n, a0[2]); v0.w = fmaf(v0.w, decay_n, a0[3]);
-      v1.x = fmaf(v1.x, decay_n, a1[0]); v1.y = fmaf(v1.y, decay_n, a1[1]);
-      v1.z = fmaf(v1.z, decay_n, a1[2]); v1.w = fmaf(v1.w, decay_n, a1[3]);
-      *reinterpret_cast<float4*>(m0) = v0;
-      *reinterpret_cast<float4*>(m1) = v1;
+      // columns 4b..4b+3 (selects keep a[] in registers)
+      float o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        o[e] = b == 0 ? a[e] : b == 1 ? a[4 + e] : b == 2 ? a[8 + e] : a[12 + e];
+      float4 v = old;
+      v.x = fmaf(v.x, decay_n, o[0]); v.y = fmaf(v.y, decay_n, o[1]);
+      v.z = fmaf(v.z, decay_n, o[2]); v.w = fmaf(v.w, decay_n, o[3]);
+      *reinterpret_cast<float4*>(M + ((size_t)unit * r + ri) * D + col0 + 4 * b) = v;
     }
   }
 }
@@ -898,7 +917,7 @@ cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, 
   dim3 fgrid(D / 16 + 1 + (sv_partials ? 1 : 0), batch * Hkv);
   // moment statistics use the identity map: the finalize skips the product
   const float* phi = c.cfg.readout == IMEM_READOUT_MOMENT ? nullptr : c.W_phi;
-  const size_t fsmem = ((size_t)r * (D + 1) + (size_t)D * 16) * sizeof(float);
+  const size_t fsmem = fin_smem(D, Gused);
   if (D == 128)
     e = launch_finalize<128>(fgrid, fsmem, st, partials, Gused, tokens_per_group, n_e, log2lam,
                              phi, r, decay_n, M, bstab, sv_partials, s_v, n_count, (float)n_e, Hkv);
@@ -974,7 +993,7 @@ cudaError_t launch_memory_static(int batch, int L, int Hkv, int r, float lambda,
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const float decay_n = (float)pow((double)lambda, (double)n_e);
-  const size_t fsmem = ((size_t)r * (D + 1) + (size_t)D * 16) * sizeof(float);
+  const size_t fsmem = fin_smem(D, Gused);
   e = launch_finalize<D>(dim3(D / 16 + 1, units), fsmem, st, scratch, Gused, tokens_per_group, n_e,
                          log2lam, W_phi, r, decay_n, M, bstab, nullptr, nullptr, nullptr, 0.f, Hkv);
   if (e != cudaSuccess) return e;

@@ -5,6 +5,7 @@ Stages and sources ("IndexMem" technical summary): §2.A indexer scores pooled
 per key by a running max; §1/§4 top-B eviction; §2.B memory update and the
 residual readout o = o_attn + g(q) m(q).
 """
+import dataclasses
 import math
 
 import numpy as np
@@ -129,14 +130,25 @@ def test_constant_context_ties_go_to_lower_positions(cuda_device):
     assert torch.equal(st.idx_evicted.cpu()[0, :640 - B], torch.arange(B, 640, dtype=torch.int32))
 
 
+def _workload(name):
+    """A workload by name; "c0-bf16" is the tiny c0 layer in bf16 (head dim 64
+    on the bf16 tensor-core memory path)."""
+    if name == "c0-bf16":
+        wl = W["c0"]
+        return dataclasses.replace(wl, shape=dataclasses.replace(wl.shape, dtype="bf16"))
+    return W[name]
+
+
 @pytest.mark.parametrize("name,L,batch,n_e,chunk", [
     ("c0", None, None, 896, 64),
+    ("c0-bf16", None, 2, 896, 64),
+    ("c0-bf16", 700, 1, 699, 64),
     ("c1", None, None, 3686, 512),
     ("c1", 1500, 3, 1499, 128),
     ("c1", 600, 2, 0, 64),
 ])
 def test_memory_update_parity(cuda_device, name, L, batch, n_e, chunk):
-    case = Case(W[name], cuda_device, L=L, batch=batch, n_decode=1)
+    case = Case(_workload(name), cuda_device, L=L, batch=batch, n_decode=1)
     E = synth.make_index_subset(case.batch, case.L, n_e, case.seed)
     M0, b0 = synth.make_memory_state(case.shape, case.batch, case.seed)
     lay = case.layer()
