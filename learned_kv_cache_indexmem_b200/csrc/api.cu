@@ -443,10 +443,10 @@ imem_status imem_update_memory(imem_ctx* h, int batch, int L, const void* K, con
   IMEM_CHECK(online_streams(h->c));
   const imem::Workspace ws = imem::workspace_layout(c, batch, L);
   float* part = (float*)((char*)workspace + ws.mem_part_off);
-  IMEM_CHECK(cuda_status(imem::clear_decode_tags(c, batch, workspace, (cudaStream_t)stream)));
+  int* tags = (int*)((char*)workspace + imem::workspace_layout(c, batch, 1).dec_tag_off);
   return cuda_status(imem::launch_memory_update(c, batch, L, K, V, idx_evicted, n_evicted, chunk,
                                                 M, bstab, part, nullptr, nullptr, nullptr,
-                                                (cudaStream_t)stream));
+                                                (cudaStream_t)stream, tags, batch));
 }
 
 imem_status imem_update_moments(imem_ctx* h, int batch, int L, const void* K, const void* V,
@@ -473,10 +473,10 @@ imem_status imem_update_moments(imem_ctx* h, int batch, int L, const void* K, co
   const imem::Workspace ws = imem::workspace_layout(c, batch, L);
   float* part = (float*)((char*)workspace + ws.mem_part_off);
   float* svp = (float*)((char*)workspace + ws.sv_part_off);
-  IMEM_CHECK(cuda_status(imem::clear_decode_tags(c, batch, workspace, (cudaStream_t)stream)));
+  int* tags = (int*)((char*)workspace + imem::workspace_layout(c, batch, 1).dec_tag_off);
   return cuda_status(imem::launch_memory_update(c, batch, L, K, V, idx_evicted, n_evicted, chunk,
                                                 S_T, s_k, part, svp, s_v, n_e,
-                                                (cudaStream_t)stream));
+                                                (cudaStream_t)stream, tags, batch));
 }
 
 namespace {

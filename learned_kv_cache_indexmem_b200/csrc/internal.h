@@ -151,11 +151,12 @@ cudaError_t launch_gather(const Ctx& c, int batch, int L, int n, const int32_t* 
                           int cap, cudaStream_t st);
 
 // sv_partials, s_v, n_count: value sums and evicted count (moment statistics);
-// all three null for the plain memory update.
+// all three null for the plain memory update. clear_tags: n_clear ints set to
+// zero on the stream before the update completes (the decode tags), or null.
 cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, const void* V,
                                  const int32_t* idx_e, int n_e, int chunk, float* M, float* bstab,
                                  float* partials, float* sv_partials, float* s_v, float* n_count,
-                                 cudaStream_t st);
+                                 cudaStream_t st, int* clear_tags = nullptr, int n_clear = 0);
 
 // s_v, n_e: the moment statistics' value sums and counts (moment readout);
 // null for the gated readout.

@@ -367,9 +367,14 @@ memory_finalize_kernel(const float* __restrict__ partials, int G, int tpg, int n
                        float log2lam, const float* __restrict__ W_phi,
                        int r, float decay_n, float* __restrict__ M, float* __restrict__ bstab,
                        const float* __restrict__ sv_partials, float* __restrict__ s_v,
-                       float* __restrict__ n_e, float n_add, int Hkv) {
+                       float* __restrict__ n_e, float n_add, int Hkv, int* __restrict__ clear_tags,
+                       int n_clear) {
   extern __shared__ float fsm[];
   __shared__ float s_fac[kMemMaxGroups];
+  // the decode tags (no kernel of the update reads them; every earlier
+  // reader has completed)
+  if (clear_tags && blockIdx.x == 0 && blockIdx.y == 0)
+    for (int i = threadIdx.x; i < n_clear; i += 256) clear_tags[i] = 0;
   for (int gg = threadIdx.x; gg < G; gg += 256) s_fac[gg] = run_factor(gg, tpg, n_tok, log2lam);
   __syncthreads();
   if (blockIdx.x == D / 16 + 1) {   // value sums (only launched with sv_partials)
@@ -790,7 +795,8 @@ template <int D>
 cudaError_t launch_finalize(dim3 grid, size_t smem, cudaStream_t st, const float* partials, int G,
                             int tpg, int n_tok, float log2lam, const float* W_phi, int r,
                             float decay_n, float* M, float* bstab, const float* sv_partials,
-                            float* s_v, float* n_count, float n_add, int Hkv) {
+                            float* s_v, float* n_count, float n_add, int Hkv,
+                            int* clear_tags = nullptr, int n_clear = 0) {
   cudaError_t e = cudaFuncSetAttribute(memory_finalize_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -805,7 +811,8 @@ cudaError_t launch_finalize(dim3 grid, size_t smem, cudaStream_t st, const float
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, memory_finalize_kernel<D>, partials, G, tpg, n_tok, log2lam,
-                            W_phi, r, decay_n, M, bstab, sv_partials, s_v, n_count, n_add, Hkv);
+                            W_phi, r, decay_n, M, bstab, sv_partials, s_v, n_count, n_add, Hkv,
+                            clear_tags, n_clear);
 }
 
 }  // namespace
@@ -865,8 +872,10 @@ size_t memory_runs_bound(int units, int L, int num_sms) {
 cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, const void* V,
                                  const int32_t* idx_e, int n_e, int chunk, float* M, float* bstab,
                                  float* partials, float* sv_partials, float* s_v, float* n_count,
-                                 cudaStream_t st) {
-  if (n_e == 0) return cudaSuccess;
+                                 cudaStream_t st, int* clear_tags, int n_clear) {
+  if (n_e == 0)
+    return clear_tags ? cudaMemsetAsync(clear_tags, 0, (size_t)n_clear * sizeof(int), st)
+                      : cudaSuccess;
   const int Hkv = c.cfg.n_kv_heads, D = c.cfg.head_dim, r = c.cfg.mem_r;
   (void)chunk;   // the split below does not change the result
   // bf16 gated memory: the cp.async-fed kernel, unless a run would exceed the
@@ -920,10 +929,12 @@ cudaError_t launch_memory_update(const Ctx& c, int batch, int L, const void* K, 
   const size_t fsmem = fin_smem(D, Gused);
   if (D == 128)
     e = launch_finalize<128>(fgrid, fsmem, st, partials, Gused, tokens_per_group, n_e, log2lam,
-                             phi, r, decay_n, M, bstab, sv_partials, s_v, n_count, (float)n_e, Hkv);
+                             phi, r, decay_n, M, bstab, sv_partials, s_v, n_count, (float)n_e, Hkv,
+                             clear_tags, n_clear);
   else
     e = launch_finalize<64>(fgrid, fsmem, st, partials, Gused, tokens_per_group, n_e, log2lam,
-                            phi, r, decay_n, M, bstab, sv_partials, s_v, n_count, (float)n_e, Hkv);
+                            phi, r, decay_n, M, bstab, sv_partials, s_v, n_count, (float)n_e, Hkv,
+                            clear_tags, n_clear);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
