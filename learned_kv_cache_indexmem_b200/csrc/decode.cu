@@ -60,8 +60,9 @@ struct Partial {   // one query head's softmax state over a block of rows
   float m;         // max of the log2-scaled logits
   float l;         // sum of 2^(s - m)
   float pad[2];
-  float o[D];      // sum of 2^(s - m) v
+  float o[D];      // sum of 2^(s - m) v (at byte 16)
 };
+static_assert(sizeof(Partial<128>) == 16 + 4 * 128, "o at byte 16");
 
 // ---- warp-level tensor-core helpers (bf16) -----------------------------------
 
@@ -578,7 +579,9 @@ __device__ void attend_f32(const float* __restrict__ Kb, const float* __restrict
 // block; ends with a barrier). dst may be another CTA's shared memory: each
 // thread writes 4 consecutive columns with one 16-byte store.
 template <int D, int G>
-__device__ void merge_warps(const Partial<D> (*w_part)[G], Partial<D>* dst) {
+__device__ void merge_warps(const Partial<D> (*w_part)[G], uint32_t dst, uint32_t bar) {
+  // dst, bar: this CTA's slots in the merge CTA and that CTA's push barrier
+  // (shared::cluster addresses); every byte written counts on the barrier
   const int tid = threadIdx.x;
   __syncthreads();
   for (int i = tid; i < G * D / 4; i += kThreads) {
@@ -596,7 +599,8 @@ __device__ void merge_warps(const Partial<D> (*w_part)[G], Partial<D>* dst) {
         o.z = fmaf(v.z, sc, o.z); o.w = fmaf(v.w, sc, o.w);
       }
     }
-    *reinterpret_cast<float4*>(&dst[g].o[c]) = o;
+    tc::st_async_v4(dst + (uint32_t)(g * sizeof(Partial<D>) + 16 + 4 * c), o.x, o.y, o.z, o.w,
+                    bar);
   }
   if (tid < G) {
     float mx = -INFINITY;
@@ -604,11 +608,13 @@ __device__ void merge_warps(const Partial<D> (*w_part)[G], Partial<D>* dst) {
     float l = 0.f;
     for (int w = 0; w < 4; ++w)
       if (w_part[w][tid].m != -INFINITY) l += w_part[w][tid].l * exp2f(w_part[w][tid].m - mx);
-    dst[tid].m = mx;
-    dst[tid].l = l;
+    tc::st_async_v2(dst + (uint32_t)(tid * sizeof(Partial<D>)), mx, l, bar);
   }
-  __syncthreads();
 }
+
+// Bytes that one attention CTA pushes into the merge CTA (G heads: o, m, l).
+template <int D, int G>
+constexpr uint32_t push_bytes() { return (uint32_t)G * (4u * D + 8u); }
 
 // Readout CTA: cp.async loads of b [r], s_v [D] (moment mode) and, if with_M,
 // M [r][D] of one unit into shared memory, as one commit group.
@@ -637,9 +643,6 @@ __device__ __forceinline__ void griddep_launch() {
 
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory");
-}
-__device__ __forceinline__ void cluster_arrive_release() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
@@ -719,7 +722,14 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   __shared__ int s_len_hint;
   __shared__ float s_wr[G], s_kq[G];   // moment readout: w_R and q.k_bar per head
   __shared__ __align__(8) uint64_t s_bar[kDecodeMaxStages];
+  // the merge CTA's push barrier: completes when the attention CTAs' states
+  // (and the second readout CTA's heads) have landed in its shared memory
+  __shared__ __align__(8) uint64_t s_pushbar;
   Partial<D>* slots = reinterpret_cast<Partial<D>*>(dyn_smem + slot_off);   // readout CTA only
+  if (rank == S && tid == 0) {   // before this CTA's arrival on the cluster barrier
+    tc::mbar_init(smem_u32(&s_pushbar), 1);
+    tc::fence_mbar_init();
+  }
 
   // readout CTA's shared memory (see DecSmem::readout)
   constexpr int RG = kThreads / (D / 4);                    // row groups of the M^T u partials
@@ -910,10 +920,10 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     // overlaps the push (an acquire would stall the warp here).
     int arrived = 0;
     if (rank == 0 && tid == 0) arrived = atomicAdd(&seq_counters[bi], 1);
-    // push this CTA's merged state into the readout CTA's slot, then arrive
-    Partial<D>* slot = cluster.map_shared_rank(slots, S) + (size_t)rank * G;
-    merge_warps<D, G>(w_part, slot);
-    cluster_arrive_release();
+    // push this CTA's merged state into the readout CTA's slot (asynchronous
+    // stores counted on its push barrier: nothing to wait for here)
+    merge_warps<D, G>(w_part, tc::mapa(smem_u32(slots + (size_t)rank * G), S),
+                      tc::mapa(smem_u32(&s_pushbar), S));
     if (rank == 0 && tid == 0 && arrived == Hkv - 1) {
       seq_counters[bi] = 0;
       cache_len[bi] = len + 1;
@@ -1021,18 +1031,22 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   if (kNro > 1 && rank > S) {
     // the second readout CTA: its heads' readout (and b . u, which the
     // moment readout's merge needs) into the merge CTA, then arrive
-    cluster_wait();   // phase 0: the merge CTA is running
-    float* ro_m = cluster.map_shared_rank(ro, S);
-    for (int i = hg0 * D + tid; i < (hg0 + HG) * D; i += kThreads) ro_m[i] = ro[i];
-    if (tid < HG) cluster.map_shared_rank(sden, S)[hg0 + tid] = sden[hg0 + tid];
-    cluster_arrive_release();   // phase 1
+    cluster_wait();   // phase 0: the merge CTA is running (its push barrier is set up)
+    const uint32_t bar = tc::mapa(smem_u32(&s_pushbar), S);
+    for (int i = hg0 * D + tid; i < (hg0 + HG) * D; i += kThreads)
+      tc::st_async_f32(tc::mapa(smem_u32(ro + i), S), ro[i], bar);
+    if (tid < HG) tc::st_async_f32(tc::mapa(smem_u32(sden + hg0 + tid), S), sden[hg0 + tid], bar);
     return;
   }
 
   // ---- merge the S attention states that the other CTAs pushed into the slots
-  cluster_wait();             // phase 0
-  cluster_arrive_release();   // phase 1: own arrival
-  cluster_wait();             // phase 1: every attention CTA has written its slot
+  cluster_wait();   // phase 0: every CTA of the cluster is running
+  // every attention CTA's state (and the second readout CTA's heads): the
+  // bytes they push, counted on this CTA's push barrier
+  if (tid == 0)
+    tc::mbar_expect_tx(smem_u32(&s_pushbar),
+                       (uint32_t)S * push_bytes<D, G>() + (uint32_t)(kNro - 1) * HG * (4u * D + 4u));
+  if (!tc::mbar_wait_cluster(smem_u32(&s_pushbar), 0)) record_error(err, DEV_TIMEOUT);
   // merge weights: a warp per head, a lane per slot (S <= 15 < 32)
   for (int g = warp; g < G; g += kThreads / 32) {
     const float mt = lane < S ? slots[lane * G + g].m : -INFINITY;

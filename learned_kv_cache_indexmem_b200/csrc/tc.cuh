@@ -127,6 +127,29 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, float a, fl
                "f"(b), "f"(c), "f"(d)
                : "memory");
 }
+// Asynchronous stores into another CTA's shared memory (addresses from mapa)
+// that count their bytes on that CTA's mbarrier (complete_tx): the receiver
+// waits on its own barrier for the bytes it expects, the sender needs no
+// fence or arrive.
+__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, float a, float b, float c,
+                                            float d, uint32_t cluster_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];\n"
+      ::"r"(cluster_addr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(cluster_bar)
+      : "memory");
+}
+__device__ __forceinline__ void st_async_v2(uint32_t cluster_addr, float a, float b,
+                                            uint32_t cluster_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];\n"
+      ::"r"(cluster_addr), "f"(a), "f"(b), "r"(cluster_bar)
+      : "memory");
+}
+__device__ __forceinline__ void st_async_f32(uint32_t cluster_addr, float a, uint32_t cluster_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];\n"
+               ::"r"(cluster_addr), "f"(a), "r"(cluster_bar)
+               : "memory");
+}
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
