@@ -223,7 +223,7 @@ __device__ void ring_issue_rows(const Ring& rg, const __nv_bfloat16* __restrict_
 // otherwise by cp.async from every thread (rows below `hi` only). TMA frees
 // the SM's issue slots and wins when CTAs stream in several waves; cp.async
 // delivers the first rows sooner and wins when the grid is one wave.
-template <int D, int G, bool kTma>
+template <int D, int G, bool kTma, bool kXtra>
 __device__ void attend_bf16(Ring& rg, const CUtensorMap* tmK, const CUtensorMap* tmV, int x0,
                             int y0, const __nv_bfloat16* __restrict__ Kb,
                             const __nv_bfloat16* __restrict__ Vb, size_t row_stride, int hi,
@@ -266,11 +266,25 @@ __device__ void attend_bf16(Ring& rg, const CUtensorMap* tmK, const CUtensorMap*
     for (int st = n_pre; st < n_stages && st < nst; ++st)
       ring_issue_lsu<D>(rg, Kb, Vb, row_stride, g0 + st, r0 + st * kStageRows, hi);
   }
-  if (!kTma && n_stages <= nst) {
+  // one stage more than the ring holds (kXtra: launches whose blocks reach
+  // it): each warp loads its 16 rows of it into its own rows of the first
+  // stage's buffer (K once its scores are done, V once its first P V is
+  // done) and adds it last (warp-local)
+  const bool extra = kXtra && !kTma && n_stages == nst + 1 && nst == kDecodeMaxStages;
+  if (!kTma && (n_stages <= nst || extra)) {
     // Every stage of this block is in the ring at once (one-wave grids): the
     // scores of all of a warp's row tiles first (independent MMA chains,
     // interleaved), one softmax over them, then all the P V products; the
     // stage-by-stage loop below would chain the tiles one after another.
+    const int xrow0 = r0 + nst * kStageRows;   // the extra stage's first row
+    auto issue_slice = [&](uint32_t dst, const __nv_bfloat16* __restrict__ src) {
+      for (int i = lane; i < 16 * CH; i += 32) {
+        const int rr = warp * 16 + i / CH, c = i % CH, row = xrow0 + rr;
+        const bool ok = row < hi;
+        cp_async16(dst + tile_off<D>(rr, c), src + (size_t)(ok ? row : 0) * row_stride + c * 8, ok);
+      }
+      cp_async_commit();
+    };
     cp_async_wait<0>();
     __syncthreads();
 #pragma unroll
@@ -319,6 +333,10 @@ __device__ void attend_bf16(Ring& rg, const CUtensorMap* tmK, const CUtensorMap*
         }
       }
     }
+    if (extra) {   // this warp's K rows of the first stage are read: its extra K rows there
+      __syncwarp();
+      issue_slice(kts[0], Kb);
+    }
     float sc[kDecodeMaxStages][4];
     float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
@@ -355,6 +373,84 @@ __device__ void attend_bf16(Ring& rg, const CUtensorMap* tmK, const CUtensorMap*
         const uint32_t pb0 = movm_trans(pack_bf16(sc[st][0], sc[st][1]));
         const uint32_t pb1 = movm_trans(pack_bf16(sc[st][2], sc[st][3]));
         const uint32_t vt = kts[st] + kTileBytes<D>;
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(vt + tile_off<D>(rv, 2 * mt + ((lane >> 3) & 1)), a0, a1, a2, a3);
+          mma_bf16_a4(o[mt], a0, a1, a2, a3, pb0, pb1);
+        }
+      }
+      if (extra && st == 0) {   // its V rows of the first stage are read: the extra V rows
+        __syncwarp();
+        issue_slice(kts[0] + kTileBytes<D>, Vb);
+      }
+    }
+    if (extra) {
+      // the extra stage, this warp's 16 rows: patch, scores, running max, P V
+      cp_async_wait<0>();
+      __syncwarp();
+      const uint32_t kt = kts[0], vt = kt + kTileBytes<D>;
+      const int kb = xrow0 + warp * 16;
+      if (kb < r1) {
+        if (kb + 16 > r1 || (len >= kb && len < kb + 16)) {
+          for (int i = lane; i < 16 * CH; i += 32) {
+            const int rr = warp * 16 + i / CH, c = i % CH, row = kb + i / CH;
+            if (row >= r1) {
+              asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};\n" ::"r"(vt + tile_off<D>(rr, c)),
+                           "r"(0u));
+            } else if (row == len) {
+              const uint4 kv = s_new[c];
+              const uint4 vv = s_new[CH + c];
+              asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(kt + tile_off<D>(rr, c)),
+                           "r"(kv.x), "r"(kv.y), "r"(kv.z), "r"(kv.w));
+              asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(vt + tile_off<D>(rr, c)),
+                           "r"(vv.x), "r"(vv.y), "r"(vv.z), "r"(vv.w));
+            }
+          }
+          __syncwarp();
+        }
+        float xa[4] = {0.f, 0.f, 0.f, 0.f}, xb[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+          const int rr = warp * 16 + (lane & 15);
+#pragma unroll
+          for (int s2 = 0; s2 < D / 16; ++s2) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(kt + tile_off<D>(rr, 2 * s2 + (lane >> 4)), a0, a1, a2, a3);
+            if (s2 & 1) mma_bf16_a4(xb, a0, a1, a2, a3, qb0[s2], qb1[s2]);
+            else mma_bf16_a4(xa, a0, a1, a2, a3, qb0[s2], qb1[s2]);
+          }
+        }
+        float xs[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int row = kb + g + ((e >> 1) << 3);
+          xs[e] = (row < r1) ? (xa[e] + xb[e]) * sscale : -INFINITY;
+        }
+        float xm[2] = {fmaxf(xs[0], xs[2]), fmaxf(xs[1], xs[3])};
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          xm[0] = fmaxf(xm[0], __shfl_xor_sync(0xffffffffu, xm[0], off));
+          xm[1] = fmaxf(xm[1], __shfl_xor_sync(0xffffffffu, xm[1], off));
+        }
+        float corr[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float m_new = fmaxf(m_run[h], xm[h]);
+          corr[h] = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - m_new);
+          m_run[h] = m_new;
+        }
+        float p[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) p[e] = (xs[e] == -INFINITY) ? 0.f : exp2f(xs[e] - m_run[e & 1]);
+        l_run[0] = l_run[0] * corr[0] + (p[0] + p[2]);
+        l_run[1] = l_run[1] * corr[1] + (p[1] + p[3]);
+#pragma unroll
+        for (int j = 0; j < D / 16; ++j) {
+          o[j][0] *= corr[0]; o[j][1] *= corr[1];
+          o[j][2] *= corr[0]; o[j][3] *= corr[1];
+        }
+        const uint32_t pb0 = movm_trans(pack_bf16(p[0], p[1]));
+        const uint32_t pb1 = movm_trans(pack_bf16(p[2], p[3]));
 #pragma unroll
         for (int mt = 0; mt < D / 16; ++mt) {
           uint32_t a0, a1, a2, a3;
@@ -685,7 +781,7 @@ struct DecSmem {
   }
 };
 
-template <typename T, int D, int G, bool kTma, int NRO>
+template <typename T, int D, int G, bool kTma, int NRO, bool kXtra>
 __global__ void __launch_bounds__(kThreads)
 decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __restrict__ v_new,
               T* __restrict__ K_ret, T* __restrict__ V_ret, int32_t* __restrict__ cache_len,
@@ -905,7 +1001,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
     auto* w_part = reinterpret_cast<Partial<D>(*)[G]>(dyn_smem);   // aliases the stages
     if constexpr (kBf16) {
       // a miss leaves TMA stages 0..n_spec-1 spent: the block starts after them
-      attend_bf16<D, G, kTma>(ring, &tmK, &tmV, kh * D, bi * cap, Kb, Vb, row_stride, r1, kn, vn,
+      attend_bf16<D, G, kTma, kXtra>(ring, &tmK, &tmV, kh * D, bi * cap, Kb, Vb, row_stride, r1, kn, vn,
                               len, r0, r1, hit ? 0 : n_spec, hit ? n_spec : 0, s_q, w_part, err,
                               s_newrow);
     }
@@ -1111,7 +1207,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   }
 }
 
-template <typename T, int D, int G, bool kTma, int NRO>
+template <typename T, int D, int G, bool kTma, int NRO, bool kXtra>
 cudaError_t launch_tgs(const Ctx& c, int S, int nst, int batch, const void* q, const void* kn,
                       const void* vn, void* K_ret, void* V_ret, int32_t* cache_len, int cap,
                       const float* M, const float* bstab, const float* s_v, const float* n_e,
@@ -1122,7 +1218,7 @@ cudaError_t launch_tgs(const Ctx& c, int S, int nst, int batch, const void* q, c
   const bool m_in_w = c.cfg.readout == IMEM_READOUT_MOMENT || kTma;
   const size_t smem = DecSmem<D, G>::total(kBf16, nst, r, S, m_in_w);
   const uint32_t slot_off = (uint32_t)DecSmem<D, G>::slot_off(r, m_in_w);
-  auto k = decode_kernel<T, D, G, kTma, NRO>;
+  auto k = decode_kernel<T, D, G, kTma, NRO, kXtra>;
   static size_t attr_smem[64] = {};   // per instantiation and device: largest size set so far
   const int dv = c.device & 63;
   if (attr_smem[dv] < smem) {
@@ -1175,16 +1271,22 @@ cudaError_t launch_tg(const Ctx& c, int S, int nst, int batch, const void* q, co
   const int units = batch * c.cfg.n_kv_heads;
   const bool tma = kBf16 && units * (S + 1) > 2 * c.num_sms;
   if (tma)
-    return launch_tgs<T, D, G, kBf16, 1>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M,
+    return launch_tgs<T, D, G, kBf16, 1, false>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M,
                                          bstab, s_v, n_e, out, counters, st);
   // a second readout CTA where the grid keeps about 1.5 CTAs per SM with it
   if constexpr (G >= 2) {
     if (S + 2 <= kDecodeMaxSplits && units * (S + 2) * 2 <= 3 * c.num_sms + 4)
-      return launch_tgs<T, D, G, false, 2>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap,
+      return launch_tgs<T, D, G, false, 2, false>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap,
                                            M, bstab, s_v, n_e, out, counters, st);
   }
-  return launch_tgs<T, D, G, false, 1>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M,
-                                       bstab, s_v, n_e, out, counters, st);
+  // blocks of up to one stage more than the ring (one-wave bf16 grids):
+  // the variant that adds that stage warp by warp
+  const int per_max = ((cap + S - 1) / S + 15) / 16 * 16;
+  if (kBf16 && nst == kDecodeMaxStages && (per_max + kStageRows - 1) / kStageRows == nst + 1)
+    return launch_tgs<T, D, G, false, 1, true>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len,
+                                               cap, M, bstab, s_v, n_e, out, counters, st);
+  return launch_tgs<T, D, G, false, 1, false>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len,
+                                              cap, M, bstab, s_v, n_e, out, counters, st);
 }
 
 template <typename T, int D>
