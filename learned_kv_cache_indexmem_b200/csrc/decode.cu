@@ -223,7 +223,7 @@ __device__ void ring_issue_rows(const Ring& rg, const __nv_bfloat16* __restrict_
 // otherwise by cp.async from every thread (rows below `hi` only). TMA frees
 // the SM's issue slots and wins when CTAs stream in several waves; cp.async
 // delivers the first rows sooner and wins when the grid is one wave.
-template <int D, int G, bool kTma, bool kXtra>
+template <int D, int G, bool kTma, int kXtra>
 __device__ void attend_bf16(Ring& rg, const CUtensorMap* tmK, const CUtensorMap* tmV, int x0,
                             int y0, const __nv_bfloat16* __restrict__ Kb,
                             const __nv_bfloat16* __restrict__ Vb, size_t row_stride, int hi,
@@ -266,24 +266,34 @@ __device__ void attend_bf16(Ring& rg, const CUtensorMap* tmK, const CUtensorMap*
     for (int st = n_pre; st < n_stages && st < nst; ++st)
       ring_issue_lsu<D>(rg, Kb, Vb, row_stride, g0 + st, r0 + st * kStageRows, hi);
   }
-  // one stage more than the ring holds (kXtra: launches whose blocks reach
-  // it): each warp loads its 16 rows of it into its own rows of the first
-  // stage's buffer (K once its scores are done, V once its first P V is
-  // done) and adds it last (warp-local)
-  const bool extra = kXtra && !kTma && n_stages == nst + 1 && nst == kDecodeMaxStages;
+  // stages beyond the ring (kXtra: launches whose blocks reach one more, 1,
+  // or more, 2): after
+  // the ring's stages, each warp streams its own 16 rows of every further
+  // stage through its own rows of the ring's buffers (warp-local copies and
+  // waits, no block barrier): the first further stage's K once the warp's
+  // scores are done and its V once its first P V is done, the next ones (K
+  // and V) once the slice they reuse has been consumed
+  const bool extra = kXtra != 0 && !kTma && n_stages > nst && nst == kDecodeMaxStages &&
+                     (kXtra == 2 || n_stages == nst + 1);
   if (!kTma && (n_stages <= nst || extra)) {
     // Every stage of this block is in the ring at once (one-wave grids): the
     // scores of all of a warp's row tiles first (independent MMA chains,
     // interleaved), one softmax over them, then all the P V products; the
     // stage-by-stage loop below would chain the tiles one after another.
-    const int xrow0 = r0 + nst * kStageRows;   // the extra stage's first row
-    auto issue_slice = [&](uint32_t dst, const __nv_bfloat16* __restrict__ src) {
+    // this warp's rows of stage xs into its rows of the buffer at kt (K, V or
+    // both: one cp.async group)
+    int xg = 0;   // warp-local groups issued
+    auto issue_slice = [&](uint32_t kt, int xs, bool k, bool v) {
+      const int row0 = r0 + xs * kStageRows;
       for (int i = lane; i < 16 * CH; i += 32) {
-        const int rr = warp * 16 + i / CH, c = i % CH, row = xrow0 + rr;
+        const int rr = warp * 16 + i / CH, c = i % CH, row = row0 + rr;
         const bool ok = row < hi;
-        cp_async16(dst + tile_off<D>(rr, c), src + (size_t)(ok ? row : 0) * row_stride + c * 8, ok);
+        const size_t off = (size_t)(ok ? row : 0) * row_stride + c * 8;
+        if (k) cp_async16(kt + tile_off<D>(rr, c), Kb + off, ok);
+        if (v) cp_async16(kt + kTileBytes<D> + tile_off<D>(rr, c), Vb + off, ok);
       }
       cp_async_commit();
+      ++xg;
     };
     cp_async_wait<0>();
     __syncthreads();
@@ -333,9 +343,9 @@ __device__ void attend_bf16(Ring& rg, const CUtensorMap* tmK, const CUtensorMap*
         }
       }
     }
-    if (extra) {   // this warp's K rows of the first stage are read: its extra K rows there
+    if (extra) {   // this warp's K rows of the first stage are read: the next stage's K there
       __syncwarp();
-      issue_slice(kts[0], Kb);
+      issue_slice(kts[0], nst, true, false);
     }
     float sc[kDecodeMaxStages][4];
     float mx[2] = {-INFINITY, -INFINITY};
@@ -380,17 +390,23 @@ __device__ void attend_bf16(Ring& rg, const CUtensorMap* tmK, const CUtensorMap*
           mma_bf16_a4(o[mt], a0, a1, a2, a3, pb0, pb1);
         }
       }
-      if (extra && st == 0) {   // its V rows of the first stage are read: the extra V rows
+      if (extra) {   // this warp's rows of stage st are consumed: refill them
         __syncwarp();
-        issue_slice(kts[0] + kTileBytes<D>, Vb);
+        if (st == 0) issue_slice(kts[0], nst, false, true);
+        else if (kXtra == 2 && st + nst < n_stages) issue_slice(kts[st], st + nst, true, true);
       }
     }
-    if (extra) {
-      // the extra stage, this warp's 16 rows: patch, scores, running max, P V
-      cp_async_wait<0>();
+    // the further stages, this warp's 16 rows each: patch, scores, running
+    // max, P V, then the slice takes the stage nst further on
+    for (int xs = nst; extra && xs < (kXtra == 1 ? nst + 1 : n_stages); ++xs) {
+      // stage xs is group 2 + (xs - nst) of this warp's (K and V of stage nst
+      // are groups 1 and 2): younger groups may stay pending
+      if (kXtra == 1) cp_async_wait<0>();
+      else cp_async_wait_dyn(xg - (2 + (xs - nst)));
       __syncwarp();
-      const uint32_t kt = kts[0], vt = kt + kTileBytes<D>;
-      const int kb = xrow0 + warp * 16;
+      const uint32_t kt = rg.buf0 + (uint32_t)((g0 + xs) % nst) * 2u * kTileBytes<D>;
+      const uint32_t vt = kt + kTileBytes<D>;
+      const int kb = r0 + xs * kStageRows + warp * 16;
       if (kb < r1) {
         if (kb + 16 > r1 || (len >= kb && len < kb + 16)) {
           for (int i = lane; i < 16 * CH; i += 32) {
@@ -457,6 +473,10 @@ __device__ void attend_bf16(Ring& rg, const CUtensorMap* tmK, const CUtensorMap*
           ldsm_x4_t(vt + tile_off<D>(rv, 2 * mt + ((lane >> 3) & 1)), a0, a1, a2, a3);
           mma_bf16_a4(o[mt], a0, a1, a2, a3, pb0, pb1);
         }
+      }
+      if (kXtra == 2 && xs + nst < n_stages) {   // this warp's rows of the slice are consumed
+        __syncwarp();
+        issue_slice(kt, xs + nst, true, true);
       }
     }
   } else
@@ -781,7 +801,7 @@ struct DecSmem {
   }
 };
 
-template <typename T, int D, int G, bool kTma, int NRO, bool kXtra>
+template <typename T, int D, int G, bool kTma, int NRO, int kXtra>
 __global__ void __launch_bounds__(kThreads)
 decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __restrict__ v_new,
               T* __restrict__ K_ret, T* __restrict__ V_ret, int32_t* __restrict__ cache_len,
@@ -1207,7 +1227,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
   }
 }
 
-template <typename T, int D, int G, bool kTma, int NRO, bool kXtra>
+template <typename T, int D, int G, bool kTma, int NRO, int kXtra>
 cudaError_t launch_tgs(const Ctx& c, int S, int nst, int batch, const void* q, const void* kn,
                       const void* vn, void* K_ret, void* V_ret, int32_t* cache_len, int cap,
                       const float* M, const float* bstab, const float* s_v, const float* n_e,
@@ -1271,22 +1291,26 @@ cudaError_t launch_tg(const Ctx& c, int S, int nst, int batch, const void* q, co
   const int units = batch * c.cfg.n_kv_heads;
   const bool tma = kBf16 && units * (S + 1) > 2 * c.num_sms;
   if (tma)
-    return launch_tgs<T, D, G, kBf16, 1, false>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M,
+    return launch_tgs<T, D, G, kBf16, 1, 0>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap, M,
                                          bstab, s_v, n_e, out, counters, st);
   // a second readout CTA where the grid keeps about 1.5 CTAs per SM with it
   if constexpr (G >= 2) {
     if (S + 2 <= kDecodeMaxSplits && units * (S + 2) * 2 <= 3 * c.num_sms + 4)
-      return launch_tgs<T, D, G, false, 2, false>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap,
+      return launch_tgs<T, D, G, false, 2, 0>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap,
                                            M, bstab, s_v, n_e, out, counters, st);
   }
-  // blocks of up to one stage more than the ring (one-wave bf16 grids):
-  // the variant that adds that stage warp by warp
+  // blocks longer than the ring (one-wave bf16 grids): the variant that
+  // streams the further stages warp by warp
   const int per_max = ((cap + S - 1) / S + 15) / 16 * 16;
-  if (kBf16 && nst == kDecodeMaxStages && (per_max + kStageRows - 1) / kStageRows == nst + 1)
-    return launch_tgs<T, D, G, false, 1, true>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len,
-                                               cap, M, bstab, s_v, n_e, out, counters, st);
-  return launch_tgs<T, D, G, false, 1, false>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len,
-                                              cap, M, bstab, s_v, n_e, out, counters, st);
+  const int st_max = (per_max + kStageRows - 1) / kStageRows;
+  if (kBf16 && nst == kDecodeMaxStages && st_max == nst + 1)
+    return launch_tgs<T, D, G, false, 1, 1>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap,
+                                            M, bstab, s_v, n_e, out, counters, st);
+  if (kBf16 && nst == kDecodeMaxStages && st_max > nst + 1)
+    return launch_tgs<T, D, G, false, 1, 2>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap,
+                                            M, bstab, s_v, n_e, out, counters, st);
+  return launch_tgs<T, D, G, false, 1, 0>(c, S, nst, batch, q, kn, vn, K_ret, V_ret, cache_len, cap,
+                                          M, bstab, s_v, n_e, out, counters, st);
 }
 
 template <typename T, int D>
