@@ -192,6 +192,11 @@ def _decode_case(case, cap, lens, gate_override=None):
     ("c1", 3, [410, 37, 1], 420, 8),        # ragged cache lengths
     ("c1", 2, [2000, 1500], 2100, 4),       # several splits
     ("c1", 4, [128, 100, 60, 1], 640, 8),   # short ragged caches, 4 splits
+    # blocks one stage longer than the ring (6 splits of up to 256 rows) and,
+    # for the shorter caches, blocks that fit it
+    ("c1", 4, [1500, 1200, 1100, 700], 1536, 4),
+    # blocks several stages longer than the ring (15 splits of up to 288 rows)
+    ("c1", 1, [4000], 4100, 3),
 ])
 def test_decode_parity(cuda_device, name, batch, lens, cap, steps):
     L = max(max(lens), 64)
