@@ -1335,7 +1335,7 @@ cudaError_t launch_t(const Ctx& c, int S, int nst, int batch, const void* q, con
 int decode_splits(int batch, int n_kv_heads, int cap) {
   const int units = batch * n_kv_heads;
   int S = (222 + units / 2) / units - 1;
-  const int by_rows = (cap + 159) / 160;
+  const int by_rows = (cap + 175) / 176;   // at least ~176 rows a CTA (c1: 4 splits measured 2% faster than 5)
   if (S > by_rows) S = by_rows;
   const int by_len = (cap + 1023) / 1024;
   if (S < by_len) S = by_len;
