@@ -928,6 +928,17 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k_new, const T* __r
       }
     }
   }
+  // The lines this step reads right after the wait, pulled into L2 while it
+  // waits (a prefetch binds no value: a write by the kernel being waited for
+  // still lands in L2 before the loads below read it).
+  if (tid < G * D / 8) {
+    const T* qp = q + ((size_t)bi * Hq + kh * G) * D + 8 * tid;
+    asm volatile("prefetch.global.L2 [%0];\n" ::"l"(qp));
+  }
+  if (rank < S && tid < 2 * D / 8) {
+    const T* np = (tid < D / 8 ? k_new : v_new) + ((size_t)bi * Hkv + kh) * D + 8 * (tid % (D / 8));
+    asm volatile("prefetch.global.L2 [%0];\n" ::"l"(np));
+  }
   // With programmatic dependent launch this kernel may start while the
   // previous kernel of the stream is still running: wait for it before
   // relying on anything another kernel may write (q, the cache, cache_len,
