@@ -28,6 +28,10 @@
  *   - A context is bound to the device that was current at imem_init; calls
  *     must be made with that device current. Calls that share a context or a
  *     workspace must be ordered on one stream.
+ *   - Calls on distinct contexts may come from several host threads at once:
+ *     the library's only process-wide host state is the one-time setting of
+ *     kernel attributes, per device, behind atomics (and a mutex where a
+ *     shared-memory size only ever grows).
  *
  * Data types: IMEM_FP32 or IMEM_BF16 (the "model dtype") applies to X, Q, K, V,
  * the indexer weights, decode inputs, the retained cache and the decode output.

@@ -46,6 +46,9 @@
 
 #include <cooperative_groups.h>
 #include <math.h>
+
+#include <atomic>
+#include <mutex>
 #include <type_traits>
 
 namespace imem {
@@ -1250,13 +1253,20 @@ cudaError_t launch_tgs(const Ctx& c, int S, int nst, int batch, const void* q, c
   const size_t smem = DecSmem<D, G>::total(kBf16, nst, r, S, m_in_w);
   const uint32_t slot_off = (uint32_t)DecSmem<D, G>::slot_off(r, m_in_w);
   auto k = decode_kernel<T, D, G, kTma, NRO, kXtra>;
-  static size_t attr_smem[64] = {};   // per instantiation and device: largest size set so far
+  // Per instantiation and device: the largest size set so far. Host threads
+  // that launch at once read it lock-free; raising it takes the mutex, so
+  // that a smaller size set late cannot undercut a larger one in use.
+  static std::atomic<size_t> attr_smem[64];
+  static std::mutex attr_mu;
   const int dv = c.device & 63;
-  if (attr_smem[dv] < smem) {
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-    attr_smem[dv] = smem;
+  if (attr_smem[dv].load(std::memory_order_acquire) < smem) {
+    std::lock_guard<std::mutex> lock(attr_mu);
+    if (attr_smem[dv].load(std::memory_order_relaxed) < smem) {
+      cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+      attr_smem[dv].store(smem, std::memory_order_release);
+    }
   }
   cudaLaunchConfig_t cfg = {};
   const int nro = NRO;   // readout CTAs per cluster

@@ -30,6 +30,8 @@
 #include "internal.h"
 #include "tc.cuh"
 
+#include <atomic>
+
 namespace imem {
 namespace {
 
@@ -326,12 +328,13 @@ cudaError_t launch_scoring(const Ctx& c, int batch, int L, const __nv_bfloat16* 
       done += cnt;
     }
   }
-  static bool attr_set[64] = {};
-  if (!attr_set[c.device & 63]) {
+  static std::atomic<uint64_t> attr_done{0};   // one bit per device
+  const uint64_t bit = 1ull << (c.device & 63);
+  if (!(attr_done.load() & bit)) {
     cudaError_t e = cudaFuncSetAttribute(scoring_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kScSmem);
     if (e != cudaSuccess) return e;
-    attr_set[c.device & 63] = true;
+    attr_done.fetch_or(bit);
   }
   scoring_tc_kernel<<<grid, kScThreads, kScSmem, st>>>(mq, mk, L, q_begin, q_end, starts,
                                                        running_max, c.err);

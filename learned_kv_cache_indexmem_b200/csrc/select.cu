@@ -26,6 +26,7 @@
 #include "common.cuh"
 #include "internal.h"
 
+#include <atomic>
 #include <cooperative_groups.h>
 
 namespace imem {
@@ -438,12 +439,15 @@ cudaError_t launch_select(int batch, const float* I, int L, int stride, int B, i
     select_kernel<<<batch, kSelThreads, 0, st>>>(I, L, stride, B, idx_r, idx_e);
     return cudaGetLastError();
   }
-  static bool attr_set = false;
-  if (!attr_set) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(select_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  static std::atomic<uint64_t> attr_done{0};   // one bit per device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(attr_done.load() & bit)) {
+    e = cudaFuncSetAttribute(select_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_done.fetch_or(bit);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(CS, batch, 1);
